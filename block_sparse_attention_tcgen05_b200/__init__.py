@@ -1,0 +1,15 @@
+"""Training-free block-sparse attention for video DiTs on NVIDIA B200 (sm_100a).
+
+The compute path lives in ``libbsa.so`` (hand-written CUDA for sm_100a behind a C ABI,
+declared in ``include/bsa.h``). This package is its thin Python binding: it checks
+arguments, allocates outputs and workspaces with torch and calls the library on the
+current CUDA stream. It has no CPU fallback; a missing library raises.
+"""
+
+from ._lib import BsaError, load as load_library  # noqa: F401
+from .ops import (  # noqa: F401
+    attention_workspace_bytes,
+    centroid_compensated_attention,
+    device_status,
+    tile_labels,
+)

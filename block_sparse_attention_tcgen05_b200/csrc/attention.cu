@@ -1,0 +1,918 @@
+// Block-sparse attention with SVG-EAR centroid compensation on sm_100a.
+//
+// Sources: "Sparse-block compensation" (mlx-arsenal notes) §The problem, §SVG-EAR —
+// centroid compensation, §No LSE needed; "Partition the Support, Reconstruct the
+// Residual" (Q, K, V permuted into group-major order; renormalised hard drop).
+//
+// Pipeline of one call (all on the caller's stream):
+//   1. label_sort_kernel (x2)   stable counting sort of the key / query labels into
+//                               cluster-major slots; each key cluster is padded to a
+//                               multiple of 16 slots, so every 16-key group belongs to
+//                               one cluster.
+//   2. mask_bits_kernel         the uint8 cluster mask -> per query cluster bitsets over
+//                               key clusters (centroid columns) and 16-key groups.
+//   3. gather_rows_kernel       Q rows into cluster-major order (zero pad rows).
+//   4. gather_kv_centroids      K, V rows into cluster-major padded order, fused with
+//                               the per-cluster mean k̄_c, v̄_c (fp32 sums).
+//   5. attn_kernel              one CTA per 128-row query tile: kept key groups are
+//                               walked as chunks of up to 128 keys (runs of kept
+//                               groups); skipped clusters follow as 128-wide centroid
+//                               chunks with column bias log2(n_c); both go through
+//                               the same online softmax, so no log-sum-exp leaves
+//                               the chip. S = QKᵀ and O += PV run on tcgen05 with
+//                               TMEM accumulators; P overwrites S in TMEM.
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdio>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace bsa {
+
+// ============================================================== label sort
+// One CTA of 1024 threads. Cluster c gets slots [off[c], off[c] + roundup(n_c,
+// cluster_pad)), filled with its tokens in increasing token order (a stable sort);
+// remaining slots hold token -1 / label -1. With group arrays given, 16-slot group g
+// is described by the cluster owning it and its number of real tokens.
+__global__ void __launch_bounds__(1024) label_sort_kernel(
+    const int32_t* __restrict__ labels, int S, int C, int cluster_pad, int n_slots,
+    int32_t* __restrict__ slot_token, int32_t* __restrict__ slot_label,
+    int32_t* __restrict__ count, int32_t* __restrict__ off, int32_t* __restrict__ group_cluster,
+    int32_t* __restrict__ group_valid, int n_groups, float* __restrict__ bias2, int C_pad,
+    uint32_t* __restrict__ nonempty_bits) {
+  extern __shared__ int32_t sm_i32[];
+  int32_t* cnt = sm_i32;     // C
+  int32_t* run = cnt + C;    // C + 1
+  __shared__ int32_t warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int c = tid; c < C; c += 1024) cnt[c] = 0;
+  for (int i = tid; i < n_slots; i += 1024) {
+    slot_token[i] = -1;
+    if (slot_label) slot_label[i] = -1;
+  }
+  __syncthreads();
+  for (int i = tid; i < S; i += 1024) {
+    const int l = labels[i];
+    if (l >= 0 && l < C) atomicAdd(&cnt[l], 1);
+    else report_device_error(kStatusBadLabel, 30);
+  }
+  __syncthreads();
+
+  // Exclusive scan of the padded cluster sizes; thread t owns a contiguous range.
+  const int per = (C + 1023) / 1024;
+  const int c0 = min(C, tid * per), c1 = min(C, c0 + per);
+  int local = 0;
+  for (int c = c0; c < c1; ++c) local += (cnt[c] + cluster_pad - 1) / cluster_pad * cluster_pad;
+  int incl = local;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int t = warp_tot[lane];
+    int ti = t;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += y;
+    }
+    warp_tot[lane] = ti - t;
+  }
+  __syncthreads();
+  int base = warp_tot[warp] + incl - local;
+  for (int c = c0; c < c1; ++c) {
+    run[c] = base;
+    off[c] = base;
+    count[c] = cnt[c];
+    base += (cnt[c] + cluster_pad - 1) / cluster_pad * cluster_pad;
+  }
+  if (tid == 1023) {
+    run[C] = base;
+    off[C] = base;
+  }
+  __syncthreads();
+
+  // Stable scatter, 1024 tokens at a time: ranks inside a warp from match_any, warps
+  // take their slots one after another so earlier tokens get earlier slots.
+  for (int t0 = 0; t0 < S; t0 += 1024) {
+    const int i = t0 + tid;
+    int l = (i < S) ? labels[i] : -1;
+    if (l >= C) l = -1;  // out-of-range labels were reported above; the token is dropped
+    const unsigned peers = __match_any_sync(0xffffffffu, l);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int leader = __ffs(peers) - 1;
+    int slot_base = 0;
+    for (int w = 0; w < 32; ++w) {
+      if (warp == w && l >= 0 && lane == leader) {
+        slot_base = run[l];
+        run[l] += __popc(peers);
+      }
+      __syncthreads();
+    }
+    slot_base = __shfl_sync(0xffffffffu, slot_base, leader);
+    if (l >= 0) {
+      const int s = slot_base + rank;
+      slot_token[s] = i;
+      if (slot_label) slot_label[s] = l;
+    }
+  }
+  __syncthreads();
+
+  if (group_cluster) {
+    const int total = off[C];
+    for (int g = tid; g < n_groups; g += 1024) {
+      const int slot = g * 16;
+      int c = -1, valid = 0;
+      if (slot < total) {
+        int lo = 0, hi = C + 1;  // first index with off > slot
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (off[mid] > slot) hi = mid; else lo = mid + 1;
+        }
+        c = lo - 1;
+        valid = min(16, cnt[c] - (slot - off[c]));
+      }
+      group_cluster[g] = c;
+      group_valid[g] = valid;
+    }
+  }
+  if (bias2) {
+    for (int c = tid; c < C_pad; c += 1024)
+      bias2[c] = (c < C && cnt[c] > 0) ? log2f(static_cast<float>(cnt[c])) : -INFINITY;
+    for (int w = tid; w < (C + 31) / 32; w += 1024) {
+      uint32_t bits = 0;
+      for (int j = 0; j < 32; ++j) {
+        const int c = w * 32 + j;
+        if (c < C && cnt[c] > 0) bits |= 1u << j;
+      }
+      nonempty_bits[w] = bits;
+    }
+  }
+}
+
+// ============================================================== mask bitsets
+// grid (Cq, n_h_slices, n_b_slices). cbits[slice][a][w]: bit c of word w = mask[a][32w+c].
+// gbits[slice][a][w]: bit j = mask[a][cluster of 16-key group 32w+j].
+__global__ void __launch_bounds__(256) mask_bits_kernel(
+    const uint8_t* __restrict__ mask, int64_t bstride, int64_t hstride, int nh, int Cq, int Ck,
+    const int32_t* __restrict__ group_cluster, const int32_t* __restrict__ group_valid,
+    int n_groups, int Wc, int Wg, uint32_t* __restrict__ cbits, uint32_t* __restrict__ gbits,
+    uint32_t* __restrict__ gfull) {
+  const int a = blockIdx.x, hs = blockIdx.y, bs = blockIdx.z;
+  const uint8_t* row = mask + bs * bstride + hs * hstride + static_cast<int64_t>(a) * Ck;
+  const size_t slice = static_cast<size_t>(bs) * nh + hs;
+  uint32_t* crow = cbits + (slice * Cq + a) * Wc;
+  uint32_t* grow = gbits + (slice * Cq + a) * Wg;
+  for (int w = threadIdx.x; w < Wc; w += blockDim.x) {
+    uint32_t bits = 0;
+    for (int j = 0; j < 32; ++j) {
+      const int c = w * 32 + j;
+      if (c < Ck && row[c]) bits |= 1u << j;
+    }
+    crow[w] = bits;
+  }
+  for (int w = threadIdx.x; w < Wg; w += blockDim.x) {
+    uint32_t bits = 0;
+    for (int j = 0; j < 32; ++j) {
+      const int g = w * 32 + j;
+      if (g < n_groups) {
+        const int c = group_cluster[g];
+        if (c >= 0 && row[c]) bits |= 1u << j;
+      }
+    }
+    grow[w] = bits;
+  }
+  if (a == 0 && slice == 0) {
+    for (int w = threadIdx.x; w < Wg; w += blockDim.x) {
+      uint32_t bits = 0;
+      for (int j = 0; j < 32; ++j) {
+        const int g = w * 32 + j;
+        if (g < n_groups && group_valid[g] == 16) bits |= 1u << j;
+      }
+      gfull[w] = bits;
+    }
+  }
+}
+
+// ============================================================== gathers
+// dst[bh][r] = src[bh][row_token[r]] (zero row when the token is -1); 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src,
+                                                          uint4* __restrict__ dst,
+                                                          const int32_t* __restrict__ row_token,
+                                                          int S, int Spad, int vpr, int H) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int r = static_cast<int>(idx / vpr), v = static_cast<int>(idx % vpr);
+  if (r >= Spad) return;
+  const int64_t bh = static_cast<int64_t>(blockIdx.z) * H + blockIdx.y;
+  const int tok = row_token[r];
+  uint4 val = make_uint4(0, 0, 0, 0);
+  if (tok >= 0) val = __ldg(src + (bh * S + tok) * vpr + v);
+  dst[(bh * Spad + r) * vpr + v] = val;
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& u, float* f);
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(h[i]);
+    f[2 * i] = x.x;
+    f[2 * i + 1] = x.y;
+  }
+}
+template <>
+__device__ __forceinline__ void unpack16<float>(const uint4& u, float* f) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void store_elt(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+__device__ __forceinline__ void store_elt(float* p, float x) { *p = x; }
+
+// grid (C_pad, Hkv, B), 256 threads. Copies the rows of cluster c into their padded
+// cluster-major slots of kp / vp and writes the cluster means k̄_c, v̄_c (fp32 sums,
+// rounded once to T). Clusters that are empty or beyond C get zero centroids.
+template <typename T>
+__global__ void __launch_bounds__(256) gather_kv_centroids_kernel(
+    const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ kp, T* __restrict__ vp,
+    T* __restrict__ kc, T* __restrict__ vc, const int32_t* __restrict__ slot_token,
+    const int32_t* __restrict__ count, const int32_t* __restrict__ off, int S, int Skpad, int C,
+    int Cpad, int D, int Hkv) {
+  constexpr int EPV = 16 / sizeof(T);
+  __shared__ float red[2][2048];
+  const int c = blockIdx.x;
+  const int64_t bh = static_cast<int64_t>(blockIdx.z) * Hkv + blockIdx.y;
+  const int vpr = D / EPV, rpi = 256 / vpr;
+  const int rin = threadIdx.x / vpr, part = threadIdx.x % vpr;
+  const int n = c < C ? count[c] : 0;
+  const int start = c < C ? off[c] : 0;
+  const int padded = (n + 15) / 16 * 16;
+  float ak[EPV], av[EPV];
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) ak[e] = av[e] = 0.f;
+  const uint4* k4 = reinterpret_cast<const uint4*>(k);
+  const uint4* v4 = reinterpret_cast<const uint4*>(v);
+  uint4* kp4 = reinterpret_cast<uint4*>(kp);
+  uint4* vp4 = reinterpret_cast<uint4*>(vp);
+  for (int s = rin; s < padded; s += rpi) {
+    const int slot = start + s;
+    const int tok = slot_token[slot];
+    uint4 xk = make_uint4(0, 0, 0, 0), xv = make_uint4(0, 0, 0, 0);
+    if (tok >= 0) {
+      xk = __ldg(k4 + (bh * S + tok) * vpr + part);
+      xv = __ldg(v4 + (bh * S + tok) * vpr + part);
+    }
+    kp4[(bh * Skpad + slot) * vpr + part] = xk;
+    vp4[(bh * Skpad + slot) * vpr + part] = xv;
+    float fk[EPV], fv[EPV];
+    unpack16<T>(xk, fk);
+    unpack16<T>(xv, fv);
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) {
+      ak[e] += fk[e];
+      av[e] += fv[e];
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) {
+    red[0][rin * D + part * EPV + e] = ak[e];
+    red[1][rin * D + part * EPV + e] = av[e];
+  }
+  __syncthreads();
+  const float inv = n > 0 ? 1.f / static_cast<float>(n) : 0.f;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float sk = 0.f, sv = 0.f;
+    for (int r = 0; r < rpi; ++r) {
+      sk += red[0][r * D + d];
+      sv += red[1][r * D + d];
+    }
+    store_elt(kc + (bh * Cpad + c) * D + d, sk * inv);
+    store_elt(vc + (bh * Cpad + c) * D + d, sv * inv);
+  }
+}
+
+// ============================================================== attention kernel
+struct AttnArgs {
+  int B, Hq, Hkv, Sq, Sqpad, Skpad, Ck, Ckpad, Cq, G, Wg, Wc;
+  int nh_slices, b_sliced, h_sliced;
+  int compensate;
+  float scale_log2;
+  const int32_t* qrow_token;
+  const int32_t* qrow_label;
+  const int32_t* group_valid;
+  const uint32_t* cbits;
+  const uint32_t* gbits;
+  const uint32_t* gfull;
+  const uint32_t* cnonempty;
+  const float* bias2;
+  float* out;
+};
+
+template <int D, bool TF32>
+struct AttnCfg {
+  static constexpr int ESIZE = TF32 ? 4 : 2;
+  static constexpr int ATOM = 128 / ESIZE;          // elements per 128-byte swizzled row
+  static constexpr int NATOM = D / ATOM;            // 128-byte column chunks per row
+  static constexpr int TILE = 128 * D * ESIZE;      // one 128-row operand tile
+  static constexpr int KSTEP = 32 / ESIZE;          // K of one MMA instruction
+  static constexpr int MISC = 4096;
+  static constexpr int SMEM = 3 * TILE + MISC + 1024;
+  // At least ~100 KB so that at most two CTAs share an SM (two 256-column TMEM
+  // allocations fill the 512 columns).
+  static constexpr int SMEM_LAUNCH = SMEM > 100 * 1024 ? SMEM : 100 * 1024;
+};
+
+enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SF, BAR_PF, BAR_OF, BAR_DRAIN, NBAR };
+
+struct Chunk {
+  int start;   // first key slot (token chunk) or first centroid (centroid chunk)
+  int n;       // number of columns, multiple of 16, <= 128
+  int g0, ng;  // token chunk: first group and number of groups
+  bool uniform, centroid;
+};
+
+__device__ __forceinline__ bool bit_at(const uint32_t* bits, int i) {
+  return (bits[i >> 5] >> (i & 31)) & 1u;
+}
+
+// Deterministic chunk walk shared by every role of the CTA: runs of kept 16-key
+// groups split into chunks of at most 8 groups, then the needed centroid chunks.
+__device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t* any,
+                                           const uint32_t* uni, int G, int Wg,
+                                           const uint32_t* cneed, int ncc, Chunk& ch) {
+  if (gcur < G) {
+    int w = gcur >> 5;
+    uint32_t bits = any[w] & (0xffffffffu << (gcur & 31));
+    while (bits == 0 && ++w < Wg) bits = any[w];
+    if (bits != 0) {
+      const int g0 = (w << 5) + __ffs(bits) - 1;
+      int ng = 1;
+      while (ng < 8 && g0 + ng < G && bit_at(any, g0 + ng)) ++ng;
+      bool uniform = true;
+      for (int j = 0; j < ng; ++j) uniform = uniform && bit_at(uni, g0 + j);
+      ch.start = g0 * 16;
+      ch.n = ng * 16;
+      ch.g0 = g0;
+      ch.ng = ng;
+      ch.uniform = uniform;
+      ch.centroid = false;
+      gcur = g0 + ng;
+      return true;
+    }
+    gcur = G;
+  }
+  while (ccur < ncc) {
+    const int i = ccur++;
+    if (bit_at(cneed, i)) {
+      ch.start = i * 128;
+      ch.n = 128;
+      ch.g0 = ch.ng = 0;
+      ch.uniform = false;
+      ch.centroid = true;
+      return true;
+    }
+  }
+  return false;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D, bool TF32>
+__global__ void __launch_bounds__(192, 2)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
+                const __grid_constant__ CUtensorMap tmVc, const AttnArgs a) {
+  using Cfg = AttnCfg<D, TF32>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sQ = smem_u32(smem), sK = sQ + Cfg::TILE, sV = sK + Cfg::TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 3 * Cfg::TILE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* n_distinct = reinterpret_cast<int*>(tmem_slot + 2);
+  int* never = reinterpret_cast<int*>(tmem_slot + 3);
+  int* distinct = reinterpret_cast<int*>(tmem_slot + 4);     // 128
+  uint32_t* any_bits = reinterpret_cast<uint32_t*>(distinct + 128);  // 128 words
+  uint32_t* uni_bits = any_bits + 128;                                // 128 words
+  uint32_t* cneed = uni_bits + 128;                                   // 4 words
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int hkv = h / (a.Hq / a.Hkv);
+  const int slice = (a.b_sliced ? b : 0) * a.nh_slices + (a.h_sliced ? h : 0);
+  const uint32_t bar0 = smem_u32(bars);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+  if (tid == 0) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(BAR(i), i == BAR_PF ? 128u : 1u);
+    *abort_flag = 0;
+    *n_distinct = 0;
+    *never = 0;
+    fence_mbarrier_init();
+  }
+  if (tid == 32) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  if (tid < 4) cneed[tid] = 0;
+  __syncthreads();
+
+  // Query clusters present in this tile (rows are sorted by label, pads last).
+  if (tid < 128) {
+    const int r = tile * 128 + tid;
+    const int lab = a.qrow_label[r];
+    const int prev = tid > 0 ? a.qrow_label[r - 1] : -2;
+    if (lab >= 0 && lab != prev) distinct[atomicAdd(n_distinct, 1)] = lab;
+  }
+  __syncthreads();
+  const int nd = *n_distinct;
+  const uint32_t* gb = a.gbits + static_cast<size_t>(slice) * a.Cq * a.Wg;
+  const uint32_t* cb = a.cbits + static_cast<size_t>(slice) * a.Cq * a.Wc;
+  for (int w = tid; w < 128; w += blockDim.x) {
+    uint32_t any = 0, all = 0;
+    if (w < a.Wg && nd > 0) {
+      all = 0xffffffffu;
+      for (int i = 0; i < nd; ++i) {
+        const uint32_t x = gb[static_cast<size_t>(distinct[i]) * a.Wg + w];
+        any |= x;
+        all &= x;
+      }
+      all &= a.gfull[w];
+    }
+    any_bits[w] = any;
+    uni_bits[w] = all & any;
+  }
+  if (a.compensate) {
+    for (int w = tid; w < a.Wc; w += blockDim.x) {
+      uint32_t need = 0;
+      for (int i = 0; i < nd; ++i) need |= ~cb[static_cast<size_t>(distinct[i]) * a.Wc + w];
+      need &= a.cnonempty[w];
+      if (need) atomicOr(&cneed[(w >> 2) >> 5], 1u << ((w >> 2) & 31));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int ncc = a.compensate ? a.Ckpad / 128 : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int qrow0 = (b * a.Hq + h) * a.Sqpad + tile * 128;
+      mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
+#pragma unroll
+      for (int c = 0; c < Cfg::NATOM; ++c)
+        tma_load_2d(sQ + c * 16384, &tmQ, BAR(BAR_Q), c * Cfg::ATOM, qrow0);
+      int gcur = 0, ccur = 0, j = 0, nk = 0, nv = 0;
+      Chunk ch;
+      while (next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
+        const CUtensorMap* mk = ch.centroid ? &tmKc : &tmK;
+        const CUtensorMap* mv = ch.centroid ? &tmVc : &tmV;
+        const int row = ch.centroid ? (b * a.Hkv + hkv) * a.Ckpad + ch.start
+                                    : (b * a.Hkv + hkv) * a.Skpad + ch.start;
+        if (j > 0 && !mbar_wait(BAR(BAR_KE), (j - 1) & 1, abort_flag, 1)) break;
+        mbar_arrive_expect_tx(BAR(BAR_KF), Cfg::TILE);
+#pragma unroll
+        for (int c = 0; c < Cfg::NATOM; ++c)
+          tma_load_2d(sK + c * 16384, mk, BAR(BAR_KF), c * Cfg::ATOM, row);
+        ++nk;
+        if (j > 0 && !mbar_wait(BAR(BAR_VE), (j - 1) & 1, abort_flag, 2)) break;
+        mbar_arrive_expect_tx(BAR(BAR_VF), Cfg::TILE);
+#pragma unroll
+        for (int c = 0; c < Cfg::NATOM; ++c)
+          tma_load_2d(sV + c * 16384, mv, BAR(BAR_VF), c * Cfg::ATOM, row);
+        ++nv;
+        ++j;
+      }
+      // Every issued copy must land before the CTA may exit.
+      mbar_wait(BAR(BAR_Q), 0, never, 20);
+      if (nk) mbar_wait(BAR(BAR_KF), (nk - 1) & 1, never, 21);
+      if (nv) mbar_wait(BAR(BAR_VF), (nv - 1) & 1, never, 22);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (one thread)
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = make_idesc(TF32, 128, 0, false, false);
+      constexpr uint32_t kIdescPV = make_idesc(TF32, 128, D, false, true);
+      bool ok = mbar_wait(BAR(BAR_Q), 0, abort_flag, 3);
+      int gcur = 0, ccur = 0, j = 0;
+      Chunk ch;
+      while (ok && next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
+        // S (and P, which aliases it) is free once the previous PV has completed.
+        if (j > 0 && !(ok = mbar_wait(BAR(BAR_VE), (j - 1) & 1, abort_flag, 4))) break;
+        if (!(ok = mbar_wait(BAR(BAR_KF), j & 1, abort_flag, 5))) break;
+        tc_fence_after();
+        const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(ch.n >> 3) << 17);
+#pragma unroll
+        for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          mma_ss<TF32>(tmem, smem_desc(sQ + off, 16, 1024), smem_desc(sK + off, 16, 1024),
+                       idesc, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(BAR(BAR_KE));
+        tc_commit(BAR(BAR_SF));
+        if (!(ok = mbar_wait(BAR(BAR_PF), j & 1, abort_flag, 6))) break;
+        if (!(ok = mbar_wait(BAR(BAR_VF), j & 1, abort_flag, 7))) break;
+        tc_fence_after();
+        const int nsteps = ch.n / Cfg::KSTEP;
+        for (int kk = 0; kk < nsteps; ++kk) {
+          // V is MN-major (d contiguous): 128-byte rows, d chunks 16 KB apart; bf16 uses
+          // 8-row swizzle groups (1 KB), tf32 the 32-byte-unit swizzle with 4-row groups.
+          const uint64_t bdesc =
+              TF32 ? smem_desc(sV + kk * Cfg::KSTEP * 128, 16384, 512, kLayoutSW128Atom32B)
+                   : smem_desc(sV + kk * Cfg::KSTEP * 128, 16384, 1024, kLayoutSW128);
+          mma_ts<TF32>(tmem + 128, tmem + kk * 8, bdesc, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(BAR(BAR_VE));
+        ++j;
+      }
+      tc_commit(BAR(BAR_OF));
+      tc_commit(BAR(BAR_DRAIN));
+      mbar_wait(BAR(BAR_DRAIN), 0, never, 23);
+    }
+  } else {
+    // ------------------------------------------------ softmax / epilogue (128 threads)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qrow = tile * 128 + r;
+    const int lab = a.qrow_label[qrow];
+    const int tok = a.qrow_token[qrow];
+    const uint32_t* grow = gb + static_cast<size_t>(lab < 0 ? 0 : lab) * a.Wg;
+    const uint32_t* crow = cb + static_cast<size_t>(lab < 0 ? 0 : lab) * a.Wc;
+    const uint32_t tS = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t tO = tS + 128;
+    float m_run = -INFINITY, l_run = 0.f;
+    int gcur = 0, ccur = 0, j = 0;
+    bool ok = true;
+    Chunk ch;
+    while (next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
+      if (!(ok = mbar_wait(BAR(BAR_SF), j & 1, abort_flag, 9))) break;
+      tc_fence_after();
+      const int npc = (ch.n + 31) >> 5;
+      float s[128];
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        if (p < npc) tmem_ld32(tS + p * 32, *reinterpret_cast<float(*)[32]>(&s[p * 32]));
+      tmem_wait_ld();
+
+      uint32_t mk[4];
+      if (lab < 0) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) mk[w] = 0;
+      } else if (ch.centroid) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int ww = (ch.start >> 5) + w;
+          mk[w] = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
+        }
+      } else if (ch.uniform) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) mk[w] = 0xffffffffu;
+      } else {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) mk[w] = 0;
+        for (int jj = 0; jj < ch.ng; ++jj) {
+          const int g = ch.g0 + jj;
+          if ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u) {
+            const int nv = bit_at(a.gfull, g) ? 16 : __ldg(a.group_valid + g);
+            const uint32_t bits = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
+            mk[jj >> 1] |= bits << ((jj & 1) * 16);
+          }
+        }
+      }
+
+      float mx = -INFINITY;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        if (p < npc) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int col = p * 32 + c;
+            float x = s[col] * a.scale_log2;
+            if (ch.centroid) x += __ldg(a.bias2 + ch.start + col);
+            const bool keep = (col < ch.n) && ((mk[p] >> c) & 1u);
+            x = keep ? x : -INFINITY;
+            s[col] = x;
+            mx = fmaxf(mx, x);
+          }
+        }
+      }
+      // Lazy rescaling: the running max only moves when the chunk max exceeds it by
+      // more than 2^8, so P stays below 256 and O is rarely touched.
+      const bool need = mx > m_run + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = need ? mx : m_run;
+        const float alpha = need ? ex2(m_run - m_new) : 1.f;
+        if (j > 0) {
+#pragma unroll
+          for (int p = 0; p < D / 32; ++p) {
+            float o[32];
+            tmem_ld32(tO + p * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= alpha;
+            tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+          }
+        }
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+      float sum = 0.f;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        if (p < npc) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float e = ex2(s[p * 32 + c] - mu);
+            sum += e;
+            s[p * 32 + c] = e;
+          }
+        }
+      }
+      l_run += sum;
+      if constexpr (TF32) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          if (p < npc) tmem_st32(tS + p * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[p * 32]));
+      } else {
+        uint32_t* pk = reinterpret_cast<uint32_t*>(s);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+        if (ch.n > 64) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(BAR_PF));
+      ++j;
+    }
+    if (ok && mbar_wait(BAR(BAR_OF), 0, abort_flag, 10)) {
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      float* orow = a.out + ((static_cast<size_t>(b) * a.Hq + h) * a.Sq + (tok >= 0 ? tok : 0)) * D;
+#pragma unroll
+      for (int p = 0; p < D / 32; ++p) {
+        float o[32];
+        tmem_ld32(tO + p * 32, o);
+        tmem_wait_ld();
+        if (tok >= 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 v4 = l_run > 0.f ? make_float4(o[4 * i] * inv, o[4 * i + 1] * inv,
+                                                  o[4 * i + 2] * inv, o[4 * i + 3] * inv)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4*>(orow + p * 32 + 4 * i) = v4;
+          }
+        }
+      }
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ============================================================== host side
+namespace {
+
+struct AttnLayout {
+  int Sqpad, Skpad, G, Wg, Ckpad, Wc, Cqpad;
+  int32_t *qrow_token, *qrow_label, *q_count, *q_off;
+  int32_t *kslot_token, *group_cluster, *group_valid, *k_count, *k_off;
+  float* bias2;
+  uint32_t *cnonempty, *cbits, *gbits, *gfull;
+  void *qp, *kp, *vp, *kc, *vc;
+  size_t bytes;
+};
+
+AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
+  AttnLayout L{};
+  const int es = s.dtype == BSA_F32 ? 4 : 2;
+  L.Sqpad = ceil_div(s.Sq, 128) * 128;
+  L.Skpad = ceil_div(s.Sk + 15 * Ck, 128) * 128;
+  L.G = L.Skpad / 16;
+  L.Wg = ceil_div(L.G, 32);
+  L.Ckpad = ceil_div(Ck, 128) * 128;
+  L.Wc = ceil_div(Ck, 32);
+  Carver cv(ws);
+  L.qrow_token = cv.take<int32_t>(L.Sqpad);
+  L.qrow_label = cv.take<int32_t>(L.Sqpad);
+  L.q_count = cv.take<int32_t>(Cq);
+  L.q_off = cv.take<int32_t>(Cq + 1);
+  L.kslot_token = cv.take<int32_t>(L.Skpad);
+  L.group_cluster = cv.take<int32_t>(L.G);
+  L.group_valid = cv.take<int32_t>(L.G);
+  L.k_count = cv.take<int32_t>(Ck);
+  L.k_off = cv.take<int32_t>(Ck + 1);
+  L.bias2 = cv.take<float>(L.Ckpad);
+  L.cnonempty = cv.take<uint32_t>(L.Wc);
+  const size_t slices = static_cast<size_t>(s.B) * s.Hq;
+  L.cbits = cv.take<uint32_t>(slices * Cq * L.Wc);
+  L.gbits = cv.take<uint32_t>(slices * Cq * L.Wg);
+  L.gfull = cv.take<uint32_t>(L.Wg);
+  L.qp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hq * L.Sqpad * s.D * es);
+  L.kp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Skpad * s.D * es);
+  L.vp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Skpad * s.D * es);
+  L.kc = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Ckpad * s.D * es);
+  L.vc = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Ckpad * s.D * es);
+  L.bytes = align_up(cv.used, 256);
+  return L;
+}
+
+template <int D, bool TF32>
+int launch_attn(const CUtensorMap* maps, const AttnArgs& args, dim3 grid, cudaStream_t st) {
+  using Cfg = AttnCfg<D, TF32>;
+  auto kern = attn_kernel<D, TF32>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg::SMEM_LAUNCH);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attn_kernel)");
+  kern<<<grid, 192, Cfg::SMEM_LAUNCH, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
+  return check_cuda(cudaGetLastError(), "attn_kernel launch");
+}
+
+}  // namespace
+
+int validate_attention_shape(const bsa_shape& s, int Cq, int Ck) {
+  if (s.B <= 0 || s.Hq <= 0 || s.Hkv <= 0 || s.Sq <= 0 || s.Sk <= 0)
+    return fail(BSA_ERR_INVALID_ARG, "non-positive shape");
+  if (s.Hq % s.Hkv) return fail(BSA_ERR_INVALID_ARG, "Hq (%d) not a multiple of Hkv (%d)", s.Hq, s.Hkv);
+  if (s.D != 64 && s.D != 128) return fail(BSA_ERR_UNSUPPORTED, "head dim %d not in {64,128}", s.D);
+  if (s.dtype != BSA_BF16 && s.dtype != BSA_F32) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", s.dtype);
+  if (Cq <= 0 || Ck <= 0 || Cq > 16384 || Ck > 16384)
+    return fail(BSA_ERR_UNSUPPORTED, "cluster counts Cq=%d Ck=%d outside [1,16384]", Cq, Ck);
+  if (static_cast<int64_t>(s.Sk) + 15LL * Ck > 65536)
+    return fail(BSA_ERR_UNSUPPORTED, "Sk + 15*Ck = %lld exceeds 65536",
+                static_cast<long long>(s.Sk) + 15LL * Ck);
+  if (s.Sq > 65536) return fail(BSA_ERR_UNSUPPORTED, "Sq %d exceeds 65536", s.Sq);
+  return BSA_OK;
+}
+
+size_t attention_workspace_bytes(const bsa_shape& s, int Cq, int Ck) {
+  return carve(s, Cq, Ck, nullptr).bytes;
+}
+
+int run_label_sort(const int32_t* labels, int S, int C, int cluster_pad, int n_slots,
+                   int32_t* slot_token, int32_t* slot_label, int32_t* count, int32_t* off,
+                   int32_t* group_cluster, int32_t* group_valid, int n_groups, float* bias2,
+                   int C_pad, uint32_t* nonempty, cudaStream_t st) {
+  const int smem = (2 * C + 1) * 4;
+  cudaError_t e = cudaFuncSetAttribute(label_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem > 48 * 1024 ? smem : 48 * 1024);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(label_sort)");
+  label_sort_kernel<<<1, 1024, smem, st>>>(labels, S, C, cluster_pad, n_slots, slot_token,
+                                           slot_label, count, off, group_cluster, group_valid,
+                                           n_groups, bias2, C_pad, nonempty);
+  return check_cuda(cudaGetLastError(), "label_sort_kernel launch");
+}
+
+int centroid_compensated_attention(const void* q, const void* k, const void* v,
+                                   const bsa_shape& s, const int32_t* q_labels, int Cq,
+                                   const int32_t* k_labels, int Ck, const uint8_t* mask,
+                                   int64_t mbs, int64_t mhs, float scale, int compensate,
+                                   float* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  int rc = validate_attention_shape(s, Cq, Ck);
+  if (rc) return rc;
+  if (s.Sq != s.Sk && false) return rc;
+  if (!q || !k || !v || !q_labels || !k_labels || !mask || !out)
+    return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+  if (mbs < 0 || mhs < 0) return fail(BSA_ERR_INVALID_ARG, "negative mask stride");
+  AttnLayout L = carve(s, Cq, Ck, ws);
+  if (!ws || ws_bytes < L.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, L.bytes);
+  if (reinterpret_cast<uintptr_t>(ws) % 256)
+    return fail(BSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  const int es = s.dtype == BSA_F32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+       reinterpret_cast<uintptr_t>(v)) % 16)
+    return fail(BSA_ERR_INVALID_ARG, "q/k/v must be 16-byte aligned");
+
+  // 1. label sorts
+  if ((rc = run_label_sort(k_labels, s.Sk, Ck, 16, L.Skpad, L.kslot_token, nullptr, L.k_count,
+                           L.k_off, L.group_cluster, L.group_valid, L.G, L.bias2, L.Ckpad,
+                           L.cnonempty, st)))
+    return rc;
+  if ((rc = run_label_sort(q_labels, s.Sq, Cq, 1, L.Sqpad, L.qrow_token, L.qrow_label, L.q_count,
+                           L.q_off, nullptr, nullptr, 0, nullptr, 0, nullptr, st)))
+    return rc;
+  // 2. mask bitsets
+  const int nb = mbs ? s.B : 1, nh = mhs ? s.Hq : 1;
+  mask_bits_kernel<<<dim3(Cq, nh, nb), 256, 0, st>>>(mask, mbs, mhs, nh, Cq, Ck, L.group_cluster,
+                                                    L.group_valid, L.G, L.Wc, L.Wg, L.cbits,
+                                                    L.gbits, L.gfull);
+  if ((rc = check_cuda(cudaGetLastError(), "mask_bits_kernel"))) return rc;
+  // 3. Q gather
+  const int vpr = s.D * es / 16;
+  {
+    const int64_t n = static_cast<int64_t>(L.Sqpad) * vpr;
+    gather_rows_kernel<<<dim3(static_cast<unsigned>((n + 255) / 256), s.Hq, s.B), 256, 0, st>>>(
+        static_cast<const uint4*>(q), static_cast<uint4*>(L.qp), L.qrow_token, s.Sq, L.Sqpad, vpr,
+        s.Hq);
+    if ((rc = check_cuda(cudaGetLastError(), "gather_rows_kernel"))) return rc;
+  }
+  // 4. K/V gather + centroids
+  if (s.dtype == BSA_F32) {
+    gather_kv_centroids_kernel<float><<<dim3(L.Ckpad, s.Hkv, s.B), 256, 0, st>>>(
+        static_cast<const float*>(k), static_cast<const float*>(v), static_cast<float*>(L.kp),
+        static_cast<float*>(L.vp), static_cast<float*>(L.kc), static_cast<float*>(L.vc),
+        L.kslot_token, L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
+  } else {
+    gather_kv_centroids_kernel<__nv_bfloat16><<<dim3(L.Ckpad, s.Hkv, s.B), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+        static_cast<__nv_bfloat16*>(L.kp), static_cast<__nv_bfloat16*>(L.vp),
+        static_cast<__nv_bfloat16*>(L.kc), static_cast<__nv_bfloat16*>(L.vc), L.kslot_token,
+        L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
+  }
+  if ((rc = check_cuda(cudaGetLastError(), "gather_kv_centroids_kernel"))) return rc;
+
+  // 5. tensor maps + attention
+  const CUtensorMapDataType tdt =
+      s.dtype == BSA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint32_t atom = 128 / es;
+  // V tiles feed the MMA as MN-major operands; for tf32 those must use the 32-byte-unit
+  // 128-byte swizzle, the other tiles use the 16-byte-unit one.
+  const CUtensorMapSwizzle vsw =
+      s.dtype == BSA_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap maps[5];
+  if ((rc = make_tmap_2d(&maps[0], L.qp, tdt, es, static_cast<uint64_t>(s.B) * s.Hq * L.Sqpad, s.D, 128, atom)) ||
+      (rc = make_tmap_2d(&maps[1], L.kp, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Skpad, s.D, 128, atom)) ||
+      (rc = make_tmap_2d(&maps[2], L.vp, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Skpad, s.D, 128, atom, vsw)) ||
+      (rc = make_tmap_2d(&maps[3], L.kc, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Ckpad, s.D, 128, atom)) ||
+      (rc = make_tmap_2d(&maps[4], L.vc, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Ckpad, s.D, 128, atom, vsw)))
+    return rc;
+  AttnArgs args{};
+  args.B = s.B;
+  args.Hq = s.Hq;
+  args.Hkv = s.Hkv;
+  args.Sq = s.Sq;
+  args.Sqpad = L.Sqpad;
+  args.Skpad = L.Skpad;
+  args.Ck = Ck;
+  args.Ckpad = L.Ckpad;
+  args.Cq = Cq;
+  args.G = L.G;
+  args.Wg = L.Wg;
+  args.Wc = L.Wc;
+  args.nh_slices = nh;
+  args.b_sliced = mbs ? 1 : 0;
+  args.h_sliced = mhs ? 1 : 0;
+  args.compensate = compensate ? 1 : 0;
+  const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(s.D));
+  args.scale_log2 = sc * 1.4426950408889634f;
+  args.qrow_token = L.qrow_token;
+  args.qrow_label = L.qrow_label;
+  args.group_valid = L.group_valid;
+  args.cbits = L.cbits;
+  args.gbits = L.gbits;
+  args.gfull = L.gfull;
+  args.cnonempty = L.cnonempty;
+  args.bias2 = L.bias2;
+  args.out = out;
+  const dim3 grid(L.Sqpad / 128, s.Hq, s.B);
+  if (s.dtype == BSA_F32) {
+    return s.D == 64 ? launch_attn<64, true>(maps, args, grid, st)
+                     : launch_attn<128, true>(maps, args, grid, st);
+  }
+  return s.D == 64 ? launch_attn<64, false>(maps, args, grid, st)
+                   : launch_attn<128, false>(maps, args, grid, st);
+}
+
+}  // namespace bsa
+
+extern "C" size_t bsa_attention_workspace_bytes(bsa_shape shape, int Cq, int Ck) {
+  if (bsa::validate_attention_shape(shape, Cq, Ck)) return 0;
+  return bsa::attention_workspace_bytes(shape, Cq, Ck);
+}
+
+extern "C" int bsa_centroid_compensated_attention(const void* q, const void* k, const void* v,
+                                                  bsa_shape shape, const int32_t* q_labels, int Cq,
+                                                  const int32_t* k_labels, int Ck,
+                                                  const uint8_t* block_mask, int64_t mask_b_stride,
+                                                  int64_t mask_h_stride, float scale, int compensate,
+                                                  float* out, void* workspace,
+                                                  size_t workspace_bytes, void* stream) {
+  return bsa::centroid_compensated_attention(q, k, v, shape, q_labels, Cq, k_labels, Ck, block_mask,
+                                             mask_b_stride, mask_h_stride, scale, compensate, out,
+                                             workspace, workspace_bytes, bsa::as_stream(stream));
+}

@@ -1,0 +1,250 @@
+/*
+ * bsa.h — C ABI of libbsa.so: training-free block-sparse attention for video DiTs
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages; cited by title and section):
+ *  [SBC]  "Sparse-block compensation" — mlx-arsenal research notes:
+ *         §The problem, §SVG-EAR — centroid compensation, §SparsePR — probe-fitted
+ *         residual repair, §What mlx-arsenal ships, §No LSE needed, §Recipe,
+ *         §Deviations from the papers.
+ *  [HMR]  "Dynamic block masks and head-wise mask reuse" — mlx-arsenal research
+ *         notes: §XAttention — anti-diagonal block scoring, §HEART — head-wise
+ *         temporal mask reuse, §What mlx-arsenal ships, §Recipe, §Deviations,
+ *         §Out of scope (padding).
+ *  [SPR]  "Partition the Support, Reconstruct the Residual: Training-Free Sparse
+ *         Attention for Video Generation and World Models" — paper summary:
+ *         probe-fitted residual reconstruction, group-major permutation, GQA.
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are caller-owned DEVICE memory, contiguous, row-major. Q is
+ *    (B, Hq, S, D); K and V are (B, Hkv, S, D) with Hq a multiple of Hkv (query head
+ *    h uses KV head h / (Hq / Hkv)). Element type: BSA_BF16 or BSA_F32.
+ *  - Cluster labels are int32 device arrays shared by every batch and head.
+ *    Masks are uint8 device arrays, 1 = block kept (computed exactly).
+ *  - The library never allocates device memory. An op that needs scratch space
+ *    has a *_workspace_bytes query; the caller passes a device buffer at least that
+ *    large (256-byte aligned). Workspace contents are undefined on return.
+ *  - Every call is asynchronous on the caller's stream (a cudaStream_t passed as
+ *    void*, NULL = legacy default stream) unless its comment says it synchronises.
+ *  - Return value: BSA_OK or a negative status. Argument errors are detected on the
+ *    host before any launch. A device-side wait that runs out of time records
+ *    BSA_ERR_TIMEOUT, read back with bsa_get_device_status().
+ *  - Output attention tensors are fp32 (B, Hq, S, D) in the ORIGINAL token order.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = -1,   /* null pointer, bad size, inconsistent shapes */
+  BSA_ERR_UNSUPPORTED = -2,   /* dtype, head dim or size outside the supported set */
+  BSA_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed */
+  BSA_ERR_TIMEOUT = -4,       /* a bounded device-side wait gave up */
+  BSA_ERR_WORKSPACE = -5      /* workspace missing or too small */
+};
+
+enum { BSA_BF16 = 0, BSA_F32 = 1 };
+
+/* Problem shape. Sq = Sk = S for self-attention; D in {64, 128}. */
+typedef struct {
+  int B, Hq, Hkv, Sq, Sk, D;
+  int dtype; /* BSA_BF16 or BSA_F32 */
+} bsa_shape;
+
+/* Human-readable name of a status code (static string). */
+const char* bsa_status_string(int status);
+
+/* Copies the calling thread's last error detail (NUL-terminated) into buf. */
+void bsa_last_error_detail(char* buf, size_t len);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int bsa_version(void);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word: BSA_OK, or
+ * BSA_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call. *where
+ * (nullable) receives the kernel-specific site code of the first failure.
+ */
+int bsa_get_device_status(void* stream, int* where);
+
+/*
+ * tile_labels — [SBC] §What mlx-arsenal ships (tile_labels: labels matching Sliding
+ * Tile Attention tiles), §Recipe. Token s = (t*H + h)*W + w of a T x H x W latent
+ * grid gets label ((t/tt)*nH + h/th)*nW + w/tw with nH = ceil(H/th),
+ * nW = ceil(W/tw); tiles at the far edges are partial when a tile size does not
+ * divide its axis.
+ *   labels     : device int32 (T*H*W), written.
+ *   n_clusters : host int, written with ceil(T/tt)*nH*nW (nullable).
+ * Errors: INVALID_ARG for non-positive sizes or a null labels pointer.
+ */
+int bsa_tile_labels(int T, int H, int W, int tt, int th, int tw, int32_t* labels,
+                    int* n_clusters, void* stream);
+
+/*
+ * antidiagonal_block_scores — [HMR] §XAttention — anti-diagonal block scoring,
+ * §Deviations (rows normalised to 1), §Out of scope (the caller pads S to a multiple
+ * of the block; padded keys take softmax mass).
+ *   A[I,J] = sum_{t<s} q[I*s+t] . k[J*s+s-1-t]        (stride x stride anti-diagonals)
+ *   P      = row-softmax(logit_scale * A) over all S/s columns
+ *   scores[b,h,i,j] = (s/block) * sum over the (block/s)^2 entries of tile (i,j)
+ * q: (B,Hq,S,D), k: (B,Hkv,S,D) with shape.Sq == shape.Sk == S; S % block == 0,
+ * block % stride == 0, block/stride <= 128, S/stride a multiple of 128,
+ * S/stride <= 8192; D in {64,128}; BSA_BF16 only. logit_scale <= 0 selects 1/sqrt(D).
+ *   scores : device float32 (B, Hq, S/block, S/block), written; each row sums to 1.
+ * The strided logit matrix is never written to device memory. No workspace.
+ */
+int bsa_antidiagonal_block_scores(const void* q, const void* k, bsa_shape shape, int block,
+                                  int stride, float logit_scale, float* scores, void* stream);
+
+/*
+ * top_p_block_mask — [HMR] §XAttention (each query block keeps the smallest set of
+ * key blocks whose mass reaches a fraction tau of its total), §Deviations (at least
+ * one block per row; key block 0 not forced), §What mlx-arsenal ships (scalar or
+ * per-head tau).
+ * Per row: sort scores descending (equal scores: lower key index first), take the
+ * running float32 sum in that order, keep ranks 0..m with m the first rank whose
+ * running sum >= tau[h]; if no running sum reaches tau the whole row is kept.
+ *   scores   : device float32 (B, H, Nq, Nk), Nk <= 1024.
+ *   tau      : device float32, n_tau == 1 (shared) or n_tau == H (per head).
+ *   mask     : device uint8 (B, H, Nq, Nk), written (1 = kept).
+ *   tie_rows : device uint8 (B, H, Nq) or NULL; 1 where a running sum lies within
+ *              1e-5 of tau or the last kept and first dropped scores differ by at most
+ *              1e-5 (rows whose decision a different rounding could flip).
+ */
+int bsa_top_p_block_mask(const float* scores, int B, int H, int Nq, int Nk, const float* tau,
+                         int n_tau, uint8_t* mask, uint8_t* tie_rows, void* stream);
+
+/*
+ * centroid_compensated_attention — [SBC] §The problem (block-sparse attention over
+ * query/key clusters), §SVG-EAR — centroid compensation (every skipped key cluster c
+ * enters the same softmax as ONE term with logit scale*q.kbar_c + ln n_c and value
+ * vbar_c), §No LSE needed (equivalently one softmax over [K; Kbar]); [SPR] (Q, K, V
+ * permuted into group-major order; hard drop renormalises over kept keys).
+ *   q_labels : device int32 (Sq), values in [0, Cq).   k_labels: device int32 (Sk),
+ *              values in [0, Ck). Labels outside the range make the output undefined.
+ *   block_mask : device uint8 with element (b,h,a,c) at
+ *              b*mask_b_stride + h*mask_h_stride + a*Ck + c; a stride of 0
+ *              broadcasts (one mask for every batch and/or head).
+ *   scale    : logit scale, <= 0 selects 1/sqrt(D).
+ *   compensate : 1 = SVG-EAR compensation of skipped non-empty clusters;
+ *              0 = hard drop (a row with no kept key outputs 0).
+ *   out      : device float32 (B, Hq, Sq, D), written in original token order.
+ *   workspace: >= bsa_attention_workspace_bytes(shape, Cq, Ck) bytes.
+ * Centroids are arithmetic means per (batch, KV head, cluster), computed in fp32 and
+ * rounded to the MMA input type. Limits: D in {64,128}; Ck <= 16384; Cq <= 16384;
+ * Sk + 15*Ck <= 65536. BSA_F32 inputs are computed with kind::tf32 MMAs.
+ */
+size_t bsa_attention_workspace_bytes(bsa_shape shape, int Cq, int Ck);
+int bsa_centroid_compensated_attention(const void* q, const void* k, const void* v,
+                                       bsa_shape shape, const int32_t* q_labels, int Cq,
+                                       const int32_t* k_labels, int Ck,
+                                       const uint8_t* block_mask, int64_t mask_b_stride,
+                                       int64_t mask_h_stride, float scale, int compensate,
+                                       float* out, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
+/*
+ * select_probe_rows — [SBC] §What mlx-arsenal ships (round-robin over query clusters,
+ * weights |G_a| / m_a), §Deviations (middle-out member; weights normalised to sum 1);
+ * [SPR] (probes stratified across query groups and ordered by distance to the group
+ * centroid).
+ * Rows of each non-empty cluster are ranked: q == NULL -> middle-out (by
+ * |r - (n-1)/2| of the row's rank r inside its cluster, ties to the lower rank),
+ * shared by all heads; q != NULL -> per (batch, query head) by the Euclidean distance
+ * to the cluster's mean query (ties to the lower index). With C' non-empty clusters,
+ * M >= C' takes rank-p rows of every cluster in pass p until M rows are taken;
+ * M < C' takes the first-ranked row of cluster floor(i*C'/M) for probe i.
+ *   labels    : device int32 (S), values in [0, C).
+ *   probe_idx : device int32 (M) if q == NULL, else (B, Hq, M); written.
+ *   weights   : device float32, same shape; written, summing to 1 per head.
+ *   shape     : used when q != NULL (B, Hq, Sq == S, D, dtype).
+ * Limits: S <= 65536, C <= 16384, M <= 1024. Workspace:
+ * bsa_probe_select_workspace_bytes(S, C).
+ */
+size_t bsa_probe_select_workspace_bytes(int S, int C);
+int bsa_select_probe_rows(const int32_t* labels, int S, int C, int M, const void* q,
+                          bsa_shape shape, int32_t* probe_idx, float* weights, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
+ * probe_dense_attention — [SBC] §Recipe (exact attention of the probe rows over every
+ * key); [SPR] (M query rows evaluated exactly against all keys).
+ *   probe_idx : device int32 (M) shared (per_head == 0) or (B, Hq, M) (per_head == 1).
+ *   o_probe   : device float32 (B, Hq, M, D), written.
+ *   scale     : <= 0 selects 1/sqrt(D). M <= 1024. Workspace:
+ *               bsa_probe_attention_workspace_bytes(shape, M).
+ */
+size_t bsa_probe_attention_workspace_bytes(bsa_shape shape, int M);
+int bsa_probe_dense_attention(const void* q, const void* k, const void* v, bsa_shape shape,
+                              const int32_t* probe_idx, int M, int per_head, float scale,
+                              float* o_probe, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * probe_residual_correction — [SBC] §SparsePR — probe-fitted residual repair; [SPR]
+ * (weighted ridge affine fit, lambda = 0.1, from the standardised sparse output,
+ * projected on the top r = 16 residual directions, applied to all rows).
+ * Per (b, h), with X = out[b,h] (S x D), Z = (X - mu) / sqrt(var + 1e-6) (column mean
+ * and population variance over all S rows), Zt = [Z, 1], W = diag(weights):
+ *   R    = o_probe - X[probe_idx]
+ *   Bc   = (Zt_p^T W Zt_p + lam*diag(1,..,1,0))^-1 Zt_p^T W R   (Cholesky)
+ *   V_r  = top-`rank` eigenvectors of R^T W R                      (Jacobi)
+ *   out <- X + Zt * Bc * V_r V_r^T                                  (every row)
+ *   out       : device float32 (B, H, S, D), updated in place.
+ *   o_probe   : device float32 (B, H, M, D).
+ *   probe_idx, weights : (M) shared (per_head == 0) or (B, H, M).
+ * Limits: D in {64,128}, 1 <= rank <= D, M <= 1024. Workspace:
+ * bsa_repair_workspace_bytes(B, H, S, D, M).
+ */
+size_t bsa_repair_workspace_bytes(int B, int H, int S, int D, int M);
+int bsa_probe_residual_correction(float* out, const float* o_probe, const int32_t* probe_idx,
+                                  const float* weights, int per_head, int B, int H, int S, int D,
+                                  int M, int rank, float lam, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
+ * Per-head drift/anchor mask cache — [HMR] §HEART — head-wise temporal mask reuse
+ * (anchor = token means qbar, kbar and the head's mask; drift = L1 distance; refresh
+ * above delta; layer gate: under gate_lo of the heads -> none, above gate_hi -> all),
+ * §Deviations (relative drift divides by the anchor's L1 norm), §Recipe (every head
+ * refreshes on the first call), "Reuse needs a fixed token grid" (reset on a grid
+ * change).
+ * State lives in a caller-owned device buffer of bsa_mask_cache_state_bytes() bytes;
+ * it can be saved and restored like any tensor. One cache per layer and CFG branch.
+ */
+size_t bsa_mask_cache_state_bytes(int B, int H, int Cq, int Ck, int D);
+/* Initialises the state (empty cache). gate_lo < 0 disables the layer gate. */
+int bsa_mask_cache_init(void* state, int B, int H, int Cq, int Ck, int D, float delta,
+                        int relative, float gate_lo, float gate_hi, void* stream);
+/*
+ * Pools q, k (B,H,S,D; Hkv must equal H) into per-head means, computes the drift
+ * against the anchors, applies delta and the layer gate, and writes refresh
+ * (device uint8 (B,H)). If n_refresh_host is non-NULL the stream is synchronised and
+ * the number of refreshed heads is written there. drift_out (nullable) receives the
+ * float32 (B,H) drift (+inf where no anchor exists yet).
+ */
+int bsa_mask_cache_should_refresh(void* state, const void* q, const void* k, bsa_shape shape,
+                                  uint8_t* refresh, float* drift_out, int* n_refresh_host,
+                                  void* stream);
+/*
+ * Replaces the cached mask of every refreshed head by new_mask (device uint8
+ * (B,H,Cq,Ck); may be NULL when no head refreshes), moves those heads' anchors to the
+ * pooled values of the last should_refresh, and writes the resulting mask to
+ * block_mask_out (device uint8 (B,H,Cq,Ck)).
+ */
+int bsa_mask_cache_update(void* state, const uint8_t* new_mask, const uint8_t* refresh,
+                          uint8_t* block_mask_out, void* stream);
+/* Forgets anchors and masks: the next should_refresh refreshes every head. */
+int bsa_mask_cache_reset(void* state, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H_ */

@@ -1,0 +1,141 @@
+"""GPU parity: libbsa centroid-compensated / hard-drop attention vs the float64 oracle.
+
+Tolerances (bf16 or fp32 inputs, fp32 accumulation): max-abs error <= 2e-2 and
+relative Frobenius error <= 5e-3 against the oracle on the same input values.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_tcgen05_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_FRO = 5e-3
+
+
+def _bsa():
+    import block_sparse_attention_tcgen05_b200 as bsa
+    return bsa
+
+
+def _check(got, ref, max_abs=MAX_ABS, rel=REL_FRO):
+    got = np.asarray(got, dtype=np.float64)
+    err = np.abs(got - ref)
+    fro = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert np.isfinite(got).all()
+    assert err.max() <= max_abs, f"max-abs {err.max():.3e}"
+    assert fro <= rel, f"rel-fro {fro:.3e}"
+    return err.max(), fro
+
+
+def _run(q, k, v, ql, kl, mask, Cq, Ck, compensate=True):
+    bsa = _bsa()
+    dev = torch.device("cuda")
+    out = bsa.centroid_compensated_attention(
+        q.to(dev), k.to(dev), v.to(dev), torch.as_tensor(ql, dtype=torch.int32, device=dev),
+        torch.as_tensor(kl, dtype=torch.int32, device=dev),
+        torch.as_tensor(np.asarray(mask), dtype=torch.uint8, device=dev), Cq=Cq, Ck=Ck,
+        compensate=compensate)
+    torch.cuda.synchronize()
+    assert bsa.device_status()[0] == 0
+    return out.cpu().numpy()
+
+
+def _ref(q, k, v, ql, kl, mask, Cq, Ck, compensate=True, rows=None):
+    return oracle.centroid_compensated_attention(
+        q.double().numpy(), k.double().numpy(), v.double().numpy(), ql, kl, mask,
+        compensate=compensate, rows=rows, Cq=Cq, Ck=Ck)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("compensate", [True, False])
+def test_tiny_workload(dtype, compensate):
+    """B=1, H=2, S=1024, D=64, labels arange//64, 25 % random cluster mask (diagonal
+    kept, seed 0)."""
+    q, k, v = wl.gaussian_qkv(1, 2, 2, 1024, 64, dtype, seed=0)
+    lab = np.arange(1024) // 64
+    mask = wl.random_cluster_mask(16, 0.25, seed=0)
+    got = _run(q, k, v, lab, lab, mask, 16, 16, compensate)
+    _check(got, _ref(q, k, v, lab, lab, mask, 16, 16, compensate))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_ragged_uneven_clusters_gqa_per_head_mask(D):
+    """S not a multiple of 128, shuffled labels with uneven sizes (some not multiples
+    of 16), Cq != Ck, an empty key cluster, per-head masks, GQA 4:2."""
+    g = np.random.default_rng(1)
+    S, Cq, Ck = 1000, 11, 13
+    ql = g.permutation(np.concatenate([np.arange(Cq), g.integers(0, Cq, S - Cq)]))
+    kl = g.permutation(np.concatenate([np.arange(Ck - 1), g.integers(0, Ck - 1, S - Ck + 1)]))
+    mask = g.random((4, Cq, Ck)) < 0.3
+    q, k, v = wl.gaussian_qkv(1, 4, 2, S, D, "bf16", seed=2)
+    for comp in (True, False):
+        got = _run(q, k, v, ql, kl, mask, Cq, Ck, comp)
+        _check(got, _ref(q, k, v, ql, kl, mask, Cq, Ck, comp))
+
+
+def test_one_key_per_cluster_equals_dense():
+    q, k, v = wl.gaussian_qkv(1, 2, 2, 384, 64, "bf16", seed=3)
+    ql = np.arange(384) // 128
+    kl = np.random.default_rng(4).permutation(384)
+    mask = np.random.default_rng(5).random((3, 384)) < 0.2
+    got = _run(q, k, v, ql, kl, mask, 3, 384)
+    dense = oracle.dense_attention(q.double().numpy(), k.double().numpy(), v.double().numpy())
+    _check(got, dense)
+
+
+def test_all_kept_equals_dense_and_batch():
+    q, k, v = wl.gaussian_qkv(2, 2, 1, 640, 128, "bf16", seed=6)
+    lab = np.arange(640) // 80
+    mask = np.ones((8, 8), dtype=bool)
+    for comp in (True, False):
+        got = _run(q, k, v, lab, lab, mask, 8, 8, comp)
+        _check(got, oracle.dense_attention(q.double().numpy(), k.double().numpy(),
+                                           v.double().numpy()))
+
+
+def test_all_skipped_rows_hard_drop_zero():
+    q, k, v = wl.gaussian_qkv(1, 1, 1, 256, 64, "bf16", seed=7)
+    lab = np.arange(256) // 64
+    mask = np.eye(4, dtype=bool)
+    mask[2, 2] = False  # query cluster 2 keeps nothing
+    got = _run(q, k, v, lab, lab, mask, 4, 4, compensate=False)
+    assert np.abs(got[0, 0, 128:192]).max() == 0.0
+    _check(got, _ref(q, k, v, lab, lab, mask, 4, 4, False))
+    got = _run(q, k, v, lab, lab, mask, 4, 4, compensate=True)
+    _check(got, _ref(q, k, v, lab, lab, mask, 4, 4, True))
+
+
+def test_dynamic_mask_workload_shape():
+    """B=1, H=8, S=8192, D=64 bf16 with 1-D positional structure; block labels
+    arange//128; a random per-head block mask at ~20 % with the diagonal kept."""
+    q, k, v, _ = wl.positional_qkv(1, 8, 8, (8192,), 64, ell=(256.0,), amp=2.0, dtype="bf16",
+                                   seed=2)
+    lab = np.arange(8192) // 128
+    mask = np.stack([wl.random_cluster_mask(64, 0.2, seed=10 + h) for h in range(8)])
+    rows = np.random.default_rng(11).choice(8192, 512, replace=False)
+    got = _run(q, k, v, lab, lab, mask, 64, 64)
+    ref = _ref(q, k, v, lab, lab, mask, 64, 64, rows=rows)
+    _check(got[:, :, rows], ref)
+
+
+def test_video_static_tiles_full_size_sampled():
+    """B=1, H=40, S=32760 (21x30x52), D=128, 3x6x8 tiles (245 clusters of 144 / 72
+    tokens), nearest-22 % tile-pair mask; sampled rows of every head vs the oracle."""
+    bsa = _bsa()
+    grid, tile = (21, 30, 52), (3, 6, 8)
+    q, k, v, _ = wl.positional_qkv(1, 40, 40, grid, 128, ell=(3.0, 6.0, 8.0), amp=2.0,
+                                   dtype="bf16", seed=3)
+    labels_gpu, C = bsa.tile_labels(*grid, tile)
+    lab_ref, C_ref = oracle.tile_labels(*grid, tile)
+    assert C == C_ref == 245
+    np.testing.assert_array_equal(labels_gpu.cpu().numpy(), lab_ref)
+    mask = wl.nearest_pair_mask(wl.tile_centroids(grid, tile), 0.22)
+    got = _run(q, k, v, lab_ref, lab_ref, mask, C, C)
+    rows = np.random.default_rng(12).choice(32760, 96, replace=False)
+    ref = _ref(q, k, v, lab_ref, lab_ref, mask, C, C, rows=rows)
+    _check(got[:, :, rows], ref)
