@@ -8,8 +8,14 @@ current CUDA stream. It has no CPU fallback; a missing library raises.
 
 from ._lib import BsaError, load as load_library  # noqa: F401
 from .ops import (  # noqa: F401
+    MaskCache,
+    antidiagonal_block_scores,
     attention_workspace_bytes,
     centroid_compensated_attention,
     device_status,
+    probe_dense_attention,
+    probe_residual_correction,
+    select_probe_rows,
     tile_labels,
+    top_p_block_mask,
 )

@@ -45,7 +45,7 @@ SIGNATURES = {
     "bsa_attention_workspace_bytes": (_sz, [Shape, _i, _i]),
     "bsa_centroid_compensated_attention": (
         _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _vp, _i64, _i64, _f, _i, _vp, _vp, _sz, _vp]),
-    "bsa_probe_select_workspace_bytes": (_sz, [_i, _i]),
+    "bsa_probe_select_workspace_bytes": (_sz, [_i, _i, _i]),
     "bsa_select_probe_rows": (_i, [_vp, _i, _i, _i, _vp, Shape, _vp, _vp, _vp, _sz, _vp]),
     "bsa_probe_attention_workspace_bytes": (_sz, [Shape, _i]),
     "bsa_probe_dense_attention": (_i, [_vp, _vp, _vp, Shape, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),

@@ -515,8 +515,9 @@ __global__ void __launch_bounds__(192, 2)
       int gcur = 0, ccur = 0, j = 0;
       Chunk ch;
       while (ok && next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
-        // S (and P, which aliases it) is free once the previous PV has completed.
-        if (j > 0 && !(ok = mbar_wait(BAR(BAR_VE), (j - 1) & 1, abort_flag, 4))) break;
+        // S is overwritten while the previous PV may still be queued: tcgen05.mma
+        // operations of one thread execute in issue order, so PV_{j-1} has read P_{j-1}
+        // before QK_j writes the same columns.
         if (!(ok = mbar_wait(BAR(BAR_KF), j & 1, abort_flag, 5))) break;
         tc_fence_after();
         const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(ch.n >> 3) << 17);
@@ -566,56 +567,74 @@ __global__ void __launch_bounds__(192, 2)
       if (!(ok = mbar_wait(BAR(BAR_SF), j & 1, abort_flag, 9))) break;
       tc_fence_after();
       const int npc = (ch.n + 31) >> 5;
-      float s[128];
+      // Logits of this chunk: a full chunk that every row of the tile keeps is used
+      // raw, scale·log2(e) folded into the FFMA feeding ex2; any other chunk gets its
+      // per-row column mask (kept groups, real keys, or skipped non-empty clusters)
+      // and, for centroid chunks, the log2(n_c) bias.
+      const bool fast = ch.uniform && ch.n == 128 && lab >= 0;
+      uint32_t mk[4] = {0u, 0u, 0u, 0u};
+      if (!fast && lab >= 0) {
+        if (ch.centroid) {
 #pragma unroll
-      for (int p = 0; p < 4; ++p)
-        if (p < npc) tmem_ld32(tS + p * 32, *reinterpret_cast<float(*)[32]>(&s[p * 32]));
-      tmem_wait_ld();
-
-      uint32_t mk[4];
-      if (lab < 0) {
+          for (int w = 0; w < 4; ++w) {
+            const int ww = (ch.start >> 5) + w;
+            mk[w] = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
+          }
+        } else if (ch.uniform) {
 #pragma unroll
-        for (int w = 0; w < 4; ++w) mk[w] = 0;
-      } else if (ch.centroid) {
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int ww = (ch.start >> 5) + w;
-          mk[w] = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
-        }
-      } else if (ch.uniform) {
-#pragma unroll
-        for (int w = 0; w < 4; ++w) mk[w] = 0xffffffffu;
-      } else {
-#pragma unroll
-        for (int w = 0; w < 4; ++w) mk[w] = 0;
-        for (int jj = 0; jj < ch.ng; ++jj) {
-          const int g = ch.g0 + jj;
-          if ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u) {
-            const int nv = bit_at(a.gfull, g) ? 16 : __ldg(a.group_valid + g);
-            const uint32_t bits = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
-            mk[jj >> 1] |= bits << ((jj & 1) * 16);
+          for (int w = 0; w < 4; ++w) mk[w] = 0xffffffffu;
+        } else {
+          for (int jj = 0; jj < ch.ng; ++jj) {
+            const int g = ch.g0 + jj;
+            if ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u) {
+              const int nv = bit_at(a.gfull, g) ? 16 : __ldg(a.group_valid + g);
+              const uint32_t bits = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
+              mk[jj >> 1] |= bits << ((jj & 1) * 16);
+            }
           }
         }
-      }
-
-      float mx = -INFINITY;
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+        for (int w = 0; w < 4; ++w)
+          if (w * 32 + 32 > ch.n) mk[w] &= (w * 32 >= ch.n) ? 0u : (0xffffffffu >> (w * 32 + 32 - ch.n));
+      }
+      const float* bias = ch.centroid ? a.bias2 + ch.start : nullptr;
+      const float scl = a.scale_log2;
+
+      // Pass 1: chunk max (log2 units). Two 32-column loads in flight per wait.
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int p = 0; p < 4; p += 2) {
         if (p < npc) {
+          float t0[32], t1[32];
+          tmem_ld32(tS + p * 32, t0);
+          if (p + 1 < npc) tmem_ld32(tS + (p + 1) * 32, t1);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int col = p * 32 + c;
-            float x = s[col] * a.scale_log2;
-            if (ch.centroid) x += __ldg(a.bias2 + ch.start + col);
-            const bool keep = (col < ch.n) && ((mk[p] >> c) & 1u);
-            x = keep ? x : -INFINITY;
-            s[col] = x;
-            mx = fmaxf(mx, x);
+          for (int h = 0; h < 2; ++h) {
+            if (p + h < npc) {
+              const float* t = h ? t1 : t0;
+              const int pp = p + h;
+              if (fast) {
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                  mx0 = fmaxf(mx0, t[c]);
+                  mx1 = fmaxf(mx1, t[c + 1]);
+                }
+              } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                  const float add = bias ? __ldg(bias + pp * 32 + c) : 0.f;
+                  const float x = ((mk[pp] >> c) & 1u) ? fmaf(t[c], scl, add) : -INFINITY;
+                  if (c & 1) mx1 = fmaxf(mx1, x); else mx0 = fmaxf(mx0, x);
+                }
+              }
+            }
           }
         }
       }
+      const float mx = fast ? fmaxf(mx0, mx1) * scl : fmaxf(mx0, mx1);
       // Lazy rescaling: the running max only moves when the chunk max exceeds it by
-      // more than 2^8, so P stays below 256 and O is rarely touched.
+      // more than 8 (log2 units), so P stays below 256 and O is rarely touched.
       const bool need = mx > m_run + 8.f;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = need ? mx : m_run;
@@ -634,31 +653,49 @@ __global__ void __launch_bounds__(192, 2)
         l_run *= alpha;
         m_run = m_new;
       }
-      const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum = 0.f;
+      const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
+
+      // Pass 2: P = 2^(x - m), written over S in place (bf16 pairs: piece p of 32
+      // logits lands in columns [16p, 16p+16), which pass 2 has already read). The load
+      // of piece p+1 is in flight while piece p is exponentiated.
+      float sum0 = 0.f, sum1 = 0.f;
+      float buf[2][32];
+      tmem_ld32(tS, buf[0]);
+      tmem_wait_ld();
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         if (p < npc) {
+          float* t = buf[p & 1];
+          if (p + 1 < npc) tmem_ld32(tS + (p + 1) * 32, buf[(p + 1) & 1]);
+          if (fast) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float e = ex2(s[p * 32 + c] - mu);
-            sum += e;
-            s[p * 32 + c] = e;
+            for (int c = 0; c < 32; c += 2) {
+              t[c] = ex2(fmaf(t[c], scl, neg_mu));
+              t[c + 1] = ex2(fmaf(t[c + 1], scl, neg_mu));
+              sum0 += t[c];
+              sum1 += t[c + 1];
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float add = bias ? __ldg(bias + p * 32 + c) : 0.f;
+              const float e = ((mk[p] >> c) & 1u) ? ex2(fmaf(t[c], scl, add + neg_mu)) : 0.f;
+              t[c] = e;
+              if (c & 1) sum1 += e; else sum0 += e;
+            }
           }
+          if constexpr (TF32) {
+            tmem_st32(tS + p * 32, *reinterpret_cast<uint32_t(*)[32]>(t));
+          } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(t[2 * i], t[2 * i + 1]);
+            tmem_st16(tS + p * 16, pk);
+          }
+          tmem_wait_ld();
         }
       }
-      l_run += sum;
-      if constexpr (TF32) {
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-          if (p < npc) tmem_st32(tS + p * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[p * 32]));
-      } else {
-        uint32_t* pk = reinterpret_cast<uint32_t*>(s);
-#pragma unroll
-        for (int i = 0; i < 64; ++i) pk[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
-        if (ch.n > 64) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
-      }
+      l_run += sum0 + sum1;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(BAR_PF));

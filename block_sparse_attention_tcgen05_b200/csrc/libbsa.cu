@@ -2,3 +2,8 @@
 // kernel without relocatable device code.
 #include "common.cu"
 #include "attention.cu"
+#include "scoring.cu"
+#include "topp.cu"
+#include "probe.cu"
+#include "repair.cu"
+#include "cache.cu"

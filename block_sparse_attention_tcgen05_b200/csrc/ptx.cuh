@@ -13,7 +13,8 @@ __device__ int g_device_status = 0;
 __device__ int g_device_status_where = 0;
 
 constexpr int kStatusTimeout = -4;
-constexpr int kStatusBadLabel = -1;  // a label outside [0, C) was seen on the device
+constexpr int kStatusBadLabel = -1;     // a label or row index outside its range was seen
+constexpr int kStatusUnsupported = -2;  // a data-dependent size exceeded a kernel limit
 
 __device__ __forceinline__ void report_device_error(int code, int where) {
   if (atomicCAS(&g_device_status, 0, code) == 0) g_device_status_where = where;
@@ -215,6 +216,32 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* u) {
       "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
       "r"(u[15])
       : "memory");
+}
+
+// Stores N (1..32, power of two) consecutive 32-bit columns per lane.
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* u) {
+  if constexpr (N == 32) {
+    tmem_st32(taddr, *reinterpret_cast<const uint32_t(*)[32]>(u));
+  } else if constexpr (N == 16) {
+    tmem_st16(taddr, u);
+  } else if constexpr (N == 8) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]),
+                 "r"(u[7])
+                 : "memory");
+  } else if constexpr (N == 4) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
+                 "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3])
+                 : "memory");
+  } else if constexpr (N == 2) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(u[0]),
+                 "r"(u[1])
+                 : "memory");
+  } else {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(u[0])
+                 : "memory");
+  }
 }
 
 __device__ __forceinline__ void tmem_wait_ld() {

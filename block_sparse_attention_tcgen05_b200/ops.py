@@ -111,3 +111,124 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
          Cq, _ptr(k_labels), Ck, _ptr(m), bs, hs, float(scale or 0.0), 1 if compensate else 0,
          _ptr(out), _ptr(workspace), workspace.numel(), _stream(q.device))
     return out
+
+
+def antidiagonal_block_scores(q, k, block=128, stride=16, logit_scale=None):
+    """XAttention block-mass estimate: fp32 (B, Hq, S/block, S/block), rows sum to 1.
+    q: (B,Hq,S,D), k: (B,Hkv,S,D) bf16 with S a multiple of ``block`` (the caller pads)."""
+    _need_cuda(q, k)
+    B, Hq, S, D = q.shape
+    nb = S // block
+    scores = torch.empty((B, Hq, nb, nb), dtype=torch.float32, device=q.device)
+    call("bsa_antidiagonal_block_scores", _ptr(q), _ptr(k), make_shape(q, k), int(block),
+         int(stride), float(logit_scale or 0.0), _ptr(scores), _stream(q.device))
+    return scores
+
+
+def top_p_block_mask(scores, tau, return_ties=False):
+    """Per-row top-p selection over fp32 (B,H,Nq,Nk) scores; ``tau`` is a float or an
+    (H,) sequence/tensor. Returns a uint8 mask (and uint8 tie flags (B,H,Nq))."""
+    _need_cuda(scores)
+    B, H, Nq, Nk = scores.shape
+    t = torch.as_tensor(tau, dtype=torch.float32).reshape(-1).to(scores.device)
+    if t.numel() not in (1, H):
+        raise ValueError("tau must be a scalar or have H entries")
+    mask = torch.empty((B, H, Nq, Nk), dtype=torch.uint8, device=scores.device)
+    ties = torch.empty((B, H, Nq), dtype=torch.uint8, device=scores.device)
+    call("bsa_top_p_block_mask", _ptr(scores), B, H, Nq, Nk, _ptr(t), t.numel(), _ptr(mask),
+         _ptr(ties), _stream(scores.device))
+    return (mask, ties) if return_ties else mask
+
+
+def select_probe_rows(labels, C, M, q=None):
+    """SparsePR probe rows. Without ``q``: head-agnostic middle-out members, (M,) int32
+    indices and (M,) fp32 weights. With ``q`` (B,Hq,S,D): per-head members nearest to
+    their cluster's mean query, (B,Hq,M) indices and weights."""
+    _need_cuda(labels, q)
+    S = labels.shape[0]
+    dev = labels.device
+    if q is not None:
+        B, Hq = q.shape[:2]
+        shape = make_shape(q, q)
+        n_heads = B * Hq
+        idx = torch.empty((B, Hq, M), dtype=torch.int32, device=dev)
+        w = torch.empty((B, Hq, M), dtype=torch.float32, device=dev)
+    else:
+        shape = Shape(1, 1, 1, S, S, 64, BSA_BF16)
+        n_heads = 1
+        idx = torch.empty((M,), dtype=torch.int32, device=dev)
+        w = torch.empty((M,), dtype=torch.float32, device=dev)
+    need = _lib.load().bsa_probe_select_workspace_bytes(S, int(C), n_heads)
+    ws = _workspace(need, dev)
+    call("bsa_select_probe_rows", _ptr(labels), S, int(C), int(M), _ptr(q), shape, _ptr(idx),
+         _ptr(w), _ptr(ws), ws.numel(), _stream(dev))
+    return idx, w
+
+
+def probe_dense_attention(q, k, v, probe_idx, scale=None, workspace=None):
+    """Exact attention of the probe rows over every key: fp32 (B, Hq, M, D)."""
+    _need_cuda(q, k, v, probe_idx)
+    B, Hq, S, D = q.shape
+    per_head = 1 if probe_idx.dim() == 3 else 0
+    M = probe_idx.shape[-1]
+    shape = make_shape(q, k)
+    out = torch.empty((B, Hq, M, v.shape[-1]), dtype=torch.float32, device=q.device)
+    need = _lib.load().bsa_probe_attention_workspace_bytes(shape, int(M))
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, q.device)
+    call("bsa_probe_dense_attention", _ptr(q), _ptr(k), _ptr(v), shape, _ptr(probe_idx), int(M),
+         per_head, float(scale or 0.0), _ptr(out), _ptr(workspace), workspace.numel(),
+         _stream(q.device))
+    return out
+
+
+def probe_residual_correction(out, o_probe, probe_idx, weights, rank=16, lam=0.1, workspace=None):
+    """SparsePR repair of ``out`` (fp32 (B,H,S,D), updated in place and returned)."""
+    _need_cuda(out, o_probe, probe_idx, weights)
+    B, H, S, D = out.shape
+    M = probe_idx.shape[-1]
+    per_head = 1 if probe_idx.dim() == 3 else 0
+    need = _lib.load().bsa_repair_workspace_bytes(B, H, S, D, int(M))
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, out.device)
+    call("bsa_probe_residual_correction", _ptr(out), _ptr(o_probe), _ptr(probe_idx), _ptr(weights),
+         per_head, B, H, S, D, int(M), int(rank), float(lam), _ptr(workspace), workspace.numel(),
+         _stream(out.device))
+    return out
+
+
+class MaskCache:
+    """HEART per-head drift/anchor mask cache; its state is one device byte buffer."""
+
+    def __init__(self, B, H, Cq, Ck, D, delta, relative=False, gate_lo=0.4, gate_hi=0.8,
+                 device="cuda"):
+        self.shape = (B, H, Cq, Ck, D)
+        n = _lib.load().bsa_mask_cache_state_bytes(B, H, Cq, Ck, D)
+        self.state = torch.empty(n, dtype=torch.uint8, device=device)
+        self.refresh = torch.empty((B, H), dtype=torch.uint8, device=device)
+        self.drift = torch.empty((B, H), dtype=torch.float32, device=device)
+        self.mask = torch.empty((B, H, Cq, Ck), dtype=torch.uint8, device=device)
+        call("bsa_mask_cache_init", _ptr(self.state), B, H, Cq, Ck, D, float(delta),
+             1 if relative else 0, float(gate_lo), float(gate_hi), _stream(self.state.device))
+
+    def should_refresh(self, q, k, sync=True):
+        """Device uint8 (B,H) refresh flags; with ``sync`` also the host count."""
+        _need_cuda(q, k)
+        n = ctypes.c_int(0)
+        call("bsa_mask_cache_should_refresh", _ptr(self.state), _ptr(q), _ptr(k), make_shape(q, k),
+             _ptr(self.refresh), _ptr(self.drift), ctypes.byref(n) if sync else None,
+             _stream(q.device))
+        return (self.refresh, n.value) if sync else self.refresh
+
+    def update(self, new_mask):
+        """Cached mask with the refreshed heads replaced by ``new_mask`` (or None)."""
+        nm = None
+        if new_mask is not None:
+            nm = new_mask.to(torch.uint8).contiguous()
+            _need_cuda(nm)
+        call("bsa_mask_cache_update", _ptr(self.state), _ptr(nm), _ptr(self.refresh),
+             _ptr(self.mask), _stream(self.state.device))
+        return self.mask
+
+    def reset(self):
+        call("bsa_mask_cache_reset", _ptr(self.state), _stream(self.state.device))

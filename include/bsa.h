@@ -165,10 +165,12 @@ int bsa_centroid_compensated_attention(const void* q, const void* k, const void*
  *   probe_idx : device int32 (M) if q == NULL, else (B, Hq, M); written.
  *   weights   : device float32, same shape; written, summing to 1 per head.
  *   shape     : used when q != NULL (B, Hq, Sq == S, D, dtype).
- * Limits: S <= 65536, C <= 16384, M <= 1024. Workspace:
- * bsa_probe_select_workspace_bytes(S, C).
+ * Limits: S <= 65536, C <= 16384, M <= 1024; with q, clusters of at most 4096 rows
+ * (a larger cluster keeps index order and records BSA_ERR_UNSUPPORTED in the device
+ * status). Workspace: bsa_probe_select_workspace_bytes(S, C, n_heads) with
+ * n_heads = B*Hq when q != NULL, else 1.
  */
-size_t bsa_probe_select_workspace_bytes(int S, int C);
+size_t bsa_probe_select_workspace_bytes(int S, int C, int n_heads);
 int bsa_select_probe_rows(const int32_t* labels, int S, int C, int M, const void* q,
                           bsa_shape shape, int32_t* probe_idx, float* weights, void* workspace,
                           size_t workspace_bytes, void* stream);
@@ -176,7 +178,9 @@ int bsa_select_probe_rows(const int32_t* labels, int S, int C, int M, const void
 /*
  * probe_dense_attention — [SBC] §Recipe (exact attention of the probe rows over every
  * key); [SPR] (M query rows evaluated exactly against all keys).
- *   probe_idx : device int32 (M) shared (per_head == 0) or (B, Hq, M) (per_head == 1).
+ *   probe_idx : device int32 (M) shared (per_head == 0) or (B, Hq, M) (per_head == 1);
+ *               an index outside [0, S) reads a zero row and records
+ *               BSA_ERR_INVALID_ARG in the device status.
  *   o_probe   : device float32 (B, Hq, M, D), written.
  *   scale     : <= 0 selects 1/sqrt(D). M <= 1024. Workspace:
  *               bsa_probe_attention_workspace_bytes(shape, M).

@@ -1,0 +1,95 @@
+"""GPU parity: anti-diagonal block scores and top-p masks vs the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_tcgen05_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+SCORE_ATOL = 1e-4   # fp32 accumulation of bf16 products vs float64 on the same values
+
+
+def _bsa():
+    import block_sparse_attention_tcgen05_b200 as bsa
+    return bsa
+
+
+def _scores(q, k, block, stride):
+    bsa = _bsa()
+    sc = bsa.antidiagonal_block_scores(q.cuda(), k.cuda(), block=block, stride=stride)
+    torch.cuda.synchronize()
+    assert bsa.device_status()[0] == 0
+    return sc.cpu().numpy()
+
+
+@pytest.mark.parametrize("D,stride,block", [(64, 16, 128), (128, 16, 128), (64, 8, 64), (128, 4, 128)])
+def test_scores_small(D, stride, block):
+    S = 128 * stride * 2  # two strided query tiles
+    q, k, _ = wl.gaussian_qkv(1, 2, 2, S, D, "bf16", seed=D + stride)
+    got = _scores(q, k, block, stride)
+    ref = oracle.antidiagonal_block_scores(q.double().numpy(), k.double().numpy(), block, stride)
+    np.testing.assert_allclose(got, ref, atol=SCORE_ATOL, rtol=0)
+    np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-4)
+
+
+def test_scores_gqa():
+    q, k, _ = wl.gaussian_qkv(1, 4, 2, 4096, 64, "bf16", seed=5)
+    got = _scores(q, k, 128, 16)
+    ref = oracle.antidiagonal_block_scores(q.double().numpy(), k.double().numpy(), 128, 16)
+    np.testing.assert_allclose(got, ref, atol=SCORE_ATOL, rtol=0)
+
+
+def test_top_p_kernel_bit_exact_on_identical_scores():
+    """Same float32 scores on both sides, decisions in float32 in the same order."""
+    g = np.random.default_rng(0)
+    sc = g.dirichlet(np.ones(64) * 0.3, size=(2, 3, 64)).astype(np.float32)
+    tau = np.array([0.85, 0.9, 0.95], dtype=np.float32)
+    bsa = _bsa()
+    got, ties = bsa.top_p_block_mask(torch.from_numpy(sc).cuda(), torch.from_numpy(tau),
+                                     return_ties=True)
+    ref, _ = oracle.top_p_block_mask(sc, tau, dtype=np.float32)
+    np.testing.assert_array_equal(got.cpu().numpy().astype(bool), ref)
+    # ragged Nk (not a power of two), scalar tau
+    sc2 = g.dirichlet(np.ones(245), size=(1, 2, 7)).astype(np.float32)
+    got2 = bsa.top_p_block_mask(torch.from_numpy(sc2).cuda(), 0.9)
+    ref2, _ = oracle.top_p_block_mask(sc2, 0.9, dtype=np.float32)
+    np.testing.assert_array_equal(got2.cpu().numpy().astype(bool), ref2)
+    assert (got2.cpu().numpy().sum(-1) >= 1).all()
+
+
+def test_dynamic_mask_workload_scores_and_masks():
+    """B=1, H=8, S=8192, D=64 bf16 with 1-D positional structure; block 128, stride 16,
+    tau 0.9. Masks must match the float64 oracle chain bit for bit outside tie rows."""
+    bsa = _bsa()
+    q, k, _, _ = wl.positional_qkv(1, 8, 8, (8192,), 64, ell=(256.0,), amp=2.0, dtype="bf16",
+                                   seed=2)
+    got = _scores(q, k, 128, 16)
+    ref = oracle.antidiagonal_block_scores(q.double().numpy(), k.double().numpy(), 128, 16)
+    np.testing.assert_allclose(got, ref, atol=SCORE_ATOL, rtol=0)
+    m_gpu = bsa.top_p_block_mask(torch.from_numpy(got).cuda(), 0.9).cpu().numpy().astype(bool)
+    m_ref, tie = oracle.top_p_block_mask(ref, 0.9)
+    diff_rows = (m_gpu != m_ref).any(-1)
+    assert not (diff_rows & ~tie).any(), f"{int((diff_rows & ~tie).sum())} non-tie rows differ"
+    print(f"tie rows {int(tie.sum())}, differing rows {int(diff_rows.sum())}, density "
+          f"{m_gpu.mean():.3f}")
+
+
+def test_video_reuse_workload_scores_sampled_heads():
+    """B=1, H=40, S=32760 padded to 32768 (XAttention pads with zeros), D=128, block 128,
+    stride 16; heads 0 and 39 against the oracle."""
+    grid = (21, 30, 52)
+    q, k, _, _ = wl.positional_qkv(1, 40, 40, grid, 128, ell=(3.0, 6.0, 8.0), amp=2.0,
+                                   dtype="bf16", seed=5)
+    pad = torch.zeros(1, 40, 8, 128, dtype=torch.bfloat16)
+    qp = torch.cat([q, pad], 2).contiguous()
+    kp = torch.cat([k, pad], 2).contiguous()
+    got = _scores(qp, kp, 128, 16)
+    assert got.shape == (1, 40, 256, 256)
+    np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-4)
+    for h in (0, 39):
+        ref = oracle.antidiagonal_block_scores(qp[:, h:h + 1].double().numpy(),
+                                               kp[:, h:h + 1].double().numpy(), 128, 16)
+        np.testing.assert_allclose(got[:, h:h + 1], ref, atol=SCORE_ATOL, rtol=0)
