@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention hot path on B200.
+
+Workload: the video-DiT shape with static tiles — B=1, H=40, S=32760 tokens on a
+21 x 30 x 52 latent grid, D=128, bf16 Q/K/V with a 3-D positional structure; labels
+from 3 x 6 x 8 sliding tiles (245 clusters); the tile-level mask keeps the 22 % of
+tile pairs nearest in (t, h, w); skipped tiles are centroid-compensated.
+One step = tile_labels + centroid_compensated_attention (label sort, Q gather, K/V
+gather with centroids, mask bitsets, fused tcgen05 attention) over one batch.
+
+Metric: effective TFLOP/s on executed pairs (4·D FLOP per token pair inside kept
+blocks; centroid terms not counted), with ms per call and % of the measured bf16
+tensor peak. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own copy of the workload (weak scaling: the path
+shards by heads and needs no collective); the step time is the max over ranks.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+GRID = (21, 30, 52)
+TILE = (3, 6, 8)
+H = 40
+D = 128
+DENSITY = 0.22
+WORKLOAD = ("video_static_tiles: B=1 H=40 S=32760 (21x30x52) D=128 bf16, 3x6x8 tile labels "
+            "(245 clusters), nearest-22% tile-pair mask, SVG-EAR compensation")
+METRIC = "effective TFLOP/s on executed pairs, centroid-compensated block-sparse attention at 40x32760x128"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="bounded CPU work for the oracle baseline")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--heads", type=int, default=H,
+                   help="number of heads (default 40; smaller only for profiler captures)")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return m, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def attention_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "block_sparse_attention_tcgen05_b200", "csrc")
+    for name in ("attention.cu", "ptx.cuh"):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
+    or None when the kernel source changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_sha") != attention_source_hash():
+        return None
+    return rec.get("bytes_per_launch_full_workload")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        self.file.close()
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(q, k, v, labels, mask, seconds):
+    """The oracle, as it stands, on the host cores over a bounded sample of the same
+    workload: head 0, query rows in chunks of 512 until ``seconds`` of work."""
+    import numpy as np
+
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    qd = q[:, :1].double().cpu().numpy()
+    kd = k[:, :1].double().cpu().numpy()
+    vd = v[:, :1].double().cpu().numpy()
+    lab = labels.cpu().numpy().astype(np.int64)
+    m = mask.cpu().numpy().astype(bool)
+    cnt = np.bincount(lab, minlength=m.shape[1])
+    kept_keys = (m[lab].astype(np.int64) * cnt[None, :]).sum(1)  # per query row
+    order = np.random.default_rng(0).permutation(len(lab))
+    t0 = time.perf_counter()
+    done, pairs = 0, 0
+    while done < len(order) and time.perf_counter() - t0 < seconds:
+        rows = np.sort(order[done:done + 512])
+        oracle.centroid_compensated_attention(qd, kd, vd, lab, lab, m, rows=rows,
+                                              Cq=m.shape[0], Ck=m.shape[1])
+        pairs += int(kept_keys[rows].sum())
+        done += len(rows)
+    dt = time.perf_counter() - t0
+    return {"value": pairs * 4 * D / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"head 0, {done} of {len(lab)} query rows (random, in chunks of 512), "
+                      f"{pairs:.3e} executed pairs in {dt:.1f} s, float64 NumPy",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank):
+    """--impl reference: the oracle on the host cores, each step a bounded sample."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from block_sparse_attention_tcgen05_b200 import workloads as wl
+    q, k, v, _ = wl.positional_qkv(1, 1, 1, GRID, D, ell=(3.0, 6.0, 8.0), amp=2.0, dtype="bf16",
+                                   seed=3)
+    lab, C = oracle.tile_labels(*GRID, TILE)
+    mask = wl.nearest_pair_mask(wl.tile_centroids(GRID, TILE), DENSITY)
+    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+    cnt = np.bincount(lab, minlength=C)
+    kept_keys = (mask[lab].astype(np.int64) * cnt[None, :]).sum(1)
+    rng = np.random.default_rng(1)
+    per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    times, pair_counts = [], []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        pairs = 0
+        while time.perf_counter() - t0 < per_step:
+            rows = np.sort(rng.choice(len(lab), 256, replace=False))
+            oracle.centroid_compensated_attention(qd, kd, vd, lab, lab, mask, rows=rows, Cq=C, Ck=C)
+            pairs += int(kept_keys[rows].sum())
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+            pair_counts.append(pairs)
+    value = sum(pair_counts) * 4 * D / sum(times) / 1e12
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_per_step": "random 256-row chunks of head 0 "
+                   f"for ~{per_step:.1f} s"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"head 0 of 40, random query rows, {sum(pair_counts):.3e} "
+                                   "executed pairs over the timed steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import ctypes
+
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_tcgen05_b200 as bsa
+    from block_sparse_attention_tcgen05_b200 import _lib
+    from block_sparse_attention_tcgen05_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    lib = _lib.load()
+
+    # ---------------------------------------------------------------- inputs (HBM-resident)
+    nh = args.heads
+    q, k, v = wl.positional_qkv_device(1, nh, nh, GRID, D, ell=(3.0, 6.0, 8.0), amp=2.0,
+                                       seed=3 + 1000 * rank, device=dev)
+    labels, C = bsa.tile_labels(*GRID, TILE, device=dev)
+    mask = torch.as_tensor(wl.nearest_pair_mask(wl.tile_centroids(GRID, TILE), DENSITY),
+                           dtype=torch.uint8, device=dev)
+    cnt = torch.bincount(labels.long(), minlength=C).double()
+    pairs = float(cnt @ mask.double() @ cnt) * nh
+    S = q.shape[2]
+    flop = pairs * 4 * D
+    ws = torch.empty(bsa.attention_workspace_bytes(q, k, C, C), dtype=torch.uint8, device=dev)
+    out = torch.empty((1, nh, S, D), dtype=torch.float32, device=dev)
+
+    def step():
+        lab, _ = bsa.tile_labels(*GRID, TILE, device=dev)
+        bsa.centroid_compensated_attention(q, k, v, lab, lab, mask, Cq=C, Ck=C, out=out, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, _ = bsa.device_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    # ---------------------------------------------------------------- timed region
+    _lib.call("bsa_profile_enable", args.steps)
+    uuid = getattr(torch.cuda.get_device_properties(dev), "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    n0 = lib.bsa_launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    launches = int(lib.bsa_launch_count() - n0)
+    ms = e0.elapsed_time(e1) / args.steps
+    attn_ms = ctypes.c_float(0.0)
+    attn_n = ctypes.c_int(0)
+    _lib.call("bsa_profile_read", 0, ctypes.byref(attn_ms), ctypes.byref(attn_n))
+    _lib.call("bsa_profile_enable", 0)
+    attn_ms_launch = attn_ms.value / max(1, attn_n.value)
+    if world > 1:
+        t = torch.tensor([ms, attn_ms_launch], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, attn_ms_launch = float(t[0]), float(t[1])
+    st, _ = bsa.device_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the timed region")
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        mh = mask.cpu().pin_memory()
+        oh = torch.empty((1, nh, S, D), dtype=torch.float32).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        md = torch.empty_like(mask)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            md.copy_(mh, non_blocking=True)
+            lab, _ = bsa.tile_labels(*GRID, TILE, device=dev)
+            bsa.centroid_compensated_attention(qd, kd, vd, lab, lab, md, Cq=C, Ck=C, out=out,
+                                               workspace=ws)
+            oh.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = a.elapsed_time(b) / args.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, mh))
+        d2h = oh.numel() * oh.element_size()
+        e2e = {"value": world * flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "block_sparse_attention_tcgen05_b200.centroid_compensated_attention"}
+        del qh, kh, vh, oh, qd, kd, vd
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(q, k, v, labels, mask, args.cpu_seconds)
+
+    if rank == 0:
+        peaks, src = measured_peaks()
+        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        achieved = flop / (attn_ms_launch * 1e-3) / 1e12
+        line = {
+            "metric": METRIC,
+            "value": world * flop / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "ms_per_call": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "pct_of_bf16_peak": 100.0 * (flop / (ms * 1e-3) / 1e12) / peak,
+            "config": {
+                "workload": WORKLOAD,
+                "B": 1, "H": nh, "S": S, "D": D, "clusters": C,
+                "executed_pairs_per_call": pairs,
+                "executed_pair_density": pairs / (nh * S * S),
+                "flop_per_call": flop,
+                "l2": "inputs larger than L2 (Q+K+V = %.2f GB per rank)" % (
+                    3 * q.numel() * 2 / 1e9),
+                "parallelism": "replicas x%d (weak, no collective on the data path)" % world,
+            },
+            "roofline": {
+                "kernel": "attn_kernel<128,bf16>",
+                "bound": "tensor",
+                "achieved": achieved,
+                "peak": peak,
+                "peak_source": f"bf16_tflops_sustained of {src} (MEASURED_PEAKS.json)"
+                if src == "measured" else "fallback sustained bf16",
+                "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "traffic": recorded_traffic(),
+                "ms_per_launch": attn_ms_launch,
+            },
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -39,6 +39,9 @@ SIGNATURES = {
     "bsa_last_error_detail": (None, [ctypes.c_char_p, _sz]),
     "bsa_version": (_i, []),
     "bsa_get_device_status": (_i, [_vp, _ip]),
+    "bsa_launch_count": (ctypes.c_longlong, []),
+    "bsa_profile_enable": (_i, [_i]),
+    "bsa_profile_read": (_i, [_i, ctypes.POINTER(ctypes.c_float), _ip]),
     "bsa_tile_labels": (_i, [_i, _i, _i, _i, _i, _i, _vp, _ip, _vp]),
     "bsa_antidiagonal_block_scores": (_i, [_vp, _vp, Shape, _i, _i, _f, _vp, _vp]),
     "bsa_top_p_block_mask": (_i, [_vp, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),

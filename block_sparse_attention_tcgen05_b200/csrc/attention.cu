@@ -779,13 +779,17 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
 }
 
 template <int D, bool TF32>
-int launch_attn(const CUtensorMap* maps, const AttnArgs& args, dim3 grid, cudaStream_t st) {
+int launch_attn(const CUtensorMap* maps, const AttnArgs& args, dim3 grid, int prof_id,
+                cudaStream_t st) {
   using Cfg = AttnCfg<D, TF32>;
   auto kern = attn_kernel<D, TF32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::SMEM_LAUNCH);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attn_kernel)");
+  prof_begin(prof_id, st);
   kern<<<grid, 192, Cfg::SMEM_LAUNCH, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
+  count_launch();
+  prof_end(prof_id, st);
   return check_cuda(cudaGetLastError(), "attn_kernel launch");
 }
 
@@ -821,6 +825,7 @@ int run_label_sort(const int32_t* labels, int S, int C, int cluster_pad, int n_s
   label_sort_kernel<<<1, 1024, smem, st>>>(labels, S, C, cluster_pad, n_slots, slot_token,
                                            slot_label, count, off, group_cluster, group_valid,
                                            n_groups, bias2, C_pad, nonempty);
+  count_launch();
   return check_cuda(cudaGetLastError(), "label_sort_kernel launch");
 }
 
@@ -828,10 +833,10 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
                                    const bsa_shape& s, const int32_t* q_labels, int Cq,
                                    const int32_t* k_labels, int Ck, const uint8_t* mask,
                                    int64_t mbs, int64_t mhs, float scale, int compensate,
-                                   float* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+                                   float* out, void* ws, size_t ws_bytes, cudaStream_t st,
+                                   int prof_id) {
   int rc = validate_attention_shape(s, Cq, Ck);
   if (rc) return rc;
-  if (s.Sq != s.Sk && false) return rc;
   if (!q || !k || !v || !q_labels || !k_labels || !mask || !out)
     return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
   if (mbs < 0 || mhs < 0) return fail(BSA_ERR_INVALID_ARG, "negative mask stride");
@@ -858,6 +863,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
   mask_bits_kernel<<<dim3(Cq, nh, nb), 256, 0, st>>>(mask, mbs, mhs, nh, Cq, Ck, L.group_cluster,
                                                     L.group_valid, L.G, L.Wc, L.Wg, L.cbits,
                                                     L.gbits, L.gfull);
+  count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "mask_bits_kernel"))) return rc;
   // 3. Q gather
   const int vpr = s.D * es / 16;
@@ -866,6 +872,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     gather_rows_kernel<<<dim3(static_cast<unsigned>((n + 255) / 256), s.Hq, s.B), 256, 0, st>>>(
         static_cast<const uint4*>(q), static_cast<uint4*>(L.qp), L.qrow_token, s.Sq, L.Sqpad, vpr,
         s.Hq);
+    count_launch();
     if ((rc = check_cuda(cudaGetLastError(), "gather_rows_kernel"))) return rc;
   }
   // 4. K/V gather + centroids
@@ -874,12 +881,14 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
         static_cast<const float*>(k), static_cast<const float*>(v), static_cast<float*>(L.kp),
         static_cast<float*>(L.vp), static_cast<float*>(L.kc), static_cast<float*>(L.vc),
         L.kslot_token, L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
+    count_launch();
   } else {
     gather_kv_centroids_kernel<__nv_bfloat16><<<dim3(L.Ckpad, s.Hkv, s.B), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
         static_cast<__nv_bfloat16*>(L.kp), static_cast<__nv_bfloat16*>(L.vp),
         static_cast<__nv_bfloat16*>(L.kc), static_cast<__nv_bfloat16*>(L.vc), L.kslot_token,
         L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
+    count_launch();
   }
   if ((rc = check_cuda(cudaGetLastError(), "gather_kv_centroids_kernel"))) return rc;
 
@@ -928,11 +937,11 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
   args.out = out;
   const dim3 grid(L.Sqpad / 128, s.Hq, s.B);
   if (s.dtype == BSA_F32) {
-    return s.D == 64 ? launch_attn<64, true>(maps, args, grid, st)
-                     : launch_attn<128, true>(maps, args, grid, st);
+    return s.D == 64 ? launch_attn<64, true>(maps, args, grid, prof_id, st)
+                     : launch_attn<128, true>(maps, args, grid, prof_id, st);
   }
-  return s.D == 64 ? launch_attn<64, false>(maps, args, grid, st)
-                   : launch_attn<128, false>(maps, args, grid, st);
+  return s.D == 64 ? launch_attn<64, false>(maps, args, grid, prof_id, st)
+                   : launch_attn<128, false>(maps, args, grid, prof_id, st);
 }
 
 }  // namespace bsa
@@ -951,5 +960,6 @@ extern "C" int bsa_centroid_compensated_attention(const void* q, const void* k, 
                                                   size_t workspace_bytes, void* stream) {
   return bsa::centroid_compensated_attention(q, k, v, shape, q_labels, Cq, k_labels, Ck, block_mask,
                                              mask_b_stride, mask_h_stride, scale, compensate, out,
-                                             workspace, workspace_bytes, bsa::as_stream(stream));
+                                             workspace, workspace_bytes, bsa::as_stream(stream),
+                                             bsa::kProfAttention);
 }

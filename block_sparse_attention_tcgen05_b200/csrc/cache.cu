@@ -247,6 +247,7 @@ extern "C" int bsa_mask_cache_init(void* state, int B, int H, int Cq, int Ck, in
   int rc;
   if ((rc = check_cuda(cudaMemsetAsync(state, 0, L.bytes, st), "memset state"))) return rc;
   cache_init_kernel<<<1, 1, 0, st>>>(L.hdr, B, H, Cq, Ck, D, delta, relative ? 1 : 0, gate_lo, gate_hi);
+  count_launch();
   return check_cuda(cudaGetLastError(), "cache_init_kernel");
 }
 
@@ -272,8 +273,10 @@ extern "C" int bsa_mask_cache_should_refresh(void* state, const void* q, const v
         shape.Sq, shape.D);
   else
     return fail(BSA_ERR_UNSUPPORTED, "dtype");
+  count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "pool_kernel"))) return rc;
   decide_kernel<<<1, 1024, 0, st>>>(state, shape.B, shape.Hq, shape.D, shape.Sq, refresh, drift_out);
+  count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "decide_kernel"))) return rc;
   if (n_refresh_host) {
     const CacheLayout L = cache_layout(state, 1, 1, 1, 1, 1);  // header offset only
@@ -292,8 +295,10 @@ extern "C" int bsa_mask_cache_update(void* state, const uint8_t* new_mask, const
   cudaStream_t st = as_stream(stream);
   int rc;
   update_mask_kernel<<<148 * 4, 256, 0, st>>>(state, new_mask, refresh, block_mask_out);
+  count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "update_mask_kernel"))) return rc;
   update_anchor_kernel<<<1, 1024, 0, st>>>(state, refresh, new_mask ? 1 : 0);
+  count_launch();
   return check_cuda(cudaGetLastError(), "update_anchor_kernel");
 }
 
@@ -302,5 +307,6 @@ extern "C" int bsa_mask_cache_reset(void* state, void* stream) {
   if (!state) return fail(BSA_ERR_INVALID_ARG, "state is null");
   const CacheLayout L = cache_layout(state, 1, 1, 1, 1, 1);
   cache_reset_kernel<<<1, 1, 0, as_stream(stream)>>>(L.hdr);
+  count_launch();
   return check_cuda(cudaGetLastError(), "cache_reset_kernel");
 }

@@ -1,7 +1,10 @@
 // Status codes, error details, tensor-map encoding and the small label kernel.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -10,6 +13,20 @@ namespace bsa {
 
 namespace {
 thread_local char g_detail[512] = "";
+
+std::atomic<long long> g_launches{0};
+
+struct ProfState {
+  std::mutex mu;
+  int enabled = 0;
+  int capacity = 0;
+  std::vector<cudaEvent_t> ev[kProfCount][2];
+  int used[kProfCount] = {0, 0, 0};
+};
+ProfState& prof() {
+  static ProfState p;
+  return p;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -35,6 +52,23 @@ int fail(int status, const char* fmt, ...) {
   vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
   va_end(ap);
   return status;
+}
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void prof_begin(int kernel, cudaStream_t st) {
+  ProfState& p = prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  if (!p.enabled || p.used[kernel] >= p.capacity) return;
+  cudaEventRecord(p.ev[kernel][0][p.used[kernel]], st);
+}
+
+void prof_end(int kernel, cudaStream_t st) {
+  ProfState& p = prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  if (!p.enabled || p.used[kernel] >= p.capacity) return;
+  cudaEventRecord(p.ev[kernel][1][p.used[kernel]], st);
+  ++p.used[kernel];
 }
 
 int check_cuda(cudaError_t e, const char* what) {
@@ -116,6 +150,46 @@ void bsa_last_error_detail(char* buf, size_t len) {
 
 int bsa_version(void) { return 100; }
 
+long long bsa_launch_count(void) { return bsa::g_launches.load(); }
+
+int bsa_profile_enable(int max_launches) {
+  bsa::ProfState& p = bsa::prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  if (max_launches < 0) return bsa::fail(BSA_ERR_INVALID_ARG, "max_launches < 0");
+  for (int k = 0; k < bsa::kProfCount; ++k) {
+    for (int j = 0; j < 2; ++j) {
+      while (static_cast<int>(p.ev[k][j].size()) < max_launches) {
+        cudaEvent_t e;
+        cudaError_t r = cudaEventCreate(&e);
+        if (r != cudaSuccess) return bsa::check_cuda(r, "cudaEventCreate");
+        p.ev[k][j].push_back(e);
+      }
+    }
+    p.used[k] = 0;
+  }
+  p.capacity = max_launches;
+  p.enabled = max_launches > 0;
+  return BSA_OK;
+}
+
+int bsa_profile_read(int kernel, float* total_ms, int* launches) {
+  bsa::ProfState& p = bsa::prof();
+  std::lock_guard<std::mutex> lk(p.mu);
+  if (kernel < 0 || kernel >= bsa::kProfCount) return bsa::fail(BSA_ERR_INVALID_ARG, "kernel id");
+  float sum = 0.f;
+  for (int i = 0; i < p.used[kernel]; ++i) {
+    cudaError_t r = cudaEventSynchronize(p.ev[kernel][1][i]);
+    if (r != cudaSuccess) return bsa::check_cuda(r, "cudaEventSynchronize");
+    float ms = 0.f;
+    r = cudaEventElapsedTime(&ms, p.ev[kernel][0][i], p.ev[kernel][1][i]);
+    if (r != cudaSuccess) return bsa::check_cuda(r, "cudaEventElapsedTime");
+    sum += ms;
+  }
+  if (total_ms) *total_ms = sum;
+  if (launches) *launches = p.used[kernel];
+  return BSA_OK;
+}
+
 int bsa_get_device_status(void* stream, int* where) {
   cudaError_t e = cudaStreamSynchronize(bsa::as_stream(stream));
   if (e != cudaSuccess) return bsa::check_cuda(e, "cudaStreamSynchronize");
@@ -144,6 +218,7 @@ int bsa_tile_labels(int T, int H, int W, int tt, int th, int tw, int32_t* labels
   if (n_clusters) *n_clusters = nT * nH * nW;
   bsa::tile_labels_kernel<<<static_cast<unsigned>((S + 255) / 256), 256, 0,
                             bsa::as_stream(stream)>>>(T, H, W, tt, th, tw, nH, nW, labels);
+  bsa::count_launch();
   return bsa::check_cuda(cudaGetLastError(), "tile_labels_kernel");
 }
 

@@ -47,4 +47,12 @@ int make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, 
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Kernel timing hooks (bsa_profile_*): when enabled, the launch sites of the main
+// kernels record a CUDA event pair around the launch on the launch stream.
+enum ProfKernel { kProfAttention = 0, kProfScoring = 1, kProfProbe = 2, kProfCount = 3 };
+void prof_begin(int kernel, cudaStream_t st);
+void prof_end(int kernel, cudaStream_t st);
+// Counts kernel launches made by the library (bsa_launch_count).
+void count_launch();
+
 }  // namespace bsa

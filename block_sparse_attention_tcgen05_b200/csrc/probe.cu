@@ -21,7 +21,8 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
                                    const bsa_shape& s, const int32_t* q_labels, int Cq,
                                    const int32_t* k_labels, int Ck, const uint8_t* mask,
                                    int64_t mbs, int64_t mhs, float scale, int compensate,
-                                   float* out, void* ws, size_t ws_bytes, cudaStream_t st);
+                                   float* out, void* ws, size_t ws_bytes, cudaStream_t st,
+                                   int prof_id);
 size_t attention_workspace_bytes(const bsa_shape& s, int Cq, int Ck);
 
 constexpr int kMaxCentroidCluster = 4096;
@@ -259,10 +260,12 @@ extern "C" int bsa_select_probe_rows(const int32_t* labels, int S, int C, int M,
       centroid_order_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), S,
                                                           shape.D, shape.Hq, L.slot_token,
                                                           L.count, L.off, L.order);
+    count_launch();
     if ((rc = check_cuda(cudaGetLastError(), "centroid_order_kernel"))) return rc;
   }
   round_robin_kernel<<<BH, 256, 0, st>>>(L.slot_token, q ? L.order : nullptr, S, C, M, L.count,
                                          L.off, probe_idx, weights);
+  count_launch();
   return check_cuda(cudaGetLastError(), "round_robin_kernel");
 }
 
@@ -307,11 +310,12 @@ extern "C" int bsa_probe_dense_attention(const void* q, const void* k, const voi
   gather_probe_rows_kernel<<<dim3(static_cast<unsigned>((n + 255) / 256), shape.Hq, shape.B), 256, 0,
                              st>>>(static_cast<const uint4*>(q), static_cast<uint4*>(qp), probe_idx,
                                    per_head, shape.Sq, M, vpr, shape.Hq);
+  count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "gather_probe_rows_kernel"))) return rc;
   bsa_shape ps = shape;
   ps.Sq = M;
   // Every probe row keeps every key: one query cluster, one key cluster, one kept block.
   return centroid_compensated_attention(qp, k, v, ps, zeros, 1, zeros, 1, one, 0, 0, scale, 0,
                                         o_probe, static_cast<char*>(workspace) + used,
-                                        workspace_bytes - used, st);
+                                        workspace_bytes - used, st, kProfProbe);
 }

@@ -446,6 +446,7 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
     return fail(BSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, L.bytes);
   int rc;
   column_stats_kernel<<<dim3(kStatSplit, BH), 256, 0, st>>>(out, S, D, L.psum, L.psq);
+  count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "column_stats_kernel"))) return rc;
   FitArgs fa{out, o_probe, probe_idx, weights, per_head, S, D, M, rank, lam, L.psum, L.psq,
              L.zt,  L.rr,    L.bc,      L.vr,    L.pp,     L.cc};
@@ -457,6 +458,7 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
                                        static_cast<int>(big));
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(repair_fit)");
   repair_fit_kernel<<<BH, kFitThreads, big, st>>>(fa);
+  count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "repair_fit_kernel"))) return rc;
   const int smem = (2 * D * rank + rank) * static_cast<int>(sizeof(float));
   auto ap = D == 64 ? repair_apply_kernel<64> : repair_apply_kernel<128>;
@@ -465,5 +467,6 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(repair_apply)");
   }
   ap<<<dim3((S + 63) / 64, BH), 256, smem, st>>>(out, S, rank, L.pp, L.cc, L.vr);
+  count_launch();
   return check_cuda(cudaGetLastError(), "repair_apply_kernel");
 }

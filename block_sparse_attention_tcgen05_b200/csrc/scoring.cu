@@ -291,7 +291,10 @@ int antidiagonal_block_scores(const void* q, const void* k, const bsa_shape& s, 
 #undef BSA_SCORE_CASE
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(score_kernel)");
+  prof_begin(kProfScoring, st);
   kern<<<dim3(ns / 128, s.Hq, s.B), 192, smem, st>>>(mq, mk, a);
+  count_launch();
+  prof_end(kProfScoring, st);
   return check_cuda(cudaGetLastError(), "score_kernel launch");
 }
 

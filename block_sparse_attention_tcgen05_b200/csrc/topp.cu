@@ -101,5 +101,6 @@ extern "C" int bsa_top_p_block_mask(const float* scores, int B, int H, int Nq, i
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(top_p)");
   top_p_kernel<<<(rows + kTopPWarps - 1) / kTopPWarps, kTopPWarps * 32, smem, as_stream(stream)>>>(
       scores, H, Nq, Nk, rows, tau, n_tau, mask, tie_rows);
+  count_launch();
   return check_cuda(cudaGetLastError(), "top_p_kernel launch");
 }

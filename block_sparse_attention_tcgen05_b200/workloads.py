@@ -149,3 +149,30 @@ def drift_steps(q0, k0, steps, sigma, boosted_heads, boost, seed=0):
             q += g.standard_normal(q.shape) * sig[None, :, None, None]
             k += g.standard_normal(k.shape) * sig[None, :, None, None]
         yield to_dtype(q, dtype), to_dtype(k, dtype)
+
+
+def positional_qkv_device(B, Hq, Hkv, grid, D, ell, amp=2.0, seed=0, device="cuda",
+                          dtype=torch.bfloat16):
+    """The ``positional_qkv`` recipe drawn with torch's generator on ``device`` (fast at
+    full video size; the stream of random numbers differs from the NumPy one, the
+    distribution and structure are the same)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    axes = [torch.arange(n, dtype=torch.float32, device=device) for n in grid]
+    mesh = torch.meshgrid(*axes, indexing="ij")
+    coords = torch.stack([m.reshape(-1) for m in mesh], dim=1)
+    S = coords.shape[0]
+    ellt = torch.tensor(ell, dtype=torch.float32, device=device).reshape(1, -1)
+    grp = Hq // Hkv
+    q = torch.empty((B, Hq, S, D), dtype=dtype, device=device)
+    k = torch.empty((B, Hkv, S, D), dtype=dtype, device=device)
+    v = torch.empty((B, Hkv, S, D), dtype=dtype, device=device)
+    for b in range(B):
+        for hk in range(Hkv):
+            omega = torch.randn((D, coords.shape[1]), generator=g, device=device) / ellt
+            phi = torch.rand((D,), generator=g, device=device) * (2.0 * math.pi)
+            pos = amp * torch.sin(coords @ omega.T + phi[None, :])
+            k[b, hk] = (torch.randn((S, D), generator=g, device=device) + pos).to(dtype)
+            v[b, hk] = torch.randn((S, D), generator=g, device=device).to(dtype)
+            for j in range(grp):
+                q[b, hk * grp + j] = (torch.randn((S, D), generator=g, device=device) + pos).to(dtype)
+    return q, k, v

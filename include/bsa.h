@@ -74,6 +74,21 @@ int bsa_version(void);
  */
 int bsa_get_device_status(void* stream, int* where);
 
+/* Number of kernel launches the library has made since it was loaded. */
+long long bsa_launch_count(void);
+
+/*
+ * Kernel timing hooks. bsa_profile_enable(n) (n > 0) makes the next n launches of each
+ * timed kernel record a CUDA event pair around the launch on its stream; n == 0 turns
+ * timing off. bsa_profile_read(kernel, &ms, &count) synchronises those events and
+ * returns the summed duration and the number of timed launches. kernel: 0 = the
+ * attention kernel of centroid_compensated_attention, 1 = the scoring kernel,
+ * 2 = the attention kernel of probe_dense_attention. Creates CUDA events (host
+ * objects), no device memory.
+ */
+int bsa_profile_enable(int max_launches);
+int bsa_profile_read(int kernel, float* total_ms, int* launches);
+
 /*
  * tile_labels — [SBC] §What mlx-arsenal ships (tile_labels: labels matching Sliding
  * Tile Attention tiles), §Recipe. Token s = (t*H + h)*W + w of a T x H x W latent
