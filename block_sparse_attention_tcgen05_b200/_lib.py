@@ -55,6 +55,8 @@ SIGNATURES = {
     "bsa_repair_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "bsa_probe_residual_correction": (
         _i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
+    "bsa_probe_residual_correction_noalloc": (
+        _i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "bsa_mask_cache_state_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "bsa_mask_cache_init": (_i, [_vp, _i, _i, _i, _i, _i, _f, _i, _f, _f, _vp]),
     "bsa_mask_cache_should_refresh": (_i, [_vp, _vp, _vp, Shape, _vp, _vp, _ip, _vp]),

@@ -7,3 +7,4 @@
 #include "probe.cu"
 #include "repair.cu"
 #include "cache.cu"
+#include "repair_noalloc.cu"

@@ -229,6 +229,28 @@ int bsa_probe_residual_correction(float* out, const float* o_probe, const int32_
                                   size_t workspace_bytes, void* stream);
 
 /*
+ * probe_residual_correction_noalloc — no counterpart in the papers: a convenience for
+ * callers that cannot allocate device memory when they repair an output (for example
+ * while a CUDA graph is being captured, or in a runtime whose device memory is fixed
+ * up front). Same arguments and result as bsa_probe_residual_correction, minus the
+ * workspace: the scratch comes from a 16 MiB buffer compiled into the library, which
+ * every GPU that loads libbsa.so holds until the process exits.
+ *  - Size limit: bsa_repair_workspace_bytes(B, H, S, D, M) must be <= 16 MiB (about
+ *    B*H <= 48 heads at D = 128, M = 64); larger problems return BSA_ERR_UNSUPPORTED
+ *    with the required size in the error detail.
+ *  - The first call on each device looks up the buffer's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call before
+ *    any stream capture begins.
+ *  - Every call uses the same buffer: calls that may overlap on the GPU (different
+ *    streams, or different host threads) race on it and must be serialised by the
+ *    caller. The buffer needs no clearing; nothing is allocated or freed.
+ */
+int bsa_probe_residual_correction_noalloc(float* out, const float* o_probe,
+                                          const int32_t* probe_idx, const float* weights,
+                                          int per_head, int B, int H, int S, int D, int M,
+                                          int rank, float lam, void* stream);
+
+/*
  * Per-head drift/anchor mask cache — [HMR] §HEART — head-wise temporal mask reuse
  * (anchor = token means qbar, kbar and the head's mask; drift = L1 distance; refresh
  * above delta; layer gate: under gate_lo of the heads -> none, above gate_hi -> all),
