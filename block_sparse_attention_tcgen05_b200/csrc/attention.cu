@@ -322,14 +322,15 @@ struct AttnCfg {
   static constexpr int NATOM = D / ATOM;            // 128-byte column chunks per row
   static constexpr int TILE = 128 * D * ESIZE;      // one 128-row operand tile
   static constexpr int KSTEP = 32 / ESIZE;          // K of one MMA instruction
-  static constexpr int MISC = 4096;
+  static constexpr int MISC = 6144;
   static constexpr int SMEM = 3 * TILE + MISC + 1024;
   // At least ~100 KB so that at most two CTAs share an SM (two 256-column TMEM
   // allocations fill the 512 columns).
   static constexpr int SMEM_LAUNCH = SMEM > 100 * 1024 ? SMEM : 100 * 1024;
 };
 
-enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SF, BAR_PF, BAR_OF, BAR_DRAIN, NBAR };
+enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SF, BAR_PF, BAR_OF, BAR_DRAIN,
+       BAR_X0, BAR_X1, BAR_X2, BAR_X3, NBAR };  // BAR_X*: row-pair exchange per lane quarter
 
 struct Chunk {
   int start;   // first key slot (token chunk) or first centroid (centroid chunk)
@@ -343,7 +344,9 @@ __device__ __forceinline__ bool bit_at(const uint32_t* bits, int i) {
 }
 
 // Deterministic chunk walk shared by every role of the CTA: runs of kept 16-key
-// groups split into chunks of at most 8 groups, then the needed centroid chunks.
+// groups split into chunks of at most 8 groups, then the needed centroid chunks. The
+// run length and the uniform test use 64-bit windows of the bitsets (trailing-ones
+// count), so one step costs a handful of shared loads whatever the run.
 __device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t* any,
                                            const uint32_t* uni, int G, int Wg,
                                            const uint32_t* cneed, int ncc, Chunk& ch) {
@@ -352,16 +355,21 @@ __device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t*
     uint32_t bits = any[w] & (0xffffffffu << (gcur & 31));
     while (bits == 0 && ++w < Wg) bits = any[w];
     if (bits != 0) {
-      const int g0 = (w << 5) + __ffs(bits) - 1;
-      int ng = 1;
-      while (ng < 8 && g0 + ng < G && bit_at(any, g0 + ng)) ++ng;
-      bool uniform = true;
-      for (int j = 0; j < ng; ++j) uniform = uniform && bit_at(uni, g0 + j);
+      const int b0 = __ffs(bits) - 1;
+      const int g0 = (w << 5) + b0;
+      const uint32_t a_hi = (w + 1 < Wg) ? any[w + 1] : 0u;
+      const uint32_t u_hi = (w + 1 < Wg) ? uni[w + 1] : 0u;
+      const uint64_t awin = ((static_cast<uint64_t>(a_hi) << 32) | any[w]) >> b0;
+      const uint64_t uwin = ((static_cast<uint64_t>(u_hi) << 32) | uni[w]) >> b0;
+      const int run = __ffsll(static_cast<long long>(~awin)) - 1;  // trailing ones
+      int ng = (run < 0 || run > 8) ? 8 : run;
+      if (ng > G - g0) ng = G - g0;
+      const uint32_t m = (1u << ng) - 1u;
       ch.start = g0 * 16;
       ch.n = ng * 16;
       ch.g0 = g0;
       ch.ng = ng;
-      ch.uniform = uniform;
+      ch.uniform = (static_cast<uint32_t>(uwin) & m) == m;
       ch.centroid = false;
       gcur = g0 + ng;
       return true;
@@ -388,7 +396,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 template <int D, bool TF32>
-__global__ void __launch_bounds__(192, 2)
+// 288 threads and at most 112 registers per thread: two CTAs share an SM.
+__global__ void __maxnreg__(112)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
                 const __grid_constant__ CUtensorMap tmVc, const AttnArgs a) {
@@ -406,6 +415,7 @@ __global__ void __launch_bounds__(192, 2)
   uint32_t* any_bits = reinterpret_cast<uint32_t*>(distinct + 128);  // 128 words
   uint32_t* uni_bits = any_bits + 128;                                // 128 words
   uint32_t* cneed = uni_bits + 128;                                   // 4 words
+  float* xchg = reinterpret_cast<float*>(cneed + 4);                  // 512 floats
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -415,18 +425,18 @@ __global__ void __launch_bounds__(192, 2)
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
 
   if (tid == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(BAR(i), i == BAR_PF ? 128u : 1u);
+    for (int i = 0; i < NBAR; ++i) mbar_init(BAR(i), i == BAR_PF ? 256u : (i >= BAR_X0 ? 64u : 1u));
     *abort_flag = 0;
     *n_distinct = 0;
     *never = 0;
     fence_mbarrier_init();
   }
-  if (tid == 32) {
+  if (tid == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
-  if (warp == 1) {
+  if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
@@ -473,84 +483,104 @@ __global__ void __launch_bounds__(192, 2)
   const int ncc = a.compensate ? a.Ckpad / 128 : 0;
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ control thread: TMA + tcgen05.mma
+    // One thread issues every copy and every MMA. The single K and V stages are
+    // refilled as soon as the MMA that read them has completed; both refills happen
+    // while the softmax warps work on the current chunk.
     if (lane == 0) {
+      constexpr uint32_t kIdescQK = make_idesc(TF32, 128, 0, false, false);
+      constexpr uint32_t kIdescPV = make_idesc(TF32, 128, D, false, true);
+      // Base descriptors; a K-step only moves the start address (bits 0..13, in
+      // 16-byte units), so each MMA adds a constant instead of rebuilding them.
+      const uint64_t dQ = smem_desc(sQ, 16, 1024);
+      const uint64_t dK = smem_desc(sK, 16, 1024);
+      const uint64_t dV = TF32 ? smem_desc(sV, 16384, 512, kLayoutSW128Atom32B)
+                               : smem_desc(sV, 16384, 1024, kLayoutSW128);
       const int qrow0 = (b * a.Hq + h) * a.Sqpad + tile * 128;
+      const int krow0 = (b * a.Hkv + hkv) * a.Skpad;
+      const int crow0 = (b * a.Hkv + hkv) * a.Ckpad;
+      auto load_kv = [&](const Chunk& c, bool is_v) {
+        const CUtensorMap* m = c.centroid ? (is_v ? &tmVc : &tmKc) : (is_v ? &tmV : &tmK);
+        const int row = (c.centroid ? crow0 : krow0) + c.start;
+        const uint32_t dst = is_v ? sV : sK;
+        const uint32_t bar = BAR(is_v ? BAR_VF : BAR_KF);
+        mbar_arrive_expect_tx(bar, Cfg::TILE);
+#pragma unroll
+        for (int cc = 0; cc < Cfg::NATOM; ++cc) tma_load_2d(dst + cc * 16384, m, bar, cc * Cfg::ATOM, row);
+      };
+      int gcur = 0, ccur = 0, j = 0, nk = 0, nv = 0;
+      Chunk cur, nxt;
+      bool have = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, cur);
       mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
 #pragma unroll
-      for (int c = 0; c < Cfg::NATOM; ++c)
-        tma_load_2d(sQ + c * 16384, &tmQ, BAR(BAR_Q), c * Cfg::ATOM, qrow0);
-      int gcur = 0, ccur = 0, j = 0, nk = 0, nv = 0;
-      Chunk ch;
-      while (next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
-        const CUtensorMap* mk = ch.centroid ? &tmKc : &tmK;
-        const CUtensorMap* mv = ch.centroid ? &tmVc : &tmV;
-        const int row = ch.centroid ? (b * a.Hkv + hkv) * a.Ckpad + ch.start
-                                    : (b * a.Hkv + hkv) * a.Skpad + ch.start;
-        if (j > 0 && !mbar_wait(BAR(BAR_KE), (j - 1) & 1, abort_flag, 1)) break;
-        mbar_arrive_expect_tx(BAR(BAR_KF), Cfg::TILE);
-#pragma unroll
-        for (int c = 0; c < Cfg::NATOM; ++c)
-          tma_load_2d(sK + c * 16384, mk, BAR(BAR_KF), c * Cfg::ATOM, row);
+      for (int cc = 0; cc < Cfg::NATOM; ++cc)
+        tma_load_2d(sQ + cc * 16384, &tmQ, BAR(BAR_Q), cc * Cfg::ATOM, qrow0);
+      if (have) {
+        load_kv(cur, false);
         ++nk;
-        if (j > 0 && !mbar_wait(BAR(BAR_VE), (j - 1) & 1, abort_flag, 2)) break;
-        mbar_arrive_expect_tx(BAR(BAR_VF), Cfg::TILE);
-#pragma unroll
-        for (int c = 0; c < Cfg::NATOM; ++c)
-          tma_load_2d(sV + c * 16384, mv, BAR(BAR_VF), c * Cfg::ATOM, row);
+        load_kv(cur, true);
         ++nv;
+      }
+      bool ok = mbar_wait(BAR(BAR_Q), 0, abort_flag, 3);
+      while (ok && have) {
+        const bool have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
+        if (!(ok = mbar_wait(BAR(BAR_KF), j & 1, abort_flag, 5))) break;
+        tc_fence_after();
+        const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(cur.n >> 3) << 17);
+        // rolled loops keep the control thread's register footprint small
+#pragma unroll 1
+        for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          mma_ss<TF32>(tmem, dQ + off, dK + off, idesc, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(BAR(BAR_KE));
+        tc_commit(BAR(BAR_SF));
+        // V stage: refill once PV_{j-1} has read it (chunk 0 was loaded up front)
+        if (j > 0) {
+          if (!(ok = mbar_wait(BAR(BAR_VE), (j - 1) & 1, abort_flag, 4))) break;
+          load_kv(cur, true);
+          ++nv;
+        }
+        // K stage: refill with the next chunk once QK_j has read it
+        if (have_next) {
+          if (!(ok = mbar_wait(BAR(BAR_KE), j & 1, abort_flag, 1))) break;
+          load_kv(nxt, false);
+          ++nk;
+        }
+        if (!(ok = mbar_wait(BAR(BAR_PF), j & 1, abort_flag, 6))) break;
+        if (!(ok = mbar_wait(BAR(BAR_VF), j & 1, abort_flag, 7))) break;
+        tc_fence_after();
+        // V is MN-major (d contiguous): 128-byte rows, d chunks 16 KB apart; bf16 uses
+        // 8-row swizzle groups (1 KB), tf32 the 32-byte-unit swizzle with 4-row groups.
+        // A K-step of KSTEP rows advances the start address by KSTEP*128 bytes.
+        const int nsteps = cur.n / Cfg::KSTEP;
+#pragma unroll 1
+        for (int kk = 0; kk < nsteps; ++kk)
+          mma_ts<TF32>(tmem + 128, tmem + kk * 8,
+                       dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(BAR(BAR_VE));
+        cur = nxt;
+        have = have_next;
         ++j;
       }
-      // Every issued copy must land before the CTA may exit.
+      tc_commit(BAR(BAR_OF));
+      // Before the CTA may exit: every issued copy has landed, every MMA has completed.
+      tc_commit(BAR(BAR_DRAIN));
+      mbar_wait(BAR(BAR_DRAIN), 0, never, 23);
       mbar_wait(BAR(BAR_Q), 0, never, 20);
       if (nk) mbar_wait(BAR(BAR_KF), (nk - 1) & 1, never, 21);
       if (nv) mbar_wait(BAR(BAR_VF), (nv - 1) & 1, never, 22);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer (one thread)
-    if (lane == 0) {
-      constexpr uint32_t kIdescQK = make_idesc(TF32, 128, 0, false, false);
-      constexpr uint32_t kIdescPV = make_idesc(TF32, 128, D, false, true);
-      bool ok = mbar_wait(BAR(BAR_Q), 0, abort_flag, 3);
-      int gcur = 0, ccur = 0, j = 0;
-      Chunk ch;
-      while (ok && next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
-        // S is overwritten while the previous PV may still be queued: tcgen05.mma
-        // operations of one thread execute in issue order, so PV_{j-1} has read P_{j-1}
-        // before QK_j writes the same columns.
-        if (!(ok = mbar_wait(BAR(BAR_KF), j & 1, abort_flag, 5))) break;
-        tc_fence_after();
-        const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(ch.n >> 3) << 17);
-#pragma unroll
-        for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
-          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          mma_ss<TF32>(tmem, smem_desc(sQ + off, 16, 1024), smem_desc(sK + off, 16, 1024),
-                       idesc, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(BAR(BAR_KE));
-        tc_commit(BAR(BAR_SF));
-        if (!(ok = mbar_wait(BAR(BAR_PF), j & 1, abort_flag, 6))) break;
-        if (!(ok = mbar_wait(BAR(BAR_VF), j & 1, abort_flag, 7))) break;
-        tc_fence_after();
-        const int nsteps = ch.n / Cfg::KSTEP;
-        for (int kk = 0; kk < nsteps; ++kk) {
-          // V is MN-major (d contiguous): 128-byte rows, d chunks 16 KB apart; bf16 uses
-          // 8-row swizzle groups (1 KB), tf32 the 32-byte-unit swizzle with 4-row groups.
-          const uint64_t bdesc =
-              TF32 ? smem_desc(sV + kk * Cfg::KSTEP * 128, 16384, 512, kLayoutSW128Atom32B)
-                   : smem_desc(sV + kk * Cfg::KSTEP * 128, 16384, 1024, kLayoutSW128);
-          mma_ts<TF32>(tmem + 128, tmem + kk * 8, bdesc, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(BAR(BAR_VE));
-        ++j;
-      }
-      tc_commit(BAR(BAR_OF));
-      tc_commit(BAR(BAR_DRAIN));
-      mbar_wait(BAR(BAR_DRAIN), 0, never, 23);
-    }
   } else {
-    // ------------------------------------------------ softmax / epilogue (128 threads)
+    // ------------------------------------------------ softmax / epilogue (256 threads)
+    // Two threads per query row: warps 1..4 own columns [0, 64) of every chunk, warps
+    // 5..8 columns [64, 128). Warp w reads TMEM lanes 32*(w%4) .. +31, so each lane
+    // quarter has one warp of each half. The row max of a chunk is combined through
+    // shared memory with a 64-thread named barrier per quarter; both threads of a row
+    // then take identical rescaling decisions.
     const int quarter = warp & 3;
+    const int half = (warp - 1) >> 2;
     const int r = quarter * 32 + lane;
     const int qrow = tile * 128 + r;
     const int lab = a.qrow_label[qrow];
@@ -558,7 +588,9 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t* grow = gb + static_cast<size_t>(lab < 0 ? 0 : lab) * a.Wg;
     const uint32_t* crow = cb + static_cast<size_t>(lab < 0 ? 0 : lab) * a.Wc;
     const uint32_t tS = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t tO = tS + 128;
+    const uint32_t tO = tS + 128 + half * (D / 2);
+    const uint32_t xbar = BAR(BAR_X0 + quarter);  // the two threads of a row meet here
+    const float scl = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     int gcur = 0, ccur = 0, j = 0;
     bool ok = true;
@@ -566,154 +598,146 @@ __global__ void __launch_bounds__(192, 2)
     while (next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
       if (!(ok = mbar_wait(BAR(BAR_SF), j & 1, abort_flag, 9))) break;
       tc_fence_after();
-      const int npc = (ch.n + 31) >> 5;
-      // Logits of this chunk: a full chunk that every row of the tile keeps is used
-      // raw, scale·log2(e) folded into the FFMA feeding ex2; any other chunk gets its
-      // per-row column mask (kept groups, real keys, or skipped non-empty clusters)
-      // and, for centroid chunks, the log2(n_c) bias.
-      const bool fast = ch.uniform && ch.n == 128 && lab >= 0;
-      uint32_t mk[4] = {0u, 0u, 0u, 0u};
-      if (!fast && lab >= 0) {
+      const int c0 = half * 64;           // first column of this thread's half
+      const int nmine = ch.n - c0;        // columns of the chunk in this half (<= 0: none)
+      const bool fast = ch.uniform && nmine >= 64 && lab >= 0;
+      // column mask of this half (bit c = column c0 + c kept) for non-fast chunks
+      uint32_t mk0 = 0u, mk1 = 0u;
+      if (!fast && lab >= 0 && nmine > 0) {
         if (ch.centroid) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int ww = (ch.start >> 5) + w;
-            mk[w] = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
-          }
-        } else if (ch.uniform) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) mk[w] = 0xffffffffu;
+          const int ww = (ch.start + c0) >> 5;
+          mk0 = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
+          mk1 = ww + 1 < a.Wc ? (~__ldg(crow + ww + 1) & __ldg(a.cnonempty + ww + 1)) : 0u;
         } else {
-          for (int jj = 0; jj < ch.ng; ++jj) {
-            const int g = ch.g0 + jj;
-            if ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u) {
+          const int gh0 = ch.g0 + half * 4;  // this half covers groups gh0 .. gh0+3
+          for (int jj = 0; jj < 4; ++jj) {
+            const int g = gh0 + jj;
+            if (half * 4 + jj < ch.ng && ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u)) {
               const int nv = bit_at(a.gfull, g) ? 16 : __ldg(a.group_valid + g);
               const uint32_t bits = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
-              mk[jj >> 1] |= bits << ((jj & 1) * 16);
+              if (jj < 2) mk0 |= bits << (jj * 16);
+              else mk1 |= bits << ((jj - 2) * 16);
             }
           }
         }
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-          if (w * 32 + 32 > ch.n) mk[w] &= (w * 32 >= ch.n) ? 0u : (0xffffffffu >> (w * 32 + 32 - ch.n));
+        if (nmine < 64) {
+          mk1 = nmine <= 32 ? 0u : (mk1 & (0xffffffffu >> (64 - nmine)));
+          if (nmine < 32) mk0 &= 0xffffffffu >> (32 - nmine);
+        }
       }
-      const float* bias = ch.centroid ? a.bias2 + ch.start : nullptr;
-      const float scl = a.scale_log2;
-
-      // Pass 1: chunk max (log2 units). Two 32-column loads in flight per wait.
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      float v0[32], v1[32];
+      float mx = -INFINITY;
+      if (nmine > 0) {
+        tmem_ld32(tS + c0, v0);
+        tmem_ld32(tS + c0 + 32, v1);
+        tmem_wait_ld();
+        if (fast) {
+          float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-      for (int p = 0; p < 4; p += 2) {
-        if (p < npc) {
-          float t0[32], t1[32];
-          tmem_ld32(tS + p * 32, t0);
-          if (p + 1 < npc) tmem_ld32(tS + (p + 1) * 32, t1);
-          tmem_wait_ld();
+          for (int c = 0; c < 32; ++c) {
+            m0 = fmaxf(m0, v0[c]);
+            m1 = fmaxf(m1, v1[c]);
+          }
+          mx = fmaxf(m0, m1) * scl;
+          // logits in log2 units
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (p + h < npc) {
-              const float* t = h ? t1 : t0;
-              const int pp = p + h;
-              if (fast) {
+          for (int c = 0; c < 32; ++c) {
+            v0[c] *= scl;
+            v1[c] *= scl;
+          }
+        } else {
+          const float* bias = ch.centroid ? a.bias2 + ch.start + c0 : nullptr;
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                  mx0 = fmaxf(mx0, t[c]);
-                  mx1 = fmaxf(mx1, t[c + 1]);
-                }
-              } else {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                  const float add = bias ? __ldg(bias + pp * 32 + c) : 0.f;
-                  const float x = ((mk[pp] >> c) & 1u) ? fmaf(t[c], scl, add) : -INFINITY;
-                  if (c & 1) mx1 = fmaxf(mx1, x); else mx0 = fmaxf(mx0, x);
-                }
-              }
-            }
+          for (int c = 0; c < 32; ++c) {
+            const float b0 = bias ? __ldg(bias + c) : 0.f;
+            const float b1 = bias ? __ldg(bias + 32 + c) : 0.f;
+            v0[c] = ((mk0 >> c) & 1u) ? fmaf(v0[c], scl, b0) : -INFINITY;
+            v1[c] = ((mk1 >> c) & 1u) ? fmaf(v1[c], scl, b1) : -INFINITY;
+            mx = fmaxf(mx, fmaxf(v0[c], v1[c]));
           }
         }
       }
-      const float mx = fast ? fmaxf(mx0, mx1) * scl : fmaxf(mx0, mx1);
+      xchg[half * 128 + r] = mx;
+      mbar_arrive(xbar);
+      if (!(ok = mbar_wait(xbar, j & 1, abort_flag, 11))) break;
+      mx = fmaxf(xchg[r], xchg[128 + r]);
       // Lazy rescaling: the running max only moves when the chunk max exceeds it by
       // more than 8 (log2 units), so P stays below 256 and O is rarely touched.
       const bool need = mx > m_run + 8.f;
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = need ? mx : m_run;
-        const float alpha = need ? ex2(m_run - m_new) : 1.f;
-        if (j > 0) {
-#pragma unroll
-          for (int p = 0; p < D / 32; ++p) {
-            float o[32];
-            tmem_ld32(tO + p * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] *= alpha;
-            tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
-          }
-        }
+      const bool any_need = __any_sync(0xffffffffu, need);
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m_run - mx);
         l_run *= alpha;
-        m_run = m_new;
+        m_run = mx;
       }
-      const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
-
-      // Pass 2: P = 2^(x - m), written over S in place (bf16 pairs: piece p of 32
-      // logits lands in columns [16p, 16p+16), which pass 2 has already read). The load
-      // of piece p+1 is in flight while piece p is exponentiated.
-      float sum0 = 0.f, sum1 = 0.f;
-      float buf[2][32];
-      tmem_ld32(tS, buf[0]);
-      tmem_wait_ld();
+      if (nmine > 0) {
+        const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        if (p < npc) {
-          float* t = buf[p & 1];
-          if (p + 1 < npc) tmem_ld32(tS + (p + 1) * 32, buf[(p + 1) & 1]);
-          if (fast) {
+        for (int c = 0; c < 32; ++c) {
+          v0[c] = ex2(v0[c] + neg_mu);
+          v1[c] = ex2(v1[c] + neg_mu);
+          s0 += v0[c];
+          s1 += v1[c];
+        }
+        l_run += s0 + s1;
+        // P over S in place: this half's 64 values become bf16 pairs in columns
+        // [32*half, 32*half + 32), or fp32 in its own 64 columns for tf32. The other
+        // half's S columns were read before the barrier above.
+        if constexpr (TF32) {
+          tmem_st32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(v0));
+          tmem_st32(tS + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v1));
+        } else {
+          // pack in place: word i of each array takes elements 2i, 2i+1 (i <= 2i)
+          uint32_t* w0 = reinterpret_cast<uint32_t*>(v0);
+          uint32_t* w1 = reinterpret_cast<uint32_t*>(v1);
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              t[c] = ex2(fmaf(t[c], scl, neg_mu));
-              t[c + 1] = ex2(fmaf(t[c + 1], scl, neg_mu));
-              sum0 += t[c];
-              sum1 += t[c + 1];
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float add = bias ? __ldg(bias + p * 32 + c) : 0.f;
-              const float e = ((mk[p] >> c) & 1u) ? ex2(fmaf(t[c], scl, add + neg_mu)) : 0.f;
-              t[c] = e;
-              if (c & 1) sum1 += e; else sum0 += e;
-            }
+          for (int i = 0; i < 16; ++i) {
+            w0[i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
+            w1[i] = pack_bf16x2(v1[2 * i], v1[2 * i + 1]);
           }
-          if constexpr (TF32) {
-            tmem_st32(tS + p * 32, *reinterpret_cast<uint32_t(*)[32]>(t));
-          } else {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(t[2 * i], t[2 * i + 1]);
-            tmem_st16(tS + p * 16, pk);
-          }
-          tmem_wait_ld();
+          tmem_st16(tS + half * 32, w0);
+          tmem_st16(tS + half * 32 + 16, w1);
         }
       }
-      l_run += sum0 + sum1;
+      // O (this half's D/2 columns) follows the running max before PV_j adds to it;
+      // nothing is in flight on O here: PV_{j-1} completed before S_j was ready.
+      if (any_need && j > 0) {
+#pragma unroll 1
+        for (int p = 0; p < D / 64; ++p) {
+          float o[32];
+          tmem_ld32(tO + p * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] *= alpha;
+          tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(BAR_PF));
       ++j;
     }
+    // row sum of both halves
+    xchg[256 + half * 128 + r] = l_run;
+    mbar_arrive(xbar);
+    if (ok) ok = mbar_wait(xbar, j & 1, abort_flag, 12);
+    const float l_tot = xchg[256 + r] + xchg[256 + 128 + r];
     if (ok && mbar_wait(BAR(BAR_OF), 0, abort_flag, 10)) {
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      float* orow = a.out + ((static_cast<size_t>(b) * a.Hq + h) * a.Sq + (tok >= 0 ? tok : 0)) * D;
-#pragma unroll
-      for (int p = 0; p < D / 32; ++p) {
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      float* orow = a.out + ((static_cast<size_t>(b) * a.Hq + h) * a.Sq + (tok >= 0 ? tok : 0)) * D +
+                    half * (D / 2);
+#pragma unroll 1
+      for (int p = 0; p < D / 64; ++p) {
         float o[32];
         tmem_ld32(tO + p * 32, o);
         tmem_wait_ld();
         if (tok >= 0) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            float4 v4 = l_run > 0.f ? make_float4(o[4 * i] * inv, o[4 * i + 1] * inv,
+            float4 v4 = l_tot > 0.f ? make_float4(o[4 * i] * inv, o[4 * i + 1] * inv,
                                                   o[4 * i + 2] * inv, o[4 * i + 3] * inv)
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
             *reinterpret_cast<float4*>(orow + p * 32 + 4 * i) = v4;
@@ -725,7 +749,7 @@ __global__ void __launch_bounds__(192, 2)
 #undef BAR
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
@@ -787,7 +811,7 @@ int launch_attn(const CUtensorMap* maps, const AttnArgs& args, dim3 grid, int pr
                                        Cfg::SMEM_LAUNCH);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attn_kernel)");
   prof_begin(prof_id, st);
-  kern<<<grid, 192, Cfg::SMEM_LAUNCH, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
+  kern<<<grid, 288, Cfg::SMEM_LAUNCH, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
   count_launch();
   prof_end(prof_id, st);
   return check_cuda(cudaGetLastError(), "attn_kernel launch");
