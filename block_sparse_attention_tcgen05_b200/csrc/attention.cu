@@ -390,6 +390,10 @@ __device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t*
   return false;
 }
 
+// Pairs of every 8 whose exponentials use the FMA-pipe polynomial instead of MUFU ex2.
+// 0: measured fastest in this kernel (the softmax warps are issue-bound, not MUFU-bound).
+constexpr int kPolyPairsOf8 = 0;
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -483,23 +487,34 @@ __global__ void __maxnreg__(112)
   const int ncc = a.compensate ? a.Ckpad / 128 : 0;
 
   if (warp == 0) {
-    // ------------------------------------------------ control thread: TMA + tcgen05.mma
-    // One thread issues every copy and every MMA. The single K and V stages are
-    // refilled as soon as the MMA that read them has completed; both refills happen
+    // ------------------------------------------------ control warp: TMA + tcgen05.mma
+    // The whole warp runs this loop on warp-uniform values, so MMA descriptors live in
+    // uniform registers and each tcgen05.mma issues without per-lane conversion; lane
+    // 0 alone issues the per-thread operations (TMA copies, expect_tx, commits). The
+    // single K and V stages are refilled as soon as the MMA that read them completes,
     // while the softmax warps work on the current chunk.
-    if (lane == 0) {
-      constexpr uint32_t kIdescQK = make_idesc(TF32, 128, 0, false, false);
-      constexpr uint32_t kIdescPV = make_idesc(TF32, 128, D, false, true);
-      // Base descriptors; a K-step only moves the start address (bits 0..13, in
-      // 16-byte units), so each MMA adds a constant instead of rebuilding them.
-      const uint64_t dQ = smem_desc(sQ, 16, 1024);
-      const uint64_t dK = smem_desc(sK, 16, 1024);
-      const uint64_t dV = TF32 ? smem_desc(sV, 16384, 512, kLayoutSW128Atom32B)
-                               : smem_desc(sV, 16384, 1024, kLayoutSW128);
-      const int qrow0 = (b * a.Hq + h) * a.Sqpad + tile * 128;
-      const int krow0 = (b * a.Hkv + hkv) * a.Skpad;
-      const int crow0 = (b * a.Hkv + hkv) * a.Ckpad;
-      auto load_kv = [&](const Chunk& c, bool is_v) {
+    const bool leader = lane == 0;
+    auto wait_all = [&](uint32_t bar, uint32_t parity, int where) -> bool {
+      const bool r = mbar_wait(bar, parity, abort_flag, where);
+      return __all_sync(0xffffffffu, r);
+    };
+    auto commit = [&](uint32_t bar) {
+      if (elect_one()) tc_commit(bar);
+      __syncwarp();
+    };
+    constexpr uint32_t kIdescQK = make_idesc(TF32, 128, 0, false, false);
+    constexpr uint32_t kIdescPV = make_idesc(TF32, 128, D, false, true);
+    // Base descriptors; a K-step only moves the start address (bits 0..13, in 16-byte
+    // units), so each MMA adds a constant instead of rebuilding them.
+    const uint64_t dQ = smem_desc(sQ, 16, 1024);
+    const uint64_t dK = smem_desc(sK, 16, 1024);
+    const uint64_t dV = TF32 ? smem_desc(sV, 16384, 512, kLayoutSW128Atom32B)
+                             : smem_desc(sV, 16384, 1024, kLayoutSW128);
+    const int qrow0 = (b * a.Hq + h) * a.Sqpad + tile * 128;
+    const int krow0 = (b * a.Hkv + hkv) * a.Skpad;
+    const int crow0 = (b * a.Hkv + hkv) * a.Ckpad;
+    auto load_kv = [&](const Chunk& c, bool is_v) {
+      if (leader) {
         const CUtensorMap* m = c.centroid ? (is_v ? &tmVc : &tmKc) : (is_v ? &tmV : &tmK);
         const int row = (c.centroid ? crow0 : krow0) + c.start;
         const uint32_t dst = is_v ? sV : sK;
@@ -507,71 +522,80 @@ __global__ void __maxnreg__(112)
         mbar_arrive_expect_tx(bar, Cfg::TILE);
 #pragma unroll
         for (int cc = 0; cc < Cfg::NATOM; ++cc) tma_load_2d(dst + cc * 16384, m, bar, cc * Cfg::ATOM, row);
-      };
-      int gcur = 0, ccur = 0, j = 0, nk = 0, nv = 0;
-      Chunk cur, nxt;
-      bool have = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, cur);
+      }
+      __syncwarp();
+    };
+    int gcur = 0, ccur = 0, j = 0, nk = 0, nv = 0;
+    Chunk cur, nxt;
+    bool have = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, cur);
+    if (leader) {
       mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
 #pragma unroll
       for (int cc = 0; cc < Cfg::NATOM; ++cc)
         tma_load_2d(sQ + cc * 16384, &tmQ, BAR(BAR_Q), cc * Cfg::ATOM, qrow0);
-      if (have) {
-        load_kv(cur, false);
-        ++nk;
+    }
+    __syncwarp();
+    if (have) {
+      load_kv(cur, false);
+      ++nk;
+      load_kv(cur, true);
+      ++nv;
+    }
+    bool ok = wait_all(BAR(BAR_Q), 0, 3);
+    while (ok && have) {
+      const bool have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
+      if (!(ok = wait_all(BAR(BAR_KF), j & 1, 5))) break;
+      tc_fence_after();
+      const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(cur.n >> 3) << 17);
+#pragma unroll
+      for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+        if (elect_one()) mma_ss<TF32>(tmem, dQ + off, dK + off, idesc, kk > 0 ? 1u : 0u);
+        __syncwarp();
+      }
+      commit(BAR(BAR_KE));
+      commit(BAR(BAR_SF));
+      // V stage: refill once PV_{j-1} has read it (chunk 0 was loaded up front)
+      if (j > 0) {
+        if (!(ok = wait_all(BAR(BAR_VE), (j - 1) & 1, 4))) break;
         load_kv(cur, true);
         ++nv;
       }
-      bool ok = mbar_wait(BAR(BAR_Q), 0, abort_flag, 3);
-      while (ok && have) {
-        const bool have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
-        if (!(ok = mbar_wait(BAR(BAR_KF), j & 1, abort_flag, 5))) break;
-        tc_fence_after();
-        const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(cur.n >> 3) << 17);
-        // rolled loops keep the control thread's register footprint small
-#pragma unroll 1
-        for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          mma_ss<TF32>(tmem, dQ + off, dK + off, idesc, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(BAR(BAR_KE));
-        tc_commit(BAR(BAR_SF));
-        // V stage: refill once PV_{j-1} has read it (chunk 0 was loaded up front)
-        if (j > 0) {
-          if (!(ok = mbar_wait(BAR(BAR_VE), (j - 1) & 1, abort_flag, 4))) break;
-          load_kv(cur, true);
-          ++nv;
-        }
-        // K stage: refill with the next chunk once QK_j has read it
-        if (have_next) {
-          if (!(ok = mbar_wait(BAR(BAR_KE), j & 1, abort_flag, 1))) break;
-          load_kv(nxt, false);
-          ++nk;
-        }
-        if (!(ok = mbar_wait(BAR(BAR_PF), j & 1, abort_flag, 6))) break;
-        if (!(ok = mbar_wait(BAR(BAR_VF), j & 1, abort_flag, 7))) break;
-        tc_fence_after();
-        // V is MN-major (d contiguous): 128-byte rows, d chunks 16 KB apart; bf16 uses
-        // 8-row swizzle groups (1 KB), tf32 the 32-byte-unit swizzle with 4-row groups.
-        // A K-step of KSTEP rows advances the start address by KSTEP*128 bytes.
-        const int nsteps = cur.n / Cfg::KSTEP;
-#pragma unroll 1
-        for (int kk = 0; kk < nsteps; ++kk)
-          mma_ts<TF32>(tmem + 128, tmem + kk * 8,
-                       dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
-                       (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(BAR(BAR_VE));
-        cur = nxt;
-        have = have_next;
-        ++j;
+      // K stage: refill with the next chunk once QK_j has read it
+      if (have_next) {
+        if (!(ok = wait_all(BAR(BAR_KE), j & 1, 1))) break;
+        load_kv(nxt, false);
+        ++nk;
       }
-      tc_commit(BAR(BAR_OF));
-      // Before the CTA may exit: every issued copy has landed, every MMA has completed.
-      tc_commit(BAR(BAR_DRAIN));
-      mbar_wait(BAR(BAR_DRAIN), 0, never, 23);
-      mbar_wait(BAR(BAR_Q), 0, never, 20);
-      if (nk) mbar_wait(BAR(BAR_KF), (nk - 1) & 1, never, 21);
-      if (nv) mbar_wait(BAR(BAR_VF), (nv - 1) & 1, never, 22);
+      if (!(ok = wait_all(BAR(BAR_PF), j & 1, 6))) break;
+      if (!(ok = wait_all(BAR(BAR_VF), j & 1, 7))) break;
+      tc_fence_after();
+      // V is MN-major (d contiguous): 128-byte rows, d chunks 16 KB apart; bf16 uses
+      // 8-row swizzle groups (1 KB), tf32 the 32-byte-unit swizzle with 4-row groups.
+      // A K-step of KSTEP rows advances the start address by KSTEP*128 bytes.
+      const int nsteps = cur.n / Cfg::KSTEP;
+#pragma unroll
+      for (int kk = 0; kk < 128 / Cfg::KSTEP; ++kk) {
+        if (kk < nsteps) {
+          if (elect_one())
+            mma_ts<TF32>(tmem + 128, tmem + kk * 8,
+                         dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+          __syncwarp();
+        }
+      }
+      commit(BAR(BAR_VE));
+      cur = nxt;
+      have = have_next;
+      ++j;
     }
+    commit(BAR(BAR_OF));
+    // Before the CTA may exit: every issued copy has landed, every MMA has completed.
+    commit(BAR(BAR_DRAIN));
+    mbar_wait(BAR(BAR_DRAIN), 0, never, 23);
+    mbar_wait(BAR(BAR_Q), 0, never, 20);
+    if (nk) mbar_wait(BAR(BAR_KF), (nk - 1) & 1, never, 21);
+    if (nv) mbar_wait(BAR(BAR_VF), (nv - 1) & 1, never, 22);
   } else {
     // ------------------------------------------------ softmax / epilogue (256 threads)
     // Two threads per query row: warps 1..4 own columns [0, 64) of every chunk, warps
@@ -632,19 +656,14 @@ __global__ void __maxnreg__(112)
         tmem_ld32(tS + c0 + 32, v1);
         tmem_wait_ld();
         if (fast) {
+          // raw logits; scale > 0, so the max of scale*s is scale*max(s)
           float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            m0 = fmaxf(m0, v0[c]);
-            m1 = fmaxf(m1, v1[c]);
+          for (int c = 0; c < 32; c += 2) {
+            m0 = max3(m0, v0[c], v0[c + 1]);
+            m1 = max3(m1, v1[c], v1[c + 1]);
           }
           mx = fmaxf(m0, m1) * scl;
-          // logits in log2 units
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            v0[c] *= scl;
-            v1[c] *= scl;
-          }
         } else {
           const float* bias = ch.centroid ? a.bias2 + ch.start + c0 : nullptr;
 #pragma unroll
@@ -673,13 +692,25 @@ __global__ void __maxnreg__(112)
       }
       if (nmine > 0) {
         const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
+        // exponent argument: fast chunks hold raw logits (x = s*scale - m), the others
+        // already hold log2-unit logits or -inf (x = v - m)
+        const float sx = fast ? scl : 1.f;
+        // 3 of every 8 pairs take the FMA-pipe polynomial, the rest MUFU ex2
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          v0[c] = ex2(v0[c] + neg_mu);
-          v1[c] = ex2(v1[c] + neg_mu);
-          s0 += v0[c];
-          s1 += v1[c];
+        for (int q = 0; q < 32; ++q) {
+          float* v = q < 16 ? v0 : v1;
+          const int c = (q & 15) * 2;
+          float x0, x1;
+          fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
+          if ((q & 7) < kPolyPairsOf8) {
+            if (fast) exp2_poly2<false>(v[c], v[c + 1], x0, x1);
+            else exp2_poly2<true>(v[c], v[c + 1], x0, x1);
+          } else {
+            v[c] = ex2(x0);
+            v[c + 1] = ex2(x1);
+          }
+          add2(s0, s1, s0, s1, v[c], v[c + 1]);
         }
         l_run += s0 + s1;
         // P over S in place: this half's 64 values become bf16 pairs in columns

@@ -91,6 +91,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// True in exactly one lane of a converged warp (elect.sync over all 32 lanes). Used
+// around per-thread instructions (tcgen05.mma, commits, TMA) inside warp-uniform code,
+// so their operands stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\t"
+      "elect.sync rx|px, %1;\n\t"
+      "@px mov.s32 %0, 1;\n\t}"
+      : "+r"(pred)
+      : "r"(0xffffffffu));
+  return pred != 0;
+}
+
 // Named barrier among `count` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -282,6 +296,59 @@ __host__ __device__ constexpr uint32_t make_idesc(bool tf32, int M, int N, bool 
          | ((tf32 ? 2u : 1u) << 10)                // B format
          | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Packed fp32 pair arithmetic (sm_100a f32x2): d = a*b + c and d = a + b, elementwise.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe (takes load off the MUFU unit). Range reduction
+// x = j + f with j = round(x), obtained by adding 1.5*2^23 (Cody-Waite style shifter),
+// f in [-1/2, 1/2]; 2^f by the degree-3 polynomial fitted for the minimax relative
+// error on [-1/2, 1/2] (gen_exp2_poly.py: 7.5e-5); 2^j added to the exponent field.
+// Inputs are clamped at -126 (the exponent add stays in range; results there are
+// below 2^-125); with kExactZero, inputs below -125.5 (masked -inf logits) return
+// exactly 0.
+constexpr float kExpC0 = 9.999280572e-01f;
+constexpr float kExpC1 = 6.932609677e-01f;
+constexpr float kExpC2 = 2.426111251e-01f;
+constexpr float kExpC3 = 5.517166853e-02f;
+template <bool kExactZero>
+__device__ __forceinline__ void exp2_poly2(float& e0, float& e1, float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  const float y0 = fmaxf(x0, -126.f), y1 = fmaxf(x1, -126.f);
+  float t0, t1, r0, r1, f0, f1, p0, p1;
+  add2(t0, t1, y0, y1, kShift, kShift);
+  add2(r0, r1, t0, t1, -kShift, -kShift);
+  fma2(f0, f1, r0, r1, -1.f, -1.f, y0, y1);
+  fma2(p0, p1, kExpC3, kExpC3, f0, f1, kExpC2, kExpC2);
+  fma2(p0, p1, p0, p1, f0, f1, kExpC1, kExpC1);
+  fma2(p0, p1, p0, p1, f0, f1, kExpC0, kExpC0);
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  if (kExactZero) {
+    e0 = x0 > -125.5f ? e0 : 0.f;
+    e1 = x1 > -125.5f ? e1 : 0.f;
+  }
 }
 
 __device__ __forceinline__ float ex2(float x) {
