@@ -329,8 +329,10 @@ struct AttnCfg {
   static constexpr int SMEM_LAUNCH = SMEM > 100 * 1024 ? SMEM : 100 * 1024;
 };
 
-enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SF, BAR_PF, BAR_OF, BAR_DRAIN,
-       BAR_X0, BAR_X1, BAR_X2, BAR_X3, NBAR };  // BAR_X*: row-pair exchange per lane quarter
+// Q/K/V full (TMA), K/V empty (MMA done reading), S full (QK done), P-low / P-high
+// ready (softmax of key columns 0..63 / 64..127 written), PV-low done, O final, drain.
+enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SF, BAR_PLO, BAR_PHI, BAR_OLO, BAR_OF,
+       BAR_DRAIN, NBAR };
 
 struct Chunk {
   int start;   // first key slot (token chunk) or first centroid (centroid chunk)
@@ -400,8 +402,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 template <int D, bool TF32>
-// 288 threads and at most 112 registers per thread: two CTAs share an SM.
-__global__ void __maxnreg__(112)
+// 160 threads (control warp + 4 softmax warps); two CTAs share an SM.
+__global__ void __launch_bounds__(160, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
                 const __grid_constant__ CUtensorMap tmVc, const AttnArgs a) {
@@ -429,7 +431,7 @@ __global__ void __maxnreg__(112)
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
 
   if (tid == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(BAR(i), i == BAR_PF ? 256u : (i >= BAR_X0 ? 64u : 1u));
+    for (int i = 0; i < NBAR; ++i) mbar_init(BAR(i), (i == BAR_PLO || i == BAR_PHI) ? 128u : 1u);
     *abort_flag = 0;
     *n_distinct = 0;
     *never = 0;
@@ -543,7 +545,6 @@ __global__ void __maxnreg__(112)
     }
     bool ok = wait_all(BAR(BAR_Q), 0, 3);
     while (ok && have) {
-      const bool have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
       if (!(ok = wait_all(BAR(BAR_KF), j & 1, 5))) break;
       tc_fence_after();
       const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(cur.n >> 3) << 17);
@@ -555,6 +556,8 @@ __global__ void __maxnreg__(112)
       }
       commit(BAR(BAR_KE));
       commit(BAR(BAR_SF));
+      // the next chunk is found while QK_j executes
+      const bool have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
       // V stage: refill once PV_{j-1} has read it (chunk 0 was loaded up front)
       if (j > 0) {
         if (!(ok = wait_all(BAR(BAR_VE), (j - 1) & 1, 4))) break;
@@ -567,20 +570,35 @@ __global__ void __maxnreg__(112)
         load_kv(nxt, false);
         ++nk;
       }
-      if (!(ok = wait_all(BAR(BAR_PF), j & 1, 6))) break;
+      // PV in two halves: keys 0..63 as soon as their P is written (P bf16 pairs in
+      // TMEM columns 0..31, fp32 in 0..63), keys 64..127 after the second half (P in
+      // columns 64..95 / 64..127). V is MN-major (d contiguous): 128-byte rows, d chunks
+      // 16 KB apart; bf16 uses 8-row swizzle groups (1 KB), tf32 the 32-byte-unit
+      // swizzle with 4-row groups; a K-step of KSTEP rows moves KSTEP*128 bytes.
+      constexpr int kHalfSteps = 64 / Cfg::KSTEP;
+      const int nsteps = cur.n / Cfg::KSTEP;
+      if (!(ok = wait_all(BAR(BAR_PLO), j & 1, 6))) break;
       if (!(ok = wait_all(BAR(BAR_VF), j & 1, 7))) break;
       tc_fence_after();
-      // V is MN-major (d contiguous): 128-byte rows, d chunks 16 KB apart; bf16 uses
-      // 8-row swizzle groups (1 KB), tf32 the 32-byte-unit swizzle with 4-row groups.
-      // A K-step of KSTEP rows advances the start address by KSTEP*128 bytes.
-      const int nsteps = cur.n / Cfg::KSTEP;
 #pragma unroll
-      for (int kk = 0; kk < 128 / Cfg::KSTEP; ++kk) {
+      for (int kk = 0; kk < kHalfSteps; ++kk) {
         if (kk < nsteps) {
           if (elect_one())
             mma_ts<TF32>(tmem + 128, tmem + kk * 8,
                          dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
                          (j > 0 || kk > 0) ? 1u : 0u);
+          __syncwarp();
+        }
+      }
+      commit(BAR(BAR_OLO));
+      if (!(ok = wait_all(BAR(BAR_PHI), j & 1, 8))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = kHalfSteps; kk < 2 * kHalfSteps; ++kk) {
+        if (kk < nsteps) {
+          if (elect_one())
+            mma_ts<TF32>(tmem + 128, tmem + 64 + (kk - kHalfSteps) * 8,
+                         dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV, 1u);
           __syncwarp();
         }
       }
@@ -597,14 +615,11 @@ __global__ void __maxnreg__(112)
     if (nk) mbar_wait(BAR(BAR_KF), (nk - 1) & 1, never, 21);
     if (nv) mbar_wait(BAR(BAR_VF), (nv - 1) & 1, never, 22);
   } else {
-    // ------------------------------------------------ softmax / epilogue (256 threads)
-    // Two threads per query row: warps 1..4 own columns [0, 64) of every chunk, warps
-    // 5..8 columns [64, 128). Warp w reads TMEM lanes 32*(w%4) .. +31, so each lane
-    // quarter has one warp of each half. The row max of a chunk is combined through
-    // shared memory with a 64-thread named barrier per quarter; both threads of a row
-    // then take identical rescaling decisions.
+    // ------------------------------------------------ softmax / epilogue (128 threads)
+    // One thread per query row (warps 1..4; warp w reads TMEM lanes 32*(w%4)..+31).
+    // Each chunk is taken as two online-softmax steps over key columns 0..63 and
+    // 64..127; after the first the PV of those keys starts while the second runs.
     const int quarter = warp & 3;
-    const int half = (warp - 1) >> 2;
     const int r = quarter * 32 + lane;
     const int qrow = tile * 128 + r;
     const int lab = a.qrow_label[qrow];
@@ -612,8 +627,7 @@ __global__ void __maxnreg__(112)
     const uint32_t* grow = gb + static_cast<size_t>(lab < 0 ? 0 : lab) * a.Wg;
     const uint32_t* crow = cb + static_cast<size_t>(lab < 0 ? 0 : lab) * a.Wc;
     const uint32_t tS = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t tO = tS + 128 + half * (D / 2);
-    const uint32_t xbar = BAR(BAR_X0 + quarter);  // the two threads of a row meet here
+    const uint32_t tO = tS + 128;
     const float scl = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     int gcur = 0, ccur = 0, j = 0;
@@ -622,153 +636,159 @@ __global__ void __maxnreg__(112)
     while (next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
       if (!(ok = mbar_wait(BAR(BAR_SF), j & 1, abort_flag, 9))) break;
       tc_fence_after();
-      const int c0 = half * 64;           // first column of this thread's half
-      const int nmine = ch.n - c0;        // columns of the chunk in this half (<= 0: none)
-      const bool fast = ch.uniform && nmine >= 64 && lab >= 0;
-      // column mask of this half (bit c = column c0 + c kept) for non-fast chunks
-      uint32_t mk0 = 0u, mk1 = 0u;
-      if (!fast && lab >= 0 && nmine > 0) {
-        if (ch.centroid) {
-          const int ww = (ch.start + c0) >> 5;
-          mk0 = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
-          mk1 = ww + 1 < a.Wc ? (~__ldg(crow + ww + 1) & __ldg(a.cnonempty + ww + 1)) : 0u;
-        } else {
-          const int gh0 = ch.g0 + half * 4;  // this half covers groups gh0 .. gh0+3
-          for (int jj = 0; jj < 4; ++jj) {
-            const int g = gh0 + jj;
-            if (half * 4 + jj < ch.ng && ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u)) {
-              const int nv = bit_at(a.gfull, g) ? 16 : __ldg(a.group_valid + g);
-              const uint32_t bits = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
-              if (jj < 2) mk0 |= bits << (jj * 16);
-              else mk1 |= bits << ((jj - 2) * 16);
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const int c0 = half * 64;         // first key column of this step
+        const int nmine = ch.n - c0;      // key columns of the chunk in this step
+        if (nmine > 0) {
+          const bool fast = ch.uniform && nmine >= 64 && lab >= 0;
+          // column mask (bit c = column c0 + c kept) for non-fast steps
+          uint32_t mk0 = 0u, mk1 = 0u;
+          if (!fast && lab >= 0) {
+            if (ch.centroid) {
+              const int ww = (ch.start + c0) >> 5;
+              mk0 = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
+              mk1 = ww + 1 < a.Wc ? (~__ldg(crow + ww + 1) & __ldg(a.cnonempty + ww + 1)) : 0u;
+            } else {
+              const int gh0 = ch.g0 + half * 4;  // this step covers groups gh0 .. gh0+3
+              for (int jj = 0; jj < 4; ++jj) {
+                const int g = gh0 + jj;
+                if (half * 4 + jj < ch.ng && ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u)) {
+                  const int nv = bit_at(a.gfull, g) ? 16 : __ldg(a.group_valid + g);
+                  const uint32_t bits = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
+                  if (jj < 2) mk0 |= bits << (jj * 16);
+                  else mk1 |= bits << ((jj - 2) * 16);
+                }
+              }
+            }
+            if (nmine < 64) {
+              mk1 = nmine <= 32 ? 0u : (mk1 & (0xffffffffu >> (64 - nmine)));
+              if (nmine < 32) mk0 &= 0xffffffffu >> (32 - nmine);
             }
           }
-        }
-        if (nmine < 64) {
-          mk1 = nmine <= 32 ? 0u : (mk1 & (0xffffffffu >> (64 - nmine)));
-          if (nmine < 32) mk0 &= 0xffffffffu >> (32 - nmine);
-        }
-      }
-      float v0[32], v1[32];
-      float mx = -INFINITY;
-      if (nmine > 0) {
-        tmem_ld32(tS + c0, v0);
-        tmem_ld32(tS + c0 + 32, v1);
-        tmem_wait_ld();
-        if (fast) {
-          // raw logits; scale > 0, so the max of scale*s is scale*max(s)
-          float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            m0 = max3(m0, v0[c], v0[c + 1]);
-            m1 = max3(m1, v1[c], v1[c + 1]);
-          }
-          mx = fmaxf(m0, m1) * scl;
-        } else {
-          const float* bias = ch.centroid ? a.bias2 + ch.start + c0 : nullptr;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float b0 = bias ? __ldg(bias + c) : 0.f;
-            const float b1 = bias ? __ldg(bias + 32 + c) : 0.f;
-            v0[c] = ((mk0 >> c) & 1u) ? fmaf(v0[c], scl, b0) : -INFINITY;
-            v1[c] = ((mk1 >> c) & 1u) ? fmaf(v1[c], scl, b1) : -INFINITY;
-            mx = fmaxf(mx, fmaxf(v0[c], v1[c]));
-          }
-        }
-      }
-      xchg[half * 128 + r] = mx;
-      mbar_arrive(xbar);
-      if (!(ok = mbar_wait(xbar, j & 1, abort_flag, 11))) break;
-      mx = fmaxf(xchg[r], xchg[128 + r]);
-      // Lazy rescaling: the running max only moves when the chunk max exceeds it by
-      // more than 8 (log2 units), so P stays below 256 and O is rarely touched.
-      const bool need = mx > m_run + 8.f;
-      const bool any_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2(m_run - mx);
-        l_run *= alpha;
-        m_run = mx;
-      }
-      if (nmine > 0) {
-        const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
-        // exponent argument: fast chunks hold raw logits (x = s*scale - m), the others
-        // already hold log2-unit logits or -inf (x = v - m)
-        const float sx = fast ? scl : 1.f;
-        // 3 of every 8 pairs take the FMA-pipe polynomial, the rest MUFU ex2
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          float* v = q < 16 ? v0 : v1;
-          const int c = (q & 15) * 2;
-          float x0, x1;
-          fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
-          if ((q & 7) < kPolyPairsOf8) {
-            if (fast) exp2_poly2<false>(v[c], v[c + 1], x0, x1);
-            else exp2_poly2<true>(v[c], v[c + 1], x0, x1);
-          } else {
-            v[c] = ex2(x0);
-            v[c + 1] = ex2(x1);
-          }
-          add2(s0, s1, s0, s1, v[c], v[c + 1]);
-        }
-        l_run += s0 + s1;
-        // P over S in place: this half's 64 values become bf16 pairs in columns
-        // [32*half, 32*half + 32), or fp32 in its own 64 columns for tf32. The other
-        // half's S columns were read before the barrier above.
-        if constexpr (TF32) {
-          tmem_st32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(v0));
-          tmem_st32(tS + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v1));
-        } else {
-          // pack in place: word i of each array takes elements 2i, 2i+1 (i <= 2i)
-          uint32_t* w0 = reinterpret_cast<uint32_t*>(v0);
-          uint32_t* w1 = reinterpret_cast<uint32_t*>(v1);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            w0[i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
-            w1[i] = pack_bf16x2(v1[2 * i], v1[2 * i + 1]);
-          }
-          tmem_st16(tS + half * 32, w0);
-          tmem_st16(tS + half * 32 + 16, w1);
-        }
-      }
-      // O (this half's D/2 columns) follows the running max before PV_j adds to it;
-      // nothing is in flight on O here: PV_{j-1} completed before S_j was ready.
-      if (any_need && j > 0) {
-#pragma unroll 1
-        for (int p = 0; p < D / 64; ++p) {
-          float o[32];
-          tmem_ld32(tO + p * 32, o);
+          float v0[32], v1[32];
+          tmem_ld32(tS + c0, v0);
+          tmem_ld32(tS + c0 + 32, v1);
           tmem_wait_ld();
+          float mx = -INFINITY;
+          if (fast) {
+            // raw logits; scale > 0, so the max of scale*s is scale*max(s)
+            float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] *= alpha;
-          tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+            for (int c = 0; c < 32; c += 2) {
+              m0 = max3(m0, v0[c], v0[c + 1]);
+              m1 = max3(m1, v1[c], v1[c + 1]);
+            }
+            mx = fmaxf(m0, m1) * scl;
+          } else {
+            const float* bias = ch.centroid ? a.bias2 + ch.start + c0 : nullptr;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float b0 = bias ? __ldg(bias + c) : 0.f;
+              const float b1 = bias ? __ldg(bias + 32 + c) : 0.f;
+              v0[c] = ((mk0 >> c) & 1u) ? fmaf(v0[c], scl, b0) : -INFINITY;
+              v1[c] = ((mk1 >> c) & 1u) ? fmaf(v1[c], scl, b1) : -INFINITY;
+              mx = fmaxf(mx, fmaxf(v0[c], v1[c]));
+            }
+          }
+          // Lazy rescaling: the running max only moves when the step max exceeds it by
+          // more than 8 (log2 units), so P stays below 256 and O is rarely touched.
+          const bool need = mx > m_run + 8.f;
+          const bool any_need = __any_sync(0xffffffffu, need);
+          float alpha = 1.f;
+          if (need) {
+            alpha = ex2(m_run - mx);
+            l_run *= alpha;
+            m_run = mx;
+          }
+          const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
+          // exponent argument: fast steps hold raw logits (x = s*scale - m), the others
+          // log2-unit logits or -inf (x = v - m)
+          const float sx = fast ? scl : 1.f;
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            float* v = q < 16 ? v0 : v1;
+            const int c = (q & 15) * 2;
+            float x0, x1;
+            fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
+            if ((q & 7) < kPolyPairsOf8) {
+              if (fast) exp2_poly2<false>(v[c], v[c + 1], x0, x1);
+              else exp2_poly2<true>(v[c], v[c + 1], x0, x1);
+            } else {
+              v[c] = ex2(x0);
+              v[c + 1] = ex2(x1);
+            }
+            add2(s0, s1, s0, s1, v[c], v[c + 1]);
+          }
+          l_run += s0 + s1;
+          // P over S in place: bf16 pairs of step h in columns [64h, 64h+32) (step 0's
+          // S columns were read above; step 1 lands on its own S columns), fp32 in the
+          // step's own 64 columns.
+          if constexpr (TF32) {
+            tmem_st32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(v0));
+            tmem_st32(tS + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v1));
+          } else {
+            uint32_t* w0 = reinterpret_cast<uint32_t*>(v0);
+            uint32_t* w1 = reinterpret_cast<uint32_t*>(v1);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              w0[i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
+              w1[i] = pack_bf16x2(v1[2 * i], v1[2 * i + 1]);
+            }
+            tmem_st16(tS + c0, w0);
+            tmem_st16(tS + c0 + 16, w1);
+          }
+          // O follows the running max before this step's PV adds to it. Step 0: PV of
+          // the previous chunk completed before S was ready. Step 1: wait for the PV of
+          // step 0, which may still run.
+          if (any_need && j > 0) {
+            if (half == 1 && !(ok = mbar_wait(BAR(BAR_OLO), j & 1, abort_flag, 12))) break;
+            if (half == 1) tc_fence_after();
+#pragma unroll 1
+            for (int p = 0; p < D / 32; ++p) {
+              float o[32];
+              tmem_ld32(tO + p * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] *= alpha;
+              tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+            }
+          } else if (any_need && half == 1 && j == 0) {
+            // first chunk: the PV of step 0 wrote O without accumulation; rescale it too
+            if (!(ok = mbar_wait(BAR(BAR_OLO), 0, abort_flag, 12))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int p = 0; p < D / 32; ++p) {
+              float o[32];
+              tmem_ld32(tO + p * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] *= alpha;
+              tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+            }
+          }
+          tmem_wait_st();
         }
+        tc_fence_before();
+        mbar_arrive(BAR(half == 0 ? BAR_PLO : BAR_PHI));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR(BAR_PF));
+      if (!ok) break;
       ++j;
     }
-    // row sum of both halves
-    xchg[256 + half * 128 + r] = l_run;
-    mbar_arrive(xbar);
-    if (ok) ok = mbar_wait(xbar, j & 1, abort_flag, 12);
-    const float l_tot = xchg[256 + r] + xchg[256 + 128 + r];
     if (ok && mbar_wait(BAR(BAR_OF), 0, abort_flag, 10)) {
       tc_fence_after();
-      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      float* orow = a.out + ((static_cast<size_t>(b) * a.Hq + h) * a.Sq + (tok >= 0 ? tok : 0)) * D +
-                    half * (D / 2);
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      float* orow = a.out + ((static_cast<size_t>(b) * a.Hq + h) * a.Sq + (tok >= 0 ? tok : 0)) * D;
 #pragma unroll 1
-      for (int p = 0; p < D / 64; ++p) {
+      for (int p = 0; p < D / 32; ++p) {
         float o[32];
         tmem_ld32(tO + p * 32, o);
         tmem_wait_ld();
         if (tok >= 0) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            float4 v4 = l_tot > 0.f ? make_float4(o[4 * i] * inv, o[4 * i + 1] * inv,
+            float4 v4 = l_run > 0.f ? make_float4(o[4 * i] * inv, o[4 * i + 1] * inv,
                                                   o[4 * i + 2] * inv, o[4 * i + 3] * inv)
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
             *reinterpret_cast<float4*>(orow + p * 32 + 4 * i) = v4;
@@ -842,7 +862,7 @@ int launch_attn(const CUtensorMap* maps, const AttnArgs& args, dim3 grid, int pr
                                        Cfg::SMEM_LAUNCH);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(attn_kernel)");
   prof_begin(prof_id, st);
-  kern<<<grid, 288, Cfg::SMEM_LAUNCH, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
+  kern<<<grid, 160, Cfg::SMEM_LAUNCH, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
   count_launch();
   prof_end(prof_id, st);
   return check_cuda(cudaGetLastError(), "attn_kernel launch");
