@@ -329,10 +329,11 @@ struct AttnCfg {
   static constexpr int SMEM_LAUNCH = SMEM > 100 * 1024 ? SMEM : 100 * 1024;
 };
 
-// Q/K/V full (TMA), K/V empty (MMA done reading), S full (QK done), P-low / P-high
-// ready (softmax of key columns 0..63 / 64..127 written), PV-low done, O final, drain.
-enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SF, BAR_PLO, BAR_PHI, BAR_OLO, BAR_OF,
-       BAR_DRAIN, NBAR };
+// Q/K/V full (TMA), K/V empty (MMA done reading), S-low / S-high full (QK of key
+// columns 0..63 / 64..127 done), P-low / P-high ready (softmax of those columns
+// written), PV-low done, O final, drain.
+enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SFLO, BAR_SFHI, BAR_PLO, BAR_PHI, BAR_OLO,
+       BAR_OF, BAR_DRAIN, NBAR };
 
 struct Chunk {
   int start;   // first key slot (token chunk) or first centroid (centroid chunk)
@@ -421,7 +422,6 @@ __global__ void __launch_bounds__(160, 2)
   uint32_t* any_bits = reinterpret_cast<uint32_t*>(distinct + 128);  // 128 words
   uint32_t* uni_bits = any_bits + 128;                                // 128 words
   uint32_t* cneed = uni_bits + 128;                                   // 4 words
-  float* xchg = reinterpret_cast<float*>(cneed + 4);                  // 512 floats
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(160, 2)
       __syncwarp();
     };
     int gcur = 0, ccur = 0, j = 0, nk = 0, nv = 0;
-    Chunk cur, nxt;
+    Chunk cur, nxt, nn;
     bool have = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, cur);
     if (leader) {
       mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
@@ -543,68 +543,110 @@ __global__ void __launch_bounds__(160, 2)
       load_kv(cur, true);
       ++nv;
     }
-    bool ok = wait_all(BAR(BAR_Q), 0, 3);
-    while (ok && have) {
-      if (!(ok = wait_all(BAR(BAR_KF), j & 1, 5))) break;
-      tc_fence_after();
-      const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(cur.n >> 3) << 17);
+    // S = Q Kᵀ for key columns [64h, 64h + n_h) of chunk c into TMEM columns 64h.. (N = n_h).
+    auto issue_qk_half = [&](const Chunk& c, int hlf) {
+      const int nh = min(64, c.n - 64 * hlf);
+      if (nh > 0) {
+        const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(nh >> 3) << 17);
+        const uint64_t krow = static_cast<uint64_t>((hlf * 64 * 128) >> 4);  // 64 rows of 128 B
 #pragma unroll
-      for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
-        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-        if (elect_one()) mma_ss<TF32>(tmem, dQ + off, dK + off, idesc, kk > 0 ? 1u : 0u);
-        __syncwarp();
+        for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          if (elect_one())
+            mma_ss<TF32>(tmem + 64 * hlf, dQ + off, dK + off + krow, idesc, kk > 0 ? 1u : 0u);
+          __syncwarp();
+        }
       }
-      commit(BAR(BAR_KE));
-      commit(BAR(BAR_SF));
-      // the next chunk is found while QK_j executes
-      const bool have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
-      // V stage: refill once PV_{j-1} has read it (chunk 0 was loaded up front)
-      if (j > 0) {
-        if (!(ok = wait_all(BAR(BAR_VE), (j - 1) & 1, 4))) break;
-        load_kv(cur, true);
-        ++nv;
-      }
-      // K stage: refill with the next chunk once QK_j has read it
-      if (have_next) {
-        if (!(ok = wait_all(BAR(BAR_KE), j & 1, 1))) break;
-        load_kv(nxt, false);
-        ++nk;
-      }
-      // PV in two halves: keys 0..63 as soon as their P is written (P bf16 pairs in
-      // TMEM columns 0..31, fp32 in 0..63), keys 64..127 after the second half (P in
-      // columns 64..95 / 64..127). V is MN-major (d contiguous): 128-byte rows, d chunks
-      // 16 KB apart; bf16 uses 8-row swizzle groups (1 KB), tf32 the 32-byte-unit
-      // swizzle with 4-row groups; a K-step of KSTEP rows moves KSTEP*128 bytes.
+    };
+    // O += P V for key rows [64h, 64h + n_h); P of step h sits at TMEM columns 64h..
+    // (bf16 pairs: 32 columns, fp32: 64). V is MN-major (d contiguous): 128-byte rows,
+    // d chunks 16 KB apart; bf16 uses 8-row swizzle groups (1 KB), tf32 the
+    // 32-byte-unit swizzle with 4-row groups; a K-step of KSTEP rows moves KSTEP*128 B.
+    auto issue_pv_half = [&](const Chunk& c, int hlf, bool first_chunk) {
       constexpr int kHalfSteps = 64 / Cfg::KSTEP;
-      const int nsteps = cur.n / Cfg::KSTEP;
+      const int nsteps = c.n / Cfg::KSTEP;
+#pragma unroll
+      for (int t = 0; t < kHalfSteps; ++t) {
+        const int kk = hlf * kHalfSteps + t;
+        if (kk < nsteps) {
+          if (elect_one())
+            mma_ts<TF32>(tmem + 128, tmem + 64 * hlf + t * 8,
+                         dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
+                         (!first_chunk || kk > 0) ? 1u : 0u);
+          __syncwarp();
+        }
+      }
+    };
+    bool ok = wait_all(BAR(BAR_Q), 0, 3);
+    bool have_next = false, have_nn = false;
+    int hi_c = 0;  // chunks with a high step whose P-high the control has waited for
+    if (ok && have) {
+      ok = wait_all(BAR(BAR_KF), 0, 5);
+      if (ok) {
+        tc_fence_after();
+        issue_qk_half(cur, 0);
+        commit(BAR(BAR_SFLO));
+        if (cur.n > 64) {
+          issue_qk_half(cur, 1);
+          commit(BAR(BAR_SFHI));
+        }
+        commit(BAR(BAR_KE));
+        have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
+        if (have_next && (ok = wait_all(BAR(BAR_KE), 0, 1))) {
+          load_kv(nxt, false);
+          ++nk;
+        }
+      }
+    }
+    // Steady state for chunk j: PV-low(j) | QK-low(j+1) | PV-high(j) | QK-high(j+1), so
+    // the tensor core works on the next chunk's low keys while the softmax warps are on
+    // chunk j's high keys, and on the next chunk's high keys while they start chunk j+1.
+    while (ok && have) {
       if (!(ok = wait_all(BAR(BAR_PLO), j & 1, 6))) break;
       if (!(ok = wait_all(BAR(BAR_VF), j & 1, 7))) break;
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kHalfSteps; ++kk) {
-        if (kk < nsteps) {
-          if (elect_one())
-            mma_ts<TF32>(tmem + 128, tmem + kk * 8,
-                         dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
-                         (j > 0 || kk > 0) ? 1u : 0u);
-          __syncwarp();
-        }
-      }
+      issue_pv_half(cur, 0, j == 0);
       commit(BAR(BAR_OLO));
-      if (!(ok = wait_all(BAR(BAR_PHI), j & 1, 8))) break;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = kHalfSteps; kk < 2 * kHalfSteps; ++kk) {
-        if (kk < nsteps) {
-          if (elect_one())
-            mma_ts<TF32>(tmem + 128, tmem + 64 + (kk - kHalfSteps) * 8,
-                         dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV, 1u);
-          __syncwarp();
-        }
+      if (have_next) {
+        // MMAs of one thread run in issue order: QK-low(j+1) overwrites P-low(j) only
+        // after PV-low(j) has read it.
+        if (!(ok = wait_all(BAR(BAR_KF), (j + 1) & 1, 5))) break;
+        tc_fence_after();
+        issue_qk_half(nxt, 0);
+        commit(BAR(BAR_SFLO));
+      }
+      // The high step exists only for chunks of more than 64 keys; its barriers count
+      // those chunks alone (hi_c / hi_n), on both sides.
+      if (cur.n > 64) {
+        if (!(ok = wait_all(BAR(BAR_PHI), hi_c & 1, 8))) break;
+        ++hi_c;
+        tc_fence_after();
+        issue_pv_half(cur, 1, j == 0);
       }
       commit(BAR(BAR_VE));
+      have_nn = false;
+      if (have_next) {
+        if (nxt.n > 64) {
+          issue_qk_half(nxt, 1);
+          commit(BAR(BAR_SFHI));
+        }
+        commit(BAR(BAR_KE));
+        // V stage: refill with the next chunk once PV(j) has read it
+        if (!(ok = wait_all(BAR(BAR_VE), j & 1, 4))) break;
+        load_kv(nxt, true);
+        ++nv;
+        // K stage: refill with the chunk after once QK(j+1) has read it
+        have_nn = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nn);
+        if (have_nn) {
+          if (!(ok = wait_all(BAR(BAR_KE), (j + 1) & 1, 1))) break;
+          load_kv(nn, false);
+          ++nk;
+        }
+      }
       cur = nxt;
+      nxt = nn;
       have = have_next;
+      have_next = have_nn;
       ++j;
     }
     commit(BAR(BAR_OF));
@@ -630,17 +672,20 @@ __global__ void __launch_bounds__(160, 2)
     const uint32_t tO = tS + 128;
     const float scl = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    int gcur = 0, ccur = 0, j = 0;
+    int gcur = 0, ccur = 0, j = 0, hi_n = 0;  // hi_n: high steps taken so far
     bool ok = true;
     Chunk ch;
     while (next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
-      if (!(ok = mbar_wait(BAR(BAR_SF), j & 1, abort_flag, 9))) break;
-      tc_fence_after();
+      const int nsteps = ch.n > 64 ? 2 : 1;
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < nsteps; ++half) {
         const int c0 = half * 64;         // first key column of this step
         const int nmine = ch.n - c0;      // key columns of the chunk in this step
-        if (nmine > 0) {
+        {
+          if (!(ok = mbar_wait(BAR(half == 0 ? BAR_SFLO : BAR_SFHI), half == 0 ? (j & 1) : (hi_n & 1),
+                               abort_flag, 9)))
+            break;
+          tc_fence_after();
           const bool fast = ch.uniform && nmine >= 64 && lab >= 0;
           // column mask (bit c = column c0 + c kept) for non-fast steps
           uint32_t mk0 = 0u, mk1 = 0u;
@@ -739,12 +784,13 @@ __global__ void __launch_bounds__(160, 2)
             tmem_st16(tS + c0, w0);
             tmem_st16(tS + c0 + 16, w1);
           }
-          // O follows the running max before this step's PV adds to it. Step 0: PV of
-          // the previous chunk completed before S was ready. Step 1: wait for the PV of
-          // step 0, which may still run.
+          // O follows the running max before this step's PV adds to it. Step 0: wait
+          // for the last PV of the previous chunk; step 1: for the PV of step 0.
           if (any_need && j > 0) {
-            if (half == 1 && !(ok = mbar_wait(BAR(BAR_OLO), j & 1, abort_flag, 12))) break;
-            if (half == 1) tc_fence_after();
+            if (!(ok = mbar_wait(BAR(half == 0 ? BAR_VE : BAR_OLO), half == 0 ? ((j - 1) & 1) : (j & 1),
+                                 abort_flag, 12)))
+              break;
+            tc_fence_after();
 #pragma unroll 1
             for (int p = 0; p < D / 32; ++p) {
               float o[32];
@@ -772,6 +818,7 @@ __global__ void __launch_bounds__(160, 2)
         }
         tc_fence_before();
         mbar_arrive(BAR(half == 0 ? BAR_PLO : BAR_PHI));
+        hi_n += half;
       }
       if (!ok) break;
       ++j;
