@@ -686,55 +686,79 @@ __global__ void __launch_bounds__(160, 2)
                                abort_flag, 9)))
             break;
           tc_fence_after();
-          const bool fast = ch.uniform && nmine >= 64 && lab >= 0;
-          // column mask (bit c = column c0 + c kept) for non-fast steps
-          uint32_t mk0 = 0u, mk1 = 0u;
-          if (!fast && lab >= 0) {
-            if (ch.centroid) {
-              const int ww = (ch.start + c0) >> 5;
-              mk0 = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
-              mk1 = ww + 1 < a.Wc ? (~__ldg(crow + ww + 1) & __ldg(a.cnonempty + ww + 1)) : 0u;
-            } else {
-              const int gh0 = ch.g0 + half * 4;  // this step covers groups gh0 .. gh0+3
-              for (int jj = 0; jj < 4; ++jj) {
-                const int g = gh0 + jj;
-                if (half * 4 + jj < ch.ng && ((__ldg(grow + (g >> 5)) >> (g & 31)) & 1u)) {
-                  const int nv = bit_at(a.gfull, g) ? 16 : __ldg(a.group_valid + g);
-                  const uint32_t bits = nv >= 16 ? 0xffffu : ((1u << nv) - 1u);
-                  if (jj < 2) mk0 |= bits << (jj * 16);
-                  else mk1 |= bits << ((jj - 2) * 16);
-                }
-              }
-            }
-            if (nmine < 64) {
-              mk1 = nmine <= 32 ? 0u : (mk1 & (0xffffffffu >> (64 - nmine)));
-              if (nmine < 32) mk0 &= 0xffffffffu >> (32 - nmine);
-            }
-          }
+          // Token chunks are masked per 16-key group (a key cluster is kept or dropped
+          // whole): a warp vote tells, per group, whether no row, every row or only some
+          // rows of the warp keep it. Groups no row keeps get P = 0 without exponentials,
+          // groups every row keeps need no select. Columns past a cluster's last token
+          // (pad slots of its last group) and pad query rows are set to -inf.
+          // Centroid chunks are masked per column and carry the log2 n_c bias.
           float v0[32], v1[32];
           tmem_ld32(tS + c0, v0);
           tmem_ld32(tS + c0 + 32, v1);
-          tmem_wait_ld();
+          uint32_t any4 = 0xfu;  // groups whose exponentials this warp computes
           float mx = -INFINITY;
-          if (fast) {
-            // raw logits; scale > 0, so the max of scale*s is scale*max(s)
-            float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              m0 = max3(m0, v0[c], v0[c + 1]);
-              m1 = max3(m1, v1[c], v1[c + 1]);
+          float sx = scl;        // exponent argument x = v * sx - m
+          if (!ch.centroid) {
+            const int ngs = nmine >= 64 ? 4 : (nmine >> 4);
+            const uint32_t present = (1u << ngs) - 1u;
+            const int gh0 = ch.g0 + half * 4;  // this step covers groups gh0 .. gh0+3
+            uint32_t kb = present, partial = 0u;
+            if (!ch.uniform) {
+              const int w = gh0 >> 5, sh = gh0 & 31;
+              const bool two = w + 1 < a.Wg;
+              const uint64_t kw = static_cast<uint64_t>(__ldg(grow + w)) |
+                                  (two ? static_cast<uint64_t>(__ldg(grow + w + 1)) << 32 : 0ull);
+              const uint64_t fw = static_cast<uint64_t>(__ldg(a.gfull + w)) |
+                                  (two ? static_cast<uint64_t>(__ldg(a.gfull + w + 1)) << 32 : 0ull);
+              kb = static_cast<uint32_t>(kw >> sh) & present;
+              partial = ~static_cast<uint32_t>(fw >> sh) & present;
             }
-            mx = fmaxf(m0, m1) * scl;
+            if (lab < 0) kb = 0u;
+            any4 = __reduce_or_sync(0xffffffffu, kb);
+            const uint32_t all4 = __reduce_and_sync(0xffffffffu, kb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              if ((any4 >> jj) & 1u) {
+                float* v = jj < 2 ? v0 : v1;
+                const int o = (jj & 1) * 16;
+                if ((partial >> jj) & 1u) {
+                  const int nv = __ldg(a.group_valid + gh0 + jj);
+#pragma unroll
+                  for (int c = 1; c < 16; ++c) v[o + c] = c < nv ? v[o + c] : -INFINITY;
+                }
+                if (!((all4 >> jj) & 1u)) {
+                  const bool keep = (kb >> jj) & 1u;
+#pragma unroll
+                  for (int c = 0; c < 16; ++c) v[o + c] = keep ? v[o + c] : -INFINITY;
+                }
+                float ma = max3(v[o], v[o + 1], v[o + 2]);
+                float mb = max3(v[o + 8], v[o + 9], v[o + 10]);
+                ma = max3(ma, v[o + 3], v[o + 4]);
+                mb = max3(mb, v[o + 11], v[o + 12]);
+                ma = max3(ma, v[o + 5], v[o + 6]);
+                mb = max3(mb, v[o + 13], v[o + 14]);
+                mx = max3(mx, fmaxf(ma, v[o + 7]), fmaxf(mb, v[o + 15]));
+              }
+            }
+            // raw logits; scale > 0, so the max of scale*s is scale*max(s)
+            mx *= scl;
           } else {
-            const float* bias = ch.centroid ? a.bias2 + ch.start + c0 : nullptr;
+            uint32_t mk0 = 0u, mk1 = 0u;  // bit c: column c0 + c (+ 32) kept
+            if (lab >= 0) {
+              const int ww = (ch.start + c0) >> 5;
+              mk0 = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
+              mk1 = ww + 1 < a.Wc ? (~__ldg(crow + ww + 1) & __ldg(a.cnonempty + ww + 1)) : 0u;
+            }
+            const float* bias = a.bias2 + ch.start + c0;
+            tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const float b0 = bias ? __ldg(bias + c) : 0.f;
-              const float b1 = bias ? __ldg(bias + 32 + c) : 0.f;
-              v0[c] = ((mk0 >> c) & 1u) ? fmaf(v0[c], scl, b0) : -INFINITY;
-              v1[c] = ((mk1 >> c) & 1u) ? fmaf(v1[c], scl, b1) : -INFINITY;
-              mx = fmaxf(mx, fmaxf(v0[c], v1[c]));
+              v0[c] = ((mk0 >> c) & 1u) ? fmaf(v0[c], scl, __ldg(bias + c)) : -INFINITY;
+              v1[c] = ((mk1 >> c) & 1u) ? fmaf(v1[c], scl, __ldg(bias + 32 + c)) : -INFINITY;
+              mx = max3(mx, v0[c], v1[c]);
             }
+            sx = 1.f;  // log2-unit logits or -inf
           }
           // Lazy rescaling: the running max only moves when the step max exceeds it by
           // more than 8 (log2 units), so P stays below 256 and O is rarely touched.
@@ -747,24 +771,25 @@ __global__ void __launch_bounds__(160, 2)
             m_run = mx;
           }
           const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
-          // exponent argument: fast steps hold raw logits (x = s*scale - m), the others
-          // log2-unit logits or -inf (x = v - m)
-          const float sx = fast ? scl : 1.f;
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll
           for (int q = 0; q < 32; ++q) {
             float* v = q < 16 ? v0 : v1;
             const int c = (q & 15) * 2;
-            float x0, x1;
-            fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
-            if ((q & 7) < kPolyPairsOf8) {
-              if (fast) exp2_poly2<false>(v[c], v[c + 1], x0, x1);
-              else exp2_poly2<true>(v[c], v[c + 1], x0, x1);
+            if ((any4 >> (q >> 3)) & 1u) {
+              float x0, x1;
+              fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
+              if ((q & 7) < kPolyPairsOf8) {
+                exp2_poly2<true>(v[c], v[c + 1], x0, x1);
+              } else {
+                v[c] = ex2(x0);
+                v[c + 1] = ex2(x1);
+              }
+              add2(s0, s1, s0, s1, v[c], v[c + 1]);
             } else {
-              v[c] = ex2(x0);
-              v[c + 1] = ex2(x1);
+              v[c] = 0.f;
+              v[c + 1] = 0.f;
             }
-            add2(s0, s1, s0, s1, v[c], v[c + 1]);
           }
           l_run += s0 + s1;
           // P over S in place: bf16 pairs of step h in columns [64h, 64h+32) (step 0's
