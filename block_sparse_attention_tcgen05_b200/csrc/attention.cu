@@ -397,6 +397,15 @@ __device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t*
 // 0: measured fastest in this kernel (the softmax warps are issue-bound, not MUFU-bound).
 constexpr int kPolyPairsOf8 = 0;
 
+// Max of 16 / 64 register values as shallow trees of 3-input maxes.
+__device__ __forceinline__ float max16(const float* v) {
+  return fmaxf(max3(max3(v[0], v[1], v[2]), max3(v[3], v[4], v[5]), fmaxf(v[6], v[7])),
+               max3(max3(v[8], v[9], v[10]), max3(v[11], v[12], v[13]), fmaxf(v[14], v[15])));
+}
+__device__ __forceinline__ float max64(const float (&a)[32], const float (&b)[32]) {
+  return fmaxf(max3(max16(a), max16(a + 16), max16(b)), max16(b + 16));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -695,8 +704,8 @@ __global__ void __launch_bounds__(160, 2)
           float v0[32], v1[32];
           tmem_ld32(tS + c0, v0);
           tmem_ld32(tS + c0 + 32, v1);
-          uint32_t any4 = 0xfu;  // groups whose exponentials this warp computes
-          float mx = -INFINITY;
+          uint32_t any4 = 0xfu;  // groups of this step whose exponentials the warp computes
+          float mx;
           float sx = scl;        // exponent argument x = v * sx - m
           if (!ch.centroid) {
             const int ngs = nmine >= 64 ? 4 : (nmine >> 4);
@@ -715,11 +724,13 @@ __global__ void __launch_bounds__(160, 2)
             }
             if (lab < 0) kb = 0u;
             any4 = __reduce_or_sync(0xffffffffu, kb);
-            const uint32_t all4 = __reduce_and_sync(0xffffffffu, kb);
+            const uint32_t mixed = any4 & ~__reduce_and_sync(0xffffffffu, kb);
             tmem_wait_ld();
+            if (partial | mixed) {
+              // -inf for the pad slots of a cluster's last group, and for rows that drop
+              // a group another row of the warp keeps
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              if ((any4 >> jj) & 1u) {
+              for (int jj = 0; jj < 4; ++jj) {
                 float* v = jj < 2 ? v0 : v1;
                 const int o = (jj & 1) * 16;
                 if ((partial >> jj) & 1u) {
@@ -727,22 +738,23 @@ __global__ void __launch_bounds__(160, 2)
 #pragma unroll
                   for (int c = 1; c < 16; ++c) v[o + c] = c < nv ? v[o + c] : -INFINITY;
                 }
-                if (!((all4 >> jj) & 1u)) {
+                if ((mixed >> jj) & 1u) {
                   const bool keep = (kb >> jj) & 1u;
 #pragma unroll
                   for (int c = 0; c < 16; ++c) v[o + c] = keep ? v[o + c] : -INFINITY;
                 }
-                float ma = max3(v[o], v[o + 1], v[o + 2]);
-                float mb = max3(v[o + 8], v[o + 9], v[o + 10]);
-                ma = max3(ma, v[o + 3], v[o + 4]);
-                mb = max3(mb, v[o + 11], v[o + 12]);
-                ma = max3(ma, v[o + 5], v[o + 6]);
-                mb = max3(mb, v[o + 13], v[o + 14]);
-                mx = max3(mx, fmaxf(ma, v[o + 7]), fmaxf(mb, v[o + 15]));
               }
             }
             // raw logits; scale > 0, so the max of scale*s is scale*max(s)
-            mx *= scl;
+            if (any4 == 0xfu) {
+              mx = max64(v0, v1) * scl;
+            } else {
+              mx = -INFINITY;
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj)
+                if ((any4 >> jj) & 1u) mx = fmaxf(mx, max16((jj < 2 ? v0 : v1) + (jj & 1) * 16));
+              mx *= scl;
+            }
           } else {
             uint32_t mk0 = 0u, mk1 = 0u;  // bit c: column c0 + c (+ 32) kept
             if (lab >= 0) {
@@ -756,8 +768,8 @@ __global__ void __launch_bounds__(160, 2)
             for (int c = 0; c < 32; ++c) {
               v0[c] = ((mk0 >> c) & 1u) ? fmaf(v0[c], scl, __ldg(bias + c)) : -INFINITY;
               v1[c] = ((mk1 >> c) & 1u) ? fmaf(v1[c], scl, __ldg(bias + 32 + c)) : -INFINITY;
-              mx = max3(mx, v0[c], v1[c]);
             }
+            mx = max64(v0, v1);
             sx = 1.f;  // log2-unit logits or -inf
           }
           // Lazy rescaling: the running max only moves when the step max exceeds it by
@@ -771,12 +783,14 @@ __global__ void __launch_bounds__(160, 2)
             m_run = mx;
           }
           const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
-          float s0 = 0.f, s1 = 0.f;
+          // Two independent pair sums keep the add chain short. Groups no row of the
+          // warp keeps are zero; the common all-groups case runs as straight-line code.
+          float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+          if (any4 == 0xfu) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            float* v = q < 16 ? v0 : v1;
-            const int c = (q & 15) * 2;
-            if ((any4 >> (q >> 3)) & 1u) {
+            for (int q = 0; q < 32; ++q) {
+              float* v = q < 16 ? v0 : v1;
+              const int c = (q & 15) * 2;
               float x0, x1;
               fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
               if ((q & 7) < kPolyPairsOf8) {
@@ -785,13 +799,32 @@ __global__ void __launch_bounds__(160, 2)
                 v[c] = ex2(x0);
                 v[c + 1] = ex2(x1);
               }
-              add2(s0, s1, s0, s1, v[c], v[c + 1]);
-            } else {
-              v[c] = 0.f;
-              v[c + 1] = 0.f;
+              if (q & 1) add2(sb0, sb1, sb0, sb1, v[c], v[c + 1]);
+              else add2(sa0, sa1, sa0, sa1, v[c], v[c + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              float* v = jj < 2 ? v0 : v1;
+              const int o = (jj & 1) * 16;
+              if ((any4 >> jj) & 1u) {
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                  const int c = o + 2 * p;
+                  float x0, x1;
+                  fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
+                  v[c] = ex2(x0);
+                  v[c + 1] = ex2(x1);
+                  if (p & 1) add2(sb0, sb1, sb0, sb1, v[c], v[c + 1]);
+                  else add2(sa0, sa1, sa0, sa1, v[c], v[c + 1]);
+                }
+              } else {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) v[o + c] = 0.f;
+              }
             }
           }
-          l_run += s0 + s1;
+          l_run += (sa0 + sa1) + (sb0 + sb1);
           // P over S in place: bf16 pairs of step h in columns [64h, 64h+32) (step 0's
           // S columns were read above; step 1 lands on its own S columns), fp32 in the
           // step's own 64 columns.
