@@ -46,7 +46,7 @@ METRIC = "effective TFLOP/s on executed pairs, centroid-compensated block-sparse
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=60)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -110,6 +110,14 @@ class ClockSampler:
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
+            return
+        # nvidia-smi takes a moment to start: wait (up to 3 s) for its first sample so
+        # that the samples cover the timed region.
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and self.proc.poll() is None:
+            if os.path.getsize(self.file.name) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:

@@ -110,8 +110,9 @@ int bsa_tile_labels(int T, int H, int W, int tt, int th, int tw, int32_t* labels
  *   P      = row-softmax(logit_scale * A) over all S/s columns
  *   scores[b,h,i,j] = (s/block) * sum over the (block/s)^2 entries of tile (i,j)
  * q: (B,Hq,S,D), k: (B,Hkv,S,D) with shape.Sq == shape.Sk == S; S % block == 0,
- * block % stride == 0, block/stride <= 128, S/stride a multiple of 128,
- * S/stride <= 8192; D in {64,128}; BSA_BF16 only. logit_scale <= 0 selects 1/sqrt(D).
+ * block % stride == 0, block/stride a power of two <= 32, S/stride a multiple of 128
+ * and <= 2048, S/block <= 256; D in {64,128}; BSA_BF16 only (other sizes return
+ * BSA_ERR_UNSUPPORTED). logit_scale <= 0 selects 1/sqrt(D).
  *   scores : device float32 (B, Hq, S/block, S/block), written; each row sums to 1.
  * The strided logit matrix is never written to device memory. No workspace.
  */
