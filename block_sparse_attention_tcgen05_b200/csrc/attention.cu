@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(256) gather_kv_centroids_kernel(
 // ============================================================== attention kernel
 struct AttnArgs {
   int B, Hq, Hkv, Sq, Sqpad, Skpad, Ck, Ckpad, Cq, G, Wg, Wc;
+  int kstride;  // rows per (batch, KV head) in the tensors the K/V maps address
   int nh_slices, b_sliced, h_sliced;
   int compensate;
   float scale_log2;
@@ -522,7 +523,7 @@ __global__ void __launch_bounds__(160, 2)
     const uint64_t dV = TF32 ? smem_desc(sV, 16384, 512, kLayoutSW128Atom32B)
                              : smem_desc(sV, 16384, 1024, kLayoutSW128);
     const int qrow0 = (b * a.Hq + h) * a.Sqpad + tile * 128;
-    const int krow0 = (b * a.Hkv + hkv) * a.Skpad;
+    const int krow0 = (b * a.Hkv + hkv) * a.kstride;
     const int crow0 = (b * a.Hkv + hkv) * a.Ckpad;
     auto load_kv = [&](const Chunk& c, bool is_v) {
       if (leader) {
@@ -1055,22 +1056,27 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     count_launch();
     if ((rc = check_cuda(cudaGetLastError(), "gather_rows_kernel"))) return rc;
   }
-  // 4. K/V gather + centroids
-  if (s.dtype == BSA_F32) {
-    gather_kv_centroids_kernel<float><<<dim3(L.Ckpad, s.Hkv, s.B), 256, 0, st>>>(
-        static_cast<const float*>(k), static_cast<const float*>(v), static_cast<float*>(L.kp),
-        static_cast<float*>(L.vp), static_cast<float*>(L.kc), static_cast<float*>(L.vc),
-        L.kslot_token, L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
-    count_launch();
-  } else {
-    gather_kv_centroids_kernel<__nv_bfloat16><<<dim3(L.Ckpad, s.Hkv, s.B), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-        static_cast<__nv_bfloat16*>(L.kp), static_cast<__nv_bfloat16*>(L.vp),
-        static_cast<__nv_bfloat16*>(L.kc), static_cast<__nv_bfloat16*>(L.vc), L.kslot_token,
-        L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
-    count_launch();
+  // 4. K/V gather + centroids. One key cluster without compensation (the probe path)
+  //    permutes nothing and needs no centroid: the K/V maps then read the caller's
+  //    tensors directly (key slot = token, rows per head = Sk).
+  const bool kv_identity = Ck == 1 && !compensate && s.Sk % 16 == 0;
+  if (!kv_identity) {
+    if (s.dtype == BSA_F32) {
+      gather_kv_centroids_kernel<float><<<dim3(L.Ckpad, s.Hkv, s.B), 256, 0, st>>>(
+          static_cast<const float*>(k), static_cast<const float*>(v), static_cast<float*>(L.kp),
+          static_cast<float*>(L.vp), static_cast<float*>(L.kc), static_cast<float*>(L.vc),
+          L.kslot_token, L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
+      count_launch();
+    } else {
+      gather_kv_centroids_kernel<__nv_bfloat16><<<dim3(L.Ckpad, s.Hkv, s.B), 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+          static_cast<__nv_bfloat16*>(L.kp), static_cast<__nv_bfloat16*>(L.vp),
+          static_cast<__nv_bfloat16*>(L.kc), static_cast<__nv_bfloat16*>(L.vc), L.kslot_token,
+          L.k_count, L.k_off, s.Sk, L.Skpad, Ck, L.Ckpad, s.D, s.Hkv);
+      count_launch();
+    }
+    if ((rc = check_cuda(cudaGetLastError(), "gather_kv_centroids_kernel"))) return rc;
   }
-  if ((rc = check_cuda(cudaGetLastError(), "gather_kv_centroids_kernel"))) return rc;
 
   // 5. tensor maps + attention
   const CUtensorMapDataType tdt =
@@ -1082,8 +1088,10 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
       s.dtype == BSA_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUtensorMap maps[5];
   if ((rc = make_tmap_2d(&maps[0], L.qp, tdt, es, static_cast<uint64_t>(s.B) * s.Hq * L.Sqpad, s.D, 128, atom)) ||
-      (rc = make_tmap_2d(&maps[1], L.kp, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Skpad, s.D, 128, atom)) ||
-      (rc = make_tmap_2d(&maps[2], L.vp, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Skpad, s.D, 128, atom, vsw)) ||
+      (rc = make_tmap_2d(&maps[1], kv_identity ? k : L.kp, tdt, es,
+                         static_cast<uint64_t>(s.B) * s.Hkv * (kv_identity ? s.Sk : L.Skpad), s.D, 128, atom)) ||
+      (rc = make_tmap_2d(&maps[2], kv_identity ? v : L.vp, tdt, es,
+                         static_cast<uint64_t>(s.B) * s.Hkv * (kv_identity ? s.Sk : L.Skpad), s.D, 128, atom, vsw)) ||
       (rc = make_tmap_2d(&maps[3], L.kc, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Ckpad, s.D, 128, atom)) ||
       (rc = make_tmap_2d(&maps[4], L.vc, tdt, es, static_cast<uint64_t>(s.B) * s.Hkv * L.Ckpad, s.D, 128, atom, vsw)))
     return rc;
@@ -1094,6 +1102,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
   args.Sq = s.Sq;
   args.Sqpad = L.Sqpad;
   args.Skpad = L.Skpad;
+  args.kstride = kv_identity ? s.Sk : L.Skpad;
   args.Ck = Ck;
   args.Ckpad = L.Ckpad;
   args.Cq = Cq;

@@ -207,8 +207,9 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   const bool small = M < D;
   const int n = small ? M : D;
   const int ne = n + (n & 1);
-  float* G = big;             // ne x ne (padding row/col zero)
-  float* V = big + ne * ne;   // ne x ne
+  const int ld = ne + 1;      // padded row stride: column sweeps hit distinct banks
+  float* G = big;             // ne x ne in ld-strided rows (padding row/col zero)
+  float* V = big + ne * ld;   // ne x ne in ld-strided rows
   for (int e = tid; e < ne * ne; e += nt) {
     const int i = e / ne, j = e % ne;
     float acc = 0.f;
@@ -221,30 +222,31 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
         for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * rr[m * D + i], rr[m * D + j], acc);
       }
     }
-    G[e] = acc;
-    V[e] = (i == j) ? 1.f : 0.f;
+    G[i * ld + j] = acc;
+    V[i * ld + j] = (i == j) ? 1.f : 0.f;
   }
   __syncthreads();
-  // 7. cyclic Jacobi sweeps
+  // 7. cyclic Jacobi sweeps, until the off-diagonal mass is below 1e-12 of the total
+  //    (about the float32 resolution of the squared entries)
   for (int sweep = 0; sweep < 20; ++sweep) {
     float off = 0.f, tot = 0.f;
     for (int e = tid; e < ne * ne; e += nt) {
-      const float g = G[e];
+      const float g = G[(e / ne) * ld + e % ne];
       tot += g * g;
       if (e / ne != e % ne) off += g * g;
     }
     off = block_sum(off, red);
     tot = block_sum(tot, red);
-    if (off <= 1e-14f * tot || tot == 0.f) break;
+    if (off <= 1e-12f * tot || tot == 0.f) break;
     for (int r = 0; r < ne - 1; ++r) {
       if (tid < ne / 2) {
         int p, q;
         round_pair(ne, r, tid, p, q);
         float c = 1.f, s = 0.f;
         if (q < n) {
-          const float apq = G[p * ne + q];
+          const float apq = G[p * ld + q];
           if (apq != 0.f) {
-            const float tau = (G[q * ne + q] - G[p * ne + p]) / (2.f * apq);
+            const float tau = (G[q * ld + q] - G[p * ld + p]) / (2.f * apq);
             const float t = (tau >= 0.f ? 1.f : -1.f) / (fabsf(tau) + sqrtf(1.f + tau * tau));
             c = 1.f / sqrtf(1.f + t * t);
             s = t * c;
@@ -260,21 +262,21 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
         const int i = e / ne, j = e % ne;
         const int p = cpq[i][0], q = cpq[i][1];
         const float c = csn[i][0], s = csn[i][1];
-        const float gp = G[p * ne + j], gq = G[q * ne + j];
-        G[p * ne + j] = c * gp - s * gq;
-        G[q * ne + j] = s * gp + c * gq;
+        const float gp = G[p * ld + j], gq = G[q * ld + j];
+        G[p * ld + j] = c * gp - s * gq;
+        G[q * ld + j] = s * gp + c * gq;
       }
       __syncthreads();
       for (int e = tid; e < (ne / 2) * ne; e += nt) {  // columns p, q  <- G J, V J
         const int i = e / ne, j = e % ne;
         const int p = cpq[i][0], q = cpq[i][1];
         const float c = csn[i][0], s = csn[i][1];
-        const float gp = G[j * ne + p], gq = G[j * ne + q];
-        G[j * ne + p] = c * gp - s * gq;
-        G[j * ne + q] = s * gp + c * gq;
-        const float vp = V[j * ne + p], vq = V[j * ne + q];
-        V[j * ne + p] = c * vp - s * vq;
-        V[j * ne + q] = s * vp + c * vq;
+        const float gp = G[j * ld + p], gq = G[j * ld + q];
+        G[j * ld + p] = c * gp - s * gq;
+        G[j * ld + q] = s * gp + c * gq;
+        const float vp = V[j * ld + p], vq = V[j * ld + q];
+        V[j * ld + p] = c * vp - s * vq;
+        V[j * ld + q] = s * vp + c * vq;
       }
       __syncthreads();
     }
@@ -288,8 +290,8 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
       for (int i = 0; i < n; ++i) {
         bool used = false;
         for (int j = 0; j < k; ++j) used |= sel[j] == i;
-        if (!used && G[i * ne + i] > bv) {
-          bv = G[i * ne + i];
+        if (!used && G[i * ld + i] > bv) {
+          bv = G[i * ld + i];
           best = i;
         }
       }
@@ -298,19 +300,19 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   }
   __syncthreads();
   float* vr = a.vr + bh * D * rk;
-  const float lmax = n > 0 && sel[0] >= 0 ? G[sel[0] * ne + sel[0]] : 0.f;
+  const float lmax = n > 0 && sel[0] >= 0 ? G[sel[0] * ld + sel[0]] : 0.f;
   for (int e = tid; e < D * rk; e += nt) {
     const int d = e / rk, k = e % rk;
     const int i = sel[k];
     float val = 0.f;
     if (i >= 0) {
       if (!small) {
-        val = V[d * ne + i];
+        val = V[d * ld + i];
       } else {
-        const float lam_i = G[i * ne + i];
+        const float lam_i = G[i * ld + i];
         if (lam_i > 1e-12f * lmax && lam_i > 0.f) {
           float acc = 0.f;
-          for (int m = 0; m < M; ++m) acc = fmaf(sqrtf(wv[m]) * rr[m * D + d], V[m * ne + i], acc);
+          for (int m = 0; m < M; ++m) acc = fmaf(sqrtf(wv[m]) * rr[m * D + d], V[m * ld + i], acc);
           val = acc / sqrtf(lam_i);
         }
       }
@@ -341,8 +343,28 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   }
 }
 
+// Sum of 16 per-lane values over the warp: a reduce-scatter butterfly (the halves a
+// lane gives away shrink 8, 4, 2, 1), then one exchange across lane pairs. Afterwards
+// lane l holds the warp total of value slot(l), slot(l) = the bits 4..1 of l
+// (i.e. (l >> 1) & 15, read MSB-first: bit 4 -> slot bit 3, ..., bit 1 -> slot bit 0).
+__device__ __forceinline__ float warp_sum16_scatter(float (&y)[16], int lane) {
+#pragma unroll
+  for (int h = 8, o = 16; h >= 1; h >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;  // this lane keeps the upper half
+#pragma unroll
+    for (int k = 0; k < h; ++k) {
+      const float give = up ? y[k] : y[k + h];
+      const float keep = up ? y[k + h] : y[k];
+      y[k] = keep + __shfl_xor_sync(0xffffffffu, give, o);
+    }
+  }
+  return y[0] + __shfl_xor_sync(0xffffffffu, y[0], 1);
+}
+
 // grid (ceil(S / 64), B*H), 256 threads (8 warps); a warp corrects one row at a time:
-// y = x P' + c' (lanes hold D/32 columns each; butterfly sums), x += y V_rᵀ.
+// y = x P' + c' (lane l holds columns l, l+32, ...; the factors sit in shared memory
+// as [k][d] so the 32 lanes read 32 consecutive words), x += y V_rᵀ. Ranks above 16
+// are taken 16 at a time.
 template <int D>
 __global__ void __launch_bounds__(256) repair_apply_kernel(float* __restrict__ out, int S, int rank,
                                                            const float* __restrict__ pp,
@@ -351,51 +373,49 @@ __global__ void __launch_bounds__(256) repair_apply_kernel(float* __restrict__ o
   constexpr int EPL = D / 32;
   extern __shared__ float sm_apply[];
   const int64_t bh = blockIdx.y;
-  float* sP = sm_apply;                // D x rank
-  float* sV = sm_apply + D * rank;     // D x rank
-  float* sc = sV + D * rank;     // rank
-  for (int e = threadIdx.x; e < D * rank; e += blockDim.x) {
-    sP[e] = pp[bh * D * rank + e];
-    sV[e] = vr[bh * D * rank + e];
+  const int nk = (rank + 15) & ~15;    // rank rounded up to 16: zero factors past it
+  float* sP = sm_apply;                // [nk][D]
+  float* sV = sm_apply + nk * D;       // [nk][D]
+  float* sc = sV + nk * D;             // [nk]
+  for (int e = threadIdx.x; e < nk * D; e += blockDim.x) {
+    const int k = e / D, d = e % D;
+    const bool in = k < rank;
+    sP[e] = in ? pp[(bh * D + d) * rank + k] : 0.f;
+    sV[e] = in ? vr[(bh * D + d) * rank + k] : 0.f;
   }
-  for (int e = threadIdx.x; e < rank; e += blockDim.x) sc[e] = cc[bh * rank + e];
+  for (int e = threadIdx.x; e < nk; e += blockDim.x) sc[e] = e < rank ? cc[bh * rank + e] : 0.f;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slot = (lane >> 1) & 15;   // the value this lane holds after warp_sum16_scatter
   const int r0 = blockIdx.x * 64;
   for (int r = r0 + warp; r < min(S, r0 + 64); r += 8) {
-    float* row = out + (bh * S + r) * D + lane * EPL;
+    float* row = out + (bh * S + r) * D + lane;
     float x[EPL], acc[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
-      x[e] = row[e];
+      x[e] = row[32 * e];
       acc[e] = x[e];
     }
-    for (int k0 = 0; k0 < rank; k0 += 16) {
+    for (int k0 = 0; k0 < nk; k0 += 16) {
       float y[16];
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         float t = 0.f;
-        if (k0 + k < rank) {
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) t = fmaf(x[e], sP[(lane * EPL + e) * rank + k0 + k], t);
-        }
+        for (int e = 0; e < EPL; ++e) t = fmaf(x[e], sP[(k0 + k) * D + lane + 32 * e], t);
         y[k] = t;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int k = 0; k < 16; ++k) y[k] += __shfl_xor_sync(0xffffffffu, y[k], o);
+      const float mine = warp_sum16_scatter(y, lane) + sc[k0 + slot];
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
-        if (k0 + k < rank) {
-          const float yk = y[k] + sc[k0 + k];
+        // the lanes 2k' .. holding slot k: lane l has slot (l >> 1) & 15, so lane 2k has k
+        const float yk = __shfl_sync(0xffffffffu, mine, 2 * k);
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) acc[e] = fmaf(yk, sV[(lane * EPL + e) * rank + k0 + k], acc[e]);
-        }
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(yk, sV[(k0 + k) * D + lane + 32 * e], acc[e]);
       }
     }
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) row[e] = acc[e];
+    for (int e = 0; e < EPL; ++e) row[32 * e] = acc[e];
   }
 }
 
@@ -453,14 +473,15 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
   const int n = M < D ? M : D;
   const int ne = n + (n & 1);
   const size_t big = std::max(static_cast<size_t>(D + 1) * (D + 1) + static_cast<size_t>(D + 1) * D,
-                              2 * static_cast<size_t>(ne) * ne) * sizeof(float);
+                              2 * static_cast<size_t>(ne) * (ne + 1)) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(repair_fit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(big));
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(repair_fit)");
   repair_fit_kernel<<<BH, kFitThreads, big, st>>>(fa);
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "repair_fit_kernel"))) return rc;
-  const int smem = (2 * D * rank + rank) * static_cast<int>(sizeof(float));
+  const int nk = (rank + 15) & ~15;
+  const int smem = (2 * D * nk + nk) * static_cast<int>(sizeof(float));
   auto ap = D == 64 ? repair_apply_kernel<64> : repair_apply_kernel<128>;
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(ap, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

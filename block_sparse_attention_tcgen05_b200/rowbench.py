@@ -1,0 +1,209 @@
+"""Per-step measurement of the hot path: each step's kernels timed at its workload
+sizes, with its algorithmic work and roofline fraction.
+
+    python -m block_sparse_attention_tcgen05_b200.rowbench [--out FILE] [--calls N]
+
+Steps and sizes follow the method's pipeline: pooled drift/gate of the per-head mask
+cache and the anti-diagonal block scoring + top-p selection at the video shape
+(H=40, S=32760 padded to 32768, D=128, block 128, stride 16, per-head tau); the
+labels -> permutation -> gather -> centroid -> bitset stages and the fused
+compensated attention at the video-tile workload (245 clusters, nearest 22 % of tile
+pairs); probe selection, probe dense attention and the probe-fitted residual repair
+at the grouped-query shape (H=24 query heads over 8 KV heads, S=32768, M=64).
+
+Timing: CUDA events on the launching stream, 5 warm-up calls, median of N calls
+(default 20), L2 flushed (a 256 MB write) before every timed call. Peaks come from
+MEASURED_PEAKS.json at the repository root (burst figures: each call is timed alone).
+All inputs are synthetic and seeded; nothing here computes reference values.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import time
+
+import torch
+
+from . import ops
+from . import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GRID, TILE, D = (21, 30, 52), (3, 6, 8), 128
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class Timer:
+    """Median device time of a callable; the L2 flush before each call is not timed."""
+
+    def __init__(self, dev, calls, warmup=5):
+        self.dev, self.calls, self.warmup = dev, calls, warmup
+        self.flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self, fn):
+        for _ in range(self.warmup):
+            fn()
+        torch.cuda.synchronize(self.dev)
+        ts = []
+        for _ in range(self.calls):
+            self.flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize(self.dev)
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+
+def row(step, what, ms, work, unit, bound, peak):
+    """One result: work per call in bytes (HBM rows) or FLOP (tensor rows)."""
+    if bound == "hbm":
+        achieved = work / (ms * 1e-3) / 1e9
+        unit_a = "GB/s"
+    elif bound == "tensor":
+        achieved = work / (ms * 1e-3) / 1e12
+        unit_a = "TFLOP/s"
+    else:
+        achieved, unit_a = None, None
+    return {"step": step, "what": what, "ms": ms, "work": work, "work_unit": unit, "bound": bound,
+            "achieved": achieved, "unit": unit_a, "peak": peak if achieved is not None else None,
+            "frac": achieved / peak if achieved is not None else None}
+
+
+def video_inputs(dev, H):
+    q, k, v = wl.positional_qkv_device(1, H, H, GRID, D, ell=(3.0, 6.0, 8.0), amp=2.0, seed=3,
+                                       device=dev)
+    return q, k, v
+
+
+def bench_cache_and_scoring(timer, dev, hbm, tc, out):
+    H, S, Sp = 40, 32760, 32768
+    q, k, _ = video_inputs(dev, H)
+    # a1: pooled means, drift and gate over Q and K of every head (one read of each)
+    cache = ops.MaskCache(1, H, Sp // 128, Sp // 128, D, delta=8.0)
+    cache.should_refresh(q, k, sync=False)  # first call: anchors
+    ms = timer(lambda: cache.should_refresh(q, k, sync=False))
+    out.append(row("a1", "mask cache: pooled means, drift, gate (H=40, S=32760)", ms,
+                   2 * q.numel() * q.element_size(), "B", "hbm", hbm))
+    # a2: anti-diagonal scoring on Q, K zero-padded to a multiple of the block
+    qp = torch.zeros((1, H, Sp, D), dtype=q.dtype, device=dev)
+    kp = torch.zeros_like(qp)
+    qp[:, :, :S] = q
+    kp[:, :, :S] = k
+    del q, k
+    stride = 16
+    ms = timer(lambda: ops.antidiagonal_block_scores(qp, kp, block=128, stride=stride))
+    flop = 2.0 * Sp * Sp * D / stride * H
+    out.append(row("a2", "anti-diagonal block scores (H=40, S=32768, D=128, stride 16)", ms, flop,
+                   "FLOP", "tensor", tc))
+    r = out[-1]
+    r["hbm_gbs"] = 2 * qp.numel() * qp.element_size() / (ms * 1e-3) / 1e9
+    # a3: top-p with tau per head from {0.85, 0.90, 0.95}
+    scores = ops.antidiagonal_block_scores(qp, kp, block=128, stride=stride)
+    tau = torch.tensor([(0.85, 0.90, 0.95)[h % 3] for h in range(H)], dtype=torch.float32)
+    ms = timer(lambda: ops.top_p_block_mask(scores, tau))
+    out.append(row("a3", "top-p block mask (1x40x256x256 scores)", ms, None, None, "latency", None))
+    del qp, kp, scores
+
+
+def bench_attention(timer, dev, hbm, tc, out):
+    import ctypes
+
+    from . import _lib
+    H, S = 40, 32760
+    q, k, v = video_inputs(dev, H)
+    labels, C = ops.tile_labels(*GRID, TILE, device=dev)
+    mask = torch.tensor(wl.nearest_pair_mask(wl.tile_centroids(GRID, TILE), 0.22),
+                        dtype=torch.uint8, device=dev)
+    ws = torch.empty(ops.attention_workspace_bytes(q, k, C, C), dtype=torch.uint8, device=dev)
+    o = torch.empty((1, H, S, D), dtype=torch.float32, device=dev)
+    cnt = torch.bincount(labels.long(), minlength=C).double()
+    pairs = float(cnt @ mask.double() @ cnt) * H
+
+    def call():
+        ops.centroid_compensated_attention(q, k, v, labels, labels, mask, Cq=C, Ck=C, out=o,
+                                           workspace=ws)
+    _lib.call("bsa_profile_enable", timer.calls + timer.warmup)
+    ms = timer(call)
+    kms, kn = ctypes.c_float(0.0), ctypes.c_int(0)
+    _lib.call("bsa_profile_read", 0, ctypes.byref(kms), ctypes.byref(kn))
+    _lib.call("bsa_profile_enable", 0)
+    kernel_ms = kms.value / max(1, kn.value)
+    prep_ms = max(ms - kernel_ms, 1e-6)
+    qkv_bytes = 3 * q.numel() * q.element_size()
+    out.append(row("a4-a7", "labels -> permutation, cluster-major gathers of Q/K/V, centroids, "
+                   "mask bitsets (call minus attention kernel)", prep_ms, 2 * qkv_bytes, "B", "hbm",
+                   hbm))
+    out.append(row("a8", f"fused compensated attention kernel ({pairs:.3e} executed pairs x 4D)",
+                   kernel_ms, pairs * 4 * D, "FLOP", "tensor", tc))
+    out.append(row("a4-a8", "whole attention call", ms, pairs * 4 * D, "FLOP", "tensor", tc))
+
+
+def bench_probe_and_repair(timer, dev, hbm, tc, out):
+    Hq, Hkv, S, M = 24, 8, 32768, 64
+    g = torch.Generator(device=dev).manual_seed(4)
+    q = torch.randn((1, Hq, S, D), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((1, Hkv, S, D), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((1, Hkv, S, D), generator=g, device=dev).to(torch.bfloat16)
+    labels = (torch.arange(S, device=dev) // 128).to(torch.int32)
+    C = S // 128
+    ms = timer(lambda: ops.select_probe_rows(labels, C, M, q=q))
+    out.append(row("a9", "probe selection, nearest-to-centroid members (H=24, 256 clusters, M=64)",
+                   ms, None, None, "latency", None))
+    idx, w = ops.select_probe_rows(labels, C, M, q=q)
+    ws = torch.empty(ops._lib.load().bsa_probe_attention_workspace_bytes(ops.make_shape(q, k), M),
+                     dtype=torch.uint8, device=dev)
+    ms = timer(lambda: ops.probe_dense_attention(q, k, v, idx, workspace=ws))
+    out.append(row("a10", "probe dense attention (24 heads x 64 rows over 32768 keys)", ms,
+                   4.0 * D * M * S * Hq, "FLOP", "tensor", tc))
+    o_probe = ops.probe_dense_attention(q, k, v, idx, workspace=ws)
+    del q, k, v
+    o = torch.randn((1, Hq, S, D), generator=g, device=dev) * 0.1
+    rws = torch.empty(ops._lib.load().bsa_repair_workspace_bytes(1, Hq, S, D, M),
+                      dtype=torch.uint8, device=dev)
+    ms = timer(lambda: ops.probe_residual_correction(o, o_probe, idx, w, workspace=rws))
+    out.append(row("a11-a14", "probe-fitted residual repair: column stats, normal equations, "
+                   "Cholesky, top-16 subspace, rank-16 apply (out 1x24x32768x128 fp32)", ms,
+                   3 * o.numel() * o.element_size(), "B", "hbm", hbm))
+
+
+def main():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--calls", type=int, default=20)
+    p.add_argument("--out", default=None, help="also write the JSON lines to this file")
+    args = p.parse_args()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm, tc, src = peaks()
+    timer = Timer(dev, args.calls)
+    out = []
+    t0 = time.time()
+    bench_cache_and_scoring(timer, dev, hbm, tc, out)
+    torch.cuda.empty_cache()
+    bench_attention(timer, dev, hbm, tc, out)
+    torch.cuda.empty_cache()
+    bench_probe_and_repair(timer, dev, hbm, tc, out)
+    st, _ = ops.device_status(dev)
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    lines = [json.dumps(dict(r, peak_source=src)) for r in out]
+    print("\n".join(lines))
+    print(f"# {len(out)} rows in {time.time() - t0:.1f} s; peaks: HBM {hbm} GB/s, bf16 {tc} TFLOP/s "
+          f"({src}, burst)")
+    if args.out:
+        with open(args.out, "w") as f:
+            f.write("\n".join(lines) + "\n")
+
+
+if __name__ == "__main__":
+    main()
