@@ -24,7 +24,7 @@
 namespace bsa {
 
 constexpr int kStatSplit = 32;
-constexpr int kFitThreads = 1024;
+constexpr int kFitThreads = 512;
 
 // grid (kStatSplit, B*H), 256 threads: partial column sums of (x - x_0) and its square,
 // x_0 = the first row, over a slice of the rows.
@@ -67,9 +67,9 @@ struct FitArgs {
   float lam;
   const float* psum;
   const float* psq;
-  float* zt;   // [BH][M][D+1]
-  float* rr;   // [BH][M][D]
-  float* bc;   // [BH][D+1][D]
+  float* zt;   // [BH][M][D+2]   (used when they do not fit in shared memory)
+  float* rr;   // [BH][M][D+1]
+  float* rv;   // [BH][M][rank]
   float* vr;   // [BH][D][rank]
   float* pp;   // [BH][D][rank]
   float* cc;   // [BH][rank]
@@ -108,23 +108,71 @@ __device__ __forceinline__ void round_pair(int n, int r, int i, int& p, int& q) 
   }
 }
 
-// One CTA (1024 threads) per (b, h): statistics, normal equations, Cholesky solve,
-// residual subspace, and the folded rank-r factors P', c' for the apply pass.
+// Shared-memory plan of the fit, in floats: the standardised probe rows Zt (M x ldz)
+// and residuals R (M x ldr) and R V_r (M x rk) when they fit (else they stay in the
+// workspace), a region W used first by the eigen step (G and V, ne x (ne + 1) each)
+// and then by the solve (A: n1 x n1, right-hand sides n1 x rk), V_r (D x rk) and the
+// Cholesky pivots. Odd row strides keep column-wise sweeps on distinct banks.
+struct FitPlan {
+  int n1, n, ne, ld, ldz, ldr, rk;
+  bool local_zr;                   // Zt, R, R V_r in shared memory
+  size_t zt, rr, rv, w, vr, piv;   // offsets (floats) into the dynamic shared memory
+  size_t floats;
+};
+__host__ __device__ inline FitPlan fit_plan(int D, int M, int rk) {
+  FitPlan p{};
+  p.n1 = D + 1;
+  p.n = M < D ? M : D;
+  p.ne = p.n + (p.n & 1);
+  p.ld = p.ne + 1;
+  p.ldz = D + 2;
+  p.ldr = D + 1;
+  p.rk = rk;
+  const size_t wa = static_cast<size_t>(2) * p.ne * p.ld;
+  const size_t wb = static_cast<size_t>(p.n1) * p.n1 + static_cast<size_t>(p.n1) * rk;
+  const size_t wsz = wa > wb ? wa : wb;
+  const size_t common = wsz + static_cast<size_t>(D) * rk + p.n1;
+  const size_t zr = static_cast<size_t>(M) * (p.ldz + p.ldr + rk);
+  p.local_zr = (common + zr) * sizeof(float) <= 200 * 1024;
+  size_t o = 0;
+  if (p.local_zr) {
+    p.zt = o; o += static_cast<size_t>(M) * p.ldz;
+    p.rr = o; o += static_cast<size_t>(M) * p.ldr;
+    p.rv = o; o += static_cast<size_t>(M) * rk;
+  }
+  p.w = o; o += wsz;
+  p.vr = o; o += static_cast<size_t>(D) * rk;
+  p.piv = o; o += p.n1;
+  p.floats = o;
+  return p;
+}
+
+// One CTA (512 threads) per (b, h): statistics, the residual subspace V_r, then the
+// ridge solve for Bc V_r only (Bc itself is never needed: the apply uses Bc V_r), and
+// the folded rank-r factors P', c' for the apply pass.
 __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArgs a) {
-  extern __shared__ float big[];
+  extern __shared__ float sm_fit[];
   __shared__ float mu[128], isg[128], red[32];
   __shared__ float wv[1024];
   __shared__ int sel[128];
   __shared__ float csn[64][2];
   __shared__ int cpq[64][2];
+  __shared__ uint8_t pairs[127][64][2];  // circle-method pair table: round, slot -> (p, q)
   const int tid = threadIdx.x, nt = blockDim.x;
   const int64_t bh = blockIdx.x;
-  const int S = a.S, D = a.D, M = a.M, n1 = D + 1;
+  const int S = a.S, D = a.D, M = a.M, rk = a.rank;
+  const FitPlan pl = fit_plan(D, M, rk);
+  const int n1 = pl.n1, n = pl.n, ne = pl.ne, ld = pl.ld, ldz = pl.ldz, ldr = pl.ldr;
+  const bool small = M < D;
   const float* X = a.out + bh * S * D;
   const int32_t* idx = a.per_head ? a.probe_idx + bh * M : a.probe_idx;
   const float* w = a.per_head ? a.weights + bh * M : a.weights;
-  float* zt = a.zt + bh * M * n1;
-  float* rr = a.rr + bh * M * D;
+  float* zt = pl.local_zr ? sm_fit + pl.zt : a.zt + bh * M * ldz;
+  float* rr = pl.local_zr ? sm_fit + pl.rr : a.rr + bh * M * ldr;
+  float* rv = pl.local_zr ? sm_fit + pl.rv : a.rv + bh * M * rk;
+  float* W = sm_fit + pl.w;
+  float* vrs = sm_fit + pl.vr;
+  float* piv = sm_fit + pl.piv;
 
   // 1. column statistics
   if (tid < D) {
@@ -139,95 +187,47 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
     isg[tid] = 1.f / sqrtf(var + 1e-6f);
   }
   for (int m = tid; m < M; m += nt) wv[m] = w[m];
+  for (int k = tid; k < 128; k += nt) sel[k] = -1;
   __syncthreads();
-  // 2. standardised probe rows and residuals
+  // 2. standardised probe rows Zt = [(x - mu) / sigma, 1] and residuals R = o_probe - x
   for (int e = tid; e < M * D; e += nt) {
     const int m = e / D, d = e % D;
     int row = idx[m];
     row = row < 0 ? 0 : (row >= S ? S - 1 : row);
     const float x = X[static_cast<int64_t>(row) * D + d];
-    zt[m * n1 + d] = (x - mu[d]) * isg[d];
-    rr[m * D + d] = a.o_probe[(bh * M + m) * D + d] - x;
+    zt[m * ldz + d] = (x - mu[d]) * isg[d];
+    rr[m * ldr + d] = a.o_probe[(bh * M + m) * D + d] - x;
   }
-  for (int m = tid; m < M; m += nt) zt[m * n1 + D] = 1.f;
+  for (int m = tid; m < M; m += nt) zt[m * ldz + D] = 1.f;
   __syncthreads();
-  // 3. normal equations: A = Ztᵀ W Zt + lam·I' (intercept unpenalised), Y = Ztᵀ W R
-  float* A = big;            // n1 x n1
-  float* Y = big + n1 * n1;  // n1 x D
-  for (int e = tid; e < n1 * n1; e += nt) {
-    const int i = e / n1, j = e % n1;
-    if (j > i) continue;
-    float acc = 0.f;
-    for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * zt[m * n1 + i], zt[m * n1 + j], acc);
-    if (i == j && i < D) acc += a.lam;
-    A[i * n1 + j] = acc;
-    A[j * n1 + i] = acc;
-  }
-  for (int e = tid; e < n1 * D; e += nt) {
-    const int i = e / D, c = e % D;
-    float acc = 0.f;
-    for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * zt[m * n1 + i], rr[m * D + c], acc);
-    Y[i * D + c] = acc;
-  }
-  __syncthreads();
-  // 4. Cholesky A = L Lᵀ (lower triangle, in place)
-  for (int k = 0; k < n1; ++k) {
-    if (tid == 0) A[k * n1 + k] = sqrtf(fmaxf(A[k * n1 + k], 1e-30f));
-    __syncthreads();
-    const float piv = A[k * n1 + k];
-    for (int i = k + 1 + tid; i < n1; i += nt) A[i * n1 + k] /= piv;
-    __syncthreads();
-    const int rem = n1 - k - 1;
-    for (int e = tid; e < rem * rem; e += nt) {
-      const int i = k + 1 + e / rem, j = k + 1 + e % rem;
-      if (j <= i) A[i * n1 + j] -= A[i * n1 + k] * A[j * n1 + k];
-    }
-    __syncthreads();
-  }
-  // 5. solve L Lᵀ Bc = Y, one right-hand side column per thread
-  if (tid < D) {
-    const int c = tid;
-    for (int i = 0; i < n1; ++i) {
-      float acc = Y[i * D + c];
-      for (int j = 0; j < i; ++j) acc -= A[i * n1 + j] * Y[j * D + c];
-      Y[i * D + c] = acc / A[i * n1 + i];
-    }
-    for (int i = n1 - 1; i >= 0; --i) {
-      float acc = Y[i * D + c];
-      for (int j = i + 1; j < n1; ++j) acc -= A[j * n1 + i] * Y[j * D + c];
-      Y[i * D + c] = acc / A[i * n1 + i];
-    }
-  }
-  __syncthreads();
-  float* bc = a.bc + bh * n1 * D;
-  for (int e = tid; e < n1 * D; e += nt) bc[e] = Y[e];
-  __syncthreads();
-
-  // 6. Gram matrix of the weighted residuals: n x n with n = min(M, D)
-  const bool small = M < D;
-  const int n = small ? M : D;
-  const int ne = n + (n & 1);
-  const int ld = ne + 1;      // padded row stride: column sweeps hit distinct banks
-  float* G = big;             // ne x ne in ld-strided rows (padding row/col zero)
-  float* V = big + ne * ld;   // ne x ne in ld-strided rows
+  // 3. Gram matrix of the weighted residuals, n x n with n = min(M, D):
+  //    W½ R Rᵀ W½ (M < D) or Rᵀ W R; padding row/column zero
+  float* G = W;
+  float* V = W + ne * ld;
   for (int e = tid; e < ne * ne; e += nt) {
     const int i = e / ne, j = e % ne;
     float acc = 0.f;
     if (i < n && j < n) {
       if (small) {
-        const float s = sqrtf(wv[i] * wv[j]);
-        for (int d = 0; d < D; ++d) acc = fmaf(rr[i * D + d], rr[j * D + d], acc);
-        acc *= s;
+        for (int d = 0; d < D; ++d) acc = fmaf(rr[i * ldr + d], rr[j * ldr + d], acc);
+        acc *= sqrtf(wv[i] * wv[j]);
       } else {
-        for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * rr[m * D + i], rr[m * D + j], acc);
+        for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * rr[m * ldr + i], rr[m * ldr + j], acc);
       }
     }
     G[i * ld + j] = acc;
     V[i * ld + j] = (i == j) ? 1.f : 0.f;
   }
   __syncthreads();
-  // 7. cyclic Jacobi sweeps, until the off-diagonal mass is below 1e-12 of the total
-  //    (about the float32 resolution of the squared entries)
+  // 4. cyclic Jacobi sweeps (circle-method pair order), until the off-diagonal mass is
+  //    below 1e-12 of the total (about the float32 resolution of the squared entries)
+  for (int e = tid; e < (ne - 1) * (ne / 2); e += nt) {
+    int p, q;
+    round_pair(ne, e / (ne / 2), e % (ne / 2), p, q);
+    pairs[e / (ne / 2)][e % (ne / 2)][0] = static_cast<uint8_t>(p);
+    pairs[e / (ne / 2)][e % (ne / 2)][1] = static_cast<uint8_t>(q);
+  }
+  __syncthreads();
   for (int sweep = 0; sweep < 20; ++sweep) {
     float off = 0.f, tot = 0.f;
     for (int e = tid; e < ne * ne; e += nt) {
@@ -240,15 +240,14 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
     if (off <= 1e-12f * tot || tot == 0.f) break;
     for (int r = 0; r < ne - 1; ++r) {
       if (tid < ne / 2) {
-        int p, q;
-        round_pair(ne, r, tid, p, q);
+        const int p = pairs[r][tid][0], q = pairs[r][tid][1];
         float c = 1.f, s = 0.f;
         if (q < n) {
           const float apq = G[p * ld + q];
           if (apq != 0.f) {
             const float tau = (G[q * ld + q] - G[p * ld + p]) / (2.f * apq);
-            const float t = (tau >= 0.f ? 1.f : -1.f) / (fabsf(tau) + sqrtf(1.f + tau * tau));
-            c = 1.f / sqrtf(1.f + t * t);
+            const float t = copysignf(1.f, tau) / (fabsf(tau) + sqrtf(fmaf(tau, tau, 1.f)));
+            c = rsqrtf(fmaf(t, t, 1.f));
             s = t * c;
           }
         }
@@ -258,49 +257,50 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
         cpq[tid][1] = q;
       }
       __syncthreads();
-      for (int e = tid; e < (ne / 2) * ne; e += nt) {  // rows p, q  <- Jᵀ G
-        const int i = e / ne, j = e % ne;
-        const int p = cpq[i][0], q = cpq[i][1];
-        const float c = csn[i][0], s = csn[i][1];
-        const float gp = G[p * ld + j], gq = G[q * ld + j];
-        G[p * ld + j] = c * gp - s * gq;
-        G[q * ld + j] = s * gp + c * gq;
+      // G <- Jᵀ G J in one pass: the 2x2 block of rows (p_a, q_a) and columns
+      // (p_b, q_b) becomes J_aᵀ B J_b, J = [[c, s], [-s, c]]; the blocks partition G.
+      // V <- V J on the columns of every pair.
+      const int half = ne / 2;
+      for (int e = tid; e < half * half; e += nt) {
+        const int ia = e / half, ib = e % half;
+        const int pa = cpq[ia][0], qa = cpq[ia][1], pb = cpq[ib][0], qb = cpq[ib][1];
+        const float ca = csn[ia][0], sa = csn[ia][1], cb = csn[ib][0], sb = csn[ib][1];
+        const float b00 = G[pa * ld + pb], b01 = G[pa * ld + qb];
+        const float b10 = G[qa * ld + pb], b11 = G[qa * ld + qb];
+        const float t00 = ca * b00 - sa * b10, t01 = ca * b01 - sa * b11;  // J_aᵀ B
+        const float t10 = sa * b00 + ca * b10, t11 = sa * b01 + ca * b11;
+        G[pa * ld + pb] = cb * t00 - sb * t01;                              // (J_aᵀ B) J_b
+        G[pa * ld + qb] = sb * t00 + cb * t01;
+        G[qa * ld + pb] = cb * t10 - sb * t11;
+        G[qa * ld + qb] = sb * t10 + cb * t11;
       }
-      __syncthreads();
-      for (int e = tid; e < (ne / 2) * ne; e += nt) {  // columns p, q  <- G J, V J
-        const int i = e / ne, j = e % ne;
-        const int p = cpq[i][0], q = cpq[i][1];
-        const float c = csn[i][0], s = csn[i][1];
-        const float gp = G[j * ld + p], gq = G[j * ld + q];
-        G[j * ld + p] = c * gp - s * gq;
-        G[j * ld + q] = s * gp + c * gq;
-        const float vp = V[j * ld + p], vq = V[j * ld + q];
-        V[j * ld + p] = c * vp - s * vq;
-        V[j * ld + q] = s * vp + c * vq;
+      for (int e = tid; e < ne * half; e += nt) {
+        const int j = e / half, ib = e % half;
+        const int pb = cpq[ib][0], qb = cpq[ib][1];
+        const float cb = csn[ib][0], sb = csn[ib][1];
+        const float vp = V[j * ld + pb], vq = V[j * ld + qb];
+        V[j * ld + pb] = cb * vp - sb * vq;
+        V[j * ld + qb] = sb * vp + cb * vq;
       }
       __syncthreads();
     }
   }
-  // 8. the `rank` largest eigenvalues
-  const int rk = a.rank;
-  if (tid == 0) {
-    for (int k = 0; k < rk; ++k) {
-      int best = -1;
-      float bv = -INFINITY;
-      for (int i = 0; i < n; ++i) {
-        bool used = false;
-        for (int j = 0; j < k; ++j) used |= sel[j] == i;
-        if (!used && G[i * ld + i] > bv) {
-          bv = G[i * ld + i];
-          best = i;
-        }
-      }
-      sel[k] = best;  // -1 when rank exceeds n: that direction is left out
+  // 5. the `rk` largest eigenvalues: eigenvalue i takes slot #{j : l_j > l_i, or equal
+  //    with j < i}; slots past n stay -1 (those directions are left out)
+  for (int i = tid; i < n; i += nt) {
+    const float li = G[i * ld + i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const float lj = G[j * ld + j];
+      rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
     }
+    if (rank < rk) sel[rank] = i;
   }
   __syncthreads();
-  float* vr = a.vr + bh * D * rk;
+  // 6. V_r (D x rk): eigenvectors of Rᵀ W R, directly (M >= D) or as
+  //    (W½ R)ᵀ u / sqrt(l) from those of W½ R Rᵀ W½ (M < D)
   const float lmax = n > 0 && sel[0] >= 0 ? G[sel[0] * ld + sel[0]] : 0.f;
+  float* vr = a.vr + bh * D * rk;
   for (int e = tid; e < D * rk; e += nt) {
     const int d = e / rk, k = e % rk;
     const int i = sel[k];
@@ -312,34 +312,88 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
         const float lam_i = G[i * ld + i];
         if (lam_i > 1e-12f * lmax && lam_i > 0.f) {
           float acc = 0.f;
-          for (int m = 0; m < M; ++m) acc = fmaf(sqrtf(wv[m]) * rr[m * D + d], V[m * ld + i], acc);
+          for (int m = 0; m < M; ++m) acc = fmaf(sqrtf(wv[m]) * rr[m * ldr + d], V[m * ld + i], acc);
           val = acc / sqrtf(lam_i);
         }
       }
     }
-    vr[d * rk + k] = val;
+    vrs[e] = val;
+    vr[e] = val;
   }
   __syncthreads();
-  // 9. folded factors: P' = diag(1/sigma) Bc[:D] V_r, c' = (Bc[D] - Σ mu/sigma Bc) V_r
-  float* c0 = big;  // D (reuses the Gram region, no longer needed)
-  __syncthreads();
-  if (tid < D) {
-    float acc = bc[D * D + tid];
-    for (int i = 0; i < D; ++i) acc -= mu[i] * isg[i] * bc[i * D + tid];
-    c0[tid] = acc;
+  // 7. R V_r (M x rk)
+  for (int e = tid; e < M * rk; e += nt) {
+    const int m = e / rk, k = e % rk;
+    float acc = 0.f;
+    for (int d = 0; d < D; ++d) acc = fmaf(rr[m * ldr + d], vrs[d * rk + k], acc);
+    rv[e] = acc;
   }
   __syncthreads();
+  // 8. normal equations, projected: A = Ztᵀ W Zt + lam·I' (intercept unpenalised) and
+  //    B = Ztᵀ W (R V_r), so that A⁻¹ B = Bc V_r
+  float* A = W;              // n1 x n1 (overwrites G, V: no longer needed)
+  float* Bm = W + n1 * n1;   // n1 x rk
+  for (int e = tid; e < n1 * n1; e += nt) {
+    const int i = e / n1, j = e % n1;
+    if (j > i) continue;
+    float acc = 0.f;
+    for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * zt[m * ldz + i], zt[m * ldz + j], acc);
+    if (i == j && i < D) acc += a.lam;
+    A[i * n1 + j] = acc;
+    A[j * n1 + i] = acc;
+  }
+  for (int e = tid; e < n1 * rk; e += nt) {
+    const int i = e / rk, k = e % rk;
+    float acc = 0.f;
+    for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * zt[m * ldz + i], rv[m * rk + k], acc);
+    Bm[e] = acc;
+  }
+  __syncthreads();
+  // 9. Cholesky without the column scaling: after step k the lower triangle holds
+  //    A[i][k] = L[i][k]·s_k with s_k = L[k][k] = sqrt(A[k][k]); one barrier per step
+  const int lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
+  for (int k = 0; k < n1; ++k) {
+    const float rdk = 1.f / fmaxf(A[k * n1 + k], 1e-30f);
+    for (int i = k + 1 + wid; i < n1; i += nw) {  // warps along rows, lanes along columns
+      const float aik = A[i * n1 + k] * rdk;
+      for (int j = k + 1 + lane; j <= i; j += 32) A[i * n1 + j] -= aik * A[j * n1 + k];
+    }
+    __syncthreads();
+  }
+  float* rpiv = piv;  // 1 / s_k
+  for (int k = tid; k < n1; k += nt) rpiv[k] = 1.f / sqrtf(fmaxf(A[k * n1 + k], 1e-30f));
+  __syncthreads();
+  // 10. solve L Lᵀ X = B in place, right-looking, one barrier per step:
+  //     forward  b_i -= (A[i][k] / s_k) (b_k / s_k), i > k;  then y_k = b_k / s_k
+  for (int k = 0; k < n1 - 1; ++k) {
+    const float r2 = rpiv[k] * rpiv[k];
+    for (int e = tid; e < (n1 - 1 - k) * rk; e += nt) {
+      const int i = k + 1 + e / rk, c = e % rk;
+      Bm[i * rk + c] -= A[i * n1 + k] * Bm[k * rk + c] * r2;
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < n1 * rk; e += nt) Bm[e] *= rpiv[e / rk];
+  __syncthreads();
+  //     backward y_i -= (A[k][i] / s_i) (y_k / s_k), i < k;  then x_k = y_k / s_k
+  for (int k = n1 - 1; k > 0; --k) {
+    const float rk_ = rpiv[k];
+    for (int e = tid; e < k * rk; e += nt) {
+      const int i = e / rk, c = e % rk;
+      Bm[i * rk + c] -= A[k * n1 + i] * rpiv[i] * Bm[k * rk + c] * rk_;
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < n1 * rk; e += nt) Bm[e] *= rpiv[e / rk];
+  __syncthreads();
+  // 11. folded factors from X = Bc V_r: P' = diag(1/sigma) X[:D],
+  //     c' = X[D] - Σ_i (mu_i / sigma_i) X[i]
   float* pp = a.pp + bh * D * rk;
-  for (int e = tid; e < D * rk; e += nt) {
-    const int d = e / rk, k = e % rk;
-    float acc = 0.f;
-    for (int c = 0; c < D; ++c) acc = fmaf(bc[d * D + c], vr[c * rk + k], acc);
-    pp[d * rk + k] = acc * isg[d];
-  }
-  if (tid < rk) {
-    float acc = 0.f;
-    for (int c = 0; c < D; ++c) acc = fmaf(c0[c], vr[c * rk + tid], acc);
-    a.cc[bh * rk + tid] = acc;
+  for (int e = tid; e < D * rk; e += nt) pp[e] = Bm[e] * isg[e / rk];
+  for (int k = tid; k < rk; k += nt) {
+    float acc = Bm[D * rk + k];
+    for (int i = 0; i < D; ++i) acc -= mu[i] * isg[i] * Bm[i * rk + k];
+    a.cc[bh * rk + k] = acc;
   }
 }
 
@@ -419,9 +473,70 @@ __global__ void __launch_bounds__(256) repair_apply_kernel(float* __restrict__ o
   }
 }
 
+// rank <= 16: one row per thread. The thread accumulates y = x P' + c' over its row
+// (each factor row d is one broadcast read of 16 floats, all lanes the same address),
+// then rereads the row (from L1/L2) and writes x + y V_rᵀ. No cross-lane sums; HBM
+// traffic is one read and one write of out. grid (ceil(S / 256), B*H), 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256) repair_apply16_kernel(float* __restrict__ out, int S, int rank,
+                                                             const float* __restrict__ pp,
+                                                             const float* __restrict__ cc,
+                                                             const float* __restrict__ vr) {
+  __shared__ float4 sP[D][4], sV[D][4];  // factor rows d, ranks 0..15 (zero past `rank`)
+  __shared__ float sc[16];
+  const int64_t bh = blockIdx.y;
+  for (int e = threadIdx.x; e < D * 16; e += blockDim.x) {
+    const int d = e / 16, k = e % 16;
+    const bool in = k < rank;
+    reinterpret_cast<float*>(sP[d])[k] = in ? pp[(bh * D + d) * rank + k] : 0.f;
+    reinterpret_cast<float*>(sV[d])[k] = in ? vr[(bh * D + d) * rank + k] : 0.f;
+  }
+  if (threadIdx.x < 16) sc[threadIdx.x] = threadIdx.x < rank ? cc[bh * rank + threadIdx.x] : 0.f;
+  __syncthreads();
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= S) return;
+  float4* row = reinterpret_cast<float4*>(out + (bh * S + r) * D);
+  float y[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) y[k] = sc[k];
+#pragma unroll 4
+  for (int d4 = 0; d4 < D / 4; ++d4) {
+    const float4 xv = row[d4];
+    const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 p = sP[4 * d4 + j][k4];
+        y[4 * k4 + 0] = fmaf(xs[j], p.x, y[4 * k4 + 0]);
+        y[4 * k4 + 1] = fmaf(xs[j], p.y, y[4 * k4 + 1]);
+        y[4 * k4 + 2] = fmaf(xs[j], p.z, y[4 * k4 + 2]);
+        y[4 * k4 + 3] = fmaf(xs[j], p.w, y[4 * k4 + 3]);
+      }
+    }
+  }
+#pragma unroll 4
+  for (int d4 = 0; d4 < D / 4; ++d4) {
+    float4 xv = row[d4];
+    float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 v = sV[4 * d4 + j][k4];
+        xs[j] = fmaf(y[4 * k4 + 0], v.x, xs[j]);
+        xs[j] = fmaf(y[4 * k4 + 1], v.y, xs[j]);
+        xs[j] = fmaf(y[4 * k4 + 2], v.z, xs[j]);
+        xs[j] = fmaf(y[4 * k4 + 3], v.w, xs[j]);
+      }
+    }
+    row[d4] = make_float4(xs[0], xs[1], xs[2], xs[3]);
+  }
+}
+
 namespace {
 struct RepairLayout {
-  float *psum, *psq, *zt, *rr, *bc, *vr, *pp, *cc;
+  float *psum, *psq, *zt, *rr, *rv, *vr, *pp, *cc;
   size_t bytes;
 };
 RepairLayout carve_repair(int BH, int D, int M, int rank, void* ws) {
@@ -429,9 +544,9 @@ RepairLayout carve_repair(int BH, int D, int M, int rank, void* ws) {
   RepairLayout L{};
   L.psum = cv.take<float>(static_cast<size_t>(BH) * kStatSplit * D);
   L.psq = cv.take<float>(static_cast<size_t>(BH) * kStatSplit * D);
-  L.zt = cv.take<float>(static_cast<size_t>(BH) * M * (D + 1));
-  L.rr = cv.take<float>(static_cast<size_t>(BH) * M * D);
-  L.bc = cv.take<float>(static_cast<size_t>(BH) * (D + 1) * D);
+  L.zt = cv.take<float>(static_cast<size_t>(BH) * M * (D + 2));
+  L.rr = cv.take<float>(static_cast<size_t>(BH) * M * (D + 1));
+  L.rv = cv.take<float>(static_cast<size_t>(BH) * M * rank);
   L.vr = cv.take<float>(static_cast<size_t>(BH) * D * rank);
   L.pp = cv.take<float>(static_cast<size_t>(BH) * D * rank);
   L.cc = cv.take<float>(static_cast<size_t>(BH) * rank);
@@ -469,17 +584,20 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "column_stats_kernel"))) return rc;
   FitArgs fa{out, o_probe, probe_idx, weights, per_head, S, D, M, rank, lam, L.psum, L.psq,
-             L.zt,  L.rr,    L.bc,      L.vr,    L.pp,     L.cc};
-  const int n = M < D ? M : D;
-  const int ne = n + (n & 1);
-  const size_t big = std::max(static_cast<size_t>(D + 1) * (D + 1) + static_cast<size_t>(D + 1) * D,
-                              2 * static_cast<size_t>(ne) * (ne + 1)) * sizeof(float);
+             L.zt,  L.rr,    L.rv,      L.vr,    L.pp,     L.cc};
+  const size_t big = fit_plan(D, M, rank).floats * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(repair_fit_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(big));
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(repair_fit)");
   repair_fit_kernel<<<BH, kFitThreads, big, st>>>(fa);
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "repair_fit_kernel"))) return rc;
+  if (rank <= 16) {
+    auto ap16 = D == 64 ? repair_apply16_kernel<64> : repair_apply16_kernel<128>;
+    ap16<<<dim3((S + 255) / 256, BH), 256, 0, st>>>(out, S, rank, L.pp, L.cc, L.vr);
+    count_launch();
+    return check_cuda(cudaGetLastError(), "repair_apply16_kernel");
+  }
   const int nk = (rank + 15) & ~15;
   const int smem = (2 * D * nk + nk) * static_cast<int>(sizeof(float));
   auto ap = D == 64 ? repair_apply_kernel<64> : repair_apply_kernel<128>;
