@@ -302,6 +302,8 @@ __global__ void __launch_bounds__(256) gather_kv_centroids_kernel(
 struct AttnArgs {
   int B, Hq, Hkv, Sq, Sqpad, Skpad, Ck, Ckpad, Cq, G, Wg, Wc;
   int kstride;  // rows per (batch, KV head) in the tensors the K/V maps address
+  int ksplit;   // CTAs per query tile, each over a contiguous range of key groups
+  float* part;  // ksplit > 1: per split, unnormalised O, running max and sum per row
   int nh_slices, b_sliced, h_sliced;
   int compensate;
   float scale_log2;
@@ -358,7 +360,8 @@ __device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t*
     int w = gcur >> 5;
     uint32_t bits = any[w] & (0xffffffffu << (gcur & 31));
     while (bits == 0 && ++w < Wg) bits = any[w];
-    if (bits != 0) {
+    // (a kept group past G belongs to another CTA's key range)
+    if (bits != 0 && (w << 5) + __ffs(bits) - 1 < G) {
       const int b0 = __ffs(bits) - 1;
       const int g0 = (w << 5) + b0;
       const uint32_t a_hi = (w + 1 < Wg) ? any[w + 1] : 0u;
@@ -434,7 +437,11 @@ __global__ void __launch_bounds__(160, 2)
   uint32_t* cneed = uni_bits + 128;                                   // 4 words
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tile = blockIdx.x / a.ksplit, split = blockIdx.x % a.ksplit;
+  const int h = blockIdx.y, b = blockIdx.z;
+  // this CTA's key groups [g_lo, g_hi); the centroid chunks belong to the last split
+  const int g_lo = static_cast<int>((static_cast<int64_t>(a.G) * split) / a.ksplit);
+  const int g_hi = static_cast<int>((static_cast<int64_t>(a.G) * (split + 1)) / a.ksplit);
   const int hkv = h / (a.Hq / a.Hkv);
   const int slice = (a.b_sliced ? b : 0) * a.nh_slices + (a.h_sliced ? h : 0);
   const uint32_t bar0 = smem_u32(bars);
@@ -496,7 +503,7 @@ __global__ void __launch_bounds__(160, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int ncc = a.compensate ? a.Ckpad / 128 : 0;
+  const int ncc = (a.compensate && split == a.ksplit - 1) ? a.Ckpad / 128 : 0;
 
   if (warp == 0) {
     // ------------------------------------------------ control warp: TMA + tcgen05.mma
@@ -537,9 +544,9 @@ __global__ void __launch_bounds__(160, 2)
       }
       __syncwarp();
     };
-    int gcur = 0, ccur = 0, j = 0, nk = 0, nv = 0;
+    int gcur = g_lo, ccur = 0, j = 0, nk = 0, nv = 0;
     Chunk cur, nxt, nn;
-    bool have = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, cur);
+    bool have = next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, cur);
     if (leader) {
       mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
 #pragma unroll
@@ -601,7 +608,7 @@ __global__ void __launch_bounds__(160, 2)
           commit(BAR(BAR_SFHI));
         }
         commit(BAR(BAR_KE));
-        have_next = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nxt);
+        have_next = next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, nxt);
         if (have_next && (ok = wait_all(BAR(BAR_KE), 0, 1))) {
           load_kv(nxt, false);
           ++nk;
@@ -646,7 +653,7 @@ __global__ void __launch_bounds__(160, 2)
         load_kv(nxt, true);
         ++nv;
         // K stage: refill with the chunk after once QK(j+1) has read it
-        have_nn = next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, nn);
+        have_nn = next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, nn);
         if (have_nn) {
           if (!(ok = wait_all(BAR(BAR_KE), (j + 1) & 1, 1))) break;
           load_kv(nn, false);
@@ -682,10 +689,10 @@ __global__ void __launch_bounds__(160, 2)
     const uint32_t tO = tS + 128;
     const float scl = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    int gcur = 0, ccur = 0, j = 0, hi_n = 0;  // hi_n: high steps taken so far
+    int gcur = g_lo, ccur = 0, j = 0, hi_n = 0;  // hi_n: high steps taken so far
     bool ok = true;
     Chunk ch;
-    while (next_chunk(gcur, ccur, any_bits, uni_bits, a.G, a.Wg, cneed, ncc, ch)) {
+    while (next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, ch)) {
       const int nsteps = ch.n > 64 ? 2 : 1;
 #pragma unroll 1
       for (int half = 0; half < nsteps; ++half) {
@@ -882,7 +889,26 @@ __global__ void __launch_bounds__(160, 2)
       if (!ok) break;
       ++j;
     }
-    if (ok && mbar_wait(BAR(BAR_OF), 0, abort_flag, 10)) {
+    const bool o_final = ok && mbar_wait(BAR(BAR_OF), 0, abort_flag, 10);
+    if (o_final && a.ksplit > 1) {
+      // one key range of several: unnormalised O plus running max and sum, merged later
+      tc_fence_after();
+      const size_t prow = (((static_cast<size_t>(b) * a.Hq + h) * a.ksplit + split) * a.Sqpad) + qrow;
+      float* po = a.part + prow * D;
+      float* pml = a.part + static_cast<size_t>(a.B) * a.Hq * a.ksplit * a.Sqpad * D + prow * 2;
+#pragma unroll 1
+      for (int p = 0; p < D / 32; ++p) {
+        float o[32];
+        tmem_ld32(tO + p * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4*>(po + p * 32 + 4 * i) =
+              make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+      }
+      pml[0] = m_run;
+      pml[1] = l_run;
+    } else if (o_final) {
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       float* orow = a.out + ((static_cast<size_t>(b) * a.Hq + h) * a.Sq + (tok >= 0 ? tok : 0)) * D;
@@ -912,11 +938,51 @@ __global__ void __launch_bounds__(160, 2)
   }
 }
 
+
+// Merge of the key-range splits of one query row (one warp per row, grid (ceil(Sqpad / 8),
+// Hq, B), 256 threads): m = max_s m_s, l = sum_s l_s 2^(m_s - m),
+// O = sum_s O_s 2^(m_s - m) / l, written to the row's token position (log2 units, as
+// the kernel keeps them). A row no split saw (l = 0) is written as zeros.
+template <int D>
+__global__ void __launch_bounds__(256) combine_splits_kernel(const float* __restrict__ part,
+                                                             const int32_t* __restrict__ qrow_token,
+                                                             int B, int Hq, int ksplit, int Sqpad,
+                                                             int Sq, float* __restrict__ out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qrow = blockIdx.x * 8 + warp;
+  const int h = blockIdx.y, b = blockIdx.z;
+  if (qrow >= Sqpad) return;
+  const int tok = qrow_token[qrow];
+  if (tok < 0) return;
+  const size_t bhs = (static_cast<size_t>(b) * Hq + h) * ksplit;
+  const float* ml = part + static_cast<size_t>(B) * Hq * ksplit * Sqpad * D;
+  float m = -INFINITY;
+  for (int s = 0; s < ksplit; ++s) m = fmaxf(m, ml[((bhs + s) * Sqpad + qrow) * 2]);
+  float l = 0.f, acc[D / 32];
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
+  for (int s = 0; s < ksplit; ++s) {
+    const size_t prow = (bhs + s) * Sqpad + qrow;
+    const float ls = ml[prow * 2 + 1];
+    if (!(ls > 0.f)) continue;
+    const float f = exp2f(ml[prow * 2] - m);
+    l = fmaf(ls, f, l);
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(part[prow * D + e * 32 + lane], f, acc[e]);
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  float* orow = out + ((static_cast<size_t>(b) * Hq + h) * Sq + tok) * D;
+#pragma unroll
+  for (int e = 0; e < D / 32; ++e) orow[e * 32 + lane] = acc[e] * inv;
+}
+
 // ============================================================== host side
 namespace {
 
 struct AttnLayout {
   int Sqpad, Skpad, G, Wg, Ckpad, Wc, Cqpad;
+  int ksplit;   // CTAs per query tile over disjoint key ranges (1 = no split)
+  float* part;  // ksplit > 1: partial O (B,Hq,ksplit,Sqpad,D), then max and sum (...,2)
   int32_t *qrow_token, *qrow_label, *q_count, *q_off;
   int32_t *kslot_token, *group_cluster, *group_valid, *k_count, *k_off;
   float* bias2;
@@ -955,6 +1021,15 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
   L.vp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Skpad * s.D * es);
   L.kc = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Ckpad * s.D * es);
   L.vc = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Ckpad * s.D * es);
+  // Key-range split when the query tiles alone leave most of the GPU idle (e.g. the
+  // 64 probe rows per head): about 2 CTAs per SM of a 148-SM part, each split at least
+  // 8 key groups (128 keys), at most 16 splits.
+  const int64_t ctas = static_cast<int64_t>(L.Sqpad / 128) * s.Hq * s.B;
+  int ks = ctas >= 148 ? 1 : static_cast<int>(296 / ctas);
+  ks = std::min(ks, std::min(16, L.G / 8));
+  L.ksplit = std::max(ks, 1);
+  L.part = L.ksplit > 1 ? cv.take<float>(static_cast<size_t>(s.B) * s.Hq * L.ksplit * L.Sqpad * (s.D + 2))
+                        : nullptr;
   L.bytes = align_up(cv.used, 256);
   return L;
 }
@@ -970,6 +1045,11 @@ int launch_attn(const CUtensorMap* maps, const AttnArgs& args, dim3 grid, int pr
   prof_begin(prof_id, st);
   kern<<<grid, 160, Cfg::SMEM_LAUNCH, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], args);
   count_launch();
+  if (args.ksplit > 1) {
+    combine_splits_kernel<D><<<dim3((args.Sqpad + 7) / 8, args.Hq, args.B), 256, 0, st>>>(
+        args.part, args.qrow_token, args.B, args.Hq, args.ksplit, args.Sqpad, args.Sq, args.out);
+    count_launch();
+  }
   prof_end(prof_id, st);
   return check_cuda(cudaGetLastError(), "attn_kernel launch");
 }
@@ -1124,7 +1204,9 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
   args.cnonempty = L.cnonempty;
   args.bias2 = L.bias2;
   args.out = out;
-  const dim3 grid(L.Sqpad / 128, s.Hq, s.B);
+  args.ksplit = L.ksplit;
+  args.part = L.part;
+  const dim3 grid((L.Sqpad / 128) * L.ksplit, s.Hq, s.B);
   if (s.dtype == BSA_F32) {
     return s.D == 64 ? launch_attn<64, true>(maps, args, grid, prof_id, st)
                      : launch_attn<128, true>(maps, args, grid, prof_id, st);

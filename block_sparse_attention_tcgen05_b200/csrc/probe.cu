@@ -65,26 +65,50 @@ __global__ void __launch_bounds__(256) centroid_order_kernel(
     if (threadIdx.x == 0) report_device_error(kStatusUnsupported, 50);
     return;
   }
+  // Rows are read warp by warp (lane l holds elements [l·D/32, (l+1)·D/32) of a row,
+  // so a warp reads whole rows coalesced); warps stride over the members.
   const T* qb = q + bh * S * D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int epl = D / 32;  // 2 or 4
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i = warp; i < n; i += nw) {
+    const T* row = qb + static_cast<int64_t>(slot_token[start + i]) * D + lane * epl;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (e < epl) acc[e] += to_f(row[e]);
+  }
+  __shared__ float part[8][128];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (e < epl) part[warp][lane * epl + e] = acc[e];
+  __syncthreads();
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < n; ++i) acc += to_f(qb[static_cast<int64_t>(slot_token[start + i]) * D + d]);
-    mean[d] = acc / static_cast<float>(n);
+    float t = 0.f;
+    for (int w = 0; w < nw; ++w) t += part[w][d];
+    mean[d] = t / static_cast<float>(n);
   }
   __syncthreads();
   int np = 1;
   while (np < n) np <<= 1;
-  for (int i = threadIdx.x; i < np; i += blockDim.x) {
+  for (int i = warp; i < np; i += nw) {
     if (i < n) {
       const int tok = slot_token[start + i];
-      float acc = 0.f;
-      for (int d = 0; d < D; ++d) {
-        const float x = to_f(qb[static_cast<int64_t>(tok) * D + d]) - mean[d];
-        acc = fmaf(x, x, acc);
+      const T* row = qb + static_cast<int64_t>(tok) * D + lane * epl;
+      float sq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (e < epl) {
+          const float x = to_f(row[e]) - mean[lane * epl + e];
+          sq = fmaf(x, x, sq);
+        }
       }
-      dist[i] = sqrtf(acc);
-      tokn[i] = tok;
-    } else {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (lane == 0) {
+        dist[i] = sqrtf(sq);
+        tokn[i] = tok;
+      }
+    } else if (lane == 0) {
       dist[i] = INFINITY;
       tokn[i] = 0x7fffffff;
     }
