@@ -58,6 +58,23 @@ def parse():
     return p.parse_args()
 
 
+def max_over_ranks(values, device, world):
+    """Element-wise maximum of per-rank timings over all ranks (every rank gets it):
+    a multi-GPU step is as slow as its slowest rank."""
+    if world <= 1:
+        return [float(x) for x in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_tflops(flop_per_rank, world, ms):
+    """Whole-job throughput: every rank processes its own copy of the workload."""
+    return world * flop_per_rank / (ms * 1e-3) / 1e12
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -305,10 +322,7 @@ def main():
     _lib.call("bsa_profile_read", 0, ctypes.byref(attn_ms), ctypes.byref(attn_n))
     _lib.call("bsa_profile_enable", 0)
     attn_ms_launch = attn_ms.value / max(1, attn_n.value)
-    if world > 1:
-        t = torch.tensor([ms, attn_ms_launch], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, attn_ms_launch = float(t[0]), float(t[1])
+    ms, attn_ms_launch = max_over_ranks([ms, attn_ms_launch], dev, world)
     st, _ = bsa.device_status(dev)
     if st != 0:
         raise RuntimeError(f"device status {st} after the timed region")
@@ -343,13 +357,10 @@ def main():
         torch.cuda.synchronize()
         barrier()
         e2e_ms = a.elapsed_time(b) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        (e2e_ms,) = max_over_ranks([e2e_ms], dev, world)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, mh))
         d2h = oh.numel() * oh.element_size()
-        e2e = {"value": world * flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": weak_scaling_tflops(flop, world, e2e_ms), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "block_sparse_attention_tcgen05_b200.centroid_compensated_attention"}
         del qh, kh, vh, oh, qd, kd, vd
@@ -364,7 +375,7 @@ def main():
         achieved = flop / (attn_ms_launch * 1e-3) / 1e12
         line = {
             "metric": METRIC,
-            "value": world * flop / (ms * 1e-3) / 1e12,
+            "value": weak_scaling_tflops(flop, world, ms),
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": args.steps,
