@@ -91,43 +91,58 @@ __device__ __forceinline__ bool header_matches(const void* state, int B, int H, 
 }
 
 // grid (kPoolSplit, B*H): partial column sums of q and k over a slice of the tokens.
+// Rows are read as 16-byte vectors (thread = one vector column of a row; the CTA walks
+// 256 / (vectors per row) rows at a time), partial sums combined in shared memory.
 template <typename T>
 __global__ void __launch_bounds__(256) pool_kernel(void* state, const T* __restrict__ q,
                                                    const T* __restrict__ k, int B, int H, int S,
                                                    int D) {
-  __shared__ float sq[256], sk[256];
+  constexpr int EPV = 16 / sizeof(T);
+  __shared__ float red[2][256 * EPV];
   if (!header_matches(state, B, H, D)) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) report_device_error(kStatusBadLabel, 60);
     return;
   }
   float* part = device_layout(state).part;
   const int64_t bh = blockIdx.y;
-  const int d = threadIdx.x % D, lr = threadIdx.x / D, rp = 256 / D;
+  const int vpr = D / EPV, rpi = 256 / vpr;
+  const int rin = threadIdx.x / vpr, v = threadIdx.x % vpr;
   const int r0 = static_cast<int>((static_cast<int64_t>(S) * blockIdx.x) / kPoolSplit);
   const int r1 = static_cast<int>((static_cast<int64_t>(S) * (blockIdx.x + 1)) / kPoolSplit);
-  float a = 0.f, b = 0.f;
-  for (int r = r0 + lr; r < r1; r += rp) {
-    const int64_t e = (bh * S + r) * D + d;
-    if constexpr (sizeof(T) == 2) {
-      a += __bfloat162float(q[e]);
-      b += __bfloat162float(k[e]);
-    } else {
-      a += q[e];
-      b += k[e];
+  const uint4* q4 = reinterpret_cast<const uint4*>(q) + bh * S * vpr;
+  const uint4* k4 = reinterpret_cast<const uint4*>(k) + bh * S * vpr;
+  float a[EPV], c[EPV];
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) a[e] = c[e] = 0.f;
+  for (int r = r0 + rin; r < r1; r += rpi) {
+    const uint4 xq = __ldg(q4 + static_cast<int64_t>(r) * vpr + v);
+    const uint4 xk = __ldg(k4 + static_cast<int64_t>(r) * vpr + v);
+    float fq[EPV], fk[EPV];
+    unpack16<T>(xq, fq);
+    unpack16<T>(xk, fk);
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) {
+      a[e] += fq[e];
+      c[e] += fk[e];
     }
   }
-  sq[threadIdx.x] = a;
-  sk[threadIdx.x] = b;
+  if (rin < rpi) {
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) {
+      red[0][rin * D + v * EPV + e] = a[e];
+      red[1][rin * D + v * EPV + e] = c[e];
+    }
+  }
   __syncthreads();
-  if (threadIdx.x < D) {
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float ta = 0.f, tb = 0.f;
-    for (int i = 0; i < rp; ++i) {
-      ta += sq[i * D + threadIdx.x];
-      tb += sk[i * D + threadIdx.x];
+    for (int i = 0; i < rpi; ++i) {
+      ta += red[0][i * D + d];
+      tb += red[1][i * D + d];
     }
     float* o = part + (bh * kPoolSplit + blockIdx.x) * 2 * D;
-    o[threadIdx.x] = ta;
-    o[D + threadIdx.x] = tb;
+    o[d] = ta;
+    o[D + d] = tb;
   }
 }
 
@@ -257,9 +272,13 @@ extern "C" int bsa_mask_cache_should_refresh(void* state, const void* q, const v
   using namespace bsa;
   if (!state || !q || !k || !refresh) return fail(BSA_ERR_INVALID_ARG, "null pointer");
   if (shape.Hq != shape.Hkv) return fail(BSA_ERR_INVALID_ARG, "the cache needs Hkv == Hq");
+  const int es = shape.dtype == BSA_F32 ? 4 : 2;
   if (shape.B <= 0 || shape.Hq <= 0 || shape.Sq <= 0 || shape.D <= 0 || shape.D > 256 ||
-      256 % shape.D)
-    return fail(BSA_ERR_UNSUPPORTED, "head dim %d must divide 256", shape.D);
+      256 % shape.D || (shape.D * es) % 16)
+    return fail(BSA_ERR_UNSUPPORTED, "head dim %d must divide 256 and rows be 16-byte multiples",
+                shape.D);
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k)) % 16)
+    return fail(BSA_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
   cudaStream_t st = as_stream(stream);
   const int BH = shape.B * shape.Hq;
   int rc;

@@ -270,7 +270,9 @@ int bsa_mask_cache_init(void* state, int B, int H, int Cq, int Ck, int D, float 
  * against the anchors, applies delta and the layer gate, and writes refresh
  * (device uint8 (B,H)). If n_refresh_host is non-NULL the stream is synchronised and
  * the number of refreshed heads is written there. drift_out (nullable) receives the
- * float32 (B,H) drift (+inf where no anchor exists yet).
+ * float32 (B,H) drift (+inf where no anchor exists yet). q and k must be 16-byte
+ * aligned and D·(element size) a multiple of 16 bytes (D dividing 256), else
+ * BSA_ERR_INVALID_ARG / BSA_ERR_UNSUPPORTED.
  */
 int bsa_mask_cache_should_refresh(void* state, const void* q, const void* k, bsa_shape shape,
                                   uint8_t* refresh, float* drift_out, int* n_refresh_host,
