@@ -36,12 +36,32 @@ namespace bsa {
 // cluster_pad)), filled with its tokens in increasing token order (a stable sort);
 // remaining slots hold token -1 / label -1. With group arrays given, 16-slot group g
 // is described by the cluster owning it and its number of real tokens.
-__global__ void __launch_bounds__(1024) label_sort_kernel(
-    const int32_t* __restrict__ labels, int S, int C, int cluster_pad, int n_slots,
-    int32_t* __restrict__ slot_token, int32_t* __restrict__ slot_label,
-    int32_t* __restrict__ count, int32_t* __restrict__ off, int32_t* __restrict__ group_cluster,
-    int32_t* __restrict__ group_valid, int n_groups, float* __restrict__ bias2, int C_pad,
-    uint32_t* __restrict__ nonempty_bits) {
+struct LabelSortJob {
+  const int32_t* labels;
+  int S, C, cluster_pad, n_slots;
+  int32_t *slot_token, *slot_label, *count, *off, *group_cluster, *group_valid;
+  int n_groups;
+  float* bias2;
+  int C_pad;
+  uint32_t* nonempty_bits;
+};
+
+// CTA b sorts job b (the query and key sorts of one call run side by side).
+__global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
+                                                          const LabelSortJob j1) {
+  const LabelSortJob& jb = blockIdx.x == 0 ? j0 : j1;
+  const int32_t* __restrict__ labels = jb.labels;
+  const int S = jb.S, C = jb.C, cluster_pad = jb.cluster_pad, n_slots = jb.n_slots;
+  int32_t* __restrict__ slot_token = jb.slot_token;
+  int32_t* __restrict__ slot_label = jb.slot_label;
+  int32_t* __restrict__ count = jb.count;
+  int32_t* __restrict__ off = jb.off;
+  int32_t* __restrict__ group_cluster = jb.group_cluster;
+  int32_t* __restrict__ group_valid = jb.group_valid;
+  const int n_groups = jb.n_groups;
+  float* __restrict__ bias2 = jb.bias2;
+  const int C_pad = jb.C_pad;
+  uint32_t* __restrict__ nonempty_bits = jb.nonempty_bits;
   extern __shared__ int32_t sm_i32[];
   int32_t* cnt = sm_i32;     // C
   int32_t* run = cnt + C;    // C + 1
@@ -1075,19 +1095,26 @@ size_t attention_workspace_bytes(const bsa_shape& s, int Cq, int Ck) {
   return carve(s, Cq, Ck, nullptr).bytes;
 }
 
+// One or two label sorts in one launch (one CTA each).
+static int launch_label_sorts(const LabelSortJob& j0, const LabelSortJob* j1, cudaStream_t st) {
+  const int c = j1 && j1->C > j0.C ? j1->C : j0.C;
+  const int smem = (2 * c + 1) * 4;
+  cudaError_t e = cudaFuncSetAttribute(label_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem > 48 * 1024 ? smem : 48 * 1024);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(label_sort)");
+  label_sort_kernel<<<j1 ? 2 : 1, 1024, smem, st>>>(j0, j1 ? *j1 : j0);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "label_sort_kernel launch");
+}
+
 int run_label_sort(const int32_t* labels, int S, int C, int cluster_pad, int n_slots,
                    int32_t* slot_token, int32_t* slot_label, int32_t* count, int32_t* off,
                    int32_t* group_cluster, int32_t* group_valid, int n_groups, float* bias2,
                    int C_pad, uint32_t* nonempty, cudaStream_t st) {
-  const int smem = (2 * C + 1) * 4;
-  cudaError_t e = cudaFuncSetAttribute(label_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       smem > 48 * 1024 ? smem : 48 * 1024);
-  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(label_sort)");
-  label_sort_kernel<<<1, 1024, smem, st>>>(labels, S, C, cluster_pad, n_slots, slot_token,
-                                           slot_label, count, off, group_cluster, group_valid,
-                                           n_groups, bias2, C_pad, nonempty);
-  count_launch();
-  return check_cuda(cudaGetLastError(), "label_sort_kernel launch");
+  const LabelSortJob j{labels,        S,           C,     cluster_pad,   n_slots, slot_token,
+                       slot_label,    count,       off,   group_cluster, group_valid,
+                       n_groups,      bias2,       C_pad, nonempty};
+  return launch_label_sorts(j, nullptr, st);
 }
 
 int centroid_compensated_attention(const void* q, const void* k, const void* v,
@@ -1112,13 +1139,15 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     return fail(BSA_ERR_INVALID_ARG, "q/k/v must be 16-byte aligned");
 
   // 1. label sorts
-  if ((rc = run_label_sort(k_labels, s.Sk, Ck, 16, L.Skpad, L.kslot_token, nullptr, L.k_count,
-                           L.k_off, L.group_cluster, L.group_valid, L.G, L.bias2, L.Ckpad,
-                           L.cnonempty, st)))
-    return rc;
-  if ((rc = run_label_sort(q_labels, s.Sq, Cq, 1, L.Sqpad, L.qrow_token, L.qrow_label, L.q_count,
-                           L.q_off, nullptr, nullptr, 0, nullptr, 0, nullptr, st)))
-    return rc;
+  {
+    const LabelSortJob jk{k_labels,       s.Sk,           Ck,      16,         L.Skpad,
+                          L.kslot_token,  nullptr,        L.k_count, L.k_off,  L.group_cluster,
+                          L.group_valid,  L.G,            L.bias2, L.Ckpad,    L.cnonempty};
+    const LabelSortJob jq{q_labels, s.Sq,    Cq,      1,       L.Sqpad, L.qrow_token, L.qrow_label,
+                          L.q_count, L.q_off, nullptr, nullptr, 0,       nullptr,      0,
+                          nullptr};
+    if ((rc = launch_label_sorts(jk, &jq, st))) return rc;
+  }
   // 2. mask bitsets
   const int nb = mbs ? s.B : 1, nh = mhs ? s.Hq : 1;
   mask_bits_kernel<<<dim3(Cq, nh, nb), 256, 0, st>>>(mask, mbs, mhs, nh, Cq, Ck, L.group_cluster,
