@@ -91,30 +91,201 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return red[0];
 }
 
-// Circle-method round robin: round r of n (even) players pairs r with n-1 and
-// (r+i) with (r-i) (mod n-1) for i = 1 .. n/2-1; every pair meets once per n-1 rounds.
-__device__ __forceinline__ void round_pair(int n, int r, int i, int& p, int& q) {
-  if (i == 0) {
-    p = r;
-    q = n - 1;
-  } else {
-    p = (r + i) % (n - 1);
-    q = (r - i + (n - 1)) % (n - 1);
+
+// Top-k eigenpairs of a symmetric n x n matrix A (n <= 128, row stride ld, in shared
+// memory), all threads of the CTA taking part:
+//  1. Householder reduction to tridiagonal form T = Hᵀ A H (reflector k in hv row k,
+//     A overwritten), diag d, off-diagonal e;
+//  2. the k largest eigenvalues of T by bisection on Sturm counts (one thread each);
+//  3. their eigenvectors by inverse iteration on T (one thread each), then modified
+//     Gram-Schmidt in order of decreasing eigenvalue;
+//  4. back-transformation by the reflectors: U = H x.
+// Output: U (n x min(k, n), row stride ld >= n) and lam[0..k) in decreasing order
+// (zero past n). hv needs n x ld floats, x n x k, work 5n + k n floats.
+__device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float* U, float* lam,
+                               float* x, float* work, float* red) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  float* d = work;
+  float* e = work + n;        // e[i] couples i and i+1
+  float* pv = work + 2 * n;   // A v
+  float* wv = work + 3 * n;   // w = 2(p - K v)
+  __shared__ float s_scal[2];
+  // 1. Householder: column k below the diagonal is mapped to (alpha, 0, ..., 0)
+  for (int c = 0; c + 2 < n; ++c) {
+    const int m = n - c - 1;  // length of the column below the diagonal
+    float ss = 0.f;
+    for (int i = tid; i < m; i += nt) {
+      const float xi = A[(c + 1 + i) * ld + c];
+      ss = fmaf(xi, xi, ss);
+    }
+    ss = block_sum(ss, red);
+    const float x0 = A[(c + 1) * ld + c];
+    const float nrm = sqrtf(ss);
+    const float alpha = x0 > 0.f ? -nrm : nrm;
+    // v = x - alpha e1, normalised; |v|^2 = ss - 2 alpha x0 + alpha^2 = 2(ss - alpha x0)
+    const float vv = 2.f * (ss - alpha * x0);
+    const bool skip = !(vv > 1e-30f * (ss + 1e-30f));
+    const float inv = skip ? 0.f : rsqrtf(vv);
+    for (int i = tid; i < m; i += nt) {
+      const float xi = A[(c + 1 + i) * ld + c];
+      hv[c * ld + i] = (i == 0 ? xi - alpha : xi) * inv;
+    }
+    __syncthreads();
+    if (!skip) {
+      // p = A' v over the trailing block A' = A[c+1.., c+1..]
+      for (int i = tid; i < m; i += nt) {
+        float acc = 0.f;
+        for (int j = 0; j < m; ++j) acc = fmaf(A[(c + 1 + i) * ld + c + 1 + j], hv[c * ld + j], acc);
+        pv[i] = acc;
+      }
+      __syncthreads();
+      float kk = 0.f;
+      for (int i = tid; i < m; i += nt) kk = fmaf(hv[c * ld + i], pv[i], kk);
+      kk = block_sum(kk, red);
+      for (int i = tid; i < m; i += nt) wv[i] = 2.f * (pv[i] - kk * hv[c * ld + i]);
+      __syncthreads();
+      // A' <- A' - v wᵀ - w vᵀ  (= H A' H with H = I - 2 v vᵀ)
+      for (int e2 = tid; e2 < m * m; e2 += nt) {
+        const int i = e2 / m, j = e2 % m;
+        A[(c + 1 + i) * ld + c + 1 + j] -= hv[c * ld + i] * wv[j] + wv[i] * hv[c * ld + j];
+      }
+    }
+    if (tid == 0) {
+      d[c] = A[c * ld + c];
+      e[c] = skip ? x0 : alpha;
+    }
+    __syncthreads();
   }
-  if (p > q) {
-    const int t = p;
-    p = q;
-    q = t;
+  if (tid == 0) {
+    for (int c = (n >= 2 ? n - 2 : 0); c < n; ++c) d[c] = A[c * ld + c];
+    if (n >= 2) e[n - 2] = A[(n - 1) * ld + (n - 2)];
   }
+  __syncthreads();
+  // 2. bisection: eigenvalue j (ascending) of T is the x where the Sturm count
+  //    #{eigenvalues < x} passes j; thread t takes the t-th largest, j = n - 1 - t
+  float* e2 = work + 4 * n;
+  for (int i = tid; i < n; i += nt) e2[i] = i + 1 < n ? e[i] * e[i] : 0.f;
+  if (tid == 0) {
+    float lo = INFINITY, hi = -INFINITY, emax = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const float r = (i > 0 ? fabsf(e[i - 1]) : 0.f) + (i + 1 < n ? fabsf(e[i]) : 0.f);
+      lo = fminf(lo, d[i] - r);
+      hi = fmaxf(hi, d[i] + r);
+      if (i + 1 < n) emax = fmaxf(emax, e2[i]);
+    }
+    const float span = fmaxf(hi - lo, 1e-30f);
+    s_scal[0] = lo - 1e-6f * span;
+    s_scal[1] = hi + 1e-6f * span;
+  }
+  __syncthreads();
+  const int kk = k < n ? k : n;
+  const float lo0 = s_scal[0], hi0 = s_scal[1];
+  const float pivmin = 1e-30f + 1e-12f * (hi0 - lo0) * (hi0 - lo0);
+  if (tid < kk) {
+    const int j = n - 1 - tid;
+    float a = lo0, b = hi0;
+    for (int it = 0; it < 60; ++it) {
+      const float mid = 0.5f * (a + b);
+      if (!(mid > a && mid < b)) break;  // float resolution reached
+      int cnt = 0;
+      float q = d[0] - mid;
+      for (int i = 0;; ++i) {
+        if (fabsf(q) < pivmin) q = -pivmin;
+        cnt += q < 0.f;
+        if (i + 1 >= n) break;
+        q = d[i + 1] - mid - __fdividef(e2[i], q);
+      }
+      if (cnt > j) b = mid;
+      else a = mid;
+    }
+    lam[tid] = 0.5f * (a + b);
+  }
+  __syncthreads();
+  // 3. inverse iteration: solve (T - lam I) y = x by elimination with guarded pivots
+  //    (thread t keeps its elimination factors in cs row t), normalise; 3 rounds
+  float* cs = work + 5 * n;  // k x n
+  if (tid < kk) {
+    const float lt = lam[tid];
+    float* f = cs + tid * n;
+    for (int i = 0; i < n; ++i) x[i * k + tid] = 1.f + 0.25f * static_cast<float>((i * 7 + tid * 13) % 11) / 11.f;
+    for (int round = 0; round < 3; ++round) {
+      // forward: m_i = (d_i - lt) - e_{i-1} f_{i-1}, f_i = e_i / m_i, y_i = (x_i - e_{i-1} y_{i-1}) / m_i
+      float yprev = 0.f, fprev = 0.f;
+      for (int i = 0; i < n; ++i) {
+        float mi = d[i] - lt - (i > 0 ? e[i - 1] * fprev : 0.f);
+        if (fabsf(mi) < pivmin) mi = mi < 0.f ? -pivmin : pivmin;
+        const float rm = 1.f / mi;
+        fprev = i + 1 < n ? e[i] * rm : 0.f;
+        f[i] = fprev;
+        yprev = (x[i * k + tid] - (i > 0 ? e[i - 1] * yprev : 0.f)) * rm;
+        x[i * k + tid] = yprev;
+      }
+      // back: y_i -= f_i y_{i+1}
+      float nrm = 0.f;
+      for (int i = n - 1; i >= 0; --i) {
+        float yi = x[i * k + tid];
+        if (i + 1 < n) yi -= f[i] * x[(i + 1) * k + tid];
+        x[i * k + tid] = yi;
+        nrm = fmaf(yi, yi, nrm);
+      }
+      const float rn = nrm > 0.f ? rsqrtf(nrm) : 0.f;
+      for (int i = 0; i < n; ++i) x[i * k + tid] *= rn;
+    }
+  }
+  __syncthreads();
+  //    modified Gram-Schmidt (warp 0) in order of decreasing eigenvalue: repairs the
+  //    loss of orthogonality of inverse iteration within clusters of eigenvalues
+  if (tid < 32) {
+    for (int t = 0; t < kk; ++t) {
+      for (int s = 0; s < t; ++s) {
+        float dot = 0.f;
+        for (int i = tid; i < n; i += 32) dot = fmaf(x[i * k + s], x[i * k + t], dot);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        for (int i = tid; i < n; i += 32) x[i * k + t] -= dot * x[i * k + s];
+        __syncwarp();
+      }
+      float nrm = 0.f;
+      for (int i = tid; i < n; i += 32) nrm = fmaf(x[i * k + t], x[i * k + t], nrm);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
+      const float rn = nrm > 0.f ? rsqrtf(nrm) : 0.f;
+      for (int i = tid; i < n; i += 32) x[i * k + t] *= rn;
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // 4. back-transformation: x <- H_c x for c = n-3 .. 0, H_c = I - 2 v_c v_cᵀ on rows c+1..
+  for (int c = n - 3; c >= 0; --c) {
+    const int m = n - c - 1;
+    if (tid < kk) {
+      float s = 0.f;
+      for (int i = 0; i < m; ++i) s = fmaf(hv[c * ld + i], x[(c + 1 + i) * k + tid], s);
+      pv[tid] = 2.f * s;
+    }
+    __syncthreads();
+    for (int e3 = tid; e3 < m * kk; e3 += nt) {
+      const int i = e3 / kk, t = e3 % kk;
+      x[(c + 1 + i) * k + t] -= hv[c * ld + i] * pv[t];
+    }
+    __syncthreads();
+  }
+  for (int e3 = tid; e3 < n * kk; e3 += nt) {  // only the kk <= n columns that exist
+    const int i = e3 / kk, t = e3 % kk;
+    U[i * ld + t] = x[i * k + t];
+  }
+  for (int t = kk + tid; t < k; t += nt) lam[t] = 0.f;
+  __syncthreads();
 }
 
 // Shared-memory plan of the fit, in floats: the standardised probe rows Zt (M x ldz)
 // and residuals R (M x ldr) and R V_r (M x rk) when they fit (else they stay in the
-// workspace), a region W used first by the eigen step (G and V, ne x (ne + 1) each)
-// and then by the solve (A: n1 x n1, right-hand sides n1 x rk), V_r (D x rk) and the
-// Cholesky pivots. Odd row strides keep column-wise sweeps on distinct banks.
+// workspace), a region W used first by the eigen step (the Gram matrix, later its
+// eigenvectors, n x ld; the reflectors n x ld; inverse-iteration vectors n x rk and
+// scratch) and then by the solve (A: n1 x n1, right-hand sides n1 x rk), V_r (D x rk)
+// and the Cholesky pivots.
 struct FitPlan {
-  int n1, n, ne, ld, ldz, ldr, rk;
+  int n1, n, ld, ldz, ldr, rk;
   bool local_zr;                   // Zt, R, R V_r in shared memory
   size_t zt, rr, rv, w, vr, piv;   // offsets (floats) into the dynamic shared memory
   size_t floats;
@@ -123,12 +294,12 @@ __host__ __device__ inline FitPlan fit_plan(int D, int M, int rk) {
   FitPlan p{};
   p.n1 = D + 1;
   p.n = M < D ? M : D;
-  p.ne = p.n + (p.n & 1);
-  p.ld = p.ne + 1;
+  p.ld = p.n + 1;
   p.ldz = D + 2;
   p.ldr = D + 1;
   p.rk = rk;
-  const size_t wa = static_cast<size_t>(2) * p.ne * p.ld;
+  const size_t wa = static_cast<size_t>(2) * p.n * p.ld + static_cast<size_t>(2) * p.n * rk +
+                    static_cast<size_t>(5) * p.n;
   const size_t wb = static_cast<size_t>(p.n1) * p.n1 + static_cast<size_t>(p.n1) * rk;
   const size_t wsz = wa > wb ? wa : wb;
   const size_t common = wsz + static_cast<size_t>(D) * rk + p.n1;
@@ -155,14 +326,12 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   __shared__ float mu[128], isg[128], red[32];
   __shared__ float wv[1024];
   __shared__ int sel[128];
-  __shared__ float csn[64][2];
-  __shared__ int cpq[64][2];
-  __shared__ uint8_t pairs[127][64][2];  // circle-method pair table: round, slot -> (p, q)
+  __shared__ float evl[128];  // eigenvalues of the residual Gram matrix, decreasing
   const int tid = threadIdx.x, nt = blockDim.x;
   const int64_t bh = blockIdx.x;
   const int S = a.S, D = a.D, M = a.M, rk = a.rank;
   const FitPlan pl = fit_plan(D, M, rk);
-  const int n1 = pl.n1, n = pl.n, ne = pl.ne, ld = pl.ld, ldz = pl.ldz, ldr = pl.ldr;
+  const int n1 = pl.n1, n = pl.n, ld = pl.ld, ldz = pl.ldz, ldr = pl.ldr;
   const bool small = M < D;
   const float* X = a.out + bh * S * D;
   const int32_t* idx = a.per_head ? a.probe_idx + bh * M : a.probe_idx;
@@ -201,105 +370,34 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   for (int m = tid; m < M; m += nt) zt[m * ldz + D] = 1.f;
   __syncthreads();
   // 3. Gram matrix of the weighted residuals, n x n with n = min(M, D):
-  //    W½ R Rᵀ W½ (M < D) or Rᵀ W R; padding row/column zero
-  float* G = W;
-  float* V = W + ne * ld;
-  for (int e = tid; e < ne * ne; e += nt) {
-    const int i = e / ne, j = e % ne;
+  //    W½ R Rᵀ W½ (M < D) or Rᵀ W R
+  float* G = W;              // n x ld; its eigenvectors later overwrite it (V)
+  float* V = W;
+  for (int e = tid; e < n * n; e += nt) {
+    const int i = e / n, j = e % n;
     float acc = 0.f;
-    if (i < n && j < n) {
-      if (small) {
-        for (int d = 0; d < D; ++d) acc = fmaf(rr[i * ldr + d], rr[j * ldr + d], acc);
-        acc *= sqrtf(wv[i] * wv[j]);
-      } else {
-        for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * rr[m * ldr + i], rr[m * ldr + j], acc);
-      }
+    if (small) {
+      for (int d = 0; d < D; ++d) acc = fmaf(rr[i * ldr + d], rr[j * ldr + d], acc);
+      acc *= sqrtf(wv[i] * wv[j]);
+    } else {
+      for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * rr[m * ldr + i], rr[m * ldr + j], acc);
     }
     G[i * ld + j] = acc;
-    V[i * ld + j] = (i == j) ? 1.f : 0.f;
   }
   __syncthreads();
-  // 4. cyclic Jacobi sweeps (circle-method pair order), until the off-diagonal mass is
-  //    below 1e-12 of the total (about the float32 resolution of the squared entries)
-  for (int e = tid; e < (ne - 1) * (ne / 2); e += nt) {
-    int p, q;
-    round_pair(ne, e / (ne / 2), e % (ne / 2), p, q);
-    pairs[e / (ne / 2)][e % (ne / 2)][0] = static_cast<uint8_t>(p);
-    pairs[e / (ne / 2)][e % (ne / 2)][1] = static_cast<uint8_t>(q);
+  // 4-5. the rk largest eigenpairs (Householder tridiagonalisation, bisection, inverse
+  //      iteration); slots past n stay -1 (those directions are left out)
+  {
+    float* hvb = W + n * ld;
+    float* xb = hvb + n * ld;
+    float* wk = xb + n * rk;
+    top_eigenpairs(G, ld, n, rk, hvb, V, evl, xb, wk, red);
+    for (int t = tid; t < 128; t += nt) sel[t] = t < rk && t < n ? t : -1;
+    __syncthreads();
   }
-  __syncthreads();
-  for (int sweep = 0; sweep < 20; ++sweep) {
-    float off = 0.f, tot = 0.f;
-    for (int e = tid; e < ne * ne; e += nt) {
-      const float g = G[(e / ne) * ld + e % ne];
-      tot += g * g;
-      if (e / ne != e % ne) off += g * g;
-    }
-    off = block_sum(off, red);
-    tot = block_sum(tot, red);
-    if (off <= 1e-12f * tot || tot == 0.f) break;
-    for (int r = 0; r < ne - 1; ++r) {
-      if (tid < ne / 2) {
-        const int p = pairs[r][tid][0], q = pairs[r][tid][1];
-        float c = 1.f, s = 0.f;
-        if (q < n) {
-          const float apq = G[p * ld + q];
-          if (apq != 0.f) {
-            const float tau = (G[q * ld + q] - G[p * ld + p]) / (2.f * apq);
-            const float t = copysignf(1.f, tau) / (fabsf(tau) + sqrtf(fmaf(tau, tau, 1.f)));
-            c = rsqrtf(fmaf(t, t, 1.f));
-            s = t * c;
-          }
-        }
-        csn[tid][0] = c;
-        csn[tid][1] = s;
-        cpq[tid][0] = p;
-        cpq[tid][1] = q;
-      }
-      __syncthreads();
-      // G <- Jᵀ G J in one pass: the 2x2 block of rows (p_a, q_a) and columns
-      // (p_b, q_b) becomes J_aᵀ B J_b, J = [[c, s], [-s, c]]; the blocks partition G.
-      // V <- V J on the columns of every pair.
-      const int half = ne / 2;
-      for (int e = tid; e < half * half; e += nt) {
-        const int ia = e / half, ib = e % half;
-        const int pa = cpq[ia][0], qa = cpq[ia][1], pb = cpq[ib][0], qb = cpq[ib][1];
-        const float ca = csn[ia][0], sa = csn[ia][1], cb = csn[ib][0], sb = csn[ib][1];
-        const float b00 = G[pa * ld + pb], b01 = G[pa * ld + qb];
-        const float b10 = G[qa * ld + pb], b11 = G[qa * ld + qb];
-        const float t00 = ca * b00 - sa * b10, t01 = ca * b01 - sa * b11;  // J_aᵀ B
-        const float t10 = sa * b00 + ca * b10, t11 = sa * b01 + ca * b11;
-        G[pa * ld + pb] = cb * t00 - sb * t01;                              // (J_aᵀ B) J_b
-        G[pa * ld + qb] = sb * t00 + cb * t01;
-        G[qa * ld + pb] = cb * t10 - sb * t11;
-        G[qa * ld + qb] = sb * t10 + cb * t11;
-      }
-      for (int e = tid; e < ne * half; e += nt) {
-        const int j = e / half, ib = e % half;
-        const int pb = cpq[ib][0], qb = cpq[ib][1];
-        const float cb = csn[ib][0], sb = csn[ib][1];
-        const float vp = V[j * ld + pb], vq = V[j * ld + qb];
-        V[j * ld + pb] = cb * vp - sb * vq;
-        V[j * ld + qb] = sb * vp + cb * vq;
-      }
-      __syncthreads();
-    }
-  }
-  // 5. the `rk` largest eigenvalues: eigenvalue i takes slot #{j : l_j > l_i, or equal
-  //    with j < i}; slots past n stay -1 (those directions are left out)
-  for (int i = tid; i < n; i += nt) {
-    const float li = G[i * ld + i];
-    int rank = 0;
-    for (int j = 0; j < n; ++j) {
-      const float lj = G[j * ld + j];
-      rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
-    }
-    if (rank < rk) sel[rank] = i;
-  }
-  __syncthreads();
   // 6. V_r (D x rk): eigenvectors of Rᵀ W R, directly (M >= D) or as
   //    (W½ R)ᵀ u / sqrt(l) from those of W½ R Rᵀ W½ (M < D)
-  const float lmax = n > 0 && sel[0] >= 0 ? G[sel[0] * ld + sel[0]] : 0.f;
+  const float lmax = n > 0 && sel[0] >= 0 ? evl[0] : 0.f;
   float* vr = a.vr + bh * D * rk;
   for (int e = tid; e < D * rk; e += nt) {
     const int d = e / rk, k = e % rk;
@@ -309,7 +407,7 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
       if (!small) {
         val = V[d * ld + i];
       } else {
-        const float lam_i = G[i * ld + i];
+        const float lam_i = evl[i];
         if (lam_i > 1e-12f * lmax && lam_i > 0.f) {
           float acc = 0.f;
           for (int m = 0; m < M; ++m) acc = fmaf(sqrtf(wv[m]) * rr[m * ldr + d], V[m * ld + i], acc);
