@@ -338,6 +338,9 @@ struct AttnArgs {
   float* out;
 };
 
+// Chunk records per CTA: at most 2048 token chunks (G <= 4096) plus 128 centroid chunks.
+constexpr int kChunkListCap = 2176;
+
 template <int D, bool TF32>
 struct AttnCfg {
   static constexpr int ESIZE = TF32 ? 4 : 2;
@@ -345,7 +348,7 @@ struct AttnCfg {
   static constexpr int NATOM = D / ATOM;            // 128-byte column chunks per row
   static constexpr int TILE = 128 * D * ESIZE;      // one 128-row operand tile
   static constexpr int KSTEP = 32 / ESIZE;          // K of one MMA instruction
-  static constexpr int MISC = 6144;
+  static constexpr int MISC = 2048 + kChunkListCap * 4 + 512;  // barriers, bitsets, chunk list
   static constexpr int SMEM = 3 * TILE + MISC + 1024;
   // At least ~100 KB so that at most two CTAs share an SM (two 256-column TMEM
   // allocations fill the 512 columns).
@@ -417,6 +420,125 @@ __device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t*
   return false;
 }
 
+// A CTA's chunk list, built once by one warp: exactly the chunks next_chunk() yields
+// from g_lo with limit g_hi, as 32-bit records (bit 31 centroid, bit 30 uniform, bits
+// 16..19 groups - 1, bits 0..15 first group or centroid chunk index), so that no role
+// re-walks the bitsets per chunk. Groups outside [g_lo, g_hi) count as dropped (a run
+// restarts at g_lo and is cut at g_hi, as in next_chunk). Lane L scans groups
+// [128 L, 128 L + 128); the position inside a run at its first group comes from the
+// trailing kept groups of the lanes before it (whole kept segments add 128 = 0 mod 8).
+// At most 2048 token chunks (runs are separated by a dropped group and G <= 4096) plus
+// 128 centroid chunks.
+__device__ __forceinline__ uint32_t kept_word(const uint32_t* any, int w, int Wg, int g_lo, int g_hi) {
+  if (w < 0 || w >= Wg) return 0u;
+  uint32_t x = any[w];
+  const int lo = g_lo - 32 * w, hi = g_hi - 32 * w;  // keep bits [lo, hi)
+  if (hi <= 0 || lo >= 32) return 0u;
+  if (hi < 32) x &= (1u << hi) - 1u;
+  if (lo > 0) x &= ~((1u << lo) - 1u);
+  return x;
+}
+
+__device__ int build_chunk_list(const uint32_t* any, const uint32_t* uni, int g_lo, int g_hi,
+                                int Wg, const uint32_t* cneed, int ncc, uint32_t* list, int lane) {
+  const int seg0 = 128 * lane;
+  int tail = 0;  // trailing kept groups of this lane's segment
+  for (int w = 4 * lane + 3; w >= 4 * lane; --w) {
+    const uint32_t x = kept_word(any, w, Wg, g_lo, g_hi);
+    if (x == 0xffffffffu) {
+      tail += 32;
+      continue;
+    }
+    tail += __clz(~x);
+    break;
+  }
+  const unsigned nonfull = __ballot_sync(0xffffffffu, tail < 128);
+  const int tail_prev = __shfl_up_sync(0xffffffffu, tail, 1);
+  const unsigned before = nonfull & ((1u << lane) - 1u);
+  const int src = before ? 31 - __clz(before) : 0;
+  const int tail_src = __shfl_sync(0xffffffffu, tail, src);
+  // groups of the run before this segment's first group, mod 8
+  const int r0 = (lane > 0 && tail_prev > 0) ? ((before ? tail_src : 0) & 7) : 0;
+  const int seg_end = min(seg0 + 128, g_hi);
+  auto run_from = [&](int g) -> int {  // consecutive kept groups from g, at most 8
+    const int w = g >> 5, sh = g & 31;
+    const uint64_t win = ((static_cast<uint64_t>(kept_word(any, w + 1, Wg, g_lo, g_hi)) << 32) |
+                          kept_word(any, w, Wg, g_lo, g_hi)) >> sh;
+    const int run = __ffsll(static_cast<long long>(~win)) - 1;
+    return (run < 0 || run > 8) ? 8 : run;
+  };
+  int total = 0, base = 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    int g = seg0, r = r0, k = 0;
+    while (g < seg_end) {
+      const int w = g >> 5;
+      uint32_t x = kept_word(any, w, Wg, g_lo, g_hi) & (0xffffffffu << (g & 31));
+      if (!(x & (1u << (g & 31)))) {
+        int ww = w;  // next kept group inside the segment
+        while (x == 0u && ++ww < 4 * lane + 4) x = kept_word(any, ww, Wg, g_lo, g_hi);
+        if (x == 0u) break;
+        g = 32 * ww + __ffs(x) - 1;
+        r = 0;
+        if (g >= seg_end) break;
+      }
+      const int run = run_from(g);
+      if (r == 0) {
+        if (pass == 1) {
+          const int wu = g >> 5, su = g & 31;
+          const uint64_t uw = ((static_cast<uint64_t>(wu + 1 < Wg ? uni[wu + 1] : 0u) << 32) |
+                               (wu < Wg ? uni[wu] : 0u)) >> su;
+          const uint64_t m = (1ull << run) - 1ull;
+          const uint32_t uniform = (uw & m) == m ? (1u << 30) : 0u;
+          list[base + k] = uniform | (static_cast<uint32_t>(run - 1) << 16) | static_cast<uint32_t>(g);
+        }
+        ++k;
+        g += run;
+      } else {
+        g += min(8 - r, run);
+      }
+      r = 0;
+    }
+    if (pass == 0) {  // exclusive prefix sum of the lanes' counts
+      int incl = k;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      base = incl - k;
+      total = __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  int nc = total;  // centroid chunks after the token chunks, in index order
+  for (int w = 0; w < 4 && 32 * w < ncc; ++w) {
+    uint32_t bits = cneed[w];
+    if (32 * w + 32 > ncc) bits &= (1u << (ncc - 32 * w)) - 1u;
+    if ((bits >> lane) & 1u) list[nc + __popc(bits & ((1u << lane) - 1u))] = 0x80000000u | (32 * w + lane);
+    nc += __popc(bits);
+  }
+  __syncwarp();
+  return nc;
+}
+
+__device__ __forceinline__ Chunk decode_chunk(uint32_t rec) {
+  Chunk c;
+  c.centroid = rec >> 31;
+  if (c.centroid) {
+    c.start = static_cast<int>(rec & 0xffffu) * 128;
+    c.n = 128;
+    c.g0 = c.ng = 0;
+    c.uniform = false;
+  } else {
+    c.g0 = static_cast<int>(rec & 0xffffu);
+    c.ng = static_cast<int>((rec >> 16) & 0xfu) + 1;
+    c.start = c.g0 * 16;
+    c.n = c.ng * 16;
+    c.uniform = (rec >> 30) & 1u;
+  }
+  return c;
+}
+
 // Pairs of every 8 whose exponentials use the FMA-pipe polynomial instead of MUFU ex2.
 // 0: measured fastest in this kernel (the softmax warps are issue-bound, not MUFU-bound).
 constexpr int kPolyPairsOf8 = 0;
@@ -455,6 +577,8 @@ __global__ void __launch_bounds__(160, 2)
   uint32_t* any_bits = reinterpret_cast<uint32_t*>(distinct + 128);  // 128 words
   uint32_t* uni_bits = any_bits + 128;                                // 128 words
   uint32_t* cneed = uni_bits + 128;                                   // 4 words
+  int* nchunks = reinterpret_cast<int*>(cneed + 4);
+  uint32_t* clist = reinterpret_cast<uint32_t*>(smem + 3 * Cfg::TILE + 2048);  // kChunkListCap
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x / a.ksplit, split = blockIdx.x % a.ksplit;
@@ -519,11 +643,17 @@ __global__ void __launch_bounds__(160, 2)
       if (need) atomicOr(&cneed[(w >> 2) >> 5], 1u << ((w >> 2) & 31));
     }
   }
+  __syncthreads();
+  const int ncc = (a.compensate && split == a.ksplit - 1) ? a.Ckpad / 128 : 0;
+  if (warp == 1) {
+    const int n = build_chunk_list(any_bits, uni_bits, g_lo, g_hi, a.Wg, cneed, ncc, clist, lane);
+    if (lane == 0) *nchunks = n;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int ncc = (a.compensate && split == a.ksplit - 1) ? a.Ckpad / 128 : 0;
+  const int nch = *nchunks;
 
   if (warp == 0) {
     // ------------------------------------------------ control warp: TMA + tcgen05.mma
@@ -564,9 +694,14 @@ __global__ void __launch_bounds__(160, 2)
       }
       __syncwarp();
     };
-    int gcur = g_lo, ccur = 0, j = 0, nk = 0, nv = 0;
+    int ci = 0, j = 0, nk = 0, nv = 0;
+    auto next = [&](Chunk& c) -> bool {
+      if (ci >= nch) return false;
+      c = decode_chunk(clist[ci++]);
+      return true;
+    };
     Chunk cur, nxt, nn;
-    bool have = next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, cur);
+    bool have = next(cur);
     if (leader) {
       mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
 #pragma unroll
@@ -628,7 +763,7 @@ __global__ void __launch_bounds__(160, 2)
           commit(BAR(BAR_SFHI));
         }
         commit(BAR(BAR_KE));
-        have_next = next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, nxt);
+        have_next = next(nxt);
         if (have_next && (ok = wait_all(BAR(BAR_KE), 0, 1))) {
           load_kv(nxt, false);
           ++nk;
@@ -673,7 +808,7 @@ __global__ void __launch_bounds__(160, 2)
         load_kv(nxt, true);
         ++nv;
         // K stage: refill with the chunk after once QK(j+1) has read it
-        have_nn = next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, nn);
+        have_nn = next(nn);
         if (have_nn) {
           if (!(ok = wait_all(BAR(BAR_KE), (j + 1) & 1, 1))) break;
           load_kv(nn, false);
@@ -709,26 +844,46 @@ __global__ void __launch_bounds__(160, 2)
     const uint32_t tO = tS + 128;
     const float scl = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    int gcur = g_lo, ccur = 0, j = 0, hi_n = 0;  // hi_n: high steps taken so far
+    int j = 0, hi_n = 0;  // hi_n: high steps taken so far
     bool ok = true;
-    Chunk ch;
-    while (next_chunk(gcur, ccur, any_bits, uni_bits, g_hi, a.Wg, cneed, ncc, ch)) {
+#pragma unroll 1
+    for (int ci = 0; ci < nch; ++ci) {
+      const Chunk ch = decode_chunk(clist[ci]);
       const int nsteps = ch.n > 64 ? 2 : 1;
+      // Token chunks are masked per 16-key group (a key cluster is kept or dropped
+      // whole): this row's keep bits for the chunk's groups, the groups holding pad
+      // slots, and the warp's votes (whether no row, every row or some rows keep each
+      // group). None of it depends on S, so it is read before S is ready.
+      uint32_t kb8 = 0u, part8 = 0u, any8 = 0xffu, mixed8 = 0u;
+      if (!ch.centroid) {
+        const uint32_t present = (1u << ch.ng) - 1u;
+        kb8 = present;
+        if (!ch.uniform) {
+          const int w = ch.g0 >> 5, sh = ch.g0 & 31;
+          const bool two = w + 1 < a.Wg;
+          const uint64_t kw = static_cast<uint64_t>(__ldg(grow + w)) |
+                              (two ? static_cast<uint64_t>(__ldg(grow + w + 1)) << 32 : 0ull);
+          const uint64_t fw = static_cast<uint64_t>(__ldg(a.gfull + w)) |
+                              (two ? static_cast<uint64_t>(__ldg(a.gfull + w + 1)) << 32 : 0ull);
+          kb8 = static_cast<uint32_t>(kw >> sh) & present;
+          part8 = ~static_cast<uint32_t>(fw >> sh) & present;
+        }
+        if (lab < 0) kb8 = 0u;
+        any8 = __reduce_or_sync(0xffffffffu, kb8);
+        mixed8 = any8 & ~__reduce_and_sync(0xffffffffu, kb8);
+      }
 #pragma unroll 1
       for (int half = 0; half < nsteps; ++half) {
         const int c0 = half * 64;         // first key column of this step
-        const int nmine = ch.n - c0;      // key columns of the chunk in this step
         {
           if (!(ok = mbar_wait(BAR(half == 0 ? BAR_SFLO : BAR_SFHI), half == 0 ? (j & 1) : (hi_n & 1),
                                abort_flag, 9)))
             break;
           tc_fence_after();
-          // Token chunks are masked per 16-key group (a key cluster is kept or dropped
-          // whole): a warp vote tells, per group, whether no row, every row or only some
-          // rows of the warp keep it. Groups no row keeps get P = 0 without exponentials,
-          // groups every row keeps need no select. Columns past a cluster's last token
-          // (pad slots of its last group) and pad query rows are set to -inf.
-          // Centroid chunks are masked per column and carry the log2 n_c bias.
+          // Groups no row of the warp keeps get P = 0 without exponentials, groups every
+          // row keeps need no select. Columns past a cluster's last token (pad slots of
+          // its last group) and pad query rows are set to -inf. Centroid chunks are
+          // masked per column and carry the log2 n_c bias.
           float v0[32], v1[32];
           tmem_ld32(tS + c0, v0);
           tmem_ld32(tS + c0 + 32, v1);
@@ -736,23 +891,11 @@ __global__ void __launch_bounds__(160, 2)
           float mx;
           float sx = scl;        // exponent argument x = v * sx - m
           if (!ch.centroid) {
-            const int ngs = nmine >= 64 ? 4 : (nmine >> 4);
-            const uint32_t present = (1u << ngs) - 1u;
             const int gh0 = ch.g0 + half * 4;  // this step covers groups gh0 .. gh0+3
-            uint32_t kb = present, partial = 0u;
-            if (!ch.uniform) {
-              const int w = gh0 >> 5, sh = gh0 & 31;
-              const bool two = w + 1 < a.Wg;
-              const uint64_t kw = static_cast<uint64_t>(__ldg(grow + w)) |
-                                  (two ? static_cast<uint64_t>(__ldg(grow + w + 1)) << 32 : 0ull);
-              const uint64_t fw = static_cast<uint64_t>(__ldg(a.gfull + w)) |
-                                  (two ? static_cast<uint64_t>(__ldg(a.gfull + w + 1)) << 32 : 0ull);
-              kb = static_cast<uint32_t>(kw >> sh) & present;
-              partial = ~static_cast<uint32_t>(fw >> sh) & present;
-            }
-            if (lab < 0) kb = 0u;
-            any4 = __reduce_or_sync(0xffffffffu, kb);
-            const uint32_t mixed = any4 & ~__reduce_and_sync(0xffffffffu, kb);
+            const uint32_t kb = (kb8 >> (4 * half)) & 0xfu;
+            const uint32_t partial = (part8 >> (4 * half)) & 0xfu;
+            const uint32_t mixed = (mixed8 >> (4 * half)) & 0xfu;
+            any4 = (any8 >> (4 * half)) & 0xfu;
             tmem_wait_ld();
             if (partial | mixed) {
               // -inf for the pad slots of a cluster's last group, and for rows that drop

@@ -139,3 +139,55 @@ def test_video_static_tiles_full_size_sampled():
     rows = np.random.default_rng(12).choice(32760, 96, replace=False)
     ref = _ref(q, k, v, lab_ref, lab_ref, mask, C, C, rows=rows)
     _check(got[:, :, rows], ref)
+
+
+# Calls with at least 148 query-tile CTAs over all heads run without a key-range split
+# (one CTA walks every kept key of its tile); the cases below reach that path with short
+# sequences and many heads.
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_unsplit_ragged_gqa(D):
+    """S = 1100 (9 query tiles, the last one ragged), shuffled uneven clusters
+    (sizes not multiples of 16), an empty key cluster, Cq != Ck, per-head masks at
+    ~30 %, GQA 40:20; compensated and hard drop."""
+    g = np.random.default_rng(21)
+    S, Cq, Ck, H, Hkv = 1100, 13, 17, 40, 20
+    ql = g.permutation(np.concatenate([np.arange(Cq), g.integers(0, Cq, S - Cq)]))
+    kl = g.permutation(np.concatenate([np.arange(Ck - 1), g.integers(0, Ck - 1, S - Ck + 1)]))
+    mask = g.random((H, Cq, Ck)) < 0.3
+    q, k, v = wl.gaussian_qkv(1, H, Hkv, S, D, "bf16", seed=22)
+    rows = np.sort(g.choice(S, 160, replace=False))
+    for comp in (True, False):
+        got = _run(q, k, v, ql, kl, mask, Cq, Ck, comp)
+        _check(got[:, :, rows], _ref(q, k, v, ql, kl, mask, Cq, Ck, comp, rows=rows))
+
+
+def test_unsplit_all_kept_equals_dense():
+    """Every block kept over many 128-key chunks: equals dense attention."""
+    q, k, v = wl.gaussian_qkv(1, 48, 48, 896, 128, "bf16", seed=23)
+    lab = np.arange(896) // 112
+    mask = np.ones((8, 8), dtype=bool)
+    got = _run(q, k, v, lab, lab, mask, 8, 8, True)
+    _check(got, oracle.dense_attention(q.double().numpy(), k.double().numpy(),
+                                       v.double().numpy()))
+
+
+def test_unsplit_large_logit_jumps():
+    """Keys 64..127 of every 128 have 20x larger logits, so the running max jumps by far
+    more than the lazy-rescale threshold between the two halves of a chunk."""
+    g = np.random.default_rng(24)
+    S, H, D = 1024, 40, 64
+    q = torch.tensor(g.standard_normal((1, H, S, D)) * 0.5, dtype=torch.float64)
+    k = torch.tensor(g.standard_normal((1, H, S, D)) * 0.5, dtype=torch.float64)
+    # keys 64..127 of every 128 are 20x larger: the second half of a chunk raises the
+    # max by far more than the lazy-rescale threshold
+    k = k * torch.tensor(1.0 + 19.0 * ((np.arange(S) % 128) >= 64))[None, None, :, None]
+    v = torch.tensor(g.standard_normal((1, H, S, D)), dtype=torch.float64)
+    q, k, v = (x.to(torch.bfloat16) for x in (q, k, v))
+    lab = np.arange(S) // 128
+    mask = np.random.default_rng(25).random((8, 8)) < 0.6
+    np.fill_diagonal(mask, True)
+    for comp in (True, False):
+        got = _run(q, k, v, lab, lab, mask, 8, 8, comp)
+        ref = _ref(q.float(), k.float(), v.float(), lab, lab, mask, 8, 8, comp)
+        _check(got, ref)
