@@ -721,13 +721,15 @@ __global__ void __launch_bounds__(160, 2)
       if (nh > 0) {
         const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(nh >> 3) << 17);
         const uint64_t krow = static_cast<uint64_t>((hlf * 64 * 128) >> 4);  // 64 rows of 128 B
+        // one elected lane issues the half's K-steps back to back
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          if (elect_one())
+          for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
             mma_ss<TF32>(tmem + 64 * hlf, dQ + off, dK + off + krow, idesc, kk > 0 ? 1u : 0u);
-          __syncwarp();
+          }
         }
+        __syncwarp();
       }
     };
     // O += P V for key rows [64h, 64h + n_h); P of step h sits at TMEM columns 64h..
@@ -737,17 +739,17 @@ __global__ void __launch_bounds__(160, 2)
     auto issue_pv_half = [&](const Chunk& c, int hlf, bool first_chunk) {
       constexpr int kHalfSteps = 64 / Cfg::KSTEP;
       const int nsteps = c.n / Cfg::KSTEP;
+      if (elect_one()) {
 #pragma unroll
-      for (int t = 0; t < kHalfSteps; ++t) {
-        const int kk = hlf * kHalfSteps + t;
-        if (kk < nsteps) {
-          if (elect_one())
+        for (int t = 0; t < kHalfSteps; ++t) {
+          const int kk = hlf * kHalfSteps + t;
+          if (kk < nsteps)
             mma_ts<TF32>(tmem + 128, tmem + 64 * hlf + t * 8,
                          dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
                          (!first_chunk || kk > 0) ? 1u : 0u);
-          __syncwarp();
         }
       }
+      __syncwarp();
     };
     bool ok = wait_all(BAR(BAR_Q), 0, 3);
     bool have_next = false, have_nn = false;
