@@ -39,6 +39,7 @@ SIGNATURES = {
     "bsa_last_error_detail": (None, [ctypes.c_char_p, _sz]),
     "bsa_version": (_i, []),
     "bsa_get_device_status": (_i, [_vp, _ip]),
+    "bsa_wait_timeout_selftest": (_i, [ctypes.c_longlong, _vp]),
     "bsa_launch_count": (ctypes.c_longlong, []),
     "bsa_profile_enable": (_i, [_i]),
     "bsa_profile_read": (_i, [_i, ctypes.POINTER(ctypes.c_float), _ip]),

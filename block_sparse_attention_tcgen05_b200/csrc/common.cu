@@ -126,6 +126,23 @@ __global__ void tile_labels_kernel(int T, int H, int W, int tt, int th, int tw, 
   labels[s] = ((t / tt) * nH + h / th) * nW + w / tw;
 }
 
+// One warp waits on an mbarrier that nothing arrives on (expected count 1, no arrival),
+// through the bounded wait every kernel uses; the wait gives up after limit_ns, which
+// records BSA_ERR_TIMEOUT (site 90) in the status word. The barrier then still has its
+// arrival pending; it lives in this CTA's shared memory and ends with it.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1u);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, 90, limit_ns);
+  __syncwarp();
+}
+
 }  // namespace bsa
 
 extern "C" {
@@ -188,6 +205,13 @@ int bsa_profile_read(int kernel, float* total_ms, int* launches) {
   if (total_ms) *total_ms = sum;
   if (launches) *launches = p.used[kernel];
   return BSA_OK;
+}
+
+int bsa_wait_timeout_selftest(long long limit_ns, void* stream) {
+  const long long lim = limit_ns < 1000 ? 1000 : (limit_ns > 2000000000LL ? 2000000000LL : limit_ns);
+  bsa::wait_timeout_selftest_kernel<<<1, 32, 0, bsa::as_stream(stream)>>>(static_cast<uint64_t>(lim));
+  bsa::count_launch();
+  return bsa::check_cuda(cudaGetLastError(), "wait_timeout_selftest_kernel");
 }
 
 int bsa_get_device_status(void* stream, int* where) {

@@ -74,6 +74,17 @@ int bsa_version(void);
  */
 int bsa_get_device_status(void* stream, int* where);
 
+/*
+ * Check of the failure path every kernel's waits share (no counterpart on the pages):
+ * launches one warp that waits, with the same bounded mbarrier wait the kernels use, on
+ * a barrier that nothing ever arrives on. After `limit_ns` nanoseconds of wall time
+ * (clamped to [1 us, 2 s]) the wait gives up, records BSA_ERR_TIMEOUT with site code
+ * 90 in the device status word and the kernel returns normally, leaving the context
+ * usable. Asynchronous on `stream`; read the outcome with bsa_get_device_status().
+ * Returns BSA_ERR_CUDA if the launch fails. Allocates nothing.
+ */
+int bsa_wait_timeout_selftest(long long limit_ns, void* stream);
+
 /* Number of kernel launches the library has made since it was loaded. */
 long long bsa_launch_count(void);
 
