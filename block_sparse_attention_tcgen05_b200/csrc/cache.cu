@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(256) pool_kernel(void* state, const T* __restr
   float a[EPV], c[EPV];
 #pragma unroll
   for (int e = 0; e < EPV; ++e) a[e] = c[e] = 0.f;
+  // four rows per thread in flight: enough outstanding bytes per SM to cover HBM latency
+#pragma unroll 4
   for (int r = r0 + rin; r < r1; r += rpi) {
     const uint4 xq = __ldg(q4 + static_cast<int64_t>(r) * vpr + v);
     const uint4 xk = __ldg(k4 + static_cast<int64_t>(r) * vpr + v);
