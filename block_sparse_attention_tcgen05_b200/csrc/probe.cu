@@ -46,15 +46,55 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return _
 template <>
 __device__ __forceinline__ float to_f<float>(float x) { return x; }
 
+// epl consecutive elements of a row as fp32, read as one vector per lane (epl * sizeof(T)
+// bytes: 4, 8 or 16; rows start on D * sizeof(T) and lanes on epl * sizeof(T) boundaries).
+template <typename T>
+__device__ __forceinline__ void load_lane(const T* p, int epl, float (&x)[4]);
+template <>
+__device__ __forceinline__ void load_lane<__nv_bfloat16>(const __nv_bfloat16* p, int epl, float (&x)[4]) {
+  if (epl == 4) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  } else {
+    const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u));
+    x[0] = a.x; x[1] = a.y; x[2] = x[3] = 0.f;
+  }
+}
+template <>
+__device__ __forceinline__ void load_lane<float>(const float* p, int epl, float (&x)[4]) {
+  if (epl == 4) {
+    const float4 u = __ldg(reinterpret_cast<const float4*>(p));
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+  } else {
+    const float2 u = __ldg(reinterpret_cast<const float2*>(p));
+    x[0] = u.x; x[1] = u.y; x[2] = x[3] = 0.f;
+  }
+}
+
+// (distance, token) order: the smaller distance first, ties to the lower token index.
+__device__ __forceinline__ bool dist_before(float da, int ta, float db, int tb) {
+  return da < db || (da == db && ta < tb);
+}
+
 // grid (C, Hq, B), 256 threads: members of cluster a ordered by the Euclidean distance
-// of q_i to the cluster's mean query (fp32), ties to the lower token index.
+// of q_i to the cluster's mean query (fp32), ties to the lower token index. When fewer
+// probes than non-empty clusters are drawn (M < C'), the selection reads only each
+// cluster's first member, so only that one (the arg-min) is written; otherwise the
+// whole cluster is sorted.
 template <typename T>
 __global__ void __launch_bounds__(256) centroid_order_kernel(
-    const T* __restrict__ q, int S, int D, int H, const int32_t* __restrict__ slot_token,
+    const T* __restrict__ q, int S, int D, int H, int C, int M, const int32_t* __restrict__ slot_token,
     const int32_t* __restrict__ count, const int32_t* __restrict__ off, int32_t* __restrict__ order) {
   __shared__ float mean[128];
   __shared__ float dist[kMaxCentroidCluster];
   __shared__ int tokn[kMaxCentroidCluster];
+  __shared__ float part[8][128];
+  __shared__ int red_n[8];
+  __shared__ float red_d[8];
+  __shared__ int red_t[8];
   const int a = blockIdx.x;
   const int64_t bh = static_cast<int64_t>(blockIdx.z) * H + blockIdx.y;
   const int n = count[a], start = off[a];
@@ -65,23 +105,30 @@ __global__ void __launch_bounds__(256) centroid_order_kernel(
     if (threadIdx.x == 0) report_device_error(kStatusUnsupported, 50);
     return;
   }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  // non-empty clusters C' (the same count the selection makes)
+  int ne = 0;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) ne += count[c] > 0;
+  ne = __reduce_add_sync(0xffffffffu, ne);
+  if (lane == 0) red_n[warp] = ne;
   // Rows are read warp by warp (lane l holds elements [l·D/32, (l+1)·D/32) of a row,
   // so a warp reads whole rows coalesced); warps stride over the members.
   const T* qb = q + bh * S * D;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int epl = D / 32;  // 2 or 4
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int i = warp; i < n; i += nw) {
-    const T* row = qb + static_cast<int64_t>(slot_token[start + i]) * D + lane * epl;
+    float x[4];
+    load_lane<T>(qb + static_cast<int64_t>(slot_token[start + i]) * D + lane * epl, epl, x);
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if (e < epl) acc[e] += to_f(row[e]);
+    for (int e = 0; e < 4; ++e) acc[e] += x[e];
   }
-  __shared__ float part[8][128];
 #pragma unroll
   for (int e = 0; e < 4; ++e)
     if (e < epl) part[warp][lane * epl + e] = acc[e];
   __syncthreads();
+  int cp = 0;
+  for (int w = 0; w < nw; ++w) cp += red_n[w];
+  const bool argmin_only = M < cp;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float t = 0.f;
     for (int w = 0; w < nw; ++w) t += part[w][d];
@@ -90,28 +137,54 @@ __global__ void __launch_bounds__(256) centroid_order_kernel(
   __syncthreads();
   int np = 1;
   while (np < n) np <<= 1;
+  float best_d = INFINITY;
+  int best_t = 0x7fffffff;
   for (int i = warp; i < np; i += nw) {
     if (i < n) {
       const int tok = slot_token[start + i];
-      const T* row = qb + static_cast<int64_t>(tok) * D + lane * epl;
+      float x[4];
+      load_lane<T>(qb + static_cast<int64_t>(tok) * D + lane * epl, epl, x);
       float sq = 0.f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if (e < epl) {
-          const float x = to_f(row[e]) - mean[lane * epl + e];
-          sq = fmaf(x, x, sq);
+          const float y = x[e] - mean[lane * epl + e];
+          sq = fmaf(y, y, sq);
         }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (lane == 0) {
-        dist[i] = sqrtf(sq);
+      const float dd = sqrtf(sq);
+      if (argmin_only) {
+        if (dist_before(dd, tok, best_d, best_t)) {
+          best_d = dd;
+          best_t = tok;
+        }
+      } else if (lane == 0) {
+        dist[i] = dd;
         tokn[i] = tok;
       }
-    } else if (lane == 0) {
+    } else if (!argmin_only && lane == 0) {
       dist[i] = INFINITY;
       tokn[i] = 0x7fffffff;
     }
+  }
+  if (argmin_only) {
+    // every lane of a warp holds the warp's best; then the best of the warps
+    if (lane == 0) {
+      red_d[warp] = best_d;
+      red_t[warp] = best_t;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < nw; ++w)
+        if (dist_before(red_d[w], red_t[w], best_d, best_t)) {
+          best_d = red_d[w];
+          best_t = red_t[w];
+        }
+      order[bh * S + start] = best_t;
+    }
+    return;
   }
   __syncthreads();
   for (int k = 2; k <= np; k <<= 1) {
@@ -122,7 +195,7 @@ __global__ void __launch_bounds__(256) centroid_order_kernel(
           const bool up = (i & k) == 0;
           const float da = dist[i], db = dist[p];
           const int ta = tokn[i], tb = tokn[p];
-          const bool a_first = da < db || (da == db && ta < tb);
+          const bool a_first = dist_before(da, ta, db, tb);
           if (up ? !a_first : a_first) {
             dist[i] = db;
             dist[p] = da;
@@ -278,11 +351,11 @@ extern "C" int bsa_select_probe_rows(const int32_t* labels, int S, int C, int M,
     const dim3 grid(C, shape.Hq, shape.B);
     if (shape.dtype == BSA_BF16)
       centroid_order_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(q), S, shape.D, shape.Hq, L.slot_token, L.count,
+          static_cast<const __nv_bfloat16*>(q), S, shape.D, shape.Hq, C, M, L.slot_token, L.count,
           L.off, L.order);
     else
       centroid_order_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), S,
-                                                          shape.D, shape.Hq, L.slot_token,
+                                                          shape.D, shape.Hq, C, M, L.slot_token,
                                                           L.count, L.off, L.order);
     count_launch();
     if ((rc = check_cuda(cudaGetLastError(), "centroid_order_kernel"))) return rc;

@@ -33,12 +33,14 @@ def test_probe_rows_shared_middle_out():
         np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-6)
 
 
-def test_probe_rows_centroid_distance_per_head():
+@pytest.mark.parametrize("dtype,D", [("bf16", 64), ("bf16", 128), ("f32", 64), ("f32", 128)])
+def test_probe_rows_centroid_distance_per_head(dtype, D):
     """Per (batch, head) nearest-to-mean members. Distances are decided in fp32 on the
     GPU: each chosen row must be in the oracle's cluster and its float64 distance must
-    equal the oracle's choice's distance to 1e-4 (equal up to near-ties)."""
+    equal the oracle's choice's distance to 1e-4 (equal up to near-ties). M=64 over 16
+    clusters takes several members per cluster (full order); M=8 one (nearest only)."""
     bsa = _bsa()
-    q, _, _ = wl.gaussian_qkv(1, 3, 3, 2048, 64, "bf16", seed=1)
+    q, _, _ = wl.gaussian_qkv(1, 3, 3, 2048, D, dtype, seed=1)
     lab = np.arange(2048) // 128
     for M in (64, 8):
         idx, w = bsa.select_probe_rows(torch.as_tensor(lab, dtype=torch.int32).cuda(), 16, M,
