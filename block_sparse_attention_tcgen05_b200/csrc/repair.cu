@@ -11,9 +11,10 @@
 // Per (b, h) with X = out[b,h] (S x D), mu / sigma its column mean and population
 // standard deviation (+1e-6 in the variance), Zt = [(X - mu)/sigma, 1], W = diag(w):
 //   Bc  = (Zt_pᵀ W Zt_p + lam·diag(1,..,1,0))⁻¹ Zt_pᵀ W R      Cholesky in shared memory
-//   V_r = top-r eigenvectors of Rᵀ W R                         cyclic Jacobi (circle-method
-//                                                              pair order) on the smaller
-//                                                              of Rᵀ W R and W½ R Rᵀ W½
+//   V_r = top-r eigenvectors of Rᵀ W R                         Householder tridiagonalisation,
+//                                                              bisection, inverse iteration on
+//                                                              the smaller of Rᵀ W R and
+//                                                              W½ R Rᵀ W½
 //   out += Zt Bc V_r V_rᵀ = (X P' + c') V_rᵀ,  P' = diag(1/sigma) Bc[:D] V_r,
 //          c' = (Bc[D] - Σ_i mu_i/sigma_i Bc[i]) V_r      (rank-r update, one HBM pass)
 #include <cmath>
@@ -571,64 +572,84 @@ __global__ void __launch_bounds__(256) repair_apply_kernel(float* __restrict__ o
   }
 }
 
-// rank <= 16: one row per thread. The thread accumulates y = x P' + c' over its row
-// (each factor row d is one broadcast read of 16 floats, all lanes the same address),
-// then rereads the row (from L1/L2) and writes x + y V_rᵀ. No cross-lane sums; HBM
-// traffic is one read and one write of out. grid (ceil(S / 256), B*H), 256 threads.
+constexpr int kApplyRows = 128;
+constexpr int apply16_smem_bytes(int D) {
+  return static_cast<int>(sizeof(float)) * (2 * D * 16 + kApplyRows * (D + 4) + 16);
+}
+
+// rank <= 16: tiles of 128 rows staged through shared memory, so that every global
+// access is a coalesced 16-byte vector (HBM traffic: one read and one write of out);
+// then one row per thread: y = x P' + c' (each factor row d is a broadcast read of 16
+// floats, all lanes the same address), x += y V_rᵀ (V_rᵀ row k broadcast likewise),
+// pairs of outputs per packed f32x2 FMA. Rows are padded to D + 4 floats, so the eight
+// rows of a quarter-warp fall on distinct 16-byte bank groups. grid (ceil(S / 128),
+// B*H), 128 threads; factors as P'[d][k], V_rᵀ[k][d], zero past `rank`.
 template <int D>
-__global__ void __launch_bounds__(256) repair_apply16_kernel(float* __restrict__ out, int S, int rank,
+__global__ void __launch_bounds__(128) repair_apply16_kernel(float* __restrict__ out, int S, int rank,
                                                              const float* __restrict__ pp,
                                                              const float* __restrict__ cc,
                                                              const float* __restrict__ vr) {
-  __shared__ float4 sP[D][4], sV[D][4];  // factor rows d, ranks 0..15 (zero past `rank`)
-  __shared__ float sc[16];
+  constexpr int TR = kApplyRows, LD = D + 4, V4 = D / 4;
+  extern __shared__ __align__(16) float apply_smem[];  // apply16_smem_bytes(D)
+  float(*sP)[16] = reinterpret_cast<float(*)[16]>(apply_smem);
+  float(*sVt)[D] = reinterpret_cast<float(*)[D]>(apply_smem + D * 16);
+  float* xs = apply_smem + 2 * D * 16;
+  float* sc = xs + TR * LD;
   const int64_t bh = blockIdx.y;
   for (int e = threadIdx.x; e < D * 16; e += blockDim.x) {
     const int d = e / 16, k = e % 16;
     const bool in = k < rank;
-    reinterpret_cast<float*>(sP[d])[k] = in ? pp[(bh * D + d) * rank + k] : 0.f;
-    reinterpret_cast<float*>(sV[d])[k] = in ? vr[(bh * D + d) * rank + k] : 0.f;
+    sP[d][k] = in ? pp[(bh * D + d) * rank + k] : 0.f;
+    sVt[k][d] = in ? vr[(bh * D + d) * rank + k] : 0.f;
   }
   if (threadIdx.x < 16) sc[threadIdx.x] = threadIdx.x < rank ? cc[bh * rank + threadIdx.x] : 0.f;
+  const int r0 = blockIdx.x * TR;
+  const int nr = min(TR, S - r0);
+  const float4* src = reinterpret_cast<const float4*>(out + (bh * S + r0) * D);
+  // fixed trip count: each thread's TR * V4 / 128 loads are in flight together
+#pragma unroll
+  for (int i = 0; i < TR * V4 / 128; ++i) {
+    const int e = threadIdx.x + 128 * i;
+    if (e < nr * V4) *reinterpret_cast<float4*>(&xs[(e / V4) * LD + 4 * (e % V4)]) = __ldg(src + e);
+  }
   __syncthreads();
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= S) return;
-  float4* row = reinterpret_cast<float4*>(out + (bh * S + r) * D);
-  float y[16];
+  if (threadIdx.x < nr) {
+    float* xr = &xs[threadIdx.x * LD];
+    float y[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) y[k] = sc[k];
-#pragma unroll 4
-  for (int d4 = 0; d4 < D / 4; ++d4) {
-    const float4 xv = row[d4];
-    const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int k = 0; k < 16; ++k) y[k] = sc[k];
+#pragma unroll 2
+    for (int d4 = 0; d4 < V4; ++d4) {
+      const float4 x = *reinterpret_cast<const float4*>(xr + 4 * d4);
+      const float xv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 4; ++j) {
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const float4 p = sP[4 * d4 + j][k4];
-        y[4 * k4 + 0] = fmaf(xs[j], p.x, y[4 * k4 + 0]);
-        y[4 * k4 + 1] = fmaf(xs[j], p.y, y[4 * k4 + 1]);
-        y[4 * k4 + 2] = fmaf(xs[j], p.z, y[4 * k4 + 2]);
-        y[4 * k4 + 3] = fmaf(xs[j], p.w, y[4 * k4 + 3]);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const float4 p = *reinterpret_cast<const float4*>(&sP[4 * d4 + j][4 * k4]);
+          fma2(y[4 * k4], y[4 * k4 + 1], xv[j], xv[j], p.x, p.y, y[4 * k4], y[4 * k4 + 1]);
+          fma2(y[4 * k4 + 2], y[4 * k4 + 3], xv[j], xv[j], p.z, p.w, y[4 * k4 + 2], y[4 * k4 + 3]);
+        }
       }
+    }
+#pragma unroll 2
+    for (int c4 = 0; c4 < V4; ++c4) {
+      float4 x = *reinterpret_cast<const float4*>(xr + 4 * c4);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float4 v = *reinterpret_cast<const float4*>(&sVt[k][4 * c4]);
+        fma2(x.x, x.y, y[k], y[k], v.x, v.y, x.x, x.y);
+        fma2(x.z, x.w, y[k], y[k], v.z, v.w, x.z, x.w);
+      }
+      *reinterpret_cast<float4*>(xr + 4 * c4) = x;
     }
   }
-#pragma unroll 4
-  for (int d4 = 0; d4 < D / 4; ++d4) {
-    float4 xv = row[d4];
-    float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+  __syncthreads();
+  float4* dst = reinterpret_cast<float4*>(out + (bh * S + r0) * D);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const float4 v = sV[4 * d4 + j][k4];
-        xs[j] = fmaf(y[4 * k4 + 0], v.x, xs[j]);
-        xs[j] = fmaf(y[4 * k4 + 1], v.y, xs[j]);
-        xs[j] = fmaf(y[4 * k4 + 2], v.z, xs[j]);
-        xs[j] = fmaf(y[4 * k4 + 3], v.w, xs[j]);
-      }
-    }
-    row[d4] = make_float4(xs[0], xs[1], xs[2], xs[3]);
+  for (int i = 0; i < TR * V4 / 128; ++i) {
+    const int e = threadIdx.x + 128 * i;
+    if (e < nr * V4) dst[e] = *reinterpret_cast<const float4*>(&xs[(e / V4) * LD + 4 * (e % V4)]);
   }
 }
 
@@ -692,7 +713,11 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
   if ((rc = check_cuda(cudaGetLastError(), "repair_fit_kernel"))) return rc;
   if (rank <= 16) {
     auto ap16 = D == 64 ? repair_apply16_kernel<64> : repair_apply16_kernel<128>;
-    ap16<<<dim3((S + 255) / 256, BH), 256, 0, st>>>(out, S, rank, L.pp, L.cc, L.vr);
+    const int smem16 = apply16_smem_bytes(D);
+    e = cudaFuncSetAttribute(ap16, cudaFuncAttributeMaxDynamicSharedMemorySize, smem16);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(repair_apply16)");
+    ap16<<<dim3((S + kApplyRows - 1) / kApplyRows, BH), kApplyRows, smem16, st>>>(out, S, rank, L.pp,
+                                                                                 L.cc, L.vr);
     count_launch();
     return check_cuda(cudaGetLastError(), "repair_apply16_kernel");
   }
