@@ -97,15 +97,17 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // memory), all threads of the CTA taking part:
 //  1. Householder reduction to tridiagonal form T = Hᵀ A H (reflector k in hv row k,
 //     A overwritten), diag d, off-diagonal e;
-//  2. the k largest eigenvalues of T by bisection on Sturm counts (one thread each);
-//  3. their eigenvectors by inverse iteration on T (one thread each), then modified
-//     Gram-Schmidt in order of decreasing eigenvalue;
+//  2. the k largest eigenvalues of T by multisection on Sturm counts (one warp each:
+//     32 points per round split the bracket into 33 parts);
+//  3. their eigenvectors by inverse iteration on T (one thread each), then Gram-Schmidt
+//     in order of decreasing eigenvalue (classical, applied twice, all warps);
 //  4. back-transformation by the reflectors: U = H x.
 // Output: U (n x min(k, n), row stride ld >= n) and lam[0..k) in decreasing order
 // (zero past n). hv needs n x ld floats, x n x k, work 5n + k n floats.
 __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float* U, float* lam,
                                float* x, float* work, float* red) {
   const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
   float* d = work;
   float* e = work + n;        // e[i] couples i and i+1
   float* pv = work + 2 * n;   // A v
@@ -133,11 +135,14 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
     }
     __syncthreads();
     if (!skip) {
-      // p = A' v over the trailing block A' = A[c+1.., c+1..]
-      for (int i = tid; i < m; i += nt) {
+      // p = A' v over the trailing block A' = A[c+1.., c+1..]: a warp per row, lanes
+      // along it, shuffle sums
+      for (int i = wid; i < m; i += nw) {
         float acc = 0.f;
-        for (int j = 0; j < m; ++j) acc = fmaf(A[(c + 1 + i) * ld + c + 1 + j], hv[c * ld + j], acc);
-        pv[i] = acc;
+        for (int j = lane; j < m; j += 32) acc = fmaf(A[(c + 1 + i) * ld + c + 1 + j], hv[c * ld + j], acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) pv[i] = acc;
       }
       __syncthreads();
       float kk = 0.f;
@@ -162,8 +167,9 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
     if (n >= 2) e[n - 2] = A[(n - 1) * ld + (n - 2)];
   }
   __syncthreads();
-  // 2. bisection: eigenvalue j (ascending) of T is the x where the Sturm count
-  //    #{eigenvalues < x} passes j; thread t takes the t-th largest, j = n - 1 - t
+  // 2. multisection: eigenvalue j (ascending) of T is the x where the Sturm count
+  //    #{eigenvalues < x} passes j; warp w takes the w-th largest (then w + nw, ...),
+  //    j = n - 1 - t
   float* e2 = work + 4 * n;
   for (int i = tid; i < n; i += nt) e2[i] = i + 1 < n ? e[i] * e[i] : 0.f;
   if (tid == 0) {
@@ -182,24 +188,33 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
   const int kk = k < n ? k : n;
   const float lo0 = s_scal[0], hi0 = s_scal[1];
   const float pivmin = 1e-30f + 1e-12f * (hi0 - lo0) * (hi0 - lo0);
-  if (tid < kk) {
-    const int j = n - 1 - tid;
+  for (int t = wid; t < kk; t += nw) {
+    const int j = n - 1 - t;
     float a = lo0, b = hi0;
-    for (int it = 0; it < 60; ++it) {
-      const float mid = 0.5f * (a + b);
-      if (!(mid > a && mid < b)) break;  // float resolution reached
+    for (int it = 0; it < 40; ++it) {
+      // lane l evaluates the count at the (l+1)-th of 32 interior points of [a, b]
+      const float xl = a + (b - a) * (static_cast<float>(lane + 1) * (1.f / 33.f));
       int cnt = 0;
-      float q = d[0] - mid;
+      float q = d[0] - xl;
       for (int i = 0;; ++i) {
         if (fabsf(q) < pivmin) q = -pivmin;
         cnt += q < 0.f;
         if (i + 1 >= n) break;
-        q = d[i + 1] - mid - __fdividef(e2[i], q);
+        q = d[i + 1] - xl - __fdividef(e2[i], q);
       }
-      if (cnt > j) b = mid;
-      else a = mid;
+      // the first point whose count exceeds j closes the new bracket, the point before
+      // it opens it (a and b when there is none)
+      const unsigned above = __ballot_sync(0xffffffffu, cnt > j);
+      const int p = above ? __ffs(above) - 1 : 32;
+      const float xa = __shfl_sync(0xffffffffu, xl, p > 0 ? p - 1 : 0);
+      const float xb = __shfl_sync(0xffffffffu, xl, p < 32 ? p : 31);
+      const float na = p > 0 ? fmaxf(xa, a) : a;
+      const float nb = p < 32 ? fminf(xb, b) : b;
+      if (!(nb - na < b - a)) break;  // float resolution reached
+      a = na;
+      b = nb;
     }
-    lam[tid] = 0.5f * (a + b);
+    if (lane == 0) lam[t] = 0.5f * (a + b);
   }
   __syncthreads();
   // 3. inverse iteration: solve (T - lam I) y = x by elimination with guarded pivots
@@ -234,28 +249,34 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
     }
   }
   __syncthreads();
-  //    modified Gram-Schmidt (warp 0) in order of decreasing eigenvalue: repairs the
-  //    loss of orthogonality of inverse iteration within clusters of eigenvalues
-  if (tid < 32) {
-    for (int t = 0; t < kk; ++t) {
-      for (int s = 0; s < t; ++s) {
+  //    Gram-Schmidt in order of decreasing eigenvalue, classical and applied twice: the
+  //    projections of vector t on the vectors before it are taken together (a warp per
+  //    projection); repairs the loss of orthogonality of inverse iteration within
+  //    clusters of eigenvalues
+  for (int t = 0; t < kk; ++t) {
+    for (int pass = 0; pass < 2; ++pass) {
+      for (int s2 = wid; s2 < t; s2 += nw) {
         float dot = 0.f;
-        for (int i = tid; i < n; i += 32) dot = fmaf(x[i * k + s], x[i * k + t], dot);
+        for (int i = lane; i < n; i += 32) dot = fmaf(x[i * k + s2], x[i * k + t], dot);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        for (int i = tid; i < n; i += 32) x[i * k + t] -= dot * x[i * k + s];
-        __syncwarp();
+        if (lane == 0) pv[s2] = dot;
       }
-      float nrm = 0.f;
-      for (int i = tid; i < n; i += 32) nrm = fmaf(x[i * k + t], x[i * k + t], nrm);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xffffffffu, nrm, o);
-      const float rn = nrm > 0.f ? rsqrtf(nrm) : 0.f;
-      for (int i = tid; i < n; i += 32) x[i * k + t] *= rn;
-      __syncwarp();
+      __syncthreads();
+      for (int i = tid; i < n; i += nt) {
+        float v = x[i * k + t];
+        for (int s2 = 0; s2 < t; ++s2) v = fmaf(-pv[s2], x[i * k + s2], v);
+        x[i * k + t] = v;
+      }
+      __syncthreads();
     }
+    float nrm = 0.f;
+    for (int i = tid; i < n; i += nt) nrm = fmaf(x[i * k + t], x[i * k + t], nrm);
+    nrm = block_sum(nrm, red);
+    const float rn = nrm > 0.f ? rsqrtf(nrm) : 0.f;
+    for (int i = tid; i < n; i += nt) x[i * k + t] *= rn;
+    __syncthreads();
   }
-  __syncthreads();
   // 4. back-transformation: x <- H_c x for c = n-3 .. 0, H_c = I - 2 v_c v_cᵀ on rows c+1..
   for (int c = n - 3; c >= 0; --c) {
     const int m = n - c - 1;
@@ -279,12 +300,54 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
   __syncthreads();
 }
 
+// Solves A X = B in place for SPD A (n x n, row stride n) and B (n x nr): Cholesky
+// without the column scaling (after step k the lower triangle holds A[i][k] = L[i][k]·s_k
+// with s_k = L[k][k] = sqrt(A[k][k]); one barrier per step), then right-looking
+// forward and backward substitution. rpiv (n floats) receives 1 / s_k. All threads of
+// the CTA take part.
+__device__ void chol_solve(float* A, int n, float* B, int nr, float* rpiv) {
+  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
+  for (int k = 0; k < n; ++k) {
+    const float rdk = 1.f / fmaxf(A[k * n + k], 1e-30f);
+    for (int i = k + 1 + wid; i < n; i += nw) {  // warps along rows, lanes along columns
+      const float aik = A[i * n + k] * rdk;
+      for (int j = k + 1 + lane; j <= i; j += 32) A[i * n + j] -= aik * A[j * n + k];
+    }
+    __syncthreads();
+  }
+  for (int k = tid; k < n; k += nt) rpiv[k] = 1.f / sqrtf(fmaxf(A[k * n + k], 1e-30f));
+  __syncthreads();
+  // forward  b_i -= (A[i][k] / s_k) (b_k / s_k), i > k;  then y_k = b_k / s_k
+  for (int k = 0; k < n - 1; ++k) {
+    const float r2 = rpiv[k] * rpiv[k];
+    for (int e = tid; e < (n - 1 - k) * nr; e += nt) {
+      const int i = k + 1 + e / nr, c = e % nr;
+      B[i * nr + c] -= A[i * n + k] * B[k * nr + c] * r2;
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < n * nr; e += nt) B[e] *= rpiv[e / nr];
+  __syncthreads();
+  // backward y_i -= (A[k][i] / s_i) (y_k / s_k), i < k;  then x_k = y_k / s_k
+  for (int k = n - 1; k > 0; --k) {
+    const float rk_ = rpiv[k];
+    for (int e = tid; e < k * nr; e += nt) {
+      const int i = e / nr, c = e % nr;
+      B[i * nr + c] -= A[k * n + i] * rpiv[i] * B[k * nr + c] * rk_;
+    }
+    __syncthreads();
+  }
+  for (int e = tid; e < n * nr; e += nt) B[e] *= rpiv[e / nr];
+  __syncthreads();
+}
+
 // Shared-memory plan of the fit, in floats: the standardised probe rows Zt (M x ldz)
 // and residuals R (M x ldr) and R V_r (M x rk) when they fit (else they stay in the
 // workspace), a region W used first by the eigen step (the Gram matrix, later its
 // eigenvectors, n x ld; the reflectors n x ld; inverse-iteration vectors n x rk and
-// scratch) and then by the solve (A: n1 x n1, right-hand sides n1 x rk), V_r (D x rk)
-// and the Cholesky pivots.
+// scratch) and then by the solve (primal: A n1 x n1 and right-hand sides n1 x rk; dual:
+// K M x M, right-hand sides M x rk and the solution n1 x rk), V_r (D x rk) and the
+// Cholesky pivots.
 struct FitPlan {
   int n1, n, ld, ldz, ldr, rk;
   bool local_zr;                   // Zt, R, R V_r in shared memory
@@ -301,7 +364,11 @@ __host__ __device__ inline FitPlan fit_plan(int D, int M, int rk) {
   p.rk = rk;
   const size_t wa = static_cast<size_t>(2) * p.n * p.ld + static_cast<size_t>(2) * p.n * rk +
                     static_cast<size_t>(5) * p.n;
-  const size_t wb = static_cast<size_t>(p.n1) * p.n1 + static_cast<size_t>(p.n1) * rk;
+  const size_t wb_primal = static_cast<size_t>(p.n1) * p.n1 + static_cast<size_t>(p.n1) * rk;
+  const size_t wb_dual = M < p.n1 ? static_cast<size_t>(M) * M + static_cast<size_t>(M) * rk +
+                                        static_cast<size_t>(p.n1) * rk
+                                  : 0;
+  const size_t wb = wb_primal > wb_dual ? wb_primal : wb_dual;
   const size_t wsz = wa > wb ? wa : wb;
   const size_t common = wsz + static_cast<size_t>(D) * rk + p.n1;
   const size_t zr = static_cast<size_t>(M) * (p.ldz + p.ldr + rk);
@@ -328,6 +395,7 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   __shared__ float wv[1024];
   __shared__ int sel[128];
   __shared__ float evl[128];  // eigenvalues of the residual Gram matrix, decreasing
+  __shared__ float zbar[128], tbar[128];  // weighted probe means of Z and R V_r (dual solve)
   const int tid = threadIdx.x, nt = blockDim.x;
   const int64_t bh = blockIdx.x;
   const int S = a.S, D = a.D, M = a.M, rk = a.rank;
@@ -428,70 +496,125 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
     rv[e] = acc;
   }
   __syncthreads();
-  // 8. normal equations, projected: A = Ztᵀ W Zt + lam·I' (intercept unpenalised) and
-  //    B = Ztᵀ W (R V_r), so that A⁻¹ B = Bc V_r
-  float* A = W;              // n1 x n1 (overwrites G, V: no longer needed)
-  float* Bm = W + n1 * n1;   // n1 x rk
-  for (int e = tid; e < n1 * n1; e += nt) {
-    const int i = e / n1, j = e % n1;
-    if (j > i) continue;
-    float acc = 0.f;
-    for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * zt[m * ldz + i], zt[m * ldz + j], acc);
-    if (i == j && i < D) acc += a.lam;
-    A[i * n1 + j] = acc;
-    A[j * n1 + i] = acc;
-  }
-  for (int e = tid; e < n1 * rk; e += nt) {
-    const int i = e / rk, k = e % rk;
-    float acc = 0.f;
-    for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * zt[m * ldz + i], rv[m * rk + k], acc);
-    Bm[e] = acc;
-  }
-  __syncthreads();
-  // 9. Cholesky without the column scaling: after step k the lower triangle holds
-  //    A[i][k] = L[i][k]·s_k with s_k = L[k][k] = sqrt(A[k][k]); one barrier per step
-  const int lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
-  for (int k = 0; k < n1; ++k) {
-    const float rdk = 1.f / fmaxf(A[k * n1 + k], 1e-30f);
-    for (int i = k + 1 + wid; i < n1; i += nw) {  // warps along rows, lanes along columns
-      const float aik = A[i * n1 + k] * rdk;
-      for (int j = k + 1 + lane; j <= i; j += 32) A[i * n1 + j] -= aik * A[j * n1 + k];
+  // 8-10. X = Bc V_r ((D+1) x rk), the ridge solution for the targets T = R V_r:
+  //   primal (M >= D+1): A X = B with A = Ztᵀ W Zt + lam·I' (intercept unpenalised) and
+  //     B = Ztᵀ W T, by Cholesky (D+1 steps);
+  //   dual (M < D+1, the same solution through M x M): the unpenalised intercept is
+  //     taken out by weighted centring (zbar, Tbar: weighted means over the probes), then
+  //     beta = Ucᵀ (Uc Ucᵀ + lam I)⁻¹ W½ T_c with Uc = W½ (Z - 1 zbarᵀ) (push-through
+  //     identity), and the intercept row Tbar - zbarᵀ beta.
+  float* Xs;
+  if (M < n1) {
+    float* Kd = W;               // M x M
+    float* Yd = Kd + M * M;      // M x rk: W½ T_c, then the dual solution
+    Xs = Yd + M * rk;            // (D+1) x rk
+    float sw = 0.f;
+    for (int m = tid; m < M; m += nt) sw += wv[m];
+    sw = block_sum(sw, red);
+    const float isw = sw > 0.f ? 1.f / sw : 0.f;
+    for (int d = tid; d < D; d += nt) {
+      float acc = 0.f;
+      for (int m = 0; m < M; ++m) acc = fmaf(wv[m], zt[m * ldz + d], acc);
+      zbar[d] = acc * isw;
+    }
+    for (int k = tid; k < rk; k += nt) {
+      float acc = 0.f;
+      for (int m = 0; m < M; ++m) acc = fmaf(wv[m], rv[m * rk + k], acc);
+      tbar[k] = acc * isw;
     }
     __syncthreads();
-  }
-  float* rpiv = piv;  // 1 / s_k
-  for (int k = tid; k < n1; k += nt) rpiv[k] = 1.f / sqrtf(fmaxf(A[k * n1 + k], 1e-30f));
-  __syncthreads();
-  // 10. solve L Lᵀ X = B in place, right-looking, one barrier per step:
-  //     forward  b_i -= (A[i][k] / s_k) (b_k / s_k), i > k;  then y_k = b_k / s_k
-  for (int k = 0; k < n1 - 1; ++k) {
-    const float r2 = rpiv[k] * rpiv[k];
-    for (int e = tid; e < (n1 - 1 - k) * rk; e += nt) {
-      const int i = k + 1 + e / rk, c = e % rk;
-      Bm[i * rk + c] -= A[i * n1 + k] * Bm[k * rk + c] * r2;
+    for (int e = tid; e < M * D; e += nt) {  // Uc in place of the probe rows of Z
+      const int m = e / D, d = e % D;
+      zt[m * ldz + d] = sqrtf(wv[m]) * (zt[m * ldz + d] - zbar[d]);
+    }
+    for (int e = tid; e < M * rk; e += nt) {
+      const int m = e / rk, k = e % rk;
+      Yd[e] = sqrtf(wv[m]) * (rv[e] - tbar[k]);
     }
     __syncthreads();
-  }
-  for (int e = tid; e < n1 * rk; e += nt) Bm[e] *= rpiv[e / rk];
-  __syncthreads();
-  //     backward y_i -= (A[k][i] / s_i) (y_k / s_k), i < k;  then x_k = y_k / s_k
-  for (int k = n1 - 1; k > 0; --k) {
-    const float rk_ = rpiv[k];
-    for (int e = tid; e < k * rk; e += nt) {
-      const int i = e / rk, c = e % rk;
-      Bm[i * rk + c] -= A[k * n1 + i] * rpiv[i] * Bm[k * rk + c] * rk_;
+    {
+      // K = Uc Ucᵀ + lam I: a warp per row i, lanes along the columns j <= i (M <= 128)
+      const int ln = tid & 31, wd = tid >> 5, nwd = nt >> 5;
+      for (int i = wd; i < M; i += nwd) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int d = 0; d < D; ++d) {
+          const float u = zt[i * ldz + d];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int j = ln + 32 * c;
+            if (j <= i) acc[c] = fmaf(u, zt[j * ldz + d], acc[c]);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int j = ln + 32 * c;
+          if (j <= i) {
+            const float v = acc[c] + (i == j ? a.lam : 0.f);
+            Kd[i * M + j] = v;
+            Kd[j * M + i] = v;
+          }
+        }
+      }
     }
     __syncthreads();
+    chol_solve(Kd, M, Yd, rk, piv);
+    for (int e = tid; e < D * rk; e += nt) {  // beta = Ucᵀ Y
+      const int d = e / rk, k = e % rk;
+      float acc = 0.f;
+      for (int m = 0; m < M; ++m) acc = fmaf(zt[m * ldz + d], Yd[m * rk + k], acc);
+      Xs[e] = acc;
+    }
+    __syncthreads();
+    for (int k = tid; k < rk; k += nt) {  // intercept row
+      float acc = tbar[k];
+      for (int d = 0; d < D; ++d) acc = fmaf(-zbar[d], Xs[d * rk + k], acc);
+      Xs[D * rk + k] = acc;
+    }
+    __syncthreads();
+  } else {
+    float* A = W;              // n1 x n1 (overwrites G, V: no longer needed)
+    float* Bm = W + n1 * n1;   // n1 x rk
+    Xs = Bm;
+    {
+      // a warp per row i, lanes along the columns j <= i (at most 5 per lane: n1 <= 129)
+      const int lane8 = tid & 31, wid8 = tid >> 5, nw8 = nt >> 5;
+      for (int i = wid8; i < n1; i += nw8) {
+        float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int m = 0; m < M; ++m) {
+          const float wz = wv[m] * zt[m * ldz + i];
+#pragma unroll
+          for (int c = 0; c < 5; ++c) {
+            const int j = lane8 + 32 * c;
+            if (j <= i) acc[c] = fmaf(wz, zt[m * ldz + j], acc[c]);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 5; ++c) {
+          const int j = lane8 + 32 * c;
+          if (j <= i) {
+            const float v = acc[c] + ((i == j && i < D) ? a.lam : 0.f);
+            A[i * n1 + j] = v;
+            A[j * n1 + i] = v;
+          }
+        }
+      }
+    }
+    for (int e = tid; e < n1 * rk; e += nt) {
+      const int i = e / rk, k = e % rk;
+      float acc = 0.f;
+      for (int m = 0; m < M; ++m) acc = fmaf(wv[m] * zt[m * ldz + i], rv[m * rk + k], acc);
+      Bm[e] = acc;
+    }
+    __syncthreads();
+    chol_solve(A, n1, Bm, rk, piv);
   }
-  for (int e = tid; e < n1 * rk; e += nt) Bm[e] *= rpiv[e / rk];
-  __syncthreads();
   // 11. folded factors from X = Bc V_r: P' = diag(1/sigma) X[:D],
   //     c' = X[D] - Σ_i (mu_i / sigma_i) X[i]
   float* pp = a.pp + bh * D * rk;
-  for (int e = tid; e < D * rk; e += nt) pp[e] = Bm[e] * isg[e / rk];
+  for (int e = tid; e < D * rk; e += nt) pp[e] = Xs[e] * isg[e / rk];
   for (int k = tid; k < rk; k += nt) {
-    float acc = Bm[D * rk + k];
-    for (int i = 0; i < D; ++i) acc -= mu[i] * isg[i] * Bm[i * rk + k];
+    float acc = Xs[D * rk + k];
+    for (int i = 0; i < D; ++i) acc -= mu[i] * isg[i] * Xs[i * rk + k];
     a.cc[bh * rk + k] = acc;
   }
 }
