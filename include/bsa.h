@@ -226,7 +226,7 @@ int bsa_probe_dense_attention(const void* q, const void* k, const void* v, bsa_s
  * and population variance over all S rows), Zt = [Z, 1], W = diag(weights):
  *   R    = o_probe - X[probe_idx]
  *   Bc   = (Zt_p^T W Zt_p + lam*diag(1,..,1,0))^-1 Zt_p^T W R   (Cholesky)
- *   V_r  = top-`rank` eigenvectors of R^T W R   (Householder, bisection, inverse iteration)
+ *   V_r  = top-`rank` eigenvectors of R^T W R   (Householder, multisection, inverse iteration)
  *   out <- X + Zt * Bc * V_r V_r^T                                  (every row)
  *   out       : device float32 (B, H, S, D), updated in place.
  *   o_probe   : device float32 (B, H, M, D).

@@ -107,3 +107,90 @@ def test_reuse_recipe_reduced():
         assert np.abs(got - o_ref).max() <= 2e-2
         assert np.linalg.norm(got - o_ref) / np.linalg.norm(o_ref) <= 5e-3
     assert bsa.device_status()[0] == 0
+
+
+def _host_means(x):
+    """Float64 token means per head of a (1, H, S, D) device tensor, shaped (1, H, 1, D)
+    (the oracle's pooling then reduces a singleton axis); computed head by head."""
+    return np.stack([x[0, h].double().mean(0).cpu().numpy() for h in range(x.shape[1])])[None, :, None]
+
+
+def test_reuse_recipe_video_full_size():
+    """The mask-reuse workload at full size: B=1, H=40, S=32760 (21x30x52), D=128,
+    20 steps of cumulative N(0, 0.05^2) drift (10x on heads 0-3), first 2 steps dense,
+    delta=8, gate 0.4/0.8, tau per head from (0.85, 0.90, 0.95), block 128, stride 16
+    (scoring on S padded to 32768), centroid-compensated attention every step.
+    Refresh decisions, counts and drifts for every head are checked against the oracle
+    cache each step; for sampled heads the oracle computes its own scores, top-p masks
+    (equal outside tie rows) and attention rows with its own masks."""
+    bsa = _bsa()
+    dev = torch.device("cuda", 0)
+    grid, H, D, S, Sp, C = (21, 30, 52), 40, 128, 32760, 32768, 256
+    heads = [0, 1, 2, 3, 17, 38]
+    q0, k0, v = wl.positional_qkv_device(1, H, H, grid, D, ell=(3.0, 6.0, 8.0), amp=2.0,
+                                         seed=5, device=dev)
+    tau = np.array([(0.85, 0.90, 0.95)[h % 3] for h in range(H)], dtype=np.float32)
+    lab = np.arange(S) // 128
+    lt = torch.as_tensor(lab, dtype=torch.int32, device=dev)
+    cache = bsa.MaskCache(1, H, C, C, D, delta=8.0, gate_lo=0.4, gate_hi=0.8)
+    ref = oracle.HeadMaskCache(8.0, gate_lo=0.4, gate_hi=0.8)
+    sig = torch.full((1, H, 1, 1), 0.05, device=dev)
+    sig[:, :4] *= 10.0
+    g = torch.Generator(device=dev).manual_seed(55)
+    qa, ka = q0.float(), k0.float()
+    pad = torch.zeros((1, H, Sp - S, D), dtype=torch.bfloat16, device=dev)
+    rng = np.random.default_rng(56)
+    n_refresh_steps = 0
+    for t in range(20):
+        if t > 0:
+            qa += torch.randn(qa.shape, generator=g, device=dev) * sig
+            ka += torch.randn(ka.shape, generator=g, device=dev) * sig
+        if t < 2:
+            continue  # dense warm-up steps leave the cache untouched
+        q, k = qa.to(torch.bfloat16), ka.to(torch.bfloat16)
+        r, n = cache.should_refresh(q, k)
+        r_ref = ref.should_refresh(_host_means(q), _host_means(k))
+        np.testing.assert_array_equal(r.cpu().numpy().astype(bool), r_ref)
+        assert n == int(r_ref.sum())
+        fin = np.isfinite(ref.last_drift)
+        np.testing.assert_allclose(cache.drift.cpu().numpy()[fin], ref.last_drift[fin],
+                                   rtol=1e-3, atol=1e-5)
+        new = None
+        new_ref = np.zeros((1, H, C, C), dtype=bool)  # heads outside `heads`: not compared
+        tie_rows = np.zeros((H, C), dtype=bool)
+        if n:
+            n_refresh_steps += 1
+            qp, kp = torch.cat([q, pad], 2), torch.cat([k, pad], 2)
+            sc = bsa.antidiagonal_block_scores(qp, kp, 128, 16)
+            new = bsa.top_p_block_mask(sc, torch.from_numpy(tau))
+            new_g = new.cpu().numpy().astype(bool)
+            for h in heads:
+                sc_ref = oracle.antidiagonal_block_scores(qp[:, h:h + 1].double().cpu().numpy(),
+                                                          kp[:, h:h + 1].double().cpu().numpy(),
+                                                          128, 16)
+                m_h, tie = oracle.top_p_block_mask(sc_ref, tau[h:h + 1])
+                new_ref[0, h] = m_h[0, 0]
+                tie_rows[h] = tie[0, 0]
+                bad = (new_g[0, h] != m_h[0, 0]).any(-1) & ~tie[0, 0]
+                assert not bad.any(), (t, h, np.nonzero(bad))
+        m = cache.update(new)
+        m_ref = ref.update(new_ref, r_ref)
+        mg = m.cpu().numpy().astype(bool)
+        out = bsa.centroid_compensated_attention(q, k, v, lt, lt, m)
+        out_h = out[0, heads].cpu().numpy()
+        for i, h in enumerate(heads):
+            diff = (mg[0, h] != m_ref[0, h]).any(-1)
+            assert not (diff & ~tie_rows[h]).any()
+            rows = rng.choice(S, 64, replace=False)
+            rows = np.sort(rows[~diff[lab[rows]]])
+            o_ref = oracle.centroid_compensated_attention(
+                q[:, h:h + 1].double().cpu().numpy(), k[:, h:h + 1].double().cpu().numpy(),
+                v[:, h:h + 1].double().cpu().numpy(), lab, lab, m_ref[:, h:h + 1], rows=rows,
+                Cq=C, Ck=C)
+            got = out_h[i][rows]
+            assert np.abs(got - o_ref[0, 0]).max() <= 2e-2
+            assert np.linalg.norm(got - o_ref[0, 0]) / np.linalg.norm(o_ref[0, 0]) <= 5e-3
+    # the recipe's expected behaviour: only the first cached step refreshes (the pooled
+    # drift stays far below delta, and 4 of 40 heads are under the gate's 40 %)
+    assert n_refresh_steps == 1
+    assert bsa.device_status()[0] == 0
