@@ -75,6 +75,26 @@ def test_dynamic_mask_workload_scores_and_masks():
     assert not (diff_rows & ~tie).any(), f"{int((diff_rows & ~tie).sum())} non-tie rows differ"
     print(f"tie rows {int(tie.sum())}, differing rows {int(diff_rows.sum())}, density "
           f"{m_gpu.mean():.3f}")
+    # the chain's last step: compensated attention on the top-p mask, labels arange // 128;
+    # sampled rows against the oracle's attention on the oracle's own mask (rows of query
+    # blocks whose masks differ, tie rows only, are left out)
+    _, _, v, _ = wl.positional_qkv(1, 8, 8, (8192,), 64, ell=(256.0,), amp=2.0, dtype="bf16",
+                                   seed=2)
+    lab = np.arange(8192) // 128
+    lt = torch.as_tensor(lab, dtype=torch.int32).cuda()
+    out = bsa.centroid_compensated_attention(q.cuda(), k.cuda(), v.cuda(), lt, lt,
+                                             torch.from_numpy(m_gpu.astype(np.uint8)).cuda())
+    got = out.cpu().numpy()
+    rows = np.sort(np.random.default_rng(21).choice(8192, 512, replace=False))
+    ref_o = oracle.centroid_compensated_attention(q.double().numpy(), k.double().numpy(),
+                                                  v.double().numpy(), lab, lab, m_ref, rows=rows,
+                                                  Cq=64, Ck=64)
+    for h in range(8):
+        keep = ~diff_rows[0, h][lab[rows]]
+        g_h, r_h = got[0, h, rows[keep]], ref_o[0, h, keep]
+        assert np.abs(g_h - r_h).max() <= 2e-2
+        assert np.linalg.norm(g_h - r_h) / np.linalg.norm(r_h) <= 5e-3
+    assert bsa.device_status()[0] == 0
 
 
 def test_video_reuse_workload_scores_sampled_heads():
