@@ -210,6 +210,10 @@ __global__ void __launch_bounds__(256) centroid_order_kernel(
   for (int i = threadIdx.x; i < n; i += blockDim.x) order[bh * S + start + i] = tokn[i];
 }
 
+// Cluster sizes staged in shared memory for the selecting thread (C above this reads
+// them from global memory).
+constexpr int kRoundRobinStage = 4096;
+
 // One CTA per head (or one in total for the shared variant): round-robin stratified
 // selection across non-empty clusters, then w = |G_a| / m_a normalised to sum 1.
 __global__ void __launch_bounds__(256) round_robin_kernel(
@@ -220,15 +224,20 @@ __global__ void __launch_bounds__(256) round_robin_kernel(
   __shared__ int chosen[kMaxProbes];
   __shared__ float wsum[256];
   __shared__ int n_taken;
+  __shared__ int cnt_s[kRoundRobinStage];  // cluster sizes, read by the selecting thread
   const int bh = blockIdx.x;
   const int32_t* ord = order ? order + static_cast<int64_t>(bh) * S : nullptr;
+  const bool staged = C <= kRoundRobinStage;
+  for (int a = threadIdx.x; a < C && staged; a += blockDim.x) cnt_s[a] = count[a];
+  __syncthreads();
+  auto cnt = [&](int a) -> int { return staged ? cnt_s[a] : count[a]; };
   auto member = [&](int a, int k) -> int {
-    const int n = count[a];
+    const int n = cnt(a);
     return ord ? ord[off[a] + k] : slot_token[off[a] + middle_out(n, k)];
   };
   if (threadIdx.x == 0) {
     int cp = 0;
-    for (int a = 0; a < C; ++a) cp += count[a] > 0;
+    for (int a = 0; a < C; ++a) cp += cnt(a) > 0;
     int taken = 0;
     if (M < cp) {
       int a = -1, seen = -1;
@@ -236,7 +245,7 @@ __global__ void __launch_bounds__(256) round_robin_kernel(
         const int target = static_cast<int>((static_cast<int64_t>(i) * cp) / M);
         while (seen < target) {
           ++a;
-          if (count[a] > 0) ++seen;
+          if (cnt(a) > 0) ++seen;
         }
         owner[taken] = a;
         chosen[taken++] = member(a, 0);
@@ -245,7 +254,7 @@ __global__ void __launch_bounds__(256) round_robin_kernel(
       for (int p = 0; taken < M; ++p) {
         bool any = false;
         for (int a = 0; a < C && taken < M; ++a) {
-          if (count[a] > p) {
+          if (cnt(a) > p) {
             owner[taken] = a;
             chosen[taken++] = member(a, p);
             any = true;
@@ -263,7 +272,7 @@ __global__ void __launch_bounds__(256) round_robin_kernel(
     if (i < taken) {
       int m = 0;
       for (int j = 0; j < taken; ++j) m += owner[j] == owner[i];
-      const float w = static_cast<float>(count[owner[i]]) / static_cast<float>(m);
+      const float w = static_cast<float>(cnt(owner[i])) / static_cast<float>(m);
       weights[static_cast<int64_t>(bh) * M + i] = w;
       local += w;
     }

@@ -65,6 +65,9 @@ __global__ void __launch_bounds__(kTopPWarps * 32) top_p_kernel(
   if (lane == 0) {
     float acc = 0.f;
     bool found = false;
+    // Scores are non-negative, so the running sum never decreases: once it is past
+    // tau by more than the tie tolerance, no later prefix decides or flags anything.
+#pragma unroll 4
     for (int i = 0; i < Nk; ++i) {
       acc = __fadd_rn(acc, sv[i]);
       if (fabsf(acc - t) <= 1e-5f) tie = 1;
@@ -72,6 +75,7 @@ __global__ void __launch_bounds__(kTopPWarps * 32) top_p_kernel(
         m = i;
         found = true;
       }
+      if (found && acc - t > 1e-5f) break;
     }
     if (m + 1 < Nk && sv[m] - sv[m + 1] <= 1e-5f) tie = 1;
   }
