@@ -333,27 +333,59 @@ def main():
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         mh = mask.cpu().pin_memory()
         oh = torch.empty((1, nh, S, D), dtype=torch.float32).pin_memory()
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        md = torch.empty_like(mask)
+        # Two device copies of a step's inputs and output: step i computes on set i % 2
+        # while the upload of step i + 1 and the download of step i - 1 run on their own
+        # streams (PCIe carries both directions at once). Every step's upload and
+        # download lies inside the timed region.
+        sets = [dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
+                     m=torch.empty_like(mask), o=torch.empty_like(out)) for _ in range(2)]
+        s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        up = [torch.cuda.Event() for _ in range(2)]    # upload into set j done
+        done = [torch.cuda.Event() for _ in range(2)]  # compute on set j done
+        down = [torch.cuda.Event() for _ in range(2)]  # download of set j's output done
 
-        def e2e_step():
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            md.copy_(mh, non_blocking=True)
-            lab, _ = bsa.tile_labels(*GRID, TILE, device=dev)
-            bsa.centroid_compensated_attention(qd, kd, vd, lab, lab, md, Cq=C, Ck=C, out=out,
-                                               workspace=ws)
-            oh.copy_(out, non_blocking=True)
+        def upload(i):
+            b = sets[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done[i % 2])  # step i - 2 no longer reads this set
+                for key, h in (("q", qh), ("k", kh), ("v", vh), ("m", mh)):
+                    b[key].copy_(h, non_blocking=True)
+                up[i % 2].record(s_in)
 
-        e2e_step()
+        def compute(i):
+            b = sets[i % 2]
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(up[i % 2])
+                if i >= 2:
+                    s_cmp.wait_event(down[i % 2])  # step i - 2's output has been read
+                lab, _ = bsa.tile_labels(*GRID, TILE, device=dev)
+                bsa.centroid_compensated_attention(b["q"], b["k"], b["v"], lab, lab, b["m"],
+                                                   Cq=C, Ck=C, out=b["o"], workspace=ws)
+                done[i % 2].record(s_cmp)
+
+        def download(i):
+            b = sets[i % 2]
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[i % 2])
+                oh.copy_(b["o"], non_blocking=True)
+                down[i % 2].record(s_out)
+
+        def run(n):
+            upload(0)
+            for i in range(n):
+                if i + 1 < n:
+                    upload(i + 1)
+                compute(i)
+                download(i)
+
+        run(2)
         torch.cuda.synchronize()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(args.steps):
-            e2e_step()
-        b.record()
+        a.record(s_in)
+        run(args.steps)
+        b.record(s_out)  # the last download follows every compute and upload
         torch.cuda.synchronize()
         barrier()
         e2e_ms = a.elapsed_time(b) / args.steps
@@ -362,8 +394,10 @@ def main():
         d2h = oh.numel() * oh.element_size()
         e2e = {"value": weak_scaling_tflops(flop, world, e2e_ms), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "block_sparse_attention_tcgen05_b200.centroid_compensated_attention"}
-        del qh, kh, vh, oh, qd, kd, vd
+               "api": "block_sparse_attention_tcgen05_b200.centroid_compensated_attention",
+               "overlap": "upload of step i+1 and download of step i-1 on their own streams "
+                          "during step i (double-buffered device tensors)"}
+        del qh, kh, vh, oh, sets
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
