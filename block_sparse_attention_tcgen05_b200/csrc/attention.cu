@@ -539,9 +539,10 @@ __device__ __forceinline__ Chunk decode_chunk(uint32_t rec) {
   return c;
 }
 
-// Pairs of every 8 whose exponentials use the FMA-pipe polynomial instead of MUFU ex2.
-// 0: measured fastest in this kernel (the softmax warps are issue-bound, not MUFU-bound).
-constexpr int kPolyPairsOf8 = 0;
+// Pairs of every 8 whose exponentials use the FMA-pipe polynomial instead of MUFU ex2
+// (the two CTAs' softmax warps share each sub-partition's MUFU). Measured at the video
+// workload: 0 -> 8.15 ms, 1 -> 7.99 ms, 2 -> 8.21 ms per kernel.
+constexpr int kPolyPairsOf8 = 1;
 
 // Max of 16 / 64 register values as shallow trees of 3-input maxes.
 __device__ __forceinline__ float max16(const float* v) {
