@@ -696,30 +696,33 @@ __global__ void __launch_bounds__(256) repair_apply_kernel(float* __restrict__ o
 }
 
 constexpr int kApplyRows = 128;
+constexpr int kApplyThreads = 64;  // two rows per thread
 constexpr int apply16_smem_bytes(int D) {
   return static_cast<int>(sizeof(float)) * (2 * D * 16 + kApplyRows * (D + 4) + 16);
 }
 
 // rank <= 16: tiles of 128 rows staged through shared memory, so that every global
 // access is a coalesced 16-byte vector (HBM traffic: one read and one write of out);
-// then one row per thread: y = x P' + c' (each factor row d is a broadcast read of 16
-// floats, all lanes the same address), x += y V_rᵀ (V_rᵀ row k broadcast likewise),
-// pairs of outputs per packed f32x2 FMA. Rows are padded to D + 4 floats, so the eight
-// rows of a quarter-warp fall on distinct 16-byte bank groups. grid (ceil(S / 128),
-// B*H), 128 threads; factors as P'[d][k], V_rᵀ[k][d], zero past `rank`.
+// then two rows per thread (rows t and t + 64): y = x P' + c' (each factor row d is a
+// broadcast read of 16 floats, all lanes the same address, used for both rows),
+// x += y V_rᵀ (V_rᵀ row k broadcast likewise), pairs of outputs per packed f32x2 FMA.
+// Rows are padded to D + 4 floats, so the eight rows of a quarter-warp fall on distinct
+// 16-byte bank groups. grid (ceil(S / 128), B*H), 64 threads; factors as P'[d][k],
+// V_rᵀ[k][d], zero past `rank`.
 template <int D>
-__global__ void __launch_bounds__(128) repair_apply16_kernel(float* __restrict__ out, int S, int rank,
-                                                             const float* __restrict__ pp,
-                                                             const float* __restrict__ cc,
-                                                             const float* __restrict__ vr) {
-  constexpr int TR = kApplyRows, LD = D + 4, V4 = D / 4;
+__global__ void __launch_bounds__(kApplyThreads) repair_apply16_kernel(float* __restrict__ out, int S,
+                                                                      int rank,
+                                                                      const float* __restrict__ pp,
+                                                                      const float* __restrict__ cc,
+                                                                      const float* __restrict__ vr) {
+  constexpr int TR = kApplyRows, LD = D + 4, V4 = D / 4, NT = kApplyThreads;
   extern __shared__ __align__(16) float apply_smem[];  // apply16_smem_bytes(D)
   float(*sP)[16] = reinterpret_cast<float(*)[16]>(apply_smem);
   float(*sVt)[D] = reinterpret_cast<float(*)[D]>(apply_smem + D * 16);
   float* xs = apply_smem + 2 * D * 16;
   float* sc = xs + TR * LD;
   const int64_t bh = blockIdx.y;
-  for (int e = threadIdx.x; e < D * 16; e += blockDim.x) {
+  for (int e = threadIdx.x; e < D * 16; e += NT) {
     const int d = e / 16, k = e % 16;
     const bool in = k < rank;
     sP[d][k] = in ? pp[(bh * D + d) * rank + k] : 0.f;
@@ -729,49 +732,56 @@ __global__ void __launch_bounds__(128) repair_apply16_kernel(float* __restrict__
   const int r0 = blockIdx.x * TR;
   const int nr = min(TR, S - r0);
   const float4* src = reinterpret_cast<const float4*>(out + (bh * S + r0) * D);
-  // fixed trip count: each thread's TR * V4 / 128 loads are in flight together
+  // fixed trip count: each thread's TR * V4 / NT loads are in flight together
 #pragma unroll
-  for (int i = 0; i < TR * V4 / 128; ++i) {
-    const int e = threadIdx.x + 128 * i;
+  for (int i = 0; i < TR * V4 / NT; ++i) {
+    const int e = threadIdx.x + NT * i;
     if (e < nr * V4) *reinterpret_cast<float4*>(&xs[(e / V4) * LD + 4 * (e % V4)]) = __ldg(src + e);
   }
   __syncthreads();
-  if (threadIdx.x < nr) {
-    float* xr = &xs[threadIdx.x * LD];
-    float y[16];
+  // rows a = t and b = t + 64 (rows past nr hold stale values and are not written back)
+  float* xa = &xs[threadIdx.x * LD];
+  float* xb = &xs[(threadIdx.x + NT) * LD];
+  float ya[16], yb[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) y[k] = sc[k];
+  for (int k = 0; k < 16; ++k) ya[k] = yb[k] = sc[k];
 #pragma unroll 2
-    for (int d4 = 0; d4 < V4; ++d4) {
-      const float4 x = *reinterpret_cast<const float4*>(xr + 4 * d4);
-      const float xv[4] = {x.x, x.y, x.z, x.w};
+  for (int d4 = 0; d4 < V4; ++d4) {
+    const float4 a4 = *reinterpret_cast<const float4*>(xa + 4 * d4);
+    const float4 b4 = *reinterpret_cast<const float4*>(xb + 4 * d4);
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < 4; ++j) {
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const float4 p = *reinterpret_cast<const float4*>(&sP[4 * d4 + j][4 * k4]);
-          fma2(y[4 * k4], y[4 * k4 + 1], xv[j], xv[j], p.x, p.y, y[4 * k4], y[4 * k4 + 1]);
-          fma2(y[4 * k4 + 2], y[4 * k4 + 3], xv[j], xv[j], p.z, p.w, y[4 * k4 + 2], y[4 * k4 + 3]);
-        }
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 p = *reinterpret_cast<const float4*>(&sP[4 * d4 + j][4 * k4]);
+        fma2(ya[4 * k4], ya[4 * k4 + 1], av[j], av[j], p.x, p.y, ya[4 * k4], ya[4 * k4 + 1]);
+        fma2(ya[4 * k4 + 2], ya[4 * k4 + 3], av[j], av[j], p.z, p.w, ya[4 * k4 + 2], ya[4 * k4 + 3]);
+        fma2(yb[4 * k4], yb[4 * k4 + 1], bv[j], bv[j], p.x, p.y, yb[4 * k4], yb[4 * k4 + 1]);
+        fma2(yb[4 * k4 + 2], yb[4 * k4 + 3], bv[j], bv[j], p.z, p.w, yb[4 * k4 + 2], yb[4 * k4 + 3]);
       }
     }
+  }
 #pragma unroll 2
-    for (int c4 = 0; c4 < V4; ++c4) {
-      float4 x = *reinterpret_cast<const float4*>(xr + 4 * c4);
+  for (int c4 = 0; c4 < V4; ++c4) {
+    float4 a4 = *reinterpret_cast<const float4*>(xa + 4 * c4);
+    float4 b4 = *reinterpret_cast<const float4*>(xb + 4 * c4);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float4 v = *reinterpret_cast<const float4*>(&sVt[k][4 * c4]);
-        fma2(x.x, x.y, y[k], y[k], v.x, v.y, x.x, x.y);
-        fma2(x.z, x.w, y[k], y[k], v.z, v.w, x.z, x.w);
-      }
-      *reinterpret_cast<float4*>(xr + 4 * c4) = x;
+    for (int k = 0; k < 16; ++k) {
+      const float4 v = *reinterpret_cast<const float4*>(&sVt[k][4 * c4]);
+      fma2(a4.x, a4.y, ya[k], ya[k], v.x, v.y, a4.x, a4.y);
+      fma2(a4.z, a4.w, ya[k], ya[k], v.z, v.w, a4.z, a4.w);
+      fma2(b4.x, b4.y, yb[k], yb[k], v.x, v.y, b4.x, b4.y);
+      fma2(b4.z, b4.w, yb[k], yb[k], v.z, v.w, b4.z, b4.w);
     }
+    *reinterpret_cast<float4*>(xa + 4 * c4) = a4;
+    *reinterpret_cast<float4*>(xb + 4 * c4) = b4;
   }
   __syncthreads();
   float4* dst = reinterpret_cast<float4*>(out + (bh * S + r0) * D);
 #pragma unroll
-  for (int i = 0; i < TR * V4 / 128; ++i) {
-    const int e = threadIdx.x + 128 * i;
+  for (int i = 0; i < TR * V4 / NT; ++i) {
+    const int e = threadIdx.x + NT * i;
     if (e < nr * V4) dst[e] = *reinterpret_cast<const float4*>(&xs[(e / V4) * LD + 4 * (e % V4)]);
   }
 }
@@ -839,8 +849,8 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
     const int smem16 = apply16_smem_bytes(D);
     e = cudaFuncSetAttribute(ap16, cudaFuncAttributeMaxDynamicSharedMemorySize, smem16);
     if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(repair_apply16)");
-    ap16<<<dim3((S + kApplyRows - 1) / kApplyRows, BH), kApplyRows, smem16, st>>>(out, S, rank, L.pp,
-                                                                                 L.cc, L.vr);
+    ap16<<<dim3((S + kApplyRows - 1) / kApplyRows, BH), kApplyThreads, smem16, st>>>(out, S, rank,
+                                                                                    L.pp, L.cc, L.vr);
     count_launch();
     return check_cuda(cudaGetLastError(), "repair_apply16_kernel");
   }
