@@ -372,63 +372,17 @@ __device__ __forceinline__ bool bit_at(const uint32_t* bits, int i) {
   return (bits[i >> 5] >> (i & 31)) & 1u;
 }
 
-// Deterministic chunk walk shared by every role of the CTA: runs of kept 16-key
-// groups split into chunks of at most 8 groups, then the needed centroid chunks. The
-// run length and the uniform test use 64-bit windows of the bitsets (trailing-ones
-// count), so one step costs a handful of shared loads whatever the run.
-__device__ __forceinline__ bool next_chunk(int& gcur, int& ccur, const uint32_t* any,
-                                           const uint32_t* uni, int G, int Wg,
-                                           const uint32_t* cneed, int ncc, Chunk& ch) {
-  if (gcur < G) {
-    int w = gcur >> 5;
-    uint32_t bits = any[w] & (0xffffffffu << (gcur & 31));
-    while (bits == 0 && ++w < Wg) bits = any[w];
-    // (a kept group past G belongs to another CTA's key range)
-    if (bits != 0 && (w << 5) + __ffs(bits) - 1 < G) {
-      const int b0 = __ffs(bits) - 1;
-      const int g0 = (w << 5) + b0;
-      const uint32_t a_hi = (w + 1 < Wg) ? any[w + 1] : 0u;
-      const uint32_t u_hi = (w + 1 < Wg) ? uni[w + 1] : 0u;
-      const uint64_t awin = ((static_cast<uint64_t>(a_hi) << 32) | any[w]) >> b0;
-      const uint64_t uwin = ((static_cast<uint64_t>(u_hi) << 32) | uni[w]) >> b0;
-      const int run = __ffsll(static_cast<long long>(~awin)) - 1;  // trailing ones
-      int ng = (run < 0 || run > 8) ? 8 : run;
-      if (ng > G - g0) ng = G - g0;
-      const uint32_t m = (1u << ng) - 1u;
-      ch.start = g0 * 16;
-      ch.n = ng * 16;
-      ch.g0 = g0;
-      ch.ng = ng;
-      ch.uniform = (static_cast<uint32_t>(uwin) & m) == m;
-      ch.centroid = false;
-      gcur = g0 + ng;
-      return true;
-    }
-    gcur = G;
-  }
-  while (ccur < ncc) {
-    const int i = ccur++;
-    if (bit_at(cneed, i)) {
-      ch.start = i * 128;
-      ch.n = 128;
-      ch.g0 = ch.ng = 0;
-      ch.uniform = false;
-      ch.centroid = true;
-      return true;
-    }
-  }
-  return false;
-}
-
-// A CTA's chunk list, built once by one warp: exactly the chunks next_chunk() yields
-// from g_lo with limit g_hi, as 32-bit records (bit 31 centroid, bit 30 uniform, bits
-// 16..19 groups - 1, bits 0..15 first group or centroid chunk index), so that no role
-// re-walks the bitsets per chunk. Groups outside [g_lo, g_hi) count as dropped (a run
-// restarts at g_lo and is cut at g_hi, as in next_chunk). Lane L scans groups
-// [128 L, 128 L + 128); the position inside a run at its first group comes from the
-// trailing kept groups of the lanes before it (whole kept segments add 128 = 0 mod 8).
-// At most 2048 token chunks (runs are separated by a dropped group and G <= 4096) plus
-// 128 centroid chunks.
+// A CTA's chunk list, built once by one warp so that no role walks the bitsets per
+// chunk. The chunks, in order: every run of consecutive kept 16-key groups inside the
+// CTA's key range [g_lo, g_hi) (groups outside it count as dropped), cut into chunks of
+// at most 8 groups from the run's start; then one 128-wide chunk per needed centroid
+// chunk. A token chunk is uniform when every row of the tile keeps all of its groups
+// and none of them holds pad slots. Records are 32-bit (bit 31 centroid, bit 30
+// uniform, bits 16..19 groups - 1, bits 0..15 first group or centroid chunk index).
+// Lane L scans groups [128 L, 128 L + 128); the position inside a run at its first
+// group comes from the trailing kept groups of the lanes before it (whole kept segments
+// add 128 = 0 mod 8). At most 2048 token chunks (runs are separated by a dropped group
+// and G <= 4096) plus 128 centroid chunks.
 __device__ __forceinline__ uint32_t kept_word(const uint32_t* any, int w, int Wg, int g_lo, int g_hi) {
   if (w < 0 || w >= Wg) return 0u;
   uint32_t x = any[w];
