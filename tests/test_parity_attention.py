@@ -206,3 +206,20 @@ def test_key_range_at_the_limit():
     for comp in (True, False):
         got = _run(q, k, v, lab, lab, mask, C, C, comp)
         _check(got[:, :, rows], _ref(q, k, v, lab, lab, mask, C, C, comp, rows=rows))
+
+
+@pytest.mark.parametrize("H,Hkv", [(40, 10), (2, 1)])
+def test_per_batch_and_head_masks(H, Hkv):
+    """B=2 with a different mask for every (batch, head) (batch and head mask strides),
+    grouped-query heads, shuffled uneven clusters; 40 heads run without a key split,
+    2 heads with one; compensated and hard drop."""
+    g = np.random.default_rng(51)
+    B, S, Cq, Ck = 2, 640, 7, 9
+    ql = g.permutation(np.concatenate([np.arange(Cq), g.integers(0, Cq, S - Cq)]))
+    kl = g.permutation(np.concatenate([np.arange(Ck), g.integers(0, Ck, S - Ck)]))
+    mask = g.random((B, H, Cq, Ck)) < 0.35
+    q, k, v = wl.gaussian_qkv(B, H, Hkv, S, 64, "bf16", seed=52)
+    rows = np.sort(g.choice(S, 128, replace=False))
+    for comp in (True, False):
+        got = _run(q, k, v, ql, kl, mask, Cq, Ck, comp)
+        _check(got[:, :, rows], _ref(q, k, v, ql, kl, mask, Cq, Ck, comp, rows=rows))
