@@ -84,10 +84,11 @@ def test_repair_kernel_matches_oracle_on_same_input():
     """GPU repair and oracle repair of the same fp32 sparse output and probes."""
     bsa = _bsa()
     g = np.random.default_rng(6)
-    # the last case has M >= D (the D x D residual Gram matrix, probe rows kept in the
-    # workspace instead of shared memory) and a rank above 16 (the general apply kernel)
+    # (1200, 128, 160, 24) has M >= D (the D x D residual Gram matrix, probe rows kept in
+    # the workspace instead of shared memory) and a rank above 16 (the general apply
+    # kernel); (512, 64, 8, 16) asks for more directions than the 8 probes span
     for (S, D, M, rank) in [(1024, 64, 64, 16), (2000, 128, 64, 16), (1500, 64, 100, 8),
-                            (1200, 128, 160, 24)]:
+                            (1200, 128, 160, 24), (512, 64, 8, 16)]:
         out = g.standard_normal((1, 2, S, D)).astype(np.float32) * 0.1
         idx = g.choice(S, M, replace=False).astype(np.int32)
         w = (g.random(M) + 0.5).astype(np.float32)

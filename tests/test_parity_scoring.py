@@ -58,6 +58,15 @@ def test_top_p_kernel_bit_exact_on_identical_scores():
     ref2, _ = oracle.top_p_block_mask(sc2, 0.9, dtype=np.float32)
     np.testing.assert_array_equal(got2.cpu().numpy().astype(bool), ref2)
     assert (got2.cpu().numpy().sum(-1) >= 1).all()
+    # degenerate tau: a tiny tau keeps the arg-max block only; tau = 1 keeps every block
+    # up to the first running sum reaching 1 (the whole row when rounding stays below 1)
+    for t in (1e-7, 1.0):
+        got3 = bsa.top_p_block_mask(torch.from_numpy(sc).cuda(), t).cpu().numpy().astype(bool)
+        ref3, _ = oracle.top_p_block_mask(sc, t, dtype=np.float32)
+        np.testing.assert_array_equal(got3, ref3)
+        if t < 1e-3:
+            assert (got3.sum(-1) == 1).all()
+            np.testing.assert_array_equal(got3.argmax(-1), sc.argmax(-1))
 
 
 def test_dynamic_mask_workload_scores_and_masks():
