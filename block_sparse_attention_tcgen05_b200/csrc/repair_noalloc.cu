@@ -2,9 +2,9 @@
 //
 // bsa_probe_residual_correction needs a few megabytes of scratch that the caller
 // normally passes in. Some callers cannot obtain that memory at the moment they call:
-// code that runs while a CUDA graph is being captured (cudaMalloc is not allowed
-// there), runtimes without a device allocator of their own, and serving loops whose
-// device memory is fixed before the first request and may not grow afterwards. For
+// runtimes without a device allocator of their own, code on a path that must not call
+// the allocator, and serving loops whose device memory is fixed before the first
+// request and may not grow afterwards. For
 // them this file keeps a fixed scratch buffer inside the library itself and runs the
 // same repair with it; nothing is allocated per call.
 //

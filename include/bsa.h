@@ -243,10 +243,10 @@ int bsa_probe_residual_correction(float* out, const float* o_probe, const int32_
 /*
  * probe_residual_correction_noalloc — no counterpart in the papers: a convenience for
  * callers that cannot allocate device memory when they repair an output (for example
- * while a CUDA graph is being captured, or in a runtime whose device memory is fixed
- * up front). Same arguments and result as bsa_probe_residual_correction, minus the
- * workspace: the scratch comes from a 16 MiB buffer compiled into the library, which
- * every GPU that loads libbsa.so holds until the process exits.
+ * a runtime whose device memory is fixed up front, or code on a path that must not
+ * call the allocator). Same arguments and result as bsa_probe_residual_correction,
+ * minus the workspace: the scratch comes from a 16 MiB buffer compiled into the
+ * library, which every GPU that loads libbsa.so holds until the process exits.
  *  - Size limit: bsa_repair_workspace_bytes(B, H, S, D, M) must be <= 16 MiB (about
  *    B*H <= 48 heads at D = 128, M = 64); larger problems return BSA_ERR_UNSUPPORTED
  *    with the required size in the error detail.

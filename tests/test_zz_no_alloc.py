@@ -1,7 +1,8 @@
 """GPU test of bsa_probe_residual_correction_noalloc, the repair entry point that takes
 its scratch from a buffer built into the library instead of a caller workspace (for
-callers that cannot allocate device memory when they call, e.g. during CUDA graph
-capture). Its output must equal the workspace entry point's on two calls in a row.
+callers that cannot allocate device memory when they call, e.g. a runtime whose device
+memory is fixed up front). Its output must equal the workspace entry point's on two
+calls in a row.
 
 This file is collected last on purpose, and must pass alone and after the others."""
 
