@@ -68,6 +68,43 @@ __global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
   __shared__ int32_t warp_tot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+  // One cluster whose labels are all valid (the probe attention's keys): the stable
+  // order is the identity, filled directly; anything else takes the general path.
+  __shared__ int n_bad;
+  if (tid == 0) n_bad = 0;
+  __syncthreads();
+  if (C == 1) {
+    int bad = 0;
+    for (int i = tid; i < S; i += 1024) bad += labels[i] != 0;
+    bad = __reduce_add_sync(0xffffffffu, bad);
+    if (lane == 0 && bad) atomicAdd(&n_bad, bad);
+    __syncthreads();
+    if (n_bad == 0) {
+      const int padded = (S + cluster_pad - 1) / cluster_pad * cluster_pad;
+      for (int i = tid; i < n_slots; i += 1024) {
+        slot_token[i] = i < S ? i : -1;
+        if (slot_label) slot_label[i] = i < S ? 0 : -1;
+      }
+      if (tid == 0) {
+        count[0] = S;
+        off[0] = 0;
+        off[1] = padded;
+      }
+      if (group_cluster) {
+        for (int g = tid; g < n_groups; g += 1024) {
+          const int slot = g * 16;
+          group_cluster[g] = slot < padded ? 0 : -1;
+          group_valid[g] = slot < padded ? min(16, S - slot) : 0;
+        }
+      }
+      if (bias2) {
+        for (int c = tid; c < C_pad; c += 1024)
+          bias2[c] = (c == 0 && S > 0) ? log2f(static_cast<float>(S)) : -INFINITY;
+        if (tid == 0) nonempty_bits[0] = S > 0 ? 1u : 0u;
+      }
+      return;
+    }
+  }
   for (int c = tid; c < C; c += 1024) cnt[c] = 0;
   for (int i = tid; i < n_slots; i += 1024) {
     slot_token[i] = -1;
