@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(256) centroid_order_kernel(
   const T* qb = q + bh * S * D;
   const int epl = D / 32;  // 2 or 4
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
   for (int i = warp; i < n; i += nw) {
     float x[4];
     load_lane<T>(qb + static_cast<int64_t>(slot_token[start + i]) * D + lane * epl, epl, x);
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__(256) centroid_order_kernel(
   while (np < n) np <<= 1;
   float best_d = INFINITY;
   int best_t = 0x7fffffff;
+#pragma unroll 4
   for (int i = warp; i < np; i += nw) {
     if (i < n) {
       const int tok = slot_token[start + i];
