@@ -84,12 +84,21 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+ATTN_SECTION = b"// ============================================================== attention kernel"
+
+
 def attention_source_hash():
+    """Hash of the source that decides the attention kernel's DRAM traffic: attention.cu
+    from the kernel's section to the end (the kernel, its helpers and its launch code;
+    the label sorts, mask bitsets and gathers above it are separate kernels) and the
+    PTX wrappers it uses."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "block_sparse_attention_tcgen05_b200", "csrc")
-    for name in ("attention.cu", "ptx.cuh"):
-        with open(os.path.join(d, name), "rb") as f:
-            h.update(f.read())
+    with open(os.path.join(d, "attention.cu"), "rb") as f:
+        src = f.read()
+    h.update(src[src.index(ATTN_SECTION):])
+    with open(os.path.join(d, "ptx.cuh"), "rb") as f:
+        h.update(f.read())
     return h.hexdigest()[:16]
 
 
