@@ -166,6 +166,17 @@ def bench_attention(timer, dev, hbm, tc, out):
     out.append(row("a8", f"fused compensated attention kernel ({pairs:.3e} executed pairs x 4D)",
                    kernel_ms, pairs * 4 * D, "FLOP", "tensor", tc))
     out.append(row("a4-a8", "whole attention call", ms, pairs * 4 * D, "FLOP", "tensor", tc))
+    # context: the same call with every tile pair kept (dense attention through the same
+    # kernel); its time over the sparse call's is the sparse path's speedup
+    full = torch.ones_like(mask)
+
+    def dense_call():
+        ops.centroid_compensated_attention(q, k, v, labels, labels, full, Cq=C, Ck=C, out=o,
+                                           workspace=ws)
+    dense_ms = timer(dense_call)
+    out.append(row("a4-a8 dense", "the same call with every tile pair kept (context)", dense_ms,
+                   float(H) * S * S * 4 * D, "FLOP", "tensor", tc))
+    out[-1]["speedup_of_sparse_call"] = dense_ms / ms
 
 
 def bench_probe_and_repair(timer, dev, hbm, tc, out):
