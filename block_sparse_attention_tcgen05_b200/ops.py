@@ -31,6 +31,36 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous")
 
 
+def _expect(t, name, dtypes=None, ndims=None, shape=None):
+    """Dtype and shape checks made before anything reaches the C ABI, which takes plain
+    pointers: a tensor of the wrong element type or size would be read or written past
+    its end there."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {list(dtypes)}")
+    if ndims is not None and t.dim() not in ndims:
+        raise ValueError(f"{name}: {t.dim()} dimensions, expected {list(ndims)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _expect_qkv(q, k, v=None):
+    """q (B,Hq,Sq,D), k and v (B,Hkv,Sk,D), one element type (bf16 or fp32)."""
+    _expect(q, "q", tuple(_DT), (4,))
+    _expect(k, "k", (q.dtype,), (4,))
+    B, Hq, _, D = q.shape
+    if k.shape[0] != B or k.shape[3] != D or k.shape[1] <= 0 or Hq % k.shape[1]:
+        raise ValueError(f"k: shape {tuple(k.shape)} does not fit q {tuple(q.shape)}")
+    if v is not None:
+        _expect(v, "v", (q.dtype,), (4,), tuple(k.shape))
+
+
+def _expect_workspace(workspace):
+    if workspace is not None:
+        _expect(workspace, "workspace", (torch.uint8,), (1,))
+
+
 def _workspace(nbytes, dev):
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
 
@@ -92,16 +122,20 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
     """SVG-EAR centroid-compensated block-sparse attention (``compensate=False``: hard
     drop). q: (B,Hq,S,D), k/v: (B,Hkv,S,D) bf16 or fp32; labels int32; block_mask
     bool/uint8 (Cq,Ck) / (H,Cq,Ck) / (B,H,Cq,Ck). Returns fp32 (B,Hq,S,D)."""
-    _need_cuda(q, k, v, q_labels, k_labels, block_mask)
+    _expect_qkv(q, k, v)
     B, Hq, Sq, D = q.shape
+    _expect(q_labels, "q_labels", (torch.int32,), (1,), (Sq,))
+    _expect(k_labels, "k_labels", (torch.int32,), (1,), (k.shape[2],))
+    if out is not None:
+        _expect(out, "out", (torch.float32,), (4,), (B, Hq, Sq, D))
+    _expect_workspace(workspace)
+    _need_cuda(q, k, v, q_labels, k_labels, block_mask, out, workspace)
     Cq = int(block_mask.shape[-2]) if Cq is None else int(Cq)
     Ck = int(block_mask.shape[-1]) if Ck is None else int(Ck)
     shape = make_shape(q, k)
     m, bs, hs = _mask_strides(block_mask, B, Hq, Cq, Ck)
-    if q_labels.dtype != torch.int32 or k_labels.dtype != torch.int32:
-        raise ValueError("labels must be int32")
     if out is None:
-        out = torch.empty((B, Hq, Sq, v.shape[-1]), dtype=torch.float32, device=q.device)
+        out = torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=q.device)
     need = _lib.load().bsa_attention_workspace_bytes(shape, Cq, Ck)
     if need == 0:
         raise _lib.BsaError("bsa_attention_workspace_bytes", _lib.BSA_ERR_UNSUPPORTED, _lib.detail())
@@ -116,8 +150,11 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
 def antidiagonal_block_scores(q, k, block=128, stride=16, logit_scale=None):
     """XAttention block-mass estimate: fp32 (B, Hq, S/block, S/block), rows sum to 1.
     q: (B,Hq,S,D), k: (B,Hkv,S,D) bf16 with S a multiple of ``block`` (the caller pads)."""
-    _need_cuda(q, k)
+    _expect_qkv(q, k)
     B, Hq, S, D = q.shape
+    if k.shape[2] != S:
+        raise ValueError(f"k has {k.shape[2]} tokens, q has {S}")
+    _need_cuda(q, k)
     nb = S // block
     scores = torch.empty((B, Hq, nb, nb), dtype=torch.float32, device=q.device)
     call("bsa_antidiagonal_block_scores", _ptr(q), _ptr(k), make_shape(q, k), int(block),
@@ -128,6 +165,7 @@ def antidiagonal_block_scores(q, k, block=128, stride=16, logit_scale=None):
 def top_p_block_mask(scores, tau, return_ties=False):
     """Per-row top-p selection over fp32 (B,H,Nq,Nk) scores; ``tau`` is a float or an
     (H,) sequence/tensor. Returns a uint8 mask (and uint8 tie flags (B,H,Nq))."""
+    _expect(scores, "scores", (torch.float32,), (4,))
     _need_cuda(scores)
     B, H, Nq, Nk = scores.shape
     t = torch.as_tensor(tau, dtype=torch.float32).reshape(-1).to(scores.device)
@@ -144,8 +182,13 @@ def select_probe_rows(labels, C, M, q=None):
     """SparsePR probe rows. Without ``q``: head-agnostic middle-out members, (M,) int32
     indices and (M,) fp32 weights. With ``q`` (B,Hq,S,D): per-head members nearest to
     their cluster's mean query, (B,Hq,M) indices and weights."""
-    _need_cuda(labels, q)
+    _expect(labels, "labels", (torch.int32,), (1,))
     S = labels.shape[0]
+    if q is not None:
+        _expect(q, "q", tuple(_DT), (4,))
+        if q.shape[2] != S:
+            raise ValueError(f"q has {q.shape[2]} tokens, labels {S}")
+    _need_cuda(labels, q)
     dev = labels.device
     if q is not None:
         B, Hq = q.shape[:2]
@@ -167,8 +210,13 @@ def select_probe_rows(labels, C, M, q=None):
 
 def probe_dense_attention(q, k, v, probe_idx, scale=None, workspace=None):
     """Exact attention of the probe rows over every key: fp32 (B, Hq, M, D)."""
-    _need_cuda(q, k, v, probe_idx)
+    _expect_qkv(q, k, v)
     B, Hq, S, D = q.shape
+    _expect(probe_idx, "probe_idx", (torch.int32,), (1, 3))
+    if probe_idx.dim() == 3 and tuple(probe_idx.shape[:2]) != (B, Hq):
+        raise ValueError(f"probe_idx: shape {tuple(probe_idx.shape)}, expected (M,) or ({B}, {Hq}, M)")
+    _expect_workspace(workspace)
+    _need_cuda(q, k, v, probe_idx, workspace)
     per_head = 1 if probe_idx.dim() == 3 else 0
     M = probe_idx.shape[-1]
     shape = make_shape(q, k)
@@ -184,9 +232,16 @@ def probe_dense_attention(q, k, v, probe_idx, scale=None, workspace=None):
 
 def probe_residual_correction(out, o_probe, probe_idx, weights, rank=16, lam=0.1, workspace=None):
     """SparsePR repair of ``out`` (fp32 (B,H,S,D), updated in place and returned)."""
-    _need_cuda(out, o_probe, probe_idx, weights)
+    _expect(out, "out", (torch.float32,), (4,))
     B, H, S, D = out.shape
+    _expect(probe_idx, "probe_idx", (torch.int32,), (1, 3))
     M = probe_idx.shape[-1]
+    if probe_idx.dim() == 3 and tuple(probe_idx.shape) != (B, H, M):
+        raise ValueError(f"probe_idx: shape {tuple(probe_idx.shape)}, expected (M,) or ({B}, {H}, M)")
+    _expect(weights, "weights", (torch.float32,), None, tuple(probe_idx.shape))
+    _expect(o_probe, "o_probe", (torch.float32,), (4,), (B, H, M, D))
+    _expect_workspace(workspace)
+    _need_cuda(out, o_probe, probe_idx, weights, workspace)
     per_head = 1 if probe_idx.dim() == 3 else 0
     need = _lib.load().bsa_repair_workspace_bytes(B, H, S, D, int(M))
     if workspace is None or workspace.numel() < need:
@@ -213,6 +268,11 @@ class MaskCache:
 
     def should_refresh(self, q, k, sync=True):
         """Device uint8 (B,H) refresh flags; with ``sync`` also the host count."""
+        B, H, _, _, D = self.shape
+        _expect(q, "q", tuple(_DT), (4,))
+        if q.shape[0] != B or q.shape[1] != H or q.shape[3] != D:
+            raise ValueError(f"q: shape {tuple(q.shape)} does not fit the cache ({B}, {H}, S, {D})")
+        _expect(k, "k", (q.dtype,), (4,), tuple(q.shape))
         _need_cuda(q, k)
         n = ctypes.c_int(0)
         call("bsa_mask_cache_should_refresh", _ptr(self.state), _ptr(q), _ptr(k), make_shape(q, k),
@@ -224,6 +284,8 @@ class MaskCache:
         """Cached mask with the refreshed heads replaced by ``new_mask`` (or None)."""
         nm = None
         if new_mask is not None:
+            B, H, Cq, Ck, _ = self.shape
+            _expect(new_mask, "new_mask", (torch.bool, torch.uint8), (4,), (B, H, Cq, Ck))
             nm = new_mask.to(torch.uint8).contiguous()
             _need_cuda(nm)
         call("bsa_mask_cache_update", _ptr(self.state), _ptr(nm), _ptr(self.refresh),

@@ -1,0 +1,79 @@
+"""CPU: the Python binding's dtype and shape checks.
+
+The C ABI takes plain pointers, so a tensor of the wrong element type or size would be
+read or written past its end inside the kernels. The binding rejects such arguments
+before anything reaches the library; these checks run before the device check, so they
+are exercised here with CPU tensors (a well-formed CPU call then fails on the device).
+"""
+
+import pytest
+import torch
+
+import block_sparse_attention_tcgen05_b200 as bsa
+
+B, H, HKV, S, D, C, M = 1, 4, 2, 256, 64, 4, 8
+
+
+def _qkv(dtype=torch.bfloat16):
+    return (torch.zeros(B, H, S, D, dtype=dtype), torch.zeros(B, HKV, S, D, dtype=dtype),
+            torch.zeros(B, HKV, S, D, dtype=dtype))
+
+
+def _labels(n=S):
+    return torch.zeros(n, dtype=torch.int32)
+
+
+def _raises(match, fn, *args, **kw):
+    with pytest.raises(ValueError, match=match):
+        fn(*args, **kw)
+
+
+def test_attention_arguments():
+    q, k, v = _qkv()
+    lab, mask = _labels(), torch.ones(C, C, dtype=torch.uint8)
+    f = bsa.centroid_compensated_attention
+    _raises("q: dtype", f, q.half(), k, v, lab, lab, mask)
+    _raises("k: dtype", f, q, k.float(), v, lab, lab, mask)
+    _raises("v: shape", f, q, k, v[:, :, :128], lab, lab, mask)
+    _raises("k: shape", f, q, torch.zeros(B, 3, S, D, dtype=q.dtype), v, lab, lab, mask)
+    _raises("q_labels: shape", f, q, k, v, _labels(S - 1), lab, mask)
+    _raises("k_labels: dtype", f, q, k, v, lab, lab.long(), mask)
+    _raises("out: dtype", f, q, k, v, lab, lab, mask, out=torch.zeros(B, H, S, D, dtype=q.dtype))
+    _raises("workspace: dtype", f, q, k, v, lab, lab, mask, workspace=torch.zeros(16))
+    _raises("CUDA tensors only", f, q, k, v, lab, lab, mask)
+
+
+def test_scoring_and_top_p_arguments():
+    q, k, _ = _qkv()
+    _raises("k has", bsa.antidiagonal_block_scores, q, k[:, :, :128])
+    _raises("k: dtype", bsa.antidiagonal_block_scores, q, k.float())
+    _raises("CUDA tensors only", bsa.antidiagonal_block_scores, q, k)
+    _raises("scores: dtype", bsa.top_p_block_mask, torch.zeros(1, H, 2, 2, dtype=torch.float64), 0.9)
+    _raises("scores: 3 dimensions", bsa.top_p_block_mask, torch.zeros(H, 2, 2), 0.9)
+    _raises("CUDA tensors only", bsa.top_p_block_mask, torch.zeros(1, H, 2, 2), 0.9)
+
+
+def test_probe_arguments():
+    q, k, v = _qkv()
+    _raises("labels: dtype", bsa.select_probe_rows, _labels().long(), C, M)
+    _raises("q has", bsa.select_probe_rows, _labels(), C, M, q=q[:, :, :128])
+    _raises("CUDA tensors only", bsa.select_probe_rows, _labels(), C, M)
+    idx = torch.zeros(M, dtype=torch.int32)
+    _raises("probe_idx: dtype", bsa.probe_dense_attention, q, k, v, idx.long())
+    _raises("probe_idx: shape", bsa.probe_dense_attention, q, k, v,
+            torch.zeros(B, H + 1, M, dtype=torch.int32))
+    _raises("CUDA tensors only", bsa.probe_dense_attention, q, k, v, idx)
+
+
+def test_repair_arguments():
+    out = torch.zeros(B, H, S, D)
+    op = torch.zeros(B, H, M, D)
+    idx = torch.zeros(M, dtype=torch.int32)
+    w = torch.full((M,), 1.0 / M)
+    f = bsa.probe_residual_correction
+    _raises("out: dtype", f, out.bfloat16(), op, idx, w)
+    _raises("o_probe: shape", f, out, op[:, :, :4], idx, w)
+    _raises("weights: shape", f, out, op, idx, w[:4])
+    _raises("weights: dtype", f, out, op, idx, w.double())
+    _raises("probe_idx: shape", f, out, op, torch.zeros(B, H + 1, M, dtype=torch.int32), w)
+    _raises("CUDA tensors only", f, out, op, idx, w)
