@@ -84,6 +84,15 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def roofline_peak(peaks, region_s):
+    """The bf16 peak a kernel timed inside a region of ``region_s`` seconds is held to:
+    the burst figure for a region shorter than the seconds-long loop the sustained
+    figure was measured over (the clocks have not settled under the power cap yet),
+    the sustained one otherwise. Returns (key, TFLOP/s)."""
+    key = "bf16_tflops" if region_s < 2.0 else "bf16_tflops_sustained"
+    return key, float(peaks.get(key, peaks.get("bf16_tflops")))
+
+
 ATTN_SECTION = b"// ============================================================== attention kernel"
 
 
@@ -414,7 +423,7 @@ def main():
 
     if rank == 0:
         peaks, src = measured_peaks()
-        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        peak_key, peak = roofline_peak(peaks, ms * args.steps * 1e-3)
         achieved = flop / (attn_ms_launch * 1e-3) / 1e12
         line = {
             "metric": METRIC,
@@ -431,6 +440,7 @@ def main():
             "dtype": "bf16",
             "data": "synthetic",
             "pct_of_bf16_peak": 100.0 * (flop / (ms * 1e-3) / 1e12) / peak,
+            "pct_of_bf16_peak_basis": peak_key,
             "config": {
                 "workload": WORKLOAD,
                 "B": 1, "H": nh, "S": S, "D": D, "clusters": C,
@@ -446,8 +456,9 @@ def main():
                 "bound": "tensor",
                 "achieved": achieved,
                 "peak": peak,
-                "peak_source": f"bf16_tflops_sustained of {src} (MEASURED_PEAKS.json)"
-                if src == "measured" else "fallback sustained bf16",
+                "peak_source": f"{peak_key} of {src} (MEASURED_PEAKS.json); timed region "
+                               f"{ms * args.steps:.0f} ms"
+                if src == "measured" else f"fallback {peak_key}",
                 "unit": "TFLOP/s",
                 "frac": achieved / peak,
                 "traffic": recorded_traffic(),

@@ -428,6 +428,10 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   for (int k = tid; k < 128; k += nt) sel[k] = -1;
   __syncthreads();
   // 2. standardised probe rows Zt = [(x - mu) / sigma, 1] and residuals R = o_probe - x
+  // A probe index outside [0, S) is reported in the device status word (site 70) and
+  // clamped, so that the reads stay inside this head's rows.
+  for (int m = tid; m < M; m += nt)
+    if (idx[m] < 0 || idx[m] >= S) report_device_error(kStatusBadLabel, 70);
   for (int e = tid; e < M * D; e += nt) {
     const int m = e / D, d = e % D;
     int row = idx[m];
@@ -809,6 +813,22 @@ RepairLayout carve_repair(int BH, int D, int M, int rank, void* ws) {
 
 }  // namespace bsa
 
+namespace bsa {
+// Argument checks of the repair, shared by the workspace and the allocation-free entry
+// points so that both return the same status for the same arguments.
+int validate_repair_args(const float* out, const float* o_probe, const int32_t* probe_idx,
+                         const float* weights, int B, int H, int S, int D, int M, int rank,
+                         float lam) {
+  if (!out || !o_probe || !probe_idx || !weights) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || H <= 0 || S <= 0 || M <= 0) return fail(BSA_ERR_INVALID_ARG, "bad sizes");
+  if (D != 64 && D != 128) return fail(BSA_ERR_UNSUPPORTED, "head dim %d", D);
+  if (M > 1024) return fail(BSA_ERR_UNSUPPORTED, "M %d > 1024", M);
+  if (rank < 1 || rank > D) return fail(BSA_ERR_INVALID_ARG, "rank %d outside [1, D]", rank);
+  if (!(lam >= 0.f)) return fail(BSA_ERR_INVALID_ARG, "lambda must be >= 0");
+  return BSA_OK;
+}
+}  // namespace bsa
+
 extern "C" size_t bsa_repair_workspace_bytes(int B, int H, int S, int D, int M) {
   if (B <= 0 || H <= 0 || S <= 0 || (D != 64 && D != 128) || M <= 0 || M > 1024) return 0;
   return bsa::carve_repair(B * H, D, M, D, nullptr).bytes;
@@ -821,17 +841,12 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
                                              size_t workspace_bytes, void* stream) {
   using namespace bsa;
   cudaStream_t st = as_stream(stream);
-  if (!out || !o_probe || !probe_idx || !weights) return fail(BSA_ERR_INVALID_ARG, "null pointer");
-  if (B <= 0 || H <= 0 || S <= 0 || M <= 0) return fail(BSA_ERR_INVALID_ARG, "bad sizes");
-  if (D != 64 && D != 128) return fail(BSA_ERR_UNSUPPORTED, "head dim %d", D);
-  if (M > 1024) return fail(BSA_ERR_UNSUPPORTED, "M %d > 1024", M);
-  if (rank < 1 || rank > D) return fail(BSA_ERR_INVALID_ARG, "rank %d outside [1, D]", rank);
-  if (!(lam >= 0.f)) return fail(BSA_ERR_INVALID_ARG, "lambda must be >= 0");
+  int rc = validate_repair_args(out, o_probe, probe_idx, weights, B, H, S, D, M, rank, lam);
+  if (rc) return rc;
   const int BH = B * H;
   RepairLayout L = carve_repair(BH, D, M, rank, workspace);
   if (!workspace || workspace_bytes < L.bytes)
     return fail(BSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", workspace_bytes, L.bytes);
-  int rc;
   column_stats_kernel<<<dim3(kStatSplit, BH), 256, 0, st>>>(out, S, D, L.psum, L.psq);
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "column_stats_kernel"))) return rc;

@@ -53,16 +53,16 @@ extern "C" int bsa_probe_residual_correction_noalloc(float* out, const float* o_
                                                      int H, int S, int D, int M, int rank,
                                                      float lam, void* stream) {
   using namespace bsa;
+  int rc = validate_repair_args(out, o_probe, probe_idx, weights, B, H, S, D, M, rank, lam);
+  if (rc) return rc;
   const size_t need = bsa_repair_workspace_bytes(B, H, S, D, M);
-  if (need == 0)
-    return fail(BSA_ERR_INVALID_ARG, "bad sizes (B=%d H=%d S=%d D=%d M=%d)", B, H, S, D, M);
   if (need > kNoAllocRepairScratchBytes)
     return fail(BSA_ERR_UNSUPPORTED,
                 "this repair needs %zu bytes of scratch; the built-in buffer holds %zu bytes "
                 "(16 MiB): use bsa_probe_residual_correction with a workspace",
                 need, kNoAllocRepairScratchBytes);
   void* scratch = nullptr;
-  int rc = noalloc_scratch(&scratch);
+  rc = noalloc_scratch(&scratch);
   if (rc) return rc;
   // Every scratch word the repair reads is written earlier in the same call, so the
   // buffer needs no clearing between calls.

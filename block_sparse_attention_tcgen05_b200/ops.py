@@ -24,11 +24,27 @@ def _ptr(t):
 
 
 def _need_cuda(*ts):
-    for t in ts:
-        if t is not None and not t.is_cuda:
+    """Every tensor passed to one call must sit on one device (the library launches on
+    the current device and reads its arguments as plain pointers: a tensor on another
+    GPU would be read through a peer address without peer access), be a CUDA tensor and
+    be contiguous."""
+    present = [t for t in ts if t is not None]
+    devs = {t.device for t in present}
+    if len(devs) > 1:
+        raise ValueError(f"all tensors of one call must be on the same device, got "
+                         f"{sorted(str(d) for d in devs)}")
+    for t in present:
+        if not t.is_cuda:
             raise ValueError("libbsa operates on CUDA tensors only")
-        if t is not None and not t.is_contiguous():
+        if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+
+
+def _call_on(dev, name, *args):
+    """Call an entry point with ``dev`` as the current CUDA device, so that the library
+    launches on the device whose stream it is given."""
+    with torch.cuda.device(dev):
+        return call(name, *args)
 
 
 def _expect(t, name, dtypes=None, ndims=None, shape=None):
@@ -86,7 +102,7 @@ def tile_labels(T, H, W, tile, device="cuda"):
     """Labels of a T×H×W token grid cut into ``tile`` boxes: (int32 (T·H·W,), n_tiles)."""
     labels = torch.empty(T * H * W, dtype=torch.int32, device=device)
     n = ctypes.c_int(0)
-    call("bsa_tile_labels", T, H, W, int(tile[0]), int(tile[1]), int(tile[2]), _ptr(labels),
+    _call_on(labels.device, "bsa_tile_labels", T, H, W, int(tile[0]), int(tile[1]), int(tile[2]), _ptr(labels),
          ctypes.byref(n), _stream(labels.device))
     return labels, n.value
 
@@ -103,17 +119,17 @@ def _mask_strides(block_mask, B, H, Cq, Ck):
         m = m.to(torch.uint8)
     if m.dtype != torch.uint8:
         raise ValueError("block_mask must be bool or uint8")
-    m = m.contiguous()
-    if m.dim() == 2:
-        m = m.view(1, 1, Cq, Ck)
-    elif m.dim() == 3:
-        m = m.view(1, m.shape[0], Cq, Ck)
+    if m.dim() not in (2, 3, 4):
+        raise ValueError(f"block_mask: {m.dim()} dimensions, expected 2, 3 or 4")
     if tuple(m.shape[-2:]) != (Cq, Ck):
         raise ValueError(f"block_mask trailing dims {tuple(m.shape[-2:])} != ({Cq},{Ck})")
+    lead = (1,) * (4 - m.dim()) + tuple(m.shape[:-2])
+    if lead[0] not in (1, B) or lead[1] not in (1, H):
+        raise ValueError(f"block_mask leading dims {tuple(m.shape[:-2])} must be 1 or (B, H) "
+                         f"= ({B}, {H})")
+    m = m.contiguous().view(*lead, Cq, Ck)
     bs = Cq * Ck * m.shape[1] if m.shape[0] > 1 else 0
     hs = Cq * Ck if m.shape[1] > 1 else 0
-    if (m.shape[0] not in (1, B)) or (m.shape[1] not in (1, H)):
-        raise ValueError("block_mask leading dims must be 1 or (B, H)")
     return m, bs, hs
 
 
@@ -129,11 +145,11 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
     if out is not None:
         _expect(out, "out", (torch.float32,), (4,), (B, Hq, Sq, D))
     _expect_workspace(workspace)
-    _need_cuda(q, k, v, q_labels, k_labels, block_mask, out, workspace)
     Cq = int(block_mask.shape[-2]) if Cq is None else int(Cq)
     Ck = int(block_mask.shape[-1]) if Ck is None else int(Ck)
-    shape = make_shape(q, k)
     m, bs, hs = _mask_strides(block_mask, B, Hq, Cq, Ck)
+    _need_cuda(q, k, v, q_labels, k_labels, m, out, workspace)
+    shape = make_shape(q, k)
     if out is None:
         out = torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=q.device)
     need = _lib.load().bsa_attention_workspace_bytes(shape, Cq, Ck)
@@ -141,7 +157,7 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
         raise _lib.BsaError("bsa_attention_workspace_bytes", _lib.BSA_ERR_UNSUPPORTED, _lib.detail())
     if workspace is None or workspace.numel() < need:
         workspace = _workspace(need, q.device)
-    call("bsa_centroid_compensated_attention", _ptr(q), _ptr(k), _ptr(v), shape, _ptr(q_labels),
+    _call_on(q.device, "bsa_centroid_compensated_attention", _ptr(q), _ptr(k), _ptr(v), shape, _ptr(q_labels),
          Cq, _ptr(k_labels), Ck, _ptr(m), bs, hs, float(scale or 0.0), 1 if compensate else 0,
          _ptr(out), _ptr(workspace), workspace.numel(), _stream(q.device))
     return out
@@ -157,7 +173,7 @@ def antidiagonal_block_scores(q, k, block=128, stride=16, logit_scale=None):
     _need_cuda(q, k)
     nb = S // block
     scores = torch.empty((B, Hq, nb, nb), dtype=torch.float32, device=q.device)
-    call("bsa_antidiagonal_block_scores", _ptr(q), _ptr(k), make_shape(q, k), int(block),
+    _call_on(q.device, "bsa_antidiagonal_block_scores", _ptr(q), _ptr(k), make_shape(q, k), int(block),
          int(stride), float(logit_scale or 0.0), _ptr(scores), _stream(q.device))
     return scores
 
@@ -173,7 +189,7 @@ def top_p_block_mask(scores, tau, return_ties=False):
         raise ValueError("tau must be a scalar or have H entries")
     mask = torch.empty((B, H, Nq, Nk), dtype=torch.uint8, device=scores.device)
     ties = torch.empty((B, H, Nq), dtype=torch.uint8, device=scores.device)
-    call("bsa_top_p_block_mask", _ptr(scores), B, H, Nq, Nk, _ptr(t), t.numel(), _ptr(mask),
+    _call_on(scores.device, "bsa_top_p_block_mask", _ptr(scores), B, H, Nq, Nk, _ptr(t), t.numel(), _ptr(mask),
          _ptr(ties), _stream(scores.device))
     return (mask, ties) if return_ties else mask
 
@@ -203,7 +219,7 @@ def select_probe_rows(labels, C, M, q=None):
         w = torch.empty((M,), dtype=torch.float32, device=dev)
     need = _lib.load().bsa_probe_select_workspace_bytes(S, int(C), n_heads)
     ws = _workspace(need, dev)
-    call("bsa_select_probe_rows", _ptr(labels), S, int(C), int(M), _ptr(q), shape, _ptr(idx),
+    _call_on(dev, "bsa_select_probe_rows", _ptr(labels), S, int(C), int(M), _ptr(q), shape, _ptr(idx),
          _ptr(w), _ptr(ws), ws.numel(), _stream(dev))
     return idx, w
 
@@ -224,7 +240,7 @@ def probe_dense_attention(q, k, v, probe_idx, scale=None, workspace=None):
     need = _lib.load().bsa_probe_attention_workspace_bytes(shape, int(M))
     if workspace is None or workspace.numel() < need:
         workspace = _workspace(need, q.device)
-    call("bsa_probe_dense_attention", _ptr(q), _ptr(k), _ptr(v), shape, _ptr(probe_idx), int(M),
+    _call_on(q.device, "bsa_probe_dense_attention", _ptr(q), _ptr(k), _ptr(v), shape, _ptr(probe_idx), int(M),
          per_head, float(scale or 0.0), _ptr(out), _ptr(workspace), workspace.numel(),
          _stream(q.device))
     return out
@@ -246,7 +262,7 @@ def probe_residual_correction(out, o_probe, probe_idx, weights, rank=16, lam=0.1
     need = _lib.load().bsa_repair_workspace_bytes(B, H, S, D, int(M))
     if workspace is None or workspace.numel() < need:
         workspace = _workspace(need, out.device)
-    call("bsa_probe_residual_correction", _ptr(out), _ptr(o_probe), _ptr(probe_idx), _ptr(weights),
+    _call_on(out.device, "bsa_probe_residual_correction", _ptr(out), _ptr(o_probe), _ptr(probe_idx), _ptr(weights),
          per_head, B, H, S, D, int(M), int(rank), float(lam), _ptr(workspace), workspace.numel(),
          _stream(out.device))
     return out
@@ -263,7 +279,7 @@ class MaskCache:
         self.refresh = torch.empty((B, H), dtype=torch.uint8, device=device)
         self.drift = torch.empty((B, H), dtype=torch.float32, device=device)
         self.mask = torch.empty((B, H, Cq, Ck), dtype=torch.uint8, device=device)
-        call("bsa_mask_cache_init", _ptr(self.state), B, H, Cq, Ck, D, float(delta),
+        _call_on(self.state.device, "bsa_mask_cache_init", _ptr(self.state), B, H, Cq, Ck, D, float(delta),
              1 if relative else 0, float(gate_lo), float(gate_hi), _stream(self.state.device))
 
     def should_refresh(self, q, k, sync=True):
@@ -273,9 +289,9 @@ class MaskCache:
         if q.shape[0] != B or q.shape[1] != H or q.shape[3] != D:
             raise ValueError(f"q: shape {tuple(q.shape)} does not fit the cache ({B}, {H}, S, {D})")
         _expect(k, "k", (q.dtype,), (4,), tuple(q.shape))
-        _need_cuda(q, k)
+        _need_cuda(q, k, self.state)
         n = ctypes.c_int(0)
-        call("bsa_mask_cache_should_refresh", _ptr(self.state), _ptr(q), _ptr(k), make_shape(q, k),
+        _call_on(q.device, "bsa_mask_cache_should_refresh", _ptr(self.state), _ptr(q), _ptr(k), make_shape(q, k),
              _ptr(self.refresh), _ptr(self.drift), ctypes.byref(n) if sync else None,
              _stream(q.device))
         return (self.refresh, n.value) if sync else self.refresh
@@ -287,10 +303,10 @@ class MaskCache:
             B, H, Cq, Ck, _ = self.shape
             _expect(new_mask, "new_mask", (torch.bool, torch.uint8), (4,), (B, H, Cq, Ck))
             nm = new_mask.to(torch.uint8).contiguous()
-            _need_cuda(nm)
-        call("bsa_mask_cache_update", _ptr(self.state), _ptr(nm), _ptr(self.refresh),
+            _need_cuda(nm, self.state)
+        _call_on(self.state.device, "bsa_mask_cache_update", _ptr(self.state), _ptr(nm), _ptr(self.refresh),
              _ptr(self.mask), _stream(self.state.device))
         return self.mask
 
     def reset(self):
-        call("bsa_mask_cache_reset", _ptr(self.state), _stream(self.state.device))
+        _call_on(self.state.device, "bsa_mask_cache_reset", _ptr(self.state), _stream(self.state.device))

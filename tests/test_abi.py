@@ -120,3 +120,26 @@ def test_python_binding_refuses_cpu_tensors():
     lab = torch.zeros(128, dtype=torch.int32)
     with pytest.raises(ValueError):
         bsa.centroid_compensated_attention(q, q, q, lab, lab, torch.ones(1, 1, dtype=torch.uint8))
+
+
+def test_noalloc_repair_returns_the_workspace_entry_points_status(lib):
+    """The allocation-free repair runs the same argument checks, with the same status
+    codes, as bsa_probe_residual_correction before it looks at its buffer's size."""
+    fake = fake_ptr()
+    null = ctypes.c_void_p(0)
+    cases = [
+        ((0, 1, 1, 100, 96, 8, 16, 0.1), _lib.BSA_ERR_UNSUPPORTED),    # head dim 96
+        ((0, 1, 1, 100, 64, 1025, 16, 0.1), _lib.BSA_ERR_UNSUPPORTED),  # M > 1024
+        ((0, 1, 1, 100, 64, 8, 65, 0.1), _lib.BSA_ERR_INVALID_ARG),     # rank > D
+        ((0, 1, 1, 100, 64, 8, 16, -1.0), _lib.BSA_ERR_INVALID_ARG),    # lambda < 0
+        ((0, 1, 0, 100, 64, 8, 16, 0.1), _lib.BSA_ERR_INVALID_ARG),     # H = 0
+    ]
+    for (ph, B, H, S, D, M, r, lam), want in cases:
+        st_ws = lib.bsa_probe_residual_correction(fake, fake, fake, fake, ph, B, H, S, D, M, r,
+                                                  lam, fake, 1 << 30, null)
+        st_na = lib.bsa_probe_residual_correction_noalloc(fake, fake, fake, fake, ph, B, H, S, D,
+                                                          M, r, lam, null)
+        assert st_ws == st_na == want, (D, M, r, lam, st_ws, st_na)
+    # null output pointer: both INVALID_ARG
+    assert lib.bsa_probe_residual_correction_noalloc(null, fake, fake, fake, 0, 1, 1, 100, 64, 8,
+                                                     16, 0.1, null) == _lib.BSA_ERR_INVALID_ARG

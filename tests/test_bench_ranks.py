@@ -53,3 +53,14 @@ def test_single_rank_passthrough():
     import bench
     assert bench.max_over_ranks([3.0, 4.0], "cpu", 1) == [3.0, 4.0]
     assert bench.weak_scaling_tflops(1e12, 1, 1.0) == pytest.approx(1000.0)
+
+
+def test_roofline_peak_follows_the_timed_region():
+    """A kernel timed inside a sub-second region is held to the burst bf16 peak; only a
+    region of seconds (the length of the sustained measurement's loop) takes the
+    sustained figure."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = {"bf16_tflops": 1653.8, "bf16_tflops_sustained": 1383.1}
+    assert bench.roofline_peak(peaks, 0.5) == ("bf16_tflops", 1653.8)
+    assert bench.roofline_peak(peaks, 4.0) == ("bf16_tflops_sustained", 1383.1)

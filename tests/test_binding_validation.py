@@ -77,3 +77,40 @@ def test_repair_arguments():
     _raises("weights: dtype", f, out, op, idx, w.double())
     _raises("probe_idx: shape", f, out, op, torch.zeros(B, H + 1, M, dtype=torch.int32), w)
     _raises("CUDA tensors only", f, out, op, idx, w)
+
+
+def test_tensors_on_different_devices_are_refused():
+    """Every tensor of one call must be on one device: the library reads plain pointers
+    on the current device. A CPU tensor mixed with a tensor on another device (the meta
+    device stands in for a second GPU here) is refused before any other device check."""
+    q, k, v = _qkv()
+    kmeta = torch.empty(k.shape, dtype=k.dtype, device="meta")
+    lab, mask = _labels(), torch.ones(C, C, dtype=torch.uint8)
+    _raises("same device", bsa.centroid_compensated_attention, q, kmeta, v, lab, lab, mask)
+    _raises("same device", bsa.centroid_compensated_attention, q, k, v, lab, lab,
+            mask.to("meta"))
+    _raises("same device", bsa.antidiagonal_block_scores, q, kmeta)
+    idx = torch.zeros(M, dtype=torch.int32)
+    _raises("same device", bsa.probe_dense_attention, q, k, v, idx.to("meta"))
+    out = torch.zeros(B, H, S, D)
+    op = torch.zeros(B, H, M, D)
+    w = torch.full((M,), 1.0 / M)
+    _raises("same device", bsa.probe_residual_correction, out, op.to("meta"), idx, w)
+    _raises("same device", bsa.centroid_compensated_attention, q, k, v, lab, lab, mask,
+            workspace=torch.empty(16, dtype=torch.uint8, device="meta"))
+
+
+def test_mask_shapes_are_checked_before_any_reshape():
+    """A mask whose trailing dims are not (Cq, Ck) is refused even when its element
+    count matches; leading dims must be 1, H or (B, H)."""
+    q, k, v = _qkv()
+    lab = _labels()
+    f = bsa.centroid_compensated_attention
+    _raises("trailing dims", f, q, k, v, lab, lab, torch.ones(H, 2, 8, dtype=torch.uint8),
+            Cq=4, Ck=4)
+    _raises("trailing dims", f, q, k, v, lab, lab, torch.ones(2, 8, dtype=torch.uint8), Cq=4,
+            Ck=4)
+    _raises("leading dims", f, q, k, v, lab, lab, torch.ones(H + 1, C, C, dtype=torch.uint8))
+    _raises("leading dims", f, q, k, v, lab, lab, torch.ones(2, H, C, C, dtype=torch.uint8))
+    _raises("dimensions", f, q, k, v, lab, lab, torch.ones(1, 1, 1, C, C, dtype=torch.uint8))
+    _raises("must be bool or uint8", f, q, k, v, lab, lab, torch.ones(C, C))

@@ -54,15 +54,35 @@ def test_probe_rows_fewer_probes_than_clusters_and_uneven():
     idx, w = oracle.select_probe_rows(lab, 4)
     assert [lab[i] for i in idx] == [0, 2, 5, 7]          # floor(i*10/4)
     assert np.isclose(w.sum(), 1)
+    # M = 14 >= C = 10: round-robin over the query clusters in ascending label order
+    # ("Sparse-block compensation", §What mlx-arsenal ships), each pass taking the next
+    # preferred member of every cluster that still has one. Cluster rows (offsets):
+    #   0: 0-4 (5)  1: 5 (1)  2: 6-7 (2)  3: 8-16 (9)  4: 17-19 (3)
+    #   5: 20-23 (4)  6: 24-27 (4)  7: 28-33 (6)  8: 34-35 (2)  9: 36 (1)
+    # Middle-out order ranks members by |2r - (n-1)|, ties to the lower rank r:
+    #   n=5 -> r 2,1,3,0,4;  n=2 -> r 0,1;  n=9 -> r 4,3,5,..;  n=3 -> r 1,0,2;
+    #   n=4 -> r 1,2,0,3;  n=6 -> r 2,3,1,4,..
+    # Pass 0 takes one row of every cluster: 2, 5, 6, 12, 18, 21, 25, 30, 34, 36.
+    # Pass 1 skips the exhausted clusters 1 and 9 and stops after four more rows, all
+    # from the first clusters in label order that still have members: 0 -> 1, 2 -> 7,
+    # 3 -> 11, 4 -> 17.
     idx, w = oracle.select_probe_rows(lab, 14)
+    np.testing.assert_array_equal(idx, [2, 5, 6, 12, 18, 21, 25, 30, 34, 36, 1, 7, 11, 17])
     owners = lab[idx]
-    assert np.bincount(owners, minlength=10).tolist() == [2, 1, 1, 2, 2, 2, 2, 2, 1, 1][:10] \
-        or len(idx) == 14
-    # weights are |G_a| / m_a normalised
-    m = np.bincount(owners, minlength=10)
-    sizes = np.bincount(lab)
-    raw = sizes[owners] / m[owners]
+    assert np.bincount(owners, minlength=10).tolist() == [2, 1, 2, 2, 2, 1, 1, 1, 1, 1]
+    # weights are |G_a| / m_a normalised: sizes 5,1,2,9,3,4,4,6,2,1 over probe counts
+    raw = np.array([5 / 2, 1, 2 / 2, 9 / 2, 3 / 2, 4, 4, 6, 2, 1, 5 / 2, 2 / 2, 9 / 2, 3 / 2])
     np.testing.assert_allclose(w, raw / raw.sum())
+    # exhaustion: M = 37 takes every row once (clusters drop out as they empty); a
+    # larger M cannot take more rows than exist
+    idx, w = oracle.select_probe_rows(lab, 37)
+    assert sorted(idx.tolist()) == list(range(37))
+    np.testing.assert_allclose(w, np.full(37, 1 / 37))
+    # passes 6, 7 and 8 only find members left in the 9-row cluster 3, whose middle-out
+    # order is r = 4,3,5,2,6,1,7,0,8: its ranks 6, 7, 8 are rows 8 + {7, 0, 8}
+    np.testing.assert_array_equal(idx[-3:], [15, 8, 16])
+    idx, _ = oracle.select_probe_rows(lab, 50)
+    assert len(idx) == 37
 
 
 def test_probe_rows_centroid_distance_brute_force():
@@ -78,6 +98,40 @@ def test_probe_rows_centroid_distance_brute_force():
             best2 = [rows[j] for j in np.argsort(d)[:2]]
             assert idx[0, h, a] == best2[0] and idx[0, h, 3 + a] == best2[1]
     np.testing.assert_allclose(w, 1 / 6)
+
+
+def test_probe_dense_attention_per_head_gqa_against_library_sdpa():
+    """Per-head probe rows under grouped-query attention ("Partition the Support,
+    Reconstruct the Residual": M query rows evaluated exactly against all keys, KV
+    heads shared by contiguous groups of query heads). Each (b, h) is checked against
+    torch's scaled_dot_product_attention on the rows probe_idx[b, h] of query head h and
+    KV head h // (Hq / Hkv). Hq = 6 over Hkv = 2 makes a wrong grouping (h % Hkv) or a
+    probe index taken from another head fail."""
+    import torch
+
+    g = np.random.default_rng(8)
+    B, Hq, Hkv, S, D, M = 2, 6, 2, 40, 8, 5
+    q = g.standard_normal((B, Hq, S, D))
+    k = g.standard_normal((B, Hkv, S, D))
+    v = g.standard_normal((B, Hkv, S, D))
+    pidx = g.integers(0, S, (B, Hq, M))
+    got = oracle.probe_dense_attention(q, k, v, pidx)
+    qt, kt, vt = (torch.from_numpy(x) for x in (q, k, v))
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // (Hq // Hkv)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qt[b, h, pidx[b, h]][None], kt[b, kv][None], vt[b, kv][None])[0]
+            np.testing.assert_allclose(got[b, h], ref.numpy(), atol=1e-12)
+    # shared rows (M,): the same rows in every head
+    rows = pidx[0, 0]
+    shared = oracle.probe_dense_attention(q, k, v, rows)
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // (Hq // Hkv)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qt[b, h, rows][None], kt[b, kv][None], vt[b, kv][None])[0]
+            np.testing.assert_allclose(shared[b, h], ref.numpy(), atol=1e-12)
 
 
 # ----------------------------------------------------------------------------- repair
