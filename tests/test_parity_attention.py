@@ -139,6 +139,20 @@ def test_video_static_tiles_full_size_sampled():
     rows = np.random.default_rng(12).choice(32760, 96, replace=False)
     ref = _ref(q, k, v, lab_ref, lab_ref, mask, C, C, rows=rows)
     _check(got[:, :, rows], ref)
+    # Coverage: one row in every 128-row query tile of the cluster-sorted order the
+    # kernel walks (tokens stably sorted by label), and one row of every cluster (the
+    # 35 partial 72-token edge tiles included), on four heads.
+    g = np.random.default_rng(13)
+    order = np.argsort(lab_ref, kind="stable")
+    cover = {int(order[t * 128 + g.integers(0, min(128, 32760 - t * 128))])
+             for t in range(-(-32760 // 128))}
+    for c in range(C):
+        cover.add(int(g.choice(np.nonzero(lab_ref == c)[0])))
+    cover = np.array(sorted(cover))
+    heads = [0, 13, 26, 39]
+    qh, kh, vh = (t[:, heads] for t in (q, k, v))
+    ref = _ref(qh, kh, vh, lab_ref, lab_ref, mask, C, C, rows=cover)
+    _check(got[:, heads][:, :, cover], ref)
 
 
 # Calls with at least 148 query-tile CTAs over all heads run without a key-range split

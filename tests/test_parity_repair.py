@@ -159,6 +159,22 @@ def test_sparsepr_video_workload_sampled():
     rep = out.cpu().numpy()
     assert bsa.device_status()[0] == 0
     qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+    # per-head centroid-distance probes (M = 64 < C = 256: the nearest member of cluster
+    # floor(i C / M)) against the oracle's selection: same clusters, and each chosen
+    # row's float64 distance to its cluster's mean query equals the oracle choice's
+    # (the GPU decides in fp32, so near-ties may pick another row at equal distance)
+    ridx, rw = oracle.select_probe_rows_centroid(qd, lab, 64)
+    gi = idx.cpu().numpy()
+    np.testing.assert_array_equal(lab[gi], lab[ridx])
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-6)
+    for h in range(24):
+        for m in range(64):
+            a = lab[ridx[0, h, m]]
+            mem = qd[0, h, a * 128:(a + 1) * 128]
+            c = mem.mean(0)
+            dg = np.linalg.norm(qd[0, h, gi[0, h, m]] - c)
+            dr = np.linalg.norm(qd[0, h, ridx[0, h, m]] - c)
+            assert abs(dg - dr) <= 1e-4 * max(dr, 1.0), (h, m, dg, dr)
     rows = np.random.default_rng(7).choice(S, 512, replace=False)
     # sparse rows against the oracle hard drop
     sp_ref = oracle.hard_drop_attention(qd, kd, vd, lab, lab, mask, rows=rows)
@@ -169,9 +185,81 @@ def test_sparsepr_video_workload_sampled():
     op_ref = oracle.probe_dense_attention(qd, kd, vd, idx_n)
     assert _rel_fro(op.cpu().numpy(), op_ref) <= 5e-3
     rep_ref = oracle.probe_residual_correction(sparse, op_ref, idx_n, w_n)
+    # the correction itself, element by element over every row: GPU (rep - sparse)
+    # against the oracle's (rep_ref - sparse) on the same sparse output and probes
+    assert _rel_fro(rep - sparse, rep_ref - sparse) <= 1e-3, _rel_fro(rep - sparse, rep_ref - sparse)
     dense_rows = oracle.dense_attention(qd, kd, vd, rows=rows)
     err_gpu = _rel_fro(rep[:, :, rows], dense_rows)
     err_ref = _rel_fro(rep_ref[:, :, rows], dense_rows)
     assert abs(err_gpu - err_ref) <= 1e-3, (err_gpu, err_ref)
     print(f"reconstruction error (sampled rows): hard drop {_rel_fro(sp_ref, dense_rows):.5f} "
           f"repaired oracle {err_ref:.5f} gpu {err_gpu:.5f}")
+
+
+def test_repair_recovers_a_planted_residual_at_video_scale():
+    """At the SparsePR video shape (H=24 over 8 KV heads, S=32768, D=128) the dense
+    output is planted as the GPU hard-drop output plus a residual that is exactly affine
+    in the standardised sparse output and lies in a rank-16 subspace ("Sparse-block
+    compensation", §SparsePR — probe-fitted residual repair: the residual is fitted from
+    the standardised sparse output and projected on the top residual directions). With
+    one probe per query cluster (M = 256 >= D + 1) and a ridge of 1e-4 the fit is
+    determined, so the repair must bring every row to the planted dense row; the GPU
+    correction must also equal the oracle's."""
+    bsa = _bsa()
+    grid = (16, 32, 64)
+    q, k, v, _ = wl.positional_qkv(1, 24, 8, grid, 128, ell=(3.0, 6.0, 8.0), amp=2.0,
+                                   dtype="bf16", seed=4, temperature_range=(0.5, 2.0))
+    S, D, r = 32768, 128, 16
+    lab = np.arange(S) // 128
+    mask = wl.nearest_pair_mask(wl.raster_block_centroids(grid, 128), 0.22)
+    lt = torch.as_tensor(lab, dtype=torch.int32).cuda()
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    out = bsa.centroid_compensated_attention(qc, kc, vc, lt, lt, torch.as_tensor(mask).cuda(),
+                                             compensate=False)
+    x = out.cpu().numpy().astype(np.float64)
+    g = np.random.default_rng(9)
+    planted = np.empty_like(x)
+    for h in range(24):
+        xh = x[0, h]
+        Zt = np.concatenate([oracle.standardise(xh), np.ones((S, 1))], 1)
+        U = np.linalg.qr(g.standard_normal((D, r)))[0]
+        Btrue = 0.05 * g.standard_normal((D + 1, r)) @ U.T
+        planted[0, h] = xh + Zt @ Btrue
+    idx, w = bsa.select_probe_rows(lt, 256, 256, q=qc)
+    gi = idx.cpu().numpy()
+    op = np.take_along_axis(planted, gi[..., None].astype(np.int64), axis=2).astype(np.float32)
+    sparse32 = out.cpu().numpy()
+    bsa.probe_residual_correction(out, torch.from_numpy(op).cuda(), idx, w, rank=r, lam=1e-4)
+    rep = out.cpu().numpy().astype(np.float64)
+    assert bsa.device_status()[0] == 0
+    corr_true = planted - x
+    err = _rel_fro(rep - x, corr_true)
+    assert err <= 2e-3, err
+    rep_ref = oracle.probe_residual_correction(sparse32, op, gi, w.cpu().numpy(), rank=r, lam=1e-4)
+    assert _rel_fro(rep - sparse32, rep_ref - sparse32) <= 1e-3
+    before = _rel_fro(x, planted)
+    after = _rel_fro(rep, planted)
+    print(f"planted residual: error before repair {before:.4e}, after {after:.4e}, "
+          f"correction error {err:.2e}")
+    assert after < 0.05 * before
+
+
+def test_repair_reports_out_of_range_probe_index():
+    """A probe index outside [0, S) is recorded in the device status word (the read is
+    clamped inside the head's rows, so nothing is read out of bounds); the status clears
+    on read and a following good call reports nothing."""
+    bsa = _bsa()
+    g = np.random.default_rng(10)
+    S, D, M = 256, 64, 16
+    out = torch.from_numpy(g.standard_normal((1, 1, S, D)).astype(np.float32)).cuda()
+    op = torch.from_numpy(g.standard_normal((1, 1, M, D)).astype(np.float32)).cuda()
+    w = torch.full((M,), 1.0 / M, device="cuda")
+    assert bsa.device_status()[0] == 0
+    bad = torch.arange(M, dtype=torch.int32, device="cuda")
+    bad[3] = S
+    bsa.probe_residual_correction(out, op, bad, w, rank=4)
+    st, where = bsa.device_status()
+    assert (st, where) == (-1, 70), (st, where)
+    bsa.probe_residual_correction(out, op, torch.arange(M, dtype=torch.int32, device="cuda"), w,
+                                  rank=4)
+    assert bsa.device_status() == (0, 0)

@@ -50,8 +50,9 @@ def test_top_p_kernel_bit_exact_on_identical_scores():
     bsa = _bsa()
     got, ties = bsa.top_p_block_mask(torch.from_numpy(sc).cuda(), torch.from_numpy(tau),
                                      return_ties=True)
-    ref, _ = oracle.top_p_block_mask(sc, tau, dtype=np.float32)
+    ref, ref_tie = oracle.top_p_block_mask(sc, tau, dtype=np.float32)
     np.testing.assert_array_equal(got.cpu().numpy().astype(bool), ref)
+    np.testing.assert_array_equal(ties.cpu().numpy().astype(bool), ref_tie)
     # ragged Nk (not a power of two), scalar tau
     sc2 = g.dirichlet(np.ones(245), size=(1, 2, 7)).astype(np.float32)
     got2 = bsa.top_p_block_mask(torch.from_numpy(sc2).cuda(), 0.9)
@@ -69,6 +70,35 @@ def test_top_p_kernel_bit_exact_on_identical_scores():
             np.testing.assert_array_equal(got3.argmax(-1), sc.argmax(-1))
 
 
+def test_top_p_tie_rows_reported():
+    """Rows built so that a decision is fragile: a running sum landing within 1e-5 of
+    tau, and a last kept score within 1e-5 of the first dropped one. The kernel's tie
+    flags equal the oracle's (float32 running sums on both sides) bit for bit, and so
+    do the masks."""
+    rows = np.array([
+        [0.5, 0.4, 0.1, 0.0],               # running sum 0.9 at rank 1: |0.9 - tau| = 0
+        [0.5, 0.399995, 0.100005, 0.0],     # 0.899995: within 1e-5 below tau
+        [0.5, 0.40002, 0.09998, 0.0],       # 0.90002: 2e-5 past tau, no tie
+        [0.6, 0.200005, 0.2, -0.0],         # kept 0.200005 vs dropped 0.2: gap 5e-6
+        [0.6, 0.21, 0.19, 0.0],             # gap 0.02, running sums far from tau: no tie
+        [0.25, 0.25, 0.25, 0.25],           # equal scores: index order decides
+    ], dtype=np.float32)
+    taus = np.array([0.9, 0.9, 0.9, 0.7, 0.7, 0.6], dtype=np.float32)
+    bsa = _bsa()
+    for r, t in zip(rows, taus):
+        sc = np.abs(r)[None, None, None, :]
+        got, ties = bsa.top_p_block_mask(torch.from_numpy(sc).cuda(), float(t), return_ties=True)
+        ref, ref_tie = oracle.top_p_block_mask(sc, float(t), dtype=np.float32)
+        np.testing.assert_array_equal(got.cpu().numpy().astype(bool), ref)
+        np.testing.assert_array_equal(ties.cpu().numpy().astype(bool), ref_tie)
+    want = [True, True, False, True, False, True]
+    got_all = []
+    for r, t in zip(rows, taus):
+        _, tie = oracle.top_p_block_mask(np.abs(r)[None, None, None, :], float(t), dtype=np.float32)
+        got_all.append(bool(tie.reshape(-1)[0]))
+    assert got_all == want, got_all
+
+
 def test_dynamic_mask_workload_scores_and_masks():
     """B=1, H=8, S=8192, D=64 bf16 with 1-D positional structure; block 128, stride 16,
     tau 0.9. Masks must match the float64 oracle chain bit for bit outside tie rows."""
@@ -78,7 +108,13 @@ def test_dynamic_mask_workload_scores_and_masks():
     got = _scores(q, k, 128, 16)
     ref = oracle.antidiagonal_block_scores(q.double().numpy(), k.double().numpy(), 128, 16)
     np.testing.assert_allclose(got, ref, atol=SCORE_ATOL, rtol=0)
-    m_gpu = bsa.top_p_block_mask(torch.from_numpy(got).cuda(), 0.9).cpu().numpy().astype(bool)
+    m_gpu_t, ties_gpu = bsa.top_p_block_mask(torch.from_numpy(got).cuda(), 0.9, return_ties=True)
+    m_gpu = m_gpu_t.cpu().numpy().astype(bool)
+    # on the GPU's own scores, decided in float32 on both sides: masks and tie flags
+    # bit for bit
+    m32, tie32 = oracle.top_p_block_mask(got, 0.9, dtype=np.float32)
+    np.testing.assert_array_equal(m_gpu, m32)
+    np.testing.assert_array_equal(ties_gpu.cpu().numpy().astype(bool), tie32)
     m_ref, tie = oracle.top_p_block_mask(ref, 0.9)
     diff_rows = (m_gpu != m_ref).any(-1)
     assert not (diff_rows & ~tie).any(), f"{int((diff_rows & ~tie).sum())} non-tie rows differ"
