@@ -40,6 +40,10 @@ D = 128
 DENSITY = 0.22
 WORKLOAD = ("video_static_tiles: B=1 H=40 S=32760 (21x30x52) D=128 bf16, 3x6x8 tile labels "
             "(245 clusters), nearest-22% tile-pair mask, SVG-EAR compensation")
+STA_WINDOW = (3, 3, 5)
+WORKLOAD_STA = ("video_static_tiles_sta: B=1 H=40 S=32760 (21x30x52) D=128 bf16, 3x6x8 tile "
+                "labels (245 clusters), sliding-tile window (3,3,5) tiles (19% of token pairs), "
+                "SVG-EAR compensation")
 METRIC = "effective TFLOP/s on executed pairs, centroid-compensated block-sparse attention at 40x32760x128"
 
 
@@ -53,6 +57,9 @@ def parse():
                    help="bounded CPU work for the oracle baseline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--mask", choices=["nearest", "sta"], default="nearest",
+                   help="nearest: the 22 %% of tile pairs nearest in (t, h, w) (default); sta: "
+                        "the recipe's sliding-tile window of STA_WINDOW tiles")
     p.add_argument("--heads", type=int, default=H,
                    help="number of heads (default 40; smaller only for profiler captures)")
     return p.parse_args()
@@ -292,8 +299,12 @@ def main():
     q, k, v = wl.positional_qkv_device(1, nh, nh, GRID, D, ell=(3.0, 6.0, 8.0), amp=2.0,
                                        seed=3 + 1000 * rank, device=dev)
     labels, C = bsa.tile_labels(*GRID, TILE, device=dev)
-    mask = torch.as_tensor(wl.nearest_pair_mask(wl.tile_centroids(GRID, TILE), DENSITY),
-                           dtype=torch.uint8, device=dev)
+    if args.mask == "sta":
+        n_tiles = tuple(-(-g // t) for g, t in zip(GRID, TILE))
+        mask = bsa.sliding_tile_block_mask(n_tiles, STA_WINDOW, device=dev)
+    else:
+        mask = torch.as_tensor(wl.nearest_pair_mask(wl.tile_centroids(GRID, TILE), DENSITY),
+                               dtype=torch.uint8, device=dev)
     cnt = torch.bincount(labels.long(), minlength=C).double()
     pairs = float(cnt @ mask.double() @ cnt) * nh
     S = q.shape[2]
@@ -442,7 +453,7 @@ def main():
             "pct_of_bf16_peak": 100.0 * (flop / (ms * 1e-3) / 1e12) / peak,
             "pct_of_bf16_peak_basis": peak_key,
             "config": {
-                "workload": WORKLOAD,
+                "workload": WORKLOAD_STA if args.mask == "sta" else WORKLOAD,
                 "B": 1, "H": nh, "S": S, "D": D, "clusters": C,
                 "executed_pairs_per_call": pairs,
                 "executed_pair_density": pairs / (nh * S * S),

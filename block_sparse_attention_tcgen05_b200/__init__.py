@@ -16,6 +16,7 @@ from .ops import (  # noqa: F401
     probe_dense_attention,
     probe_residual_correction,
     select_probe_rows,
+    sliding_tile_block_mask,
     tile_labels,
     top_p_block_mask,
 )

@@ -44,6 +44,7 @@ SIGNATURES = {
     "bsa_profile_enable": (_i, [_i]),
     "bsa_profile_read": (_i, [_i, ctypes.POINTER(ctypes.c_float), _ip]),
     "bsa_tile_labels": (_i, [_i, _i, _i, _i, _i, _i, _vp, _ip, _vp]),
+    "bsa_sliding_tile_block_mask": (_i, [_i, _i, _i, _i, _i, _i, _vp, _vp]),
     "bsa_antidiagonal_block_scores": (_i, [_vp, _vp, Shape, _i, _i, _f, _vp, _vp]),
     "bsa_top_p_block_mask": (_i, [_vp, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "bsa_attention_workspace_bytes": (_sz, [Shape, _i, _i]),

@@ -255,6 +255,168 @@ __global__ void __launch_bounds__(256) mask_bits_kernel(
   }
 }
 
+// ============================================================== query tile plan
+// The attention kernel computes every key group that any row of a 128-row query tile
+// keeps, for all 128 rows. With query rows in plain cluster order a tile straddles two
+// clusters whenever cluster sizes are not multiples of 128 (3x6x8 video tiles hold 144
+// tokens), and the rows of one cluster then also compute the other cluster's kept keys.
+// The plan lays the rows out so that tiles mix as few kept sets as possible:
+//   1. every query cluster fills floor(n_a / 128) whole tiles with its own rows (no mix);
+//   2. the remaining n_a mod 128 rows of each cluster are packed into the following
+//      tiles greedily: a tile starts with the cluster that has the most rows left
+//      (ties: lower label) and is then filled, run by run, with the cluster whose kept
+//      key clusters add the fewest new key clusters to the tile's union so far (ties:
+//      lower label), a cluster's rows staying contiguous inside a tile.
+// Kept sets are the OR of the mask over every (batch, head) slice. When the greedy
+// search would be too expensive (Cq * Wc > kPlanGreedyWords) the leftover rows follow
+// in label order instead. Any layout gives the same result; only the work differs.
+// One CTA of 1024 threads; the greedy loop runs in warp 0.
+constexpr int kPlanGreedyWords = 16384;
+
+struct PlanArgs {
+  const int32_t* sort_token;  // stable label sort of the query rows (cluster-major)
+  const int32_t* sort_label;  // label of each sorted slot (-1 past the valid rows)
+  const int32_t* count;       // rows per query cluster
+  const int32_t* off;         // first sorted slot of each cluster
+  const uint32_t* cbits;      // mask bitsets (slice, Cq, Wc) over key clusters
+  int n_slices, Cq, Wc, Sqpad;
+  int greedy;
+  int32_t* row_token;         // out: token of each planned row (-1 = pad)
+  int32_t* row_label;         // out: its label (-1 = pad)
+};
+
+__global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs pa) {
+  extern __shared__ uint32_t sm_plan[];
+  const int Cq = pa.Cq, Wc = pa.Wc;
+  int32_t* rem = reinterpret_cast<int32_t*>(sm_plan);                 // Cq
+  int32_t* poff = rem + Cq;                                           // Cq
+  uint32_t* uni = reinterpret_cast<uint32_t*>(poff + Cq);             // Wc
+  uint32_t* any = uni + Wc;                                           // Cq * Wc (greedy only)
+  __shared__ int warp_tot[32];
+  __shared__ int s_total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (pa.greedy) {
+    for (int e = tid; e < Cq * Wc; e += 1024) {
+      uint32_t x = 0;
+      for (int sl = 0; sl < pa.n_slices; ++sl) x |= pa.cbits[static_cast<size_t>(sl) * Cq * Wc + e];
+      any[e] = x;
+    }
+  }
+  // exclusive scan of 128 * floor(n_a / 128): first row of cluster a's whole tiles
+  const int per = (Cq + 1023) / 1024;
+  const int c0 = min(Cq, tid * per), c1 = min(Cq, c0 + per);
+  int local = 0, valid = 0;
+  for (int c = c0; c < c1; ++c) {
+    local += pa.count[c] / 128 * 128;
+    valid += pa.count[c];
+  }
+  int incl = local;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  valid = __reduce_add_sync(0xffffffffu, valid);
+  if (lane == 31) warp_tot[warp] = incl;
+  if (tid == 0) s_total = 0;
+  __syncthreads();
+  if (lane == 0) atomicAdd(&s_total, valid);
+  if (warp == 0) {
+    const int t = warp_tot[lane];
+    int ti = t;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += y;
+    }
+    warp_tot[lane] = ti - t;
+  }
+  __syncthreads();
+  const int total = s_total;  // rows with a valid label
+  int base = warp_tot[warp] + incl - local;
+  for (int c = c0; c < c1; ++c) {
+    const int n = pa.count[c], full = n / 128 * 128;
+    rem[c] = n - full;
+    poff[c] = base;
+    base += full;
+  }
+  __syncthreads();
+  // whole tiles: rows [0, 128 k_a) of each cluster, in cluster order
+  for (int p = tid; p < total; p += 1024) {
+    const int c = pa.sort_label[p];
+    const int i = p - pa.off[c];
+    if (i < pa.count[c] / 128 * 128) {
+      pa.row_token[poff[c] + i] = pa.sort_token[p];
+      pa.row_label[poff[c] + i] = c;
+    }
+  }
+  for (int r = total + tid; r < pa.Sqpad; r += 1024) {
+    pa.row_token[r] = -1;
+    pa.row_label[r] = -1;
+  }
+  if (warp != 0) return;
+
+  // ------------------------------------------------ leftover rows (warp 0)
+  int dst = 0;  // rows placed by the whole-tile pass = sum of 128 k_a
+  for (int c = lane; c < Cq; c += 32) dst += pa.count[c] / 128 * 128;
+  dst = __reduce_add_sync(0xffffffffu, dst);
+  int left = total - dst;
+  int room = 0, cur = -1, next_in_order = 0;
+  while (left > 0) {
+    if (room == 0) {
+      // new tile: the cluster with the most rows left, ties to the lower label
+      int best = -1, bc = 0x7fffffff;
+      for (int c = lane; c < Cq; c += 32)
+        if (rem[c] > best) { best = rem[c]; bc = c; }
+      for (int o = 16; o > 0; o >>= 1) {
+        const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+        if (ob > best || (ob == best && oc < bc)) { best = ob; bc = oc; }
+      }
+      cur = pa.greedy ? bc : -1;
+      room = 128;
+      if (pa.greedy)
+        for (int w = lane; w < Wc; w += 32) uni[w] = 0u;
+      __syncwarp();
+    } else if (pa.greedy) {
+      // the cluster adding the fewest new kept key clusters to this tile
+      int best = 0x7fffffff, bc = 0x7fffffff;
+      for (int c = lane; c < Cq; c += 32) {
+        if (rem[c] == 0) continue;
+        int add = 0;
+        for (int w = 0; w < Wc; ++w) add += __popc(any[c * Wc + w] & ~uni[w]);
+        if (add < best) { best = add; bc = c; }
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+        if (ob < best || (ob == best && oc < bc)) { best = ob; bc = oc; }
+      }
+      cur = bc;
+    } else {
+      cur = -1;
+    }
+    if (cur < 0) {  // label order
+      while (rem[next_in_order] == 0) ++next_in_order;
+      cur = next_in_order;
+    }
+    const int r_all = pa.count[cur] % 128;
+    const int take = min(room, rem[cur]);
+    const int src = pa.off[cur] + pa.count[cur] - r_all + (r_all - rem[cur]);
+    for (int i = lane; i < take; i += 32) {
+      pa.row_token[dst + i] = pa.sort_token[src + i];
+      pa.row_label[dst + i] = cur;
+    }
+    if (pa.greedy)
+      for (int w = lane; w < Wc; w += 32) uni[w] |= any[cur * Wc + w];
+    __syncwarp();
+    if (lane == 0) rem[cur] -= take;
+    __syncwarp();
+    dst += take;
+    room -= take;
+    left -= take;
+  }
+}
+
 // ============================================================== gathers
 // dst[bh][r] = src[bh][row_token[r]] (zero row when the token is -1); 16-byte vectors.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src,
@@ -1140,7 +1302,7 @@ struct AttnLayout {
   int Sqpad, Skpad, G, Wg, Ckpad, Wc, Cqpad;
   int ksplit;   // CTAs per query tile over disjoint key ranges (1 = no split)
   float* part;  // ksplit > 1: partial O (B,Hq,ksplit,Sqpad,D), then max and sum (...,2)
-  int32_t *qrow_token, *qrow_label, *q_count, *q_off;
+  int32_t *qrow_token, *qrow_label, *qsort_token, *qsort_label, *q_count, *q_off;
   int32_t *kslot_token, *group_cluster, *group_valid, *k_count, *k_off;
   float* bias2;
   uint32_t *cnonempty, *cbits, *gbits, *gfull;
@@ -1160,6 +1322,8 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
   Carver cv(ws);
   L.qrow_token = cv.take<int32_t>(L.Sqpad);
   L.qrow_label = cv.take<int32_t>(L.Sqpad);
+  L.qsort_token = cv.take<int32_t>(L.Sqpad);
+  L.qsort_label = cv.take<int32_t>(L.Sqpad);
   L.q_count = cv.take<int32_t>(Cq);
   L.q_off = cv.take<int32_t>(Cq + 1);
   L.kslot_token = cv.take<int32_t>(L.Skpad);
@@ -1280,7 +1444,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     const LabelSortJob jk{k_labels,       s.Sk,           Ck,      16,         L.Skpad,
                           L.kslot_token,  nullptr,        L.k_count, L.k_off,  L.group_cluster,
                           L.group_valid,  L.G,            L.bias2, L.Ckpad,    L.cnonempty};
-    const LabelSortJob jq{q_labels, s.Sq,    Cq,      1,       L.Sqpad, L.qrow_token, L.qrow_label,
+    const LabelSortJob jq{q_labels, s.Sq,    Cq,      1,       L.Sqpad, L.qsort_token, L.qsort_label,
                           L.q_count, L.q_off, nullptr, nullptr, 0,       nullptr,      0,
                           nullptr};
     if ((rc = launch_label_sorts(jk, &jq, st))) return rc;
@@ -1292,6 +1456,30 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
                                                     L.gbits, L.gfull);
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "mask_bits_kernel"))) return rc;
+  // 2b. query tile plan (row order of the query tiles)
+  {
+    PlanArgs pa{};
+    pa.sort_token = L.qsort_token;
+    pa.sort_label = L.qsort_label;
+    pa.count = L.q_count;
+    pa.off = L.q_off;
+    pa.cbits = L.cbits;
+    pa.n_slices = nb * nh;
+    pa.Cq = Cq;
+    pa.Wc = L.Wc;
+    pa.Sqpad = L.Sqpad;
+    pa.greedy = static_cast<int64_t>(Cq) * L.Wc <= kPlanGreedyWords ? 1 : 0;
+    pa.row_token = L.qrow_token;
+    pa.row_label = L.qrow_label;
+    const int smem = (2 * Cq + L.Wc + (pa.greedy ? Cq * L.Wc : 0)) * 4;
+    cudaError_t e = cudaFuncSetAttribute(plan_query_tiles_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem > 48 * 1024 ? smem : 48 * 1024);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(plan_query_tiles)");
+    plan_query_tiles_kernel<<<1, 1024, smem, st>>>(pa);
+    count_launch();
+    if ((rc = check_cuda(cudaGetLastError(), "plan_query_tiles_kernel"))) return rc;
+  }
   // 3. Q gather
   const int vpr = s.D * es / 16;
   {

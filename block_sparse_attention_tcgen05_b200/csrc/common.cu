@@ -126,6 +126,33 @@ __global__ void tile_labels_kernel(int T, int H, int W, int tt, int th, int tw, 
   labels[s] = ((t / tt) * nH + h / th) * nW + w / tw;
 }
 
+// Sliding Tile Attention window along one axis of n tiles, w tiles wide: key tile c is
+// inside query tile a's window when |c - centre| <= w / 2, the centre being a moved
+// inward at the borders (clamped to [w / 2, n - 1 - w / 2]); a window at least as wide
+// as the axis holds every tile.
+__device__ __forceinline__ bool sta_axis_keep(int a, int c, int n, int w) {
+  const int r = w / 2;
+  if (2 * r + 1 >= n) return true;
+  const int centre = min(max(a, r), n - 1 - r);
+  return abs(c - centre) <= r;
+}
+
+// Tile-resolution STA mask: one thread per (query tile, key tile) byte, tiles in the
+// raster order of tile_labels.
+__global__ void sliding_tile_mask_kernel(int nT, int nH, int nW, int wt, int wh, int ww,
+                                         uint8_t* __restrict__ mask) {
+  const int64_t C = static_cast<int64_t>(nT) * nH * nW;
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (e >= C * C) return;
+  const int a = static_cast<int>(e / C), c = static_cast<int>(e % C);
+  const int at = a / (nH * nW), ah = (a / nW) % nH, aw = a % nW;
+  const int ct = c / (nH * nW), ch = (c / nW) % nH, cw = c % nW;
+  mask[e] = (sta_axis_keep(at, ct, nT, wt) && sta_axis_keep(ah, ch, nH, wh) &&
+             sta_axis_keep(aw, cw, nW, ww))
+                ? 1
+                : 0;
+}
+
 // One warp waits on an mbarrier that nothing arrives on (expected count 1, no arrival),
 // through the bounded wait every kernel uses; the wait gives up after limit_ns, which
 // records BSA_ERR_TIMEOUT (site 90) in the status word. The barrier then still has its
@@ -244,6 +271,19 @@ int bsa_tile_labels(int T, int H, int W, int tt, int th, int tw, int32_t* labels
                             bsa::as_stream(stream)>>>(T, H, W, tt, th, tw, nH, nW, labels);
   bsa::count_launch();
   return bsa::check_cuda(cudaGetLastError(), "tile_labels_kernel");
+}
+
+int bsa_sliding_tile_block_mask(int nT, int nH, int nW, int wt, int wh, int ww, uint8_t* mask,
+                                void* stream) {
+  if (nT <= 0 || nH <= 0 || nW <= 0 || wt <= 0 || wh <= 0 || ww <= 0)
+    return bsa::fail(BSA_ERR_INVALID_ARG, "non-positive tile grid or window");
+  if (!mask) return bsa::fail(BSA_ERR_INVALID_ARG, "mask is null");
+  const int64_t C = static_cast<int64_t>(nT) * nH * nW;
+  if (C > 16384) return bsa::fail(BSA_ERR_UNSUPPORTED, "%lld tiles > 16384", static_cast<long long>(C));
+  bsa::sliding_tile_mask_kernel<<<static_cast<unsigned>((C * C + 255) / 256), 256, 0,
+                                  bsa::as_stream(stream)>>>(nT, nH, nW, wt, wh, ww, mask);
+  bsa::count_launch();
+  return bsa::check_cuda(cudaGetLastError(), "sliding_tile_mask_kernel");
 }
 
 }  // extern "C"

@@ -107,6 +107,18 @@ def tile_labels(T, H, W, tile, device="cuda"):
     return labels, n.value
 
 
+def sliding_tile_block_mask(n_tiles, window, device="cuda"):
+    """Tile-resolution Sliding Tile Attention mask over a (nT, nH, nW) tile grid with a
+    (wt, wh, ww) window in tiles: uint8 (C, C), C = nT·nH·nW, tiles in the order of
+    ``tile_labels``."""
+    nT, nH, nW = (int(x) for x in n_tiles)
+    C = nT * nH * nW
+    mask = torch.empty((C, C), dtype=torch.uint8, device=device)
+    _call_on(mask.device, "bsa_sliding_tile_block_mask", nT, nH, nW, int(window[0]),
+             int(window[1]), int(window[2]), _ptr(mask), _stream(mask.device))
+    return mask
+
+
 def attention_workspace_bytes(q, k, Cq, Ck):
     return _lib.load().bsa_attention_workspace_bytes(make_shape(q, k), int(Cq), int(Ck))
 

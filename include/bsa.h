@@ -114,6 +114,23 @@ int bsa_tile_labels(int T, int H, int W, int tt, int th, int tw, int32_t* labels
                     int* n_clusters, void* stream);
 
 /*
+ * sliding_tile_block_mask — [SBC] §What mlx-arsenal ships (sliding_tile_block_mask),
+ * §Recipe: STA with both repairs (evaluated at tile resolution it is the cluster-level
+ * mask for tile_labels: expanding it through the labels reproduces the token-level
+ * Sliding Tile Attention mask). Tiles of an nT x nH x nW tile grid in the raster order
+ * of bsa_tile_labels; query tile a keeps key tile c when, on every axis, c lies in a's
+ * window: the tiles within w/2 of a centre that is a moved inward at the borders
+ * (clamped to [w/2, n-1-w/2]), so an odd window keeps w tiles; a window at least as
+ * wide as the axis keeps all of them.
+ *   wt, wh, ww : window sizes in tiles (>= 1).
+ *   mask       : device uint8 (C, C), C = nT*nH*nW <= 16384; written (1 = kept).
+ * Errors: INVALID_ARG for non-positive sizes or a null mask; UNSUPPORTED past 16384
+ * tiles.
+ */
+int bsa_sliding_tile_block_mask(int nT, int nH, int nW, int wt, int wh, int ww, uint8_t* mask,
+                                void* stream);
+
+/*
  * antidiagonal_block_scores — [HMR] §XAttention — anti-diagonal block scoring,
  * §Deviations (rows normalised to 1), §Out of scope (the caller pads S to a multiple
  * of the block; padded keys take softmax mass).

@@ -32,7 +32,7 @@ from .attention import (  # noqa: F401
     kv_head,
 )
 from .scoring import antidiagonal_block_scores, top_p_block_mask  # noqa: F401
-from .labels import tile_labels  # noqa: F401
+from .labels import sliding_tile_block_mask, sta_token_mask, tile_labels  # noqa: F401
 from .repair import (  # noqa: F401
     select_probe_rows,
     select_probe_rows_centroid,
@@ -42,3 +42,4 @@ from .repair import (  # noqa: F401
 )
 from .cache import HeadMaskCache, pooled_qk, qk_drift  # noqa: F401
 from .accounting import executed_pairs  # noqa: F401
+from .routing import compensation_errors, error_aware_block_mask  # noqa: F401

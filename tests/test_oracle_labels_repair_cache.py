@@ -41,6 +41,50 @@ def test_tile_labels_encode_tile_coordinates():
     np.testing.assert_array_equal(tmask[lab][:, lab], tok)
 
 
+@pytest.mark.parametrize("grid,tile,window", [
+    ((4, 6, 10), (2, 3, 4), (1, 1, 3)),      # partial edge tiles along W (10 = 4 + 4 + 2)
+    ((6, 6, 8), (2, 2, 2), (3, 3, 3)),       # 3 x 3 x 4 tiles, windows clamped at the borders
+    ((5, 4, 9), (1, 2, 2), (5, 1, 3)),       # window as wide as the T axis keeps all of it
+    ((3, 5, 7), (1, 1, 1), (3, 5, 9)),       # token resolution, windows past the grid
+])
+def test_sliding_tile_mask_expands_to_the_token_level_sta_mask(grid, tile, window):
+    """"Sparse-block compensation", §Recipe: the tile-resolution sliding-tile mask,
+    expanded through tile_labels, reproduces the token-level STA mask (computed token
+    pair by token pair from the tokens' own tile coordinates)."""
+    lab, C = oracle.tile_labels(*grid, tile)
+    n = [-(-g // t) for g, t in zip(grid, tile)]
+    m = oracle.sliding_tile_block_mask(*n, window)
+    assert m.shape == (C, C)
+    np.testing.assert_array_equal(m[lab][:, lab], oracle.sta_token_mask(*grid, tile, window))
+
+
+def test_sliding_tile_mask_window_by_explicit_loops():
+    """The window written the other way round, by loops: along an axis of n tiles a
+    window of w = 2r + 1 tiles starts at min(max(a − r, 0), n − w) (shifted inward at
+    the borders) and holds w consecutive tiles; a window of at least n tiles holds
+    them all. Every query tile therefore keeps exactly the product of min(w, n) key
+    tiles, the diagonal is always kept, (1,1,1) is the identity."""
+    nT, nH, nW, window = 4, 3, 6, (3, 1, 5)
+    m = oracle.sliding_tile_block_mask(nT, nH, nW, window)
+
+    def axis_keep(a, c, n, w):
+        if w >= n:
+            return True
+        start = min(max(a - w // 2, 0), n - w)
+        return start <= c < start + w
+
+    for a in range(nT * nH * nW):
+        at, ah, aw = a // (nH * nW), (a // nW) % nH, a % nW
+        for c in range(nT * nH * nW):
+            ct, ch, cw = c // (nH * nW), (c // nW) % nH, c % nW
+            want = (axis_keep(at, ct, nT, 3) and axis_keep(ah, ch, nH, 1)
+                    and axis_keep(aw, cw, nW, 5))
+            assert m[a, c] == want, (a, c)
+    assert (m.sum(1) == 3 * 1 * 5).all() and m.diagonal().all()
+    np.testing.assert_array_equal(oracle.sliding_tile_block_mask(3, 4, 5, (1, 1, 1)), np.eye(60))
+    assert oracle.sliding_tile_block_mask(3, 4, 5, (3, 5, 5)).all()
+
+
 # ----------------------------------------------------------------------------- probes
 def test_probe_rows_tiny_golden():
     rows = np.loadtxt(os.path.join(GOLDEN, "probe_rows_tiny.txt"), comments="#")

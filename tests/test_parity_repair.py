@@ -185,9 +185,13 @@ def test_sparsepr_video_workload_sampled():
     op_ref = oracle.probe_dense_attention(qd, kd, vd, idx_n)
     assert _rel_fro(op.cpu().numpy(), op_ref) <= 5e-3
     rep_ref = oracle.probe_residual_correction(sparse, op_ref, idx_n, w_n)
-    # the correction itself, element by element over every row: GPU (rep - sparse)
-    # against the oracle's (rep_ref - sparse) on the same sparse output and probes
-    assert _rel_fro(rep - sparse, rep_ref - sparse) <= 1e-3, _rel_fro(rep - sparse, rep_ref - sparse)
+    # The correction itself, element by element over every row: GPU (rep - sparse)
+    # against the oracle's repair of the same sparse output with the same probe rows and
+    # the same probe outputs (the GPU's). The residual at the probes is ~0.3 % of the
+    # output here, the size of the fp32-vs-float64 difference of the probe attention, so
+    # the probe outputs must be shared for the corrections to be comparable.
+    rep_same = oracle.probe_residual_correction(sparse, op.cpu().numpy(), idx_n, w_n)
+    assert _rel_fro(rep - sparse, rep_same - sparse) <= 1e-3, _rel_fro(rep - sparse, rep_same - sparse)
     dense_rows = oracle.dense_attention(qd, kd, vd, rows=rows)
     err_gpu = _rel_fro(rep[:, :, rows], dense_rows)
     err_ref = _rel_fro(rep_ref[:, :, rows], dense_rows)
