@@ -60,6 +60,9 @@ def parse():
     p.add_argument("--mask", choices=["nearest", "sta"], default="nearest",
                    help="nearest: the 22 %% of tile pairs nearest in (t, h, w) (default); sta: "
                         "the recipe's sliding-tile window of STA_WINDOW tiles")
+    p.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                   help="replicas: every rank runs the whole workload (weak scaling, default); "
+                        "heads: the layer's 40 heads are split over the ranks (strong scaling)")
     p.add_argument("--heads", type=int, default=H,
                    help="number of heads (default 40; smaller only for profiler captures)")
     return p.parse_args()
@@ -80,6 +83,14 @@ def max_over_ranks(values, device, world):
 def weak_scaling_tflops(flop_per_rank, world, ms):
     """Whole-job throughput: every rank processes its own copy of the workload."""
     return world * flop_per_rank / (ms * 1e-3) / 1e12
+
+
+def job_flop(flop_local, heads_local, heads_layer, world, shard):
+    """FLOPs of the whole job: N copies of the workload (replicas) or the one layer whose
+    heads the ranks share (heads)."""
+    if shard == "heads":
+        return flop_local / heads_local * heads_layer
+    return flop_local * world
 
 
 def measured_peaks():
@@ -296,8 +307,14 @@ def main():
 
     # ---------------------------------------------------------------- inputs (HBM-resident)
     nh = args.heads
+    seed = 3 + 1000 * rank
+    if args.shard == "heads":
+        # this rank's heads of the one layer (KV-aligned ranges; no exchange of data)
+        from block_sparse_attention_tcgen05_b200.sharding import head_range
+        h0, h1, _, _ = head_range(args.heads, args.heads, world, rank)
+        nh, seed = h1 - h0, 3 + h0
     q, k, v = wl.positional_qkv_device(1, nh, nh, GRID, D, ell=(3.0, 6.0, 8.0), amp=2.0,
-                                       seed=3 + 1000 * rank, device=dev)
+                                       seed=seed, device=dev)
     labels, C = bsa.tile_labels(*GRID, TILE, device=dev)
     if args.mask == "sta":
         n_tiles = tuple(-(-g // t) for g, t in zip(GRID, TILE))
@@ -421,7 +438,8 @@ def main():
         (e2e_ms,) = max_over_ranks([e2e_ms], dev, world)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, mh))
         d2h = oh.numel() * oh.element_size()
-        e2e = {"value": weak_scaling_tflops(flop, world, e2e_ms), "unit": "TFLOP/s",
+        e2e = {"value": job_flop(flop, nh, args.heads, world, args.shard) / (e2e_ms * 1e-3) / 1e12,
+               "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "block_sparse_attention_tcgen05_b200.centroid_compensated_attention",
                "overlap": "upload of step i+1 and download of step i-1 on their own streams "
@@ -438,7 +456,7 @@ def main():
         achieved = flop / (attn_ms_launch * 1e-3) / 1e12
         line = {
             "metric": METRIC,
-            "value": weak_scaling_tflops(flop, world, ms),
+            "value": job_flop(flop, nh, args.heads, world, args.shard) / (ms * 1e-3) / 1e12,
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -446,7 +464,7 @@ def main():
             "ms_per_step": ms,
             "ms_per_call": ms,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if args.shard == "heads" else "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
@@ -460,7 +478,9 @@ def main():
                 "flop_per_call": flop,
                 "l2": "inputs larger than L2 (Q+K+V = %.2f GB per rank)" % (
                     3 * q.numel() * 2 / 1e9),
-                "parallelism": "replicas x%d (weak, no collective on the data path)" % world,
+                "parallelism": ("heads split over %d ranks (strong, no collective on the data path)"
+                                if args.shard == "heads" else
+                                "replicas x%d (weak, no collective on the data path)") % world,
             },
             "roofline": {
                 "kernel": "attn_kernel<128,bf16>",

@@ -13,6 +13,7 @@ from .ops import (  # noqa: F401
     attention_workspace_bytes,
     centroid_compensated_attention,
     device_status,
+    error_aware_block_mask,
     probe_dense_attention,
     probe_residual_correction,
     select_probe_rows,

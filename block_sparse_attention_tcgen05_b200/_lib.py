@@ -50,6 +50,9 @@ SIGNATURES = {
     "bsa_attention_workspace_bytes": (_sz, [Shape, _i, _i]),
     "bsa_centroid_compensated_attention": (
         _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _vp, _i64, _i64, _f, _i, _vp, _vp, _sz, _vp]),
+    "bsa_routing_workspace_bytes": (_sz, [Shape, _i, _i]),
+    "bsa_error_aware_block_mask": (
+        _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _f, _f, _vp, _vp, _vp, _sz, _vp]),
     "bsa_probe_select_workspace_bytes": (_sz, [_i, _i, _i]),
     "bsa_select_probe_rows": (_i, [_vp, _i, _i, _i, _vp, Shape, _vp, _vp, _vp, _sz, _vp]),
     "bsa_probe_attention_workspace_bytes": (_sz, [Shape, _i]),
@@ -62,6 +65,7 @@ SIGNATURES = {
     "bsa_mask_cache_state_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "bsa_mask_cache_init": (_i, [_vp, _i, _i, _i, _i, _i, _f, _i, _f, _f, _vp]),
     "bsa_mask_cache_should_refresh": (_i, [_vp, _vp, _vp, Shape, _vp, _vp, _ip, _vp]),
+    "bsa_mask_cache_layer_gate": (_i, [_vp, _vp, _i, _i, _f, _f, _vp]),
     "bsa_mask_cache_update": (_i, [_vp, _vp, _vp, _vp, _vp]),
     "bsa_mask_cache_reset": (_i, [_vp, _vp]),
 }

@@ -206,6 +206,26 @@ __global__ void __launch_bounds__(1024) decide_kernel(void* state, int B, int H,
   if (threadIdx.x == 0) hdr->n_refresh = n;
 }
 
+// Layer gate over heads held by several caches (a layer's heads split across GPUs):
+// with the layer-wide refresh count n_layer of n_heads heads, fewer than gate_lo of them
+// -> no local head refreshes, more than gate_hi -> every local head does; otherwise the
+// per-head decisions stand. Not applied on a cache's first call (no anchors: every head
+// refreshes). One CTA; the header's n_refresh becomes the local count after the gate.
+__global__ void __launch_bounds__(256) layer_gate_kernel(void* state, uint8_t* __restrict__ refresh,
+                                                         int n_layer, int n_heads, float gate_lo,
+                                                         float gate_hi) {
+  const CacheLayout L = device_layout(state);
+  CacheHeader* hdr = L.hdr;
+  if (hdr->magic != kCacheMagic) return;
+  const int BH = hdr->B * hdr->H;
+  if (!hdr->has_anchor || gate_lo < 0.f) return;
+  const float frac = static_cast<float>(n_layer) / static_cast<float>(n_heads);
+  const int force = frac < gate_lo ? 0 : (frac > gate_hi ? 1 : -1);
+  if (force < 0) return;
+  for (int bh = threadIdx.x; bh < BH; bh += blockDim.x) refresh[bh] = static_cast<uint8_t>(force);
+  if (threadIdx.x == 0) hdr->n_refresh = force ? BH : 0;
+}
+
 // Grid-stride over the cached mask: refreshed heads (every head on the first update)
 // take new_mask; the result is copied to out.
 __global__ void update_mask_kernel(void* state, const uint8_t* __restrict__ new_mask,
@@ -307,6 +327,19 @@ extern "C" int bsa_mask_cache_should_refresh(void* state, const void* q, const v
     if ((rc = check_cuda(cudaStreamSynchronize(st), "cudaStreamSynchronize"))) return rc;
   }
   return BSA_OK;
+}
+
+extern "C" int bsa_mask_cache_layer_gate(void* state, uint8_t* refresh, int n_refresh_layer,
+                                         int n_heads_layer, float gate_lo, float gate_hi,
+                                         void* stream) {
+  using namespace bsa;
+  if (!state || !refresh) return fail(BSA_ERR_INVALID_ARG, "null pointer");
+  if (n_heads_layer <= 0 || n_refresh_layer < 0 || n_refresh_layer > n_heads_layer)
+    return fail(BSA_ERR_INVALID_ARG, "refresh count %d of %d heads", n_refresh_layer, n_heads_layer);
+  layer_gate_kernel<<<1, 256, 0, as_stream(stream)>>>(state, refresh, n_refresh_layer, n_heads_layer,
+                                                      gate_lo, gate_hi);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "layer_gate_kernel");
 }
 
 extern "C" int bsa_mask_cache_update(void* state, const uint8_t* new_mask, const uint8_t* refresh,

@@ -2,6 +2,7 @@
 // kernel without relocatable device code.
 #include "common.cu"
 #include "attention.cu"
+#include "routing.cu"
 #include "scoring.cu"
 #include "topp.cu"
 #include "probe.cu"

@@ -1,0 +1,465 @@
+// SVG-EAR error-aware routing: which (query cluster, key cluster) blocks to compute
+// exactly.
+//
+// Sources: "Sparse-block compensation" (mlx-arsenal notes), §SVG-EAR — centroid
+// compensation (the paper adds an error-aware router choosing which blocks to compute
+// exactly); the SVG-EAR abstract (a lightweight probe estimates each block's
+// compensation error; the blocks with the highest error-to-cost ratio are computed
+// exactly, the others compensated).
+//
+// Per (batch, query head):
+//   probe of query cluster a   q̄_a, the mean query of the cluster
+//   block error                err_ac = || E_ac - A_ac ||_2 with, for dense logits
+//                              l_j = scale q̄_a . k_j, m their max, Z = sum_j exp(l_j - m):
+//                              E_ac = sum_{j in c} exp(l_j - m) v_j / Z (exact) and
+//                              A_ac = n_c exp(scale q̄_a . k̄_c - m) v̄_c / Z (centroid term)
+//   cost, ratio                n_a n_c token pairs; ratio = err_ac / n_c
+//   selection                  blocks of non-empty clusters by descending ratio (equal
+//                              ratios: lower a*Ck + c), the longest prefix whose pairs
+//                              sum to at most floor(density * Sq * Sk)
+//
+// Kernels (caller's stream): label sorts of both label arrays (the attention's sort),
+// per-cluster means of Q, K and V (fp32), the probe kernel (one CTA per 16 probes of a
+// head, streaming the head's keys cluster by cluster through shared memory), and one
+// CTA per head that selects the prefix exactly by a radix descent over the ratios'
+// bits with 64-bit pair counts.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace bsa {
+
+// ---------------------------------------------------------------- cluster means
+// grid (C, H, B), 128 threads: dst[b,h,c,:] = mean of src[b,h,tok,:] over the tokens of
+// cluster c (slots off[c] .. off[c] + count[c] of the sorted order); 0 if empty.
+template <typename T>
+__global__ void __launch_bounds__(128) cluster_mean_kernel(const T* __restrict__ src,
+                                                           const int32_t* __restrict__ sort_token,
+                                                           const int32_t* __restrict__ count,
+                                                           const int32_t* __restrict__ off, int C,
+                                                           int S, int D, int H,
+                                                           float* __restrict__ dst) {
+  const int c = blockIdx.x;
+  const int64_t bh = static_cast<int64_t>(blockIdx.z) * H + blockIdx.y;
+  const int n = count[c], o = off[c];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const int tok = sort_token[o + i];
+      acc += static_cast<float>(src[(bh * S + tok) * D + d]);
+    }
+    dst[(bh * C + c) * D + d] = n > 0 ? acc / static_cast<float>(n) : 0.f;
+  }
+}
+
+// ---------------------------------------------------------------- probe errors
+constexpr int kRouteProbes = 16;   // probes per CTA
+constexpr int kRouteKeys = 32;     // keys per shared-memory chunk
+constexpr int kRouteThreads = 256; // 16 threads per probe
+
+__device__ __forceinline__ float route_f(float x) { return x; }
+__device__ __forceinline__ float route_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+struct RouteArgs {
+  int B, Hq, Hkv, S, D, Cq, Ck;
+  float scale;
+  const float* qbar;   // (B, Hq, Cq, D)
+  const float* kbar;   // (B, Hkv, Ck, D)
+  const float* vbar;   // (B, Hkv, Ck, D)
+  const int32_t* q_count;
+  const int32_t* k_sort_token;
+  const int32_t* k_count;
+  const int32_t* k_off;
+  float* err;   // (B, Hq, Cq, Ck): written
+  float* mref;  // (B, Hq, Cq, Ck): per-block reference of the unscaled error (scratch)
+};
+
+// grid (ceil(Cq / 16), Hq, B). Thread t serves probe p = t / 16 and dims
+// [8 (t % 16), 8 (t % 16) + 8) of its running difference vector; for D = 64 only the
+// first 8 lanes of each probe hold dims. Keys of one cluster are streamed 32 at a time
+// through shared memory; a running reference m (the largest logit seen, centroid
+// logits included) keeps every exponential <= 1. At the end of cluster c the norm of
+// the difference vector and the reference it was taken with are stored; once every
+// cluster is done they are brought to the final reference and divided by Z.
+template <typename T, int D>
+__global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __restrict__ k,
+                                                                     const T* __restrict__ v,
+                                                                     const RouteArgs a) {
+  __shared__ float sq[kRouteProbes][D];
+  __shared__ float sk[kRouteKeys][D + 1];
+  __shared__ float sv[kRouteKeys][D];
+  __shared__ float sw[kRouteProbes][kRouteKeys];
+  const int tid = threadIdx.x, p = tid >> 4, sub = tid & 15;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hkv = h / (a.Hq / a.Hkv);
+  const int a0 = blockIdx.x * kRouteProbes;
+  const int pa = a0 + p;                    // this thread's query cluster (probe)
+  const bool live = pa < a.Cq && a.q_count[pa] > 0;
+  const int64_t bq = static_cast<int64_t>(b) * a.Hq + h;
+  const int64_t bk = static_cast<int64_t>(b) * a.Hkv + hkv;
+  for (int e = tid; e < kRouteProbes * D; e += kRouteThreads) {
+    const int pp = e / D, d = e % D;
+    sq[pp][d] = (a0 + pp < a.Cq) ? a.qbar[(bq * a.Cq + a0 + pp) * D + d] : 0.f;
+  }
+  constexpr int DPT = 8;                    // dims per thread
+  const bool has_dims = sub * DPT < D;
+  const int d0 = sub * DPT;
+  float m = -INFINITY, z = 0.f;             // running reference and sum of exp(l - m)
+  float diff[DPT];
+  const float* kb = a.kbar + bk * a.Ck * D;
+  const float* vb = a.vbar + bk * a.Ck * D;
+  float* err = a.err + (bq * a.Cq + (pa < a.Cq ? pa : 0)) * a.Ck;
+  float* mref = a.mref + (bq * a.Cq + (pa < a.Cq ? pa : 0)) * a.Ck;
+  __syncthreads();
+  for (int c = 0; c < a.Ck; ++c) {
+    const int n = a.k_count[c], o = a.k_off[c];
+#pragma unroll
+    for (int i = 0; i < DPT; ++i) diff[i] = 0.f;
+    // centroid logit of this probe (16 lanes of the probe reduce their dims)
+    float lc = 0.f;
+    if (has_dims)
+#pragma unroll
+      for (int i = 0; i < DPT; ++i) lc = fmaf(sq[p][d0 + i], kb[c * D + d0 + i], lc);
+#pragma unroll
+    for (int s = 8; s > 0; s >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, s);
+    lc *= a.scale;
+    if (n > 0 && lc > m) {
+      const float f = __expf(m - lc);
+      z *= f;
+      m = lc;
+    }
+    for (int j0 = 0; j0 < n; j0 += kRouteKeys) {
+      const int nk = min(kRouteKeys, n - j0);
+      __syncthreads();
+      for (int e = tid; e < kRouteKeys * D; e += kRouteThreads) {
+        const int j = e / D, d = e % D;
+        float kx = 0.f, vx = 0.f;
+        if (j < nk) {
+          const int tok = a.k_sort_token[o + j0 + j];
+          kx = route_f(k[(bk * a.S + tok) * D + d]);
+          vx = route_f(v[(bk * a.S + tok) * D + d]);
+        }
+        sk[j][d] = kx;
+        sv[j][d] = vx;
+      }
+      __syncthreads();
+      // logits of keys sub and sub + 16 for this probe
+      float l0 = 0.f, l1 = 0.f;
+#pragma unroll 8
+      for (int d = 0; d < D; ++d) {
+        const float x = sq[p][d];
+        l0 = fmaf(x, sk[sub][d], l0);
+        l1 = fmaf(x, sk[sub + 16][d], l1);
+      }
+      l0 = sub < nk ? l0 * a.scale : -INFINITY;
+      l1 = sub + 16 < nk ? l1 * a.scale : -INFINITY;
+      float mx = fmaxf(l0, l1);
+#pragma unroll
+      for (int s = 8; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+      if (mx > m) {
+        const float f = __expf(m - mx);
+        z *= f;
+#pragma unroll
+        for (int i = 0; i < DPT; ++i) diff[i] *= f;
+        m = mx;
+      }
+      const float w0 = __expf(l0 - m), w1 = __expf(l1 - m);
+      float ws = w0 + w1;
+#pragma unroll
+      for (int s = 8; s > 0; s >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, s);
+      z += ws;
+      sw[p][sub] = w0;
+      sw[p][sub + 16] = w1;
+      __syncwarp();
+      if (has_dims)
+        for (int j = 0; j < nk; ++j) {
+          const float w = sw[p][j];
+#pragma unroll
+          for (int i = 0; i < DPT; ++i) diff[i] = fmaf(w, sv[j][d0 + i], diff[i]);
+        }
+    }
+    // minus the centroid term, then the norm (taken with reference m)
+    float e2 = 0.f;
+    if (n > 0) {
+      const float wc = static_cast<float>(n) * __expf(lc - m);
+      if (has_dims)
+#pragma unroll
+        for (int i = 0; i < DPT; ++i) {
+          const float dd = diff[i] - wc * vb[c * D + d0 + i];
+          e2 = fmaf(dd, dd, e2);
+        }
+    }
+#pragma unroll
+    for (int s = 8; s > 0; s >>= 1) e2 += __shfl_xor_sync(0xffffffffu, e2, s);
+    if (sub == 0 && pa < a.Cq) {
+      err[c] = sqrtf(e2);
+      mref[c] = m;
+    }
+  }
+  __syncwarp();
+  if (pa < a.Cq) {
+    for (int c = sub; c < a.Ck; c += 16) {
+      const bool ok = live && a.k_count[c] > 0 && z > 0.f;
+      err[c] = ok ? err[c] * __expf(mref[c] - m) / z : 0.f;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- budgeted selection
+// One CTA (1024 threads) per (batch, head). Keys are the bit patterns of the
+// non-negative float ratios err / n_c (monotone in the value); invalid blocks (an
+// empty cluster) take no part. A radix descent, 8 bits per pass from the top, finds
+// the key k* at which the pair count of the blocks above it, plus those at k*, first
+// exceeds the budget; blocks above k* are kept, and those equal to k* in index order
+// while the running count stays within the budget.
+__global__ void __launch_bounds__(1024) route_select_kernel(const float* __restrict__ err,
+                                                            const int32_t* __restrict__ q_count,
+                                                            const int32_t* __restrict__ k_count,
+                                                            int Cq, int Ck, float density,
+                                                            uint8_t* __restrict__ mask) {
+  __shared__ unsigned long long hist[256];
+  __shared__ unsigned long long s_part[32];
+  __shared__ unsigned long long s_sq, s_sk;
+  __shared__ uint32_t s_prefix;
+  __shared__ long long s_rem;
+  __shared__ int s_all;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t bh = blockIdx.x;
+  const int64_t E = static_cast<int64_t>(Cq) * Ck;
+  const float* e_bh = err + bh * E;
+  uint8_t* m_bh = mask + bh * E;
+  // totals of valid query and key rows
+  unsigned long long sq = 0, sk = 0;
+  for (int a = tid; a < Cq; a += 1024) sq += static_cast<unsigned long long>(max(q_count[a], 0));
+  for (int c = tid; c < Ck; c += 1024) sk += static_cast<unsigned long long>(max(k_count[c], 0));
+  if (tid == 0) { s_sq = 0; s_sk = 0; }
+  __syncthreads();
+  sq = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(sq));
+  sk = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(sk));
+  if (lane == 0) { atomicAdd(&s_sq, sq); atomicAdd(&s_sk, sk); }
+  __syncthreads();
+  const long long budget = static_cast<long long>(
+      floor(static_cast<double>(density) * static_cast<double>(s_sq) * static_cast<double>(s_sk)));
+  auto key_of = [&](int64_t e, uint32_t& key, long long& cost) -> bool {
+    const int a_ = static_cast<int>(e / Ck), c_ = static_cast<int>(e % Ck);
+    const int na = q_count[a_], nc = k_count[c_];
+    if (na <= 0 || nc <= 0) return false;
+    const float r = __fdiv_rn(e_bh[e], static_cast<float>(nc));
+    key = __float_as_uint(fmaxf(r, 0.f));
+    cost = static_cast<long long>(na) * nc;
+    return true;
+  };
+  if (tid == 0) { s_prefix = 0; s_rem = budget; s_all = 0; }
+  __syncthreads();
+  // radix descent: after pass p the top 8(p+1) bits of k* are known
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < 256; i += 1024) hist[i] = 0;
+    __syncthreads();
+    const uint32_t pre = s_prefix;
+    const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+    for (int64_t e = tid; e < E; e += 1024) {
+      uint32_t key;
+      long long cost;
+      if (!key_of(e, key, cost)) continue;
+      if ((key & hi_mask) != (pre & hi_mask)) continue;
+      atomicAdd(&hist[(key >> shift) & 255u], static_cast<unsigned long long>(cost));
+    }
+    __syncthreads();
+    if (tid == 0) {
+      long long rem = s_rem;
+      int digit = -1;
+      for (int d = 255; d >= 0; --d) {
+        const long long hcost = static_cast<long long>(hist[d]);
+        if (hcost > rem) { digit = d; break; }
+        rem -= hcost;
+      }
+      if (digit < 0) {
+        s_all = 1;  // every block under this prefix fits
+      } else {
+        s_prefix = pre | (static_cast<uint32_t>(digit) << shift);
+        s_rem = rem;
+      }
+    }
+    __syncthreads();
+    if (s_all) break;
+  }
+  const bool all = s_all != 0;
+  const uint32_t kstar = s_prefix;
+  const long long rem_at_k = s_rem;  // budget left for the blocks equal to k*
+  // blocks above k* (or every block when all fit); blocks at k* in index order
+  unsigned long long carry = 0;
+  for (int64_t t0 = 0; t0 < E; t0 += 1024) {
+    const int64_t e = t0 + tid;
+    uint32_t key = 0;
+    long long cost = 0;
+    const bool valid = e < E && key_of(e, key, cost);
+    uint8_t keep = 0;
+    unsigned long long tie_cost = 0;
+    if (valid) {
+      if (all || key > kstar) keep = 1;
+      else if (key == kstar) tie_cost = static_cast<unsigned long long>(cost);
+    }
+    // inclusive block scan of tie_cost
+    unsigned long long x = tie_cost;
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_part[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      unsigned long long w = s_part[lane];
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      s_part[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const unsigned long long before = warp > 0 ? s_part[warp - 1] : 0ull;
+    const unsigned long long incl = carry + before + x;
+    if (tie_cost > 0 && static_cast<long long>(incl) <= rem_at_k) keep = 1;
+    carry += s_part[31];
+    __syncthreads();
+    if (e < E) m_bh[e] = keep;
+  }
+}
+
+namespace {
+struct RouteLayout {
+  int32_t *q_tok, *q_count, *q_off, *k_tok, *k_count, *k_off;
+  float *qbar, *kbar, *vbar, *err, *mref;
+  size_t bytes;
+};
+RouteLayout carve_route(const bsa_shape& s, int Cq, int Ck, void* ws) {
+  Carver cv(ws);
+  RouteLayout L{};
+  L.q_tok = cv.take<int32_t>(s.Sq);
+  L.q_count = cv.take<int32_t>(Cq);
+  L.q_off = cv.take<int32_t>(Cq + 1);
+  L.k_tok = cv.take<int32_t>(s.Sk);
+  L.k_count = cv.take<int32_t>(Ck);
+  L.k_off = cv.take<int32_t>(Ck + 1);
+  L.qbar = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * s.D);
+  L.kbar = cv.take<float>(static_cast<size_t>(s.B) * s.Hkv * Ck * s.D);
+  L.vbar = cv.take<float>(static_cast<size_t>(s.B) * s.Hkv * Ck * s.D);
+  L.err = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
+  L.mref = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
+  L.bytes = align_up(cv.used, 256);
+  return L;
+}
+
+int validate_route(const bsa_shape& s, int Cq, int Ck) {
+  if (s.B <= 0 || s.Hq <= 0 || s.Hkv <= 0 || s.Sq <= 0 || s.Sk <= 0)
+    return fail(BSA_ERR_INVALID_ARG, "non-positive shape");
+  if (s.Hq % s.Hkv) return fail(BSA_ERR_INVALID_ARG, "Hq (%d) not a multiple of Hkv (%d)", s.Hq, s.Hkv);
+  if (s.D != 64 && s.D != 128) return fail(BSA_ERR_UNSUPPORTED, "head dim %d not in {64,128}", s.D);
+  if (s.dtype != BSA_BF16 && s.dtype != BSA_F32) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", s.dtype);
+  if (Cq <= 0 || Ck <= 0 || Cq > 16384 || Ck > 16384)
+    return fail(BSA_ERR_UNSUPPORTED, "cluster counts Cq=%d Ck=%d outside [1,16384]", Cq, Ck);
+  if (static_cast<int64_t>(Cq) * Ck > (int64_t(1) << 24))
+    return fail(BSA_ERR_UNSUPPORTED, "Cq * Ck = %lld blocks per head exceeds 2^24",
+                static_cast<long long>(Cq) * Ck);
+  return BSA_OK;
+}
+
+template <typename T, int D>
+void launch_route_probe(const void* k, const void* v, const RouteArgs& ra, cudaStream_t st) {
+  route_probe_kernel<T, D><<<dim3((ra.Cq + kRouteProbes - 1) / kRouteProbes, ra.Hq, ra.B),
+                             kRouteThreads, 0, st>>>(static_cast<const T*>(k),
+                                                     static_cast<const T*>(v), ra);
+}
+}  // namespace
+
+}  // namespace bsa
+
+extern "C" size_t bsa_routing_workspace_bytes(bsa_shape shape, int Cq, int Ck) {
+  if (bsa::validate_route(shape, Cq, Ck)) return 0;
+  return bsa::carve_route(shape, Cq, Ck, nullptr).bytes;
+}
+
+extern "C" int bsa_error_aware_block_mask(const void* q, const void* k, const void* v,
+                                          bsa_shape shape, const int32_t* q_labels, int Cq,
+                                          const int32_t* k_labels, int Ck, float density,
+                                          float scale, uint8_t* mask, float* err,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  using namespace bsa;
+  int rc = validate_route(shape, Cq, Ck);
+  if (rc) return rc;
+  if (!q || !k || !v || !q_labels || !k_labels || !mask)
+    return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!(density >= 0.f && density <= 1.f))
+    return fail(BSA_ERR_INVALID_ARG, "density %g outside [0, 1]", static_cast<double>(density));
+  RouteLayout L = carve_route(shape, Cq, Ck, workspace);
+  if (!workspace || workspace_bytes < L.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, L.bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(BSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  cudaStream_t st = as_stream(stream);
+  const bsa_shape& s = shape;
+  // 1. stable label sorts (cluster-major token order, counts, offsets)
+  {
+    const LabelSortJob jk{k_labels, s.Sk, Ck, 1, s.Sk, L.k_tok, nullptr, L.k_count, L.k_off,
+                          nullptr, nullptr, 0, nullptr, 0, nullptr};
+    const LabelSortJob jq{q_labels, s.Sq, Cq, 1, s.Sq, L.q_tok, nullptr, L.q_count, L.q_off,
+                          nullptr, nullptr, 0, nullptr, 0, nullptr};
+    if ((rc = launch_label_sorts(jk, &jq, st))) return rc;
+  }
+  // 2. cluster means of Q (probes), K and V (centroids), fp32
+  if (s.dtype == BSA_F32) {
+    cluster_mean_kernel<float><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(
+        static_cast<const float*>(q), L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.D, s.Hq, L.qbar);
+    cluster_mean_kernel<float><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
+        static_cast<const float*>(k), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.kbar);
+    cluster_mean_kernel<float><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
+        static_cast<const float*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
+  } else {
+    using bf = __nv_bfloat16;
+    cluster_mean_kernel<bf><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(
+        static_cast<const bf*>(q), L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.D, s.Hq, L.qbar);
+    cluster_mean_kernel<bf><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
+        static_cast<const bf*>(k), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.kbar);
+    cluster_mean_kernel<bf><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
+        static_cast<const bf*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
+  }
+  for (int i = 0; i < 3; ++i) count_launch();
+  if ((rc = check_cuda(cudaGetLastError(), "cluster_mean_kernel"))) return rc;
+  // 3. probe errors
+  RouteArgs ra{};
+  ra.B = s.B;
+  ra.Hq = s.Hq;
+  ra.Hkv = s.Hkv;
+  ra.S = s.Sk;
+  ra.D = s.D;
+  ra.Cq = Cq;
+  ra.Ck = Ck;
+  ra.scale = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(s.D));
+  ra.qbar = L.qbar;
+  ra.kbar = L.kbar;
+  ra.vbar = L.vbar;
+  ra.q_count = L.q_count;
+  ra.k_sort_token = L.k_tok;
+  ra.k_count = L.k_count;
+  ra.k_off = L.k_off;
+  ra.err = err ? err : L.err;
+  ra.mref = L.mref;
+  if (s.dtype == BSA_F32) {
+    if (s.D == 64) launch_route_probe<float, 64>(k, v, ra, st);
+    else launch_route_probe<float, 128>(k, v, ra, st);
+  } else {
+    if (s.D == 64) launch_route_probe<__nv_bfloat16, 64>(k, v, ra, st);
+    else launch_route_probe<__nv_bfloat16, 128>(k, v, ra, st);
+  }
+  count_launch();
+  if ((rc = check_cuda(cudaGetLastError(), "route_probe_kernel"))) return rc;
+  // 4. budgeted prefix per (batch, head)
+  route_select_kernel<<<s.B * s.Hq, 1024, 0, st>>>(ra.err, L.q_count, L.k_count, Cq, Ck, density,
+                                                   mask);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "route_select_kernel");
+}

@@ -175,6 +175,32 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
     return out
 
 
+def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=None,
+                           return_err=False, workspace=None):
+    """SVG-EAR error-aware routing: uint8 (B, Hq, Cq, Ck) mask of the blocks to compute
+    exactly, the highest compensation-error-per-pair blocks within ``density`` of the
+    token pairs (and, with ``return_err``, the fp32 block errors)."""
+    _expect_qkv(q, k, v)
+    B, Hq, Sq, D = q.shape
+    _expect(q_labels, "q_labels", (torch.int32,), (1,), (Sq,))
+    _expect(k_labels, "k_labels", (torch.int32,), (1,), (k.shape[2],))
+    _expect_workspace(workspace)
+    _need_cuda(q, k, v, q_labels, k_labels, workspace)
+    shape = make_shape(q, k)
+    Cq, Ck = int(Cq), int(Ck)
+    need = _lib.load().bsa_routing_workspace_bytes(shape, Cq, Ck)
+    if need == 0:
+        raise _lib.BsaError("bsa_routing_workspace_bytes", _lib.BSA_ERR_UNSUPPORTED, _lib.detail())
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, q.device)
+    mask = torch.empty((B, Hq, Cq, Ck), dtype=torch.uint8, device=q.device)
+    err = torch.empty((B, Hq, Cq, Ck), dtype=torch.float32, device=q.device) if return_err else None
+    _call_on(q.device, "bsa_error_aware_block_mask", _ptr(q), _ptr(k), _ptr(v), shape,
+             _ptr(q_labels), Cq, _ptr(k_labels), Ck, float(density), float(scale or 0.0),
+             _ptr(mask), _ptr(err), _ptr(workspace), workspace.numel(), _stream(q.device))
+    return (mask, err) if return_err else mask
+
+
 def antidiagonal_block_scores(q, k, block=128, stride=16, logit_scale=None):
     """XAttention block-mass estimate: fp32 (B, Hq, S/block, S/block), rows sum to 1.
     q: (B,Hq,S,D), k: (B,Hkv,S,D) bf16 with S a multiple of ``block`` (the caller pads)."""

@@ -195,6 +195,38 @@ int bsa_centroid_compensated_attention(const void* q, const void* k, const void*
                                        void* stream);
 
 /*
+ * error_aware_block_mask — SVG-EAR error-aware routing: [SBC] §SVG-EAR — centroid
+ * compensation (an error-aware router chooses which blocks to compute exactly) and the
+ * SVG-EAR abstract (a lightweight probe estimates each block's compensation error; the
+ * blocks with the highest error-to-cost ratio are computed exactly, the rest
+ * compensated). Per (b, query head h), with KV head h / (Hq / Hkv):
+ *   probe of query cluster a : qbar_a, the mean query of the cluster;
+ *   block error  err[a][c]   : || E - A ||_2 with, over the dense logits
+ *                              l_j = scale qbar_a . k_j (max m, Z = sum_j exp(l_j - m)),
+ *                              E = sum_{j in c} exp(l_j - m) v_j / Z (exact contribution)
+ *                              A = n_c exp(scale qbar_a . kbar_c - m) vbar_c / Z (centroid);
+ *   ratio                    : err[a][c] / n_c (error per computed pair), float32;
+ *   mask[a][c] = 1           : the longest prefix of the blocks of non-empty clusters in
+ *                              descending ratio (equal ratios: lower a*Ck + c) whose token
+ *                              pairs n_a n_c sum to at most floor(density * Sq' * Sk'),
+ *                              Sq', Sk' the rows with a valid label.
+ *   q, k, v   : (B,Hq,Sq,D), (B,Hkv,Sk,D), (B,Hkv,Sk,D) device, BSA_BF16 or BSA_F32.
+ *   q_labels  : device int32 (Sq) in [0, Cq);  k_labels : device int32 (Sk) in [0, Ck).
+ *   density   : fraction of token pairs to compute exactly, in [0, 1].
+ *   scale     : <= 0 selects 1/sqrt(D).
+ *   mask      : device uint8 (B, Hq, Cq, Ck), written.
+ *   err       : device float32 (B, Hq, Cq, Ck) or NULL; the block errors when given.
+ *   workspace : >= bsa_routing_workspace_bytes(shape, Cq, Ck) bytes, 256-byte aligned.
+ * Limits: D in {64,128}, Cq, Ck <= 16384, Cq*Ck <= 2^24. Errors: INVALID_ARG for null
+ * pointers or a density outside [0, 1]; UNSUPPORTED past the limits; WORKSPACE.
+ */
+size_t bsa_routing_workspace_bytes(bsa_shape shape, int Cq, int Ck);
+int bsa_error_aware_block_mask(const void* q, const void* k, const void* v, bsa_shape shape,
+                               const int32_t* q_labels, int Cq, const int32_t* k_labels, int Ck,
+                               float density, float scale, uint8_t* mask, float* err,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * select_probe_rows — [SBC] §What mlx-arsenal ships (round-robin over query clusters,
  * weights |G_a| / m_a), §Deviations (middle-out member; weights normalised to sum 1);
  * [SPR] (probes stratified across query groups and ordered by distance to the group
@@ -313,6 +345,19 @@ int bsa_mask_cache_should_refresh(void* state, const void* q, const void* k, bsa
  */
 int bsa_mask_cache_update(void* state, const uint8_t* new_mask, const uint8_t* refresh,
                           uint8_t* block_mask_out, void* stream);
+/*
+ * Layer gate for a layer whose heads are split over several caches (one per GPU,
+ * [HMR] §HEART: the gate looks at the fraction of the layer's heads asking for a
+ * refresh). Each cache is initialised with gate_lo < 0 (no gate of its own); after
+ * should_refresh the callers add their refresh counts over all GPUs (one integer
+ * all-reduce) and pass the sum here: n_refresh_layer of n_heads_layer heads under
+ * gate_lo -> none of this cache's heads refresh, above gate_hi -> all do, otherwise the
+ * per-head flags stand. Not applied on a cache's first call. Updates `refresh` (device
+ * uint8 (B, H) of this cache) in place. Errors: INVALID_ARG for null pointers or a
+ * count outside [0, n_heads_layer].
+ */
+int bsa_mask_cache_layer_gate(void* state, uint8_t* refresh, int n_refresh_layer,
+                              int n_heads_layer, float gate_lo, float gate_hi, void* stream);
 /* Forgets anchors and masks: the next should_refresh refreshes every head. */
 int bsa_mask_cache_reset(void* state, void* stream);
 

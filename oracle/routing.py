@@ -72,23 +72,25 @@ def compensation_errors(q, k, v, q_labels, k_labels, Cq, Ck, scale=None):
     return err
 
 
-def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=None):
-    """SVG-EAR routing: (mask (B, Hq, Cq, Ck) bool, err (B, Hq, Cq, Ck)).
-
-    Per (batch, head), blocks are ranked by err_ac / n_c descending (ties: lower
-    a · Ck + c) and the longest prefix whose token pairs n_a · n_c sum to at most
-    floor(density · Sq · Sk) is kept."""
-    err = compensation_errors(q, k, v, q_labels, k_labels, Cq, Ck, scale)
+def route_blocks(err, q_labels, k_labels, Cq, Ck, density, dtype=np.float64):
+    """The budgeted prefix selection of SVG-EAR routing, given block errors
+    (B, Hq, Cq, Ck): per (batch, head), blocks ranked by err_ac / n_c descending (ties:
+    lower a · Ck + c); the longest prefix whose token pairs n_a · n_c sum to at most
+    floor(density · Sq · Sk) is kept. ``dtype`` is the precision of the ratio (float32
+    when deciding on a kernel's own float32 errors, as the kernel does). Returns a bool
+    mask (B, Hq, Cq, Ck)."""
     n_q = np.bincount(np.asarray(q_labels, dtype=np.int64), minlength=Cq).astype(np.int64)
     n_k = np.bincount(np.asarray(k_labels, dtype=np.int64), minlength=Ck).astype(np.int64)
     cost = np.outer(n_q, n_k)
-    budget = int(np.floor(density * float(n_q.sum()) * float(n_k.sum())))
+    budget = int(np.floor(float(density) * float(n_q.sum()) * float(n_k.sum())))
+    err = np.asarray(err)
     B, Hq = err.shape[:2]
     mask = np.zeros(err.shape, dtype=bool)
     valid = cost > 0
     for b in range(B):
         for h in range(Hq):
-            ratio = np.where(valid, err[b, h] / np.maximum(n_k, 1)[None, :], -1.0)
+            ratio = np.where(valid, err[b, h].astype(dtype) / np.maximum(n_k, 1).astype(dtype)[None, :],
+                             dtype(-1.0))
             flat = ratio.reshape(-1)
             idx = np.arange(flat.size)
             order = np.lexsort((idx, -flat))
@@ -101,4 +103,11 @@ def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=N
                     break
                 total += int(cost[a, c])
                 mask[b, h, a, c] = True
-    return mask, err
+    return mask
+
+
+def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=None):
+    """SVG-EAR routing: (mask (B, Hq, Cq, Ck) bool, err (B, Hq, Cq, Ck)): the block
+    errors of ``compensation_errors`` and the selection of ``route_blocks``."""
+    err = compensation_errors(q, k, v, q_labels, k_labels, Cq, Ck, scale)
+    return route_blocks(err, q_labels, k_labels, Cq, Ck, density), err

@@ -64,3 +64,13 @@ def test_roofline_peak_follows_the_timed_region():
     peaks = {"bf16_tflops": 1653.8, "bf16_tflops_sustained": 1383.1}
     assert bench.roofline_peak(peaks, 0.5) == ("bf16_tflops", 1653.8)
     assert bench.roofline_peak(peaks, 4.0) == ("bf16_tflops_sustained", 1383.1)
+
+
+def test_job_flop_for_replicas_and_head_sharding():
+    """Replicas: N copies of the workload. Heads: the one layer, whatever share of its
+    heads each rank holds."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.job_flop(10.0, 40, 40, 4, "replicas") == 40.0
+    assert bench.job_flop(10.0, 10, 40, 4, "heads") == 40.0
+    assert bench.job_flop(14.0, 14, 40, 3, "heads") == 40.0
