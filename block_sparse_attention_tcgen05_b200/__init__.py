@@ -16,6 +16,7 @@ from .ops import (  # noqa: F401
     error_aware_block_mask,
     probe_dense_attention,
     probe_residual_correction,
+    response_coupled_partition,
     select_probe_rows,
     sliding_tile_block_mask,
     tile_labels,

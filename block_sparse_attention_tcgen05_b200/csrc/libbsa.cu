@@ -3,6 +3,7 @@
 #include "common.cu"
 #include "attention.cu"
 #include "routing.cu"
+#include "partition.cu"
 #include "scoring.cu"
 #include "topp.cu"
 #include "probe.cu"

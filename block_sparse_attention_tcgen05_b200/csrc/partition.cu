@@ -1,0 +1,335 @@
+// SparsePR Response-Coupled Partitioning: query and key clusters from the current
+// call's responses.
+//
+// Source: "Partition the Support, Reconstruct the Residual" (paper summary): queries
+// are sampled from the call and keys grouped by their pre-softmax response; key-group
+// centroids define query coordinates, so queries with a similar response direction
+// share a route; one asymmetric pass; feature ranks rK = 48 and rQ = 64; K/V partitions
+// and routes shared by a KV head's query heads; an online k-means.
+//
+// Per (batch, KV head g) with G = Hq / Hkv query heads:
+//   samples         rK query rows: sample s = token floor((s + 1/2) Sq / rK) of query
+//                   head g G + (s mod G)
+//   key features    f_j = scale * Q_s k_j                                 (Sk x rK)
+//   key groups      k-means of the key features into Ck clusters
+//   query coords    x_i = (scale * q_{h,i} . kbar_{c_t}) over the rQ' = min(rQ, Ck)
+//                   groups c_t = floor((t + 1/2) Ck / rQ') and the G heads, divided by
+//                   its norm                                              (Sq x rQ' G)
+//   query groups    k-means of the query coordinates into Cq clusters
+// k-means (Lloyd): centroids start at rows floor((c + 1/2) N / C); each round assigns
+// rows to the nearest centroid (squared distance, ties to the lower index) and moves
+// each centroid to its rows' mean (an empty cluster keeps its centroid); after `iters`
+// rounds a last assignment gives the labels. Every sum runs in a fixed order, so a
+// call is deterministic.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace bsa {
+
+constexpr int kRcpMaxF = 256;       // feature dimension limit (rK, rQ' G)
+constexpr int kRcpRows = 128;       // rows per assignment CTA
+constexpr int kRcpCentChunk = 32;   // centroids per shared-memory chunk
+
+__device__ __forceinline__ float rcp_f(float x) { return x; }
+__device__ __forceinline__ float rcp_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// grid (ceil(Sk / 64), Hkv, B), 256 threads: feat[b,g,j,s] = scale * q[b, h_s, t_s] . k[b,g,j].
+template <typename T, int D>
+__global__ void __launch_bounds__(256) rcp_key_features_kernel(const T* __restrict__ q,
+                                                               const T* __restrict__ k, int Hq,
+                                                               int Hkv, int Sq, int Sk, int rk,
+                                                               float scale,
+                                                               float* __restrict__ feat) {
+  extern __shared__ float sm_rcp[];
+  float* qs = sm_rcp;              // rk x D
+  float* ks = qs + rk * D;         // 64 x (D + 1)
+  const int g = blockIdx.y, b = blockIdx.z, G = Hq / Hkv;
+  const int j0 = blockIdx.x * 64;
+  for (int e = threadIdx.x; e < rk * D; e += 256) {
+    const int s = e / D, d = e % D;
+    const int tok = static_cast<int>((static_cast<int64_t>(2 * s + 1) * Sq) / (2 * rk));
+    const int h = g * G + s % G;
+    qs[e] = rcp_f(q[((static_cast<int64_t>(b) * Hq + h) * Sq + tok) * D + d]);
+  }
+  const int64_t kb = (static_cast<int64_t>(b) * Hkv + g) * Sk;
+  for (int e = threadIdx.x; e < 64 * D; e += 256) {
+    const int j = e / D, d = e % D;
+    ks[j * (D + 1) + d] = j0 + j < Sk ? rcp_f(k[(kb + j0 + j) * D + d]) : 0.f;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 64 * rk; e += 256) {
+    const int j = e / rk, s = e % rk;
+    if (j0 + j >= Sk) continue;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < D; ++d) acc = fmaf(qs[s * D + d], ks[j * (D + 1) + d], acc);
+    feat[(kb + j0 + j) * rk + s] = scale * acc;
+  }
+}
+
+// grid (C, n_problems): cent[p, c, :] = x[p, floor((2c + 1) N / (2C)), :].
+__global__ void kmeans_init_kernel(const float* __restrict__ x, int N, int F, int C,
+                                   float* __restrict__ cent) {
+  const int c = blockIdx.x;
+  const int64_t p = blockIdx.y;
+  const int row = static_cast<int>((static_cast<int64_t>(2 * c + 1) * N) / (2 * C));
+  for (int f = threadIdx.x; f < F; f += blockDim.x)
+    cent[(p * C + c) * F + f] = x[(p * N + row) * F + f];
+}
+
+// grid (ceil(N / 128), n_problems), 128 threads, one row per thread: the nearest of the
+// C centroids (squared distance, ties to the lower index). Rows are staged feature-major
+// in shared memory, centroids 32 at a time.
+__global__ void __launch_bounds__(kRcpRows) kmeans_assign_kernel(const float* __restrict__ x,
+                                                                 int N, int F, int C,
+                                                                 const float* __restrict__ cent,
+                                                                 int32_t* __restrict__ label) {
+  extern __shared__ float sm_km[];
+  float* xs = sm_km;                       // F x 128
+  float* cs = xs + F * kRcpRows;           // 32 x F
+  const int64_t p = blockIdx.y;
+  const int i0 = blockIdx.x * kRcpRows, tid = threadIdx.x;
+  for (int e = tid; e < kRcpRows * F; e += kRcpRows) {
+    const int r = e / F, f = e % F;
+    xs[f * kRcpRows + r] = i0 + r < N ? x[(p * N + i0 + r) * F + f] : 0.f;
+  }
+  float best = INFINITY;
+  int bc = 0;
+  for (int c0 = 0; c0 < C; c0 += kRcpCentChunk) {
+    const int nc = min(kRcpCentChunk, C - c0);
+    __syncthreads();
+    for (int e = tid; e < nc * F; e += kRcpRows) cs[e] = cent[(p * C + c0) * F + e];
+    __syncthreads();
+    float d[kRcpCentChunk];
+#pragma unroll
+    for (int c = 0; c < kRcpCentChunk; ++c) d[c] = 0.f;
+    for (int f = 0; f < F; ++f) {
+      const float xv = xs[f * kRcpRows + tid];
+#pragma unroll
+      for (int c = 0; c < kRcpCentChunk; ++c) {
+        const float t = xv - cs[(c < nc ? c : 0) * F + f];
+        d[c] = fmaf(t, t, d[c]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < kRcpCentChunk; ++c)
+      if (c < nc && d[c] < best) {
+        best = d[c];
+        bc = c0 + c;
+      }
+  }
+  if (i0 + tid < N) label[p * N + i0 + tid] = bc;
+}
+
+// grid (C, n_problems), 256 threads (thread f holds feature f): the mean of the rows of
+// cluster c, summed in index order; an empty cluster keeps its centroid. With
+// `gather_rows` the rows come from a (n_problems, N, F) source of type T instead of x.
+template <typename T>
+__global__ void __launch_bounds__(256) kmeans_update_kernel(const T* __restrict__ x, int N, int F,
+                                                            int C, const int32_t* __restrict__ label,
+                                                            float* __restrict__ cent) {
+  __shared__ int members[256];
+  __shared__ int n_members;
+  const int c = blockIdx.x, tid = threadIdx.x;
+  const int64_t p = blockIdx.y;
+  const int lane = tid & 31, warp = tid >> 5;
+  __shared__ int warp_n[8];
+  float acc = 0.f;
+  int count = 0;
+  for (int i0 = 0; i0 < N; i0 += 256) {
+    const int i = i0 + tid;
+    const bool mine = i < N && label[p * N + i] == c;
+    const unsigned bal = __ballot_sync(0xffffffffu, mine);
+    if (lane == 0) warp_n[warp] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < 8; ++w) {
+      if (w < warp) before += warp_n[w];
+      total += warp_n[w];
+    }
+    if (mine) members[before + __popc(bal & ((1u << lane) - 1u))] = i;
+    if (tid == 0) n_members = total;
+    __syncthreads();
+    const int nm = n_members;
+    if (tid < F)
+      for (int m = 0; m < nm; ++m) acc += rcp_f(x[(p * N + members[m]) * F + tid]);
+    count += nm;
+    __syncthreads();
+  }
+  if (tid < F && count > 0) cent[(p * C + c) * F + tid] = acc / static_cast<float>(count);
+}
+
+// grid (ceil(Sq / 64), Hkv, B), 256 threads: x[b,g,i,:] = (scale q_{h,i} . kbar_{c_t})
+// over t < rq and the G heads h of KV head g, divided by its norm.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) rcp_query_coords_kernel(const T* __restrict__ q,
+                                                               const float* __restrict__ kbar,
+                                                               int Hq, int Hkv, int Sq, int Ck,
+                                                               int rq, float scale,
+                                                               float* __restrict__ xq) {
+  extern __shared__ float sm_rq[];
+  float* kc = sm_rq;                 // rq x D
+  float* out = kc + rq * D;          // 64 x F
+  const int g = blockIdx.y, b = blockIdx.z, G = Hq / Hkv, F = rq * G;
+  const int i0 = blockIdx.x * 64;
+  const int64_t pg = static_cast<int64_t>(b) * Hkv + g;
+  for (int e = threadIdx.x; e < rq * D; e += 256) {
+    const int t = e / D, d = e % D;
+    const int c = static_cast<int>((static_cast<int64_t>(2 * t + 1) * Ck) / (2 * rq));
+    kc[e] = kbar[(pg * Ck + c) * D + d];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 64 * F; e += 256) {
+    const int i = e / F, f = e % F;
+    const int hh = f / rq, t = f % rq;
+    float acc = 0.f;
+    if (i0 + i < Sq) {
+      const T* qrow = q + ((static_cast<int64_t>(b) * Hq + g * G + hh) * Sq + i0 + i) * D;
+#pragma unroll 8
+      for (int d = 0; d < D; ++d) acc = fmaf(rcp_f(qrow[d]), kc[t * D + d], acc);
+    }
+    out[i * F + f] = scale * acc;
+  }
+  __syncthreads();
+  // one warp per row: norm, then the normalised row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < 64; i += 8) {
+    if (i0 + i >= Sq) continue;
+    float ss = 0.f;
+    for (int f = lane; f < F; f += 32) ss = fmaf(out[i * F + f], out[i * F + f], ss);
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+    for (int f = lane; f < F; f += 32) xq[(pg * Sq + i0 + i) * F + f] = out[i * F + f] * inv;
+  }
+}
+
+namespace {
+struct RcpLayout {
+  float *fk, *xq, *kcent, *qcent, *kbar;
+  size_t bytes;
+};
+RcpLayout carve_rcp(const bsa_shape& s, int Cq, int Ck, int rk, int rq, void* ws) {
+  Carver cv(ws);
+  RcpLayout L{};
+  const size_t P = static_cast<size_t>(s.B) * s.Hkv;
+  const int G = s.Hq / s.Hkv;
+  const int rqe = rq < Ck ? rq : Ck;
+  L.fk = cv.take<float>(P * s.Sk * rk);
+  L.xq = cv.take<float>(P * s.Sq * rqe * G);
+  L.kcent = cv.take<float>(P * Ck * rk);
+  L.qcent = cv.take<float>(P * Cq * rqe * G);
+  L.kbar = cv.take<float>(P * Ck * s.D);
+  L.bytes = align_up(cv.used, 256);
+  return L;
+}
+
+int validate_rcp(const bsa_shape& s, int Cq, int Ck, int rk, int rq, int iters) {
+  if (s.B <= 0 || s.Hq <= 0 || s.Hkv <= 0 || s.Sq <= 0 || s.Sk <= 0)
+    return fail(BSA_ERR_INVALID_ARG, "non-positive shape");
+  if (s.Hq % s.Hkv) return fail(BSA_ERR_INVALID_ARG, "Hq (%d) not a multiple of Hkv (%d)", s.Hq, s.Hkv);
+  if (s.D != 64 && s.D != 128) return fail(BSA_ERR_UNSUPPORTED, "head dim %d not in {64,128}", s.D);
+  if (s.dtype != BSA_BF16 && s.dtype != BSA_F32) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", s.dtype);
+  if (Cq < 1 || Ck < 1 || Cq > s.Sq || Ck > s.Sk)
+    return fail(BSA_ERR_INVALID_ARG, "cluster counts Cq=%d Ck=%d outside [1, S]", Cq, Ck);
+  if (Cq > 4096 || Ck > 4096) return fail(BSA_ERR_UNSUPPORTED, "cluster counts above 4096");
+  if (rk < 1 || rq < 1 || iters < 0) return fail(BSA_ERR_INVALID_ARG, "rK, rQ >= 1, iters >= 0");
+  const int G = s.Hq / s.Hkv;
+  const int rqe = rq < Ck ? rq : Ck;
+  if (rk > kRcpMaxF || rqe * G > kRcpMaxF)
+    return fail(BSA_ERR_UNSUPPORTED, "feature dims rK=%d, rQ'*G=%d above %d", rk, rqe * G, kRcpMaxF);
+  return BSA_OK;
+}
+
+// Lloyd iterations on (P, N, F) features: init, `iters` rounds, last assignment.
+int run_kmeans(const float* x, int P, int N, int F, int C, int iters, float* cent,
+               int32_t* label, cudaStream_t st) {
+  kmeans_init_kernel<<<dim3(C, P), 128, 0, st>>>(x, N, F, C, cent);
+  count_launch();
+  const int smem = (F * kRcpRows + kRcpCentChunk * F) * 4;
+  cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem > 48 * 1024 ? smem : 48 * 1024);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(kmeans_assign)");
+  for (int it = 0; it <= iters; ++it) {
+    kmeans_assign_kernel<<<dim3((N + kRcpRows - 1) / kRcpRows, P), kRcpRows, smem, st>>>(x, N, F, C,
+                                                                                        cent, label);
+    count_launch();
+    if (it == iters) break;
+    kmeans_update_kernel<float><<<dim3(C, P), 256, 0, st>>>(x, N, F, C, label, cent);
+    count_launch();
+  }
+  return check_cuda(cudaGetLastError(), "k-means kernels");
+}
+
+template <typename T, int D>
+int run_rcp(const void* qv, const void* kv, const bsa_shape& s, int Cq, int Ck, int rk, int rq,
+            int iters, float scale, int32_t* q_labels, int32_t* k_labels, const RcpLayout& L,
+            cudaStream_t st) {
+  const T* q = static_cast<const T*>(qv);
+  const T* k = static_cast<const T*>(kv);
+  const int P = s.B * s.Hkv, G = s.Hq / s.Hkv;
+  const int rqe = rq < Ck ? rq : Ck;
+  int rc;
+  {
+    const int smem = (rk * D + 64 * (D + 1)) * 4;
+    cudaError_t e = cudaFuncSetAttribute(rcp_key_features_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem > 48 * 1024 ? smem : 48 * 1024);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(rcp_key_features)");
+    rcp_key_features_kernel<T, D><<<dim3((s.Sk + 63) / 64, s.Hkv, s.B), 256, smem, st>>>(
+        q, k, s.Hq, s.Hkv, s.Sq, s.Sk, rk, scale, L.fk);
+    count_launch();
+  }
+  if ((rc = run_kmeans(L.fk, P, s.Sk, rk, Ck, iters, L.kcent, k_labels, st))) return rc;
+  // key-group centroids in key space
+  kmeans_update_kernel<T><<<dim3(Ck, P), 256, 0, st>>>(k, s.Sk, D, Ck, k_labels, L.kbar);
+  count_launch();
+  {
+    const int smem = (rqe * D + 64 * rqe * G) * 4;
+    cudaError_t e = cudaFuncSetAttribute(rcp_query_coords_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem > 48 * 1024 ? smem : 48 * 1024);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(rcp_query_coords)");
+    rcp_query_coords_kernel<T, D><<<dim3((s.Sq + 63) / 64, s.Hkv, s.B), 256, smem, st>>>(
+        q, L.kbar, s.Hq, s.Hkv, s.Sq, Ck, rqe, scale, L.xq);
+    count_launch();
+  }
+  return run_kmeans(L.xq, P, s.Sq, rqe * G, Cq, iters, L.qcent, q_labels, st);
+}
+}  // namespace
+
+}  // namespace bsa
+
+extern "C" size_t bsa_partition_workspace_bytes(bsa_shape shape, int Cq, int Ck, int r_k, int r_q) {
+  if (bsa::validate_rcp(shape, Cq, Ck, r_k, r_q, 0)) return 0;
+  return bsa::carve_rcp(shape, Cq, Ck, r_k, r_q, nullptr).bytes;
+}
+
+extern "C" int bsa_response_coupled_partition(const void* q, const void* k, bsa_shape shape, int Cq,
+                                              int Ck, int r_k, int r_q, int iters, float scale,
+                                              int32_t* q_labels, int32_t* k_labels, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  using namespace bsa;
+  int rc = validate_rcp(shape, Cq, Ck, r_k, r_q, iters);
+  if (rc) return rc;
+  if (!q || !k || !q_labels || !k_labels) return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+  RcpLayout L = carve_rcp(shape, Cq, Ck, r_k, r_q, workspace);
+  if (!workspace || workspace_bytes < L.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, L.bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(BSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(shape.D));
+  cudaStream_t st = as_stream(stream);
+  if (shape.dtype == BSA_F32)
+    return shape.D == 64 ? run_rcp<float, 64>(q, k, shape, Cq, Ck, r_k, r_q, iters, sc, q_labels,
+                                              k_labels, L, st)
+                         : run_rcp<float, 128>(q, k, shape, Cq, Ck, r_k, r_q, iters, sc, q_labels,
+                                               k_labels, L, st);
+  return shape.D == 64 ? run_rcp<__nv_bfloat16, 64>(q, k, shape, Cq, Ck, r_k, r_q, iters, sc,
+                                                    q_labels, k_labels, L, st)
+                       : run_rcp<__nv_bfloat16, 128>(q, k, shape, Cq, Ck, r_k, r_q, iters, sc,
+                                                     q_labels, k_labels, L, st);
+}

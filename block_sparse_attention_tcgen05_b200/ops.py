@@ -201,6 +201,28 @@ def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=N
     return (mask, err) if return_err else mask
 
 
+def response_coupled_partition(q, k, Cq, Ck, r_k=48, r_q=64, iters=8, scale=None, workspace=None):
+    """SparsePR Response-Coupled Partitioning: int32 query labels (B, Hkv, Sq) and key
+    labels (B, Hkv, Sk), one partition per KV head shared by its query heads."""
+    _expect_qkv(q, k)
+    _expect_workspace(workspace)
+    _need_cuda(q, k, workspace)
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    shape = make_shape(q, k)
+    need = _lib.load().bsa_partition_workspace_bytes(shape, int(Cq), int(Ck), int(r_k), int(r_q))
+    if need == 0:
+        raise _lib.BsaError("bsa_partition_workspace_bytes", _lib.BSA_ERR_UNSUPPORTED, _lib.detail())
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, q.device)
+    ql = torch.empty((B, Hkv, Sq), dtype=torch.int32, device=q.device)
+    kl = torch.empty((B, Hkv, Sk), dtype=torch.int32, device=q.device)
+    _call_on(q.device, "bsa_response_coupled_partition", _ptr(q), _ptr(k), shape, int(Cq), int(Ck),
+             int(r_k), int(r_q), int(iters), float(scale or 0.0), _ptr(ql), _ptr(kl),
+             _ptr(workspace), workspace.numel(), _stream(q.device))
+    return ql, kl
+
+
 def antidiagonal_block_scores(q, k, block=128, stride=16, logit_scale=None):
     """XAttention block-mass estimate: fp32 (B, Hq, S/block, S/block), rows sum to 1.
     q: (B,Hq,S,D), k: (B,Hkv,S,D) bf16 with S a multiple of ``block`` (the caller pads)."""

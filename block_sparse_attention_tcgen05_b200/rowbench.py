@@ -179,6 +179,51 @@ def bench_attention(timer, dev, hbm, tc, out):
     out[-1]["speedup_of_sparse_call"] = dense_ms / ms
 
 
+def fp32_alu_tflops(dev):
+    """CUDA-core fp32 peak of the part: SMs x 128 FMA lanes x 2 FLOP x the maximum SM
+    clock (for kernels that run on the FMA pipe rather than the tensor cores)."""
+    props = torch.cuda.get_device_properties(dev)
+    mhz = 1965.0
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def bench_routing_and_sta(timer, dev, hbm, tc, out):
+    H = 40
+    q, k, v = video_inputs(dev, H)
+    labels, C = ops.tile_labels(*GRID, TILE, device=dev)
+    S = q.shape[2]
+    # f1: SVG-EAR error-aware routing at density 0.22: the probe kernel computes, per
+    # head, every query cluster's mean query against every key (logits and the
+    # exp-weighted values): 4 D FLOP per (probe, key) pair on the FMA pipe
+    ws = torch.empty(ops._lib.load().bsa_routing_workspace_bytes(ops.make_shape(q, k), C, C),
+                     dtype=torch.uint8, device=dev)
+    ms = timer(lambda: ops.error_aware_block_mask(q, k, v, labels, labels, C, C, 0.22,
+                                                  workspace=ws))
+    r = row("f1", "SVG-EAR error-aware routing (H=40, 245 probes per head over 32760 keys, "
+            "density 0.22)", ms, 4.0 * D * C * S * H, "FLOP", "alu", None)
+    alu = fp32_alu_tflops(dev)
+    r.update({"achieved": 4.0 * D * C * S * H / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+              "peak": alu, "frac": 4.0 * D * C * S * H / (ms * 1e-3) / 1e12 / alu,
+              "peak_note": "fp32 FMA pipe: SMs x 128 lanes x 2 x max SM clock"})
+    out.append(r)
+    # f3: the recipe's sliding-tile window mask, (3, 3, 5) tiles, driving the attention
+    n_tiles = tuple(-(-g // t) for g, t in zip(GRID, TILE))
+    mask = ops.sliding_tile_block_mask(n_tiles, (3, 3, 5), device=dev)
+    ws = torch.empty(ops.attention_workspace_bytes(q, k, C, C), dtype=torch.uint8, device=dev)
+    o = torch.empty((1, H, S, D), dtype=torch.float32, device=dev)
+    cnt = torch.bincount(labels.long(), minlength=C).double()
+    pairs = float(cnt @ mask.double() @ cnt) * H
+    ms = timer(lambda: ops.centroid_compensated_attention(q, k, v, labels, labels, mask, Cq=C, Ck=C,
+                                                          out=o, workspace=ws))
+    out.append(row("f3", "compensated attention call on the sliding-tile (3,3,5) window mask "
+                   f"({pairs / (H * S * S):.3f} of token pairs)", ms, pairs * 4 * D, "FLOP",
+                   "tensor", tc))
+
+
 def bench_probe_and_repair(timer, dev, hbm, tc, out):
     Hq, Hkv, S, M = 24, 8, 32768, 64
     g = torch.Generator(device=dev).manual_seed(4)
@@ -222,6 +267,8 @@ def main():
     bench_cache_and_scoring(timer, dev, hbm, tc, out)
     torch.cuda.empty_cache()
     bench_attention(timer, dev, hbm, tc, out)
+    torch.cuda.empty_cache()
+    bench_routing_and_sta(timer, dev, hbm, tc, out)
     torch.cuda.empty_cache()
     bench_probe_and_repair(timer, dev, hbm, tc, out)
     st, _ = ops.device_status(dev)

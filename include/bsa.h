@@ -227,6 +227,36 @@ int bsa_error_aware_block_mask(const void* q, const void* k, const void* v, bsa_
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * response_coupled_partition — SparsePR Response-Coupled Partitioning: [SPR] (queries
+ * sampled from the call; keys grouped by their pre-softmax response, values following
+ * their keys; key-group centroids define query coordinates so that queries with a
+ * similar response direction share a route; one asymmetric pass; ranks rK = 48, rQ = 64;
+ * K/V partitions and routes shared by a KV head's query heads; online k-means).
+ * Per (b, KV head g), G = Hq / Hkv:
+ *   samples      : rK query rows, sample s = token floor((s+1/2) Sq / rK) of query head
+ *                  g*G + s % G;
+ *   key features : f_j = scale * Q_s k_j (rK values per key), k-means into Ck groups;
+ *   query coords : x_i = (scale * q_{h,i} . kbar_{c_t}) over rQ' = min(rQ, Ck) groups
+ *                  c_t = floor((t+1/2) Ck / rQ') and the G heads, divided by its norm;
+ *                  k-means into Cq groups.
+ *   k-means      : Lloyd; centroids start at rows floor((c+1/2) N / C); `iters` rounds
+ *                  of (nearest centroid by squared distance, ties to the lower index;
+ *                  centroid = mean of its rows, an empty cluster keeps its centroid),
+ *                  then a last assignment. Sums run in a fixed order (deterministic).
+ *   q, k      : (B,Hq,Sq,D), (B,Hkv,Sk,D) device, BSA_BF16 or BSA_F32; D in {64,128}.
+ *   q_labels  : device int32 (B, Hkv, Sq), written (one partition per KV head).
+ *   k_labels  : device int32 (B, Hkv, Sk), written.
+ *   scale     : <= 0 selects 1/sqrt(D).
+ *   workspace : >= bsa_partition_workspace_bytes(shape, Cq, Ck, r_k, r_q), 256-aligned.
+ * Limits: 1 <= Cq <= min(Sq, 4096), 1 <= Ck <= min(Sk, 4096), rK <= 256, rQ'*G <= 256.
+ */
+size_t bsa_partition_workspace_bytes(bsa_shape shape, int Cq, int Ck, int r_k, int r_q);
+int bsa_response_coupled_partition(const void* q, const void* k, bsa_shape shape, int Cq, int Ck,
+                                   int r_k, int r_q, int iters, float scale, int32_t* q_labels,
+                                   int32_t* k_labels, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
  * select_probe_rows — [SBC] §What mlx-arsenal ships (round-robin over query clusters,
  * weights |G_a| / m_a), §Deviations (middle-out member; weights normalised to sum 1);
  * [SPR] (probes stratified across query groups and ordered by distance to the group
