@@ -15,6 +15,7 @@ from .ops import (  # noqa: F401
     device_status,
     error_aware_block_mask,
     probe_dense_attention,
+    probe_budget_block_mask,
     probe_residual_correction,
     response_coupled_partition,
     select_probe_rows,

@@ -53,6 +53,8 @@ SIGNATURES = {
     "bsa_routing_workspace_bytes": (_sz, [Shape, _i, _i]),
     "bsa_error_aware_block_mask": (
         _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _f, _f, _vp, _vp, _vp, _sz, _vp]),
+    "bsa_probe_budget_block_mask": (
+        _i, [_vp, _vp, Shape, _vp, _i, _vp, _i, _f, _i, _f, _vp, _vp, _vp, _sz, _vp]),
     "bsa_partition_workspace_bytes": (_sz, [Shape, _i, _i, _i, _i]),
     "bsa_response_coupled_partition": (
         _i, [_vp, _vp, Shape, _i, _i, _i, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]),

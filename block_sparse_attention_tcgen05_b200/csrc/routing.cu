@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
 __global__ void __launch_bounds__(1024) route_select_kernel(const float* __restrict__ err,
                                                             const int32_t* __restrict__ q_count,
                                                             const int32_t* __restrict__ k_count,
-                                                            int Cq, int Ck, float density,
+                                                            int Cq, int Ck, double density,
                                                             uint8_t* __restrict__ mask) {
   __shared__ unsigned long long hist[256];
   __shared__ unsigned long long s_part[32];
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(1024) route_select_kernel(const float* __restr
   if (lane == 0) { atomicAdd(&s_sq, sq); atomicAdd(&s_sk, sk); }
   __syncthreads();
   const long long budget = static_cast<long long>(
-      floor(static_cast<double>(density) * static_cast<double>(s_sq) * static_cast<double>(s_sk)));
+      floor(density * static_cast<double>(s_sq) * static_cast<double>(s_sk)));
   auto key_of = [&](int64_t e, uint32_t& key, long long& cost) -> bool {
     const int a_ = static_cast<int>(e / Ck), c_ = static_cast<int>(e % Ck);
     const int na = q_count[a_], nc = k_count[c_];
@@ -329,6 +329,59 @@ __global__ void __launch_bounds__(1024) route_select_kernel(const float* __restr
   }
 }
 
+// ---------------------------------------------------------------- centroid mass
+// grid (Cq, Hq, B), 128 threads: mass[b,h,a,c] = softmax over the key clusters of
+// scale * qbar_a . kbar_c + ln n_c (empty key clusters 0; an empty query cluster's row
+// is 0): the share of the mean query's attention that falls on each key cluster when
+// every key is replaced by its cluster centroid.
+template <int D>
+__global__ void __launch_bounds__(128) centroid_mass_kernel(const RouteArgs a,
+                                                            float* __restrict__ mass) {
+  __shared__ float qa[D];
+  __shared__ float red[4];
+  const int c0 = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int hkv = h / (a.Hq / a.Hkv);
+  const int64_t bq = static_cast<int64_t>(b) * a.Hq + h;
+  const int64_t bk = static_cast<int64_t>(b) * a.Hkv + hkv;
+  float* row = mass + (bq * a.Cq + c0) * a.Ck;
+  if (a.q_count[c0] <= 0) {
+    for (int c = tid; c < a.Ck; c += 128) row[c] = 0.f;
+    return;
+  }
+  for (int d = tid; d < D; d += 128) qa[d] = a.qbar[(bq * a.Cq + c0) * D + d];
+  __syncthreads();
+  float mx = -INFINITY;
+  for (int c = tid; c < a.Ck; c += 128) {
+    const int n = a.k_count[c];
+    float l = -INFINITY;
+    if (n > 0) {
+      float acc = 0.f;
+      const float* kc = a.kbar + (bk * a.Ck + c) * D;
+#pragma unroll 8
+      for (int d = 0; d < D; ++d) acc = fmaf(qa[d], kc[d], acc);
+      l = a.scale * acc + logf(static_cast<float>(n));
+    }
+    row[c] = l;
+    mx = fmaxf(mx, l);
+  }
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  float sum = 0.f;
+  for (int c = tid; c < a.Ck; c += 128) {
+    const float e = row[c] == -INFINITY ? 0.f : __expf(row[c] - mx);
+    row[c] = e;
+    sum += e;
+  }
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if ((tid & 31) == 0) red[tid >> 5] = sum;
+  __syncthreads();
+  const float inv = 1.f / ((red[0] + red[1]) + (red[2] + red[3]));
+  for (int c = tid; c < a.Ck; c += 128) row[c] *= inv;
+}
+
 namespace {
 struct RouteLayout {
   int32_t *q_tok, *q_count, *q_off, *k_tok, *k_count, *k_off;
@@ -375,6 +428,11 @@ void launch_route_probe(const void* k, const void* v, const RouteArgs& ra, cudaS
 }
 }  // namespace
 
+int route_prologue(const void* q, const void* k, const void* v, const bsa_shape& shape,
+                   const int32_t* q_labels, int Cq, const int32_t* k_labels, int Ck, float scale,
+                   uint8_t* mask, float* err, const RouteLayout& L, cudaStream_t st, float density,
+                   int M);
+
 }  // namespace bsa
 
 extern "C" size_t bsa_routing_workspace_bytes(bsa_shape shape, int Cq, int Ck) {
@@ -400,7 +458,19 @@ extern "C" int bsa_error_aware_block_mask(const void* q, const void* k, const vo
     return fail(BSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, L.bytes);
   if (reinterpret_cast<uintptr_t>(workspace) % 256)
     return fail(BSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
-  cudaStream_t st = as_stream(stream);
+  return route_prologue(q, k, v, shape, q_labels, Cq, k_labels, Ck, scale, mask, err, L,
+                        as_stream(stream), density, -1);
+}
+
+namespace bsa {
+// Shared steps of both routers: label sorts, cluster means, then either the probe
+// errors (M < 0: SVG-EAR) or the centroid masses (M >= 0: probe budget), and the exact
+// budgeted selection at `density` (less M / Sq for the probe budget).
+int route_prologue(const void* q, const void* k, const void* v, const bsa_shape& shape,
+                   const int32_t* q_labels, int Cq, const int32_t* k_labels, int Ck, float scale,
+                   uint8_t* mask, float* err, const RouteLayout& L, cudaStream_t st, float density,
+                   int M) {
+  int rc;
   const bsa_shape& s = shape;
   // 1. stable label sorts (cluster-major token order, counts, offsets)
   {
@@ -411,23 +481,26 @@ extern "C" int bsa_error_aware_block_mask(const void* q, const void* k, const vo
     if ((rc = launch_label_sorts(jk, &jq, st))) return rc;
   }
   // 2. cluster means of Q (probes), K and V (centroids), fp32
+  const bool with_v = M < 0;
   if (s.dtype == BSA_F32) {
     cluster_mean_kernel<float><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(
         static_cast<const float*>(q), L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.D, s.Hq, L.qbar);
     cluster_mean_kernel<float><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
         static_cast<const float*>(k), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.kbar);
-    cluster_mean_kernel<float><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
-        static_cast<const float*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
+    if (with_v)
+      cluster_mean_kernel<float><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
+          static_cast<const float*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
   } else {
     using bf = __nv_bfloat16;
     cluster_mean_kernel<bf><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(
         static_cast<const bf*>(q), L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.D, s.Hq, L.qbar);
     cluster_mean_kernel<bf><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
         static_cast<const bf*>(k), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.kbar);
-    cluster_mean_kernel<bf><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
-        static_cast<const bf*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
+    if (with_v)
+      cluster_mean_kernel<bf><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
+          static_cast<const bf*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
   }
-  for (int i = 0; i < 3; ++i) count_launch();
+  for (int i = 0; i < (with_v ? 3 : 2); ++i) count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "cluster_mean_kernel"))) return rc;
   // 3. probe errors
   RouteArgs ra{};
@@ -448,18 +521,53 @@ extern "C" int bsa_error_aware_block_mask(const void* q, const void* k, const vo
   ra.k_off = L.k_off;
   ra.err = err ? err : L.err;
   ra.mref = L.mref;
-  if (s.dtype == BSA_F32) {
-    if (s.D == 64) launch_route_probe<float, 64>(k, v, ra, st);
-    else launch_route_probe<float, 128>(k, v, ra, st);
+  double route_density = static_cast<double>(density);
+  if (with_v) {
+    if (s.dtype == BSA_F32) {
+      if (s.D == 64) launch_route_probe<float, 64>(k, v, ra, st);
+      else launch_route_probe<float, 128>(k, v, ra, st);
+    } else {
+      if (s.D == 64) launch_route_probe<__nv_bfloat16, 64>(k, v, ra, st);
+      else launch_route_probe<__nv_bfloat16, 128>(k, v, ra, st);
+    }
   } else {
-    if (s.D == 64) launch_route_probe<__nv_bfloat16, 64>(k, v, ra, st);
-    else launch_route_probe<__nv_bfloat16, 128>(k, v, ra, st);
+    if (s.D == 64)
+      centroid_mass_kernel<64><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(ra, ra.err);
+    else
+      centroid_mass_kernel<128><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(ra, ra.err);
+    // the probe rows' M x Sk pairs come out of the budget first
+    route_density = route_density - static_cast<double>(M) / static_cast<double>(s.Sq);
+    if (route_density < 0.0) route_density = 0.0;
   }
   count_launch();
-  if ((rc = check_cuda(cudaGetLastError(), "route_probe_kernel"))) return rc;
+  if ((rc = check_cuda(cudaGetLastError(), "route score kernel"))) return rc;
   // 4. budgeted prefix per (batch, head)
-  route_select_kernel<<<s.B * s.Hq, 1024, 0, st>>>(ra.err, L.q_count, L.k_count, Cq, Ck, density,
-                                                   mask);
+  route_select_kernel<<<s.B * s.Hq, 1024, 0, st>>>(ra.err, L.q_count, L.k_count, Cq, Ck,
+                                                   route_density, mask);
   count_launch();
   return check_cuda(cudaGetLastError(), "route_select_kernel");
+}
+}  // namespace bsa
+
+extern "C" int bsa_probe_budget_block_mask(const void* q, const void* k, bsa_shape shape,
+                                           const int32_t* q_labels, int Cq,
+                                           const int32_t* k_labels, int Ck, float density, int M,
+                                           float scale, uint8_t* mask, float* mass,
+                                           void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+  using namespace bsa;
+  int rc = validate_route(shape, Cq, Ck);
+  if (rc) return rc;
+  if (!q || !k || !q_labels || !k_labels || !mask)
+    return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!(density >= 0.f && density <= 1.f))
+    return fail(BSA_ERR_INVALID_ARG, "density %g outside [0, 1]", static_cast<double>(density));
+  if (M < 0) return fail(BSA_ERR_INVALID_ARG, "M %d < 0", M);
+  RouteLayout L = carve_route(shape, Cq, Ck, workspace);
+  if (!workspace || workspace_bytes < L.bytes)
+    return fail(BSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", workspace_bytes, L.bytes);
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(BSA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  return route_prologue(q, k, nullptr, shape, q_labels, Cq, k_labels, Ck, scale, mask, mass, L,
+                        as_stream(stream), density, M);
 }

@@ -201,6 +201,32 @@ def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=N
     return (mask, err) if return_err else mask
 
 
+def probe_budget_block_mask(q, k, q_labels, k_labels, Cq, Ck, density, M, scale=None,
+                            return_mass=False, workspace=None):
+    """SparsePR's router: uint8 (B, Hq, Cq, Ck) mask of the highest attention-mass-per-pair
+    cells within ``density`` of the token pairs after the M probe rows' pairs are
+    reserved (and, with ``return_mass``, the fp32 cell masses)."""
+    _expect_qkv(q, k)
+    B, Hq, Sq, D = q.shape
+    _expect(q_labels, "q_labels", (torch.int32,), (1,), (Sq,))
+    _expect(k_labels, "k_labels", (torch.int32,), (1,), (k.shape[2],))
+    _expect_workspace(workspace)
+    _need_cuda(q, k, q_labels, k_labels, workspace)
+    shape = make_shape(q, k)
+    Cq, Ck = int(Cq), int(Ck)
+    need = _lib.load().bsa_routing_workspace_bytes(shape, Cq, Ck)
+    if need == 0:
+        raise _lib.BsaError("bsa_routing_workspace_bytes", _lib.BSA_ERR_UNSUPPORTED, _lib.detail())
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, q.device)
+    mask = torch.empty((B, Hq, Cq, Ck), dtype=torch.uint8, device=q.device)
+    mass = torch.empty((B, Hq, Cq, Ck), dtype=torch.float32, device=q.device) if return_mass else None
+    _call_on(q.device, "bsa_probe_budget_block_mask", _ptr(q), _ptr(k), shape, _ptr(q_labels), Cq,
+             _ptr(k_labels), Ck, float(density), int(M), float(scale or 0.0), _ptr(mask), _ptr(mass),
+             _ptr(workspace), workspace.numel(), _stream(q.device))
+    return (mask, mass) if return_mass else mask
+
+
 def response_coupled_partition(q, k, Cq, Ck, r_k=48, r_q=64, iters=8, scale=None, workspace=None):
     """SparsePR Response-Coupled Partitioning: int32 query labels (B, Hkv, Sq) and key
     labels (B, Hkv, Sk), one partition per KV head shared by its query heads."""

@@ -227,6 +227,26 @@ int bsa_error_aware_block_mask(const void* q, const void* k, const void* v, bsa_
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * probe_budget_block_mask — SparsePR's router with the probe cost reserved first: [SPR]
+ * (executed-pair density is the routing density plus M/Nq; the router reserves the
+ * probe cost first; whole cells are atomic). Per (b, query head), cells are scored by
+ * their centroid-estimated attention mass: for the mean query qbar_a of query cluster a,
+ *   mass[a][c] = softmax over non-empty key clusters of (scale qbar_a . kbar_c + ln n_c)
+ * (0 for empty clusters), ranked by mass / n_c (mass per computed pair, equal ratios:
+ * lower a*Ck + c), and the longest prefix whose pairs fit
+ * floor(max(0, density - M / Sq) * Sq' * Sk') is kept (Sq', Sk' rows with a valid label).
+ *   q, k      : (B,Hq,Sq,D), (B,Hkv,Sk,D) device, BSA_BF16 or BSA_F32.
+ *   M         : probe rows reserved (>= 0).
+ *   mask      : device uint8 (B, Hq, Cq, Ck), written. mass: float32 (B,Hq,Cq,Ck) or NULL.
+ *   workspace : >= bsa_routing_workspace_bytes(shape, Cq, Ck) bytes, 256-byte aligned.
+ * Limits and errors as error_aware_block_mask; INVALID_ARG for M < 0.
+ */
+int bsa_probe_budget_block_mask(const void* q, const void* k, bsa_shape shape,
+                                const int32_t* q_labels, int Cq, const int32_t* k_labels, int Ck,
+                                float density, int M, float scale, uint8_t* mask, float* mass,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * response_coupled_partition — SparsePR Response-Coupled Partitioning: [SPR] (queries
  * sampled from the call; keys grouped by their pre-softmax response, values following
  * their keys; key-group centroids define query coordinates so that queries with a

@@ -43,4 +43,10 @@ from .repair import (  # noqa: F401
 from .cache import HeadMaskCache, pooled_qk, qk_drift  # noqa: F401
 from .accounting import executed_pairs  # noqa: F401
 from .partition import kmeans, response_coupled_partition  # noqa: F401
-from .routing import compensation_errors, error_aware_block_mask, route_blocks  # noqa: F401
+from .routing import (  # noqa: F401
+    centroid_mass,
+    compensation_errors,
+    error_aware_block_mask,
+    probe_budget_block_mask,
+    route_blocks,
+)

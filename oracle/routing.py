@@ -111,3 +111,46 @@ def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=N
     errors of ``compensation_errors`` and the selection of ``route_blocks``."""
     err = compensation_errors(q, k, v, q_labels, k_labels, Cq, Ck, scale)
     return route_blocks(err, q_labels, k_labels, Cq, Ck, density), err
+
+
+def centroid_mass(q, k, q_labels, k_labels, Cq, Ck, scale=None):
+    """Block mass estimate (B, Hq, Cq, Ck): for the mean query q̄_a of each query
+    cluster, the softmax over key clusters of scale · q̄_a · k̄_c + ln n_c (empty key
+    clusters: 0), the share of q̄_a's attention that falls on each key cluster when
+    every key is replaced by its cluster centroid ("Sparse-block compensation",
+    §SVG-EAR: a cluster enters the softmax as one term with the log-count prior).
+    Rows of empty query clusters are 0."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = D ** -0.5
+    kl = np.asarray(k_labels, dtype=np.int64)
+    v0 = np.zeros_like(k[0, 0])
+    out = np.zeros((B, Hq, Cq, Ck))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head(h, Hq, Hkv)
+            n_q, qbar = _query_centroids(q[b, h], q_labels, Cq)
+            n_k, kbar, _ = cluster_centroids(k[b, g], v0, kl, Ck)
+            with np.errstate(divide="ignore"):
+                logits = scale * (qbar @ kbar.T) + np.log(n_k.astype(np.float64))[None, :]
+            m = logits.max(1, keepdims=True)
+            e = np.exp(logits - m)
+            out[b, h] = e / e.sum(1, keepdims=True)
+            out[b, h, n_q == 0] = 0.0
+    return out
+
+
+def probe_budget_block_mask(q, k, q_labels, k_labels, Cq, Ck, density, M, scale=None):
+    """SparsePR's router with the probe cost reserved first ("Partition the Support,
+    Reconstruct the Residual": executed-pair density is the routing density plus M/Nq,
+    and the router reserves the probe cost before routing). Reading: cells are ranked
+    by their centroid-estimated attention mass per computed pair (``centroid_mass`` /
+    n_c) and the budgeted prefix of ``route_blocks`` is taken with the routing density
+    max(0, density − M / Sq). Returns (mask (B, Hq, Cq, Ck) bool, mass)."""
+    mass = centroid_mass(q, k, q_labels, k_labels, Cq, Ck, scale)
+    Sq = len(np.asarray(q_labels))
+    route = max(0.0, float(density) - float(M) / Sq)
+    return route_blocks(mass, q_labels, k_labels, Cq, Ck, route), mass

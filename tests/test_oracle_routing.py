@@ -101,3 +101,39 @@ def test_empty_clusters_are_never_kept():
     assert not mask[:, :, 4].any() and not mask[:, :, :, 3:].any()
     assert mask[:, :, :4, :3].all()
     assert (err[:, :, 4] == 0).all() and (err[:, :, :, 3:] == 0).all()
+
+
+def test_centroid_mass_is_the_softmax_over_centroid_terms_by_library():
+    """The cell mass equals torch's softmax of scale · q̄_a · k̄_c + ln n_c over the
+    non-empty key clusters; rows sum to 1."""
+    q, k, v, ql, kl = _case(seed=4, Hq=2, Hkv=1, C=5)
+    kl = np.where(kl == 2, 0, kl)          # key cluster 2 empty
+    mass = oracle.centroid_mass(q, k, ql, kl, 5, 5)
+    for h in range(2):
+        for a in range(5):
+            qbar = torch.from_numpy(q[0, h, ql == a].mean(0))
+            logits = []
+            for c in (0, 1, 3, 4):
+                kb = torch.from_numpy(k[0, 0, kl == c].mean(0))
+                logits.append((qbar @ kb) * 8 ** -0.5 + np.log((kl == c).sum()))
+            p = torch.softmax(torch.stack(logits), 0).numpy()
+            np.testing.assert_allclose(mass[0, h, a, [0, 1, 3, 4]], p, rtol=1e-12)
+            assert mass[0, h, a, 2] == 0.0
+    np.testing.assert_allclose(mass.sum(-1), 1.0)
+
+
+def test_probe_budget_reserves_the_probe_cost_first():
+    """With M probe rows the routing budget is (density − M/Sq)·Sq·Sk pairs: the kept
+    cells plus the M·Sk probe pairs never exceed density·Sq·Sk, and the mask is the
+    budgeted prefix of the mass-per-pair order."""
+    q, k, v, ql, kl = _case(seed=5, Hq=2, Hkv=2, C=6)
+    nq, nk = np.bincount(ql, minlength=6), np.bincount(kl, minlength=6)
+    for density, M in ((0.3, 8), (0.5, 12), (0.1, 10)):
+        mask, mass = oracle.probe_budget_block_mask(q, k, ql, kl, 6, 6, density, M)
+        for h in range(2):
+            pairs = (nq[:, None] * nk[None, :])[mask[0, h]].sum()
+            assert pairs <= max(0.0, density * 48 * 48 - M * 48) + 1e-9
+            if M / 48 >= density:            # the probes alone use the whole budget
+                assert pairs == 0
+        want = oracle.route_blocks(mass, ql, kl, 6, 6, max(0.0, density - M / 48))
+        np.testing.assert_array_equal(mask, want)

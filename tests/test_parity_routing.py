@@ -121,3 +121,31 @@ def test_routing_video_static_then_attention():
     assert np.abs(g - ref).max() <= 2e-2
     assert np.linalg.norm(g - ref) / np.linalg.norm(ref) <= 5e-3
     assert bsa.device_status()[0] == 0
+
+
+@pytest.mark.parametrize("dtype,D,Hq,Hkv", [("bf16", 128, 6, 2), ("f32", 64, 2, 2)])
+def test_probe_budget_router(dtype, D, Hq, Hkv):
+    """SparsePR's router ("Partition the Support, Reconstruct the Residual": the router
+    reserves the probe cost first): cell masses against the oracle at a tolerance, and
+    the mask bit for bit against the oracle's budgeted prefix on the GPU's own masses with
+    the routing density max(0, density - M / Sq)."""
+    bsa = _bsa()
+    g = np.random.default_rng(35)
+    S, Cq, Ck, M = 2048, 16, 16, 64
+    ql = g.permutation(np.arange(S) % Cq)
+    kl = g.permutation(np.concatenate([np.arange(Ck - 1), g.integers(0, Ck - 1, S - Ck + 1)]))
+    q, k, _ = wl.gaussian_qkv(1, Hq, Hkv, S, D, dtype, seed=36)
+    ref_mass = oracle.centroid_mass(q.double().numpy(), k.double().numpy(), ql, kl, Cq, Ck)
+    for density in (0.22, 0.5, 0.02):
+        mask, mass = bsa.probe_budget_block_mask(
+            q.cuda(), k.cuda(), torch.as_tensor(ql, dtype=torch.int32).cuda(),
+            torch.as_tensor(kl, dtype=torch.int32).cuda(), Cq, Ck, density, M, return_mass=True)
+        mask, mass = mask.cpu().numpy().astype(bool), mass.cpu().numpy()
+        assert np.abs(mass - ref_mass).max() <= 1e-4
+        route = max(0.0, float(np.float32(density)) - M / S)
+        same = oracle.route_blocks(mass, ql, kl, Cq, Ck, route, dtype=np.float32)
+        np.testing.assert_array_equal(mask, same)
+        nq, nk = np.bincount(ql, minlength=Cq), np.bincount(kl, minlength=Ck)
+        pairs = [(nq[:, None] * nk[None, :])[mask[0, h]].sum() for h in range(Hq)]
+        assert max(pairs) + M * S <= max(density * S * S, M * S)
+    assert bsa.device_status()[0] == 0
