@@ -283,6 +283,8 @@ struct PlanArgs {
   int greedy;
   int32_t* row_token;         // out: token of each planned row (-1 = pad)
   int32_t* row_label;         // out: its label (-1 = pad)
+  int4* pieces;               // scratch: (cluster, first sorted slot, rows, first row)
+  int max_pieces;
 };
 
 __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs pa) {
@@ -296,11 +298,11 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
   __shared__ int s_total;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  if (pa.greedy) {
+  if (pa.greedy) {  // word-major (any[w * Cq + c]): candidate threads read consecutive words
     for (int e = tid; e < Cq * Wc; e += 1024) {
       uint32_t x = 0;
       for (int sl = 0; sl < pa.n_slices; ++sl) x |= pa.cbits[static_cast<size_t>(sl) * Cq * Wc + e];
-      any[e] = x;
+      any[(e % Wc) * Cq + e / Wc] = x;
     }
   }
   // exclusive scan of 128 * floor(n_a / 128): first row of cluster a's whole tiles
@@ -353,67 +355,81 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
     pa.row_token[r] = -1;
     pa.row_label[r] = -1;
   }
-  if (warp != 0) return;
-
-  // ------------------------------------------------ leftover rows (warp 0)
-  int dst = 0;  // rows placed by the whole-tile pass = sum of 128 k_a
-  for (int c = lane; c < Cq; c += 32) dst += pa.count[c] / 128 * 128;
-  dst = __reduce_add_sync(0xffffffffu, dst);
-  int left = total - dst;
-  int room = 0, cur = -1, next_in_order = 0;
-  while (left > 0) {
-    if (room == 0) {
-      // new tile: the cluster with the most rows left, ties to the lower label
-      int best = -1, bc = 0x7fffffff;
-      for (int c = lane; c < Cq; c += 32)
-        if (rem[c] > best) { best = rem[c]; bc = c; }
-      for (int o = 16; o > 0; o >>= 1) {
-        const int ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
-        if (ob > best || (ob == best && oc < bc)) { best = ob; bc = oc; }
-      }
-      cur = pa.greedy ? bc : -1;
-      room = 128;
-      if (pa.greedy)
-        for (int w = lane; w < Wc; w += 32) uni[w] = 0u;
-      __syncwarp();
-    } else if (pa.greedy) {
-      // the cluster adding the fewest new kept key clusters to this tile
-      int best = 0x7fffffff, bc = 0x7fffffff;
-      for (int c = lane; c < Cq; c += 32) {
-        if (rem[c] == 0) continue;
+  // ------------------------------------------------ leftover rows: one piece per step,
+  // the candidates scored by all threads (one cluster each), the choice taken by a
+  // block-wide minimum of (score, label); the rows are copied once the order is known.
+  __shared__ unsigned long long s_red[32];
+  __shared__ int s_left, s_room, s_dst, s_npieces, s_cur, s_new;
+  if (tid == 0) {
+    s_dst = 0;
+    s_room = 0;
+    s_npieces = 0;
+  }
+  __syncthreads();
+  const int full_part = __reduce_add_sync(0xffffffffu, local);  // rows in whole tiles
+  if (lane == 0) atomicAdd(&s_dst, full_part);
+  __syncthreads();
+  if (tid == 0) s_left = total - s_dst;
+  __syncthreads();
+  while (s_left > 0) {
+    const bool new_tile = s_room == 0;
+    unsigned long long best = ~0ull;
+    for (int c = tid; c < Cq; c += 1024) {
+      const int rc = rem[c];
+      if (rc == 0) continue;
+      unsigned long long key;
+      if (!pa.greedy) {
+        key = static_cast<unsigned long long>(c);                         // label order
+      } else if (new_tile) {
+        key = (static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(rc)) << 32) | c;
+      } else {
         int add = 0;
-        for (int w = 0; w < Wc; ++w) add += __popc(any[c * Wc + w] & ~uni[w]);
-        if (add < best) { best = add; bc = c; }
+        for (int w = 0; w < Wc; ++w) add += __popc(any[w * Cq + c] & ~uni[w]);
+        key = (static_cast<unsigned long long>(add) << 32) | c;
       }
+      best = key < best ? key : best;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+      best = y < best ? y : best;
+    }
+    if (lane == 0) s_red[warp] = best;
+    __syncthreads();
+    if (warp == 0) {
+      best = s_red[lane];
       for (int o = 16; o > 0; o >>= 1) {
-        const int ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
-        if (ob < best || (ob == best && oc < bc)) { best = ob; bc = oc; }
+        const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+        best = y < best ? y : best;
       }
-      cur = bc;
-    } else {
-      cur = -1;
+      if (lane == 0) {
+        const int cur = static_cast<int>(best & 0xffffffffull);
+        const int room = new_tile ? 128 : s_room;
+        const int take = min(room, rem[cur]);
+        const int r_all = pa.count[cur] % 128;
+        const int src = pa.off[cur] + pa.count[cur] - r_all + (r_all - rem[cur]);
+        if (s_npieces < pa.max_pieces) pa.pieces[s_npieces] = make_int4(cur, src, take, s_dst);
+        ++s_npieces;
+        rem[cur] -= take;
+        s_room = room - take;
+        s_dst += take;
+        s_left -= take;
+        s_cur = cur;
+        s_new = new_tile ? 1 : 0;
+      }
     }
-    if (cur < 0) {  // label order
-      while (rem[next_in_order] == 0) ++next_in_order;
-      cur = next_in_order;
-    }
-    const int r_all = pa.count[cur] % 128;
-    const int take = min(room, rem[cur]);
-    const int src = pa.off[cur] + pa.count[cur] - r_all + (r_all - rem[cur]);
-    for (int i = lane; i < take; i += 32) {
-      pa.row_token[dst + i] = pa.sort_token[src + i];
-      pa.row_label[dst + i] = cur;
-    }
+    __syncthreads();
     if (pa.greedy)
-      for (int w = lane; w < Wc; w += 32) uni[w] |= any[cur * Wc + w];
-    __syncwarp();
-    if (lane == 0) rem[cur] -= take;
-    __syncwarp();
-    dst += take;
-    room -= take;
-    left -= take;
+      for (int w = tid; w < Wc; w += 1024) uni[w] = (s_new ? 0u : uni[w]) | any[w * Cq + s_cur];
+    __syncthreads();
+  }
+  // copy the leftover rows piece by piece, one warp per piece
+  const int np = min(s_npieces, pa.max_pieces);
+  for (int pc = warp; pc < np; pc += 32) {
+    const int4 pe = pa.pieces[pc];
+    for (int i = lane; i < pe.z; i += 32) {
+      pa.row_token[pe.w + i] = pa.sort_token[pe.y + i];
+      pa.row_label[pe.w + i] = pe.x;
+    }
   }
 }
 
@@ -521,6 +537,8 @@ __global__ void __launch_bounds__(256) gather_kv_centroids_kernel(
 struct AttnArgs {
   int B, Hq, Hkv, Sq, Sqpad, Skpad, Ck, Ckpad, Cq, G, Wg, Wc;
   int kstride;  // rows per (batch, KV head) in the tensors the K/V maps address
+  int q_gather;   // 1: the Q map addresses the caller's q (B*Hq*Sq rows, one-row boxes) and
+                  // the tile's rows are gathered through qrow_token; 0: a permuted copy
   int ksplit;   // CTAs per query tile, each over a contiguous range of key groups
   float* part;  // ksplit > 1: per split, unnormalised O, running max and sum per row
   int nh_slices, b_sliced, h_sliced;
@@ -547,18 +565,18 @@ struct AttnCfg {
   static constexpr int NATOM = D / ATOM;            // 128-byte column chunks per row
   static constexpr int TILE = 128 * D * ESIZE;      // one 128-row operand tile
   static constexpr int KSTEP = 32 / ESIZE;          // K of one MMA instruction
-  // barriers, bitsets, chunk list, centroid column biases (2 x 128 floats)
-  static constexpr int MISC = 2048 + kChunkListCap * 4 + 512 + 1024;
+  static constexpr int MISC = 2048 + kChunkListCap * 4 + 512;  // barriers, bitsets, chunk list
   static constexpr int SMEM = 3 * TILE + MISC + 1024;
   // At least ~100 KB so that at most two CTAs share an SM (two 256-column TMEM
   // allocations fill the 512 columns).
   static constexpr int SMEM_LAUNCH = SMEM > 100 * 1024 ? SMEM : 100 * 1024;
 };
 
-// Q/K/V full (TMA), K/V empty (the MMA reading the stage has completed), S full (QK of
-// the current chunk done), P full (softmax of the chunk written), O final, drain.
-// CB: the softmax threads have staged a centroid chunk's column biases.
-enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SF, BAR_PF, BAR_OF, BAR_DRAIN, BAR_CB, NBAR };
+// Q/K/V full (TMA), K/V empty (MMA done reading), S-low / S-high full (QK of key
+// columns 0..63 / 64..127 done), P-low / P-high ready (softmax of those columns
+// written), PV-low done, O final, drain.
+enum { BAR_Q = 0, BAR_KF, BAR_KE, BAR_VF, BAR_VE, BAR_SFLO, BAR_SFHI, BAR_PLO, BAR_PHI, BAR_OLO,
+       BAR_OF, BAR_DRAIN, NBAR };
 
 struct Chunk {
   int start;   // first key slot (token chunk) or first centroid (centroid chunk)
@@ -712,9 +730,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 template <int D, bool TF32>
-// 160 threads (control warp + 4 softmax warps); two CTAs share an SM (at most 200
-// registers a thread: 2 x 160 x 200 fits the SM's 65536).
-__global__ void __maxnreg__(200)
+// 160 threads (control warp + 4 softmax warps); two CTAs share an SM.
+__global__ void __launch_bounds__(160, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
                 const __grid_constant__ CUtensorMap tmVc, const AttnArgs a) {
@@ -734,7 +751,6 @@ __global__ void __maxnreg__(200)
   uint32_t* cneed = uni_bits + 128;                                   // 4 words
   int* nchunks = reinterpret_cast<int*>(cneed + 4);
   uint32_t* clist = reinterpret_cast<uint32_t*>(smem + 3 * Cfg::TILE + 2048);  // kChunkListCap
-  float* sbias = reinterpret_cast<float*>(smem + 3 * Cfg::TILE + 2048 + kChunkListCap * 4 + 512);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x / a.ksplit, split = blockIdx.x % a.ksplit;
@@ -748,7 +764,7 @@ __global__ void __maxnreg__(200)
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
 
   if (tid == 0) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(BAR(i), (i == BAR_PF || i == BAR_CB) ? 128u : 1u);
+    for (int i = 0; i < NBAR; ++i) mbar_init(BAR(i), (i == BAR_PLO || i == BAR_PHI) ? 128u : 1u);
     *abort_flag = 0;
     *n_distinct = 0;
     *never = 0;
@@ -815,12 +831,9 @@ __global__ void __maxnreg__(200)
     // ------------------------------------------------ control warp: TMA + tcgen05.mma
     // The whole warp runs this loop on warp-uniform values, so MMA descriptors live in
     // uniform registers and each tcgen05.mma issues without per-lane conversion; lane
-    // 0 alone issues the per-thread operations (TMA copies, expect_tx, commits).
-    // Per chunk j, once the softmax has written P(j): PV(j), then QK(j+1). One thread
-    // issues both, so they run in that order: QK(j+1) overwrites P(j) only after PV(j)
-    // has read it, and the commit after QK(j+1) also covers PV(j). The single K and V
-    // stages are refilled as soon as the MMA that read them completes; the softmax of
-    // the next chunk gives the copies time to land.
+    // 0 alone issues the per-thread operations (TMA copies, expect_tx, commits). The
+    // single K and V stages are refilled as soon as the MMA that read them completes,
+    // while the softmax warps work on the current chunk.
     const bool leader = lane == 0;
     auto wait_all = [&](uint32_t bar, uint32_t parity, int where) -> bool {
       const bool r = mbar_wait(bar, parity, abort_flag, where);
@@ -861,42 +874,70 @@ __global__ void __maxnreg__(200)
     };
     Chunk cur, nxt, nn;
     bool have = next(cur);
-    if (leader) {
-      mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
-#pragma unroll
-      for (int cc = 0; cc < Cfg::NATOM; ++cc)
-        tma_load_2d(sQ + cc * 16384, &tmQ, BAR(BAR_Q), cc * Cfg::ATOM, qrow0);
-    }
-    __syncwarp();
     if (have) {
       load_kv(cur, false);
       ++nk;
       load_kv(cur, true);
       ++nv;
     }
-    // S = Q Kᵀ for the n key columns of chunk c into TMEM columns 0..n-1 (N = n).
-    auto issue_qk = [&](const Chunk& c) {
-      const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(c.n >> 3) << 17);
-      if (elect_one()) {
+    if (a.q_gather) {
+      // the tile's 128 rows straight from the caller's q: lane L gathers rows 4L..4L+3
+      // (their tokens through the row map; pad rows point past the last row and read
+      // zeros), one tile::gather4 per 128-byte column chunk
+      if (leader) mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
+      __syncwarp();
+      const int64_t qbase = (static_cast<int64_t>(b) * a.Hq + h) * a.Sq;
+      const int oob = a.B * a.Hq * a.Sq;
+      int rr[4];
 #pragma unroll
-        for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          mma_ss<TF32>(tmem, dQ + off, dK + off, idesc, kk > 0 ? 1u : 0u);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const int t = a.qrow_token[tile * 128 + 4 * lane + i];
+        rr[i] = t >= 0 ? static_cast<int>(qbase + t) : oob;
+      }
+#pragma unroll
+      for (int cc = 0; cc < Cfg::NATOM; ++cc)
+        tma_gather4_2d(sQ + cc * 16384 + lane * 512, &tmQ, BAR(BAR_Q), cc * Cfg::ATOM, rr[0], rr[1],
+                       rr[2], rr[3]);
+      __syncwarp();
+    } else {
+      if (leader) {
+        mbar_arrive_expect_tx(BAR(BAR_Q), Cfg::TILE);
+#pragma unroll
+        for (int cc = 0; cc < Cfg::NATOM; ++cc)
+          tma_load_2d(sQ + cc * 16384, &tmQ, BAR(BAR_Q), cc * Cfg::ATOM, qrow0);
       }
       __syncwarp();
+    }
+    // S = Q Kᵀ for key columns [64h, 64h + n_h) of chunk c into TMEM columns 64h.. (N = n_h).
+    auto issue_qk_half = [&](const Chunk& c, int hlf) {
+      const int nh = min(64, c.n - 64 * hlf);
+      if (nh > 0) {
+        const uint32_t idesc = kIdescQK | (static_cast<uint32_t>(nh >> 3) << 17);
+        const uint64_t krow = static_cast<uint64_t>((hlf * 64 * 128) >> 4);  // 64 rows of 128 B
+        // one elected lane issues the half's K-steps back to back
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / Cfg::KSTEP; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss<TF32>(tmem + 64 * hlf, dQ + off, dK + off + krow, idesc, kk > 0 ? 1u : 0u);
+          }
+        }
+        __syncwarp();
+      }
     };
-    // O += P V over the n key rows of chunk c; P sits at TMEM columns 0.. (bf16 pairs:
-    // n/2 columns, fp32: n). V is MN-major (d contiguous): 128-byte rows, d chunks 16 KB
-    // apart; bf16 uses 8-row swizzle groups (1 KB), tf32 the 32-byte-unit swizzle with
-    // 4-row groups; a K-step of KSTEP rows moves KSTEP*128 B.
-    auto issue_pv = [&](const Chunk& c, bool first_chunk) {
+    // O += P V for key rows [64h, 64h + n_h); P of step h sits at TMEM columns 64h..
+    // (bf16 pairs: 32 columns, fp32: 64). V is MN-major (d contiguous): 128-byte rows,
+    // d chunks 16 KB apart; bf16 uses 8-row swizzle groups (1 KB), tf32 the
+    // 32-byte-unit swizzle with 4-row groups; a K-step of KSTEP rows moves KSTEP*128 B.
+    auto issue_pv_half = [&](const Chunk& c, int hlf, bool first_chunk) {
+      constexpr int kHalfSteps = 64 / Cfg::KSTEP;
       const int nsteps = c.n / Cfg::KSTEP;
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 128 / Cfg::KSTEP; ++kk) {
+        for (int t = 0; t < kHalfSteps; ++t) {
+          const int kk = hlf * kHalfSteps + t;
           if (kk < nsteps)
-            mma_ts<TF32>(tmem + 128, tmem + kk * 8,
+            mma_ts<TF32>(tmem + 128, tmem + 64 * hlf + t * 8,
                          dV + static_cast<uint64_t>((kk * Cfg::KSTEP * 128) >> 4), kIdescPV,
                          (!first_chunk || kk > 0) ? 1u : 0u);
         }
@@ -905,12 +946,17 @@ __global__ void __maxnreg__(200)
     };
     bool ok = wait_all(BAR(BAR_Q), 0, 3);
     bool have_next = false, have_nn = false;
+    int hi_c = 0;  // chunks with a high step whose P-high the control has waited for
     if (ok && have) {
       ok = wait_all(BAR(BAR_KF), 0, 5);
       if (ok) {
         tc_fence_after();
-        issue_qk(cur);
-        commit(BAR(BAR_SF));
+        issue_qk_half(cur, 0);
+        commit(BAR(BAR_SFLO));
+        if (cur.n > 64) {
+          issue_qk_half(cur, 1);
+          commit(BAR(BAR_SFHI));
+        }
         commit(BAR(BAR_KE));
         have_next = next(nxt);
         if (have_next && (ok = wait_all(BAR(BAR_KE), 0, 1))) {
@@ -919,18 +965,38 @@ __global__ void __maxnreg__(200)
         }
       }
     }
+    // Steady state for chunk j: PV-low(j) | QK-low(j+1) | PV-high(j) | QK-high(j+1), so
+    // the tensor core works on the next chunk's low keys while the softmax warps are on
+    // chunk j's high keys, and on the next chunk's high keys while they start chunk j+1.
     while (ok && have) {
-      if (!(ok = wait_all(BAR(BAR_PF), j & 1, 6))) break;
+      if (!(ok = wait_all(BAR(BAR_PLO), j & 1, 6))) break;
       if (!(ok = wait_all(BAR(BAR_VF), j & 1, 7))) break;
       tc_fence_after();
-      issue_pv(cur, j == 0);
+      issue_pv_half(cur, 0, j == 0);
+      commit(BAR(BAR_OLO));
+      if (have_next) {
+        // MMAs of one thread run in issue order: QK-low(j+1) overwrites P-low(j) only
+        // after PV-low(j) has read it.
+        if (!(ok = wait_all(BAR(BAR_KF), (j + 1) & 1, 5))) break;
+        tc_fence_after();
+        issue_qk_half(nxt, 0);
+        commit(BAR(BAR_SFLO));
+      }
+      // The high step exists only for chunks of more than 64 keys; its barriers count
+      // those chunks alone (hi_c / hi_n), on both sides.
+      if (cur.n > 64) {
+        if (!(ok = wait_all(BAR(BAR_PHI), hi_c & 1, 8))) break;
+        ++hi_c;
+        tc_fence_after();
+        issue_pv_half(cur, 1, j == 0);
+      }
       commit(BAR(BAR_VE));
       have_nn = false;
       if (have_next) {
-        if (!(ok = wait_all(BAR(BAR_KF), (j + 1) & 1, 5))) break;
-        tc_fence_after();
-        issue_qk(nxt);
-        commit(BAR(BAR_SF));
+        if (nxt.n > 64) {
+          issue_qk_half(nxt, 1);
+          commit(BAR(BAR_SFHI));
+        }
         commit(BAR(BAR_KE));
         // V stage: refill with the next chunk once PV(j) has read it
         if (!(ok = wait_all(BAR(BAR_VE), j & 1, 4))) break;
@@ -960,8 +1026,8 @@ __global__ void __maxnreg__(200)
   } else {
     // ------------------------------------------------ softmax / epilogue (128 threads)
     // One thread per query row (warps 1..4; warp w reads TMEM lanes 32*(w%4)..+31).
-    // Each chunk is one online-softmax step over its up to 128 key columns: S is read
-    // from TMEM, P is written back over it, and the control warp then issues PV.
+    // Each chunk is taken as two online-softmax steps over key columns 0..63 and
+    // 64..127; after the first the PV of those keys starts while the second runs.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int qrow = tile * 128 + r;
@@ -973,20 +1039,20 @@ __global__ void __maxnreg__(200)
     const uint32_t tO = tS + 128;
     const float scl = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    int j = 0, ncent = 0;
+    int j = 0, hi_n = 0;  // hi_n: high steps taken so far
     bool ok = true;
 #pragma unroll 1
     for (int ci = 0; ci < nch; ++ci) {
       const Chunk ch = decode_chunk(clist[ci]);
+      const int nsteps = ch.n > 64 ? 2 : 1;
       // Token chunks are masked per 16-key group (a key cluster is kept or dropped
       // whole): this row's keep bits for the chunk's groups, the groups holding pad
       // slots, and the warp's votes (whether no row, every row or some rows keep each
-      // group). None of it depends on S, so it is read before S is ready. Groups past
-      // the chunk's end count as kept by no row.
-      uint32_t kb = 0u, part = 0u, anyg = 0xffu, mixed = 0u;
+      // group). None of it depends on S, so it is read before S is ready.
+      uint32_t kb8 = 0u, part8 = 0u, any8 = 0xffu, mixed8 = 0u;
       if (!ch.centroid) {
         const uint32_t present = (1u << ch.ng) - 1u;
-        kb = present;
+        kb8 = present;
         if (!ch.uniform) {
           const int w = ch.g0 >> 5, sh = ch.g0 & 31;
           const bool two = w + 1 < a.Wg;
@@ -994,139 +1060,191 @@ __global__ void __maxnreg__(200)
                               (two ? static_cast<uint64_t>(__ldg(grow + w + 1)) << 32 : 0ull);
           const uint64_t fw = static_cast<uint64_t>(__ldg(a.gfull + w)) |
                               (two ? static_cast<uint64_t>(__ldg(a.gfull + w + 1)) << 32 : 0ull);
-          kb = static_cast<uint32_t>(kw >> sh) & present;
-          part = ~static_cast<uint32_t>(fw >> sh) & present;
+          kb8 = static_cast<uint32_t>(kw >> sh) & present;
+          part8 = ~static_cast<uint32_t>(fw >> sh) & present;
         }
-        if (lab < 0) kb = 0u;
-        anyg = __reduce_or_sync(0xffffffffu, kb);
-        mixed = anyg & ~__reduce_and_sync(0xffffffffu, kb);
+        if (lab < 0) kb8 = 0u;
+        any8 = __reduce_or_sync(0xffffffffu, kb8);
+        mixed8 = any8 & ~__reduce_and_sync(0xffffffffu, kb8);
       }
-      uint32_t mk[4] = {0u, 0u, 0u, 0u};  // centroid chunk: bit c of word w = column 32w+c kept
-      const float* cbias = sbias + 128 * (ncent & 1);
-      if (ch.centroid) {
-        if (lab >= 0) {
-          const int w0 = ch.start >> 5;
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            mk[w] = w0 + w < a.Wc ? (~__ldg(crow + w0 + w) & __ldg(a.cnonempty + w0 + w)) : 0u;
-        }
-        // the chunk's column biases log2 n_c, one per softmax thread, shared through
-        // shared memory (two buffers by centroid-chunk parity: no thread can be a whole
-        // chunk ahead of another, every chunk ends on P full)
-        sbias[128 * (ncent & 1) + r] = __ldg(a.bias2 + ch.start + r);
-        mbar_arrive(BAR(BAR_CB));
-        if (!(ok = mbar_wait(BAR(BAR_CB), ncent & 1, abort_flag, 13))) break;
-        ++ncent;
-      }
-      if (!(ok = mbar_wait(BAR(BAR_SF), j & 1, abort_flag, 9))) break;
-      tc_fence_after();
-      float v[128];
-      const int nblk = ch.n > 96 ? 4 : (ch.n > 64 ? 3 : (ch.n > 32 ? 2 : 1));
-      tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(v));
-      tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-      tmem_ld32(tS + 64, *reinterpret_cast<float(*)[32]>(v + 64));
-      tmem_ld32(tS + 96, *reinterpret_cast<float(*)[32]>(v + 96));
-      float mx;
-      float sx = scl;  // exponent argument x = v * sx - m
-      tmem_wait_ld();
-      // blocks not loaded (past the chunk's end) take no part
-#pragma unroll
-      for (int c = 32; c < 128; ++c) v[c] = (c >> 5) < nblk ? v[c] : -INFINITY;
-      if (!ch.centroid) {
-        // -inf for key columns past the chunk's end (in its last 32-column block), for
-        // the pad slots of a cluster's last group, for rows that drop a group another
-        // row of the warp keeps, and for groups no row of the warp keeps
-        const uint32_t drop = ~anyg & ((1u << (2 * nblk)) - 1u);
-        if (part | mixed | drop) {
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            if ((part >> g) & 1u) {
-              const int nvalid = __ldg(a.group_valid + ch.g0 + g);
-#pragma unroll
-              for (int c = 1; c < 16; ++c) v[16 * g + c] = c < nvalid ? v[16 * g + c] : -INFINITY;
-            }
-            if (((mixed | drop) >> g) & 1u) {
-              const bool keep = ((kb & ~drop) >> g) & 1u;
-#pragma unroll
-              for (int c = 0; c < 16; ++c) v[16 * g + c] = keep ? v[16 * g + c] : -INFINITY;
-            }
-          }
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          v[c] = fmaf(v[c], scl, ((mk[c >> 5] >> (c & 31)) & 1u) ? cbias[c] : -INFINITY);
-        sx = 1.f;  // log2-unit logits or -inf
-      }
-      // max over the loaded blocks (raw logits for token chunks: scale > 0, so the max
-      // of scale*s is scale*max(s))
-      mx = fmaxf(max64(*reinterpret_cast<float(*)[32]>(v), *reinterpret_cast<float(*)[32]>(v + 32)),
-                 max64(*reinterpret_cast<float(*)[32]>(v + 64), *reinterpret_cast<float(*)[32]>(v + 96)));
-      if (!ch.centroid) mx *= scl;
-      // Lazy rescaling: the running max only moves when the step max exceeds it by
-      // more than 8 (log2 units), so P stays below 256 and O is rarely touched.
-      const bool need = mx > m_run + 8.f;
-      const bool any_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2(m_run - mx);
-        l_run *= alpha;
-        m_run = mx;
-      }
-      const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
-      // Two independent pair sums keep the add chain short. Straight-line code over all
-      // 128 columns (masked columns give exact zeros).
-      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-#pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        {
-#pragma unroll
-          for (int p = 0; p < 16; ++p) {
-            const int c = 32 * blk + 2 * p;
-            float x0, x1;
-            fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
-            if ((p & 7) < kPolyPairsOf8) {
-              exp2_poly2<true>(v[c], v[c + 1], x0, x1);
-            } else {
-              v[c] = ex2(x0);
-              v[c + 1] = ex2(x1);
-            }
-            if (p & 1) add2(sb0, sb1, sb0, sb1, v[c], v[c + 1]);
-            else add2(sa0, sa1, sa0, sa1, v[c], v[c + 1]);
-          }
-        }
-      }
-      l_run += (sa0 + sa1) + (sb0 + sb1);
-      // P over S in place: bf16 pairs in columns [0, 64), fp32 in [0, 128).
-      if constexpr (TF32) {
-        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(v));
-        if (nblk > 1) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        if (nblk > 2) tmem_st32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
-        if (nblk > 3) tmem_st32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
-      } else {
-        uint32_t* w = reinterpret_cast<uint32_t*>(v);
-#pragma unroll
-        for (int i = 0; i < 64; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(w));
-        if (nblk > 2) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(w + 32));
-      }
-      // O follows the running max before this chunk's PV adds to it (after P
-      // is stored, so that its registers are free). S(j) full means
-      // QK(j) has completed, and with it PV(j-1), which was issued before it.
-      if (any_need && j > 0) {
 #pragma unroll 1
-        for (int p = 0; p < D / 32; ++p) {
-          float o[32];
-          tmem_ld32(tO + p * 32, o);
-          tmem_wait_ld();
+      for (int half = 0; half < nsteps; ++half) {
+        const int c0 = half * 64;         // first key column of this step
+        {
+          if (!(ok = mbar_wait(BAR(half == 0 ? BAR_SFLO : BAR_SFHI), half == 0 ? (j & 1) : (hi_n & 1),
+                               abort_flag, 9)))
+            break;
+          tc_fence_after();
+          // Groups no row of the warp keeps get P = 0 without exponentials, groups every
+          // row keeps need no select. Columns past a cluster's last token (pad slots of
+          // its last group) and pad query rows are set to -inf. Centroid chunks are
+          // masked per column and carry the log2 n_c bias.
+          float v0[32], v1[32];
+          tmem_ld32(tS + c0, v0);
+          tmem_ld32(tS + c0 + 32, v1);
+          uint32_t any4 = 0xfu;  // groups of this step whose exponentials the warp computes
+          float mx;
+          float sx = scl;        // exponent argument x = v * sx - m
+          if (!ch.centroid) {
+            const int gh0 = ch.g0 + half * 4;  // this step covers groups gh0 .. gh0+3
+            const uint32_t kb = (kb8 >> (4 * half)) & 0xfu;
+            const uint32_t partial = (part8 >> (4 * half)) & 0xfu;
+            const uint32_t mixed = (mixed8 >> (4 * half)) & 0xfu;
+            any4 = (any8 >> (4 * half)) & 0xfu;
+            tmem_wait_ld();
+            if (partial | mixed) {
+              // -inf for the pad slots of a cluster's last group, and for rows that drop
+              // a group another row of the warp keeps
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] *= alpha;
-          tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+              for (int jj = 0; jj < 4; ++jj) {
+                float* v = jj < 2 ? v0 : v1;
+                const int o = (jj & 1) * 16;
+                if ((partial >> jj) & 1u) {
+                  const int nv = __ldg(a.group_valid + gh0 + jj);
+#pragma unroll
+                  for (int c = 1; c < 16; ++c) v[o + c] = c < nv ? v[o + c] : -INFINITY;
+                }
+                if ((mixed >> jj) & 1u) {
+                  const bool keep = (kb >> jj) & 1u;
+#pragma unroll
+                  for (int c = 0; c < 16; ++c) v[o + c] = keep ? v[o + c] : -INFINITY;
+                }
+              }
+            }
+            // raw logits; scale > 0, so the max of scale*s is scale*max(s)
+            if (any4 == 0xfu) {
+              mx = max64(v0, v1) * scl;
+            } else {
+              mx = -INFINITY;
+#pragma unroll
+              for (int jj = 0; jj < 4; ++jj)
+                if ((any4 >> jj) & 1u) mx = fmaxf(mx, max16((jj < 2 ? v0 : v1) + (jj & 1) * 16));
+              mx *= scl;
+            }
+          } else {
+            uint32_t mk0 = 0u, mk1 = 0u;  // bit c: column c0 + c (+ 32) kept
+            if (lab >= 0) {
+              const int ww = (ch.start + c0) >> 5;
+              mk0 = ww < a.Wc ? (~__ldg(crow + ww) & __ldg(a.cnonempty + ww)) : 0u;
+              mk1 = ww + 1 < a.Wc ? (~__ldg(crow + ww + 1) & __ldg(a.cnonempty + ww + 1)) : 0u;
+            }
+            const float* bias = a.bias2 + ch.start + c0;
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              v0[c] = ((mk0 >> c) & 1u) ? fmaf(v0[c], scl, __ldg(bias + c)) : -INFINITY;
+              v1[c] = ((mk1 >> c) & 1u) ? fmaf(v1[c], scl, __ldg(bias + 32 + c)) : -INFINITY;
+            }
+            mx = max64(v0, v1);
+            sx = 1.f;  // log2-unit logits or -inf
+          }
+          // Lazy rescaling: the running max only moves when the step max exceeds it by
+          // more than 8 (log2 units), so P stays below 256 and O is rarely touched.
+          const bool need = mx > m_run + 8.f;
+          const bool any_need = __any_sync(0xffffffffu, need);
+          float alpha = 1.f;
+          if (need) {
+            alpha = ex2(m_run - mx);
+            l_run *= alpha;
+            m_run = mx;
+          }
+          const float neg_mu = (m_run == -INFINITY) ? 0.f : -m_run;
+          // Two independent pair sums keep the add chain short. Groups no row of the
+          // warp keeps are zero; the common all-groups case runs as straight-line code.
+          float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+          if (any4 == 0xfu) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              float* v = q < 16 ? v0 : v1;
+              const int c = (q & 15) * 2;
+              float x0, x1;
+              fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
+              if ((q & 7) < kPolyPairsOf8) {
+                exp2_poly2<true>(v[c], v[c + 1], x0, x1);
+              } else {
+                v[c] = ex2(x0);
+                v[c + 1] = ex2(x1);
+              }
+              if (q & 1) add2(sb0, sb1, sb0, sb1, v[c], v[c + 1]);
+              else add2(sa0, sa1, sa0, sa1, v[c], v[c + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              float* v = jj < 2 ? v0 : v1;
+              const int o = (jj & 1) * 16;
+              if ((any4 >> jj) & 1u) {
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                  const int c = o + 2 * p;
+                  float x0, x1;
+                  fma2(x0, x1, v[c], v[c + 1], sx, sx, neg_mu, neg_mu);
+                  v[c] = ex2(x0);
+                  v[c + 1] = ex2(x1);
+                  if (p & 1) add2(sb0, sb1, sb0, sb1, v[c], v[c + 1]);
+                  else add2(sa0, sa1, sa0, sa1, v[c], v[c + 1]);
+                }
+              } else {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) v[o + c] = 0.f;
+              }
+            }
+          }
+          l_run += (sa0 + sa1) + (sb0 + sb1);
+          // P over S in place: bf16 pairs of step h in columns [64h, 64h+32) (step 0's
+          // S columns were read above; step 1 lands on its own S columns), fp32 in the
+          // step's own 64 columns.
+          if constexpr (TF32) {
+            tmem_st32(tS + c0, *reinterpret_cast<uint32_t(*)[32]>(v0));
+            tmem_st32(tS + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v1));
+          } else {
+            uint32_t* w0 = reinterpret_cast<uint32_t*>(v0);
+            uint32_t* w1 = reinterpret_cast<uint32_t*>(v1);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              w0[i] = pack_bf16x2(v0[2 * i], v0[2 * i + 1]);
+              w1[i] = pack_bf16x2(v1[2 * i], v1[2 * i + 1]);
+            }
+            tmem_st16(tS + c0, w0);
+            tmem_st16(tS + c0 + 16, w1);
+          }
+          // O follows the running max before this step's PV adds to it. Step 0: wait
+          // for the last PV of the previous chunk; step 1: for the PV of step 0.
+          if (any_need && j > 0) {
+            if (!(ok = mbar_wait(BAR(half == 0 ? BAR_VE : BAR_OLO), half == 0 ? ((j - 1) & 1) : (j & 1),
+                                 abort_flag, 12)))
+              break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int p = 0; p < D / 32; ++p) {
+              float o[32];
+              tmem_ld32(tO + p * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] *= alpha;
+              tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+            }
+          } else if (any_need && half == 1 && j == 0) {
+            // first chunk: the PV of step 0 wrote O without accumulation; rescale it too
+            if (!(ok = mbar_wait(BAR(BAR_OLO), 0, abort_flag, 12))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int p = 0; p < D / 32; ++p) {
+              float o[32];
+              tmem_ld32(tO + p * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] *= alpha;
+              tmem_st32(tO + p * 32, *reinterpret_cast<uint32_t(*)[32]>(o));
+            }
+          }
+          tmem_wait_st();
         }
+        tc_fence_before();
+        mbar_arrive(BAR(half == 0 ? BAR_PLO : BAR_PHI));
+        hi_n += half;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR(BAR_PF));
+      if (!ok) break;
       ++j;
     }
     const bool o_final = ok && mbar_wait(BAR(BAR_OF), 0, abort_flag, 10);
@@ -1224,6 +1342,9 @@ struct AttnLayout {
   int ksplit;   // CTAs per query tile over disjoint key ranges (1 = no split)
   float* part;  // ksplit > 1: partial O (B,Hq,ksplit,Sqpad,D), then max and sum (...,2)
   int32_t *qrow_token, *qrow_label, *qsort_token, *qsort_label, *q_count, *q_off;
+  int4* pieces;     // query tile plan: leftover pieces
+  int max_pieces;
+  int q_gather;     // the kernel gathers Q rows itself (no permuted copy)
   int32_t *kslot_token, *group_cluster, *group_valid, *k_count, *k_off;
   float* bias2;
   uint32_t *cnonempty, *cbits, *gbits, *gfull;
@@ -1245,6 +1366,8 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
   L.qrow_label = cv.take<int32_t>(L.Sqpad);
   L.qsort_token = cv.take<int32_t>(L.Sqpad);
   L.qsort_label = cv.take<int32_t>(L.Sqpad);
+  L.max_pieces = Cq + L.Sqpad / 128 + 1;
+  L.pieces = cv.take<int4>(L.max_pieces);
   L.q_count = cv.take<int32_t>(Cq);
   L.q_off = cv.take<int32_t>(Cq + 1);
   L.kslot_token = cv.take<int32_t>(L.Skpad);
@@ -1258,7 +1381,11 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
   L.cbits = cv.take<uint32_t>(slices * Cq * L.Wc);
   L.gbits = cv.take<uint32_t>(slices * Cq * L.Wg);
   L.gfull = cv.take<uint32_t>(L.Wg);
-  L.qp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hq * L.Sqpad * s.D * es);
+  // Q rows are gathered straight from the caller's q by the attention kernel whenever
+  // every row index fits a TMA coordinate; otherwise a cluster-major copy is made.
+  L.q_gather = static_cast<int64_t>(s.B) * s.Hq * s.Sq < (int64_t(1) << 31) - 1;
+  L.qp = L.q_gather ? nullptr
+                    : cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hq * L.Sqpad * s.D * es);
   L.kp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Skpad * s.D * es);
   L.vp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Skpad * s.D * es);
   L.kc = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * L.Ckpad * s.D * es);
@@ -1392,6 +1519,8 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     pa.greedy = static_cast<int64_t>(Cq) * L.Wc <= kPlanGreedyWords ? 1 : 0;
     pa.row_token = L.qrow_token;
     pa.row_label = L.qrow_label;
+    pa.pieces = L.pieces;
+    pa.max_pieces = L.max_pieces;
     const int smem = (2 * Cq + L.Wc + (pa.greedy ? Cq * L.Wc : 0)) * 4;
     cudaError_t e = cudaFuncSetAttribute(plan_query_tiles_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1401,9 +1530,9 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     count_launch();
     if ((rc = check_cuda(cudaGetLastError(), "plan_query_tiles_kernel"))) return rc;
   }
-  // 3. Q gather
+  // 3. Q gather (only when the kernel cannot gather the rows itself)
   const int vpr = s.D * es / 16;
-  {
+  if (!L.q_gather) {
     const int64_t n = static_cast<int64_t>(L.Sqpad) * vpr;
     gather_rows_kernel<<<dim3(static_cast<unsigned>((n + 255) / 256), s.Hq, s.B), 256, 0, st>>>(
         static_cast<const uint4*>(q), static_cast<uint4*>(L.qp), L.qrow_token, s.Sq, L.Sqpad, vpr,
@@ -1442,7 +1571,10 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
   const CUtensorMapSwizzle vsw =
       s.dtype == BSA_F32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUtensorMap maps[5];
-  if ((rc = make_tmap_2d(&maps[0], L.qp, tdt, es, static_cast<uint64_t>(s.B) * s.Hq * L.Sqpad, s.D, 128, atom)) ||
+  if ((rc = L.q_gather
+                ? make_tmap_2d(&maps[0], q, tdt, es, static_cast<uint64_t>(s.B) * s.Hq * s.Sq, s.D, 1, atom)
+                : make_tmap_2d(&maps[0], L.qp, tdt, es, static_cast<uint64_t>(s.B) * s.Hq * L.Sqpad, s.D, 128,
+                               atom)) ||
       (rc = make_tmap_2d(&maps[1], kv_identity ? k : L.kp, tdt, es,
                          static_cast<uint64_t>(s.B) * s.Hkv * (kv_identity ? s.Sk : L.Skpad), s.D, 128, atom)) ||
       (rc = make_tmap_2d(&maps[2], kv_identity ? v : L.vp, tdt, es,
@@ -1458,6 +1590,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
   args.Sqpad = L.Sqpad;
   args.Skpad = L.Skpad;
   args.kstride = kv_identity ? s.Sk : L.Skpad;
+  args.q_gather = L.q_gather;
   args.Ck = Ck;
   args.Ckpad = L.Ckpad;
   args.Cq = Cq;

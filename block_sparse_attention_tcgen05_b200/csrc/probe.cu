@@ -377,15 +377,29 @@ extern "C" int bsa_select_probe_rows(const int32_t* labels, int S, int C, int M,
   return check_cuda(cudaGetLastError(), "round_robin_kernel");
 }
 
+namespace bsa {
+// The gathered probe rows, (B, Hq, M, D), are the same memory as (B, Hkv, G M, D) with
+// G = Hq / Hkv: the probe rows of the G query heads that share a KV head run as one
+// attention problem of G M rows per KV head (fewer, fuller 128-row tiles than one
+// problem of M rows per query head), and o_probe comes out in the same layout.
+inline bsa_shape probe_attention_shape(const bsa_shape& shape, int M) {
+  bsa_shape ps = shape;
+  const int G = shape.Hkv > 0 ? shape.Hq / shape.Hkv : 1;
+  ps.Hq = shape.Hkv;
+  ps.Sq = G * M;
+  return ps;
+}
+}  // namespace bsa
+
 extern "C" size_t bsa_probe_attention_workspace_bytes(bsa_shape shape, int M) {
   using namespace bsa;
   if (M <= 0 || M > kMaxProbes) return 0;
+  if (shape.Hkv <= 0 || shape.Hq <= 0 || shape.Hq % shape.Hkv) return 0;
   const int es = shape.dtype == BSA_F32 ? 4 : 2;
-  bsa_shape ps = shape;
-  ps.Sq = M;
+  const bsa_shape ps = probe_attention_shape(shape, M);
   Carver cv(nullptr);
   cv.take<uint8_t>(static_cast<size_t>(shape.B) * shape.Hq * M * shape.D * es);
-  cv.take<int32_t>(static_cast<size_t>(M > shape.Sk ? M : shape.Sk));
+  cv.take<int32_t>(static_cast<size_t>(ps.Sq > shape.Sk ? ps.Sq : shape.Sk));
   cv.take<uint8_t>(16);
   const size_t att = attention_workspace_bytes(ps, 1, 1);
   return align_up(cv.used, 256) + att;
@@ -399,6 +413,8 @@ extern "C" int bsa_probe_dense_attention(const void* q, const void* k, const voi
   cudaStream_t st = as_stream(stream);
   if (!q || !k || !v || !probe_idx || !o_probe) return fail(BSA_ERR_INVALID_ARG, "null pointer");
   if (M <= 0 || M > kMaxProbes) return fail(BSA_ERR_UNSUPPORTED, "M must be in [1, %d]", kMaxProbes);
+  if (shape.Hkv <= 0 || shape.Hq <= 0 || shape.Hq % shape.Hkv)
+    return fail(BSA_ERR_INVALID_ARG, "Hq (%d) not a positive multiple of Hkv (%d)", shape.Hq, shape.Hkv);
   const size_t need = bsa_probe_attention_workspace_bytes(shape, M);
   if (!need) return fail(BSA_ERR_INVALID_ARG, "bad shape");
   if (!workspace || workspace_bytes < need)
@@ -406,7 +422,8 @@ extern "C" int bsa_probe_dense_attention(const void* q, const void* k, const voi
   const int es = shape.dtype == BSA_F32 ? 4 : 2;
   Carver cv(workspace);
   void* qp = cv.take<uint8_t>(static_cast<size_t>(shape.B) * shape.Hq * M * shape.D * es);
-  const int nz = M > shape.Sk ? M : shape.Sk;
+  const bsa_shape ps = probe_attention_shape(shape, M);
+  const int nz = ps.Sq > shape.Sk ? ps.Sq : shape.Sk;
   int32_t* zeros = cv.take<int32_t>(nz);
   uint8_t* one = cv.take<uint8_t>(16);
   const size_t used = align_up(cv.used, 256);
@@ -420,8 +437,6 @@ extern "C" int bsa_probe_dense_attention(const void* q, const void* k, const voi
                                    per_head, shape.Sq, M, vpr, shape.Hq);
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "gather_probe_rows_kernel"))) return rc;
-  bsa_shape ps = shape;
-  ps.Sq = M;
   // Every probe row keeps every key: one query cluster, one key cluster, one kept block.
   return centroid_compensated_attention(qp, k, v, ps, zeros, 1, zeros, 1, one, 0, 0, scale, 0,
                                         o_probe, static_cast<char*>(workspace) + used,

@@ -79,18 +79,25 @@ struct RouteArgs {
 
 // grid (ceil(Cq / 16), Hq, B). Thread t serves probe p = t / 16 and dims
 // [8 (t % 16), 8 (t % 16) + 8) of its running difference vector; for D = 64 only the
-// first 8 lanes of each probe hold dims. Keys of one cluster are streamed 32 at a time
-// through shared memory; a running reference m (the largest logit seen, centroid
-// logits included) keeps every exponential <= 1. At the end of cluster c the norm of
-// the difference vector and the reference it was taken with are stored; once every
-// cluster is done they are brought to the final reference and divided by Z.
+// first 8 lanes of each probe hold dims. kp / vp hold the keys and values of each
+// (batch, KV head) in cluster-major order (cluster c at rows off[c] .. off[c] + n_c),
+// read 32 rows at a time with 16-byte loads; the next chunk's loads are issued into
+// registers before the current chunk is computed. A running reference m (the largest
+// logit seen, centroid logits included) keeps every exponential <= 1. At the end of
+// cluster c the norm of the difference vector and the reference it was taken with are
+// stored; once every cluster is done they are brought to the final reference and
+// divided by Z.
 template <typename T, int D>
-__global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __restrict__ k,
-                                                                     const T* __restrict__ v,
+__global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __restrict__ kp,
+                                                                     const T* __restrict__ vp,
                                                                      const RouteArgs a) {
+  constexpr int EPV = 16 / sizeof(T);                       // elements per 16-byte vector
+  constexpr int VPR = D / EPV;                              // vectors per row
+  constexpr int VPT = kRouteKeys * VPR / kRouteThreads;     // vectors per thread per chunk
+  static_assert(VPT >= 1 && kRouteKeys * VPR % kRouteThreads == 0, "chunk split");
   __shared__ float sq[kRouteProbes][D];
   __shared__ float sk[kRouteKeys][D + 1];
-  __shared__ float sv[kRouteKeys][D];
+  __shared__ __align__(16) float sv[kRouteKeys][D];
   __shared__ float sw[kRouteProbes][kRouteKeys];
   const int tid = threadIdx.x, p = tid >> 4, sub = tid & 15;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -113,97 +120,146 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
   const float* vb = a.vbar + bk * a.Ck * D;
   float* err = a.err + (bq * a.Cq + (pa < a.Cq ? pa : 0)) * a.Ck;
   float* mref = a.mref + (bq * a.Cq + (pa < a.Cq ? pa : 0)) * a.Ck;
+  const uint4* k4 = reinterpret_cast<const uint4*>(kp) + bk * a.S * VPR;
+  const uint4* v4 = reinterpret_cast<const uint4*>(vp) + bk * a.S * VPR;
+  // chunk cursor: cluster c, first key j0 of the chunk inside it
+  int c = 0, j0 = 0;
+  while (c < a.Ck && a.k_count[c] == 0) ++c;
+  uint4 rk[VPT], rv[VPT];
+  auto fetch = [&](int cc, int jj) {
+    const int n = a.k_count[cc], o = a.k_off[cc];
+    const int nk = min(kRouteKeys, n - jj);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int e = tid + i * kRouteThreads, j = e / VPR, part = e % VPR;
+      if (j < nk) {
+        rk[i] = __ldg(k4 + static_cast<int64_t>(o + jj + j) * VPR + part);
+        rv[i] = __ldg(v4 + static_cast<int64_t>(o + jj + j) * VPR + part);
+      } else {
+        rk[i] = make_uint4(0, 0, 0, 0);
+        rv[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  if (c < a.Ck) fetch(c, 0);
   __syncthreads();
-  for (int c = 0; c < a.Ck; ++c) {
-    const int n = a.k_count[c], o = a.k_off[c];
+  // clusters before the first non-empty one, and empty ones later, store 0
+  for (int cc = 0; cc < c; ++cc)
+    if (sub == 0 && pa < a.Cq) { err[cc] = 0.f; mref[cc] = 0.f; }
+  float lc = 0.f;
+  while (c < a.Ck) {
+    const int n = a.k_count[c];
+    const int nk = min(kRouteKeys, n - j0);
+    if (j0 == 0) {
 #pragma unroll
-    for (int i = 0; i < DPT; ++i) diff[i] = 0.f;
-    // centroid logit of this probe (16 lanes of the probe reduce their dims)
-    float lc = 0.f;
-    if (has_dims)
-#pragma unroll
-      for (int i = 0; i < DPT; ++i) lc = fmaf(sq[p][d0 + i], kb[c * D + d0 + i], lc);
-#pragma unroll
-    for (int s = 8; s > 0; s >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, s);
-    lc *= a.scale;
-    if (n > 0 && lc > m) {
-      const float f = __expf(m - lc);
-      z *= f;
-      m = lc;
-    }
-    for (int j0 = 0; j0 < n; j0 += kRouteKeys) {
-      const int nk = min(kRouteKeys, n - j0);
-      __syncthreads();
-      for (int e = tid; e < kRouteKeys * D; e += kRouteThreads) {
-        const int j = e / D, d = e % D;
-        float kx = 0.f, vx = 0.f;
-        if (j < nk) {
-          const int tok = a.k_sort_token[o + j0 + j];
-          kx = route_f(k[(bk * a.S + tok) * D + d]);
-          vx = route_f(v[(bk * a.S + tok) * D + d]);
-        }
-        sk[j][d] = kx;
-        sv[j][d] = vx;
-      }
-      __syncthreads();
-      // logits of keys sub and sub + 16 for this probe
-      float l0 = 0.f, l1 = 0.f;
-#pragma unroll 8
-      for (int d = 0; d < D; ++d) {
-        const float x = sq[p][d];
-        l0 = fmaf(x, sk[sub][d], l0);
-        l1 = fmaf(x, sk[sub + 16][d], l1);
-      }
-      l0 = sub < nk ? l0 * a.scale : -INFINITY;
-      l1 = sub + 16 < nk ? l1 * a.scale : -INFINITY;
-      float mx = fmaxf(l0, l1);
-#pragma unroll
-      for (int s = 8; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
-      if (mx > m) {
-        const float f = __expf(m - mx);
-        z *= f;
-#pragma unroll
-        for (int i = 0; i < DPT; ++i) diff[i] *= f;
-        m = mx;
-      }
-      const float w0 = __expf(l0 - m), w1 = __expf(l1 - m);
-      float ws = w0 + w1;
-#pragma unroll
-      for (int s = 8; s > 0; s >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, s);
-      z += ws;
-      sw[p][sub] = w0;
-      sw[p][sub + 16] = w1;
-      __syncwarp();
+      for (int i = 0; i < DPT; ++i) diff[i] = 0.f;
+      // centroid logit of this probe (16 lanes of the probe reduce their dims)
+      lc = 0.f;
       if (has_dims)
-        for (int j = 0; j < nk; ++j) {
-          const float w = sw[p][j];
 #pragma unroll
-          for (int i = 0; i < DPT; ++i) diff[i] = fmaf(w, sv[j][d0 + i], diff[i]);
-        }
+        for (int i = 0; i < DPT; ++i) lc = fmaf(sq[p][d0 + i], kb[c * D + d0 + i], lc);
+#pragma unroll
+      for (int s = 8; s > 0; s >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, s);
+      lc *= a.scale;
+      if (lc > m) {
+        z *= __expf(m - lc);
+#pragma unroll
+        for (int i = 0; i < DPT; ++i) diff[i] = 0.f;
+        m = lc;
+      }
     }
-    // minus the centroid term, then the norm (taken with reference m)
-    float e2 = 0.f;
-    if (n > 0) {
+    // the fetched chunk into shared memory (fp32)
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int e = tid + i * kRouteThreads, j = e / VPR, part = e % VPR;
+      float fk[EPV], fv[EPV];
+      unpack16<T>(rk[i], fk);
+      unpack16<T>(rv[i], fv);
+#pragma unroll
+      for (int u = 0; u < EPV; ++u) {
+        sk[j][part * EPV + u] = fk[u];
+        sv[j][part * EPV + u] = fv[u];
+      }
+    }
+    __syncthreads();
+    // next chunk's loads in flight while this one is computed
+    const int c_now = c, j_now = j0;
+    j0 += kRouteKeys;
+    if (j0 >= n) {
+      j0 = 0;
+      ++c;
+      while (c < a.Ck && a.k_count[c] == 0) {
+        if (sub == 0 && pa < a.Cq) { err[c] = 0.f; mref[c] = m; }
+        ++c;
+      }
+    }
+    if (c < a.Ck) fetch(c, j0);
+    // logits of keys sub and sub + 16 for this probe
+    float l0 = 0.f, l1 = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < D; ++d) {
+      const float x = sq[p][d];
+      l0 = fmaf(x, sk[sub][d], l0);
+      l1 = fmaf(x, sk[sub + 16][d], l1);
+    }
+    l0 = sub < nk ? l0 * a.scale : -INFINITY;
+    l1 = sub + 16 < nk ? l1 * a.scale : -INFINITY;
+    float mx = fmaxf(l0, l1);
+#pragma unroll
+    for (int s = 8; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+    if (mx > m) {
+      const float f = __expf(m - mx);
+      z *= f;
+#pragma unroll
+      for (int i = 0; i < DPT; ++i) diff[i] *= f;
+      m = mx;
+    }
+    const float w0 = __expf(l0 - m), w1 = __expf(l1 - m);
+    float ws = w0 + w1;
+#pragma unroll
+    for (int s = 8; s > 0; s >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, s);
+    z += ws;
+    sw[p][sub] = w0;
+    sw[p][sub + 16] = w1;
+    __syncwarp();
+    if (has_dims)
+      for (int j = 0; j < nk; ++j) {
+        const float w = sw[p][j];
+        const float4 va = *reinterpret_cast<const float4*>(&sv[j][d0]);
+        const float4 vb4 = *reinterpret_cast<const float4*>(&sv[j][d0 + 4]);
+        diff[0] = fmaf(w, va.x, diff[0]);
+        diff[1] = fmaf(w, va.y, diff[1]);
+        diff[2] = fmaf(w, va.z, diff[2]);
+        diff[3] = fmaf(w, va.w, diff[3]);
+        diff[4] = fmaf(w, vb4.x, diff[4]);
+        diff[5] = fmaf(w, vb4.y, diff[5]);
+        diff[6] = fmaf(w, vb4.z, diff[6]);
+        diff[7] = fmaf(w, vb4.w, diff[7]);
+      }
+    if (j_now + kRouteKeys >= n) {
+      // cluster c_now done: minus the centroid term, the norm (taken with reference m)
       const float wc = static_cast<float>(n) * __expf(lc - m);
+      float e2 = 0.f;
       if (has_dims)
 #pragma unroll
         for (int i = 0; i < DPT; ++i) {
-          const float dd = diff[i] - wc * vb[c * D + d0 + i];
+          const float dd = diff[i] - wc * vb[c_now * D + d0 + i];
           e2 = fmaf(dd, dd, e2);
         }
-    }
 #pragma unroll
-    for (int s = 8; s > 0; s >>= 1) e2 += __shfl_xor_sync(0xffffffffu, e2, s);
-    if (sub == 0 && pa < a.Cq) {
-      err[c] = sqrtf(e2);
-      mref[c] = m;
+      for (int s = 8; s > 0; s >>= 1) e2 += __shfl_xor_sync(0xffffffffu, e2, s);
+      if (sub == 0 && pa < a.Cq) {
+        err[c_now] = sqrtf(e2);
+        mref[c_now] = m;
+      }
     }
+    __syncthreads();  // the chunk's shared-memory rows are read; the next may overwrite
   }
   __syncwarp();
   if (pa < a.Cq) {
-    for (int c = sub; c < a.Ck; c += 16) {
-      const bool ok = live && a.k_count[c] > 0 && z > 0.f;
-      err[c] = ok ? err[c] * __expf(mref[c] - m) / z : 0.f;
+    for (int cc = sub; cc < a.Ck; cc += 16) {
+      const bool ok = live && a.k_count[cc] > 0 && z > 0.f;
+      err[cc] = ok ? err[cc] * __expf(mref[cc] - m) / z : 0.f;
     }
   }
 }
@@ -220,6 +276,9 @@ __global__ void __launch_bounds__(1024) route_select_kernel(const float* __restr
                                                             const int32_t* __restrict__ k_count,
                                                             int Cq, int Ck, double density,
                                                             uint8_t* __restrict__ mask) {
+  // per-warp histograms (most ratios share their top bits: one histogram for the whole
+  // CTA would serialise its atomics), summed into hist after each pass
+  extern __shared__ unsigned long long whist[];  // 32 x 256
   __shared__ unsigned long long hist[256];
   __shared__ unsigned long long s_part[32];
   __shared__ unsigned long long s_sq, s_sk;
@@ -257,7 +316,7 @@ __global__ void __launch_bounds__(1024) route_select_kernel(const float* __restr
   // radix descent: after pass p the top 8(p+1) bits of k* are known
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += 1024) hist[i] = 0;
+    for (int i = tid; i < 32 * 256; i += 1024) whist[i] = 0;
     __syncthreads();
     const uint32_t pre = s_prefix;
     const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
@@ -266,7 +325,13 @@ __global__ void __launch_bounds__(1024) route_select_kernel(const float* __restr
       long long cost;
       if (!key_of(e, key, cost)) continue;
       if ((key & hi_mask) != (pre & hi_mask)) continue;
-      atomicAdd(&hist[(key >> shift) & 255u], static_cast<unsigned long long>(cost));
+      atomicAdd(&whist[warp * 256 + ((key >> shift) & 255u)], static_cast<unsigned long long>(cost));
+    }
+    __syncthreads();
+    for (int i = tid; i < 256; i += 1024) {
+      unsigned long long t = 0;
+      for (int w = 0; w < 32; ++w) t += whist[w * 256 + i];
+      hist[i] = t;
     }
     __syncthreads();
     if (tid == 0) {
@@ -386,6 +451,7 @@ namespace {
 struct RouteLayout {
   int32_t *q_tok, *q_count, *q_off, *k_tok, *k_count, *k_off;
   float *qbar, *kbar, *vbar, *err, *mref;
+  void *kp, *vp;  // keys and values in cluster-major order
   size_t bytes;
 };
 RouteLayout carve_route(const bsa_shape& s, int Cq, int Ck, void* ws) {
@@ -402,6 +468,9 @@ RouteLayout carve_route(const bsa_shape& s, int Cq, int Ck, void* ws) {
   L.vbar = cv.take<float>(static_cast<size_t>(s.B) * s.Hkv * Ck * s.D);
   L.err = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
   L.mref = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
+  const int es = s.dtype == BSA_F32 ? 4 : 2;
+  L.kp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * s.Sk * s.D * es);
+  L.vp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * s.Sk * s.D * es);
   L.bytes = align_up(cv.used, 256);
   return L;
 }
@@ -523,12 +592,23 @@ int route_prologue(const void* q, const void* k, const void* v, const bsa_shape&
   ra.mref = L.mref;
   double route_density = static_cast<double>(density);
   if (with_v) {
+    // keys and values in cluster-major order (rows off[c] .. off[c] + n_c per head)
+    const int es = s.dtype == BSA_F32 ? 4 : 2;
+    const int vpr = s.D * es / 16;
+    const int64_t nvec = static_cast<int64_t>(s.Sk) * vpr;
+    const dim3 gg(static_cast<unsigned>((nvec + 255) / 256), s.Hkv, s.B);
+    gather_rows_kernel<<<gg, 256, 0, st>>>(static_cast<const uint4*>(k), static_cast<uint4*>(L.kp),
+                                           L.k_tok, s.Sk, s.Sk, vpr, s.Hkv);
+    gather_rows_kernel<<<gg, 256, 0, st>>>(static_cast<const uint4*>(v), static_cast<uint4*>(L.vp),
+                                           L.k_tok, s.Sk, s.Sk, vpr, s.Hkv);
+    count_launch();
+    count_launch();
     if (s.dtype == BSA_F32) {
-      if (s.D == 64) launch_route_probe<float, 64>(k, v, ra, st);
-      else launch_route_probe<float, 128>(k, v, ra, st);
+      if (s.D == 64) launch_route_probe<float, 64>(L.kp, L.vp, ra, st);
+      else launch_route_probe<float, 128>(L.kp, L.vp, ra, st);
     } else {
-      if (s.D == 64) launch_route_probe<__nv_bfloat16, 64>(k, v, ra, st);
-      else launch_route_probe<__nv_bfloat16, 128>(k, v, ra, st);
+      if (s.D == 64) launch_route_probe<__nv_bfloat16, 64>(L.kp, L.vp, ra, st);
+      else launch_route_probe<__nv_bfloat16, 128>(L.kp, L.vp, ra, st);
     }
   } else {
     if (s.D == 64)
@@ -542,8 +622,14 @@ int route_prologue(const void* q, const void* k, const void* v, const bsa_shape&
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "route score kernel"))) return rc;
   // 4. budgeted prefix per (batch, head)
-  route_select_kernel<<<s.B * s.Hq, 1024, 0, st>>>(ra.err, L.q_count, L.k_count, Cq, Ck,
-                                                   route_density, mask);
+  {
+    const int smem = 32 * 256 * 8;
+    cudaError_t e = cudaFuncSetAttribute(route_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(route_select)");
+    route_select_kernel<<<s.B * s.Hq, 1024, smem, st>>>(ra.err, L.q_count, L.k_count, Cq, Ck,
+                                                         route_density, mask);
+  }
   count_launch();
   return check_cuda(cudaGetLastError(), "route_select_kernel");
 }

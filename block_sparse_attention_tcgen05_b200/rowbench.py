@@ -257,20 +257,22 @@ def main():
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--calls", type=int, default=20)
     p.add_argument("--out", default=None, help="also write the JSON lines to this file")
+    p.add_argument("--only", default=None,
+                   help="comma-separated groups to run (cache_scoring, attention, routing, "
+                        "probe_repair); default all")
     args = p.parse_args()
+    groups = set(args.only.split(",")) if args.only else None
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     hbm, tc, src = peaks()
     timer = Timer(dev, args.calls)
     out = []
     t0 = time.time()
-    bench_cache_and_scoring(timer, dev, hbm, tc, out)
-    torch.cuda.empty_cache()
-    bench_attention(timer, dev, hbm, tc, out)
-    torch.cuda.empty_cache()
-    bench_routing_and_sta(timer, dev, hbm, tc, out)
-    torch.cuda.empty_cache()
-    bench_probe_and_repair(timer, dev, hbm, tc, out)
+    for name, fn in (("cache_scoring", bench_cache_and_scoring), ("attention", bench_attention),
+                     ("routing", bench_routing_and_sta), ("probe_repair", bench_probe_and_repair)):
+        if groups is None or name in groups:
+            fn(timer, dev, hbm, tc, out)
+            torch.cuda.empty_cache()
     st, _ = ops.device_status(dev)
     if st != 0:
         raise RuntimeError(f"device status {st}")

@@ -46,8 +46,9 @@ def test_status_strings(lib):
 def test_workspace_queries(lib):
     sh = _lib.Shape(1, 40, 40, 32760, 32760, 128, _lib.BSA_BF16)
     n = lib.bsa_attention_workspace_bytes(sh, 245, 245)
-    # permuted Q, K, V copies dominate: about 3 x 40 x 36k x 128 x 2 bytes
-    assert 1.0e9 < n < 1.5e9
+    # the permuted K and V copies dominate (Q rows are gathered by the attention kernel
+    # itself): about 2 x 40 x 36k x 128 x 2 bytes
+    assert 0.6e9 < n < 0.9e9
     assert lib.bsa_attention_workspace_bytes(_lib.Shape(1, 1, 1, 100, 100, 96, 0), 1, 1) == 0
     assert lib.bsa_repair_workspace_bytes(1, 24, 32768, 128, 64) > 0
     assert lib.bsa_repair_workspace_bytes(1, 24, 32768, 96, 64) == 0
