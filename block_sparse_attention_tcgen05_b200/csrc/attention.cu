@@ -332,9 +332,21 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
     }
     warp_tot[lane] = ti - t;
   }
+  __shared__ int s_full;
+  if (tid == 0) s_full = 0;
   __syncthreads();
   const int total = s_total;  // rows with a valid label
-  int base = warp_tot[warp] + incl - local;
+  {
+    const int fp = __reduce_add_sync(0xffffffffu, local);
+    if (lane == 0) atomicAdd(&s_full, fp);
+  }
+  __syncthreads();
+  // The mixed tiles (leftover rows, the costliest: they walk several clusters' kept
+  // keys) come first, padded to a tile boundary, so that they start early; the whole
+  // tiles follow. The tile count stays ceil(Sq / 128).
+  const int full_rows = s_full, left_rows = total - full_rows;
+  const int pure0 = (left_rows + 127) / 128 * 128;
+  int base = pure0 + warp_tot[warp] + incl - local;
   for (int c = c0; c < c1; ++c) {
     const int n = pa.count[c], full = n / 128 * 128;
     rem[c] = n - full;
@@ -351,77 +363,64 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
       pa.row_label[poff[c] + i] = c;
     }
   }
-  for (int r = total + tid; r < pa.Sqpad; r += 1024) {
+  for (int r = left_rows + tid; r < pure0; r += 1024) {  // pad of the last mixed tile
+    pa.row_token[r] = -1;
+    pa.row_label[r] = -1;
+  }
+  for (int r = pure0 + full_rows + tid; r < pa.Sqpad; r += 1024) {
     pa.row_token[r] = -1;
     pa.row_label[r] = -1;
   }
   // ------------------------------------------------ leftover rows: one piece per step,
-  // the candidates scored by all threads (one cluster each), the choice taken by a
-  // block-wide minimum of (score, label); the rows are copied once the order is known.
-  __shared__ unsigned long long s_red[32];
-  __shared__ int s_left, s_room, s_dst, s_npieces, s_cur, s_new;
-  if (tid == 0) {
-    s_dst = 0;
-    s_room = 0;
-    s_npieces = 0;
-  }
-  __syncthreads();
-  const int full_part = __reduce_add_sync(0xffffffffu, local);  // rows in whole tiles
-  if (lane == 0) atomicAdd(&s_dst, full_part);
-  __syncthreads();
-  if (tid == 0) s_left = total - s_dst;
-  __syncthreads();
-  while (s_left > 0) {
-    const bool new_tile = s_room == 0;
-    unsigned long long best = ~0ull;
-    for (int c = tid; c < Cq; c += 1024) {
-      const int rc = rem[c];
-      if (rc == 0) continue;
-      unsigned long long key;
-      if (!pa.greedy) {
-        key = static_cast<unsigned long long>(c);                         // label order
-      } else if (new_tile) {
-        key = (static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(rc)) << 32) | c;
-      } else {
-        int add = 0;
-        for (int w = 0; w < Wc; ++w) add += __popc(any[w * Cq + c] & ~uni[w]);
-        key = (static_cast<unsigned long long>(add) << 32) | c;
+  // chosen by warp 0 alone (no CTA barrier per step): each lane scores the clusters
+  // lane, lane + 32, ... (word-major bitsets: conflict-free reads), a warp minimum of
+  // (score, label) picks the piece; the rows are copied once the order is known.
+  __shared__ int s_npieces;
+  if (warp == 0) {
+    int left = left_rows, room = 0, dst = 0, npieces = 0;
+    while (left > 0) {
+      const bool new_tile = room == 0;
+      unsigned long long best = ~0ull;
+      for (int c = lane; c < Cq; c += 32) {
+        const int rc = rem[c];
+        if (rc == 0) continue;
+        unsigned long long key;
+        if (!pa.greedy) {
+          key = static_cast<unsigned long long>(c);                       // label order
+        } else if (new_tile) {
+          key = (static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(rc)) << 32) | c;
+        } else {
+          int add = 0;
+          for (int w = 0; w < Wc; ++w) add += __popc(any[w * Cq + c] & ~uni[w]);
+          key = (static_cast<unsigned long long>(add) << 32) | c;
+        }
+        best = key < best ? key : best;
       }
-      best = key < best ? key : best;
-    }
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
-      best = y < best ? y : best;
-    }
-    if (lane == 0) s_red[warp] = best;
-    __syncthreads();
-    if (warp == 0) {
-      best = s_red[lane];
+#pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
         best = y < best ? y : best;
       }
-      if (lane == 0) {
-        const int cur = static_cast<int>(best & 0xffffffffull);
-        const int room = new_tile ? 128 : s_room;
-        const int take = min(room, rem[cur]);
-        const int r_all = pa.count[cur] % 128;
-        const int src = pa.off[cur] + pa.count[cur] - r_all + (r_all - rem[cur]);
-        if (s_npieces < pa.max_pieces) pa.pieces[s_npieces] = make_int4(cur, src, take, s_dst);
-        ++s_npieces;
-        rem[cur] -= take;
-        s_room = room - take;
-        s_dst += take;
-        s_left -= take;
-        s_cur = cur;
-        s_new = new_tile ? 1 : 0;
-      }
+      const int cur = static_cast<int>(best & 0xffffffffull);
+      const int room_now = new_tile ? 128 : room;
+      const int rc = rem[cur];
+      const int take = min(room_now, rc);
+      const int r_all = pa.count[cur] % 128;
+      const int src = pa.off[cur] + pa.count[cur] - r_all + (r_all - rc);
+      if (lane == 0 && npieces < pa.max_pieces) pa.pieces[npieces] = make_int4(cur, src, take, dst);
+      if (pa.greedy)
+        for (int w = lane; w < Wc; w += 32) uni[w] = (new_tile ? 0u : uni[w]) | any[w * Cq + cur];
+      __syncwarp();
+      if (lane == 0) rem[cur] = rc - take;
+      __syncwarp();
+      ++npieces;
+      room = room_now - take;
+      dst += take;
+      left -= take;
     }
-    __syncthreads();
-    if (pa.greedy)
-      for (int w = tid; w < Wc; w += 1024) uni[w] = (s_new ? 0u : uni[w]) | any[w * Cq + s_cur];
-    __syncthreads();
+    if (lane == 0) s_npieces = npieces;
   }
+  __syncthreads();
   // copy the leftover rows piece by piece, one warp per piece
   const int np = min(s_npieces, pa.max_pieces);
   for (int pc = warp; pc < np; pc += 32) {

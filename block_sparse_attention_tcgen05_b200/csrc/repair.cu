@@ -699,117 +699,94 @@ __global__ void __launch_bounds__(256) repair_apply_kernel(float* __restrict__ o
   }
 }
 
-constexpr int kApplyWarps = 8;        // warps per CTA
-constexpr int kApplyRowsPerWarp = 32;  // rows per warp
+constexpr int kApplyRows = 128;
+constexpr int kApplyThreads = 64;  // two rows per thread
+constexpr int apply16_smem_bytes(int D) {
+  return static_cast<int>(sizeof(float)) * (2 * D * 16 + kApplyRows * (D + 4) + 16);
+}
 
-// rank <= 16: one warp per row at a time. Lane l holds dims [DPL l, DPL l + DPL) of the
-// row (one coalesced 8- or 16-byte access per lane) and, in registers, the same dims of
-// both factors: P'[d][0..16) and V_r[d][0..16). y = x P' + c' is summed across the
-// lanes by a halving butterfly (lanes trade the half of their 16 partial sums the
-// partner keeps: 8 + 4 + 2 + 1 + 1 shuffles), after which lane l holds y_k for
-// k = l >> 1, and 16 more shuffles give every lane all of y; then x += y V_rᵀ on the
-// lane's own dims. HBM traffic: one read and one write of out; many warps per SM keep
-// the loads in flight. grid (ceil(S / (8 * 32)), B*H), 256 threads; factors zero past
-// `rank`.
+// rank <= 16: tiles of 128 rows staged through shared memory, so that every global
+// access is a coalesced 16-byte vector (HBM traffic: one read and one write of out);
+// then two rows per thread (rows t and t + 64): y = x P' + c' (each factor row d is a
+// broadcast read of 16 floats, all lanes the same address, used for both rows),
+// x += y V_rᵀ (V_rᵀ row k broadcast likewise), pairs of outputs per packed f32x2 FMA.
+// Rows are padded to D + 4 floats, so the eight rows of a quarter-warp fall on distinct
+// 16-byte bank groups. grid (ceil(S / 128), B*H), 64 threads; factors as P'[d][k],
+// V_rᵀ[k][d], zero past `rank`.
 template <int D>
-__global__ void __launch_bounds__(kApplyWarps * 32) repair_apply16_kernel(float* __restrict__ out, int S,
-                                                                         int rank,
-                                                                         const float* __restrict__ pp,
-                                                                         const float* __restrict__ cc,
-                                                                         const float* __restrict__ vr) {
-  constexpr int DPL = D / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__global__ void __launch_bounds__(kApplyThreads) repair_apply16_kernel(float* __restrict__ out, int S,
+                                                                      int rank,
+                                                                      const float* __restrict__ pp,
+                                                                      const float* __restrict__ cc,
+                                                                      const float* __restrict__ vr) {
+  constexpr int TR = kApplyRows, LD = D + 4, V4 = D / 4, NT = kApplyThreads;
+  extern __shared__ __align__(16) float apply_smem[];  // apply16_smem_bytes(D)
+  float(*sP)[16] = reinterpret_cast<float(*)[16]>(apply_smem);
+  float(*sVt)[D] = reinterpret_cast<float(*)[D]>(apply_smem + D * 16);
+  float* xs = apply_smem + 2 * D * 16;
+  float* sc = xs + TR * LD;
   const int64_t bh = blockIdx.y;
-  float fp[DPL][16], fv[DPL][16];
+  for (int e = threadIdx.x; e < D * 16; e += NT) {
+    const int d = e / 16, k = e % 16;
+    const bool in = k < rank;
+    sP[d][k] = in ? pp[(bh * D + d) * rank + k] : 0.f;
+    sVt[k][d] = in ? vr[(bh * D + d) * rank + k] : 0.f;
+  }
+  if (threadIdx.x < 16) sc[threadIdx.x] = threadIdx.x < rank ? cc[bh * rank + threadIdx.x] : 0.f;
+  const int r0 = blockIdx.x * TR;
+  const int nr = min(TR, S - r0);
+  const float4* src = reinterpret_cast<const float4*>(out + (bh * S + r0) * D);
+  // fixed trip count: each thread's TR * V4 / NT loads are in flight together
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) {
-    const int d = DPL * lane + i;
+  for (int i = 0; i < TR * V4 / NT; ++i) {
+    const int e = threadIdx.x + NT * i;
+    if (e < nr * V4) *reinterpret_cast<float4*>(&xs[(e / V4) * LD + 4 * (e % V4)]) = __ldg(src + e);
+  }
+  __syncthreads();
+  // rows a = t and b = t + 64 (rows past nr hold stale values and are not written back)
+  float* xa = &xs[threadIdx.x * LD];
+  float* xb = &xs[(threadIdx.x + NT) * LD];
+  float ya[16], yb[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      fp[i][k] = k < rank ? pp[(bh * D + d) * rank + k] : 0.f;
-      fv[i][k] = k < rank ? vr[(bh * D + d) * rank + k] : 0.f;
+  for (int k = 0; k < 16; ++k) ya[k] = yb[k] = sc[k];
+#pragma unroll 2
+  for (int d4 = 0; d4 < V4; ++d4) {
+    const float4 a4 = *reinterpret_cast<const float4*>(xa + 4 * d4);
+    const float4 b4 = *reinterpret_cast<const float4*>(xb + 4 * d4);
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 p = *reinterpret_cast<const float4*>(&sP[4 * d4 + j][4 * k4]);
+        fma2(ya[4 * k4], ya[4 * k4 + 1], av[j], av[j], p.x, p.y, ya[4 * k4], ya[4 * k4 + 1]);
+        fma2(ya[4 * k4 + 2], ya[4 * k4 + 3], av[j], av[j], p.z, p.w, ya[4 * k4 + 2], ya[4 * k4 + 3]);
+        fma2(yb[4 * k4], yb[4 * k4 + 1], bv[j], bv[j], p.x, p.y, yb[4 * k4], yb[4 * k4 + 1]);
+        fma2(yb[4 * k4 + 2], yb[4 * k4 + 3], bv[j], bv[j], p.z, p.w, yb[4 * k4 + 2], yb[4 * k4 + 3]);
+      }
     }
   }
-  // lane l ends up holding y_k, k = l >> 1; its constant term
-  const float ck = (lane >> 1) < rank ? cc[bh * rank + (lane >> 1)] : 0.f;
-  const int r0 = (blockIdx.x * kApplyWarps + warp) * kApplyRowsPerWarp;
-  const int r1 = min(S, r0 + kApplyRowsPerWarp);
-  constexpr int kBatch = 8;  // rows whose loads are in flight together
-  for (int rb = r0; rb < r1; rb += kBatch) {
-    float xb[kBatch][DPL];
+#pragma unroll 2
+  for (int c4 = 0; c4 < V4; ++c4) {
+    float4 a4 = *reinterpret_cast<const float4*>(xa + 4 * c4);
+    float4 b4 = *reinterpret_cast<const float4*>(xb + 4 * c4);
 #pragma unroll
-    for (int t = 0; t < kBatch; ++t) {
-      const int r = min(rb + t, r1 - 1);  // rows past the end repeat the last (not stored)
-      const float* row = out + (bh * S + r) * D + DPL * lane;
-      if constexpr (DPL == 4) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(row));
-        xb[t][0] = v.x; xb[t][1] = v.y; xb[t][2] = v.z; xb[t][3] = v.w;
-      } else {
-        const float2 v = __ldg(reinterpret_cast<const float2*>(row));
-        xb[t][0] = v.x; xb[t][1] = v.y;
-      }
+    for (int k = 0; k < 16; ++k) {
+      const float4 v = *reinterpret_cast<const float4*>(&sVt[k][4 * c4]);
+      fma2(a4.x, a4.y, ya[k], ya[k], v.x, v.y, a4.x, a4.y);
+      fma2(a4.z, a4.w, ya[k], ya[k], v.z, v.w, a4.z, a4.w);
+      fma2(b4.x, b4.y, yb[k], yb[k], v.x, v.y, b4.x, b4.y);
+      fma2(b4.z, b4.w, yb[k], yb[k], v.z, v.w, b4.z, b4.w);
     }
+    *reinterpret_cast<float4*>(xa + 4 * c4) = a4;
+    *reinterpret_cast<float4*>(xb + 4 * c4) = b4;
+  }
+  __syncthreads();
+  float4* dst = reinterpret_cast<float4*>(out + (bh * S + r0) * D);
 #pragma unroll
-    for (int t = 0; t < kBatch; ++t) {
-      if (rb + t >= r1) continue;
-      float* row = out + (bh * S + rb + t) * D + DPL * lane;
-      float x[DPL];
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) x[i] = xb[t][i];
-      float y[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc = fmaf(x[i], fp[i][k], acc);
-        y[k] = acc;
-      }
-      // halving butterfly over the 16 partial sums
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {  // xor 16: lanes < 16 keep k in [0, 8), others [8, 16)
-        const bool hi = lane & 16;
-        const float send = hi ? y[k] : y[k + 8];
-        const float got = __shfl_xor_sync(0xffffffffu, send, 16);
-        y[k] = (hi ? y[k + 8] : y[k]) + got;
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {  // xor 8
-        const bool hi = lane & 8;
-        const float send = hi ? y[k] : y[k + 4];
-        const float got = __shfl_xor_sync(0xffffffffu, send, 8);
-        y[k] = (hi ? y[k + 4] : y[k]) + got;
-      }
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {  // xor 4
-        const bool hi = lane & 4;
-        const float send = hi ? y[k] : y[k + 2];
-        const float got = __shfl_xor_sync(0xffffffffu, send, 4);
-        y[k] = (hi ? y[k + 2] : y[k]) + got;
-      }
-      {  // xor 2
-        const bool hi = lane & 2;
-        const float send = hi ? y[0] : y[1];
-        const float got = __shfl_xor_sync(0xffffffffu, send, 2);
-        y[0] = (hi ? y[1] : y[0]) + got;
-      }
-      // xor 1: both lanes of a pair hold the same slot; the full sum. Lane l holds slot
-      // 8 [l&16] + 4 [l&8] + 2 [l&4] + [l&2] = (l >> 1) & 15
-      const float mine = y[0] + __shfl_xor_sync(0xffffffffu, y[0], 1) + ck;
-      float acc[DPL];
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[i] = x[i];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float yk = __shfl_sync(0xffffffffu, mine, 2 * k);
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[i] = fmaf(yk, fv[i][k], acc[i]);
-      }
-      if constexpr (DPL == 4) {
-        *reinterpret_cast<float4*>(row) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      } else {
-        *reinterpret_cast<float2*>(row) = make_float2(acc[0], acc[1]);
-      }
-    }
+  for (int i = 0; i < TR * V4 / NT; ++i) {
+    const int e = threadIdx.x + NT * i;
+    if (e < nr * V4) dst[e] = *reinterpret_cast<const float4*>(&xs[(e / V4) * LD + 4 * (e % V4)]);
   }
 }
 
@@ -884,9 +861,11 @@ extern "C" int bsa_probe_residual_correction(float* out, const float* o_probe,
   if ((rc = check_cuda(cudaGetLastError(), "repair_fit_kernel"))) return rc;
   if (rank <= 16) {
     auto ap16 = D == 64 ? repair_apply16_kernel<64> : repair_apply16_kernel<128>;
-    constexpr int rows = kApplyWarps * kApplyRowsPerWarp;
-    ap16<<<dim3((S + rows - 1) / rows, BH), kApplyWarps * 32, 0, st>>>(out, S, rank, L.pp, L.cc,
-                                                                       L.vr);
+    const int smem16 = apply16_smem_bytes(D);
+    e = cudaFuncSetAttribute(ap16, cudaFuncAttributeMaxDynamicSharedMemorySize, smem16);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(repair_apply16)");
+    ap16<<<dim3((S + kApplyRows - 1) / kApplyRows, BH), kApplyThreads, smem16, st>>>(out, S, rank,
+                                                                                    L.pp, L.cc, L.vr);
     count_launch();
     return check_cuda(cudaGetLastError(), "repair_apply16_kernel");
   }
