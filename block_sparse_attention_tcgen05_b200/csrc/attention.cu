@@ -262,16 +262,18 @@ __global__ void __launch_bounds__(256) mask_bits_kernel(
 // tokens), and the rows of one cluster then also compute the other cluster's kept keys.
 // The plan lays the rows out so that tiles mix as few kept sets as possible:
 //   1. every query cluster fills floor(n_a / 128) whole tiles with its own rows (no mix);
-//   2. the remaining n_a mod 128 rows of each cluster are packed into the following
-//      tiles greedily: a tile starts with the cluster that has the most rows left
-//      (ties: lower label) and is then filled, run by run, with the cluster whose kept
-//      key clusters add the fewest new key clusters to the tile's union so far (ties:
-//      lower label), a cluster's rows staying contiguous inside a tile.
-// Kept sets are the OR of the mask over every (batch, head) slice. When the greedy
-// search would be too expensive (Cq * Wc > kPlanGreedyWords) the leftover rows follow
-// in label order instead. Any layout gives the same result; only the work differs.
-// One CTA of 1024 threads; the greedy loop runs in warp 0.
-constexpr int kPlanGreedyWords = 16384;
+//   2. the remaining n_a mod 128 rows of each cluster (its leftover) are laid out in the
+//      order of a nearest-neighbour chain over the clusters' kept sets: the chain starts
+//      at the lowest label with a leftover and moves, step by step, to the unvisited
+//      cluster whose mask row differs from the current one in the fewest key clusters
+//      (Hamming distance; ties: lower label); consecutive leftovers then share tiles.
+// Kept sets are the OR of the mask over every (batch, head) slice. The leftover tiles
+// come first (padded to a tile boundary: they are the costliest and start earliest), the
+// whole tiles follow; the tile count stays ceil(Sq / 128). When the distance matrix
+// does not fit in shared memory (more than kPlanChainMax clusters with a leftover) the
+// leftovers follow in label order. Any layout gives the same result; only the work
+// differs. One CTA of 1024 threads.
+constexpr int kPlanChainMax = 288;  // distance matrix <= 288^2 x 2 bytes
 
 struct PlanArgs {
   const int32_t* sort_token;  // stable label sort of the query rows (cluster-major)
@@ -280,29 +282,31 @@ struct PlanArgs {
   const int32_t* off;         // first sorted slot of each cluster
   const uint32_t* cbits;      // mask bitsets (slice, Cq, Wc) over key clusters
   int n_slices, Cq, Wc, Sqpad;
-  int greedy;
+  int chain;                  // 1: nearest-neighbour chain over the leftovers, 0: label order
   int32_t* row_token;         // out: token of each planned row (-1 = pad)
   int32_t* row_label;         // out: its label (-1 = pad)
-  int4* pieces;               // scratch: (cluster, first sorted slot, rows, first row)
-  int max_pieces;
+  int32_t* scratch;           // 5 * Cq ints of workspace
 };
 
 __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs pa) {
   extern __shared__ uint32_t sm_plan[];
   const int Cq = pa.Cq, Wc = pa.Wc;
-  int32_t* rem = reinterpret_cast<int32_t*>(sm_plan);                 // Cq
+  int32_t* rem = pa.scratch;                                          // Cq
   int32_t* poff = rem + Cq;                                           // Cq
-  uint32_t* uni = reinterpret_cast<uint32_t*>(poff + Cq);             // Wc
-  uint32_t* any = uni + Wc;                                           // Cq * Wc (greedy only)
+  int32_t* lcl = poff + Cq;                                           // Cq: clusters with a leftover
+  int32_t* ord = lcl + Cq;                                            // Cq: chain order (indices into lcl)
+  int32_t* dstp = ord + Cq;                                           // Cq: first row of each leftover
+  uint32_t* any = sm_plan;                                            // Cq * Wc (chain only)
+  uint16_t* dist = reinterpret_cast<uint16_t*>(any + (pa.chain ? Cq * Wc : 0));  // L x L (chain only)
   __shared__ int warp_tot[32];
-  __shared__ int s_total;
+  __shared__ int s_total, s_full, s_L;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  if (pa.greedy) {  // word-major (any[w * Cq + c]): candidate threads read consecutive words
+  if (pa.chain) {
     for (int e = tid; e < Cq * Wc; e += 1024) {
       uint32_t x = 0;
       for (int sl = 0; sl < pa.n_slices; ++sl) x |= pa.cbits[static_cast<size_t>(sl) * Cq * Wc + e];
-      any[(e % Wc) * Cq + e / Wc] = x;
+      any[e] = x;
     }
   }
   // exclusive scan of 128 * floor(n_a / 128): first row of cluster a's whole tiles
@@ -319,10 +323,17 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
     if (lane >= o) incl += y;
   }
   valid = __reduce_add_sync(0xffffffffu, valid);
+  const int fsum = __reduce_add_sync(0xffffffffu, local);
   if (lane == 31) warp_tot[warp] = incl;
-  if (tid == 0) s_total = 0;
+  if (tid == 0) {
+    s_total = 0;
+    s_full = 0;
+  }
   __syncthreads();
-  if (lane == 0) atomicAdd(&s_total, valid);
+  if (lane == 0) {
+    atomicAdd(&s_total, valid);
+    atomicAdd(&s_full, fsum);
+  }
   if (warp == 0) {
     const int t = warp_tot[lane];
     int ti = t;
@@ -332,18 +343,9 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
     }
     warp_tot[lane] = ti - t;
   }
-  __shared__ int s_full;
-  if (tid == 0) s_full = 0;
   __syncthreads();
   const int total = s_total;  // rows with a valid label
-  {
-    const int fp = __reduce_add_sync(0xffffffffu, local);
-    if (lane == 0) atomicAdd(&s_full, fp);
-  }
-  __syncthreads();
-  // The mixed tiles (leftover rows, the costliest: they walk several clusters' kept
-  // keys) come first, padded to a tile boundary, so that they start early; the whole
-  // tiles follow. The tile count stays ceil(Sq / 128).
+  // The leftover tiles come first, padded to a tile boundary; the whole tiles follow.
   const int full_rows = s_full, left_rows = total - full_rows;
   const int pure0 = (left_rows + 127) / 128 * 128;
   int base = pure0 + warp_tot[warp] + incl - local;
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
       pa.row_label[poff[c] + i] = c;
     }
   }
-  for (int r = left_rows + tid; r < pure0; r += 1024) {  // pad of the last mixed tile
+  for (int r = left_rows + tid; r < pure0; r += 1024) {  // pad of the last leftover tile
     pa.row_token[r] = -1;
     pa.row_label[r] = -1;
   }
@@ -371,63 +373,81 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
     pa.row_token[r] = -1;
     pa.row_label[r] = -1;
   }
-  // ------------------------------------------------ leftover rows: one piece per step,
-  // chosen by warp 0 alone (no CTA barrier per step): each lane scores the clusters
-  // lane, lane + 32, ... (word-major bitsets: conflict-free reads), a warp minimum of
-  // (score, label) picks the piece; the rows are copied once the order is known.
-  __shared__ int s_npieces;
+  // ------------------------------------------------ leftovers: the clusters that have
+  // one, in label order (warp 0 compacts them)
   if (warp == 0) {
-    int left = left_rows, room = 0, dst = 0, npieces = 0;
-    while (left > 0) {
-      const bool new_tile = room == 0;
-      unsigned long long best = ~0ull;
-      for (int c = lane; c < Cq; c += 32) {
-        const int rc = rem[c];
-        if (rc == 0) continue;
-        unsigned long long key;
-        if (!pa.greedy) {
-          key = static_cast<unsigned long long>(c);                       // label order
-        } else if (new_tile) {
-          key = (static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(rc)) << 32) | c;
-        } else {
-          int add = 0;
-          for (int w = 0; w < Wc; ++w) add += __popc(any[w * Cq + c] & ~uni[w]);
-          key = (static_cast<unsigned long long>(add) << 32) | c;
-        }
-        best = key < best ? key : best;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
-        best = y < best ? y : best;
-      }
-      const int cur = static_cast<int>(best & 0xffffffffull);
-      const int room_now = new_tile ? 128 : room;
-      const int rc = rem[cur];
-      const int take = min(room_now, rc);
-      const int r_all = pa.count[cur] % 128;
-      const int src = pa.off[cur] + pa.count[cur] - r_all + (r_all - rc);
-      if (lane == 0 && npieces < pa.max_pieces) pa.pieces[npieces] = make_int4(cur, src, take, dst);
-      if (pa.greedy)
-        for (int w = lane; w < Wc; w += 32) uni[w] = (new_tile ? 0u : uni[w]) | any[w * Cq + cur];
-      __syncwarp();
-      if (lane == 0) rem[cur] = rc - take;
-      __syncwarp();
-      ++npieces;
-      room = room_now - take;
-      dst += take;
-      left -= take;
+    int L = 0;
+    for (int c0w = 0; c0w < Cq; c0w += 32) {
+      const int c = c0w + lane;
+      const bool has = c < Cq && rem[c] > 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, has);
+      if (has) lcl[L + __popc(bal & ((1u << lane) - 1u))] = c;
+      L += __popc(bal);
     }
-    if (lane == 0) s_npieces = npieces;
+    if (lane == 0) s_L = L;
   }
   __syncthreads();
-  // copy the leftover rows piece by piece, one warp per piece
-  const int np = min(s_npieces, pa.max_pieces);
-  for (int pc = warp; pc < np; pc += 32) {
-    const int4 pe = pa.pieces[pc];
-    for (int i = lane; i < pe.z; i += 32) {
-      pa.row_token[pe.w + i] = pa.sort_token[pe.y + i];
-      pa.row_label[pe.w + i] = pe.x;
+  const int L = s_L;
+  const bool chain = pa.chain && L <= kPlanChainMax;
+  if (chain) {
+    // Hamming distances between the leftover clusters' kept sets
+    for (int e = tid; e < L * L; e += 1024) {
+      const int i = e / L, j = e % L;
+      const int ci = lcl[i], cj = lcl[j];
+      int d = 0;
+      for (int w = 0; w < Wc; ++w) d += __popc(any[ci * Wc + w] ^ any[cj * Wc + w]);
+      dist[e] = static_cast<uint16_t>(min(d, 65535));
+    }
+    __syncthreads();
+    // the chain (warp 0): from the lowest label, always to the nearest unvisited one. A
+    // visited cluster's column is set to the largest distance (real ones are <= Ck).
+    if (warp == 0) {
+      int cur = 0;
+      for (int i = lane; i < L; i += 32) dist[i * L] = 0xffffu;
+      if (lane == 0) ord[0] = 0;
+      __syncwarp();
+      for (int step = 1; step < L; ++step) {
+        uint32_t best = 0xffffffffu;
+        for (int j = lane; j < L; j += 32) {
+          const uint32_t key = (static_cast<uint32_t>(dist[cur * L + j]) << 16) | static_cast<uint32_t>(j);
+          best = key < best ? key : best;
+        }
+        best = __reduce_min_sync(0xffffffffu, best);
+        cur = static_cast<int>(best & 0xffffu);
+        for (int i = lane; i < L; i += 32) dist[i * L + cur] = 0xffffu;
+        if (lane == 0) ord[step] = cur;
+        __syncwarp();
+      }
+    }
+  } else {
+    for (int t = tid; t < L; t += 1024) ord[t] = t;  // label order
+  }
+  __syncthreads();
+  // first row of each leftover in chain order (warp 0 scans)
+  if (warp == 0) {
+    int run = 0;
+    for (int t0 = 0; t0 < L; t0 += 32) {
+      const int t = t0 + lane;
+      const int r = t < L ? rem[lcl[ord[t]]] : 0;
+      int x = r;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (t < L) dstp[t] = run + x - r;
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+  }
+  __syncthreads();
+  // copy the leftover rows, one warp per cluster
+  for (int t = warp; t < L; t += 32) {
+    const int c = lcl[ord[t]];
+    const int r = rem[c];
+    const int src = pa.off[c] + pa.count[c] - r;
+    const int dst = dstp[t];
+    for (int i = lane; i < r; i += 32) {
+      pa.row_token[dst + i] = pa.sort_token[src + i];
+      pa.row_label[dst + i] = c;
     }
   }
 }
@@ -1341,8 +1361,7 @@ struct AttnLayout {
   int ksplit;   // CTAs per query tile over disjoint key ranges (1 = no split)
   float* part;  // ksplit > 1: partial O (B,Hq,ksplit,Sqpad,D), then max and sum (...,2)
   int32_t *qrow_token, *qrow_label, *qsort_token, *qsort_label, *q_count, *q_off;
-  int4* pieces;     // query tile plan: leftover pieces
-  int max_pieces;
+  int32_t* plan_scratch;  // query tile plan: 5 * Cq ints
   int q_gather;     // the kernel gathers Q rows itself (no permuted copy)
   int32_t *kslot_token, *group_cluster, *group_valid, *k_count, *k_off;
   float* bias2;
@@ -1365,8 +1384,7 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
   L.qrow_label = cv.take<int32_t>(L.Sqpad);
   L.qsort_token = cv.take<int32_t>(L.Sqpad);
   L.qsort_label = cv.take<int32_t>(L.Sqpad);
-  L.max_pieces = Cq + L.Sqpad / 128 + 1;
-  L.pieces = cv.take<int4>(L.max_pieces);
+  L.plan_scratch = cv.take<int32_t>(static_cast<size_t>(5) * Cq);
   L.q_count = cv.take<int32_t>(Cq);
   L.q_off = cv.take<int32_t>(Cq + 1);
   L.kslot_token = cv.take<int32_t>(L.Skpad);
@@ -1515,12 +1533,14 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     pa.Cq = Cq;
     pa.Wc = L.Wc;
     pa.Sqpad = L.Sqpad;
-    pa.greedy = static_cast<int64_t>(Cq) * L.Wc <= kPlanGreedyWords ? 1 : 0;
+    // the chain needs the OR-ed mask rows and the distance matrix in shared memory
+    const size_t chain_bytes = static_cast<size_t>(Cq) * L.Wc * 4 +
+                               static_cast<size_t>(kPlanChainMax) * kPlanChainMax * 2;
+    pa.chain = chain_bytes <= 200 * 1024 ? 1 : 0;
     pa.row_token = L.qrow_token;
     pa.row_label = L.qrow_label;
-    pa.pieces = L.pieces;
-    pa.max_pieces = L.max_pieces;
-    const int smem = (2 * Cq + L.Wc + (pa.greedy ? Cq * L.Wc : 0)) * 4;
+    pa.scratch = L.plan_scratch;
+    const int smem = pa.chain ? static_cast<int>(chain_bytes) : 0;
     cudaError_t e = cudaFuncSetAttribute(plan_query_tiles_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem > 48 * 1024 ? smem : 48 * 1024);

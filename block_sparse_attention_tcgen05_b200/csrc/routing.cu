@@ -77,190 +77,194 @@ struct RouteArgs {
   float* mref;  // (B, Hq, Cq, Ck): per-block reference of the unscaled error (scratch)
 };
 
-// grid (ceil(Cq / 16), Hq, B). Thread t serves probe p = t / 16 and dims
-// [8 (t % 16), 8 (t % 16) + 8) of its running difference vector; for D = 64 only the
-// first 8 lanes of each probe hold dims. kp / vp hold the keys and values of each
-// (batch, KV head) in cluster-major order (cluster c at rows off[c] .. off[c] + n_c),
-// read 32 rows at a time with 16-byte loads; the next chunk's loads are issued into
-// registers before the current chunk is computed. A running reference m (the largest
-// logit seen, centroid logits included) keeps every exponential <= 1. At the end of
-// cluster c the norm of the difference vector and the reference it was taken with are
-// stored; once every cluster is done they are brought to the final reference and
-// divided by Z.
+// grid (ceil(Cq / 16), Hq, B), 256 threads: the 16 probes (query clusters a0 .. a0+15)
+// of one head against every key of its KV head. kp / vp hold the keys and values of each
+// (batch, KV head) in cluster-major order (cluster c at rows off[c] .. off[c] + n_c).
+// Warp w takes the key clusters w, w + 8, ...; inside a cluster lane j holds key j of
+// each 32-key chunk and computes its 16 probe logits (probe rows stored transposed, so
+// one broadcast float4 feeds four probes through packed f32x2 FMAs); each lane also
+// owns dims [DL lane, DL lane + DL) of the 16 running difference vectors
+// sum_j exp(l_j - m) v_j, fed by shuffles of the keys' weights. Every warp keeps its
+// own running reference m (the largest logit it has seen, centroid logits included)
+// and sum z per probe; at the end of a cluster the norm of (difference - n_c exp(lc - m)
+// vbar_c) is stored with the reference it was taken with, and once all warps are done
+// every error is brought to the common reference and divided by the total Z.
 template <typename T, int D>
 __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __restrict__ kp,
                                                                      const T* __restrict__ vp,
                                                                      const RouteArgs a) {
-  constexpr int EPV = 16 / sizeof(T);                       // elements per 16-byte vector
-  constexpr int VPR = D / EPV;                              // vectors per row
-  constexpr int VPT = kRouteKeys * VPR / kRouteThreads;     // vectors per thread per chunk
-  static_assert(VPT >= 1 && kRouteKeys * VPR % kRouteThreads == 0, "chunk split");
-  __shared__ float sq[kRouteProbes][D];
-  __shared__ float sk[kRouteKeys][D + 1];
-  __shared__ __align__(16) float sv[kRouteKeys][D];
-  __shared__ float sw[kRouteProbes][kRouteKeys];
-  const int tid = threadIdx.x, p = tid >> 4, sub = tid & 15;
+  constexpr int NP = kRouteProbes;        // 16
+  constexpr int NW = kRouteThreads / 32;  // 8 warps
+  constexpr int DL = D / 32;              // dims per lane
+  constexpr int EPV = 16 / sizeof(T);     // elements per 16-byte vector
+  __shared__ __align__(16) float sqt[D][NP];   // probe rows, transposed
+  __shared__ float s_m[NW][NP], s_z[NW][NP];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.y, b = blockIdx.z;
   const int hkv = h / (a.Hq / a.Hkv);
-  const int a0 = blockIdx.x * kRouteProbes;
-  const int pa = a0 + p;                    // this thread's query cluster (probe)
-  const bool live = pa < a.Cq && a.q_count[pa] > 0;
+  const int a0 = blockIdx.x * NP;
   const int64_t bq = static_cast<int64_t>(b) * a.Hq + h;
   const int64_t bk = static_cast<int64_t>(b) * a.Hkv + hkv;
-  for (int e = tid; e < kRouteProbes * D; e += kRouteThreads) {
+  for (int e = tid; e < NP * D; e += kRouteThreads) {
     const int pp = e / D, d = e % D;
-    sq[pp][d] = (a0 + pp < a.Cq) ? a.qbar[(bq * a.Cq + a0 + pp) * D + d] : 0.f;
+    sqt[d][pp] = (a0 + pp < a.Cq) ? a.qbar[(bq * a.Cq + a0 + pp) * D + d] : 0.f;
   }
-  constexpr int DPT = 8;                    // dims per thread
-  const bool has_dims = sub * DPT < D;
-  const int d0 = sub * DPT;
-  float m = -INFINITY, z = 0.f;             // running reference and sum of exp(l - m)
-  float diff[DPT];
+  __syncthreads();
   const float* kb = a.kbar + bk * a.Ck * D;
   const float* vb = a.vbar + bk * a.Ck * D;
-  float* err = a.err + (bq * a.Cq + (pa < a.Cq ? pa : 0)) * a.Ck;
-  float* mref = a.mref + (bq * a.Cq + (pa < a.Cq ? pa : 0)) * a.Ck;
-  const uint4* k4 = reinterpret_cast<const uint4*>(kp) + bk * a.S * VPR;
-  const uint4* v4 = reinterpret_cast<const uint4*>(vp) + bk * a.S * VPR;
-  // chunk cursor: cluster c, first key j0 of the chunk inside it
-  int c = 0, j0 = 0;
-  while (c < a.Ck && a.k_count[c] == 0) ++c;
-  uint4 rk[VPT], rv[VPT];
-  auto fetch = [&](int cc, int jj) {
-    const int n = a.k_count[cc], o = a.k_off[cc];
-    const int nk = min(kRouteKeys, n - jj);
+  const T* kbase = kp + bk * a.S * D;
+  const T* vbase = vp + bk * a.S * D;
+  float m[NP], z[NP], diff[NP][DL];
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int e = tid + i * kRouteThreads, j = e / VPR, part = e % VPR;
-      if (j < nk) {
-        rk[i] = __ldg(k4 + static_cast<int64_t>(o + jj + j) * VPR + part);
-        rv[i] = __ldg(v4 + static_cast<int64_t>(o + jj + j) * VPR + part);
-      } else {
-        rk[i] = make_uint4(0, 0, 0, 0);
-        rv[i] = make_uint4(0, 0, 0, 0);
+  for (int p = 0; p < NP; ++p) {
+    m[p] = -INFINITY;
+    z[p] = 0.f;
+  }
+  for (int c = warp; c < a.Ck; c += NW) {
+    const int n = a.k_count[c], o = a.k_off[c];
+    // the (probe, cluster) slots of this cluster: lane p < 16 writes probe p's
+    float* err_p = a.err + (bq * a.Cq + a0 + (lane & (NP - 1))) * a.Ck;
+    float* mref_p = a.mref + (bq * a.Cq + a0 + (lane & (NP - 1))) * a.Ck;
+    const bool writer = lane < NP && a0 + lane < a.Cq;
+    if (n == 0) {
+      if (writer) {
+        err_p[c] = 0.f;
+        mref_p[c] = 0.f;
       }
+      continue;
     }
-  };
-  if (c < a.Ck) fetch(c, 0);
-  __syncthreads();
-  // clusters before the first non-empty one, and empty ones later, store 0
-  for (int cc = 0; cc < c; ++cc)
-    if (sub == 0 && pa < a.Cq) { err[cc] = 0.f; mref[cc] = 0.f; }
-  float lc = 0.f;
-  while (c < a.Ck) {
-    const int n = a.k_count[c];
-    const int nk = min(kRouteKeys, n - j0);
-    if (j0 == 0) {
-#pragma unroll
-      for (int i = 0; i < DPT; ++i) diff[i] = 0.f;
-      // centroid logit of this probe (16 lanes of the probe reduce their dims)
-      lc = 0.f;
-      if (has_dims)
-#pragma unroll
-        for (int i = 0; i < DPT; ++i) lc = fmaf(sq[p][d0 + i], kb[c * D + d0 + i], lc);
-#pragma unroll
-      for (int s = 8; s > 0; s >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, s);
-      lc *= a.scale;
-      if (lc > m) {
-        z *= __expf(m - lc);
-#pragma unroll
-        for (int i = 0; i < DPT; ++i) diff[i] = 0.f;
-        m = lc;
-      }
-    }
-    // the fetched chunk into shared memory (fp32)
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int e = tid + i * kRouteThreads, j = e / VPR, part = e % VPR;
-      float fk[EPV], fv[EPV];
-      unpack16<T>(rk[i], fk);
-      unpack16<T>(rv[i], fv);
-#pragma unroll
-      for (int u = 0; u < EPV; ++u) {
-        sk[j][part * EPV + u] = fk[u];
-        sv[j][part * EPV + u] = fv[u];
-      }
-    }
-    __syncthreads();
-    // next chunk's loads in flight while this one is computed
-    const int c_now = c, j_now = j0;
-    j0 += kRouteKeys;
-    if (j0 >= n) {
-      j0 = 0;
-      ++c;
-      while (c < a.Ck && a.k_count[c] == 0) {
-        if (sub == 0 && pa < a.Cq) { err[c] = 0.f; mref[c] = m; }
-        ++c;
-      }
-    }
-    if (c < a.Ck) fetch(c, j0);
-    // logits of keys sub and sub + 16 for this probe
-    float l0 = 0.f, l1 = 0.f;
+    // centroid logits: lane p (< 16) computes probe p's, then every lane gets all 16
+    float lcl = 0.f;
+    if (lane < NP)
 #pragma unroll 8
-    for (int d = 0; d < D; ++d) {
-      const float x = sq[p][d];
-      l0 = fmaf(x, sk[sub][d], l0);
-      l1 = fmaf(x, sk[sub + 16][d], l1);
-    }
-    l0 = sub < nk ? l0 * a.scale : -INFINITY;
-    l1 = sub + 16 < nk ? l1 * a.scale : -INFINITY;
-    float mx = fmaxf(l0, l1);
+      for (int d = 0; d < D; ++d) lcl = fmaf(sqt[d][lane], kb[c * D + d], lcl);
+    float lc[NP];
 #pragma unroll
-    for (int s = 8; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
-    if (mx > m) {
-      const float f = __expf(m - mx);
-      z *= f;
-#pragma unroll
-      for (int i = 0; i < DPT; ++i) diff[i] *= f;
-      m = mx;
-    }
-    const float w0 = __expf(l0 - m), w1 = __expf(l1 - m);
-    float ws = w0 + w1;
-#pragma unroll
-    for (int s = 8; s > 0; s >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, s);
-    z += ws;
-    sw[p][sub] = w0;
-    sw[p][sub + 16] = w1;
-    __syncwarp();
-    if (has_dims)
-      for (int j = 0; j < nk; ++j) {
-        const float w = sw[p][j];
-        const float4 va = *reinterpret_cast<const float4*>(&sv[j][d0]);
-        const float4 vb4 = *reinterpret_cast<const float4*>(&sv[j][d0 + 4]);
-        diff[0] = fmaf(w, va.x, diff[0]);
-        diff[1] = fmaf(w, va.y, diff[1]);
-        diff[2] = fmaf(w, va.z, diff[2]);
-        diff[3] = fmaf(w, va.w, diff[3]);
-        diff[4] = fmaf(w, vb4.x, diff[4]);
-        diff[5] = fmaf(w, vb4.y, diff[5]);
-        diff[6] = fmaf(w, vb4.z, diff[6]);
-        diff[7] = fmaf(w, vb4.w, diff[7]);
+    for (int p = 0; p < NP; ++p) {
+      lc[p] = __shfl_sync(0xffffffffu, lcl, p) * a.scale;
+      if (lc[p] > m[p]) {
+        z[p] *= __expf(m[p] - lc[p]);
+        m[p] = lc[p];
       }
-    if (j_now + kRouteKeys >= n) {
-      // cluster c_now done: minus the centroid term, the norm (taken with reference m)
-      const float wc = static_cast<float>(n) * __expf(lc - m);
-      float e2 = 0.f;
-      if (has_dims)
 #pragma unroll
-        for (int i = 0; i < DPT; ++i) {
-          const float dd = diff[i] - wc * vb[c_now * D + d0 + i];
-          e2 = fmaf(dd, dd, e2);
+      for (int i = 0; i < DL; ++i) diff[p][i] = 0.f;
+    }
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int nk = min(32, n - j0);
+      const bool mine = lane < nk;
+      // 16 logits of this lane's key
+      float l[NP];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) l[p] = 0.f;
+      const T* krow = kbase + static_cast<int64_t>(o + j0 + (mine ? lane : 0)) * D;
+#pragma unroll 2
+      for (int v0 = 0; v0 < D; v0 += EPV) {
+        float kx[EPV];
+        unpack16<T>(__ldg(reinterpret_cast<const uint4*>(krow + v0)), kx);
+#pragma unroll
+        for (int t = 0; t < EPV; ++t) {
+#pragma unroll
+          for (int p4 = 0; p4 < NP; p4 += 4) {
+            const float4 qv = *reinterpret_cast<const float4*>(&sqt[v0 + t][p4]);
+            fma2(l[p4], l[p4 + 1], kx[t], kx[t], qv.x, qv.y, l[p4], l[p4 + 1]);
+            fma2(l[p4 + 2], l[p4 + 3], kx[t], kx[t], qv.z, qv.w, l[p4 + 2], l[p4 + 3]);
+          }
+        }
+      }
+      // chunk maxima, new references, weights and their sums
+      float w[NP];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) {
+        const float lp = mine ? l[p] * a.scale : -INFINITY;
+        float mx = lp;
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o2));
+        if (mx > m[p]) {
+          const float f = __expf(m[p] - mx);
+          z[p] *= f;
+#pragma unroll
+          for (int i = 0; i < DL; ++i) diff[p][i] *= f;
+          m[p] = mx;
+        }
+        w[p] = mine ? __expf(lp - m[p]) : 0.f;
+        float ws = w[p];
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o2);
+        z[p] += ws;
+      }
+      // difference vectors: the lane's dims of each key's value row
+      for (int jj = 0; jj < nk; ++jj) {
+        const T* vrow = vbase + static_cast<int64_t>(o + j0 + jj) * D + DL * lane;
+        float vx[DL];
+        if constexpr (DL == 4) {
+          const uint2 u = *reinterpret_cast<const uint2*>(vrow);
+          if constexpr (sizeof(T) == 2) {
+            const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+            const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+            vx[0] = lo.x; vx[1] = lo.y; vx[2] = hi.x; vx[3] = hi.y;
+          }
+        }
+        if constexpr (sizeof(T) == 4 || DL != 4) {
+#pragma unroll
+          for (int i = 0; i < DL; ++i) vx[i] = route_f(vrow[i]);
         }
 #pragma unroll
-      for (int s = 8; s > 0; s >>= 1) e2 += __shfl_xor_sync(0xffffffffu, e2, s);
-      if (sub == 0 && pa < a.Cq) {
-        err[c_now] = sqrtf(e2);
-        mref[c_now] = m;
+        for (int p = 0; p < NP; p += 2) {
+          const float w0 = __shfl_sync(0xffffffffu, w[p], jj);
+          const float w1 = __shfl_sync(0xffffffffu, w[p + 1], jj);
+#pragma unroll
+          for (int i = 0; i < DL; ++i) fma2(diff[p][i], diff[p + 1][i], w0, w1, vx[i], vx[i], diff[p][i],
+                                            diff[p + 1][i]);
+        }
       }
     }
-    __syncthreads();  // the chunk's shared-memory rows are read; the next may overwrite
-  }
-  __syncwarp();
-  if (pa < a.Cq) {
-    for (int cc = sub; cc < a.Ck; cc += 16) {
-      const bool ok = live && a.k_count[cc] > 0 && z > 0.f;
-      err[cc] = ok ? err[cc] * __expf(mref[cc] - m) / z : 0.f;
+    // cluster c done: the norm of (difference - centroid term), taken with reference m
+    float vbl[DL];
+#pragma unroll
+    for (int i = 0; i < DL; ++i) vbl[i] = vb[c * D + DL * lane + i];
+    float e2w = 0.f;  // lane p (< 16) ends with probe p's squared norm
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      const float wc = static_cast<float>(n) * __expf(lc[p] - m[p]);
+      float e2 = 0.f;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) {
+        const float dd = diff[p][i] - wc * vbl[i];
+        e2 = fmaf(dd, dd, e2);
+      }
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) e2 += __shfl_xor_sync(0xffffffffu, e2, o2);
+      if (lane == p) e2w = e2;
     }
+    float mw = m[0];
+#pragma unroll
+    for (int p = 1; p < NP; ++p) mw = lane == p ? m[p] : mw;
+    if (writer) {
+      err_p[c] = sqrtf(e2w);
+      mref_p[c] = mw;
+    }
+  }
+  // every warp's references and sums, combined per probe
+  if (lane == 0) {
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+      s_m[warp][p] = m[p];
+      s_z[warp][p] = z[p];
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < NP * a.Ck; e += kRouteThreads) {
+    const int pp = e / a.Ck, c = e % a.Ck;
+    if (a0 + pp >= a.Cq) continue;
+    float M = -INFINITY;
+    for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, s_m[ww][pp]);
+    float Z = 0.f;
+    for (int ww = 0; ww < NW; ++ww)
+      if (s_z[ww][pp] > 0.f) Z += s_z[ww][pp] * __expf(s_m[ww][pp] - M);
+    float* err = a.err + (bq * a.Cq + a0 + pp) * a.Ck;
+    const float* mref = a.mref + (bq * a.Cq + a0 + pp) * a.Ck;
+    const bool ok = a.q_count[a0 + pp] > 0 && a.k_count[c] > 0 && Z > 0.f;
+    err[c] = ok ? err[c] * __expf(mref[c] - M) / Z : 0.f;
   }
 }
 

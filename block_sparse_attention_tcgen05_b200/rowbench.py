@@ -224,6 +224,36 @@ def bench_routing_and_sta(timer, dev, hbm, tc, out):
                    "tensor", tc))
 
 
+def bench_partition(timer, dev, hbm, tc, out):
+    """f2 at the grouped-query shape: response-coupled partition of 24 query heads over 8 KV
+    heads, S=32768, 256 query and key groups; and the probe-budget router on the result's
+    first KV head labels (all 24 heads, density 0.22, M=64)."""
+    Hq, Hkv, S = 24, 8, 32768
+    g = torch.Generator(device=dev).manual_seed(4)
+    q = torch.randn((1, Hq, S, D), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((1, Hkv, S, D), generator=g, device=dev).to(torch.bfloat16)
+    C = S // 128
+    ws = torch.empty(ops._lib.load().bsa_partition_workspace_bytes(ops.make_shape(q, k), C, C, 48, 64),
+                     dtype=torch.uint8, device=dev)
+    ms = timer(lambda: ops.response_coupled_partition(q, k, C, C, workspace=ws))
+    # FMA-pipe work: key features 2 rK D per key, 9 k-means assignments of 2 C rK per key,
+    # query coordinates 2 rQ G D per query row, 9 assignments of 2 C rQ G per query row
+    G = Hq // Hkv
+    flop = Hkv * S * (2 * 48 * D + 9 * 2 * C * 48 + 2 * 64 * G * D + 9 * 2 * C * 64 * G)
+    r = row("f2", "response-coupled partition (24 query / 8 KV heads, S=32768, 256 + 256 groups, "
+            "8 k-means rounds)", ms, flop, "FLOP", "alu", None)
+    alu = fp32_alu_tflops(dev)
+    r.update({"achieved": flop / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "peak": alu,
+              "frac": flop / (ms * 1e-3) / 1e12 / alu,
+              "peak_note": "fp32 FMA pipe: SMs x 128 lanes x 2 x max SM clock"})
+    out.append(r)
+    ql, kl = ops.response_coupled_partition(q, k, C, C, workspace=ws)
+    qlab, klab = ql[0, 0].contiguous(), kl[0, 0].contiguous()
+    ms = timer(lambda: ops.probe_budget_block_mask(q, k, qlab, klab, C, C, 0.22, 64))
+    out.append(row("f2r", "probe-budget router (24 heads, 256 x 256 cells, density 0.22, M=64)", ms,
+                   None, None, "latency", None))
+
+
 def bench_probe_and_repair(timer, dev, hbm, tc, out):
     Hq, Hkv, S, M = 24, 8, 32768, 64
     g = torch.Generator(device=dev).manual_seed(4)
@@ -259,7 +289,7 @@ def main():
     p.add_argument("--out", default=None, help="also write the JSON lines to this file")
     p.add_argument("--only", default=None,
                    help="comma-separated groups to run (cache_scoring, attention, routing, "
-                        "probe_repair); default all")
+                        "partition, probe_repair); default all")
     args = p.parse_args()
     groups = set(args.only.split(",")) if args.only else None
     dev = torch.device("cuda", 0)
@@ -269,7 +299,8 @@ def main():
     out = []
     t0 = time.time()
     for name, fn in (("cache_scoring", bench_cache_and_scoring), ("attention", bench_attention),
-                     ("routing", bench_routing_and_sta), ("probe_repair", bench_probe_and_repair)):
+                     ("routing", bench_routing_and_sta), ("partition", bench_partition),
+                     ("probe_repair", bench_probe_and_repair)):
         if groups is None or name in groups:
             fn(timer, dev, hbm, tc, out)
             torch.cuda.empty_cache()
