@@ -5,16 +5,24 @@
 // Residual" (Q, K, V permuted into group-major order; renormalised hard drop).
 //
 // Pipeline of one call (all on the caller's stream):
-//   1. label_sort_kernel (x2)   stable counting sort of the key / query labels into
-//                               cluster-major slots; each key cluster is padded to a
-//                               multiple of 16 slots, so every 16-key group belongs to
-//                               one cluster.
-//   2. mask_bits_kernel         the uint8 cluster mask -> per query cluster bitsets over
-//                               key clusters (centroid columns) and 16-key groups.
-//   3. gather_rows_kernel       Q rows into cluster-major order (zero pad rows).
-//   4. gather_kv_centroids      K, V rows into cluster-major padded order, fused with
+//   1. mask_cbits_kernel        the uint8 cluster mask -> per query cluster bitsets over
+//                               key clusters (centroid columns).
+//   2. prep_kernel (2 CTAs)     CTA 0: slot-layout order of the key clusters (a nearest-
+//                               neighbour chain over the mask columns, so clusters kept
+//                               by the same query clusters sit side by side), then the
+//                               stable counting sort of the key labels into cluster-
+//                               major slots in that order, each key cluster padded to a
+//                               multiple of 16 slots (every 16-key group belongs to one
+//                               cluster). CTA 1: the query label sort, then the row
+//                               order of the 128-row query tiles (whole tiles of one
+//                               cluster, then the leftover rows packed by a nearest-
+//                               neighbour chain over the clusters' mask rows).
+//   3. mask_gbits_kernel        per query cluster bitsets over the 16-key groups.
+//   4. gather_rows_kernel       Q rows into tile order, only when the attention kernel
+//                               cannot gather them itself by TMA.
+//   5. gather_kv_centroids      K, V rows into cluster-major padded order, fused with
 //                               the per-cluster mean k̄_c, v̄_c (fp32 sums).
-//   5. attn_kernel              one CTA per 128-row query tile: kept key groups are
+//   6. attn_kernel              one CTA per 128-row query tile: kept key groups are
 //                               walked as chunks of up to 128 keys (runs of kept
 //                               groups); skipped clusters follow as 128-wide centroid
 //                               chunks with column bias log2(n_c); both go through
@@ -44,12 +52,22 @@ struct LabelSortJob {
   float* bias2;
   int C_pad;
   uint32_t* nonempty_bits;
+  const int32_t* order;  // nullable: position p of the slot layout holds cluster order[p]
 };
 
-// CTA b sorts job b (the query and key sorts of one call run side by side).
-__global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
-                                                          const LabelSortJob j1) {
-  const LabelSortJob& jb = blockIdx.x == 0 ? j0 : j1;
+// Label sorts with at most kSortFastC clusters take a stable path without CTA-wide
+// barriers inside the token loops: warp w owns the contiguous tokens
+// [w ceil(S/32), (w+1) ceil(S/32)), counts them per label in its own histogram row,
+// and after one scan over (label, warp) scatters them again in token order.
+constexpr int kSortFastC = 512;
+
+// Dynamic shared memory (bytes) a label sort of C clusters needs.
+__host__ __device__ constexpr int label_sort_smem(int C) {
+  return (C <= kSortFastC ? 34 * C + 1 : 2 * C + 1) * 4;
+}
+
+// One CTA of 1024 threads sorts one job; `sm` is label_sort_smem(C) bytes of shared memory.
+__device__ void label_sort_cta(const LabelSortJob& jb, int32_t* sm) {
   const int32_t* __restrict__ labels = jb.labels;
   const int S = jb.S, C = jb.C, cluster_pad = jb.cluster_pad, n_slots = jb.n_slots;
   int32_t* __restrict__ slot_token = jb.slot_token;
@@ -62,9 +80,10 @@ __global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
   float* __restrict__ bias2 = jb.bias2;
   const int C_pad = jb.C_pad;
   uint32_t* __restrict__ nonempty_bits = jb.nonempty_bits;
-  extern __shared__ int32_t sm_i32[];
-  int32_t* cnt = sm_i32;     // C
-  int32_t* run = cnt + C;    // C + 1
+  const int32_t* __restrict__ order = jb.order;
+  int32_t* cnt = sm;           // C
+  int32_t* run = cnt + C;      // C + 1
+  int32_t* hist = run + C + 1;  // 32 x C (fast path): warp-major counts, then slot cursors
   __shared__ int32_t warp_tot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -105,24 +124,62 @@ __global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
       return;
     }
   }
+  const bool fast = C <= kSortFastC;
+  const int per_w = (S + 31) / 32;
+  const int t_lo = min(S, warp * per_w), t_hi = min(S, t_lo + per_w);
   for (int c = tid; c < C; c += 1024) cnt[c] = 0;
+  if (fast)
+    for (int e = tid; e < 32 * C; e += 1024) hist[e] = 0;
   for (int i = tid; i < n_slots; i += 1024) {
     slot_token[i] = -1;
     if (slot_label) slot_label[i] = -1;
   }
   __syncthreads();
-  for (int i = tid; i < S; i += 1024) {
-    const int l = labels[i];
-    if (l >= 0 && l < C) atomicAdd(&cnt[l], 1);
-    else report_device_error(kStatusBadLabel, 30);
+  if (fast) {
+    // eight loads of 32 labels in flight per warp, then their counts
+    for (int b8 = t_lo; b8 < t_hi; b8 += 256) {
+      int lb[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = b8 + 32 * u + lane;
+        lb[u] = i < t_hi ? labels[i] : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool in = b8 + 32 * u + lane < t_hi;
+        int l = lb[u];
+        if (in && (l < 0 || l >= C)) report_device_error(kStatusBadLabel, 30);
+        if (!in || l < 0 || l >= C) l = -1;
+        const unsigned peers = __match_any_sync(0xffffffffu, l);
+        if (l >= 0 && lane == __ffs(peers) - 1) hist[warp * C + l] += __popc(peers);
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    for (int c = tid; c < C; c += 1024) {
+      int t = 0;
+#pragma unroll 8
+      for (int w = 0; w < 32; ++w) t += hist[w * C + c];
+      cnt[c] = t;
+    }
+  } else {
+    for (int i = tid; i < S; i += 1024) {
+      const int l = labels[i];
+      if (l >= 0 && l < C) atomicAdd(&cnt[l], 1);
+      else report_device_error(kStatusBadLabel, 30);
+    }
   }
   __syncthreads();
 
-  // Exclusive scan of the padded cluster sizes; thread t owns a contiguous range.
+  // Exclusive scan of the padded cluster sizes in slot-layout order (label order, or
+  // `order`); thread t owns a contiguous range of positions.
   const int per = (C + 1023) / 1024;
   const int c0 = min(C, tid * per), c1 = min(C, c0 + per);
   int local = 0;
-  for (int c = c0; c < c1; ++c) local += (cnt[c] + cluster_pad - 1) / cluster_pad * cluster_pad;
+  for (int q = c0; q < c1; ++q) {
+    const int c = order ? order[q] : q;
+    local += (cnt[c] + cluster_pad - 1) / cluster_pad * cluster_pad;
+  }
   int incl = local;
   for (int o = 1; o < 32; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -141,7 +198,8 @@ __global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
   }
   __syncthreads();
   int base = warp_tot[warp] + incl - local;
-  for (int c = c0; c < c1; ++c) {
+  for (int q = c0; q < c1; ++q) {
+    const int c = order ? order[q] : q;
     run[c] = base;
     off[c] = base;
     count[c] = cnt[c];
@@ -149,52 +207,88 @@ __global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
   }
   if (tid == 1023) {
     run[C] = base;
-    off[C] = base;
+    off[C] = base;  // total slots in use
   }
   __syncthreads();
 
-  // Stable scatter, 1024 tokens at a time: ranks inside a warp from match_any, warps
-  // take their slots one after another so earlier tokens get earlier slots.
-  for (int t0 = 0; t0 < S; t0 += 1024) {
-    const int i = t0 + tid;
-    int l = (i < S) ? labels[i] : -1;
-    if (l >= C) l = -1;  // out-of-range labels were reported above; the token is dropped
-    const unsigned peers = __match_any_sync(0xffffffffu, l);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    const int leader = __ffs(peers) - 1;
-    int slot_base = 0;
-    for (int w = 0; w < 32; ++w) {
-      if (warp == w && l >= 0 && lane == leader) {
-        slot_base = run[l];
-        run[l] += __popc(peers);
+  if (fast) {
+    // slot cursor of (warp, label): the label's first slot plus the tokens of the
+    // warps before it
+    for (int c = tid; c < C; c += 1024) {
+      int r = run[c];
+      for (int w = 0; w < 32; ++w) {
+        const int t = hist[w * C + c];
+        hist[w * C + c] = r;
+        r += t;
       }
-      __syncthreads();
     }
-    slot_base = __shfl_sync(0xffffffffu, slot_base, leader);
-    if (l >= 0) {
-      const int s = slot_base + rank;
-      slot_token[s] = i;
-      if (slot_label) slot_label[s] = l;
+    __syncthreads();
+    for (int b8 = t_lo; b8 < t_hi; b8 += 256) {
+      int lb[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = b8 + 32 * u + lane;
+        lb[u] = i < t_hi ? labels[i] : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = b8 + 32 * u + lane;
+        int l = lb[u];
+        if (l >= C) l = -1;  // out-of-range labels were reported above; the token is dropped
+        const unsigned peers = __match_any_sync(0xffffffffu, l);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int sb = l >= 0 ? hist[warp * C + l] : 0;
+        __syncwarp();
+        if (l >= 0 && lane == __ffs(peers) - 1) hist[warp * C + l] = sb + __popc(peers);
+        __syncwarp();
+        if (l >= 0) {
+          slot_token[sb + rank] = i;
+          if (slot_label) slot_label[sb + rank] = l;
+        }
+      }
+    }
+  } else {
+    // Stable scatter, 1024 tokens at a time: ranks inside a warp from match_any, warps
+    // take their slots one after another so earlier tokens get earlier slots.
+    for (int t0 = 0; t0 < S; t0 += 1024) {
+      const int i = t0 + tid;
+      int l = (i < S) ? labels[i] : -1;
+      if (l >= C) l = -1;  // out-of-range labels were reported above; the token is dropped
+      const unsigned peers = __match_any_sync(0xffffffffu, l);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int leader = __ffs(peers) - 1;
+      int slot_base = 0;
+      for (int w = 0; w < 32; ++w) {
+        if (warp == w && l >= 0 && lane == leader) {
+          slot_base = run[l];
+          run[l] += __popc(peers);
+        }
+        __syncthreads();
+      }
+      slot_base = __shfl_sync(0xffffffffu, slot_base, leader);
+      if (l >= 0) {
+        const int s = slot_base + rank;
+        slot_token[s] = i;
+        if (slot_label) slot_label[s] = l;
+      }
     }
   }
   __syncthreads();
 
   if (group_cluster) {
+    // groups of every cluster, written by the thread owning it; groups past the last
+    // cluster's slots belong to none
     const int total = off[C];
-    for (int g = tid; g < n_groups; g += 1024) {
-      const int slot = g * 16;
-      int c = -1, valid = 0;
-      if (slot < total) {
-        int lo = 0, hi = C + 1;  // first index with off > slot
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (off[mid] > slot) hi = mid; else lo = mid + 1;
-        }
-        c = lo - 1;
-        valid = min(16, cnt[c] - (slot - off[c]));
+    for (int g = total / 16 + tid; g < n_groups; g += 1024) {
+      group_cluster[g] = -1;
+      group_valid[g] = 0;
+    }
+    for (int c = tid; c < C; c += 1024) {
+      const int n = cnt[c], g0 = off[c] / 16, ng = (n + 15) / 16;  // cluster_pad is 16 here
+      for (int i = 0; i < ng; ++i) {
+        group_cluster[g0 + i] = c;
+        group_valid[g0 + i] = min(16, n - 16 * i);
       }
-      group_cluster[g] = c;
-      group_valid[g] = valid;
     }
   }
   if (bias2) {
@@ -211,19 +305,23 @@ __global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
   }
 }
 
+// CTA b sorts job b (two sorts of one call side by side).
+__global__ void __launch_bounds__(1024) label_sort_kernel(const LabelSortJob j0,
+                                                          const LabelSortJob j1) {
+  extern __shared__ int32_t sm_i32[];
+  label_sort_cta(blockIdx.x == 0 ? j0 : j1, sm_i32);
+}
+
 // ============================================================== mask bitsets
 // grid (Cq, n_h_slices, n_b_slices). cbits[slice][a][w]: bit c of word w = mask[a][32w+c].
-// gbits[slice][a][w]: bit j = mask[a][cluster of 16-key group 32w+j].
-__global__ void __launch_bounds__(256) mask_bits_kernel(
-    const uint8_t* __restrict__ mask, int64_t bstride, int64_t hstride, int nh, int Cq, int Ck,
-    const int32_t* __restrict__ group_cluster, const int32_t* __restrict__ group_valid,
-    int n_groups, int Wc, int Wg, uint32_t* __restrict__ cbits, uint32_t* __restrict__ gbits,
-    uint32_t* __restrict__ gfull) {
+__global__ void __launch_bounds__(256) mask_cbits_kernel(const uint8_t* __restrict__ mask,
+                                                         int64_t bstride, int64_t hstride, int nh,
+                                                         int Cq, int Ck, int Wc,
+                                                         uint32_t* __restrict__ cbits) {
   const int a = blockIdx.x, hs = blockIdx.y, bs = blockIdx.z;
   const uint8_t* row = mask + bs * bstride + hs * hstride + static_cast<int64_t>(a) * Ck;
   const size_t slice = static_cast<size_t>(bs) * nh + hs;
   uint32_t* crow = cbits + (slice * Cq + a) * Wc;
-  uint32_t* grow = gbits + (slice * Cq + a) * Wg;
   for (int w = threadIdx.x; w < Wc; w += blockDim.x) {
     uint32_t bits = 0;
     for (int j = 0; j < 32; ++j) {
@@ -232,13 +330,28 @@ __global__ void __launch_bounds__(256) mask_bits_kernel(
     }
     crow[w] = bits;
   }
+}
+
+// grid (Cq, n_slices). gbits[slice][a][w]: bit j = kept(a, cluster of 16-key group 32w+j),
+// from the cluster bitsets; gfull: bit j = group 32w+j holds 16 real keys.
+__global__ void __launch_bounds__(256) mask_gbits_kernel(const uint32_t* __restrict__ cbits,
+                                                         int Cq, int Wc,
+                                                         const int32_t* __restrict__ group_cluster,
+                                                         const int32_t* __restrict__ group_valid,
+                                                         int n_groups, int Wg,
+                                                         uint32_t* __restrict__ gbits,
+                                                         uint32_t* __restrict__ gfull) {
+  const int a = blockIdx.x;
+  const size_t slice = blockIdx.y;
+  const uint32_t* crow = cbits + (slice * Cq + a) * Wc;
+  uint32_t* grow = gbits + (slice * Cq + a) * Wg;
   for (int w = threadIdx.x; w < Wg; w += blockDim.x) {
     uint32_t bits = 0;
     for (int j = 0; j < 32; ++j) {
       const int g = w * 32 + j;
       if (g < n_groups) {
         const int c = group_cluster[g];
-        if (c >= 0 && row[c]) bits |= 1u << j;
+        if (c >= 0 && ((crow[c >> 5] >> (c & 31)) & 1u)) bits |= 1u << j;
       }
     }
     grow[w] = bits;
@@ -255,6 +368,143 @@ __global__ void __launch_bounds__(256) mask_bits_kernel(
   }
 }
 
+// ============================================================== nearest-neighbour chain
+// Order of n items (n <= kChainMax) given as bitsets of W words, stored transposed in
+// shared memory (bitsT[w * n + i] = word w of item i): start at item 0, then move, step
+// by step, to the unvisited item whose bitset differs from the current one in the
+// fewest bits (Hamming distance; ties: lower index). `dist` is shared scratch of
+// n x chain_stride(n) uint16. All threads of the CTA call it; warp 0 walks the chain and
+// writes ord[0..n).
+constexpr int kChainMax = 288;
+
+// Row stride of the distance matrix: even (two entries per 32-bit load) with an odd
+// number of words, so that the mirrored column writes hit distinct banks.
+__host__ __device__ constexpr int chain_stride(int n) {
+  return ((n + 1) / 2 % 2 == 0) ? (n + 1) / 2 * 2 + 2 : (n + 1) / 2 * 2;
+}
+
+__device__ void nn_chain(const uint32_t* bitsT, int n, int W, uint16_t* dist, int32_t* ord) {
+  if (n <= 0) return;
+  constexpr int kK = (kChainMax + 31) / 32;   // items per lane in the distance rows
+  constexpr int kK2 = (kChainMax + 63) / 64;  // item pairs per lane in the chain
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int np = chain_stride(n);
+  // distances: warp per item i, lane per item j > i (mirrored into column i); 8 words
+  // of item i at a time in registers
+  for (int i = warp; i < n; i += nwarps) {
+    int d[kK];
+#pragma unroll
+    for (int k = 0; k < kK; ++k) d[k] = 0;
+    for (int w0 = 0; w0 < W; w0 += 8) {
+      uint32_t ri[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) ri[t] = w0 + t < W ? bitsT[(w0 + t) * n + i] : 0u;
+#pragma unroll
+      for (int k = 0; k < kK; ++k) {
+        const int j = lane + 32 * k;
+        if (j > i && j < n) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (w0 + t < W) d[k] += __popc(ri[t] ^ bitsT[(w0 + t) * n + j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kK; ++k) {
+      const int j = lane + 32 * k;
+      if (j > i && j < n) {
+        const uint16_t v = static_cast<uint16_t>(min(d[k], 65534));
+        dist[i * np + j] = v;
+        dist[j * np + i] = v;
+      } else if (j == i) {
+        dist[i * np + i] = 0;
+      } else if (j >= n && j < np) {
+        dist[i * np + j] = 0xffffu;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // lane owns items 2 lane + 64 k and 2 lane + 64 k + 1; bit 2k (+1) of `vis` marks
+    // them visited
+    uint32_t vis = lane == 0 ? 1u : 0u;
+    int cur = 0;
+    if (lane == 0) ord[0] = 0;
+    for (int step = 1; step < n; ++step) {
+      const uint32_t* row = reinterpret_cast<const uint32_t*>(dist + cur * np);
+      uint32_t best = 0xffffffffu;
+#pragma unroll
+      for (int k = 0; k < kK2; ++k) {
+        const int j = 2 * lane + 64 * k;
+        if (j < n) {
+          const uint32_t wd = row[j >> 1];
+          const uint32_t k0 = ((vis >> (2 * k)) & 1u) ? 0xffffffffu : ((wd & 0xffffu) << 16) | j;
+          const uint32_t k1 = (j + 1 >= n || ((vis >> (2 * k + 1)) & 1u))
+                                  ? 0xffffffffu
+                                  : ((wd >> 16) << 16) | (j + 1);
+          best = min(best, min(k0, k1));
+        }
+      }
+      best = __reduce_min_sync(0xffffffffu, best);
+      cur = static_cast<int>(best & 0xffffu);
+      if (lane == ((cur & 63) >> 1)) vis |= 1u << (2 * (cur >> 6) + (cur & 1));
+      if (lane == 0) ord[step] = cur;
+    }
+  }
+}
+
+// OR of the mask bitsets over every (batch, head) slice: any[a][w] (Cq x Wc words).
+__device__ void or_slices(const uint32_t* __restrict__ cbits, int n_slices, int Cq, int Wc,
+                          uint32_t* any) {
+  for (int e = threadIdx.x; e < Cq * Wc; e += blockDim.x) {
+    uint32_t x = 0;
+    for (int sl = 0; sl < n_slices; ++sl) x |= cbits[static_cast<size_t>(sl) * Cq * Wc + e];
+    any[e] = x;
+  }
+}
+
+// ============================================================== key cluster order
+// The slot layout of the key clusters decides how a query tile's kept key groups fall
+// into runs, and so how many chunks (of at most 128 keys) the attention kernel walks.
+// Clusters whose columns of the mask (the query clusters keeping them, OR-ed over every
+// (batch, head) slice) are alike are laid out next to each other: the nearest-neighbour
+// chain above over the key clusters' columns. Without room for it (more than kChainMax
+// key clusters, or too many query clusters) the label order is kept.
+struct KeyOrderArgs {
+  const uint32_t* cbits;
+  int n_slices, Cq, Ck, Wc;
+  int chain;
+  int32_t* order;  // out: Ck
+};
+
+// Shared memory of the chain over the key clusters.
+__host__ __device__ constexpr size_t key_order_smem(int Cq, int Ck) {
+  return (static_cast<size_t>(Cq) * ((Ck + 31) / 32) + static_cast<size_t>((Cq + 31) / 32) * Ck) * 4 +
+         static_cast<size_t>(Ck) * chain_stride(Ck) * 2;
+}
+
+__device__ void key_order_cta(const KeyOrderArgs& ka, uint8_t* sm) {
+  const int Cq = ka.Cq, Ck = ka.Ck, Wc = ka.Wc, Wq = (Cq + 31) / 32;
+  if (!ka.chain) {
+    for (int c = threadIdx.x; c < Ck; c += blockDim.x) ka.order[c] = c;
+    return;
+  }
+  uint32_t* any = reinterpret_cast<uint32_t*>(sm);  // Cq x Wc
+  uint32_t* colT = any + Cq * Wc;                    // Wq x Ck: word w of column c at w*Ck + c
+  uint16_t* dist = reinterpret_cast<uint16_t*>(colT + Wq * Ck);
+  or_slices(ka.cbits, ka.n_slices, Cq, Wc, any);
+  __syncthreads();
+  for (int e = threadIdx.x; e < Wq * Ck; e += blockDim.x) {
+    const int w = e / Ck, c = e % Ck;
+    uint32_t bits = 0;
+    for (int j = 0; j < 32 && 32 * w + j < Cq; ++j)
+      bits |= ((any[(32 * w + j) * Wc + (c >> 5)] >> (c & 31)) & 1u) << j;
+    colT[e] = bits;
+  }
+  __syncthreads();
+  nn_chain(colT, Ck, Wq, dist, ka.order);
+}
+
 // ============================================================== query tile plan
 // The attention kernel computes every key group that any row of a 128-row query tile
 // keeps, for all 128 rows. With query rows in plain cluster order a tile straddles two
@@ -269,11 +519,10 @@ __global__ void __launch_bounds__(256) mask_bits_kernel(
 //      (Hamming distance; ties: lower label); consecutive leftovers then share tiles.
 // Kept sets are the OR of the mask over every (batch, head) slice. The leftover tiles
 // come first (padded to a tile boundary: they are the costliest and start earliest), the
-// whole tiles follow; the tile count stays ceil(Sq / 128). When the distance matrix
-// does not fit in shared memory (more than kPlanChainMax clusters with a leftover) the
-// leftovers follow in label order. Any layout gives the same result; only the work
+// whole tiles follow; the tile count stays ceil(Sq / 128). When the chain does not fit
+// in shared memory (more than kChainMax clusters with a leftover, or mask rows too long)
+// the leftovers follow in label order. Any layout gives the same result; only the work
 // differs. One CTA of 1024 threads.
-constexpr int kPlanChainMax = 288;  // distance matrix <= 288^2 x 2 bytes
 
 struct PlanArgs {
   const int32_t* sort_token;  // stable label sort of the query rows (cluster-major)
@@ -288,27 +537,27 @@ struct PlanArgs {
   int32_t* scratch;           // 5 * Cq ints of workspace
 };
 
-__global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs pa) {
-  extern __shared__ uint32_t sm_plan[];
+// Shared memory of the chain over the leftover clusters.
+__host__ __device__ constexpr size_t plan_smem(int Cq, int Wc) {
+  return (static_cast<size_t>(Cq) * Wc + static_cast<size_t>(Wc) * kChainMax) * 4 +
+         static_cast<size_t>(kChainMax) * chain_stride(kChainMax) * 2;
+}
+
+__device__ void plan_cta(const PlanArgs& pa, uint8_t* sm) {
   const int Cq = pa.Cq, Wc = pa.Wc;
   int32_t* rem = pa.scratch;                                          // Cq
   int32_t* poff = rem + Cq;                                           // Cq
   int32_t* lcl = poff + Cq;                                           // Cq: clusters with a leftover
   int32_t* ord = lcl + Cq;                                            // Cq: chain order (indices into lcl)
   int32_t* dstp = ord + Cq;                                           // Cq: first row of each leftover
-  uint32_t* any = sm_plan;                                            // Cq * Wc (chain only)
-  uint16_t* dist = reinterpret_cast<uint16_t*>(any + (pa.chain ? Cq * Wc : 0));  // L x L (chain only)
+  uint32_t* any = reinterpret_cast<uint32_t*>(sm);   // Cq x Wc (chain only)
+  uint32_t* anyT = any + Cq * Wc;                     // Wc x L: the leftovers' rows, transposed
+  uint16_t* dist = reinterpret_cast<uint16_t*>(anyT + Wc * kChainMax);  // L x chain_stride(L)
   __shared__ int warp_tot[32];
   __shared__ int s_total, s_full, s_L;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  if (pa.chain) {
-    for (int e = tid; e < Cq * Wc; e += 1024) {
-      uint32_t x = 0;
-      for (int sl = 0; sl < pa.n_slices; ++sl) x |= pa.cbits[static_cast<size_t>(sl) * Cq * Wc + e];
-      any[e] = x;
-    }
-  }
+  if (pa.chain) or_slices(pa.cbits, pa.n_slices, Cq, Wc, any);
   // exclusive scan of 128 * floor(n_a / 128): first row of cluster a's whole tiles
   const int per = (Cq + 1023) / 1024;
   const int c0 = min(Cq, tid * per), c1 = min(Cq, c0 + per);
@@ -356,13 +605,23 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
     base += full;
   }
   __syncthreads();
-  // whole tiles: rows [0, 128 k_a) of each cluster, in cluster order
-  for (int p = tid; p < total; p += 1024) {
-    const int c = pa.sort_label[p];
-    const int i = p - pa.off[c];
-    if (i < pa.count[c] / 128 * 128) {
-      pa.row_token[poff[c] + i] = pa.sort_token[p];
-      pa.row_label[poff[c] + i] = c;
+  // whole tiles: rows [0, 128 k_a) of each cluster, in cluster order (warp per cluster)
+  {
+    const int32_t* __restrict__ st = pa.sort_token;
+    int32_t* __restrict__ rt = pa.row_token;
+    int32_t* __restrict__ rl = pa.row_label;
+    for (int c = warp; c < Cq; c += 32) {
+      const int full = pa.count[c] / 128 * 128, src = pa.off[c], dst = poff[c];
+      for (int i0 = 0; i0 < full; i0 += 128) {
+        int tk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tk[u] = st[src + i0 + 32 * u + lane];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          rt[dst + i0 + 32 * u + lane] = tk[u];
+          rl[dst + i0 + 32 * u + lane] = c;
+        }
+      }
     }
   }
   for (int r = left_rows + tid; r < pure0; r += 1024) {  // pad of the last leftover tile
@@ -388,37 +647,11 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
   }
   __syncthreads();
   const int L = s_L;
-  const bool chain = pa.chain && L <= kPlanChainMax;
+  const bool chain = pa.chain && L <= kChainMax;
   if (chain) {
-    // Hamming distances between the leftover clusters' kept sets
-    for (int e = tid; e < L * L; e += 1024) {
-      const int i = e / L, j = e % L;
-      const int ci = lcl[i], cj = lcl[j];
-      int d = 0;
-      for (int w = 0; w < Wc; ++w) d += __popc(any[ci * Wc + w] ^ any[cj * Wc + w]);
-      dist[e] = static_cast<uint16_t>(min(d, 65535));
-    }
+    for (int e = tid; e < Wc * L; e += 1024) anyT[e] = any[lcl[e % L] * Wc + e / L];
     __syncthreads();
-    // the chain (warp 0): from the lowest label, always to the nearest unvisited one. A
-    // visited cluster's column is set to the largest distance (real ones are <= Ck).
-    if (warp == 0) {
-      int cur = 0;
-      for (int i = lane; i < L; i += 32) dist[i * L] = 0xffffu;
-      if (lane == 0) ord[0] = 0;
-      __syncwarp();
-      for (int step = 1; step < L; ++step) {
-        uint32_t best = 0xffffffffu;
-        for (int j = lane; j < L; j += 32) {
-          const uint32_t key = (static_cast<uint32_t>(dist[cur * L + j]) << 16) | static_cast<uint32_t>(j);
-          best = key < best ? key : best;
-        }
-        best = __reduce_min_sync(0xffffffffu, best);
-        cur = static_cast<int>(best & 0xffffu);
-        for (int i = lane; i < L; i += 32) dist[i * L + cur] = 0xffffu;
-        if (lane == 0) ord[step] = cur;
-        __syncwarp();
-      }
-    }
+    nn_chain(anyT, L, Wc, dist, ord);
   } else {
     for (int t = tid; t < L; t += 1024) ord[t] = t;  // label order
   }
@@ -449,6 +682,23 @@ __global__ void __launch_bounds__(1024) plan_query_tiles_kernel(const PlanArgs p
       pa.row_token[dst + i] = pa.sort_token[src + i];
       pa.row_label[dst + i] = c;
     }
+  }
+}
+
+// ============================================================== call preparation
+// CTA 0: key cluster order, then the key label sort in that order. CTA 1: query label
+// sort, then the query tile plan. The two chains are independent and run side by side.
+__global__ void __launch_bounds__(1024) prep_kernel(const KeyOrderArgs ka, const LabelSortJob jk,
+                                                    const LabelSortJob jq, const PlanArgs pa) {
+  extern __shared__ __align__(16) uint8_t sm_prep[];
+  if (blockIdx.x == 0) {
+    key_order_cta(ka, sm_prep);
+    __syncthreads();
+    label_sort_cta(jk, reinterpret_cast<int32_t*>(sm_prep));
+  } else {
+    label_sort_cta(jq, reinterpret_cast<int32_t*>(sm_prep));
+    __syncthreads();
+    plan_cta(pa, sm_prep);
   }
 }
 
@@ -1364,6 +1614,7 @@ struct AttnLayout {
   int32_t* plan_scratch;  // query tile plan: 5 * Cq ints
   int q_gather;     // the kernel gathers Q rows itself (no permuted copy)
   int32_t *kslot_token, *group_cluster, *group_valid, *k_count, *k_off;
+  int32_t* korder;  // slot-layout order of the key clusters
   float* bias2;
   uint32_t *cnonempty, *cbits, *gbits, *gfull;
   void *qp, *kp, *vp, *kc, *vc;
@@ -1392,6 +1643,7 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
   L.group_valid = cv.take<int32_t>(L.G);
   L.k_count = cv.take<int32_t>(Ck);
   L.k_off = cv.take<int32_t>(Ck + 1);
+  L.korder = cv.take<int32_t>(Ck);
   L.bias2 = cv.take<float>(L.Ckpad);
   L.cnonempty = cv.take<uint32_t>(L.Wc);
   const size_t slices = static_cast<size_t>(s.B) * s.Hq;
@@ -1463,8 +1715,8 @@ size_t attention_workspace_bytes(const bsa_shape& s, int Cq, int Ck) {
 
 // One or two label sorts in one launch (one CTA each).
 static int launch_label_sorts(const LabelSortJob& j0, const LabelSortJob* j1, cudaStream_t st) {
-  const int c = j1 && j1->C > j0.C ? j1->C : j0.C;
-  const int smem = (2 * c + 1) * 4;
+  const int smem = j1 && label_sort_smem(j1->C) > label_sort_smem(j0.C) ? label_sort_smem(j1->C)
+                                                                        : label_sort_smem(j0.C);
   cudaError_t e = cudaFuncSetAttribute(label_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        smem > 48 * 1024 ? smem : 48 * 1024);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(label_sort)");
@@ -1504,25 +1756,24 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
        reinterpret_cast<uintptr_t>(v)) % 16)
     return fail(BSA_ERR_INVALID_ARG, "q/k/v must be 16-byte aligned");
 
-  // 1. label sorts
+  // 1. cluster bitsets of the mask (label order)
+  const int nb = mbs ? s.B : 1, nh = mhs ? s.Hq : 1;
+  mask_cbits_kernel<<<dim3(Cq, nh, nb), 256, 0, st>>>(mask, mbs, mhs, nh, Cq, Ck, L.Wc, L.cbits);
+  count_launch();
+  if ((rc = check_cuda(cudaGetLastError(), "mask_cbits_kernel"))) return rc;
+  // 2. key cluster order + key label sort (CTA 0) beside query label sort + query tile
+  //    plan (CTA 1)
   {
-    const LabelSortJob jk{k_labels,       s.Sk,           Ck,      16,         L.Skpad,
-                          L.kslot_token,  nullptr,        L.k_count, L.k_off,  L.group_cluster,
-                          L.group_valid,  L.G,            L.bias2, L.Ckpad,    L.cnonempty};
+    KeyOrderArgs ka{L.cbits, nb * nh, Cq, Ck, L.Wc, 0, L.korder};
+    const size_t ko_bytes = key_order_smem(Cq, Ck);
+    ka.chain = Ck <= kChainMax && ko_bytes <= 200 * 1024 ? 1 : 0;
+    LabelSortJob jk{k_labels,       s.Sk,           Ck,      16,         L.Skpad,
+                    L.kslot_token,  nullptr,        L.k_count, L.k_off,  L.group_cluster,
+                    L.group_valid,  L.G,            L.bias2, L.Ckpad,    L.cnonempty};
+    jk.order = L.korder;
     const LabelSortJob jq{q_labels, s.Sq,    Cq,      1,       L.Sqpad, L.qsort_token, L.qsort_label,
                           L.q_count, L.q_off, nullptr, nullptr, 0,       nullptr,      0,
                           nullptr};
-    if ((rc = launch_label_sorts(jk, &jq, st))) return rc;
-  }
-  // 2. mask bitsets
-  const int nb = mbs ? s.B : 1, nh = mhs ? s.Hq : 1;
-  mask_bits_kernel<<<dim3(Cq, nh, nb), 256, 0, st>>>(mask, mbs, mhs, nh, Cq, Ck, L.group_cluster,
-                                                    L.group_valid, L.G, L.Wc, L.Wg, L.cbits,
-                                                    L.gbits, L.gfull);
-  count_launch();
-  if ((rc = check_cuda(cudaGetLastError(), "mask_bits_kernel"))) return rc;
-  // 2b. query tile plan (row order of the query tiles)
-  {
     PlanArgs pa{};
     pa.sort_token = L.qsort_token;
     pa.sort_label = L.qsort_label;
@@ -1533,23 +1784,27 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     pa.Cq = Cq;
     pa.Wc = L.Wc;
     pa.Sqpad = L.Sqpad;
-    // the chain needs the OR-ed mask rows and the distance matrix in shared memory
-    const size_t chain_bytes = static_cast<size_t>(Cq) * L.Wc * 4 +
-                               static_cast<size_t>(kPlanChainMax) * kPlanChainMax * 2;
-    pa.chain = chain_bytes <= 200 * 1024 ? 1 : 0;
+    const size_t plan_bytes = plan_smem(Cq, L.Wc);
+    pa.chain = plan_bytes <= 200 * 1024 ? 1 : 0;
     pa.row_token = L.qrow_token;
     pa.row_label = L.qrow_label;
     pa.scratch = L.plan_scratch;
-    const int smem = pa.chain ? static_cast<int>(chain_bytes) : 0;
-    cudaError_t e = cudaFuncSetAttribute(plan_query_tiles_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem > 48 * 1024 ? smem : 48 * 1024);
-    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(plan_query_tiles)");
-    plan_query_tiles_kernel<<<1, 1024, smem, st>>>(pa);
+    size_t smem = std::max(label_sort_smem(Ck), label_sort_smem(Cq));
+    if (ka.chain) smem = std::max(smem, ko_bytes);
+    if (pa.chain) smem = std::max(smem, plan_bytes);
+    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem > 48 * 1024 ? static_cast<int>(smem) : 48 * 1024);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(prep_kernel)");
+    prep_kernel<<<2, 1024, smem, st>>>(ka, jk, jq, pa);
     count_launch();
-    if ((rc = check_cuda(cudaGetLastError(), "plan_query_tiles_kernel"))) return rc;
+    if ((rc = check_cuda(cudaGetLastError(), "prep_kernel"))) return rc;
   }
-  // 3. Q gather (only when the kernel cannot gather the rows itself)
+  // 3. key-group bitsets (slot layout)
+  mask_gbits_kernel<<<dim3(Cq, nb * nh), 256, 0, st>>>(L.cbits, Cq, L.Wc, L.group_cluster,
+                                                       L.group_valid, L.G, L.Wg, L.gbits, L.gfull);
+  count_launch();
+  if ((rc = check_cuda(cudaGetLastError(), "mask_gbits_kernel"))) return rc;
+  // 4. Q gather (only when the kernel cannot gather the rows itself)
   const int vpr = s.D * es / 16;
   if (!L.q_gather) {
     const int64_t n = static_cast<int64_t>(L.Sqpad) * vpr;
@@ -1559,7 +1814,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     count_launch();
     if ((rc = check_cuda(cudaGetLastError(), "gather_rows_kernel"))) return rc;
   }
-  // 4. K/V gather + centroids. One key cluster without compensation (the probe path)
+  // 5. K/V gather + centroids. One key cluster without compensation (the probe path)
   //    permutes nothing and needs no centroid: the K/V maps then read the caller's
   //    tensors directly (key slot = token, rows per head = Sk).
   const bool kv_identity = Ck == 1 && !compensate && s.Sk % 16 == 0;
@@ -1581,7 +1836,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
     if ((rc = check_cuda(cudaGetLastError(), "gather_kv_centroids_kernel"))) return rc;
   }
 
-  // 5. tensor maps + attention
+  // 6. tensor maps + attention
   const CUtensorMapDataType tdt =
       s.dtype == BSA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint32_t atom = 128 / es;
