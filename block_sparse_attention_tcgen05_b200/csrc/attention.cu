@@ -702,6 +702,50 @@ __global__ void __launch_bounds__(1024) prep_kernel(const KeyOrderArgs ka, const
   }
 }
 
+// ============================================================== dense call preparation
+// One query cluster, one key cluster, the block kept, no compensation (the probe rows'
+// dense attention): the sorts and the plan are identities, so their outputs are filled
+// directly (grid-stride, 256 threads per CTA) instead of by the sparse call's chain.
+__global__ void __launch_bounds__(256) dense_prep_kernel(int Sq, int Sqpad, int Sk, int Skpad, int G,
+                                                         int Wg, int Ckpad, int32_t* qrow_token,
+                                                         int32_t* qrow_label, int32_t* kslot_token,
+                                                         int32_t* group_cluster, int32_t* group_valid,
+                                                         int32_t* k_count, int32_t* k_off,
+                                                         uint32_t* cbits, uint32_t* gbits,
+                                                         uint32_t* gfull, uint32_t* cnonempty,
+                                                         float* bias2) {
+  const int stride = gridDim.x * blockDim.x;
+  const int t0 = blockIdx.x * blockDim.x + threadIdx.x;
+  for (int i = t0; i < Sqpad; i += stride) {
+    qrow_token[i] = i < Sq ? i : -1;
+    qrow_label[i] = i < Sq ? 0 : -1;
+  }
+  for (int i = t0; i < Skpad; i += stride) kslot_token[i] = i < Sk ? i : -1;
+  for (int g = t0; g < G; g += stride) {
+    const int nv = min(16, max(0, Sk - 16 * g));
+    group_cluster[g] = nv > 0 ? 0 : -1;
+    group_valid[g] = nv;
+  }
+  for (int w = t0; w < Wg; w += stride) {
+    uint32_t kept = 0, full = 0;
+    for (int j = 0; j < 32; ++j) {
+      const int g = 32 * w + j;
+      if (g < G && 16 * g < Sk) kept |= 1u << j;
+      if (g < G && 16 * g + 16 <= Sk) full |= 1u << j;
+    }
+    gbits[w] = kept;
+    gfull[w] = full;
+  }
+  for (int c = t0; c < Ckpad; c += stride) bias2[c] = c == 0 && Sk > 0 ? log2f(static_cast<float>(Sk)) : -INFINITY;
+  if (t0 == 0) {
+    cbits[0] = 1u;
+    cnonempty[0] = Sk > 0 ? 1u : 0u;
+    k_count[0] = Sk;
+    k_off[0] = 0;
+    k_off[1] = (Sk + 15) / 16 * 16;
+  }
+}
+
 // ============================================================== gathers
 // dst[bh][r] = src[bh][row_token[r]] (zero row when the token is -1); 16-byte vectors.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src,
@@ -1740,7 +1784,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
                                    const int32_t* k_labels, int Ck, const uint8_t* mask,
                                    int64_t mbs, int64_t mhs, float scale, int compensate,
                                    float* out, void* ws, size_t ws_bytes, cudaStream_t st,
-                                   int prof_id) {
+                                   int prof_id, bool dense) {
   int rc = validate_attention_shape(s, Cq, Ck);
   if (rc) return rc;
   if (!q || !k || !v || !q_labels || !k_labels || !mask || !out)
@@ -1756,8 +1800,20 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
        reinterpret_cast<uintptr_t>(v)) % 16)
     return fail(BSA_ERR_INVALID_ARG, "q/k/v must be 16-byte aligned");
 
-  // 1. cluster bitsets of the mask (label order)
   const int nb = mbs ? s.B : 1, nh = mhs ? s.Hq : 1;
+  if (dense) {
+    // every query row keeps every key: identities instead of steps 1-3
+    if (Cq != 1 || Ck != 1 || compensate || mbs || mhs)
+      return fail(BSA_ERR_INVALID_ARG, "dense preparation needs one cluster each, no compensation");
+    const int n = std::max(L.Sqpad, L.Skpad);
+    dense_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(
+        s.Sq, L.Sqpad, s.Sk, L.Skpad, L.G, L.Wg, L.Ckpad, L.qrow_token, L.qrow_label, L.kslot_token,
+        L.group_cluster, L.group_valid, L.k_count, L.k_off, L.cbits, L.gbits, L.gfull, L.cnonempty,
+        L.bias2);
+    count_launch();
+    if ((rc = check_cuda(cudaGetLastError(), "dense_prep_kernel"))) return rc;
+  } else {
+  // 1. cluster bitsets of the mask (label order)
   mask_cbits_kernel<<<dim3(Cq, nh, nb), 256, 0, st>>>(mask, mbs, mhs, nh, Cq, Ck, L.Wc, L.cbits);
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "mask_cbits_kernel"))) return rc;
@@ -1804,6 +1860,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
                                                        L.group_valid, L.G, L.Wg, L.gbits, L.gfull);
   count_launch();
   if ((rc = check_cuda(cudaGetLastError(), "mask_gbits_kernel"))) return rc;
+  }
   // 4. Q gather (only when the kernel cannot gather the rows itself)
   const int vpr = s.D * es / 16;
   if (!L.q_gather) {
@@ -1914,5 +1971,5 @@ extern "C" int bsa_centroid_compensated_attention(const void* q, const void* k, 
   return bsa::centroid_compensated_attention(q, k, v, shape, q_labels, Cq, k_labels, Ck, block_mask,
                                              mask_b_stride, mask_h_stride, scale, compensate, out,
                                              workspace, workspace_bytes, bsa::as_stream(stream),
-                                             bsa::kProfAttention);
+                                             bsa::kProfAttention, false);
 }

@@ -103,7 +103,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 //     in order of decreasing eigenvalue (classical, applied twice, all warps);
 //  4. back-transformation by the reflectors: U = H x.
 // Output: U (n x min(k, n), row stride ld >= n) and lam[0..k) in decreasing order
-// (zero past n). hv needs n x ld floats, x n x k, work 5n + k n floats.
+// (zero past n). hv needs n x ld floats, x n x k, work 5n + 2 k n floats.
 __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float* U, float* lam,
                                float* x, float* work, float* red) {
   const int tid = threadIdx.x, nt = blockDim.x;
@@ -111,54 +111,79 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
   float* d = work;
   float* e = work + n;        // e[i] couples i and i+1
   float* pv = work + 2 * n;   // A v
-  float* wv = work + 3 * n;   // w = 2(p - K v)
   __shared__ float s_scal[2];
-  // 1. Householder: column k below the diagonal is mapped to (alpha, 0, ..., 0)
+  // 1. Householder: column c below the diagonal is mapped to (alpha, 0, ..., 0). Three
+  //    block barriers per step: warp 0 forms the reflector (column norm by shuffles);
+  //    the warps form p = A' v; every warp then takes v·p on its own (the same sum in
+  //    the same order) and applies the rank-2 update with w = 2 (p - (v·p) v) formed in
+  //    place.
+  __shared__ int s_skip;
   for (int c = 0; c + 2 < n; ++c) {
     const int m = n - c - 1;  // length of the column below the diagonal
-    float ss = 0.f;
-    for (int i = tid; i < m; i += nt) {
-      const float xi = A[(c + 1 + i) * ld + c];
-      ss = fmaf(xi, xi, ss);
-    }
-    ss = block_sum(ss, red);
-    const float x0 = A[(c + 1) * ld + c];
-    const float nrm = sqrtf(ss);
-    const float alpha = x0 > 0.f ? -nrm : nrm;
-    // v = x - alpha e1, normalised; |v|^2 = ss - 2 alpha x0 + alpha^2 = 2(ss - alpha x0)
-    const float vv = 2.f * (ss - alpha * x0);
-    const bool skip = !(vv > 1e-30f * (ss + 1e-30f));
-    const float inv = skip ? 0.f : rsqrtf(vv);
-    for (int i = tid; i < m; i += nt) {
-      const float xi = A[(c + 1 + i) * ld + c];
-      hv[c * ld + i] = (i == 0 ? xi - alpha : xi) * inv;
+    float* v = hv + c * ld;
+    if (wid == 0) {
+      float ss = 0.f;
+      for (int i = lane; i < m; i += 32) {
+        const float xi = A[(c + 1 + i) * ld + c];
+        ss = fmaf(xi, xi, ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float x0 = A[(c + 1) * ld + c];
+      const float nrm = sqrtf(ss);
+      const float alpha = x0 > 0.f ? -nrm : nrm;
+      // v = x - alpha e1, normalised; |v|^2 = ss - 2 alpha x0 + alpha^2 = 2(ss - alpha x0)
+      const float vv = 2.f * (ss - alpha * x0);
+      const bool skip = !(vv > 1e-30f * (ss + 1e-30f));
+      const float inv = skip ? 0.f : rsqrtf(vv);
+      for (int i = lane; i < m; i += 32) {
+        const float xi = A[(c + 1 + i) * ld + c];
+        v[i] = (i == 0 ? xi - alpha : xi) * inv;
+      }
+      if (lane == 0) {
+        d[c] = A[c * ld + c];
+        e[c] = skip ? x0 : alpha;
+        s_skip = skip ? 1 : 0;
+      }
     }
     __syncthreads();
-    if (!skip) {
+    if (!s_skip) {
       // p = A' v over the trailing block A' = A[c+1.., c+1..]: a warp per row, lanes
-      // along it, shuffle sums
-      for (int i = wid; i < m; i += nw) {
-        float acc = 0.f;
-        for (int j = lane; j < m; j += 32) acc = fmaf(A[(c + 1 + i) * ld + c + 1 + j], hv[c * ld + j], acc);
+      // along it; four rows of a warp at a time, their shuffle sums interleaved
+      for (int i0 = wid; i0 < m; i0 += 4 * nw) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) pv[i] = acc;
+        for (int r = 0; r < 4; ++r) {
+          const int i = i0 + r * nw;
+          if (i < m)
+            for (int j = lane; j < m; j += 32) acc[r] = fmaf(A[(c + 1 + i) * ld + c + 1 + j], v[j], acc[r]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            if (i0 + r * nw < m) pv[i0 + r * nw] = acc[r];
+        }
       }
       __syncthreads();
       float kk = 0.f;
-      for (int i = tid; i < m; i += nt) kk = fmaf(hv[c * ld + i], pv[i], kk);
-      kk = block_sum(kk, red);
-      for (int i = tid; i < m; i += nt) wv[i] = 2.f * (pv[i] - kk * hv[c * ld + i]);
-      __syncthreads();
+      for (int i = lane; i < m; i += 32) kk = fmaf(v[i], pv[i], kk);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) kk += __shfl_xor_sync(0xffffffffu, kk, o);
       // A' <- A' - v wᵀ - w vᵀ  (= H A' H with H = I - 2 v vᵀ)
-      for (int e2 = tid; e2 < m * m; e2 += nt) {
-        const int i = e2 / m, j = e2 % m;
-        A[(c + 1 + i) * ld + c + 1 + j] -= hv[c * ld + i] * wv[j] + wv[i] * hv[c * ld + j];
+      // a warp per row, lanes along it (no index division)
+      for (int i = wid; i < m; i += nw) {
+        const float vi = v[i], wi = 2.f * (pv[i] - kk * vi);
+        float* row = A + (c + 1 + i) * ld + c + 1;
+        for (int j = lane; j < m; j += 32) {
+          const float vj = v[j], wj = 2.f * (pv[j] - kk * vj);
+          row[j] -= vi * wj + wi * vj;
+        }
       }
-    }
-    if (tid == 0) {
-      d[c] = A[c * ld + c];
-      e[c] = skip ? x0 : alpha;
     }
     __syncthreads();
   }
@@ -218,34 +243,57 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
   }
   __syncthreads();
   // 3. inverse iteration: solve (T - lam I) y = x by elimination with guarded pivots
-  //    (thread t keeps its elimination factors in cs row t), normalise; 3 rounds
-  float* cs = work + 5 * n;  // k x n
+  //    (thread t factors T - lam_t I once, its factors in cs and rmv row t), normalise;
+  //    3 rounds. The next step's operands are loaded ahead of the recurrence.
+  float* cs = work + 5 * n;   // k x n: f_i = e_i / m_i
+  float* rmv = cs + k * n;    // k x n: 1 / m_i
   if (tid < kk) {
     const float lt = lam[tid];
     float* f = cs + tid * n;
-    for (int i = 0; i < n; ++i) x[i * k + tid] = 1.f + 0.25f * static_cast<float>((i * 7 + tid * 13) % 11) / 11.f;
-    for (int round = 0; round < 3; ++round) {
-      // forward: m_i = (d_i - lt) - e_{i-1} f_{i-1}, f_i = e_i / m_i, y_i = (x_i - e_{i-1} y_{i-1}) / m_i
-      float yprev = 0.f, fprev = 0.f;
+    float* rm = rmv + tid * n;
+    {
+      float fprev = 0.f;
       for (int i = 0; i < n; ++i) {
         float mi = d[i] - lt - (i > 0 ? e[i - 1] * fprev : 0.f);
         if (fabsf(mi) < pivmin) mi = mi < 0.f ? -pivmin : pivmin;
-        const float rm = 1.f / mi;
-        fprev = i + 1 < n ? e[i] * rm : 0.f;
+        const float r = 1.f / mi;
+        rm[i] = r;
+        fprev = i + 1 < n ? e[i] * r : 0.f;
         f[i] = fprev;
-        yprev = (x[i * k + tid] - (i > 0 ? e[i - 1] * yprev : 0.f)) * rm;
+      }
+    }
+    for (int i = 0; i < n; ++i) x[i * k + tid] = 1.f + 0.25f * static_cast<float>((i * 7 + tid * 13) % 11) / 11.f;
+    for (int round = 0; round < 3; ++round) {
+      // forward: y_i = (x_i - e_{i-1} y_{i-1}) / m_i
+      float yprev = 0.f;
+      float xn = x[tid], rn_ = rm[0], en = 0.f;
+      for (int i = 0; i < n; ++i) {
+        const float xi = xn, ri = rn_, ei = en;
+        if (i + 1 < n) {
+          xn = x[(i + 1) * k + tid];
+          rn_ = rm[i + 1];
+          en = e[i];
+        }
+        yprev = (xi - ei * yprev) * ri;
         x[i * k + tid] = yprev;
       }
       // back: y_i -= f_i y_{i+1}
-      float nrm = 0.f;
-      for (int i = n - 1; i >= 0; --i) {
-        float yi = x[i * k + tid];
-        if (i + 1 < n) yi -= f[i] * x[(i + 1) * k + tid];
+      float nrm = yprev * yprev;
+      float ynext = yprev;
+      float xp = n >= 2 ? x[(n - 2) * k + tid] : 0.f, fp = n >= 2 ? f[n - 2] : 0.f;
+      for (int i = n - 2; i >= 0; --i) {
+        const float xi = xp, fi = fp;
+        if (i > 0) {
+          xp = x[(i - 1) * k + tid];
+          fp = f[i - 1];
+        }
+        const float yi = xi - fi * ynext;
         x[i * k + tid] = yi;
         nrm = fmaf(yi, yi, nrm);
+        ynext = yi;
       }
-      const float rn = nrm > 0.f ? rsqrtf(nrm) : 0.f;
-      for (int i = 0; i < n; ++i) x[i * k + tid] *= rn;
+      const float rs = nrm > 0.f ? rsqrtf(nrm) : 0.f;
+      for (int i = 0; i < n; ++i) x[i * k + tid] *= rs;
     }
   }
   __syncthreads();
@@ -300,44 +348,82 @@ __device__ void top_eigenpairs(float* A, int ld, int n, int k, float* hv, float*
   __syncthreads();
 }
 
-// Solves A X = B in place for SPD A (n x n, row stride n) and B (n x nr): Cholesky
+// Solves A X = B in place for SPD A (n x n, row stride lda) and B (n x nr): Cholesky
 // without the column scaling (after step k the lower triangle holds A[i][k] = L[i][k]·s_k
-// with s_k = L[k][k] = sqrt(A[k][k]); one barrier per step), then right-looking
-// forward and backward substitution. rpiv (n floats) receives 1 / s_k. All threads of
+// with s_k = L[k][k] = sqrt(A[k][k]); one barrier per step), then forward and backward
+// substitution by one warp (lanes across 16 right-hand side columns and two row
+// parities, no block barrier per step). rpiv (n floats) receives 1 / s_k. All threads of
 // the CTA take part.
-__device__ void chol_solve(float* A, int n, float* B, int nr, float* rpiv) {
+__device__ void chol_solve(float* A, int n, int lda, float* B, int nr, float* rpiv) {
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
   for (int k = 0; k < n; ++k) {
-    const float rdk = 1.f / fmaxf(A[k * n + k], 1e-30f);
+    const float rdk = 1.f / fmaxf(A[k * lda + k], 1e-30f);
     for (int i = k + 1 + wid; i < n; i += nw) {  // warps along rows, lanes along columns
-      const float aik = A[i * n + k] * rdk;
-      for (int j = k + 1 + lane; j <= i; j += 32) A[i * n + j] -= aik * A[j * n + k];
+      const float aik = A[i * lda + k] * rdk;
+      for (int j = k + 1 + lane; j <= i; j += 32) A[i * lda + j] -= aik * A[j * lda + k];
     }
     __syncthreads();
   }
-  for (int k = tid; k < n; k += nt) rpiv[k] = 1.f / sqrtf(fmaxf(A[k * n + k], 1e-30f));
+  for (int k = tid; k < n; k += nt) rpiv[k] = 1.f / sqrtf(fmaxf(A[k * lda + k], 1e-30f));
   __syncthreads();
-  // forward  b_i -= (A[i][k] / s_k) (b_k / s_k), i > k;  then y_k = b_k / s_k
-  for (int k = 0; k < n - 1; ++k) {
-    const float r2 = rpiv[k] * rpiv[k];
-    for (int e = tid; e < (n - 1 - k) * nr; e += nt) {
-      const int i = k + 1 + e / nr, c = e % nr;
-      B[i * nr + c] -= A[i * n + k] * B[k * nr + c] * r2;
+  if (wid == 0) {
+    // one warp: lane (c, h) = (l % 16, l / 16) takes right-hand side column c0 + c over
+    // the rows of parity h (consecutive lanes on consecutive words of a row of B); eight
+    // rows loaded before any is stored
+    const int cl = lane & 15, hl = lane >> 4;
+    for (int c0 = 0; c0 < nr; c0 += 16) {
+      const int c = c0 + cl;
+      const bool on = c < nr;
+      // forward  b_i -= (A[i][k] / s_k) (b_k / s_k), i > k;  then y_k = b_k / s_k
+      for (int k = 0; k < n - 1; ++k) {
+        if (on) {
+          const float bk = B[k * nr + c] * (rpiv[k] * rpiv[k]);
+          for (int i0 = k + 1 + hl; i0 < n; i0 += 16) {
+            float bv[8], av[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = i0 + 2 * u;
+              bv[u] = i < n ? B[i * nr + c] : 0.f;
+              av[u] = i < n ? A[i * lda + k] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = i0 + 2 * u;
+              if (i < n) B[i * nr + c] = bv[u] - av[u] * bk;
+            }
+          }
+        }
+        __syncwarp();
+      }
+      if (on)
+        for (int i = hl; i < n; i += 2) B[i * nr + c] *= rpiv[i];
+      __syncwarp();
+      // backward y_i -= (A[k][i] / s_i) (y_k / s_k), i < k;  then x_k = y_k / s_k
+      for (int k = n - 1; k > 0; --k) {
+        if (on) {
+          const float bk = B[k * nr + c] * rpiv[k];
+          for (int i0 = hl; i0 < k; i0 += 16) {
+            float bv[8], av[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = i0 + 2 * u;
+              bv[u] = i < k ? B[i * nr + c] : 0.f;
+              av[u] = i < k ? A[k * lda + i] * rpiv[i] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = i0 + 2 * u;
+              if (i < k) B[i * nr + c] = bv[u] - av[u] * bk;
+            }
+          }
+        }
+        __syncwarp();
+      }
+      if (on)
+        for (int i = hl; i < n; i += 2) B[i * nr + c] *= rpiv[i];
+      __syncwarp();
     }
-    __syncthreads();
   }
-  for (int e = tid; e < n * nr; e += nt) B[e] *= rpiv[e / nr];
-  __syncthreads();
-  // backward y_i -= (A[k][i] / s_i) (y_k / s_k), i < k;  then x_k = y_k / s_k
-  for (int k = n - 1; k > 0; --k) {
-    const float rk_ = rpiv[k];
-    for (int e = tid; e < k * nr; e += nt) {
-      const int i = e / nr, c = e % nr;
-      B[i * nr + c] -= A[k * n + i] * rpiv[i] * B[k * nr + c] * rk_;
-    }
-    __syncthreads();
-  }
-  for (int e = tid; e < n * nr; e += nt) B[e] *= rpiv[e / nr];
   __syncthreads();
 }
 
@@ -358,14 +444,14 @@ __host__ __device__ inline FitPlan fit_plan(int D, int M, int rk) {
   FitPlan p{};
   p.n1 = D + 1;
   p.n = M < D ? M : D;
-  p.ld = p.n + 1;
-  p.ldz = D + 2;
+  p.ld = (p.n + 1) | 1;  // odd: rows on distinct banks
+  p.ldz = D + 3;  // odd: probe rows on distinct banks
   p.ldr = D + 1;
   p.rk = rk;
-  const size_t wa = static_cast<size_t>(2) * p.n * p.ld + static_cast<size_t>(2) * p.n * rk +
+  const size_t wa = static_cast<size_t>(2) * p.n * p.ld + static_cast<size_t>(3) * p.n * rk +
                     static_cast<size_t>(5) * p.n;
-  const size_t wb_primal = static_cast<size_t>(p.n1) * p.n1 + static_cast<size_t>(p.n1) * rk;
-  const size_t wb_dual = M < p.n1 ? static_cast<size_t>(M) * M + static_cast<size_t>(M) * rk +
+  const size_t wb_primal = static_cast<size_t>(p.n1) * (p.n1 | 1) + static_cast<size_t>(p.n1) * rk;
+  const size_t wb_dual = M < p.n1 ? static_cast<size_t>(M) * (M | 1) + static_cast<size_t>(M) * rk +
                                         static_cast<size_t>(p.n1) * rk
                                   : 0;
   const size_t wb = wb_primal > wb_dual ? wb_primal : wb_dual;
@@ -392,7 +478,7 @@ __host__ __device__ inline FitPlan fit_plan(int D, int M, int rk) {
 __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArgs a) {
   extern __shared__ float sm_fit[];
   __shared__ float mu[128], isg[128], red[32];
-  __shared__ float wv[1024];
+  __shared__ float wv[1024], sqw[1024];  // probe weights and their square roots
   __shared__ int sel[128];
   __shared__ float evl[128];  // eigenvalues of the residual Gram matrix, decreasing
   __shared__ float zbar[128], tbar[128];  // weighted probe means of Z and R V_r (dual solve)
@@ -424,7 +510,10 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
     mu[tid] = X[tid] + m1;
     isg[tid] = 1.f / sqrtf(var + 1e-6f);
   }
-  for (int m = tid; m < M; m += nt) wv[m] = w[m];
+  for (int m = tid; m < M; m += nt) {
+    wv[m] = w[m];
+    sqw[m] = sqrtf(w[m]);
+  }
   for (int k = tid; k < 128; k += nt) sel[k] = -1;
   __syncthreads();
   // 2. standardised probe rows Zt = [(x - mu) / sigma, 1] and residuals R = o_probe - x
@@ -483,7 +572,7 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
         const float lam_i = evl[i];
         if (lam_i > 1e-12f * lmax && lam_i > 0.f) {
           float acc = 0.f;
-          for (int m = 0; m < M; ++m) acc = fmaf(sqrtf(wv[m]) * rr[m * ldr + d], V[m * ld + i], acc);
+          for (int m = 0; m < M; ++m) acc = fmaf(sqw[m] * rr[m * ldr + d], V[m * ld + i], acc);
           val = acc / sqrtf(lam_i);
         }
       }
@@ -509,8 +598,9 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
   //     identity), and the intercept row Tbar - zbarᵀ beta.
   float* Xs;
   if (M < n1) {
+    const int ldk = M | 1;       // odd row stride (distinct banks per row)
     float* Kd = W;               // M x M
-    float* Yd = Kd + M * M;      // M x rk: W½ T_c, then the dual solution
+    float* Yd = Kd + M * ldk;    // M x rk: W½ T_c, then the dual solution
     Xs = Yd + M * rk;            // (D+1) x rk
     float sw = 0.f;
     for (int m = tid; m < M; m += nt) sw += wv[m];
@@ -529,11 +619,11 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
     __syncthreads();
     for (int e = tid; e < M * D; e += nt) {  // Uc in place of the probe rows of Z
       const int m = e / D, d = e % D;
-      zt[m * ldz + d] = sqrtf(wv[m]) * (zt[m * ldz + d] - zbar[d]);
+      zt[m * ldz + d] = sqw[m] * (zt[m * ldz + d] - zbar[d]);
     }
     for (int e = tid; e < M * rk; e += nt) {
       const int m = e / rk, k = e % rk;
-      Yd[e] = sqrtf(wv[m]) * (rv[e] - tbar[k]);
+      Yd[e] = sqw[m] * (rv[e] - tbar[k]);
     }
     __syncthreads();
     {
@@ -554,14 +644,14 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
           const int j = ln + 32 * c;
           if (j <= i) {
             const float v = acc[c] + (i == j ? a.lam : 0.f);
-            Kd[i * M + j] = v;
-            Kd[j * M + i] = v;
+            Kd[i * ldk + j] = v;
+            Kd[j * ldk + i] = v;
           }
         }
       }
     }
     __syncthreads();
-    chol_solve(Kd, M, Yd, rk, piv);
+    chol_solve(Kd, M, ldk, Yd, rk, piv);
     for (int e = tid; e < D * rk; e += nt) {  // beta = Ucᵀ Y
       const int d = e / rk, k = e % rk;
       float acc = 0.f;
@@ -576,8 +666,9 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
     }
     __syncthreads();
   } else {
+    const int lda = n1 | 1;    // odd row stride
     float* A = W;              // n1 x n1 (overwrites G, V: no longer needed)
-    float* Bm = W + n1 * n1;   // n1 x rk
+    float* Bm = W + n1 * lda;  // n1 x rk
     Xs = Bm;
     {
       // a warp per row i, lanes along the columns j <= i (at most 5 per lane: n1 <= 129)
@@ -597,8 +688,8 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
           const int j = lane8 + 32 * c;
           if (j <= i) {
             const float v = acc[c] + ((i == j && i < D) ? a.lam : 0.f);
-            A[i * n1 + j] = v;
-            A[j * n1 + i] = v;
+            A[i * lda + j] = v;
+            A[j * lda + i] = v;
           }
         }
       }
@@ -610,7 +701,7 @@ __global__ void __launch_bounds__(kFitThreads, 1) repair_fit_kernel(const FitArg
       Bm[e] = acc;
     }
     __syncthreads();
-    chol_solve(A, n1, Bm, rk, piv);
+    chol_solve(A, n1, lda, Bm, rk, piv);
   }
   // 11. folded factors from X = Bc V_r: P' = diag(1/sigma) X[:D],
   //     c' = X[D] - Σ_i (mu_i / sigma_i) X[i]
@@ -800,7 +891,7 @@ RepairLayout carve_repair(int BH, int D, int M, int rank, void* ws) {
   RepairLayout L{};
   L.psum = cv.take<float>(static_cast<size_t>(BH) * kStatSplit * D);
   L.psq = cv.take<float>(static_cast<size_t>(BH) * kStatSplit * D);
-  L.zt = cv.take<float>(static_cast<size_t>(BH) * M * (D + 2));
+  L.zt = cv.take<float>(static_cast<size_t>(BH) * M * (D + 3));  // row stride ldz of the fit plan
   L.rr = cv.take<float>(static_cast<size_t>(BH) * M * (D + 1));
   L.rv = cv.take<float>(static_cast<size_t>(BH) * M * rank);
   L.vr = cv.take<float>(static_cast<size_t>(BH) * D * rank);
