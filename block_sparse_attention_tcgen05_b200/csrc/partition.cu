@@ -45,15 +45,15 @@ __global__ void __launch_bounds__(256) rcp_key_features_kernel(const T* __restri
                                                                float scale,
                                                                float* __restrict__ feat) {
   extern __shared__ float sm_rcp[];
-  float* qs = sm_rcp;              // rk x D
-  float* ks = qs + rk * D;         // 64 x (D + 1)
+  float* qs = sm_rcp;              // rk x (D + 1): odd row stride, the lanes' samples on distinct banks
+  float* ks = qs + rk * (D + 1);   // 64 x (D + 1)
   const int g = blockIdx.y, b = blockIdx.z, G = Hq / Hkv;
   const int j0 = blockIdx.x * 64;
   for (int e = threadIdx.x; e < rk * D; e += 256) {
     const int s = e / D, d = e % D;
     const int tok = static_cast<int>((static_cast<int64_t>(2 * s + 1) * Sq) / (2 * rk));
     const int h = g * G + s % G;
-    qs[e] = rcp_f(q[((static_cast<int64_t>(b) * Hq + h) * Sq + tok) * D + d]);
+    qs[s * (D + 1) + d] = rcp_f(q[((static_cast<int64_t>(b) * Hq + h) * Sq + tok) * D + d]);
   }
   const int64_t kb = (static_cast<int64_t>(b) * Hkv + g) * Sk;
   for (int e = threadIdx.x; e < 64 * D; e += 256) {
@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(256) rcp_key_features_kernel(const T* __restri
     if (j0 + j >= Sk) continue;
     float acc = 0.f;
 #pragma unroll 8
-    for (int d = 0; d < D; ++d) acc = fmaf(qs[s * D + d], ks[j * (D + 1) + d], acc);
+    for (int d = 0; d < D; ++d) acc = fmaf(qs[s * (D + 1) + d], ks[j * (D + 1) + d], acc);
     feat[(kb + j0 + j) * rk + s] = scale * acc;
   }
 }
@@ -82,36 +82,50 @@ __global__ void kmeans_init_kernel(const float* __restrict__ x, int N, int F, in
 }
 
 // grid (ceil(N / 128), n_problems), 128 threads, one row per thread: the nearest of the
-// C centroids (squared distance, ties to the lower index). Rows are staged feature-major
-// in shared memory, centroids 32 at a time.
+// C centroids (squared distance summed in feature order, ties to the lower index). Rows
+// are staged feature-major in shared memory, centroids 32 at a time as rows of F4 =
+// ceil(F / 4) * 4 floats (zero padded, which adds exact zeros), read four features per
+// broadcast load.
 __global__ void __launch_bounds__(kRcpRows) kmeans_assign_kernel(const float* __restrict__ x,
                                                                  int N, int F, int C,
                                                                  const float* __restrict__ cent,
                                                                  int32_t* __restrict__ label) {
-  extern __shared__ float sm_km[];
-  float* xs = sm_km;                       // F x 128
-  float* cs = xs + F * kRcpRows;           // 32 x F
+  extern __shared__ __align__(16) float sm_km[];
+  const int F4 = (F + 3) / 4 * 4;
+  float* xs = sm_km;                       // F4 x 128
+  float* cs = xs + F4 * kRcpRows;          // 32 x F4
   const int64_t p = blockIdx.y;
   const int i0 = blockIdx.x * kRcpRows, tid = threadIdx.x;
-  for (int e = tid; e < kRcpRows * F; e += kRcpRows) {
-    const int r = e / F, f = e % F;
-    xs[f * kRcpRows + r] = i0 + r < N ? x[(p * N + i0 + r) * F + f] : 0.f;
+  for (int e = tid; e < kRcpRows * F4; e += kRcpRows) {
+    const int r = e / F4, f = e % F4;
+    xs[f * kRcpRows + r] = (i0 + r < N && f < F) ? x[(p * N + i0 + r) * F + f] : 0.f;
   }
   float best = INFINITY;
   int bc = 0;
   for (int c0 = 0; c0 < C; c0 += kRcpCentChunk) {
     const int nc = min(kRcpCentChunk, C - c0);
     __syncthreads();
-    for (int e = tid; e < nc * F; e += kRcpRows) cs[e] = cent[(p * C + c0) * F + e];
+    for (int e = tid; e < kRcpCentChunk * F4; e += kRcpRows) {
+      const int c = e / F4, f = e % F4;
+      cs[e] = (c < nc && f < F) ? cent[(p * C + c0 + c) * F + f] : 0.f;
+    }
     __syncthreads();
     float d[kRcpCentChunk];
 #pragma unroll
     for (int c = 0; c < kRcpCentChunk; ++c) d[c] = 0.f;
-    for (int f = 0; f < F; ++f) {
-      const float xv = xs[f * kRcpRows + tid];
+    for (int f = 0; f < F4; f += 4) {
+      const float x0 = xs[f * kRcpRows + tid], x1 = xs[(f + 1) * kRcpRows + tid];
+      const float x2 = xs[(f + 2) * kRcpRows + tid], x3 = xs[(f + 3) * kRcpRows + tid];
 #pragma unroll
       for (int c = 0; c < kRcpCentChunk; ++c) {
-        const float t = xv - cs[(c < nc ? c : 0) * F + f];
+        const float4 cv = *reinterpret_cast<const float4*>(cs + c * F4 + f);
+        float t = x0 - cv.x;
+        d[c] = fmaf(t, t, d[c]);
+        t = x1 - cv.y;
+        d[c] = fmaf(t, t, d[c]);
+        t = x2 - cv.z;
+        d[c] = fmaf(t, t, d[c]);
+        t = x3 - cv.w;
         d[c] = fmaf(t, t, d[c]);
       }
     }
@@ -125,42 +139,52 @@ __global__ void __launch_bounds__(kRcpRows) kmeans_assign_kernel(const float* __
   if (i0 + tid < N) label[p * N + i0 + tid] = bc;
 }
 
+// grid (n_problems), 1024 threads: stable sort of each problem's labels into member
+// lists (cluster c's rows, in index order, at slot[p][off[p][c] ..]).
+__global__ void __launch_bounds__(1024) kmeans_members_kernel(const int32_t* __restrict__ label, int N,
+                                                              int C, int32_t* slot, int32_t* count,
+                                                              int32_t* off) {
+  extern __shared__ int32_t sm_mem[];
+  const int64_t p = blockIdx.x;
+  LabelSortJob j{};
+  j.labels = label + p * N;
+  j.S = N;
+  j.C = C;
+  j.cluster_pad = 1;
+  j.n_slots = N;
+  j.slot_token = slot + p * N;
+  j.count = count + p * C;
+  j.off = off + p * (C + 1);
+  label_sort_cta(j, sm_mem);
+}
+
 // grid (C, n_problems), 256 threads (thread f holds feature f): the mean of the rows of
-// cluster c, summed in index order; an empty cluster keeps its centroid. With
-// `gather_rows` the rows come from a (n_problems, N, F) source of type T instead of x.
+// cluster c, summed in index order from its member list (eight rows in flight); an
+// empty cluster keeps its centroid. With T != float the rows come from a (n_problems,
+// N, F) source of that type (the key-space centroids).
 template <typename T>
 __global__ void __launch_bounds__(256) kmeans_update_kernel(const T* __restrict__ x, int N, int F,
-                                                            int C, const int32_t* __restrict__ label,
+                                                            int C, const int32_t* __restrict__ slot,
+                                                            const int32_t* __restrict__ count,
+                                                            const int32_t* __restrict__ off,
                                                             float* __restrict__ cent) {
-  __shared__ int members[256];
-  __shared__ int n_members;
   const int c = blockIdx.x, tid = threadIdx.x;
   const int64_t p = blockIdx.y;
-  const int lane = tid & 31, warp = tid >> 5;
-  __shared__ int warp_n[8];
+  const int n = count[p * C + c];
+  if (tid >= F || n == 0) return;
+  const int32_t* mem = slot + p * N + off[p * (C + 1) + c];
+  const T* xp = x + p * N * F + tid;
   float acc = 0.f;
-  int count = 0;
-  for (int i0 = 0; i0 < N; i0 += 256) {
-    const int i = i0 + tid;
-    const bool mine = i < N && label[p * N + i] == c;
-    const unsigned bal = __ballot_sync(0xffffffffu, mine);
-    if (lane == 0) warp_n[warp] = __popc(bal);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < 8; ++w) {
-      if (w < warp) before += warp_n[w];
-      total += warp_n[w];
-    }
-    if (mine) members[before + __popc(bal & ((1u << lane) - 1u))] = i;
-    if (tid == 0) n_members = total;
-    __syncthreads();
-    const int nm = n_members;
-    if (tid < F)
-      for (int m = 0; m < nm; ++m) acc += rcp_f(x[(p * N + members[m]) * F + tid]);
-    count += nm;
-    __syncthreads();
+  int m = 0;
+  for (; m + 8 <= n; m += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = rcp_f(xp[static_cast<int64_t>(mem[m + u]) * F]);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += v[u];
   }
-  if (tid < F && count > 0) cent[(p * C + c) * F + tid] = acc / static_cast<float>(count);
+  for (; m < n; ++m) acc += rcp_f(xp[static_cast<int64_t>(mem[m]) * F]);
+  cent[(p * C + c) * F + tid] = acc / static_cast<float>(n);
 }
 
 // grid (ceil(Sq / 64), Hkv, B), 256 threads: x[b,g,i,:] = (scale q_{h,i} . kbar_{c_t})
@@ -172,15 +196,15 @@ __global__ void __launch_bounds__(256) rcp_query_coords_kernel(const T* __restri
                                                                int rq, float scale,
                                                                float* __restrict__ xq) {
   extern __shared__ float sm_rq[];
-  float* kc = sm_rq;                 // rq x D
-  float* out = kc + rq * D;          // 64 x F
+  float* kc = sm_rq;                 // rq x (D + 1): odd row stride, the lanes' groups on distinct banks
+  float* out = kc + rq * (D + 1);    // 64 x F
   const int g = blockIdx.y, b = blockIdx.z, G = Hq / Hkv, F = rq * G;
   const int i0 = blockIdx.x * 64;
   const int64_t pg = static_cast<int64_t>(b) * Hkv + g;
   for (int e = threadIdx.x; e < rq * D; e += 256) {
     const int t = e / D, d = e % D;
     const int c = static_cast<int>((static_cast<int64_t>(2 * t + 1) * Ck) / (2 * rq));
-    kc[e] = kbar[(pg * Ck + c) * D + d];
+    kc[t * (D + 1) + d] = kbar[(pg * Ck + c) * D + d];
   }
   __syncthreads();
   for (int e = threadIdx.x; e < 64 * F; e += 256) {
@@ -190,7 +214,7 @@ __global__ void __launch_bounds__(256) rcp_query_coords_kernel(const T* __restri
     if (i0 + i < Sq) {
       const T* qrow = q + ((static_cast<int64_t>(b) * Hq + g * G + hh) * Sq + i0 + i) * D;
 #pragma unroll 8
-      for (int d = 0; d < D; ++d) acc = fmaf(rcp_f(qrow[d]), kc[t * D + d], acc);
+      for (int d = 0; d < D; ++d) acc = fmaf(rcp_f(qrow[d]), kc[t * (D + 1) + d], acc);
     }
     out[i * F + f] = scale * acc;
   }
@@ -210,6 +234,7 @@ __global__ void __launch_bounds__(256) rcp_query_coords_kernel(const T* __restri
 namespace {
 struct RcpLayout {
   float *fk, *xq, *kcent, *qcent, *kbar;
+  int32_t *mslot, *mcount, *moff;  // k-means member lists: rows of each cluster, per problem
   size_t bytes;
 };
 RcpLayout carve_rcp(const bsa_shape& s, int Cq, int Ck, int rk, int rq, void* ws) {
@@ -223,6 +248,11 @@ RcpLayout carve_rcp(const bsa_shape& s, int Cq, int Ck, int rk, int rq, void* ws
   L.kcent = cv.take<float>(P * Ck * rk);
   L.qcent = cv.take<float>(P * Cq * rqe * G);
   L.kbar = cv.take<float>(P * Ck * s.D);
+  const size_t Nmax = s.Sq > s.Sk ? s.Sq : s.Sk;
+  const size_t Cmax = Cq > Ck ? Cq : Ck;
+  L.mslot = cv.take<int32_t>(P * Nmax);
+  L.mcount = cv.take<int32_t>(P * Cmax);
+  L.moff = cv.take<int32_t>(P * (Cmax + 1));
   L.bytes = align_up(cv.used, 256);
   return L;
 }
@@ -245,11 +275,23 @@ int validate_rcp(const bsa_shape& s, int Cq, int Ck, int rk, int rq, int iters) 
 }
 
 // Lloyd iterations on (P, N, F) features: init, `iters` rounds, last assignment.
+// Member lists of every cluster (stable sort of each problem's labels).
+int run_members(const int32_t* label, int P, int N, int C, const RcpLayout& L, cudaStream_t st) {
+  const int smem = label_sort_smem(C);
+  cudaError_t e = cudaFuncSetAttribute(kmeans_members_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem > 48 * 1024 ? smem : 48 * 1024);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(kmeans_members)");
+  kmeans_members_kernel<<<P, 1024, smem, st>>>(label, N, C, L.mslot, L.mcount, L.moff);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "kmeans_members_kernel");
+}
+
 int run_kmeans(const float* x, int P, int N, int F, int C, int iters, float* cent,
-               int32_t* label, cudaStream_t st) {
+               int32_t* label, const RcpLayout& L, cudaStream_t st) {
   kmeans_init_kernel<<<dim3(C, P), 128, 0, st>>>(x, N, F, C, cent);
   count_launch();
-  const int smem = (F * kRcpRows + kRcpCentChunk * F) * 4;
+  const int F4 = (F + 3) / 4 * 4;
+  const int smem = (F4 * kRcpRows + kRcpCentChunk * F4) * 4;
   cudaError_t e = cudaFuncSetAttribute(kmeans_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        smem > 48 * 1024 ? smem : 48 * 1024);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(kmeans_assign)");
@@ -258,7 +300,9 @@ int run_kmeans(const float* x, int P, int N, int F, int C, int iters, float* cen
                                                                                         cent, label);
     count_launch();
     if (it == iters) break;
-    kmeans_update_kernel<float><<<dim3(C, P), 256, 0, st>>>(x, N, F, C, label, cent);
+    int rc = run_members(label, P, N, C, L, st);
+    if (rc) return rc;
+    kmeans_update_kernel<float><<<dim3(C, P), 256, 0, st>>>(x, N, F, C, L.mslot, L.mcount, L.moff, cent);
     count_launch();
   }
   return check_cuda(cudaGetLastError(), "k-means kernels");
@@ -274,7 +318,7 @@ int run_rcp(const void* qv, const void* kv, const bsa_shape& s, int Cq, int Ck, 
   const int rqe = rq < Ck ? rq : Ck;
   int rc;
   {
-    const int smem = (rk * D + 64 * (D + 1)) * 4;
+    const int smem = (rk * (D + 1) + 64 * (D + 1)) * 4;
     cudaError_t e = cudaFuncSetAttribute(rcp_key_features_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem > 48 * 1024 ? smem : 48 * 1024);
@@ -283,12 +327,13 @@ int run_rcp(const void* qv, const void* kv, const bsa_shape& s, int Cq, int Ck, 
         q, k, s.Hq, s.Hkv, s.Sq, s.Sk, rk, scale, L.fk);
     count_launch();
   }
-  if ((rc = run_kmeans(L.fk, P, s.Sk, rk, Ck, iters, L.kcent, k_labels, st))) return rc;
+  if ((rc = run_kmeans(L.fk, P, s.Sk, rk, Ck, iters, L.kcent, k_labels, L, st))) return rc;
   // key-group centroids in key space
-  kmeans_update_kernel<T><<<dim3(Ck, P), 256, 0, st>>>(k, s.Sk, D, Ck, k_labels, L.kbar);
+  if ((rc = run_members(k_labels, P, s.Sk, Ck, L, st))) return rc;
+  kmeans_update_kernel<T><<<dim3(Ck, P), 256, 0, st>>>(k, s.Sk, D, Ck, L.mslot, L.mcount, L.moff, L.kbar);
   count_launch();
   {
-    const int smem = (rqe * D + 64 * rqe * G) * 4;
+    const int smem = (rqe * (D + 1) + 64 * rqe * G) * 4;
     cudaError_t e = cudaFuncSetAttribute(rcp_query_coords_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem > 48 * 1024 ? smem : 48 * 1024);
@@ -297,7 +342,7 @@ int run_rcp(const void* qv, const void* kv, const bsa_shape& s, int Cq, int Ck, 
         q, L.kbar, s.Hq, s.Hkv, s.Sq, Ck, rqe, scale, L.xq);
     count_launch();
   }
-  return run_kmeans(L.xq, P, s.Sq, rqe * G, Cq, iters, L.qcent, q_labels, st);
+  return run_kmeans(L.xq, P, s.Sq, rqe * G, Cq, iters, L.qcent, q_labels, L, st);
 }
 }  // namespace
 

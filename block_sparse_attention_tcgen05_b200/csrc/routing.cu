@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
   constexpr int DL = D / 32;              // dims per lane
   constexpr int EPV = 16 / sizeof(T);     // elements per 16-byte vector
   __shared__ __align__(16) float sqt[D][NP];   // probe rows, transposed
+  __shared__ __align__(16) float s_w[NW][32][NP];  // per warp: the 16 weights of each key of a chunk
   __shared__ float s_m[NW][NP], s_z[NW][NP];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -149,29 +150,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
 #pragma unroll
       for (int i = 0; i < DL; ++i) diff[p][i] = 0.f;
     }
-    for (int j0 = 0; j0 < n; j0 += 32) {
-      const int nk = min(32, n - j0);
+    // one 32-key group: chunk maxima, new references, weights and their sums, then the
+    // difference vectors (the lane's dims of each key's value row; a key's 16 weights
+    // come as four broadcast loads)
+    auto group = [&](const float (&l)[NP], int jb, int nk) {
       const bool mine = lane < nk;
-      // 16 logits of this lane's key
-      float l[NP];
-#pragma unroll
-      for (int p = 0; p < NP; ++p) l[p] = 0.f;
-      const T* krow = kbase + static_cast<int64_t>(o + j0 + (mine ? lane : 0)) * D;
-#pragma unroll 2
-      for (int v0 = 0; v0 < D; v0 += EPV) {
-        float kx[EPV];
-        unpack16<T>(__ldg(reinterpret_cast<const uint4*>(krow + v0)), kx);
-#pragma unroll
-        for (int t = 0; t < EPV; ++t) {
-#pragma unroll
-          for (int p4 = 0; p4 < NP; p4 += 4) {
-            const float4 qv = *reinterpret_cast<const float4*>(&sqt[v0 + t][p4]);
-            fma2(l[p4], l[p4 + 1], kx[t], kx[t], qv.x, qv.y, l[p4], l[p4 + 1]);
-            fma2(l[p4 + 2], l[p4 + 3], kx[t], kx[t], qv.z, qv.w, l[p4 + 2], l[p4 + 3]);
-          }
-        }
-      }
-      // chunk maxima, new references, weights and their sums
       float w[NP];
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
@@ -187,14 +170,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
           m[p] = mx;
         }
         w[p] = mine ? __expf(lp - m[p]) : 0.f;
+        s_w[warp][lane][p] = w[p];
         float ws = w[p];
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o2);
         z[p] += ws;
       }
-      // difference vectors: the lane's dims of each key's value row
+      __syncwarp();
       for (int jj = 0; jj < nk; ++jj) {
-        const T* vrow = vbase + static_cast<int64_t>(o + j0 + jj) * D + DL * lane;
+        const T* vrow = vbase + static_cast<int64_t>(o + jb + jj) * D + DL * lane;
         float vx[DL];
         if constexpr (DL == 4) {
           const uint2 u = *reinterpret_cast<const uint2*>(vrow);
@@ -209,14 +193,46 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
           for (int i = 0; i < DL; ++i) vx[i] = route_f(vrow[i]);
         }
 #pragma unroll
-        for (int p = 0; p < NP; p += 2) {
-          const float w0 = __shfl_sync(0xffffffffu, w[p], jj);
-          const float w1 = __shfl_sync(0xffffffffu, w[p + 1], jj);
+        for (int p4 = 0; p4 < NP; p4 += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(&s_w[warp][jj][p4]);
 #pragma unroll
-          for (int i = 0; i < DL; ++i) fma2(diff[p][i], diff[p + 1][i], w0, w1, vx[i], vx[i], diff[p][i],
-                                            diff[p + 1][i]);
+          for (int i = 0; i < DL; ++i) {
+            fma2(diff[p4][i], diff[p4 + 1][i], w4.x, w4.y, vx[i], vx[i], diff[p4][i], diff[p4 + 1][i]);
+            fma2(diff[p4 + 2][i], diff[p4 + 3][i], w4.z, w4.w, vx[i], vx[i], diff[p4 + 2][i],
+                 diff[p4 + 3][i]);
+          }
         }
       }
+      __syncwarp();
+    };
+    // 64 keys at a time: the 16 logits of the lane's two keys (j0 + lane, j0 + 32 + lane),
+    // one broadcast float4 of probe rows feeding both
+    for (int j0 = 0; j0 < n; j0 += 64) {
+      const int nk0 = min(32, n - j0), nk1 = max(0, min(32, n - j0 - 32));
+      float l0[NP], l1[NP];
+#pragma unroll
+      for (int p = 0; p < NP; ++p) l0[p] = l1[p] = 0.f;
+      const T* krow0 = kbase + static_cast<int64_t>(o + j0 + (lane < nk0 ? lane : 0)) * D;
+      const T* krow1 = kbase + static_cast<int64_t>(o + j0 + 32 + (lane < nk1 ? lane : 0) - (nk1 ? 0 : 32)) * D;
+#pragma unroll 2
+      for (int v0 = 0; v0 < D; v0 += EPV) {
+        float k0[EPV], k1[EPV];
+        unpack16<T>(__ldg(reinterpret_cast<const uint4*>(krow0 + v0)), k0);
+        unpack16<T>(__ldg(reinterpret_cast<const uint4*>(krow1 + v0)), k1);
+#pragma unroll
+        for (int t = 0; t < EPV; ++t) {
+#pragma unroll
+          for (int p4 = 0; p4 < NP; p4 += 4) {
+            const float4 qv = *reinterpret_cast<const float4*>(&sqt[v0 + t][p4]);
+            fma2(l0[p4], l0[p4 + 1], k0[t], k0[t], qv.x, qv.y, l0[p4], l0[p4 + 1]);
+            fma2(l0[p4 + 2], l0[p4 + 3], k0[t], k0[t], qv.z, qv.w, l0[p4 + 2], l0[p4 + 3]);
+            fma2(l1[p4], l1[p4 + 1], k1[t], k1[t], qv.x, qv.y, l1[p4], l1[p4 + 1]);
+            fma2(l1[p4 + 2], l1[p4 + 3], k1[t], k1[t], qv.z, qv.w, l1[p4 + 2], l1[p4 + 3]);
+          }
+        }
+      }
+      group(l0, j0, nk0);
+      if (nk1 > 0) group(l1, j0 + 32, nk1);
     }
     // cluster c done: the norm of (difference - centroid term), taken with reference m
     float vbl[DL];

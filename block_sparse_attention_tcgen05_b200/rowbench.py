@@ -159,10 +159,12 @@ def bench_attention(timer, dev, hbm, tc, out):
     _lib.call("bsa_profile_enable", 0)
     kernel_ms = kms.value / max(1, kn.value)
     prep_ms = max(ms - kernel_ms, 1e-6)
-    qkv_bytes = 3 * q.numel() * q.element_size()
-    out.append(row("a4-a7", "labels -> permutation, cluster-major gathers of Q/K/V, centroids, "
-                   "mask bitsets (call minus attention kernel)", prep_ms, 2 * qkv_bytes, "B", "hbm",
-                   hbm))
+    # Q is not copied (the attention kernel gathers its tile's rows by TMA): the bytes
+    # that must cross HBM are one read and one write of K and V
+    kv_bytes = 2 * k.numel() * k.element_size()
+    out.append(row("a4-a7", "key cluster order, label sorts, query tile plan, cluster-major K/V "
+                   "gather, centroids, mask bitsets (call minus attention kernel)", prep_ms,
+                   2 * kv_bytes, "B", "hbm", hbm))
     out.append(row("a8", f"fused compensated attention kernel ({pairs:.3e} executed pairs x 4D)",
                    kernel_ms, pairs * 4 * D, "FLOP", "tensor", tc))
     out.append(row("a4-a8", "whole attention call", ms, pairs * 4 * D, "FLOP", "tensor", tc))
