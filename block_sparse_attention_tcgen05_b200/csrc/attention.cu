@@ -924,7 +924,8 @@ __device__ __forceinline__ uint32_t kept_word(const uint32_t* any, int w, int Wg
 }
 
 __device__ int build_chunk_list(const uint32_t* any, const uint32_t* uni, int g_lo, int g_hi,
-                                int Wg, const uint32_t* cneed, int ncc, uint32_t* list, int lane) {
+                                int Wg, const uint32_t* cneed, int ncc, uint32_t* list, int lane,
+                                int gbase) {
   const int seg0 = 128 * lane;
   int tail = 0;  // trailing kept groups of this lane's segment
   for (int w = 4 * lane + 3; w >= 4 * lane; --w) {
@@ -974,7 +975,7 @@ __device__ int build_chunk_list(const uint32_t* any, const uint32_t* uni, int g_
                                (wu < Wg ? uni[wu] : 0u)) >> su;
           const uint64_t m = (1ull << run) - 1ull;
           const uint32_t uniform = (uw & m) == m ? (1u << 30) : 0u;
-          list[base + k] = uniform | (static_cast<uint32_t>(run - 1) << 16) | static_cast<uint32_t>(g);
+          list[base + k] = uniform | (static_cast<uint32_t>(run - 1) << 16) | static_cast<uint32_t>(g + gbase);
         }
         ++k;
         g += run;
@@ -1069,8 +1070,12 @@ __global__ void __launch_bounds__(160, 2)
   const int tile = blockIdx.x / a.ksplit, split = blockIdx.x % a.ksplit;
   const int h = blockIdx.y, b = blockIdx.z;
   // this CTA's key groups [g_lo, g_hi); the centroid chunks belong to the last split
-  const int g_lo = static_cast<int>((static_cast<int64_t>(a.G) * split) / a.ksplit);
-  const int g_hi = static_cast<int>((static_cast<int64_t>(a.G) * (split + 1)) / a.ksplit);
+  // (ranges start on 32-group words; one range spans at most 4096 groups, the window of
+  // the CTA's bitsets, which start at word wbase)
+  const int g_lo = static_cast<int>((static_cast<int64_t>(a.G) * split) / a.ksplit) & ~31;
+  const int g_hi = split + 1 == a.ksplit ? a.G
+                                         : static_cast<int>((static_cast<int64_t>(a.G) * (split + 1)) / a.ksplit) & ~31;
+  const int wbase = g_lo >> 5;
   const int hkv = h / (a.Hq / a.Hkv);
   const int slice = (a.b_sliced ? b : 0) * a.nh_slices + (a.h_sliced ? h : 0);
   const uint32_t bar0 = smem_u32(bars);
@@ -1108,14 +1113,15 @@ __global__ void __launch_bounds__(160, 2)
   const uint32_t* cb = a.cbits + static_cast<size_t>(slice) * a.Cq * a.Wc;
   for (int w = tid; w < 128; w += blockDim.x) {
     uint32_t any = 0, all = 0;
-    if (w < a.Wg && nd > 0) {
+    const int wa = wbase + w;  // absolute word
+    if (wa < a.Wg && nd > 0) {
       all = 0xffffffffu;
       for (int i = 0; i < nd; ++i) {
-        const uint32_t x = gb[static_cast<size_t>(distinct[i]) * a.Wg + w];
+        const uint32_t x = gb[static_cast<size_t>(distinct[i]) * a.Wg + wa];
         any |= x;
         all &= x;
       }
-      all &= a.gfull[w];
+      all &= a.gfull[wa];
     }
     any_bits[w] = any;
     uni_bits[w] = all & any;
@@ -1131,7 +1137,8 @@ __global__ void __launch_bounds__(160, 2)
   __syncthreads();
   const int ncc = (a.compensate && split == a.ksplit - 1) ? a.Ckpad / 128 : 0;
   if (warp == 1) {
-    const int n = build_chunk_list(any_bits, uni_bits, g_lo, g_hi, a.Wg, cneed, ncc, clist, lane);
+    const int n = build_chunk_list(any_bits, uni_bits, g_lo - 32 * wbase, g_hi - 32 * wbase,
+                                   min(128, a.Wg - wbase), cneed, ncc, clist, lane, 32 * wbase);
     if (lane == 0) *nchunks = n;
   }
   tc_fence_before();
@@ -1709,6 +1716,9 @@ AttnLayout carve(const bsa_shape& s, int Cq, int Ck, void* ws) {
   const int64_t ctas = static_cast<int64_t>(L.Sqpad / 128) * s.Hq * s.B;
   int ks = ctas >= 148 ? 1 : static_cast<int>(296 / ctas);
   ks = std::min(ks, std::min(16, L.G / 8));
+  // one CTA's key range spans at most 4096 groups (its bitset window); longer key
+  // sequences are always split (ranges start on 32-group words)
+  ks = std::max(ks, ceil_div(L.G, 4064));
   L.ksplit = std::max(ks, 1);
   L.part = L.ksplit > 1 ? cv.take<float>(static_cast<size_t>(s.B) * s.Hq * L.ksplit * L.Sqpad * (s.D + 2))
                         : nullptr;
@@ -1746,10 +1756,16 @@ int validate_attention_shape(const bsa_shape& s, int Cq, int Ck) {
   if (s.dtype != BSA_BF16 && s.dtype != BSA_F32) return fail(BSA_ERR_UNSUPPORTED, "dtype %d", s.dtype);
   if (Cq <= 0 || Ck <= 0 || Cq > 16384 || Ck > 16384)
     return fail(BSA_ERR_UNSUPPORTED, "cluster counts Cq=%d Ck=%d outside [1,16384]", Cq, Ck);
-  if (static_cast<int64_t>(s.Sk) + 15LL * Ck > 65536)
-    return fail(BSA_ERR_UNSUPPORTED, "Sk + 15*Ck = %lld exceeds 65536",
-                static_cast<long long>(s.Sk) + 15LL * Ck);
-  if (s.Sq > 65536) return fail(BSA_ERR_UNSUPPORTED, "Sq %d exceeds 65536", s.Sq);
+  // chunk records hold a 16-bit first key group: at most 65536 groups of 16 slots
+  if (static_cast<int64_t>(s.Sk) + 15LL * Ck > (int64_t(1) << 20) - 128)
+    return fail(BSA_ERR_UNSUPPORTED, "Sk + 15*Ck = %lld exceeds %lld",
+                static_cast<long long>(s.Sk) + 15LL * Ck, static_cast<long long>((1 << 20) - 128));
+  // row indices of the query maps, the key maps and the split partials fit 32 bits
+  const int64_t sqpad = (static_cast<int64_t>(s.Sq) + 127) / 128 * 128;
+  const int64_t skpad = (static_cast<int64_t>(s.Sk) + 15LL * Ck + 127) / 128 * 128;
+  if (static_cast<int64_t>(s.B) * s.Hq * sqpad * 16 >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(s.B) * s.Hkv * skpad >= (int64_t(1) << 31))
+    return fail(BSA_ERR_UNSUPPORTED, "B*Hq*Sq or B*Hkv*Sk too large for 32-bit row indices");
   return BSA_OK;
 }
 

@@ -18,6 +18,12 @@
 // tile each row rescales its partials to the global row max and total, and groups of
 // r consecutive rows (r lanes of a warp) add their rows up with shuffles. The strided
 // logit matrix never reaches device memory.
+//
+// Long sequences (more than 2048 strided rows or 256 key blocks, where the per-tile
+// partials no longer fit next to the accumulator) take two passes of the same GEMM: the
+// first keeps each row's running max and sum (online over the tiles) and parks them in
+// the row's own query block of the output (2 r floats of its nb), the second reads them
+// back and writes every tile's normalised block sums directly.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -37,7 +43,9 @@ struct ScoreArgs {
 constexpr int kScoreStages = 3;
 constexpr int kScoreStageBytes = 16384 + 32768;  // Q box (128 x 128 B) + K box (256 x 128 B)
 
-template <int D, int R>
+// MODE 0: one pass (partials in TMEM); 1: row max and sum only; 2: normalised block sums
+// from the first pass's row statistics.
+template <int D, int R, int MODE>
 __global__ void __launch_bounds__(192, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const ScoreArgs a) {
@@ -143,81 +151,157 @@ __global__ void __launch_bounds__(192, 1)
     const int row = quarter * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float scl = a.scale_log2;
-    constexpr int per_tile = 256 / R;  // key blocks per full tile
-    bool ok = true;
-    for (int jt = 0; jt < a.n_tiles; ++jt) {
-      if (!(ok = mbar_wait(ACC_FULL, jt & 1, abort_flag, 45))) break;
-      tc_fence_after();
-      const int ncols = min(256, a.ns - jt * 256);
-      const int npc = ncols / 32;
-      float mx = -INFINITY;  // raw logits; scale > 0 so the max commutes with it
-      for (int p = 0; p < npc; ++p) {
-        float t[32];
-        tmem_ld32(tl + p * 32, t);
-        tmem_wait_ld();
+    if constexpr (MODE == 0) {
+      constexpr int per_tile = 256 / R;  // key blocks per full tile
+      bool ok = true;
+      for (int jt = 0; jt < a.n_tiles; ++jt) {
+        if (!(ok = mbar_wait(ACC_FULL, jt & 1, abort_flag, 45))) break;
+        tc_fence_after();
+        const int ncols = min(256, a.ns - jt * 256);
+        const int npc = ncols / 32;
+        float mx = -INFINITY;  // raw logits; scale > 0 so the max commutes with it
+        for (int p = 0; p < npc; ++p) {
+          float t[32];
+          tmem_ld32(tl + p * 32, t);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, t[c]);
-      }
-      float lsum = 0.f;
-      // partial block sums of this tile, written to TMEM columns 256 + jt*per_tile + ...
-      for (int p = 0; p < npc; ++p) {
-        float t[32];
-        tmem_ld32(tl + p * 32, t);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          t[c] = ex2((t[c] - mx) * scl);
-          lsum += t[c];
+          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, t[c]);
         }
-        // sums over groups of R consecutive columns = one key block each
-        constexpr int G = 32 / R;
-        uint32_t gs[G];
+        float lsum = 0.f;
+        // partial block sums of this tile, written to TMEM columns 256 + jt*per_tile + ...
+        for (int p = 0; p < npc; ++p) {
+          float t[32];
+          tmem_ld32(tl + p * 32, t);
+          tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float acc = 0.f;
+          for (int c = 0; c < 32; ++c) {
+            t[c] = ex2((t[c] - mx) * scl);
+            lsum += t[c];
+          }
+          // sums over groups of R consecutive columns = one key block each
+          constexpr int G = 32 / R;
+          uint32_t gs[G];
 #pragma unroll
-          for (int c = 0; c < R; ++c) acc += t[g * R + c];
-          gs[g] = __float_as_uint(acc);
+          for (int g = 0; g < G; ++g) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < R; ++c) acc += t[g * R + c];
+            gs[g] = __float_as_uint(acc);
+          }
+          tmem_st_n<G>(tl + 256 + jt * per_tile + p * G, gs);
+          tmem_wait_st();
         }
-        tmem_st_n<G>(tl + 256 + jt * per_tile + p * G, gs);
-        tmem_wait_st();
+        mtile[jt * 128 + row] = mx;
+        ltile[jt * 128 + row] = lsum;
+        tc_fence_before();
+        mbar_arrive(ACC_FREE);
       }
-      mtile[jt * 128 + row] = mx;
-      ltile[jt * 128 + row] = lsum;
-      tc_fence_before();
-      mbar_arrive(ACC_FREE);
-    }
-    if (ok && !*abort_flag) {
-      float M = -INFINITY;
-      for (int jt = 0; jt < a.n_tiles; ++jt) M = fmaxf(M, mtile[jt * 128 + row]);
-      float L = 0.f;
-      for (int jt = 0; jt < a.n_tiles; ++jt)
-        L += ltile[jt * 128 + row] * ex2((mtile[jt * 128 + row] - M) * scl);
-      const float inv_rl = 1.f / (L * static_cast<float>(R));
-      // query block of this row and the lane leading its group of r rows
+      if (ok && !*abort_flag) {
+        float M = -INFINITY;
+        for (int jt = 0; jt < a.n_tiles; ++jt) M = fmaxf(M, mtile[jt * 128 + row]);
+        float L = 0.f;
+        for (int jt = 0; jt < a.n_tiles; ++jt)
+          L += ltile[jt * 128 + row] * ex2((mtile[jt * 128 + row] - M) * scl);
+        const float inv_rl = 1.f / (L * static_cast<float>(R));
+        // query block of this row and the lane leading its group of r rows
+        const int qrow_global = itile * 128 + row;
+        const int iblk = qrow_global / R;
+        const bool leader = (qrow_global % R) == 0;
+        float* out = a.scores + ((static_cast<size_t>(b) * a.Hq + h) * a.nb + iblk) * a.nb;
+        for (int jt = 0; jt < a.n_tiles; ++jt) {
+          const float f = ex2((mtile[jt * 128 + row] - M) * scl) * inv_rl;
+          const int ncols = min(256, a.ns - jt * 256);
+          const int nblk = ncols / R;
+          for (int c0 = 0; c0 < nblk; c0 += 32) {
+            float t[32];
+            tmem_ld32(tl + 256 + jt * per_tile + c0, t);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              float v = t[c] * f;
+              // sum over the r rows of the query block (r consecutive lanes, r <= 32)
+#pragma unroll
+              for (int o = 1; o < R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              t[c] = v;
+            }
+            if (leader) {
+              for (int c = 0; c < 32 && c0 + c < nblk; ++c) out[jt * per_tile + c0 + c] = t[c];
+            }
+          }
+        }
+      }
+    } else {
+      // the row's query block and the lane leading its group of r rows; the block row of
+      // the output first holds the r rows' (max, sum) pairs from the first pass
       const int qrow_global = itile * 128 + row;
       const int iblk = qrow_global / R;
       const bool leader = (qrow_global % R) == 0;
       float* out = a.scores + ((static_cast<size_t>(b) * a.Hq + h) * a.nb + iblk) * a.nb;
+      float M = -INFINITY, L = 0.f;
+      if constexpr (MODE == 2) {
+        M = out[2 * (qrow_global % R)];
+        L = out[2 * (qrow_global % R) + 1];
+      }
+      __syncwarp();  // every row of the block has its statistics before the leader writes
+      const float inv_rl = 1.f / (L * static_cast<float>(R));
+      bool ok = true;
       for (int jt = 0; jt < a.n_tiles; ++jt) {
-        const float f = ex2((mtile[jt * 128 + row] - M) * scl) * inv_rl;
+        if (!(ok = mbar_wait(ACC_FULL, jt & 1, abort_flag, 45))) break;
+        tc_fence_after();
         const int ncols = min(256, a.ns - jt * 256);
-        const int nblk = ncols / R;
-        for (int c0 = 0; c0 < nblk; c0 += 32) {
-          float t[32];
-          tmem_ld32(tl + 256 + jt * per_tile + c0, t);
-          tmem_wait_ld();
+        const int npc = ncols / 32;
+        if constexpr (MODE == 1) {
+          float mx = -INFINITY;  // raw logits; scale > 0 so the max commutes with it
+          for (int p = 0; p < npc; ++p) {
+            float t[32];
+            tmem_ld32(tl + p * 32, t);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float v = t[c] * f;
-            // sum over the r rows of the query block (r consecutive lanes, r <= 32)
+            for (int c = 0; c < 32; ++c) mx = fmaxf(mx, t[c]);
+          }
+          if (mx > M) {
+            L *= ex2((M - mx) * scl);
+            M = mx;
+          }
+          for (int p = 0; p < npc; ++p) {
+            float t[32];
+            tmem_ld32(tl + p * 32, t);
+            tmem_wait_ld();
 #pragma unroll
-            for (int o = 1; o < R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            t[c] = v;
+            for (int c = 0; c < 32; ++c) L += ex2((t[c] - M) * scl);
           }
-          if (leader) {
-            for (int c = 0; c < 32 && c0 + c < nblk; ++c) out[jt * per_tile + c0 + c] = t[c];
+        } else {
+          constexpr int G = 32 / R;
+          constexpr int per_tile = 256 / R;
+          for (int p = 0; p < npc; ++p) {
+            float t[32];
+            tmem_ld32(tl + p * 32, t);
+            tmem_wait_ld();
+            float gs[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              float acc = 0.f;
+#pragma unroll
+              for (int c = 0; c < R; ++c) acc += ex2((t[g * R + c] - M) * scl);
+              // sum over the r rows of the query block (r consecutive lanes, r <= 32)
+              float v = acc * inv_rl;
+#pragma unroll
+              for (int o = 1; o < R; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              gs[g] = v;
+            }
+            if (leader) {
+#pragma unroll
+              for (int g = 0; g < G; ++g) out[jt * per_tile + p * G + g] = gs[g];
+            }
           }
+        }
+        tc_fence_before();
+        mbar_arrive(ACC_FREE);
+      }
+      if constexpr (MODE == 1) {
+        if (ok && !*abort_flag) {
+          out[2 * (qrow_global % R)] = M;
+          out[2 * (qrow_global % R) + 1] = L;
         }
       }
     }
@@ -248,8 +332,15 @@ int antidiagonal_block_scores(const void* q, const void* k, const bsa_shape& s, 
   const int ns = N / stride;
   if (ns % 128) return fail(BSA_ERR_UNSUPPORTED, "S/stride (%d) must be a multiple of 128", ns);
   const int nb = N / block;
-  if (ns > 2048 || nb > 256)
-    return fail(BSA_ERR_UNSUPPORTED, "S/stride (%d) > 2048 or S/block (%d) > 256", ns, nb);
+  // one pass while the per-tile partials fit beside the accumulator in TMEM (at most 8
+  // tiles of 256 strided columns, 256 key blocks); two passes beyond, which park each
+  // row's statistics in its query block of the output (2 r floats of nb)
+  const bool one_pass = ns <= 2048 && nb <= 256;
+  if (!one_pass && nb < 2 * r)
+    return fail(BSA_ERR_UNSUPPORTED, "two-pass scoring needs S/block (%d) >= 2 block/stride (%d)", nb,
+                2 * r);
+  if (static_cast<int64_t>(s.B) * s.Hq * ns >= (int64_t(1) << 31))
+    return fail(BSA_ERR_UNSUPPORTED, "B * Hq * S/stride exceeds the TMA row range");
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k)) % 16)
     return fail(BSA_ERR_INVALID_ARG, "q/k must be 16-byte aligned");
 
@@ -274,10 +365,13 @@ int antidiagonal_block_scores(const void* q, const void* k, const bsa_shape& s, 
   a.scale_log2 = sc * 1.4426950408889634f;
   a.scores = scores;
   const int smem = kScoreStages * kScoreStageBytes + 1024 + 2 * 8 * 128 * 4 + 1024;
-  void (*kern)(CUtensorMap, CUtensorMap, ScoreArgs) = nullptr;
-#define BSA_SCORE_CASE(RR)                                          \
-  case RR:                                                          \
-    kern = s.D == 64 ? score_kernel<64, RR> : score_kernel<128, RR>; \
+  using Kern = void (*)(CUtensorMap, CUtensorMap, ScoreArgs);
+  Kern k0 = nullptr, k1 = nullptr, k2 = nullptr;
+#define BSA_SCORE_CASE(RR)                                                        \
+  case RR:                                                                        \
+    k0 = s.D == 64 ? score_kernel<64, RR, 0> : score_kernel<128, RR, 0>;           \
+    k1 = s.D == 64 ? score_kernel<64, RR, 1> : score_kernel<128, RR, 1>;           \
+    k2 = s.D == 64 ? score_kernel<64, RR, 2> : score_kernel<128, RR, 2>;           \
     break;
   switch (r) {
     BSA_SCORE_CASE(1)
@@ -289,13 +383,18 @@ int antidiagonal_block_scores(const void* q, const void* k, const bsa_shape& s, 
     default: return fail(BSA_ERR_UNSUPPORTED, "block/stride = %d", r);
   }
 #undef BSA_SCORE_CASE
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(score_kernel)");
+  const dim3 grid(ns / 128, s.Hq, s.B);
   prof_begin(kProfScoring, st);
-  kern<<<dim3(ns / 128, s.Hq, s.B), 192, smem, st>>>(mq, mk, a);
-  count_launch();
+  for (Kern kern : {one_pass ? k0 : k1, one_pass ? nullptr : k2}) {
+    if (!kern) continue;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(score_kernel)");
+    kern<<<grid, 192, smem, st>>>(mq, mk, a);
+    count_launch();
+    if ((rc = check_cuda(cudaGetLastError(), "score_kernel launch"))) return rc;
+  }
   prof_end(kProfScoring, st);
-  return check_cuda(cudaGetLastError(), "score_kernel launch");
+  return BSA_OK;
 }
 
 }  // namespace bsa

@@ -138,8 +138,9 @@ int bsa_sliding_tile_block_mask(int nT, int nH, int nW, int wt, int wh, int ww, 
  *   P      = row-softmax(logit_scale * A) over all S/s columns
  *   scores[b,h,i,j] = (s/block) * sum over the (block/s)^2 entries of tile (i,j)
  * q: (B,Hq,S,D), k: (B,Hkv,S,D) with shape.Sq == shape.Sk == S; S % block == 0,
- * block % stride == 0, block/stride a power of two <= 32, S/stride a multiple of 128
- * and <= 2048, S/block <= 256; D in {64,128}; BSA_BF16 only (other sizes return
+ * block % stride == 0, block/stride a power of two <= 32, S/stride a multiple of 128;
+ * past S/stride = 2048 or S/block = 256 the GEMM runs twice (row statistics, then block
+ * sums) and S/block >= 2 block/stride is needed; D in {64,128}; BSA_BF16 only (other sizes return
  * BSA_ERR_UNSUPPORTED). logit_scale <= 0 selects 1/sqrt(D).
  *   scores : device float32 (B, Hq, S/block, S/block), written; each row sums to 1.
  * The strided logit matrix is never written to device memory. No workspace.
@@ -183,7 +184,9 @@ int bsa_top_p_block_mask(const float* scores, int B, int H, int Nq, int Nk, cons
  *   workspace: >= bsa_attention_workspace_bytes(shape, Cq, Ck) bytes.
  * Centroids are arithmetic means per (batch, KV head, cluster), computed in fp32 and
  * rounded to the MMA input type. Limits: D in {64,128}; Ck <= 16384; Cq <= 16384;
- * Sk + 15*Ck <= 65536. BSA_F32 inputs are computed with kind::tf32 MMAs.
+ * Sk + 15*Ck <= 2^20 - 128 (key sequences longer than one CTA's window of 4096 key
+ * groups are split into key ranges whose partial results are merged); B*Hq*Sq*16 and
+ * B*Hkv*(Sk + 15*Ck) below 2^31. BSA_F32 inputs are computed with kind::tf32 MMAs.
  */
 size_t bsa_attention_workspace_bytes(bsa_shape shape, int Cq, int Ck);
 int bsa_centroid_compensated_attention(const void* q, const void* k, const void* v,

@@ -80,20 +80,22 @@ def test_host_side_argument_errors(lib):
     st = lib.bsa_centroid_compensated_attention(null, null, null, d96, null, 16, null, 16, null, 0,
                                                 0, 0.0, 1, null, null, 0, null)
     assert st == _lib.BSA_ERR_UNSUPPORTED
-    # empty sequences, and key ranges past the kernel's limit (Sk + 15 Ck <= 65536)
+    # empty sequences, and key ranges past the limit of 16-bit key-group indices
+    # (Sk + 15 Ck <= 2^20 - 128)
     empty = _lib.Shape(1, 2, 2, 0, 1024, 64, _lib.BSA_BF16)
     st = lib.bsa_centroid_compensated_attention(null, null, null, empty, null, 16, null, 16, null,
                                                 0, 0, 0.0, 1, null, null, 0, null)
     assert st == _lib.BSA_ERR_INVALID_ARG
     assert lib.bsa_attention_workspace_bytes(empty, 16, 16) == 0
-    at_max = _lib.Shape(1, 1, 1, 1024, 65536 - 15 * 16, 64, _lib.BSA_BF16)
+    lim = (1 << 20) - 128
+    at_max = _lib.Shape(1, 1, 1, 1024, lim - 15 * 16, 64, _lib.BSA_BF16)
     assert lib.bsa_attention_workspace_bytes(at_max, 16, 16) > 0
-    past = _lib.Shape(1, 1, 1, 1024, 65536 - 15 * 16 + 1, 64, _lib.BSA_BF16)
+    past = _lib.Shape(1, 1, 1, 1024, lim - 15 * 16 + 1, 64, _lib.BSA_BF16)
     assert lib.bsa_attention_workspace_bytes(past, 16, 16) == 0
     st = lib.bsa_centroid_compensated_attention(fake_ptr(), fake_ptr(), fake_ptr(), past, fake_ptr(),
                                                 16, fake_ptr(), 16, fake_ptr(), 0, 0, 0.0, 1,
                                                 fake_ptr(), fake_ptr(), 1 << 30, null)
-    assert st == _lib.BSA_ERR_UNSUPPORTED and "65536" in _lib.detail()
+    assert st == _lib.BSA_ERR_UNSUPPORTED and str(lim) in _lib.detail()
     # scoring: S not a multiple of the block
     fake = ctypes.c_void_p(256)
     s2 = _lib.Shape(1, 1, 1, 1000, 1000, 64, _lib.BSA_BF16)

@@ -207,16 +207,31 @@ def test_unsplit_large_logit_jumps():
         _check(got, ref)
 
 
-def test_key_range_at_the_limit():
-    """Sk + 15 Ck = 65536, the largest key range the kernel takes: 4096 key groups, so
-    the per-tile bitsets and chunk lists are at their capacity. 16 clusters of ~4081
-    tokens (none a multiple of 16), a random mask with the diagonal kept; compensated
-    and hard drop; sampled rows vs the oracle."""
+def test_key_range_at_one_window():
+    """Sk + 15 Ck = 65536: 4096 key groups, the size of one CTA's bitset window, here
+    taken as two key ranges. 16 clusters of ~4081 tokens (none a multiple of 16), a
+    random mask with the diagonal kept; compensated and hard drop; sampled rows vs the
+    oracle."""
     S, C = 65536 - 15 * 16, 16
     q, k, v = wl.gaussian_qkv(1, 1, 1, S, 64, "bf16", seed=41)
     lab = (np.arange(S) * C) // S
     mask = wl.random_cluster_mask(C, 0.4, seed=42)
     rows = np.sort(np.random.default_rng(43).choice(S, 96, replace=False))
+    for comp in (True, False):
+        got = _run(q, k, v, lab, lab, mask, C, C, comp)
+        _check(got[:, :, rows], _ref(q, k, v, lab, lab, mask, C, C, comp, rows=rows))
+
+
+def test_long_key_sequence_split_into_windows():
+    """S = 81920 (a long video latent, past one window of 4096 key groups): the key
+    groups are split into ranges of at most 4096 per CTA, merged afterwards. 20 clusters
+    of 4096 tokens, a random mask with the diagonal kept; compensated and hard drop;
+    sampled rows vs the oracle."""
+    S, C = 81920, 20
+    q, k, v = wl.gaussian_qkv(1, 1, 1, S, 64, "bf16", seed=61)
+    lab = (np.arange(S) * C) // S
+    mask = wl.random_cluster_mask(C, 0.3, seed=62)
+    rows = np.sort(np.random.default_rng(63).choice(S, 96, replace=False))
     for comp in (True, False):
         got = _run(q, k, v, lab, lab, mask, C, C, comp)
         _check(got[:, :, rows], _ref(q, k, v, lab, lab, mask, C, C, comp, rows=rows))

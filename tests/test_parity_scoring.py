@@ -42,6 +42,20 @@ def test_scores_gqa():
     np.testing.assert_allclose(got, ref, atol=SCORE_ATOL, rtol=0)
 
 
+@pytest.mark.parametrize("S,D,stride,block", [
+    (40960, 64, 16, 128),   # 2560 strided rows: more than one pass's 2048
+    (32768, 128, 16, 64),   # 512 key blocks: more than one pass's 256
+])
+def test_scores_two_pass_long_sequences(S, D, stride, block):
+    """Sequences past the one-pass limits take the two-pass path (row statistics first,
+    then normalised block sums); same oracle, same tolerance, rows sum to 1."""
+    q, k, _ = wl.gaussian_qkv(1, 2, 1, S, D, "bf16", seed=S % 97 + D)
+    got = _scores(q, k, block, stride)
+    ref = oracle.antidiagonal_block_scores(q.double().numpy(), k.double().numpy(), block, stride)
+    np.testing.assert_allclose(got, ref, atol=SCORE_ATOL, rtol=0)
+    np.testing.assert_allclose(got.sum(-1), 1.0, atol=1e-4)
+
+
 def test_top_p_kernel_bit_exact_on_identical_scores():
     """Same float32 scores on both sides, decisions in float32 in the same order."""
     g = np.random.default_rng(0)
