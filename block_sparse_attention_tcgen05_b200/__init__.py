@@ -14,6 +14,7 @@ from .ops import (  # noqa: F401
     centroid_compensated_attention,
     device_status,
     error_aware_block_mask,
+    per_kv_head_attention,
     probe_dense_attention,
     probe_budget_block_mask,
     probe_residual_correction,

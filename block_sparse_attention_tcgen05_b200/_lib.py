@@ -50,6 +50,9 @@ SIGNATURES = {
     "bsa_attention_workspace_bytes": (_sz, [Shape, _i, _i]),
     "bsa_centroid_compensated_attention": (
         _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _vp, _i64, _i64, _f, _i, _vp, _vp, _sz, _vp]),
+    "bsa_per_kv_head_attention_workspace_bytes": (_sz, [Shape, _i, _i]),
+    "bsa_per_kv_head_attention": (
+        _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _vp, _i64, _i64, _f, _i, _vp, _vp, _sz, _vp]),
     "bsa_routing_workspace_bytes": (_sz, [Shape, _i, _i]),
     "bsa_error_aware_block_mask": (
         _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _f, _f, _vp, _vp, _vp, _sz, _vp]),

@@ -1634,20 +1634,38 @@ __global__ void __launch_bounds__(256) combine_splits_kernel(const float* __rest
   if (tok < 0) return;
   const size_t bhs = (static_cast<size_t>(b) * Hq + h) * ksplit;
   const float* ml = part + static_cast<size_t>(B) * Hq * ksplit * Sqpad * D;
+  // the splits' maxima and sums read by the lanes side by side (lane s, s + 32, ...)
   float m = -INFINITY;
-  for (int s = 0; s < ksplit; ++s) m = fmaxf(m, ml[((bhs + s) * Sqpad + qrow) * 2]);
+  for (int s = lane; s < ksplit; s += 32) m = fmaxf(m, ml[((bhs + s) * Sqpad + qrow) * 2]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float l = 0.f, acc[D / 32];
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
-  for (int s = 0; s < ksplit; ++s) {
-    const size_t prow = (bhs + s) * Sqpad + qrow;
-    const float ls = ml[prow * 2 + 1];
-    if (!(ls > 0.f)) continue;
-    const float f = exp2f(ml[prow * 2] - m);
-    l = fmaf(ls, f, l);
+  for (int s0 = 0; s0 < ksplit; s0 += 32) {
+    // weight of split s0 + lane (0 for a split that saw no key of this row)
+    float f = 0.f;
+    if (s0 + lane < ksplit) {
+      const size_t prow = (bhs + s0 + lane) * Sqpad + qrow;
+      const float ls = ml[prow * 2 + 1];
+      if (ls > 0.f) {
+        f = exp2f(ml[prow * 2] - m);
+        l = fmaf(ls, f, l);
+      }
+    }
+    const int ns = min(32, ksplit - s0);
+#pragma unroll 4
+    for (int t = 0; t < ns; ++t) {
+      const float ft = __shfl_sync(0xffffffffu, f, t);
+      if (ft > 0.f) {  // a split that saw no key of this row left its partial row unset
+        const size_t prow = (bhs + s0 + t) * Sqpad + qrow;
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(part[prow * D + e * 32 + lane], f, acc[e]);
+        for (int e = 0; e < D / 32; ++e) acc[e] = fmaf(part[prow * D + e * 32 + lane], ft, acc[e]);
+      }
+    }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
   const float inv = l > 0.f ? 1.f / l : 0.f;
   float* orow = out + ((static_cast<size_t>(b) * Hq + h) * Sq + tok) * D;
 #pragma unroll
@@ -1988,4 +2006,56 @@ extern "C" int bsa_centroid_compensated_attention(const void* q, const void* k, 
                                              mask_b_stride, mask_h_stride, scale, compensate, out,
                                              workspace, workspace_bytes, bsa::as_stream(stream),
                                              bsa::kProfAttention, false);
+}
+
+namespace bsa {
+namespace {
+// One (batch, KV head) problem of the per-KV-head call: its G query heads and one KV head.
+bsa_shape kv_head_problem(const bsa_shape& s) {
+  bsa_shape p = s;
+  p.B = 1;
+  p.Hkv = 1;
+  p.Hq = s.Hkv > 0 ? s.Hq / s.Hkv : s.Hq;
+  return p;
+}
+}  // namespace
+}  // namespace bsa
+
+extern "C" size_t bsa_per_kv_head_attention_workspace_bytes(bsa_shape shape, int Cq, int Ck) {
+  if (shape.B <= 0 || shape.Hkv <= 0 || shape.Hq <= 0 || shape.Hq % shape.Hkv) return 0;
+  return bsa_attention_workspace_bytes(bsa::kv_head_problem(shape), Cq, Ck);
+}
+
+extern "C" int bsa_per_kv_head_attention(const void* q, const void* k, const void* v, bsa_shape shape,
+                                         const int32_t* q_labels, int Cq, const int32_t* k_labels,
+                                         int Ck, const uint8_t* block_mask, int64_t mask_b_stride,
+                                         int64_t mask_g_stride, float scale, int compensate, float* out,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  using namespace bsa;
+  if (shape.B <= 0 || shape.Hkv <= 0 || shape.Hq <= 0 || shape.Sq <= 0 || shape.Sk <= 0)
+    return fail(BSA_ERR_INVALID_ARG, "non-positive shape");
+  if (shape.Hq % shape.Hkv)
+    return fail(BSA_ERR_INVALID_ARG, "Hq (%d) not a multiple of Hkv (%d)", shape.Hq, shape.Hkv);
+  if (!q || !k || !v || !q_labels || !k_labels || !block_mask || !out)
+    return fail(BSA_ERR_INVALID_ARG, "null pointer argument");
+  if (mask_b_stride < 0 || mask_g_stride < 0) return fail(BSA_ERR_INVALID_ARG, "negative mask stride");
+  const bsa_shape p = kv_head_problem(shape);
+  const int es = shape.dtype == BSA_F32 ? 4 : 2;
+  const int G = p.Hq;
+  for (int b = 0; b < shape.B; ++b) {
+    for (int g = 0; g < shape.Hkv; ++g) {
+      const int64_t qh = static_cast<int64_t>(b) * shape.Hq + static_cast<int64_t>(g) * G;
+      const int64_t kh = static_cast<int64_t>(b) * shape.Hkv + g;
+      const char* qs = static_cast<const char*>(q) + qh * shape.Sq * shape.D * es;
+      const char* ks = static_cast<const char*>(k) + kh * shape.Sk * shape.D * es;
+      const char* vs = static_cast<const char*>(v) + kh * shape.Sk * shape.D * es;
+      const int rc = centroid_compensated_attention(
+          qs, ks, vs, p, q_labels + kh * shape.Sq, Cq, k_labels + kh * shape.Sk, Ck,
+          block_mask + b * mask_b_stride + g * mask_g_stride, 0, 0, scale, compensate,
+          out + qh * shape.Sq * shape.D, workspace, workspace_bytes, as_stream(stream),
+          kProfAttention, false);
+      if (rc) return rc;
+    }
+  }
+  return BSA_OK;
 }

@@ -175,6 +175,39 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
     return out
 
 
+def per_kv_head_attention(q, k, v, q_labels, k_labels, block_mask, Cq=None, Ck=None, scale=None,
+                          compensate=True, out=None, workspace=None):
+    """The compensated attention with labels per (batch, KV head), as the response-coupled
+    partition produces them: q_labels int32 (B, Hkv, Sq), k_labels int32 (B, Hkv, Sk);
+    block_mask bool/uint8 (Cq,Ck) / (Hkv,Cq,Ck) / (B,Hkv,Cq,Ck), shared by the query
+    heads of a KV head. Returns fp32 (B,Hq,S,D)."""
+    _expect_qkv(q, k, v)
+    B, Hq, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    _expect(q_labels, "q_labels", (torch.int32,), (3,), (B, Hkv, Sq))
+    _expect(k_labels, "k_labels", (torch.int32,), (3,), (B, Hkv, Sk))
+    if out is not None:
+        _expect(out, "out", (torch.float32,), (4,), (B, Hq, Sq, D))
+    _expect_workspace(workspace)
+    Cq = int(block_mask.shape[-2]) if Cq is None else int(Cq)
+    Ck = int(block_mask.shape[-1]) if Ck is None else int(Ck)
+    m, bs, gs = _mask_strides(block_mask, B, Hkv, Cq, Ck)
+    _need_cuda(q, k, v, q_labels, k_labels, m, out, workspace)
+    shape = make_shape(q, k)
+    if out is None:
+        out = torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=q.device)
+    need = _lib.load().bsa_per_kv_head_attention_workspace_bytes(shape, Cq, Ck)
+    if need == 0:
+        raise _lib.BsaError("bsa_per_kv_head_attention_workspace_bytes", _lib.BSA_ERR_UNSUPPORTED,
+                            _lib.detail())
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, q.device)
+    _call_on(q.device, "bsa_per_kv_head_attention", _ptr(q), _ptr(k), _ptr(v), shape, _ptr(q_labels),
+             Cq, _ptr(k_labels), Ck, _ptr(m), bs, gs, float(scale or 0.0), 1 if compensate else 0,
+             _ptr(out), _ptr(workspace), workspace.numel(), _stream(q.device))
+    return out
+
+
 def error_aware_block_mask(q, k, v, q_labels, k_labels, Cq, Ck, density, scale=None,
                            return_err=False, workspace=None):
     """SVG-EAR error-aware routing: uint8 (B, Hq, Cq, Ck) mask of the blocks to compute

@@ -198,6 +198,30 @@ int bsa_centroid_compensated_attention(const void* q, const void* k, const void*
                                        void* stream);
 
 /*
+ * per_kv_head_attention — the same attention with labels of their own per (batch, KV
+ * head): [SPR] (K/V partitions and routes are shared by the query heads of a KV head;
+ * the partition step produces one label set per KV head); [SBC] §Recipe (one
+ * block-sparse call per label set).
+ * For every (b, g) the G = Hq / Hkv query heads g*G .. g*G+G-1 attend to KV head g with
+ * q_labels[b, g], k_labels[b, g] and mask slice (b, g):
+ *   q_labels : device int32 (B, Hkv, Sq), values in [0, Cq).
+ *   k_labels : device int32 (B, Hkv, Sk), values in [0, Ck).
+ *   block_mask : device uint8, element (b, g, a, c) at b*mask_b_stride +
+ *              g*mask_g_stride + a*Ck + c (a stride of 0 broadcasts).
+ *   out      : device float32 (B, Hq, Sq, D), written in original token order.
+ *   workspace: >= bsa_per_kv_head_attention_workspace_bytes(shape, Cq, Ck) bytes, used
+ *              by the (b, g) problems one after another on the stream.
+ * Other arguments, limits and errors as centroid_compensated_attention (the limits apply
+ * to one (b, g) problem: B = Hkv = 1, Hq = G).
+ */
+size_t bsa_per_kv_head_attention_workspace_bytes(bsa_shape shape, int Cq, int Ck);
+int bsa_per_kv_head_attention(const void* q, const void* k, const void* v, bsa_shape shape,
+                              const int32_t* q_labels, int Cq, const int32_t* k_labels, int Ck,
+                              const uint8_t* block_mask, int64_t mask_b_stride,
+                              int64_t mask_g_stride, float scale, int compensate, float* out,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * error_aware_block_mask — SVG-EAR error-aware routing: [SBC] §SVG-EAR — centroid
  * compensation (an error-aware router chooses which blocks to compute exactly) and the
  * SVG-EAR abstract (a lightweight probe estimates each block's compensation error; the

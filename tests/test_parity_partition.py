@@ -109,3 +109,35 @@ def test_partition_drives_per_kv_head_attention():
         assert np.abs(gg - ref).max() <= 2e-2
         assert np.linalg.norm(gg - ref) / np.linalg.norm(ref) <= 5e-3
     assert bsa.device_status()[0] == 0
+
+
+def test_per_kv_head_attention_one_call():
+    """The per-KV-head labels of the partition drive one call that runs every (batch,
+    KV head) problem with its own labels and mask slice: B=2, 6 query heads over 2 KV
+    heads, a mask per (batch, KV head); compensated and hard drop; sampled rows of every
+    head against the oracle."""
+    bsa = _bsa()
+    B, Hq, Hkv, D, C = 2, 6, 2, 64, 24
+    q, k, v, _ = wl.positional_qkv(B, Hq, Hkv, (8, 16, 16), D, ell=(3.0, 6.0, 8.0), amp=2.0,
+                                   dtype="bf16", seed=9)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    ql, kl = bsa.response_coupled_partition(qc, kc, C, C)
+    G, S = Hq // Hkv, q.shape[2]
+    mask = np.random.default_rng(10).random((B, Hkv, C, C)) < 0.3
+    for b in range(B):
+        for g in range(Hkv):
+            np.fill_diagonal(mask[b, g], True)
+    mt = torch.from_numpy(mask.astype(np.uint8)).cuda()
+    rows = np.sort(np.random.default_rng(11).choice(S, 128, replace=False))
+    for comp in (True, False):
+        got = bsa.per_kv_head_attention(qc, kc, vc, ql, kl, mt, Cq=C, Ck=C, compensate=comp).cpu().numpy()
+        for b in range(B):
+            for g in range(Hkv):
+                ref = oracle.centroid_compensated_attention(
+                    q[b:b + 1, g * G:(g + 1) * G].double().numpy(), k[b:b + 1, g:g + 1].double().numpy(),
+                    v[b:b + 1, g:g + 1].double().numpy(), ql[b, g].cpu().numpy(), kl[b, g].cpu().numpy(),
+                    mask[b, g], rows=rows, Cq=C, Ck=C, compensate=comp)
+                gg = got[b:b + 1, g * G:(g + 1) * G][:, :, rows]
+                assert np.abs(gg - ref).max() <= 2e-2
+                assert np.linalg.norm(gg - ref) / np.linalg.norm(ref) <= 5e-3
+    assert bsa.device_status()[0] == 0
