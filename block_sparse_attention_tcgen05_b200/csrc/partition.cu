@@ -81,44 +81,52 @@ __global__ void kmeans_init_kernel(const float* __restrict__ x, int N, int F, in
     cent[(p * C + c) * F + f] = x[(p * N + row) * F + f];
 }
 
-// grid (ceil(N / 128), n_problems), 128 threads, one row per thread: the nearest of the
-// C centroids (squared distance summed in feature order, ties to the lower index). Rows
-// are staged feature-major in shared memory, centroids 32 at a time as rows of F4 =
+// grid (ceil(N / 128), n_problems), 256 threads: the nearest of the C centroids for 128
+// rows (squared distance summed in feature order, ties to the lower index). Rows are
+// staged feature-major in shared memory, centroids 32 at a time as rows of F4 =
 // ceil(F / 4) * 4 floats (zero padded, which adds exact zeros), read four features per
-// broadcast load.
-__global__ void __launch_bounds__(kRcpRows) kmeans_assign_kernel(const float* __restrict__ x,
-                                                                 int N, int F, int C,
-                                                                 const float* __restrict__ cent,
-                                                                 int32_t* __restrict__ label) {
+// broadcast load. Thread t takes row t % 128 against centroid half t / 128 of every
+// chunk (warp-uniform, so every centroid read is a broadcast); the two halves' bests
+// are merged at the end.
+constexpr int kRcpThreads = 2 * kRcpRows;
+__global__ void __launch_bounds__(kRcpThreads) kmeans_assign_kernel(const float* __restrict__ x,
+                                                                    int N, int F, int C,
+                                                                    const float* __restrict__ cent,
+                                                                    int32_t* __restrict__ label) {
   extern __shared__ __align__(16) float sm_km[];
+  constexpr int HC = kRcpCentChunk / 2;   // centroids per half
+  __shared__ float s_best[kRcpRows];
+  __shared__ int s_bc[kRcpRows];
   const int F4 = (F + 3) / 4 * 4;
   float* xs = sm_km;                       // F4 x 128
   float* cs = xs + F4 * kRcpRows;          // 32 x F4
   const int64_t p = blockIdx.y;
   const int i0 = blockIdx.x * kRcpRows, tid = threadIdx.x;
-  for (int e = tid; e < kRcpRows * F4; e += kRcpRows) {
-    const int r = e / F4, f = e % F4;
-    xs[f * kRcpRows + r] = (i0 + r < N && f < F) ? x[(p * N + i0 + r) * F + f] : 0.f;
+  const int r = tid % kRcpRows, half = tid / kRcpRows;
+  for (int e = tid; e < kRcpRows * F4; e += kRcpThreads) {
+    const int rr = e / F4, f = e % F4;
+    xs[f * kRcpRows + rr] = (i0 + rr < N && f < F) ? x[(p * N + i0 + rr) * F + f] : 0.f;
   }
   float best = INFINITY;
-  int bc = 0;
+  int bc = 0x7fffffff;
   for (int c0 = 0; c0 < C; c0 += kRcpCentChunk) {
     const int nc = min(kRcpCentChunk, C - c0);
     __syncthreads();
-    for (int e = tid; e < kRcpCentChunk * F4; e += kRcpRows) {
+    for (int e = tid; e < kRcpCentChunk * F4; e += kRcpThreads) {
       const int c = e / F4, f = e % F4;
       cs[e] = (c < nc && f < F) ? cent[(p * C + c0 + c) * F + f] : 0.f;
     }
     __syncthreads();
-    float d[kRcpCentChunk];
+    const float* ch = cs + half * HC * F4;
+    float d[HC];
 #pragma unroll
-    for (int c = 0; c < kRcpCentChunk; ++c) d[c] = 0.f;
+    for (int c = 0; c < HC; ++c) d[c] = 0.f;
     for (int f = 0; f < F4; f += 4) {
-      const float x0 = xs[f * kRcpRows + tid], x1 = xs[(f + 1) * kRcpRows + tid];
-      const float x2 = xs[(f + 2) * kRcpRows + tid], x3 = xs[(f + 3) * kRcpRows + tid];
+      const float x0 = xs[f * kRcpRows + r], x1 = xs[(f + 1) * kRcpRows + r];
+      const float x2 = xs[(f + 2) * kRcpRows + r], x3 = xs[(f + 3) * kRcpRows + r];
 #pragma unroll
-      for (int c = 0; c < kRcpCentChunk; ++c) {
-        const float4 cv = *reinterpret_cast<const float4*>(cs + c * F4 + f);
+      for (int c = 0; c < HC; ++c) {
+        const float4 cv = *reinterpret_cast<const float4*>(ch + c * F4 + f);
         float t = x0 - cv.x;
         d[c] = fmaf(t, t, d[c]);
         t = x1 - cv.y;
@@ -130,13 +138,25 @@ __global__ void __launch_bounds__(kRcpRows) kmeans_assign_kernel(const float* __
       }
     }
 #pragma unroll
-    for (int c = 0; c < kRcpCentChunk; ++c)
-      if (c < nc && d[c] < best) {
+    for (int c = 0; c < HC; ++c) {
+      const int ci = half * HC + c;
+      if (ci < nc && d[c] < best) {
         best = d[c];
-        bc = c0 + c;
+        bc = c0 + ci;
       }
+    }
   }
-  if (i0 + tid < N) label[p * N + i0 + tid] = bc;
+  if (half == 1) {
+    s_best[r] = best;
+    s_bc[r] = bc;
+  }
+  __syncthreads();
+  if (half == 0 && i0 + r < N) {
+    const float b1 = s_best[r];
+    const int c1 = s_bc[r];
+    if (b1 < best || (b1 == best && c1 < bc)) bc = c1;
+    label[p * N + i0 + r] = bc == 0x7fffffff ? 0 : bc;  // no finite distance: cluster 0
+  }
 }
 
 // grid (n_problems), 1024 threads: stable sort of each problem's labels into member
@@ -296,8 +316,8 @@ int run_kmeans(const float* x, int P, int N, int F, int C, int iters, float* cen
                                        smem > 48 * 1024 ? smem : 48 * 1024);
   if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(kmeans_assign)");
   for (int it = 0; it <= iters; ++it) {
-    kmeans_assign_kernel<<<dim3((N + kRcpRows - 1) / kRcpRows, P), kRcpRows, smem, st>>>(x, N, F, C,
-                                                                                        cent, label);
+    kmeans_assign_kernel<<<dim3((N + kRcpRows - 1) / kRcpRows, P), kRcpThreads, smem, st>>>(x, N, F, C,
+                                                                                           cent, label);
     count_launch();
     if (it == iters) break;
     int rc = run_members(label, P, N, C, L, st);
