@@ -115,6 +115,24 @@ def test_host_side_argument_errors(lib):
     assert lib.bsa_tile_labels(0, 1, 1, 1, 1, 1, fake, None, null) == _lib.BSA_ERR_INVALID_ARG
 
 
+def test_per_kv_head_attention_host_errors(lib):
+    """The per-KV-head call rejects a bad head split and null pointers on the host, and
+    sizes its workspace for one (batch, KV head) problem."""
+    null = ctypes.c_void_p(0)
+    sh = _lib.Shape(2, 6, 2, 4096, 4096, 64, _lib.BSA_BF16)
+    one = _lib.Shape(1, 3, 1, 4096, 4096, 64, _lib.BSA_BF16)
+    assert lib.bsa_per_kv_head_attention_workspace_bytes(sh, 16, 16) == \
+        lib.bsa_attention_workspace_bytes(one, 16, 16) > 0
+    bad = _lib.Shape(1, 5, 2, 4096, 4096, 64, _lib.BSA_BF16)
+    assert lib.bsa_per_kv_head_attention_workspace_bytes(bad, 16, 16) == 0
+    st = lib.bsa_per_kv_head_attention(null, null, null, bad, null, 16, null, 16, null, 0, 0, 0.0, 1,
+                                       null, null, 0, null)
+    assert st == _lib.BSA_ERR_INVALID_ARG
+    st = lib.bsa_per_kv_head_attention(null, null, null, sh, null, 16, null, 16, null, 0, 0, 0.0, 1,
+                                       null, null, 0, null)
+    assert st == _lib.BSA_ERR_INVALID_ARG and "null" in _lib.detail()
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
 

@@ -28,6 +28,19 @@ def _raises(match, fn, *args, **kw):
         fn(*args, **kw)
 
 
+def test_per_kv_head_attention_arguments():
+    q, k, v = _qkv()
+    ql = torch.zeros(B, HKV, S, dtype=torch.int32)
+    mask = torch.ones(HKV, C, C, dtype=torch.uint8)
+    f = bsa.per_kv_head_attention
+    _raises("q_labels: shape", f, q, k, v, torch.zeros(B, H, S, dtype=torch.int32), ql, mask)
+    _raises("k_labels: 1 dimensions", f, q, k, v, ql, _labels(), mask)
+    _raises("k_labels: dtype", f, q, k, v, ql, ql.long(), mask)
+    _raises("block_mask leading dims", f, q, k, v, ql, ql, torch.ones(H, C, C, dtype=torch.uint8))
+    _raises("block_mask trailing dims", f, q, k, v, ql, ql, mask, Cq=C + 1)
+    _raises("CUDA tensors only", f, q, k, v, ql, ql, mask)
+
+
 def test_attention_arguments():
     q, k, v = _qkv()
     lab, mask = _labels(), torch.ones(C, C, dtype=torch.uint8)
