@@ -85,24 +85,25 @@ __global__ void kmeans_init_kernel(const float* __restrict__ x, int N, int F, in
 // rows (squared distance summed in feature order, ties to the lower index). Rows are
 // staged feature-major in shared memory, centroids 32 at a time as rows of F4 =
 // ceil(F / 4) * 4 floats (zero padded, which adds exact zeros), read four features per
-// broadcast load. Thread t takes row t % 128 against centroid half t / 128 of every
-// chunk (warp-uniform, so every centroid read is a broadcast); the two halves' bests
+// broadcast load. Thread t takes row t % 128 against centroid quarter t / 128 of every
+// chunk (warp-uniform, so every centroid read is a broadcast); the four quarters' bests
 // are merged at the end.
-constexpr int kRcpThreads = 2 * kRcpRows;
+constexpr int kRcpGroups = 4;
+constexpr int kRcpThreads = kRcpGroups * kRcpRows;
 __global__ void __launch_bounds__(kRcpThreads) kmeans_assign_kernel(const float* __restrict__ x,
                                                                     int N, int F, int C,
                                                                     const float* __restrict__ cent,
                                                                     int32_t* __restrict__ label) {
   extern __shared__ __align__(16) float sm_km[];
-  constexpr int HC = kRcpCentChunk / 2;   // centroids per half
-  __shared__ float s_best[kRcpRows];
-  __shared__ int s_bc[kRcpRows];
+  constexpr int HC = kRcpCentChunk / kRcpGroups;   // centroids per group
+  __shared__ float s_best[kRcpGroups][kRcpRows];
+  __shared__ int s_bc[kRcpGroups][kRcpRows];
   const int F4 = (F + 3) / 4 * 4;
   float* xs = sm_km;                       // F4 x 128
   float* cs = xs + F4 * kRcpRows;          // 32 x F4
   const int64_t p = blockIdx.y;
   const int i0 = blockIdx.x * kRcpRows, tid = threadIdx.x;
-  const int r = tid % kRcpRows, half = tid / kRcpRows;
+  const int r = tid % kRcpRows, grp = tid / kRcpRows;
   for (int e = tid; e < kRcpRows * F4; e += kRcpThreads) {
     const int rr = e / F4, f = e % F4;
     xs[f * kRcpRows + rr] = (i0 + rr < N && f < F) ? x[(p * N + i0 + rr) * F + f] : 0.f;
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(kRcpThreads) kmeans_assign_kernel(const float*
       cs[e] = (c < nc && f < F) ? cent[(p * C + c0 + c) * F + f] : 0.f;
     }
     __syncthreads();
-    const float* ch = cs + half * HC * F4;
+    const float* ch = cs + grp * HC * F4;
     float d[HC];
 #pragma unroll
     for (int c = 0; c < HC; ++c) d[c] = 0.f;
@@ -139,22 +140,26 @@ __global__ void __launch_bounds__(kRcpThreads) kmeans_assign_kernel(const float*
     }
 #pragma unroll
     for (int c = 0; c < HC; ++c) {
-      const int ci = half * HC + c;
+      const int ci = grp * HC + c;
       if (ci < nc && d[c] < best) {
         best = d[c];
         bc = c0 + ci;
       }
     }
   }
-  if (half == 1) {
-    s_best[r] = best;
-    s_bc[r] = bc;
-  }
+  s_best[grp][r] = best;
+  s_bc[grp][r] = bc;
   __syncthreads();
-  if (half == 0 && i0 + r < N) {
-    const float b1 = s_best[r];
-    const int c1 = s_bc[r];
-    if (b1 < best || (b1 == best && c1 < bc)) bc = c1;
+  if (grp == 0 && i0 + r < N) {
+#pragma unroll
+    for (int g = 1; g < kRcpGroups; ++g) {
+      const float b1 = s_best[g][r];
+      const int c1 = s_bc[g][r];
+      if (b1 < best || (b1 == best && c1 < bc)) {
+        best = b1;
+        bc = c1;
+      }
+    }
     label[p * N + i0 + r] = bc == 0x7fffffff ? 0 : bc;  // no finite distance: cluster 0
   }
 }
@@ -208,35 +213,51 @@ __global__ void __launch_bounds__(256) kmeans_update_kernel(const T* __restrict_
 }
 
 // grid (ceil(Sq / 64), Hkv, B), 256 threads: x[b,g,i,:] = (scale q_{h,i} . kbar_{c_t})
-// over t < rq and the G heads h of KV head g, divided by its norm.
+// over t < rq and the G heads h of KV head g, divided by its norm. The group vectors sit
+// transposed in shared memory (d-major, rq padded to rq4 = ceil(rq / 4) * 4 with zeros),
+// so a thread takes four groups of one (row, head) per query element: one load of q and
+// one broadcast-free float4 of the four groups' components per d.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) rcp_query_coords_kernel(const T* __restrict__ q,
                                                                const float* __restrict__ kbar,
                                                                int Hq, int Hkv, int Sq, int Ck,
                                                                int rq, float scale,
                                                                float* __restrict__ xq) {
-  extern __shared__ float sm_rq[];
-  float* kc = sm_rq;                 // rq x (D + 1): odd row stride, the lanes' groups on distinct banks
-  float* out = kc + rq * (D + 1);    // 64 x F
+  extern __shared__ __align__(16) float sm_rq[];
+  const int rq4 = (rq + 3) / 4 * 4, n4 = rq4 / 4;
+  float* kcT = sm_rq;                // D x rq4
+  float* out = kcT + D * rq4;        // 64 x F
   const int g = blockIdx.y, b = blockIdx.z, G = Hq / Hkv, F = rq * G;
   const int i0 = blockIdx.x * 64;
   const int64_t pg = static_cast<int64_t>(b) * Hkv + g;
-  for (int e = threadIdx.x; e < rq * D; e += 256) {
-    const int t = e / D, d = e % D;
+  for (int e = threadIdx.x; e < D * rq4; e += 256) {
+    const int d = e / rq4, t = e % rq4;
     const int c = static_cast<int>((static_cast<int64_t>(2 * t + 1) * Ck) / (2 * rq));
-    kc[t * (D + 1) + d] = kbar[(pg * Ck + c) * D + d];
+    kcT[e] = t < rq ? kbar[(pg * Ck + c) * D + d] : 0.f;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < 64 * F; e += 256) {
-    const int i = e / F, f = e % F;
-    const int hh = f / rq, t = f % rq;
-    float acc = 0.f;
+  for (int item = threadIdx.x; item < 64 * G * n4; item += 256) {
+    const int g4 = item % n4, rest = item / n4;
+    const int hh = rest % G, i = rest / G;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     if (i0 + i < Sq) {
       const T* qrow = q + ((static_cast<int64_t>(b) * Hq + g * G + hh) * Sq + i0 + i) * D;
 #pragma unroll 8
-      for (int d = 0; d < D; ++d) acc = fmaf(rcp_f(qrow[d]), kc[t * (D + 1) + d], acc);
+      for (int d = 0; d < D; ++d) {
+        const float qv = rcp_f(qrow[d]);
+        const float4 k4 = *reinterpret_cast<const float4*>(kcT + d * rq4 + 4 * g4);
+        a0 = fmaf(qv, k4.x, a0);
+        a1 = fmaf(qv, k4.y, a1);
+        a2 = fmaf(qv, k4.z, a2);
+        a3 = fmaf(qv, k4.w, a3);
+      }
     }
-    out[i * F + f] = scale * acc;
+    const float av[4] = {a0, a1, a2, a3};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int t = 4 * g4 + u;
+      if (t < rq) out[i * F + hh * rq + t] = scale * av[u];
+    }
   }
   __syncthreads();
   // one warp per row: norm, then the normalised row
@@ -353,7 +374,7 @@ int run_rcp(const void* qv, const void* kv, const bsa_shape& s, int Cq, int Ck, 
   kmeans_update_kernel<T><<<dim3(Ck, P), 256, 0, st>>>(k, s.Sk, D, Ck, L.mslot, L.mcount, L.moff, L.kbar);
   count_launch();
   {
-    const int smem = (rqe * (D + 1) + 64 * rqe * G) * 4;
+    const int smem = (D * ((rqe + 3) / 4 * 4) + 64 * rqe * G) * 4;
     cudaError_t e = cudaFuncSetAttribute(rcp_query_coords_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem > 48 * 1024 ? smem : 48 * 1024);
