@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
       for (int p = 0; p < NP; ++p) l0[p] = l1[p] = 0.f;
       const T* krow0 = kbase + static_cast<int64_t>(o + j0 + (lane < nk0 ? lane : 0)) * D;
       const T* krow1 = kbase + static_cast<int64_t>(o + j0 + 32 + (lane < nk1 ? lane : 0) - (nk1 ? 0 : 32)) * D;
-#pragma unroll 2
+#pragma unroll 4
       for (int v0 = 0; v0 < D; v0 += EPV) {
         float k0[EPV], k1[EPV];
         unpack16<T>(__ldg(reinterpret_cast<const uint4*>(krow0 + v0)), k0);
