@@ -25,6 +25,7 @@
 // bits with 64-bit pair counts.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "common.cuh"
@@ -33,26 +34,76 @@
 namespace bsa {
 
 // ---------------------------------------------------------------- cluster means
-// grid (C, H, B), 128 threads: dst[b,h,c,:] = mean of src[b,h,tok,:] over the tokens of
-// cluster c (slots off[c] .. off[c] + count[c] of the sorted order); 0 if empty.
-template <typename T>
-__global__ void __launch_bounds__(128) cluster_mean_kernel(const T* __restrict__ src,
-                                                           const int32_t* __restrict__ sort_token,
-                                                           const int32_t* __restrict__ count,
-                                                           const int32_t* __restrict__ off, int C,
-                                                           int S, int D, int H,
-                                                           float* __restrict__ dst) {
-  const int c = blockIdx.x;
+// grid (C, H, B), 256 threads: mean[b,h,c,:] = mean of src[b,h,tok,:] over the tokens of
+// cluster c (slots off[c] .. off[c] + count[c] of the sorted order; 0 if empty), fp32.
+// With dst, the rows are also copied to dst in cluster-major order (row off[c] + i of
+// the (b, h) slab), so one pass gathers and averages. Each warp takes 32 / VPR rows per
+// pass (VPR 16-byte vectors per row, one per lane) and each thread keeps four rows in
+// flight; the row slots' partial sums meet in shared memory.
+template <typename T, int VPR>
+__global__ void __launch_bounds__(256) gather_mean_kernel(const uint4* __restrict__ src,
+                                                          uint4* __restrict__ dst,
+                                                          const int32_t* __restrict__ sort_token,
+                                                          const int32_t* __restrict__ count,
+                                                          const int32_t* __restrict__ off, int C,
+                                                          int S, int H, float* __restrict__ mean) {
+  constexpr int EPV = 16 / sizeof(T);   // elements per vector
+  constexpr int RPW = 32 / VPR;         // rows per warp pass
+  constexpr int SLOTS = 8 * RPW;        // row slots of the CTA
+  constexpr int D = VPR * EPV;
+  __shared__ float part[SLOTS][D];
+  const int c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t bh = static_cast<int64_t>(blockIdx.z) * H + blockIdx.y;
   const int n = count[c], o = off[c];
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const int tok = sort_token[o + i];
-      acc += static_cast<float>(src[(bh * S + tok) * D + d]);
+  const int slot = warp * RPW + lane / VPR, vi = lane % VPR;
+  float acc[EPV];
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
+  for (int r0 = slot; r0 < n; r0 += 4 * SLOTS) {
+    int tok[4];
+    uint4 u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int rr = r0 + j * SLOTS;
+      tok[j] = rr < n ? __ldg(sort_token + o + rr) : -1;
     }
-    dst[(bh * C + c) * D + d] = n > 0 ? acc / static_cast<float>(n) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (tok[j] >= 0) u[j] = __ldg(src + (bh * S + tok[j]) * VPR + vi);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (tok[j] < 0) continue;
+      float f[EPV];
+      unpack16<T>(u[j], f);
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) acc[e] += f[e];
+      if (dst) dst[(bh * S + o + r0 + j * SLOTS) * VPR + vi] = u[j];
+    }
   }
+#pragma unroll
+  for (int e = 0; e < EPV; ++e) part[slot][vi * EPV + e] = acc[e];
+  __syncthreads();
+  const float inv = n > 0 ? 1.f / static_cast<float>(n) : 0.f;
+  for (int d = tid; d < D; d += 256) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k) t += part[k][d];
+    mean[(bh * C + c) * D + d] = t * inv;
+  }
+}
+
+template <typename T>
+void launch_gather_mean(const void* src, void* dst, const int32_t* tok, const int32_t* cnt,
+                        const int32_t* off, int C, int S, int H, int B, int D, float* mean,
+                        cudaStream_t st) {
+  const dim3 g(C, H, B);
+  const uint4* s4 = static_cast<const uint4*>(src);
+  uint4* d4 = static_cast<uint4*>(dst);
+  const int vpr = D * static_cast<int>(sizeof(T)) / 16;
+  if (vpr == 8) gather_mean_kernel<T, 8><<<g, 256, 0, st>>>(s4, d4, tok, cnt, off, C, S, H, mean);
+  else if (vpr == 16) gather_mean_kernel<T, 16><<<g, 256, 0, st>>>(s4, d4, tok, cnt, off, C, S, H, mean);
+  else gather_mean_kernel<T, 32><<<g, 256, 0, st>>>(s4, d4, tok, cnt, off, C, S, H, mean);
+  count_launch();
 }
 
 // ---------------------------------------------------------------- probe errors
@@ -284,6 +335,548 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
   }
 }
 
+// ---------------------------------------------------------------- probe errors, tensor cores
+// bf16 keys and values. The two sums per (probe, key) of the error above, the logit
+// q̄_a . k_j and the weighted value sum over a cluster's keys, are dense contractions:
+// S = Q̄ Kᵀ over a piece of up to 128 keys of one cluster, then E += P V over the same
+// keys, on tcgen05 with fp32 accumulators in TMEM. Both bf16 operands that are not
+// exact in bf16 are carried as a high and a low bf16 part (x = hi + lo to about 16
+// mantissa bits; keys and values are bf16 already): Q̄ = q̄ scale log2(e) is split once
+// per CTA, the weights w = 2^(s - m) once per piece, and each K-step issues one MMA per
+// part, so logits and sums keep close to fp32 precision.
+//
+// One CTA (one per SM: 512 TMEM columns, ~194 KB of shared memory) takes 128 probes of
+// one head and a range of key clusters (balanced by keys); clusters are cut into pieces
+// of at most 128 keys. 160 threads: warp 0 issues the TMA copies (double-buffered K and
+// V stages) and the MMAs; warps 1..4 hold one probe per thread. TMEM columns: S/P of
+// pieces i even / odd at 0 / 128 (P's high part over S columns 0..63, low part over
+// 64..127), E of clusters k even / odd at 256 / 384. The MMA order is QK(i+1), PV(i),
+// QK(i+2), ..., so the next piece's logits are computed while the softmax threads take
+// the weights of this one. Per cluster the running reference m starts at the centroid
+// logit and follows the largest logit seen (E rescaled in TMEM when a later piece
+// raises it); after the cluster's last piece the softmax threads read E and store
+// || E - n_c 2^(lc - m) v̄_c ||, m and the weight sum z of the cluster (all in log2
+// units), one piece later so that its PV runs meanwhile. route_finish_kernel brings the
+// clusters of a probe to one reference and divides by the dense sum.
+struct RouteTcArgs {
+  int B, Hq, Hkv, S, Cq, Ck, nsplit;
+  float scale_log2;       // scale * log2(e)
+  const float* qbar;      // (B, Hq, Cq, D)
+  const float* lc;        // (B, Hq, Cq, Ck): scale_log2 * q̄_a . k̄_c
+  const float* vbar;      // (B, Hkv, Ck, D)
+  const int32_t* q_count;
+  const int32_t* k_count;
+  const int32_t* k_off;   // Ck + 1 offsets into the cluster-major key rows
+  float* err;             // (B, Hq, Cq, Ck): || E - A || against reference mref
+  float* mref;            // (B, Hq, Cq, Ck)
+  float* zc;              // (B, Hq, Cq, Ck): sum of the cluster's weights against mref
+};
+
+// Pieces of the non-empty clusters in [c, c_hi), in order; k counts the clusters.
+struct RtIter {
+  int c, c_hi, p, nc, off, k;
+  __device__ __forceinline__ void seek(const int32_t* cnt, const int32_t* offs) {
+    while (c < c_hi && (nc = __ldg(cnt + c)) <= 0) ++c;
+    if (c < c_hi) off = __ldg(offs + c);
+  }
+  __device__ __forceinline__ void init(int lo, int hi, const int32_t* cnt, const int32_t* offs) {
+    c = lo;
+    c_hi = hi;
+    p = 0;
+    k = 0;
+    nc = 0;
+    off = 0;
+    seek(cnt, offs);
+  }
+  __device__ __forceinline__ void advance(const int32_t* cnt, const int32_t* offs) {
+    if (++p * 128 >= nc) {
+      p = 0;
+      ++c;
+      ++k;
+      seek(cnt, offs);
+    }
+  }
+  __device__ __forceinline__ bool valid() const { return c < c_hi; }
+  __device__ __forceinline__ int n() const { return min(128, nc - 128 * p); }
+  __device__ __forceinline__ int row() const { return off + 128 * p; }
+  __device__ __forceinline__ bool first() const { return p == 0; }
+  __device__ __forceinline__ bool last() const { return (p + 1) * 128 >= nc; }
+};
+
+enum {
+  RT_QR = 0, RT_KF0, RT_KF1, RT_KE0, RT_KE1, RT_VF0, RT_VF1, RT_VE0, RT_VE1, RT_SF0, RT_SF1,
+  RT_PF0, RT_PF1, RT_OF0, RT_OF1, RT_OE0, RT_OE1, RT_XB0, RT_XB1, RT_XE, RT_DRAIN, RT_NBAR
+};
+
+template <int D>
+struct RouteTcCfg {
+  static constexpr int NATOM = D / 64;        // 128-byte column chunks of a bf16 row
+  static constexpr int TILE = 128 * D * 2;    // one 128-row bf16 operand tile
+  static constexpr int SMEM = 6 * TILE + 1024 + 8192;  // tiles, alignment, barriers + exchange
+};
+
+// First cluster of key-balanced range `split` of nsplit (offsets are non-decreasing).
+__device__ __forceinline__ int route_range_start(const int32_t* off, int Ck, int S, int split,
+                                                 int nsplit) {
+  if (split <= 0) return 0;
+  if (split >= nsplit) return Ck;
+  const int target = static_cast<int>((static_cast<int64_t>(S) * split) / nsplit);
+  int lo = 0, hi = Ck;  // first c with off[c] >= target
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(off + mid) < target) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+template <int D>
+__global__ void __launch_bounds__(288, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const RouteTcArgs a) {
+  using Cfg = RouteTcCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sQh = smem_u32(smem), sQl = sQh + Cfg::TILE;
+  const uint32_t sK = sQh + 2 * Cfg::TILE, sV = sQh + 4 * Cfg::TILE;  // two stages each
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * Cfg::TILE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + RT_NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* never = reinterpret_cast<int*>(tmem_slot + 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x / a.nsplit, split = blockIdx.x % a.nsplit;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hkv = h / (a.Hq / a.Hkv);
+  const int64_t bq = static_cast<int64_t>(b) * a.Hq + h;
+  const int64_t bk = static_cast<int64_t>(b) * a.Hkv + hkv;
+  const int a0 = tile * 128;
+  const int c_lo = route_range_start(a.k_off, a.Ck, a.S, split, a.nsplit);
+  const int c_hi = route_range_start(a.k_off, a.Ck, a.S, split + 1, a.nsplit);
+  const uint32_t bar0 = smem_u32(bars);
+#define RBAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+  if (tid == 0) {
+    for (int i = 0; i < RT_NBAR; ++i)
+      mbar_init(RBAR(i), (i == RT_QR || i == RT_PF0 || i == RT_PF1 || i == RT_OE0 || i == RT_OE1 ||
+                          i == RT_XB0 || i == RT_XB1 || i == RT_XE)
+                             ? 256u
+                             : 1u);
+    *abort_flag = 0;
+    *never = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ control warp: TMA + tcgen05.mma
+    const bool leader = lane == 0;
+    auto wait_all = [&](uint32_t bar, uint32_t parity, int where) -> bool {
+      const bool r = mbar_wait(bar, parity, abort_flag, where);
+      return __all_sync(0xffffffffu, r);
+    };
+    auto commit = [&](uint32_t bar) {
+      if (elect_one()) tc_commit(bar);
+      __syncwarp();
+    };
+    constexpr uint32_t kIdescQK = make_idesc(false, 128, 0, false, false);
+    constexpr uint32_t kIdescPV = make_idesc(false, 128, D, false, true);
+    const uint64_t dQh = smem_desc(sQh, 16, 1024), dQl = smem_desc(sQl, 16, 1024);
+    const int grow0 = static_cast<int>(bk * a.S);
+    int lk0 = 0, lk1 = 0, lv0 = 0, lv1 = 0;  // copies issued into each K / V stage
+    auto load = [&](bool is_v, int stage, int row) {
+      if (leader) {
+        const uint32_t bar = RBAR((is_v ? RT_VF0 : RT_KF0) + stage);
+        const uint32_t dst = (is_v ? sV : sK) + stage * Cfg::TILE;
+        mbar_arrive_expect_tx(bar, Cfg::TILE);
+#pragma unroll
+        for (int cc = 0; cc < Cfg::NATOM; ++cc)
+          tma_load_2d(dst + cc * 16384, is_v ? &tmV : &tmK, bar, cc * 64, grow0 + row);
+      }
+      __syncwarp();
+      if (is_v) (stage ? lv1 : lv0) += 1;
+      else (stage ? lk1 : lk0) += 1;
+    };
+    // S[stage] = Q̄_hi Kᵀ + Q̄_lo Kᵀ over the piece's n16 key columns
+    auto issue_qk = [&](int stage, int n) {
+      const uint32_t n16 = static_cast<uint32_t>((n + 15) & ~15);
+      const uint32_t idesc = kIdescQK | ((n16 >> 3) << 17);
+      const uint64_t dK = smem_desc(sK + stage * Cfg::TILE, 16, 1024);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          mma_ss<false>(tmem + 128 * stage, dQh + off, dK + off, idesc, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          mma_ss<false>(tmem + 128 * stage, dQl + off, dK + off, idesc, 1u);
+        }
+      }
+      __syncwarp();
+    };
+    // E[o] (+)= P_hi V + P_lo V over the piece's keys, 16 per K-step
+    auto issue_pv = [&](int stage, int o, int n, bool first) {
+      const int nst = (n + 15) >> 4;
+      const uint64_t dV = smem_desc(sV + stage * Cfg::TILE, 16384, 1024, kLayoutSW128);
+      const uint32_t tE = tmem + 256 + 128 * o, tP = tmem + 128 * stage;
+      if (elect_one()) {
+        for (int t = 0; t < nst; ++t) {
+          const uint64_t bv = dV + static_cast<uint64_t>((t * 16 * 128) >> 4);
+          mma_ts<false>(tE, tP + 8 * t, bv, kIdescPV, (first && t == 0) ? 0u : 1u);
+          mma_ts<false>(tE, tP + 64 + 8 * t, bv, kIdescPV, 1u);
+        }
+      }
+      __syncwarp();
+    };
+    RtIter it;
+    it.init(c_lo, c_hi, a.k_count, a.k_off);
+    bool ok = true;
+    if (it.valid()) {
+      load(false, 0, it.row());
+      load(true, 0, it.row());
+      RtIter n1 = it;
+      n1.advance(a.k_count, a.k_off);
+      if (n1.valid()) load(false, 1, n1.row());
+      ok = wait_all(RBAR(RT_QR), 0, 40) && wait_all(RBAR(RT_KF0), 0, 41);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, it.n());
+        commit(RBAR(RT_SF0));
+        commit(RBAR(RT_KE0));
+      }
+    }
+    int i = 0;
+    while (ok && it.valid()) {
+      const int s = i & 1, s1 = s ^ 1;
+      RtIter nx = it;
+      nx.advance(a.k_count, a.k_off);
+      if (nx.valid()) {
+        // the next piece's logits go first, so they are ready when this softmax ends
+        if (!(ok = wait_all(RBAR(RT_KF0 + s1), ((i + 1) >> 1) & 1, 42))) break;
+        tc_fence_after();
+        issue_qk(s1, nx.n());
+        commit(RBAR(RT_SF0 + s1));
+        commit(RBAR(RT_KE0 + s1));
+        // K of piece i + 2 as soon as QK(i) has read its stage (it has, or nearly: the
+        // softmax of piece i started from it), a whole softmax ahead of its QK
+        RtIter nn = nx;
+        nn.advance(a.k_count, a.k_off);
+        if (nn.valid()) {
+          if (!(ok = wait_all(RBAR(RT_KE0 + s), (i >> 1) & 1, 47))) break;
+          load(false, s, nn.row());
+        }
+        // V of piece i + 1: its stage was last read by PV(i - 1)
+        if (i >= 1 && !(ok = wait_all(RBAR(RT_VE0 + s1), ((i - 1) >> 1) & 1, 43))) break;
+        load(true, s1, nx.row());
+      }
+      if (!(ok = wait_all(RBAR(RT_PF0 + s), (i >> 1) & 1, 44))) break;
+      // a cluster's first PV overwrites its E buffer: the epilogue of cluster k - 2 is done
+      if (it.first() && it.k >= 2 &&
+          !(ok = wait_all(RBAR(RT_OE0 + (it.k & 1)), ((it.k - 2) >> 1) & 1, 45)))
+        break;
+      if (!(ok = wait_all(RBAR(RT_VF0 + s), (i >> 1) & 1, 46))) break;
+      tc_fence_after();
+      issue_pv(s, it.k & 1, it.n(), it.first());
+      commit(RBAR(RT_VE0 + s));
+      if (it.last()) commit(RBAR(RT_OF0 + (it.k & 1)));
+      it = nx;
+      ++i;
+    }
+    // Before the CTA may exit: every MMA has completed and every issued copy has landed.
+    commit(RBAR(RT_DRAIN));
+    mbar_wait(RBAR(RT_DRAIN), 0, never, 48);
+    if (lk0) mbar_wait(RBAR(RT_KF0), (lk0 - 1) & 1, never, 49);
+    if (lk1) mbar_wait(RBAR(RT_KF1), (lk1 - 1) & 1, never, 49);
+    if (lv0) mbar_wait(RBAR(RT_VF0), (lv0 - 1) & 1, never, 49);
+    if (lv1) mbar_wait(RBAR(RT_VF1), (lv1 - 1) & 1, never, 49);
+  } else {
+    // ------------------------------------------------ softmax / epilogue (256 threads)
+    // Two threads per probe: warps 1..4 take key columns 0..63 of each piece and E's
+    // first half of dims, warps 5..8 columns 64..127 and the second half (warp w reads
+    // TMEM lanes 32*(w%4)..+31). The pair exchanges its piece maxima, and at a cluster's
+    // end its halves of the error and of the weight sum, through shared memory, each
+    // exchange closed by an mbarrier of the 256 threads (bounded waits).
+    constexpr int DH = D / 2;  // E columns per thread
+    const int quarter = warp & 3, hh = (warp - 1) >> 2;
+    const int r = quarter * 32 + lane;
+    const int pa = a0 + r;  // this thread's probe (query cluster)
+    const bool live = pa < a.Cq;
+    const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+    float* xmax = reinterpret_cast<float*>(tmem_slot + 4);   // [2 parity][2 halves][128]
+    float* xe2 = xmax + 2 * 2 * 128;                         // [2 halves][128]
+    float* xz = xe2 + 2 * 128;                               // [2 halves][128]
+    // Q̄ rows, high and low bf16 parts, into the K-major 128-byte-swizzled tiles (each
+    // thread of the pair writes half of the row's 16-byte chunks)
+    {
+      const float* qrow = a.qbar + (bq * a.Cq + (live ? pa : 0)) * D;
+#pragma unroll
+      for (int j = 0; j < Cfg::NATOM * 4; ++j) {
+        const int g = hh * Cfg::NATOM * 4 + j;  // 16-byte chunk of the row (8 elements)
+        const int cc = g >> 3, ch = g & 7;
+        float x[8];
+        if (live) {
+          const float4 u0 = __ldg(reinterpret_cast<const float4*>(qrow + g * 8));
+          const float4 u1 = __ldg(reinterpret_cast<const float4*>(qrow + g * 8 + 4));
+          x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w;
+          x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        }
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = x[2 * e] * a.scale_log2, x1 = x[2 * e + 1] * a.scale_log2;
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+          const float2 hf = __bfloat1622float2(hb);
+          hw[e] = *reinterpret_cast<const uint32_t*>(&hb);
+          lw[e] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+        }
+        const uint32_t off = cc * 16384 + r * 128 + ((ch ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sQh + off), "r"(hw[0]),
+                     "r"(hw[1]), "r"(hw[2]), "r"(hw[3]) : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sQl + off), "r"(lw[0]),
+                     "r"(lw[1]), "r"(lw[2]), "r"(lw[3]) : "memory");
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(RBAR(RT_QR));
+    }
+    const float* lc_row = a.lc + (bq * a.Cq + (live ? pa : 0)) * a.Ck;
+    const int64_t out_row = (bq * a.Cq + (live ? pa : 0)) * a.Ck;
+    bool ok = true;
+    // the cluster whose E is still to be read: ordinal, index, count, m, z, lc
+    bool pend = false;
+    int pk = 0, pc = 0, pn = 0, ne = 0;  // ne: epilogues done
+    float pm = 0.f, pz = 0.f, plc = 0.f;
+    auto epilogue = [&]() -> bool {
+      if (!mbar_wait(RBAR(RT_OF0 + (pk & 1)), (pk >> 1) & 1, abort_flag, 50)) return false;
+      tc_fence_after();
+      const float wc = static_cast<float>(pn) * ex2(plc - pm);
+      const float* vb = a.vbar + (bk * a.Ck + pc) * D + hh * DH;
+      const uint32_t tE = tmem + lanes + 256 + 128 * (pk & 1) + hh * DH;
+      float e2a = 0.f, e2b = 0.f;
+#pragma unroll
+      for (int q = 0; q < DH / 32; ++q) {
+        float o[32];
+        tmem_ld32(tE + 32 * q, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 v4 = __ldg(reinterpret_cast<const float4*>(vb + 32 * q + 4 * c4));
+          const float d0 = fmaf(-wc, v4.x, o[4 * c4]), d1 = fmaf(-wc, v4.y, o[4 * c4 + 1]);
+          const float d2 = fmaf(-wc, v4.z, o[4 * c4 + 2]), d3 = fmaf(-wc, v4.w, o[4 * c4 + 3]);
+          e2a = fmaf(d0, d0, fmaf(d1, d1, e2a));
+          e2b = fmaf(d2, d2, fmaf(d3, d3, e2b));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(RBAR(RT_OE0 + (pk & 1)));
+      xe2[hh * 128 + r] = e2a + e2b;
+      xz[hh * 128 + r] = pz;
+      mbar_arrive(RBAR(RT_XE));
+      if (!mbar_wait(RBAR(RT_XE), ne & 1, abort_flag, 53)) return false;
+      ++ne;
+      if (live && hh == 0) {
+        a.err[out_row + pc] = sqrtf(xe2[r] + xe2[128 + r]);
+        a.mref[out_row + pc] = pm;
+        a.zc[out_row + pc] = xz[r] + xz[128 + r];
+      }
+      pend = false;
+      return true;
+    };
+    RtIter it;
+    it.init(c_lo, c_hi, a.k_count, a.k_off);
+    float m = 0.f, z = 0.f, lc2 = 0.f;
+    int i = 0;
+#pragma unroll 1
+    while (it.valid()) {
+      const int s = i & 1;
+      const int nh = min(64, it.n() - 64 * hh);  // this thread's key columns (may be <= 0)
+      if (it.first()) {
+        lc2 = live ? __ldg(lc_row + it.c) : 0.f;
+        m = lc2;
+        z = 0.f;
+      }
+      if (!(ok = mbar_wait(RBAR(RT_SF0 + s), (i >> 1) & 1, abort_flag, 51))) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + lanes + 128 * s;
+      float v[2][32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        if (32 * q < nh) tmem_ld32(tS + 64 * hh + 32 * q, v[q]);
+      tmem_wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          v[q][c] = 32 * q + c < nh ? v[q][c] : -INFINITY;
+          mx = fmaxf(mx, v[q][c]);
+        }
+      // (the exchange also orders both threads' S loads before either's P stores, which
+      // overlap the partner's S columns)
+      xmax[(s * 2 + hh) * 128 + r] = mx;
+      tc_fence_before();
+      mbar_arrive(RBAR(RT_XB0 + s));
+      if (!(ok = mbar_wait(RBAR(RT_XB0 + s), (i >> 1) & 1, abort_flag, 54))) break;
+      tc_fence_after();
+      mx = fmaxf(mx, xmax[(s * 2 + (hh ^ 1)) * 128 + r]);
+      const bool need = mx > m;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m - mx);
+        z *= alpha;
+        m = mx;
+      }
+      if (!it.first() && __any_sync(0xffffffffu, need)) {
+        // E holds this cluster's earlier pieces against the old reference: wait for
+        // PV(i - 1), then scale this thread's half of it
+        if (!(ok = mbar_wait(RBAR(RT_VE0 + (s ^ 1)), ((i - 1) >> 1) & 1, abort_flag, 52))) break;
+        tc_fence_after();
+        const uint32_t tE = tmem + lanes + 256 + 128 * (it.k & 1) + hh * DH;
+#pragma unroll 1
+        for (int q = 0; q < DH / 32; ++q) {
+          float o[32];
+          tmem_ld32(tE + 32 * q, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] *= alpha;
+          tmem_st32(tE + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(o));
+        }
+      }
+      // weights, their sum, and the high / low bf16 parts over S
+      float za = 0.f, zb = 0.f;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (32 * q < nh) {
+          uint32_t hw[16], lw[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float w0 = ex2(v[q][2 * e] - m), w1 = ex2(v[q][2 * e + 1] - m);
+            za += w0;
+            zb += w1;
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(w0, w1);
+            const float2 hf = __bfloat1622float2(hb);
+            hw[e] = *reinterpret_cast<const uint32_t*>(&hb);
+            lw[e] = pack_bf16x2(w0 - hf.x, w1 - hf.y);
+          }
+          tmem_st16(tS + 32 * hh + 16 * q, hw);
+          tmem_st16(tS + 64 + 32 * hh + 16 * q, lw);
+        }
+      }
+      z += za + zb;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(RBAR(RT_PF0 + s));
+      // the previous cluster's E: its last PV was issued before this piece's
+      if (pend && !(ok = epilogue())) break;
+      if (it.last()) {
+        pend = true;
+        pk = it.k;
+        pc = it.c;
+        pn = it.nc;
+        pm = m;
+        pz = z;
+        plc = lc2;
+      }
+      it.advance(a.k_count, a.k_off);
+      ++i;
+    }
+    if (ok && pend) epilogue();
+  }
+#undef RBAR
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// grid (ceil(Cq / 32), Hq, B), 256 threads: lc[b,h,a,c] = scale_log2 * q̄_a . k̄_c (fp32)
+// for 32 probes a per CTA; thread c streams k̄_c once (float4) against the 32 probe rows
+// held in shared memory (broadcast reads).
+constexpr int kLcProbes = 32;
+template <int D>
+__global__ void __launch_bounds__(256) centroid_logit_kernel(const float* __restrict__ qbar,
+                                                             const float* __restrict__ kbar,
+                                                             int Hq, int Hkv, int Cq, int Ck,
+                                                             float scale_log2,
+                                                             float* __restrict__ lc) {
+  __shared__ __align__(16) float qa[kLcProbes][D];
+  const int a0 = blockIdx.x * kLcProbes, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int hkv = h / (Hq / Hkv);
+  const int64_t bq = static_cast<int64_t>(b) * Hq + h;
+  const int64_t bk = static_cast<int64_t>(b) * Hkv + hkv;
+  const int np = min(kLcProbes, Cq - a0);
+  for (int e = tid; e < kLcProbes * D; e += 256) {
+    const int p = e / D, d = e % D;
+    qa[p][d] = p < np ? qbar[(bq * Cq + a0 + p) * D + d] : 0.f;
+  }
+  __syncthreads();
+  for (int c = tid; c < Ck; c += 256) {
+    const float4* kc = reinterpret_cast<const float4*>(kbar + (bk * Ck + c) * D);
+    float acc[kLcProbes];
+#pragma unroll
+    for (int p = 0; p < kLcProbes; ++p) acc[p] = 0.f;
+#pragma unroll 2
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      const float4 k4 = __ldg(kc + d4);
+#pragma unroll
+      for (int p = 0; p < kLcProbes; ++p) {
+        const float4 q4 = *reinterpret_cast<const float4*>(&qa[p][4 * d4]);
+        acc[p] = fmaf(q4.x, k4.x, fmaf(q4.y, k4.y, fmaf(q4.z, k4.z, fmaf(q4.w, k4.w, acc[p]))));
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < kLcProbes; ++p)
+      if (p < np) lc[(bq * Cq + a0 + p) * Ck + c] = scale_log2 * acc[p];
+  }
+}
+
+// One warp per (batch, head, probe) row: M = max_c mref, Z = sum_c zc 2^(mref - M) over
+// the non-empty key clusters; err <- err 2^(mref - M) / Z (0 for an empty probe or key
+// cluster, or Z = 0).
+__global__ void __launch_bounds__(256) route_finish_kernel(const int32_t* __restrict__ q_count,
+                                                           const int32_t* __restrict__ k_count,
+                                                           int Cq, int Ck, int64_t rows,
+                                                           const float* __restrict__ mref,
+                                                           const float* __restrict__ zc,
+                                                           float* __restrict__ err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int pa = static_cast<int>(row % Cq);
+  const float* mr = mref + row * Ck;
+  const float* zr = zc + row * Ck;
+  float* er = err + row * Ck;
+  float M = -INFINITY;
+  for (int c = lane; c < Ck; c += 32)
+    if (__ldg(k_count + c) > 0) M = fmaxf(M, mr[c]);
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float Z = 0.f;
+  if (M > -INFINITY)
+    for (int c = lane; c < Ck; c += 32)
+      if (__ldg(k_count + c) > 0) Z += zr[c] * ex2(mr[c] - M);
+  for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+  const bool qok = __ldg(q_count + pa) > 0 && Z > 0.f;
+  const float invZ = qok ? 1.f / Z : 0.f;
+  for (int c = lane; c < Ck; c += 32) {
+    const bool ok = qok && __ldg(k_count + c) > 0;
+    er[c] = ok ? er[c] * ex2(mr[c] - M) * invZ : 0.f;
+  }
+}
+
 // ---------------------------------------------------------------- budgeted selection
 // One CTA (1024 threads) per (batch, head). Keys are the bit patterns of the
 // non-negative float ratios err / n_c (monotone in the value); invalid blocks (an
@@ -470,7 +1063,7 @@ __global__ void __launch_bounds__(128) centroid_mass_kernel(const RouteArgs a,
 namespace {
 struct RouteLayout {
   int32_t *q_tok, *q_count, *q_off, *k_tok, *k_count, *k_off;
-  float *qbar, *kbar, *vbar, *err, *mref;
+  float *qbar, *kbar, *vbar, *err, *mref, *lc, *zc;
   void *kp, *vp;  // keys and values in cluster-major order
   size_t bytes;
 };
@@ -488,6 +1081,8 @@ RouteLayout carve_route(const bsa_shape& s, int Cq, int Ck, void* ws) {
   L.vbar = cv.take<float>(static_cast<size_t>(s.B) * s.Hkv * Ck * s.D);
   L.err = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
   L.mref = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
+  L.lc = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
+  L.zc = cv.take<float>(static_cast<size_t>(s.B) * s.Hq * Cq * Ck);
   const int es = s.dtype == BSA_F32 ? 4 : 2;
   L.kp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * s.Sk * s.D * es);
   L.vp = cv.take<uint8_t>(static_cast<size_t>(s.B) * s.Hkv * s.Sk * s.D * es);
@@ -506,7 +1101,78 @@ int validate_route(const bsa_shape& s, int Cq, int Ck) {
   if (static_cast<int64_t>(Cq) * Ck > (int64_t(1) << 24))
     return fail(BSA_ERR_UNSUPPORTED, "Cq * Ck = %lld blocks per head exceeds 2^24",
                 static_cast<long long>(Cq) * Ck);
+  if (static_cast<int64_t>(s.B) * s.Hkv * s.Sk >= (int64_t(1) << 31))
+    return fail(BSA_ERR_UNSUPPORTED, "B * Hkv * Sk = %lld key rows exceeds 2^31 - 1",
+                static_cast<long long>(s.B) * s.Hkv * s.Sk);
   return BSA_OK;
+}
+
+// Probe errors of bf16 keys and values on the tensor cores: centroid logits, the probe
+// kernel over key-balanced cluster ranges, and the common-reference normalisation.
+template <int D>
+int launch_route_tc(const RouteLayout& L, const bsa_shape& s, int Cq, int Ck, float scale,
+                    float* err, cudaStream_t st) {
+  int rc;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  centroid_logit_kernel<D><<<dim3((Cq + kLcProbes - 1) / kLcProbes, s.Hq, s.B), 256, 0, st>>>(
+      L.qbar, L.kbar, s.Hq, s.Hkv, Cq, Ck, scale_log2, L.lc);
+  count_launch();
+  if ((rc = check_cuda(cudaGetLastError(), "centroid_logit_kernel"))) return rc;
+  CUtensorMap mk, mv;
+  const uint64_t rows = static_cast<uint64_t>(s.B) * s.Hkv * s.Sk;
+  if ((rc = make_tmap_2d(&mk, L.kp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, s.D, 128, 64)) ||
+      (rc = make_tmap_2d(&mv, L.vp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, s.D, 128, 64)))
+    return rc;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // one CTA per SM: split the key clusters so that the grid fills whole waves best
+  const int tiles = (Cq + 127) / 128;
+  const int64_t units = static_cast<int64_t>(tiles) * s.Hq * s.B;
+  int nsplit = 1;
+  double best = -1.0;
+  const int lo = static_cast<int>(std::max<int64_t>(1, (2 * sms + units - 1) / units));
+  for (int n = lo; n <= 2 * lo && n <= Ck; ++n) {
+    const int64_t ctas = units * n;
+    const double fill = static_cast<double>(ctas) / (static_cast<double>((ctas + sms - 1) / sms) * sms);
+    if (fill > best + 1e-9) {
+      best = fill;
+      nsplit = n;
+    }
+  }
+  if (nsplit > Ck) nsplit = Ck;
+  if (units * nsplit > 0x7fffffffLL || static_cast<int64_t>(tiles) * nsplit > 0x7fffffffLL)
+    return fail(BSA_ERR_UNSUPPORTED, "routing grid too large");
+  RouteTcArgs ta{};
+  ta.B = s.B;
+  ta.Hq = s.Hq;
+  ta.Hkv = s.Hkv;
+  ta.S = s.Sk;
+  ta.Cq = Cq;
+  ta.Ck = Ck;
+  ta.nsplit = nsplit;
+  ta.scale_log2 = scale_log2;
+  ta.qbar = L.qbar;
+  ta.lc = L.lc;
+  ta.vbar = L.vbar;
+  ta.q_count = L.q_count;
+  ta.k_count = L.k_count;
+  ta.k_off = L.k_off;
+  ta.err = err;
+  ta.mref = L.mref;
+  ta.zc = L.zc;
+  auto kern = route_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       RouteTcCfg<D>::SMEM);
+  if (e != cudaSuccess) return check_cuda(e, "cudaFuncSetAttribute(route_tc_kernel)");
+  kern<<<dim3(tiles * nsplit, s.Hq, s.B), 288, RouteTcCfg<D>::SMEM, st>>>(mk, mv, ta);
+  count_launch();
+  if ((rc = check_cuda(cudaGetLastError(), "route_tc_kernel"))) return rc;
+  const int64_t nrows = static_cast<int64_t>(s.B) * s.Hq * Cq;
+  route_finish_kernel<<<static_cast<unsigned>((nrows + 7) / 8), 256, 0, st>>>(
+      L.q_count, L.k_count, Cq, Ck, nrows, L.mref, L.zc, err);
+  count_launch();
+  return check_cuda(cudaGetLastError(), "route_finish_kernel");
 }
 
 template <typename T, int D>
@@ -569,28 +1235,28 @@ int route_prologue(const void* q, const void* k, const void* v, const bsa_shape&
                           nullptr, nullptr, 0, nullptr, 0, nullptr};
     if ((rc = launch_label_sorts(jk, &jq, st))) return rc;
   }
-  // 2. cluster means of Q (probes), K and V (centroids), fp32
+  // 2. cluster means of Q (probes), K and V (centroids), fp32; for the probe errors K and
+  // V are gathered into cluster-major order in the same pass
   const bool with_v = M < 0;
   if (s.dtype == BSA_F32) {
-    cluster_mean_kernel<float><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(
-        static_cast<const float*>(q), L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.D, s.Hq, L.qbar);
-    cluster_mean_kernel<float><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
-        static_cast<const float*>(k), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.kbar);
+    launch_gather_mean<float>(q, nullptr, L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.Hq, s.B, s.D,
+                              L.qbar, st);
+    launch_gather_mean<float>(k, with_v ? L.kp : nullptr, L.k_tok, L.k_count, L.k_off, Ck, s.Sk,
+                              s.Hkv, s.B, s.D, L.kbar, st);
     if (with_v)
-      cluster_mean_kernel<float><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
-          static_cast<const float*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
+      launch_gather_mean<float>(v, L.vp, L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.Hkv, s.B, s.D,
+                                L.vbar, st);
   } else {
     using bf = __nv_bfloat16;
-    cluster_mean_kernel<bf><<<dim3(Cq, s.Hq, s.B), 128, 0, st>>>(
-        static_cast<const bf*>(q), L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.D, s.Hq, L.qbar);
-    cluster_mean_kernel<bf><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
-        static_cast<const bf*>(k), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.kbar);
+    launch_gather_mean<bf>(q, nullptr, L.q_tok, L.q_count, L.q_off, Cq, s.Sq, s.Hq, s.B, s.D,
+                           L.qbar, st);
+    launch_gather_mean<bf>(k, with_v ? L.kp : nullptr, L.k_tok, L.k_count, L.k_off, Ck, s.Sk,
+                           s.Hkv, s.B, s.D, L.kbar, st);
     if (with_v)
-      cluster_mean_kernel<bf><<<dim3(Ck, s.Hkv, s.B), 128, 0, st>>>(
-          static_cast<const bf*>(v), L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.D, s.Hkv, L.vbar);
+      launch_gather_mean<bf>(v, L.vp, L.k_tok, L.k_count, L.k_off, Ck, s.Sk, s.Hkv, s.B, s.D,
+                             L.vbar, st);
   }
-  for (int i = 0; i < (with_v ? 3 : 2); ++i) count_launch();
-  if ((rc = check_cuda(cudaGetLastError(), "cluster_mean_kernel"))) return rc;
+  if ((rc = check_cuda(cudaGetLastError(), "gather_mean_kernel"))) return rc;
   // 3. probe errors
   RouteArgs ra{};
   ra.B = s.B;
@@ -612,23 +1278,14 @@ int route_prologue(const void* q, const void* k, const void* v, const bsa_shape&
   ra.mref = L.mref;
   double route_density = static_cast<double>(density);
   if (with_v) {
-    // keys and values in cluster-major order (rows off[c] .. off[c] + n_c per head)
-    const int es = s.dtype == BSA_F32 ? 4 : 2;
-    const int vpr = s.D * es / 16;
-    const int64_t nvec = static_cast<int64_t>(s.Sk) * vpr;
-    const dim3 gg(static_cast<unsigned>((nvec + 255) / 256), s.Hkv, s.B);
-    gather_rows_kernel<<<gg, 256, 0, st>>>(static_cast<const uint4*>(k), static_cast<uint4*>(L.kp),
-                                           L.k_tok, s.Sk, s.Sk, vpr, s.Hkv);
-    gather_rows_kernel<<<gg, 256, 0, st>>>(static_cast<const uint4*>(v), static_cast<uint4*>(L.vp),
-                                           L.k_tok, s.Sk, s.Sk, vpr, s.Hkv);
-    count_launch();
-    count_launch();
+    // keys and values are in cluster-major order (rows off[c] .. off[c] + n_c per head)
     if (s.dtype == BSA_F32) {
       if (s.D == 64) launch_route_probe<float, 64>(L.kp, L.vp, ra, st);
       else launch_route_probe<float, 128>(L.kp, L.vp, ra, st);
     } else {
-      if (s.D == 64) launch_route_probe<__nv_bfloat16, 64>(L.kp, L.vp, ra, st);
-      else launch_route_probe<__nv_bfloat16, 128>(L.kp, L.vp, ra, st);
+      rc = s.D == 64 ? launch_route_tc<64>(L, s, Cq, Ck, ra.scale, ra.err, st)
+                     : launch_route_tc<128>(L, s, Cq, Ck, ra.scale, ra.err, st);
+      if (rc) return rc;
     }
   } else {
     if (s.D == 64)
@@ -639,8 +1296,10 @@ int route_prologue(const void* q, const void* k, const void* v, const bsa_shape&
     route_density = route_density - static_cast<double>(M) / static_cast<double>(s.Sq);
     if (route_density < 0.0) route_density = 0.0;
   }
-  count_launch();
-  if ((rc = check_cuda(cudaGetLastError(), "route score kernel"))) return rc;
+  if (!(with_v && s.dtype != BSA_F32)) {  // the tensor-core path counts and checks its own
+    count_launch();
+    if ((rc = check_cuda(cudaGetLastError(), "route score kernel"))) return rc;
+  }
   // 4. budgeted prefix per (batch, head)
   {
     const int smem = 32 * 256 * 8;

@@ -79,6 +79,27 @@ def test_routing_small_uneven_clusters(dtype, D, Hq, Hkv):
         assert not mask[:, :, Cq - 1].any() and not mask[:, :, :, 5].any()
 
 
+def test_routing_large_clusters_two_probe_tiles():
+    """Key clusters of several hundred keys (several 128-key pieces each, so the running
+    reference moves between pieces), 200 query clusters (two 128-probe tiles, the second
+    partly padding), GQA 4 over 2 KV heads, bf16 D=128; density 0.3."""
+    g = np.random.default_rng(41)
+    S, Cq, Ck = 2400, 200, 5
+    ql = g.permutation(np.concatenate([np.arange(Cq), g.integers(0, Cq, S - Cq)]))
+    kl = np.sort(g.integers(0, Ck, S))
+    kl[:Ck] = np.arange(Ck)
+    kl = g.permutation(kl)
+    q, k, v = wl.gaussian_qkv(1, 4, 2, S, 128, "bf16", seed=42)
+    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+    ref_err = oracle.compensation_errors(qd, kd, vd, ql, kl, Cq, Ck)
+    mask, err = _route(q, k, v, ql, kl, Cq, Ck, 0.3)
+    _check_errors(err, ref_err)
+    same = oracle.route_blocks(err, ql, kl, Cq, Ck, np.float32(0.3), dtype=np.float32)
+    np.testing.assert_array_equal(mask, same)
+    ref_mask = oracle.route_blocks(ref_err, ql, kl, Cq, Ck, np.float32(0.3))
+    _check_chain(mask, ref_mask, ref_err, ql, kl, Cq, Ck)
+
+
 def test_routing_density_edges():
     """Density 1 keeps every block of non-empty clusters, density 0 none."""
     q, k, v = wl.gaussian_qkv(1, 2, 2, 512, 64, "bf16", seed=33)
