@@ -372,12 +372,39 @@ struct RouteTcArgs {
   float* zc;              // (B, Hq, Cq, Ck): sum of the cluster's weights against mref
 };
 
-// Pieces of the non-empty clusters in [c, c_hi), in order; k counts the clusters.
+// Tile (x, y) of a 2-D tensor map into L2 only (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x),
+               "r"(y)
+               : "memory");
+}
+
+// Pieces of the non-empty clusters in [c, c_hi), in order; k counts the clusters. Run by
+// a whole warp on warp-uniform values: the lanes hold the counts and offsets of a window
+// of 32 consecutive clusters (one coalesced load each), so finding the next non-empty
+// cluster is a ballot rather than a chain of dependent loads.
 struct RtIter {
   int c, c_hi, p, nc, off, k;
+  int wbase, wcnt, woff;  // window [wbase, wbase + 32): this lane's cluster wbase + lane
   __device__ __forceinline__ void seek(const int32_t* cnt, const int32_t* offs) {
-    while (c < c_hi && (nc = __ldg(cnt + c)) <= 0) ++c;
-    if (c < c_hi) off = __ldg(offs + c);
+    const int lane = threadIdx.x & 31;
+    while (c < c_hi) {
+      if (c < wbase || c >= wbase + 32) {
+        wbase = c;
+        const int cc = c + lane;
+        wcnt = cc < c_hi ? __ldg(cnt + cc) : 0;
+        woff = cc < c_hi ? __ldg(offs + cc) : 0;
+      }
+      const uint32_t nz = __ballot_sync(0xffffffffu, wcnt > 0) & (0xffffffffu << (c - wbase));
+      if (nz) {
+        const int j = __ffs(nz) - 1;
+        c = wbase + j;
+        nc = __shfl_sync(0xffffffffu, wcnt, j);
+        off = __shfl_sync(0xffffffffu, woff, j);
+        return;
+      }
+      c = wbase + 32;
+    }
   }
   __device__ __forceinline__ void init(int lo, int hi, const int32_t* cnt, const int32_t* offs) {
     c = lo;
@@ -386,6 +413,8 @@ struct RtIter {
     k = 0;
     nc = 0;
     off = 0;
+    wbase = -64;
+    wcnt = woff = 0;
     seek(cnt, offs);
   }
   __device__ __forceinline__ void advance(const int32_t* cnt, const int32_t* offs) {
@@ -445,7 +474,10 @@ __global__ void __launch_bounds__(288, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* never = reinterpret_cast<int*>(tmem_slot + 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x / a.nsplit, split = blockIdx.x % a.nsplit;
+  // the probe tiles of one key range are neighbours in the grid, so they run together
+  // and share the range's K and V through L2
+  const int tiles = (a.Cq + 127) / 128;
+  const int tile = blockIdx.x % tiles, split = blockIdx.x / tiles;
   const int h = blockIdx.y, b = blockIdx.z;
   const int hkv = h / (a.Hq / a.Hkv);
   const int64_t bq = static_cast<int64_t>(b) * a.Hq + h;
@@ -459,7 +491,7 @@ __global__ void __launch_bounds__(288, 1)
     for (int i = 0; i < RT_NBAR; ++i)
       mbar_init(RBAR(i), (i == RT_QR || i == RT_PF0 || i == RT_PF1 || i == RT_OE0 || i == RT_OE1 ||
                           i == RT_XB0 || i == RT_XB1 || i == RT_XE)
-                             ? 256u
+                             ? 8u   // one arrival per softmax warp
                              : 1u);
     *abort_flag = 0;
     *never = 0;
@@ -574,6 +606,18 @@ __global__ void __launch_bounds__(288, 1)
         if (nn.valid()) {
           if (!(ok = wait_all(RBAR(RT_KE0 + s), (i >> 1) & 1, 47))) break;
           load(false, s, nn.row());
+          // K and V of piece i + 4 into L2, two pieces ahead of their copies
+          RtIter n4 = nn;
+          n4.advance(a.k_count, a.k_off);
+          if (n4.valid()) n4.advance(a.k_count, a.k_off);
+          if (n4.valid() && leader) {
+#pragma unroll
+            for (int cc = 0; cc < Cfg::NATOM; ++cc) {
+              tma_prefetch_l2_2d(&tmK, cc * 64, grow0 + n4.row());
+              tma_prefetch_l2_2d(&tmV, cc * 64, grow0 + n4.row());
+            }
+          }
+          __syncwarp();
         }
         // V of piece i + 1: its stage was last read by PV(i - 1)
         if (i >= 1 && !(ok = wait_all(RBAR(RT_VE0 + s1), ((i - 1) >> 1) & 1, 43))) break;
@@ -605,7 +649,8 @@ __global__ void __launch_bounds__(288, 1)
     // first half of dims, warps 5..8 columns 64..127 and the second half (warp w reads
     // TMEM lanes 32*(w%4)..+31). The pair exchanges its piece maxima, and at a cluster's
     // end its halves of the error and of the weight sum, through shared memory, each
-    // exchange closed by an mbarrier of the 256 threads (bounded waits).
+    // exchange closed by an mbarrier (bounded waits). Every hand-off is one arrival per
+    // warp: the lanes fence their own stores, meet at __syncwarp, and lane 0 arrives.
     constexpr int DH = D / 2;  // E columns per thread
     const int quarter = warp & 3, hh = (warp - 1) >> 2;
     const int r = quarter * 32 + lane;
@@ -649,8 +694,17 @@ __global__ void __launch_bounds__(288, 1)
                      "r"(lw[1]), "r"(lw[2]), "r"(lw[3]) : "memory");
       }
       fence_proxy_async_smem();
-      mbar_arrive(RBAR(RT_QR));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(RBAR(RT_QR));
     }
+    auto warp_arrive = [&](uint32_t bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    // waits are warp-uniform: the iterator's ballots need every lane of the warp
+    auto wait_w = [&](uint32_t bar, uint32_t parity, int where) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, where));
+    };
     const float* lc_row = a.lc + (bq * a.Cq + (live ? pa : 0)) * a.Ck;
     const int64_t out_row = (bq * a.Cq + (live ? pa : 0)) * a.Ck;
     bool ok = true;
@@ -659,10 +713,11 @@ __global__ void __launch_bounds__(288, 1)
     int pk = 0, pc = 0, pn = 0, ne = 0;  // ne: epilogues done
     float pm = 0.f, pz = 0.f, plc = 0.f;
     auto epilogue = [&]() -> bool {
-      if (!mbar_wait(RBAR(RT_OF0 + (pk & 1)), (pk >> 1) & 1, abort_flag, 50)) return false;
+      // v̄_c (this thread's half; prefetched into L1 when the cluster started)
+      const float4* vb = reinterpret_cast<const float4*>(a.vbar + (bk * a.Ck + pc) * D + hh * DH);
+      if (!wait_w(RBAR(RT_OF0 + (pk & 1)), (pk >> 1) & 1, 50)) return false;
       tc_fence_after();
       const float wc = static_cast<float>(pn) * ex2(plc - pm);
-      const float* vb = a.vbar + (bk * a.Ck + pc) * D + hh * DH;
       const uint32_t tE = tmem + lanes + 256 + 128 * (pk & 1) + hh * DH;
       float e2a = 0.f, e2b = 0.f;
 #pragma unroll
@@ -672,7 +727,7 @@ __global__ void __launch_bounds__(288, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 v4 = __ldg(reinterpret_cast<const float4*>(vb + 32 * q + 4 * c4));
+          const float4 v4 = __ldg(vb + 8 * q + c4);
           const float d0 = fmaf(-wc, v4.x, o[4 * c4]), d1 = fmaf(-wc, v4.y, o[4 * c4 + 1]);
           const float d2 = fmaf(-wc, v4.z, o[4 * c4 + 2]), d3 = fmaf(-wc, v4.w, o[4 * c4 + 3]);
           e2a = fmaf(d0, d0, fmaf(d1, d1, e2a));
@@ -680,11 +735,14 @@ __global__ void __launch_bounds__(288, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(RBAR(RT_OE0 + (pk & 1)));
       xe2[hh * 128 + r] = e2a + e2b;
       xz[hh * 128 + r] = pz;
-      mbar_arrive(RBAR(RT_XE));
-      if (!mbar_wait(RBAR(RT_XE), ne & 1, abort_flag, 53)) return false;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(RBAR(RT_OE0 + (pk & 1)));
+        mbar_arrive(RBAR(RT_XE));
+      }
+      if (!wait_w(RBAR(RT_XE), ne & 1, 53)) return false;
       ++ne;
       if (live && hh == 0) {
         a.err[out_row + pc] = sqrtf(xe2[r] + xe2[128 + r]);
@@ -706,8 +764,12 @@ __global__ void __launch_bounds__(288, 1)
         lc2 = live ? __ldg(lc_row + it.c) : 0.f;
         m = lc2;
         z = 0.f;
+        const float* vh = a.vbar + (bk * a.Ck + it.c) * D + hh * DH;
+#pragma unroll
+        for (int j = 0; j < DH; j += 32)
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(vh + j));
       }
-      if (!(ok = mbar_wait(RBAR(RT_SF0 + s), (i >> 1) & 1, abort_flag, 51))) break;
+      if (!(ok = wait_w(RBAR(RT_SF0 + s), (i >> 1) & 1, 51))) break;
       tc_fence_after();
       const uint32_t tS = tmem + lanes + 128 * s;
       float v[2][32];
@@ -727,8 +789,8 @@ __global__ void __launch_bounds__(288, 1)
       // overlap the partner's S columns)
       xmax[(s * 2 + hh) * 128 + r] = mx;
       tc_fence_before();
-      mbar_arrive(RBAR(RT_XB0 + s));
-      if (!(ok = mbar_wait(RBAR(RT_XB0 + s), (i >> 1) & 1, abort_flag, 54))) break;
+      warp_arrive(RBAR(RT_XB0 + s));
+      if (!(ok = wait_w(RBAR(RT_XB0 + s), (i >> 1) & 1, 54))) break;
       tc_fence_after();
       mx = fmaxf(mx, xmax[(s * 2 + (hh ^ 1)) * 128 + r]);
       const bool need = mx > m;
@@ -741,7 +803,7 @@ __global__ void __launch_bounds__(288, 1)
       if (!it.first() && __any_sync(0xffffffffu, need)) {
         // E holds this cluster's earlier pieces against the old reference: wait for
         // PV(i - 1), then scale this thread's half of it
-        if (!(ok = mbar_wait(RBAR(RT_VE0 + (s ^ 1)), ((i - 1) >> 1) & 1, abort_flag, 52))) break;
+        if (!(ok = wait_w(RBAR(RT_VE0 + (s ^ 1)), ((i - 1) >> 1) & 1, 52))) break;
         tc_fence_after();
         const uint32_t tE = tmem + lanes + 256 + 128 * (it.k & 1) + hh * DH;
 #pragma unroll 1
@@ -777,7 +839,7 @@ __global__ void __launch_bounds__(288, 1)
       z += za + zb;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(RBAR(RT_PF0 + s));
+      warp_arrive(RBAR(RT_PF0 + s));
       // the previous cluster's E: its last PV was issued before this piece's
       if (pend && !(ok = epilogue())) break;
       if (it.last()) {

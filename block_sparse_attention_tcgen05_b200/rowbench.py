@@ -200,18 +200,17 @@ def bench_routing_and_sta(timer, dev, hbm, tc, out):
     S = q.shape[2]
     # f1: SVG-EAR error-aware routing at density 0.22: the probe kernel computes, per
     # head, every query cluster's mean query against every key (logits and the
-    # exp-weighted values): 4 D FLOP per (probe, key) pair on the FMA pipe
+    # exp-weighted values): 4 D FLOP per (probe, key) pair, on the tensor cores with
+    # both operands that are not bf16-exact carried as two bf16 parts (the executed
+    # MMA work is about twice this, plus 16-key padding of each cluster's last piece)
     ws = torch.empty(ops._lib.load().bsa_routing_workspace_bytes(ops.make_shape(q, k), C, C),
                      dtype=torch.uint8, device=dev)
     ms = timer(lambda: ops.error_aware_block_mask(q, k, v, labels, labels, C, C, 0.22,
                                                   workspace=ws))
-    r = row("f1", "SVG-EAR error-aware routing (H=40, 245 probes per head over 32760 keys, "
-            "density 0.22)", ms, 4.0 * D * C * S * H, "FLOP", "alu", None)
-    alu = fp32_alu_tflops(dev)
-    r.update({"achieved": 4.0 * D * C * S * H / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-              "peak": alu, "frac": 4.0 * D * C * S * H / (ms * 1e-3) / 1e12 / alu,
-              "peak_note": "fp32 FMA pipe: SMs x 128 lanes x 2 x max SM clock"})
-    out.append(r)
+    out.append(row("f1", "SVG-EAR error-aware routing (H=40, 245 probes per head over 32760 "
+                   "keys, density 0.22; whole call: sorts, gathers and means, centroid "
+                   "logits, probe kernel, normalisation, selection)", ms,
+                   4.0 * D * C * S * H, "FLOP", "tensor", tc))
     # f3: the recipe's sliding-tile window mask, (3, 3, 5) tiles, driving the attention
     n_tiles = tuple(-(-g // t) for g, t in zip(GRID, TILE))
     mask = ops.sliding_tile_block_mask(n_tiles, (3, 3, 5), device=dev)
