@@ -8,6 +8,7 @@ LIB_PATH = os.path.join(_HERE, "libbsa.so")
 
 BSA_OK = 0
 BSA_ERR_INVALID_ARG = -1
+BSA_REUSE_PLAN = 1
 BSA_ERR_UNSUPPORTED = -2
 BSA_ERR_CUDA = -3
 BSA_ERR_TIMEOUT = -4
@@ -50,6 +51,8 @@ SIGNATURES = {
     "bsa_attention_workspace_bytes": (_sz, [Shape, _i, _i]),
     "bsa_centroid_compensated_attention": (
         _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _vp, _i64, _i64, _f, _i, _vp, _vp, _sz, _vp]),
+    "bsa_centroid_compensated_attention_ex": (
+        _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _vp, _i64, _i64, _f, _i, _vp, _vp, _sz, _i, _vp]),
     "bsa_per_kv_head_attention_workspace_bytes": (_sz, [Shape, _i, _i]),
     "bsa_per_kv_head_attention": (
         _i, [_vp, _vp, _vp, Shape, _vp, _i, _vp, _i, _vp, _i64, _i64, _f, _i, _vp, _vp, _sz, _vp]),

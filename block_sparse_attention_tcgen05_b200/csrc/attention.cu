@@ -1818,7 +1818,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
                                    const int32_t* k_labels, int Ck, const uint8_t* mask,
                                    int64_t mbs, int64_t mhs, float scale, int compensate,
                                    float* out, void* ws, size_t ws_bytes, cudaStream_t st,
-                                   int prof_id, bool dense) {
+                                   int prof_id, bool dense, bool reuse_plan) {
   int rc = validate_attention_shape(s, Cq, Ck);
   if (rc) return rc;
   if (!q || !k || !v || !q_labels || !k_labels || !mask || !out)
@@ -1846,7 +1846,9 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
         L.bias2);
     count_launch();
     if ((rc = check_cuda(cudaGetLastError(), "dense_prep_kernel"))) return rc;
-  } else {
+  } else if (!reuse_plan) {
+  // Steps 1-3 depend only on the labels and the mask: a call that reuses the plan of an
+  // earlier call on this workspace (same shape, labels, mask) skips them.
   // 1. cluster bitsets of the mask (label order)
   mask_cbits_kernel<<<dim3(Cq, nh, nb), 256, 0, st>>>(mask, mbs, mhs, nh, Cq, Ck, L.Wc, L.cbits);
   count_launch();
@@ -2005,7 +2007,20 @@ extern "C" int bsa_centroid_compensated_attention(const void* q, const void* k, 
   return bsa::centroid_compensated_attention(q, k, v, shape, q_labels, Cq, k_labels, Ck, block_mask,
                                              mask_b_stride, mask_h_stride, scale, compensate, out,
                                              workspace, workspace_bytes, bsa::as_stream(stream),
-                                             bsa::kProfAttention, false);
+                                             bsa::kProfAttention, false, false);
+}
+
+extern "C" int bsa_centroid_compensated_attention_ex(
+    const void* q, const void* k, const void* v, bsa_shape shape, const int32_t* q_labels, int Cq,
+    const int32_t* k_labels, int Ck, const uint8_t* block_mask, int64_t mask_b_stride,
+    int64_t mask_h_stride, float scale, int compensate, float* out, void* workspace,
+    size_t workspace_bytes, int flags, void* stream) {
+  if (flags & ~BSA_REUSE_PLAN) return bsa::fail(BSA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  return bsa::centroid_compensated_attention(q, k, v, shape, q_labels, Cq, k_labels, Ck, block_mask,
+                                             mask_b_stride, mask_h_stride, scale, compensate, out,
+                                             workspace, workspace_bytes, bsa::as_stream(stream),
+                                             bsa::kProfAttention, false,
+                                             (flags & BSA_REUSE_PLAN) != 0);
 }
 
 namespace bsa {
@@ -2053,7 +2068,7 @@ extern "C" int bsa_per_kv_head_attention(const void* q, const void* k, const voi
           qs, ks, vs, p, q_labels + kh * shape.Sq, Cq, k_labels + kh * shape.Sk, Ck,
           block_mask + b * mask_b_stride + g * mask_g_stride, 0, 0, scale, compensate,
           out + qh * shape.Sq * shape.D, workspace, workspace_bytes, as_stream(stream),
-          kProfAttention, false);
+          kProfAttention, false, false);
       if (rc) return rc;
     }
   }

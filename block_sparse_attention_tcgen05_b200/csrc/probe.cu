@@ -22,7 +22,7 @@ int centroid_compensated_attention(const void* q, const void* k, const void* v,
                                    const int32_t* k_labels, int Ck, const uint8_t* mask,
                                    int64_t mbs, int64_t mhs, float scale, int compensate,
                                    float* out, void* ws, size_t ws_bytes, cudaStream_t st,
-                                   int prof_id, bool dense);
+                                   int prof_id, bool dense, bool reuse_plan);
 size_t attention_workspace_bytes(const bsa_shape& s, int Cq, int Ck);
 
 constexpr int kMaxCentroidCluster = 4096;
@@ -440,5 +440,5 @@ extern "C" int bsa_probe_dense_attention(const void* q, const void* k, const voi
   // buffers passed along are never read on that path).
   return centroid_compensated_attention(qp, k, v, ps, zeros, 1, zeros, 1, one, 0, 0, scale, 0,
                                         o_probe, static_cast<char*>(workspace) + used,
-                                        workspace_bytes - used, st, kProfProbe, true);
+                                        workspace_bytes - used, st, kProfProbe, true, false);
 }

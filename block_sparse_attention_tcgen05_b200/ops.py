@@ -6,6 +6,7 @@ current torch stream. There is no CPU path.
 """
 
 import ctypes
+import weakref
 
 import torch
 
@@ -145,11 +146,32 @@ def _mask_strides(block_mask, B, H, Cq, Ck):
     return m, bs, hs
 
 
+# Workspace address -> the arguments of the last attention call that prepared it (labels
+# and mask by identity and in-place version) and the workspace tensor itself (weakly, so a
+# new tensor at a recycled address never matches), for calls that reuse that preparation.
+_PLANS = {}
+
+
+def _plan_key(shape, q_labels, k_labels, block_mask, Cq, Ck, compensate):
+    return (tuple(getattr(shape, f) for f, _ in shape._fields_), Cq, Ck, bool(compensate),
+            q_labels.data_ptr(), q_labels._version, tuple(q_labels.shape),
+            k_labels.data_ptr(), k_labels._version, tuple(k_labels.shape),
+            block_mask.data_ptr(), block_mask._version, tuple(block_mask.shape),
+            tuple(block_mask.stride()), block_mask.dtype)
+
+
 def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=None, Ck=None,
-                                   scale=None, compensate=True, out=None, workspace=None):
+                                   scale=None, compensate=True, out=None, workspace=None,
+                                   reuse_plan=False):
     """SVG-EAR centroid-compensated block-sparse attention (``compensate=False``: hard
     drop). q: (B,Hq,S,D), k/v: (B,Hkv,S,D) bf16 or fp32; labels int32; block_mask
-    bool/uint8 (Cq,Ck) / (H,Cq,Ck) / (B,H,Cq,Ck). Returns fp32 (B,Hq,S,D)."""
+    bool/uint8 (Cq,Ck) / (H,Cq,Ck) / (B,H,Cq,Ck). Returns fp32 (B,Hq,S,D).
+
+    ``reuse_plan=True`` skips the label sorts, key cluster order, query tile plan and
+    mask bitsets, reusing those of the last call on ``workspace``; that call must have
+    had the same shapes, label and mask tensors (unmodified since), Cq, Ck and
+    compensate, and no other call may have used the workspace in between. q, k, v and
+    scale may differ (the K/V gather, centroids and attention always run)."""
     _expect_qkv(q, k, v)
     B, Hq, Sq, D = q.shape
     _expect(q_labels, "q_labels", (torch.int32,), (1,), (Sq,))
@@ -160,18 +182,27 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
     Cq = int(block_mask.shape[-2]) if Cq is None else int(Cq)
     Ck = int(block_mask.shape[-1]) if Ck is None else int(Ck)
     m, bs, hs = _mask_strides(block_mask, B, Hq, Cq, Ck)
-    _need_cuda(q, k, v, q_labels, k_labels, m, out, workspace)
     shape = make_shape(q, k)
+    key = _plan_key(shape, q_labels, k_labels, block_mask, Cq, Ck, compensate)
+    rec = _PLANS.get(workspace.data_ptr()) if workspace is not None else None
+    if reuse_plan and (rec is None or rec[0] != key or rec[1]() is not workspace):
+        raise ValueError("reuse_plan needs the workspace of an earlier call with the same "
+                         "shapes, labels, mask, Cq, Ck and compensate (tensors unmodified)")
+    _need_cuda(q, k, v, q_labels, k_labels, m, out, workspace)
     if out is None:
         out = torch.empty((B, Hq, Sq, D), dtype=torch.float32, device=q.device)
     need = _lib.load().bsa_attention_workspace_bytes(shape, Cq, Ck)
     if need == 0:
         raise _lib.BsaError("bsa_attention_workspace_bytes", _lib.BSA_ERR_UNSUPPORTED, _lib.detail())
-    if workspace is None or workspace.numel() < need:
+    if not reuse_plan and (workspace is None or workspace.numel() < need):
         workspace = _workspace(need, q.device)
-    _call_on(q.device, "bsa_centroid_compensated_attention", _ptr(q), _ptr(k), _ptr(v), shape, _ptr(q_labels),
-         Cq, _ptr(k_labels), Ck, _ptr(m), bs, hs, float(scale or 0.0), 1 if compensate else 0,
-         _ptr(out), _ptr(workspace), workspace.numel(), _stream(q.device))
+    if workspace is not None:
+        _PLANS.pop(workspace.data_ptr(), None)
+    _call_on(q.device, "bsa_centroid_compensated_attention_ex", _ptr(q), _ptr(k), _ptr(v), shape,
+             _ptr(q_labels), Cq, _ptr(k_labels), Ck, _ptr(m), bs, hs, float(scale or 0.0),
+             1 if compensate else 0, _ptr(out), _ptr(workspace), workspace.numel(),
+             _lib.BSA_REUSE_PLAN if reuse_plan else 0, _stream(q.device))
+    _PLANS[workspace.data_ptr()] = (key, weakref.ref(workspace))
     return out
 
 

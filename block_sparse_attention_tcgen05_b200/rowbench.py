@@ -168,6 +168,24 @@ def bench_attention(timer, dev, hbm, tc, out):
     out.append(row("a8", f"fused compensated attention kernel ({pairs:.3e} executed pairs x 4D)",
                    kernel_ms, pairs * 4 * D, "FLOP", "tensor", tc))
     out.append(row("a4-a8", "whole attention call", ms, pairs * 4 * D, "FLOP", "tensor", tc))
+    # the same call reusing the label sorts, key order, tile plan and bitsets of the
+    # previous call on the workspace (labels and mask unchanged, as across denoising
+    # steps whose mask cache refreshes no head): only the K/V gather and centroids remain
+
+    def reuse_call():
+        ops.centroid_compensated_attention(q, k, v, labels, labels, mask, Cq=C, Ck=C, out=o,
+                                           workspace=ws, reuse_plan=True)
+    call()
+    _lib.call("bsa_profile_enable", timer.calls + timer.warmup)
+    ms_r = timer(reuse_call)
+    _lib.call("bsa_profile_read", 0, ctypes.byref(kms), ctypes.byref(kn))
+    _lib.call("bsa_profile_enable", 0)
+    kernel_r = kms.value / max(1, kn.value)
+    out.append(row("a4-a7 reused", "K/V gather and centroids only: preparation of a call that "
+                   "reuses the previous call's plan (call minus attention kernel)",
+                   max(ms_r - kernel_r, 1e-6), 2 * kv_bytes, "B", "hbm", hbm))
+    out.append(row("a4-a8 reused", "whole attention call reusing the plan", ms_r, pairs * 4 * D,
+                   "FLOP", "tensor", tc))
     # context: the same call with every tile pair kept (dense attention through the same
     # kernel); its time over the sparse call's is the sparse path's speedup
     full = torch.ones_like(mask)

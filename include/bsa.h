@@ -52,6 +52,9 @@ enum {
 
 enum { BSA_BF16 = 0, BSA_F32 = 1 };
 
+/* Flags of bsa_centroid_compensated_attention_ex. */
+enum { BSA_REUSE_PLAN = 1 };
+
 /* Problem shape. Sq = Sk = S for self-attention; D in {64, 128}. */
 typedef struct {
   int B, Hq, Hkv, Sq, Sk, D;
@@ -196,6 +199,32 @@ int bsa_centroid_compensated_attention(const void* q, const void* k, const void*
                                        int64_t mask_h_stride, float scale, int compensate,
                                        float* out, void* workspace, size_t workspace_bytes,
                                        void* stream);
+
+/*
+ * centroid_compensated_attention_ex — the same call with flags. [HMR] §HEART and
+ * "Reuse needs a fixed token grid" (labels fixed by the grid; masks reused across
+ * denoising steps while the mask cache refreshes no head).
+ *   flags & BSA_REUSE_PLAN : the workspace holds the preparation of an earlier call on
+ *              it (label sorts, key cluster order, query tile plan, mask bitsets) with
+ *              the same shape, q_labels, Cq, k_labels, Ck, block_mask contents and
+ *              strides; those steps are skipped and the labels are not checked again.
+ *              The K/V gather, the centroids and the attention run as usual, so q, k, v
+ *              and scale may change between the calls. The caller owns that
+ *              precondition: if the workspace does not hold such a preparation (or
+ *              another call used it in between) the behaviour is undefined, and the
+ *              kernels may read and write out of bounds. The Python binding passes the
+ *              flag only for a workspace whose last attention call it recorded with
+ *              the same arguments and unmodified label and mask tensors.
+ * Other flag bits: BSA_ERR_INVALID_ARG. Arguments otherwise as
+ * centroid_compensated_attention.
+ */
+int bsa_centroid_compensated_attention_ex(const void* q, const void* k, const void* v,
+                                          bsa_shape shape, const int32_t* q_labels, int Cq,
+                                          const int32_t* k_labels, int Ck,
+                                          const uint8_t* block_mask, int64_t mask_b_stride,
+                                          int64_t mask_h_stride, float scale, int compensate,
+                                          float* out, void* workspace, size_t workspace_bytes,
+                                          int flags, void* stream);
 
 /*
  * per_kv_head_attention — the same attention with labels of their own per (batch, KV

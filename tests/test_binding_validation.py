@@ -56,6 +56,29 @@ def test_attention_arguments():
     _raises("CUDA tensors only", f, q, k, v, lab, lab, mask)
 
 
+def test_plan_reuse_needs_a_prepared_workspace():
+    """reuse_plan skips the label sorts, tile plan and bitsets, which the kernels then
+    read from the workspace: the binding refuses it unless the workspace's last
+    attention call had the same arguments (no workspace, a fresh one, or a recorded one
+    whose mask was modified in place since)."""
+    from block_sparse_attention_tcgen05_b200 import ops
+    q, k, v = _qkv()
+    lab, mask = _labels(), torch.ones(C, C, dtype=torch.uint8)
+    ws = torch.zeros(1024, dtype=torch.uint8)
+    f = bsa.centroid_compensated_attention
+    _raises("reuse_plan needs", f, q, k, v, lab, lab, mask, reuse_plan=True)
+    _raises("reuse_plan needs", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True)
+    # a record as a successful call leaves it, then an in-place change of the mask
+    shape = ops.make_shape(q, k)
+    ops._PLANS[ws.data_ptr()] = (ops._plan_key(shape, lab, lab, mask, C, C, True), ops.weakref.ref(ws))
+    _raises("CUDA tensors only", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True)
+    _raises("reuse_plan needs", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True,
+            compensate=False)
+    mask[0, 0] = 0
+    _raises("reuse_plan needs", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True)
+    ops._PLANS.clear()
+
+
 def test_scoring_and_top_p_arguments():
     q, k, _ = _qkv()
     _raises("k has", bsa.antidiagonal_block_scores, q, k[:, :, :128])

@@ -252,3 +252,33 @@ def test_per_batch_and_head_masks(H, Hkv):
     for comp in (True, False):
         got = _run(q, k, v, ql, kl, mask, Cq, Ck, comp)
         _check(got[:, :, rows], _ref(q, k, v, ql, kl, mask, Cq, Ck, comp, rows=rows))
+
+
+def test_plan_reuse_with_new_qkv():
+    """A call that reuses the label sorts, key order, tile plan and bitsets of the previous
+    call on the same workspace ("Dynamic block masks and head-wise mask reuse": masks and
+    the token grid fixed across denoising steps) with new Q, K, V: bit-identical to a
+    fresh call on those values, and within tolerance of the oracle. Video-grid tiles
+    (72- and 144-token clusters), per-head masks, GQA, bf16 D=128."""
+    bsa = _bsa()
+    dev = torch.device("cuda")
+    grid, tile = (3, 12, 20), (3, 6, 8)
+    lab, C = oracle.tile_labels(*grid, tile)
+    S = int(np.prod(grid))
+    g = np.random.default_rng(51)
+    mask = g.random((4, C, C)) < 0.4
+    mask[:, np.arange(C), np.arange(C)] = True
+    lt = torch.as_tensor(lab, dtype=torch.int32, device=dev)
+    mt = torch.as_tensor(mask, dtype=torch.uint8, device=dev)
+    q0, k0, v0 = (t.to(dev) for t in wl.gaussian_qkv(1, 4, 2, S, 128, "bf16", seed=52))
+    q1, k1, v1 = wl.gaussian_qkv(1, 4, 2, S, 128, "bf16", seed=53)
+    ws = torch.empty(bsa.attention_workspace_bytes(q0, k0, C, C), dtype=torch.uint8, device=dev)
+    bsa.centroid_compensated_attention(q0, k0, v0, lt, lt, mt, Cq=C, Ck=C, workspace=ws)
+    reused = bsa.centroid_compensated_attention(q1.to(dev), k1.to(dev), v1.to(dev), lt, lt, mt,
+                                                Cq=C, Ck=C, workspace=ws, reuse_plan=True)
+    fresh = bsa.centroid_compensated_attention(q1.to(dev), k1.to(dev), v1.to(dev), lt, lt, mt,
+                                               Cq=C, Ck=C)
+    torch.cuda.synchronize()
+    assert bsa.device_status()[0] == 0
+    assert torch.equal(reused, fresh)
+    _check(reused.cpu().numpy(), _ref(q1, k1, v1, lab, lab, mask[None], C, C))
