@@ -19,10 +19,14 @@
 //                              sum to at most floor(density * Sq * Sk)
 //
 // Kernels (caller's stream): label sorts of both label arrays (the attention's sort),
-// per-cluster means of Q, K and V (fp32), the probe kernel (one CTA per 16 probes of a
-// head, streaming the head's keys cluster by cluster through shared memory), and one
-// CTA per head that selects the prefix exactly by a radix descent over the ratios'
-// bits with 64-bit pair counts.
+// one gather-and-mean pass per operand (fp32 means of Q, K and V; K and V also copied
+// into cluster-major order), then the probe errors: for bf16 inputs the centroid
+// logits and a tensor-core kernel (tcgen05 MMAs for q̄ . k_j and the weighted value
+// sums, per 128 probes and a key-balanced range of clusters) followed by a
+// normalisation to one reference per probe; for fp32 inputs an FMA-pipe kernel (one CTA
+// per 16 probes of a head, streaming the head's keys cluster by cluster through shared
+// memory). Last, one CTA per head selects the prefix exactly by a radix descent over
+// the ratios' bits with 64-bit pair counts.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -345,12 +349,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_probe_kernel(const T* __r
 // per CTA, the weights w = 2^(s - m) once per piece, and each K-step issues one MMA per
 // part, so logits and sums keep close to fp32 precision.
 //
-// One CTA (one per SM: 512 TMEM columns, ~194 KB of shared memory) takes 128 probes of
+// One CTA (one per SM: 512 TMEM columns, ~205 KB of shared memory) takes 128 probes of
 // one head and a range of key clusters (balanced by keys); clusters are cut into pieces
-// of at most 128 keys. 160 threads: warp 0 issues the TMA copies (double-buffered K and
-// V stages) and the MMAs; warps 1..4 hold one probe per thread. TMEM columns: S/P of
-// pieces i even / odd at 0 / 128 (P's high part over S columns 0..63, low part over
-// 64..127), E of clusters k even / odd at 256 / 384. The MMA order is QK(i+1), PV(i),
+// of at most 128 keys. 288 threads: warp 0 issues the TMA copies (double-buffered K and
+// V stages) and the MMAs; warps 1..8 hold each probe as a pair of threads (one per half
+// of a piece's key columns and of E's dims). TMEM columns: S/P of pieces i even / odd
+// at 0 / 128 (P's high part over S columns 0..63, low part over 64..127), E of
+// clusters k even / odd at 256 / 384. The MMA order is QK(i+1), PV(i),
 // QK(i+2), ..., so the next piece's logits are computed while the softmax threads take
 // the weights of this one. Per cluster the running reference m starts at the centroid
 // logit and follows the largest logit seen (E rescaled in TMEM when a later piece
