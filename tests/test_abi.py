@@ -96,6 +96,20 @@ def test_host_side_argument_errors(lib):
                                                 16, fake_ptr(), 16, fake_ptr(), 0, 0, 0.0, 1,
                                                 fake_ptr(), fake_ptr(), 1 << 30, null)
     assert st == _lib.BSA_ERR_UNSUPPORTED and str(lim) in _lib.detail()
+    # the flagged entry point: unknown flag bits, and the usual checks with the
+    # plan-reuse flag set
+    st = lib.bsa_centroid_compensated_attention_ex(null, null, null, sh, null, 16, null, 16, null,
+                                                   0, 0, 0.0, 1, null, null, 0, 2, null)
+    assert st == _lib.BSA_ERR_INVALID_ARG and "flags" in _lib.detail()
+    st = lib.bsa_centroid_compensated_attention_ex(null, null, null, sh, null, 16, null, 16, null,
+                                                   0, 0, 0.0, 1, null, null, 0,
+                                                   _lib.BSA_REUSE_PLAN, null)
+    assert st == _lib.BSA_ERR_INVALID_ARG and "null" in _lib.detail()
+    st = lib.bsa_centroid_compensated_attention_ex(fake_ptr(), fake_ptr(), fake_ptr(), sh,
+                                                   fake_ptr(), 16, fake_ptr(), 16, fake_ptr(), 0, 0,
+                                                   0.0, 1, fake_ptr(), fake_ptr(), 256,
+                                                   _lib.BSA_REUSE_PLAN, null)
+    assert st == _lib.BSA_ERR_WORKSPACE
     # scoring: S not a multiple of the block
     fake = ctypes.c_void_p(256)
     s2 = _lib.Shape(1, 1, 1, 1000, 1000, 64, _lib.BSA_BF16)
