@@ -152,6 +152,17 @@ def _mask_strides(block_mask, B, H, Cq, Ck):
 _PLANS = {}
 
 
+def _record_plan(workspace, key):
+    """Remember which call prepared ``workspace``; the record goes when the tensor does."""
+    ptr = workspace.data_ptr()
+
+    def drop(ref, ptr=ptr):
+        rec = _PLANS.get(ptr)
+        if rec is not None and rec[1] is ref:
+            del _PLANS[ptr]
+    _PLANS[ptr] = (key, weakref.ref(workspace, drop))
+
+
 def _plan_key(shape, q_labels, k_labels, block_mask, Cq, Ck, compensate):
     return (tuple(getattr(shape, f) for f, _ in shape._fields_), Cq, Ck, bool(compensate),
             q_labels.data_ptr(), q_labels._version, tuple(q_labels.shape),
@@ -202,7 +213,7 @@ def centroid_compensated_attention(q, k, v, q_labels, k_labels, block_mask, Cq=N
              _ptr(q_labels), Cq, _ptr(k_labels), Ck, _ptr(m), bs, hs, float(scale or 0.0),
              1 if compensate else 0, _ptr(out), _ptr(workspace), workspace.numel(),
              _lib.BSA_REUSE_PLAN if reuse_plan else 0, _stream(q.device))
-    _PLANS[workspace.data_ptr()] = (key, weakref.ref(workspace))
+    _record_plan(workspace, key)
     return out
 
 

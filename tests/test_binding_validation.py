@@ -70,13 +70,17 @@ def test_plan_reuse_needs_a_prepared_workspace():
     _raises("reuse_plan needs", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True)
     # a record as a successful call leaves it, then an in-place change of the mask
     shape = ops.make_shape(q, k)
-    ops._PLANS[ws.data_ptr()] = (ops._plan_key(shape, lab, lab, mask, C, C, True), ops.weakref.ref(ws))
+    ops._record_plan(ws, ops._plan_key(shape, lab, lab, mask, C, C, True))
     _raises("CUDA tensors only", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True)
     _raises("reuse_plan needs", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True,
             compensate=False)
     mask[0, 0] = 0
     _raises("reuse_plan needs", f, q, k, v, lab, lab, mask, workspace=ws, reuse_plan=True)
-    ops._PLANS.clear()
+    # the record goes with the workspace tensor
+    ptr = ws.data_ptr()
+    assert ptr in ops._PLANS
+    del ws
+    assert ptr not in ops._PLANS
 
 
 def test_scoring_and_top_p_arguments():
